@@ -1,0 +1,427 @@
+"""Pins for the fp64 CPU oracle: each test checks the oracle against something
+other than itself -- a closed form, an exact integer identity, an exhaustive
+enumeration, a library conversion routine, a hand-derived example, or a fact
+printed on the model cards (tests/golden/format_facts.json) -- chosen so that a
+dropped term, a wrong sign or index, or a transposed operand fails one of them.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "format_facts.json")
+FACTS = json.load(open(GOLDEN))
+RNG = np.random.default_rng(1234)
+
+
+def popcount(v):
+    return bin(v).count("1")
+
+
+# --------------------------------------------------------------------------
+# Walsh-Hadamard transform
+# --------------------------------------------------------------------------
+def hadamard_matrix_from_oracle():
+    H = np.empty((128, 128))
+    for j in range(128):
+        e = np.zeros(128)
+        e[j] = 1.0
+        H[:, j] = O.fwht128_f64(e)
+    return H
+
+
+def test_fwht_matrix_is_sylvester_and_orthogonal():
+    H = hadamard_matrix_from_oracle()
+    closed = np.array([[(-1) ** popcount(i & j) for j in range(128)] for i in range(128)], dtype=np.float64)
+    assert np.array_equal(H, closed)  # natural (Sylvester) order, entries +-1
+    assert np.array_equal(H @ H.T, 128.0 * np.eye(128))  # H . H^T = 128 I, exact in integers
+
+
+def test_fwht_involution_and_parseval():
+    for _ in range(20):
+        v = RNG.integers(-1000, 1000, 128).astype(np.float64)
+        w = O.fwht128_f64(v)
+        assert np.array_equal(O.fwht128_f64(w), 128.0 * v)  # H(Hv) = 128 v, exact
+        assert np.isclose(w @ w, 128.0 * (v @ v), rtol=0, atol=0)  # integer Parseval
+    # dot products survive the transform: (Hx).(Hw) = 128 x.w (integers, exact)
+    x = RNG.integers(-50, 50, 128).astype(np.float64)
+    w = RNG.integers(-50, 50, 128).astype(np.float64)
+    assert O.fwht128_f64(x) @ O.fwht128_f64(w) == 128.0 * (x @ w)
+
+
+def test_fwht_spec_scale_constant_and_closed_forms():
+    c = np.float32(1.0 / np.sqrt(128.0))
+    assert hex(c.view(np.uint32)) == FACTS["fwht128_scale_f32_bits"]["value"].lower()
+    # constant vector: all energy in the first output, 128 * c
+    out = O.fwht128_spec_f32(np.ones(128, np.float32))
+    assert out[0] == np.float32(128.0) * c and np.all(out[1:] == 0)
+    # unit vectors give +-c times the Sylvester column, exactly
+    for j in (0, 1, 5, 64, 127):
+        e = np.zeros(128, np.float32)
+        e[j] = 1.0
+        col = np.array([(-1) ** popcount(i & j) for i in range(128)], np.float32) * c
+        assert np.array_equal(O.fwht128_spec_f32(e), col)
+
+
+def test_fwht_spec_f32_error_bound():
+    # fp32 butterflies then one multiply: |spec - c.H.v| <= (7 + 1) 2^-24 sum|v| c (7 rounded levels + scale)
+    c = 1.0 / np.sqrt(128.0)
+    for _ in range(50):
+        v = RNG.standard_normal(128).astype(np.float32) * np.float32(RNG.uniform(0.01, 100))
+        exact = O.fwht128_f64(v.astype(np.float64)) * c
+        got = O.fwht128_spec_f32(v).astype(np.float64)
+        bound = 9 * 2.0 ** -24 * np.abs(v).astype(np.float64).sum() * c
+        assert np.max(np.abs(got - exact)) <= bound
+
+
+def test_hadamard_rotate_matches_spec_then_bf16():
+    x = O.bf16_encode(RNG.standard_normal(256))[None, :].repeat(2, 0)
+    y = O.hadamard128_rotate(x)
+    for g in range(2):
+        v = torch.from_numpy(x[0, g * 128:(g + 1) * 128].view(np.int16)).view(torch.bfloat16).float().numpy()
+        r = O.fwht128_spec_f32(v)
+        ref = torch.from_numpy(r).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(y[0, g * 128:(g + 1) * 128], ref)
+
+
+# --------------------------------------------------------------------------
+# Number formats
+# --------------------------------------------------------------------------
+def test_bf16_codec_exhaustive_and_vs_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = O.bf16_decode(bits)
+    tv = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    finite = ~np.isnan(tv)
+    assert np.array_equal(vals[finite], tv[finite])
+    assert np.array_equal(O.bf16_encode(vals[finite]), bits[finite])  # decode -> encode is identity
+    # round to nearest even on random fp32 (incl. exact ties) vs torch's cast
+    f = np.concatenate([RNG.standard_normal(3000).astype(np.float32) * 10.0 ** RNG.integers(-30, 30, 3000),
+                        (bits[:2000].astype(np.uint32) << 16 | 0x8000).view(np.float32)])
+    f = f[np.isfinite(f)].astype(np.float32)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.bf16_encode(f.astype(np.float64)), ref)
+
+
+def test_f16_codec_exhaustive_and_vs_numpy():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = O.f16_decode(bits)
+    nv = bits.view(np.float16).astype(np.float64)
+    finite = np.isfinite(nv)
+    assert np.array_equal(vals[finite], nv[finite])
+    assert np.array_equal(O.f16_encode(vals[finite]), bits[finite])
+    f = RNG.standard_normal(4000) * 10.0 ** RNG.integers(-9, 5, 4000)
+    f = f.astype(np.float32).astype(np.float64)
+    assert np.array_equal(O.f16_encode(f), f.astype(np.float16).view(np.uint16))
+
+
+def test_e4m3_decode_table_and_vs_torch():
+    tab = FACTS["e4m3_values"]
+    for hx, v in tab["table"]:
+        d = O.e4m3_decode(np.array([int(hx, 16)], np.uint8))[0]
+        assert d == v and np.signbit(d) == np.signbit(v)
+    for hx in tab["nan"]:
+        assert np.isnan(O.e4m3_decode(np.array([int(hx, 16)], np.uint8))[0])
+    allb = np.arange(256, dtype=np.uint8)
+    mine = O.e4m3_decode(allb)
+    ref = torch.from_numpy(allb).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+
+
+def test_e4m3_encode_roundtrip_rne_and_saturation():
+    allb = np.arange(256, dtype=np.uint8)
+    vals = O.e4m3_decode(allb)
+    ok = ~np.isnan(vals)
+    assert np.array_equal(O.e4m3_encode(vals[ok]), allb[ok])
+    f = (RNG.standard_normal(5000) * 10.0 ** RNG.integers(-3, 3, 5000)).astype(np.float32)
+    f = f[np.abs(f) <= 448].astype(np.float64)
+    ref = torch.from_numpy(f.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(f), ref)
+    assert list(O.e4m3_encode(np.array([1000.0, -1e9, 460.0, 470.0]))) == [0x7E, 0xFE, 0x7E, 0x7E]
+    # a tie between 1.0 (0x38) and 1.125 (0x39) goes to the even code
+    assert O.e4m3_encode(np.array([1.0625]))[0] == 0x38
+    assert O.e4m3_encode(np.array([1.1875]))[0] == 0x3A
+
+
+# --------------------------------------------------------------------------
+# Activation quantiser
+# --------------------------------------------------------------------------
+def test_act_quant_hand_example_ties_and_zero():
+    v = np.zeros(128, np.float32)
+    v[:8] = [127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -127.0]
+    q, s = O.act_quant_group(v)
+    assert s == np.float32(1.0)
+    assert list(q[:8]) == [127, 2, 4, -2, -4, 0, 2, -127] and not q[8:].any()
+    q, s = O.act_quant_group(np.zeros(128, np.float32))
+    assert s == 0 and not q.any()
+
+
+def test_act_quant_invariants_and_idempotence():
+    for _ in range(50):
+        v = (RNG.standard_normal(128) * RNG.uniform(1e-3, 1e3)).astype(np.float32)
+        q, s = O.act_quant_group(v)
+        amax = np.max(np.abs(v))
+        assert s == np.float32(amax / np.float32(127))
+        assert np.max(np.abs(q.astype(int))) == 127
+        assert np.all(np.abs(v.astype(np.float64) - float(s) * q) <= 0.5 * float(s) * (1 + 1e-6))
+        # quantising the dequantised group gives back the same codes
+        q2, s2 = O.act_quant_group((np.float32(s) * q.astype(np.float32)).astype(np.float32))
+        assert np.array_equal(q2, q)
+
+
+def test_act_quant_rotate_is_spec_transform_then_quant():
+    x = O.bf16_encode(RNG.standard_normal(256) * 3)[None, :]
+    q, s = O.act_quant_i8_g128(x, rotate=True)
+    c = 1.0 / np.sqrt(128.0)
+    xv = O.bf16_decode(x)[0]
+    for g in range(2):
+        rot = O.fwht128_f64(xv[g * 128:(g + 1) * 128]) * c  # exact rotation
+        deq = float(s[0, g]) * q[0, g * 128:(g + 1) * 128]
+        assert np.max(np.abs(deq - rot)) <= 0.5 * float(s[0, g]) * (1 + 1e-4) + 1e-5 * np.abs(rot).max()
+
+
+# --------------------------------------------------------------------------
+# Weight quantisers
+# --------------------------------------------------------------------------
+def test_quant_i8_scale_rule_bound_and_idempotence():
+    W = (RNG.standard_normal((6, 256)) * 0.02).astype(np.float32)
+    W[2, :128] = 0.0  # an all-zero group
+    for f16 in (False, True):
+        q, s = O.quant_i8_g128(W, scale_f16=f16)
+        dec = O.f16_decode(s) if f16 else O.bf16_decode(s)
+        assert dec[2, 0] == 0 and not q[2, :128].any()
+        for n in range(6):
+            for g in range(2):
+                grp = W[n, g * 128:(g + 1) * 128]
+                amax = np.float32(np.max(np.abs(grp)))
+                want = np.float32(amax / np.float32(127))
+                ref = (np.float16(want).view(np.uint16) if f16 else
+                       torch.tensor([want]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)[0])
+                assert s[n, g] == ref
+                if amax == 0:
+                    continue
+                qq = q[n, g * 128:(g + 1) * 128].astype(np.float64)
+                assert np.max(np.abs(qq)) <= 127
+                err = np.abs(grp.astype(np.float64) - dec[n, g] * qq)
+                clamped = np.abs(grp / dec[n, g]) > 127.5
+                assert np.all(err[~clamped] <= 0.5 * dec[n, g] * (1 + 1e-6))
+        # re-quantising the dequantised weights gives the same codes
+        Wd = O.dequant(O.I8_G128_F16 if f16 else O.I8_G128_BF16, q.view(np.uint8), s, None, 6, 256)
+        q2, s2 = O.quant_i8_g128(Wd.astype(np.float32), scale_f16=f16)
+        assert np.array_equal(q2, q) and np.array_equal(s2, s)
+
+
+def test_quant_i8_hadamard_domain_reproduces_product():
+    # weights quantised in the rotated domain, applied to rotated activations,
+    # approximate the unrotated fp64 product x . W^T
+    N, K, M = 16, 512, 3
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    x = O.bf16_encode(RNG.standard_normal((M, K)))
+    q, s = O.quant_i8_g128(W, hadamard=True)
+    y = O.forward(x, q.view(np.uint8), s, None, O.I8_G128_BF16, O.HADAMARD, N)
+    exact = O.bf16_decode(x) @ W.astype(np.float64).T
+    assert np.linalg.norm(y - exact) <= 2e-2 * np.linalg.norm(exact)
+    # and the rotation itself is orthonormal: de-rotating the dequantised
+    # weights (H / sqrt(128) is its own inverse) recovers W within the
+    # quantisation error
+    H = hadamard_matrix_from_oracle() / np.sqrt(128.0)
+    Wd = O.dequant(O.I8_G128_BF16, q.view(np.uint8), s, None, N, K)
+    back = np.concatenate([Wd[:, g * 128:(g + 1) * 128] @ H for g in range(K // 128)], axis=1)
+    assert np.max(np.abs(back - W)) < 0.02 * 4 / 127 * 4
+
+
+def test_quant_fp8_block_rule():
+    N, K = 200, 256  # a ragged last row block (72 rows)
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    q, s = O.quant_fp8_b128(W)
+    assert s.shape == (2, 2)
+    for nb in range(2):
+        for g in range(2):
+            blk = W[nb * 128:(nb + 1) * 128, g * 128:(g + 1) * 128]
+            amax = np.float32(np.max(np.abs(blk)))
+            want = torch.tensor([np.float32(amax / np.float32(448))]).to(torch.bfloat16)
+            assert s[nb, g] == want.view(torch.int16).numpy().view(np.uint16)[0]
+            sd = float(want.float())
+            codes = q[nb * 128:(nb + 1) * 128, g * 128:(g + 1) * 128]
+            ref = torch.from_numpy((blk / np.float32(sd)).astype(np.float32).clip(-448, 448)).to(
+                torch.float8_e4m3fn).view(torch.uint8).numpy()
+            assert np.array_equal(codes, ref)
+
+
+def test_quant_i4_rule():
+    W = (RNG.standard_normal((4, 128)) * 0.02).astype(np.float32)
+    q, s = O.quant_i4_g64(W)
+    dec = O.bf16_decode(s)
+    assert q.min() >= -8 and q.max() <= 7
+    for n in range(4):
+        for g in range(2):
+            grp = W[n, g * 64:(g + 1) * 64].astype(np.float64)
+            assert np.all(np.abs(grp - dec[n, g] * q[n, g * 64:(g + 1) * 64]) <= 0.5 * dec[n, g] * (1 + 1e-6) + 1e-12)
+
+
+# --------------------------------------------------------------------------
+# Packing and sizes
+# --------------------------------------------------------------------------
+def test_pack_i4_layout_and_roundtrip():
+    q = np.zeros((1, 64), np.int8)
+    q[0, :4] = [1, 2, -8, 7]
+    p = O.pack_i4(q)
+    assert p[0, 0] == (9 | (10 << 4)) and p[0, 1] == (0 | (15 << 4))  # low nibble first, offset +8
+    for _ in range(5):
+        q = RNG.integers(-8, 8, (7, 192)).astype(np.int8)
+        q[0, :] = -8
+        q[1, :] = 7
+        assert np.array_equal(O.unpack_i4(O.pack_i4(q), 192), q)
+
+
+def test_pack_i5_layout_and_roundtrip():
+    q = np.zeros((1, 128), np.uint8)
+    q[0, 0] = 1
+    q[0, 1] = 31
+    p = O.pack_i5(q)
+    # code 0 in bits 0-4, code 1 in bits 5-9 of the little-endian stream
+    assert p[0, 0] == (1 | (31 << 5) & 0xFF) and p[0, 1] == (31 >> 3) and not p[0, 2:].any()
+    for _ in range(5):
+        q = RNG.integers(0, 32, (5, 256)).astype(np.uint8)
+        q[0, :] = 31
+        q[1, :] = 0
+        assert np.array_equal(O.unpack_i5(O.pack_i5(q), 256), q)
+
+
+@pytest.mark.parametrize("fmt,bpw", [(O.I4_G64_BF16, 4.25), (O.I8_G128_BF16, 8.125), (O.I8_G128_F16, 8.125),
+                                     (O.I8A8_G128_BF16, 8.125), (O.I5Z_G128_F16, 5.1875),
+                                     (O.FP8_B128_BF16, 8 + 16 / 16384)])
+def test_packed_sizes_bits_per_weight(fmt, bpw):
+    N, K = 21504, 5376
+    c, s, z = O.packed_sizes(fmt, N, K)
+    assert 8 * (c + s + z) / (N * K) == pytest.approx(bpw, rel=0, abs=1e-12)
+    if fmt == O.I4_G64_BF16:
+        assert bpw == FACTS["int4_g64_bf16_bits_per_weight"]["value"]
+
+
+# --------------------------------------------------------------------------
+# Dequantise-then-matmul
+# --------------------------------------------------------------------------
+def _exact_case(fmt, M=3, N=5, K=256):
+    """Scales 1, small integer codes and integer activations: y is an exact
+    integer matrix, equal to an int64 matmul of the codes."""
+    x_int = RNG.integers(-3, 4, (M, K))
+    x = O.bf16_encode(x_int.astype(np.float64))
+    one_bf16, one_f16 = 0x3F80, 0x3C00
+    if fmt in (O.I8_G128_BF16, O.I8_G128_F16):
+        q = RNG.integers(-3, 4, (N, K)).astype(np.int8)
+        s = np.full((N, K // 128), one_f16 if fmt == O.I8_G128_F16 else one_bf16, np.uint16)
+        return x, x_int, q.view(np.uint8), s, None, q.astype(np.int64)
+    if fmt == O.I4_G64_BF16:
+        q = RNG.integers(-8, 8, (N, K)).astype(np.int8)
+        return x, x_int, O.pack_i4(q), np.full((N, K // 64), one_bf16, np.uint16), None, q.astype(np.int64)
+    if fmt == O.I5Z_G128_F16:
+        q = RNG.integers(0, 32, (N, K)).astype(np.uint8)
+        z = RNG.integers(0, 32, (N, K // 128)).astype(np.uint8)
+        wq = q.astype(np.int64) - np.repeat(z.astype(np.int64), 128, axis=1)
+        return x, x_int, O.pack_i5(q), np.full((N, K // 128), one_f16, np.uint16), z, wq
+    if fmt == O.FP8_B128_BF16:
+        ints = RNG.integers(-3, 4, (N, K))
+        codes = O.e4m3_encode(ints.astype(np.float64).ravel()).reshape(N, K)
+        return x, x_int, codes, np.full(((N + 127) // 128, K // 128), one_bf16, np.uint16), None, ints
+
+
+@pytest.mark.parametrize("fmt", [O.I8_G128_BF16, O.I8_G128_F16, O.I4_G64_BF16, O.I5Z_G128_F16, O.FP8_B128_BF16])
+def test_forward_exact_integer_case(fmt):
+    x, x_int, codes, s, z, wq = _exact_case(fmt)
+    N = wq.shape[0]
+    y = O.forward(x, codes, s, z, fmt, 0, N)
+    assert np.array_equal(y, (x_int @ wq.T).astype(np.float64))  # not y^T, not a transposed operand
+
+
+def test_forward_brute_force_random_scales():
+    # explicit fp64 matrix from independently decoded scales (torch's bf16 / numpy's f16)
+    M, N, K = 4, 3, 256
+    q = RNG.integers(-127, 128, (N, K)).astype(np.int8)
+    s = O.bf16_encode(np.exp(RNG.normal(-4, 0.5, (N, K // 128))))
+    x = O.bf16_encode(RNG.standard_normal((M, K)))
+    sd = torch.from_numpy(s.view(np.int16)).view(torch.bfloat16).double().numpy()
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).double().numpy()
+    Wt = q.astype(np.float64) * np.repeat(sd, 128, axis=1)
+    y = O.forward(x, q.view(np.uint8), s, None, O.I8_G128_BF16, 0, N)
+    ref = np.array([[sum(xd[m, k] * Wt[n, k] for k in range(K)) for n in range(N)] for m in range(M)])
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-15)
+    # int5 with zero points and f16 scales, and fp8 with block scales
+    q5 = RNG.integers(0, 32, (N, K)).astype(np.uint8)
+    z5 = RNG.integers(0, 32, (N, K // 128)).astype(np.uint8)
+    s5 = (np.exp(RNG.normal(-4, 0.5, (N, K // 128)))).astype(np.float16)
+    W5 = (q5.astype(np.float64) - np.repeat(z5, 128, axis=1)) * np.repeat(s5.astype(np.float64), 128, axis=1)
+    y5 = O.forward(x, O.pack_i5(q5), s5.view(np.uint16), z5, O.I5Z_G128_F16, 0, N)
+    assert np.allclose(y5, xd @ W5.T, rtol=1e-12, atol=1e-14)
+    c8 = RNG.integers(0, 256, (N, K)).astype(np.uint8)
+    c8[(c8 & 0x7F) == 0x7F] = 0x10  # no NaN codes
+    s8 = O.bf16_encode(np.exp(RNG.normal(-4, 0.5, (1, K // 128))))
+    W8 = torch.from_numpy(c8).view(torch.float8_e4m3fn).double().numpy() * np.repeat(
+        torch.from_numpy(s8.view(np.int16)).view(torch.bfloat16).double().numpy(), 128, axis=1)
+    y8 = O.forward(x, c8, s8, None, O.FP8_B128_BF16, 0, N)
+    assert np.allclose(y8, xd @ W8.T, rtol=1e-12, atol=1e-14)
+
+
+def test_w8a8_int32_accumulators_and_combination():
+    M, N, K = 3, 4, 384
+    q = RNG.integers(-127, 128, (N, K)).astype(np.int8)
+    q[0, :128] = 127
+    s = O.bf16_encode(np.exp(RNG.normal(-4, 0.5, (N, K // 128))))
+    x = O.bf16_encode(RNG.standard_normal((M, K)) * 5)
+    x[0, :128] = O.bf16_encode(np.full(128, -2.0))  # a group at full scale: acc = -128 * 127 * 127
+    for rot in (0, O.HADAMARD):
+        y, acc = O.forward(x, q.view(np.uint8), s, None, O.I8A8_G128_BF16, rot, N, want_acc=True)
+        qx, sx = O.act_quant_i8_g128(x, rotate=bool(rot))
+        for m in range(M):
+            for n in range(N):
+                for g in range(K // 128):
+                    ref = int(np.dot(qx[m, g * 128:(g + 1) * 128].astype(np.int64),
+                                     q[n, g * 128:(g + 1) * 128].astype(np.int64)))
+                    assert acc[m, n, g] == ref and abs(ref) <= 128 * 127 * 127
+        if not rot:
+            assert acc[0, 0, 0] == -128 * 127 * 127
+        sd = O.bf16_decode(s)
+        ref_y = np.einsum("mg,ng,mng->mn", sx.astype(np.float64), sd, acc.astype(np.float64))
+        assert np.allclose(y, ref_y, rtol=1e-14, atol=0)
+
+
+# --------------------------------------------------------------------------
+# MoE routing and gate_up
+# --------------------------------------------------------------------------
+def test_moe_permute_brute_force():
+    for T, E in ((1, 8), (7, 16), (33, 128)):
+        ids = np.stack([RNG.permutation(E)[:8] for _ in range(T)]).astype(np.int32)
+        counts, offsets, perm, bad = O.moe_permute(ids, E)
+        assert bad == 0 and counts.sum() == T * 8 and offsets[-1] == T * 8
+        assert np.array_equal(np.sort(perm), np.arange(T * 8))  # a permutation
+        assert np.array_equal(perm, np.argsort(ids.ravel(), kind="stable"))  # stable by (expert, t, j)
+        assert np.array_equal(counts, np.bincount(ids.ravel(), minlength=E))
+    # every token on the same expert; an invalid id is dropped and counted
+    ids = np.zeros((5, 8), np.int32)
+    ids[4, 7] = 99
+    counts, offsets, perm, bad = O.moe_permute(ids, 4)
+    assert bad == 1 and counts[0] == 39 and offsets[1] == 39
+
+
+def test_moe_gate_up_reduces_to_dense():
+    T, E, N, K, topk = 5, 6, 48, 256, 3
+    ids = np.stack([RNG.permutation(E)[:topk] for _ in range(T)]).astype(np.int32)
+    x = O.bf16_encode(RNG.standard_normal((T, K)))
+    qs, ss = [], []
+    for e in range(E):
+        q, s = O.quant_i8_g128((RNG.standard_normal((N, K)) * 0.02).astype(np.float32), hadamard=True)
+        qs.append(q)
+        ss.append(s)
+    codes = np.stack(qs).view(np.uint8)
+    scales = np.stack(ss)
+    out = O.moe_gate_up(x, ids, codes, scales, O.I8_G128_BF16, O.HADAMARD, E, N)
+    for t in range(T):
+        for j in range(topk):
+            e = ids[t, j]
+            dense = O.forward(x[t:t + 1], codes[e], scales[e], None, O.I8_G128_BF16, O.HADAMARD, N)
+            assert np.array_equal(out[t, j], dense[0])
