@@ -1,0 +1,467 @@
+"""Benchmark of the quantized linear layer on B200.
+
+Workload (the headline): dense decode W8A8 int8 g128 in the Hadamard domain,
+N = 21504, K = 5376, tokens M in {1, 4, 8, 16}.  One step = the whole hot path
+once per M: rotate + quantise the activations, then the skinny GEMM over the
+packed weight.  Metric: decode qGEMV HBM GB/s, counted from the algorithmic
+bytes (packed codes + scales + bf16 x read + fp32 y written).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+
+Timing: W eager warm-up steps, then the K timed steps replayed from a CUDA
+graph, bracketed by a barrier and device synchronisation, measured with CUDA
+events on the launching stream; max over ranks.  Four packed copies of the
+weight (470 MB, more than the 126 MB L2) rotate between the forward calls, so
+no call finds its weight in L2.  The library's own launch trace (CUDA events
+around each of its kernels, captured into the graph) gives the per-kernel
+durations of the last timed graph replay for the roofline.
+Multi-GPU: replicas only -- the layer does not shard in this workload, every
+rank runs the same step on its own GPU and value sums the ranks' bytes.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+N_FULL, K_FULL = 21504, 5376
+MS = (1, 4, 8, 16)
+COPIES = 4
+METRIC = "decode qGEMV HBM GB/s (% of peak); prefill qGEMM TOPS (% of int8/fp8 peak)"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return p.parse_args()
+
+
+def step_bytes():
+    """Algorithmic bytes of one step: per M, codes + scales + x (bf16) + y (fp32)."""
+    G = K_FULL // 128
+    w = N_FULL * K_FULL + N_FULL * G * 2
+    return sum(w + m * K_FULL * 2 + m * N_FULL * 4 for m in MS)
+
+
+def skinny_bytes(m):
+    """Algorithmic bytes of one skinny-GEMM launch: codes + scales + int8 x + fp32 x scales + fp32 y."""
+    G = K_FULL // 128
+    return N_FULL * K_FULL + N_FULL * G * 2 + m * K_FULL + m * G * 4 + m * N_FULL * 4
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_traffic(name: str, src: Path):
+    """Per-launch DRAM bytes of a kernel from its committed ncu summary, if the
+    summary was taken on the current source (matching sha256 of the .cu file)."""
+    md = ROOT / "profiles" / f"{name}.md"
+    if not md.exists():
+        return None
+    text = md.read_text()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr:
+        return None
+    if hashlib.sha256(src.read_bytes()).hexdigest() != m_sha.group(1):
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle arm
+# --------------------------------------------------------------------------
+def oracle_sample(rows: int):
+    """Inputs of a bounded sample of the workload: the first `rows` weight rows,
+    quantised by the oracle, and the activations of each M."""
+    from moe_hadamard128_act_b200 import synth
+    from oracle import oracle as O
+
+    W = synth.weight_rows(0, "W", K_FULL, 0, rows)
+    q, s = O.quant_i8_g128(W, hadamard=True)
+    xs = {m: synth.activations(0, f"x_M{m}", m, K_FULL, outlier_frac=0.01) for m in MS}
+    return q.view(np.uint8), s, xs
+
+
+def oracle_step(q, s, xs, rows):
+    from oracle import oracle as O
+
+    t0 = time.perf_counter()
+    for m in MS:
+        O.forward(xs[m], q, s, None, O.I8A8_G128_BF16, O.HADAMARD, rows)
+    return time.perf_counter() - t0
+
+
+def sample_bytes(rows):
+    G = K_FULL // 128
+    return sum(rows * (K_FULL + G * 2) + m * K_FULL * 2 + m * rows * 4 for m in MS)
+
+
+def cpu_baseline(target_s: float = 10.0):
+    rows = 512
+    q, s, xs = oracle_sample(rows)
+    t = oracle_step(q, s, xs, rows)
+    rows = int(min(N_FULL, max(64, rows * target_s / max(t, 1e-3))))
+    q, s, xs = oracle_sample(rows)
+    t = oracle_step(q, s, xs, rows)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": sample_bytes(rows) / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle, W8A8 Hadamard forward of the first {rows} of {N_FULL} weight rows for "
+                      f"M in {list(MS)} (one step), {t:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from oracle import oracle as O
+
+    O.build()
+    rows = 512
+    q, s, xs = oracle_sample(rows)
+    t = oracle_step(q, s, xs, rows)
+    budget = 120.0 / max(1, args.steps + args.warmup)  # whole run within a few minutes
+    rows = int(min(N_FULL, max(32, rows * budget / max(t, 1e-3))))
+    q, s, xs = oracle_sample(rows)
+    for _ in range(args.warmup):
+        oracle_step(q, s, xs, rows)
+    tot = sum(oracle_step(q, s, xs, rows) for _ in range(args.steps))
+    value = args.steps * sample_bytes(rows) / tot / 1e9
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "dense decode W8A8 int8 g128 Hadamard, N=21504 K=5376, M in [1,4,8,16]",
+                   "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {rows} of {N_FULL} weight rows per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------------------
+# Secondary workloads (reported under "extras"; the headline is the W8A8 step)
+# --------------------------------------------------------------------------
+def _traced(Q, fn, iters, kind):
+    """Run fn(i) iters times with the library trace on; mean ms of `kind` launches."""
+    Q.ql_trace_enable(64 * iters)
+    for i in range(iters):
+        fn(i)
+    tr = Q.ql_trace_read(64 * iters)
+    Q.ql_trace_enable(0)
+    ks = [t for k, t in tr if k == kind]
+    return float(np.mean(ks)) if ks else None, len(tr) / iters
+
+
+def run_extras(torch, Q, synth, dev, stream, hbm):
+    out = {}
+    G = K_FULL // 128
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    with torch.cuda.stream(stream):
+        # weight-only decode, int4 g64 and int5 + zero point g128
+        for name, fmt in (("w4a16_decode", Q.I4_G64_BF16), ("w5a16_decode", Q.I5Z_G128_F16)):
+            d = synth.w4a16(16) if fmt == Q.I4_G64_BF16 else synth.w5a16(16)
+            z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None
+            c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
+                                      scales=torch.from_numpy(d["scales"].view(np.int16)).to(dev), zeros=z)
+            cp = [(c, s, zz)] + [(c.clone(), s.clone(), None if zz is None else zz.clone()) for _ in range(3)]
+            res = {}
+            for m in (1, 5, 16) if fmt == Q.I4_G64_BF16 else (1, 4, 16):
+                x = bf(synth.activations(0, f"x_M{m}", m, K_FULL))
+                y = torch.empty((m, N_FULL), dtype=torch.float32, device=dev)
+                ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, m, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
+                run = lambda i: Q.qlinear_forward(x, cp[i % 4][0], cp[i % 4][1], cp[i % 4][2], fmt, N_FULL,  # noqa
+                                                  y=y, ws=ws, stream=stream)
+                for i in range(8):
+                    run(i)
+                t, _ = _traced(Q, run, 40, "skinny")
+                cb, sb, zb = Q.qlinear_packed_sizes(fmt, N_FULL, K_FULL)
+                byts = cb + sb + zb + m * K_FULL * 2 + m * N_FULL * 4
+                res[str(m)] = {"us": 1e3 * t, "GB/s": byts / (t * 1e-3) / 1e9, "frac": byts / (t * 1e-3) / 1e9 / hbm}
+            out[name] = res
+            del cp, c, s, zz
+        # MoE gate_up, int8 Hadamard-domain experts, decode batches
+        E, topk, Ke, Ne = 128, 8, 2816, 1408
+        Ws = synth.moe_gate_up(1, experts=range(E))["W"]
+        codes = torch.empty((E, Ne, Ke), dtype=torch.int8, device=dev)
+        scales = torch.empty((E, Ne, Ke // 128), dtype=torch.int16, device=dev)
+        for e in range(E):
+            c, s, _ = Q.qlinear_pack(Q.I8_G128_BF16, Ne, Ke, W=torch.from_numpy(Ws[e]).to(dev), flags=Q.HADAMARD)
+            codes[e] = c.view(torch.int8).reshape(Ne, Ke)
+            scales[e] = s.view(torch.int16).reshape(Ne, Ke // 128)
+        del Ws
+        res = {}
+        for T in (1, 8, 16):
+            batches = []
+            for b in range(8):
+                ids, w = synth.routing(100 + b, T, E, topk)
+                batches.append((bf(synth.activations(b, f"x_T{T}", T, Ke)), torch.from_numpy(ids).to(dev),
+                                len(set(ids.ravel().tolist()))))
+            y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+            run = lambda i: Q.moe_gate_up(batches[i % 8][0], batches[i % 8][1], codes, scales, E, Ne, y=y,  # noqa
+                                          stream=stream)
+            for i in range(8):
+                run(i)
+            t, per = _traced(Q, run, 40, "moe_gemm")
+            touched = float(np.mean([b[2] for b in batches]))
+            byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
+            res[str(T)] = {"us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
+                           "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per}
+        out["moe_gate_up_decode"] = res
+        del codes, scales
+    torch.cuda.synchronize()
+    return out
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    from moe_hadamard128_act_b200 import build as qbuild
+    from moe_hadamard128_act_b200 import qlinear as Q
+    from moe_hadamard128_act_b200 import synth
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    if rank == 0:
+        qbuild.build()
+    if world > 1:
+        dist.barrier()
+    Q.lib()
+    dev = torch.device("cuda", local)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    # ---- inputs: the weight packed on the GPU from the seeded fp32 draw ----
+    W = torch.from_numpy(synth.weight_rows(0, "W", K_FULL, 0, N_FULL)).to(dev)
+    codes0, scales0, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N_FULL, K_FULL, W=W, flags=Q.HADAMARD)
+    del W
+    copies = [(codes0, scales0)] + [(codes0.clone(), scales0.clone()) for _ in range(COPIES - 1)]
+    xs_host = {m: synth.activations(0, f"x_M{m}", m, K_FULL, outlier_frac=0.01) for m in MS}
+    xs = {m: torch.from_numpy(xs_host[m].view(np.int16)).view(torch.bfloat16).to(dev) for m in MS}
+    ys = {m: torch.empty((m, N_FULL), dtype=torch.float32, device=dev) for m in MS}
+    ws = torch.empty(Q.qlinear_workspace_size(Q.I8A8_G128_BF16, Q.HADAMARD, 16, N_FULL, K_FULL), dtype=torch.uint8,
+                     device=dev)
+    L = Q.lib()
+    stream = torch.cuda.Stream(device=dev)
+
+    def forward_args(i, m, s):
+        c, sc = copies[i % COPIES]
+        return (ctypes.c_void_p(xs[m].data_ptr()), ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(sc.data_ptr()),
+                None, Q.I8A8_G128_BF16, Q.HADAMARD, m, N_FULL, K_FULL, ctypes.c_void_p(ys[m].data_ptr()),
+                ctypes.c_void_p(ws.data_ptr()), ws.numel(), ctypes.c_void_p(s.cuda_stream))
+
+    calls = [forward_args(i, m, stream) for i, m in enumerate(MS)]
+
+    def step():
+        for a in calls:
+            st = L.qlinear_forward(*a)
+            if st:
+                raise Q.QLError("qlinear_forward", st)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+
+    # ---- graph of S steps with the launch trace captured in it ----
+    S = max(d for d in range(1, min(args.steps, 50) + 1) if args.steps % d == 0)
+    R = args.steps // S
+    launches_per_step = 2 * len(MS)
+    Q.ql_trace_enable(S * launches_per_step)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(S):
+                step()
+    g.replay()  # untimed graph warm-up
+    stream.synchronize()
+
+    # clocks pre-roll: about a second of the same load while nvidia-smi samples
+    per_replay = None
+    with ClockSampler(local) as clk:
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < 1.0:
+            g.replay()
+            n += 1
+            if n % 10 == 0:
+                stream.synchronize()
+        stream.synchronize()
+        per_replay = (time.perf_counter() - t0) / n
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(R):
+            g.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    trace = Q.ql_trace_read(S * launches_per_step)
+    Q.ql_trace_enable(0)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    value = world * args.steps * step_bytes() / (ms * 1e-3) / 1e9
+
+    # ---- roofline of the dominant kernel (the skinny GEMM) from the trace ----
+    hbm, bf16_tf, peak_src = peaks()
+    sk = [t for k, t in trace if k == "skinny"]
+    sk_bytes = [skinny_bytes(MS[i % len(MS)]) for i in range(len(sk))]
+    sk_ms = float(np.sum(sk))
+    achieved = float(np.sum(sk_bytes)) / (sk_ms * 1e-3) / 1e9 if sk_ms > 0 else None
+    share = sk_ms / max(1e-9, float(np.sum([t for _, t in trace])))
+    traffic = kernel_traffic("skinny_w8a8_decode", ROOT / "moe_hadamard128_act_b200" / "csrc" / "k_skinny.cu")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm if achieved else None, "traffic": traffic,
+                "kernel": "k_skinny<W8A8>", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "share_of_traced_time": share,
+                "per_m_us": {str(m): 1e3 * float(np.mean(sk[i::len(MS)])) for i, m in enumerate(MS)}}
+
+    # ---- end to end through the C ABI with host buffers ----
+    e2e_steps = min(args.steps, 200)
+    xh = {m: torch.from_numpy(xs_host[m].view(np.int16)).view(torch.bfloat16).pin_memory() for m in MS}
+    yh = {m: torch.empty((m, N_FULL), dtype=torch.float32).pin_memory() for m in MS}
+    h2d = sum(m * K_FULL * 2 for m in MS)
+    d2h = sum(m * N_FULL * 4 for m in MS)
+    with torch.cuda.stream(stream):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(e2e_steps):
+            for j, m in enumerate(MS):
+                xs[m].copy_(xh[m], non_blocking=True)
+                st = L.qlinear_forward(*calls[j])
+                if st:
+                    raise Q.QLError("qlinear_forward", st)
+                yh[m].copy_(ys[m], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e = {"value": world * e2e_steps * step_bytes() / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    extras = None
+    if not args.no_extras:
+        del copies, codes0, scales0
+        torch.cuda.empty_cache()
+        extras = run_extras(torch, Q, synth, dev, stream, hbm)
+
+    st, bits = Q.ql_get_device_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error word set: {bits}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8 x int8 -> int32 (fp32 scales)", "data": "synthetic",
+            "config": {"workload": "dense decode W8A8 int8 g128 Hadamard, N=21504 K=5376, M in [1,4,8,16]",
+                       "parallelism": f"replicas x{world}", "l2": f"{COPIES} rotating weight copies (470 MB > L2)",
+                       "graph_steps": S, "frac_of_hbm": value / world / hbm},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * launches_per_step,
+            "clocks": clk.summary(),
+            "extras": extras,
+        }
+        print(json.dumps(out), flush=True)
+    del g
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+// k_act.cu -- activation-side kernels: the 128-wide Walsh-Hadamard rotation
+// ("transform=fwht128" of the int8 experts in "gemma4-26b-a4b-dflash-i8"), the
+// fused rotation + int8 quantiser with one scale per token per 128 values
+// ("keptn/gemma4-12b-i8g", table "Format"), and the preparation of bf16
+// activations for the weight-only skinny GEMM.
+//
+// Both transform kernels put one warp on one (token, 128-group): each lane
+// loads 4 consecutive bf16 (8 bytes, so a warp reads one 256-byte group fully
+// coalesced), the butterflies run in registers and through warp shuffles, and
+// the max for the quantiser is a shuffle reduction.  They are bound by HBM
+// (2 bytes in and 2 or 1 + 4/128 bytes out per element).
+#include "ql_device.cuh"
+#include "ql_internal.h"
+
+namespace ql {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+__device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float v[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(raw.x << 16);
+    v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(raw.y << 16);
+    v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_rotate_bf16(const __nv_bfloat16* x, int M, int K,
+                                                                     __nv_bfloat16* y) {
+    const int lane = threadIdx.x & 31;
+    const long long G = K / 128;
+    const long long nw = (long long)gridDim.x * kWarpsPerBlock;
+    for (long long u = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); u < (long long)M * G; u += nw) {
+        const long long off = (u / G) * K + (u % G) * 128 + 4 * lane;
+        float v[4];
+        load4_bf16(x + off, v);
+        fwht128_warp(v, lane);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 out;
+        out.x = *reinterpret_cast<const uint32_t*>(&lo);
+        out.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(y + off) = out;
+    }
+}
+
+// Grid-stride zero of y[0 .. n) (16-byte stores; y is 16-byte aligned).
+__device__ __forceinline__ void zero_fill(float* y, long long n) {
+    if (!y) return;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    float4* y4 = reinterpret_cast<float4*>(y);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n / 4; i += stride)
+        y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (long long i = (n & ~3LL) + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) y[i] = 0.f;
+}
+
+// s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127).
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bfloat16* x, int M, int K, int rotate,
+                                                                   int8_t* q, float* sx, float* yz, long long nz) {
+    zero_fill(yz, nz);  // the GEMM that follows accumulates into y
+    const int lane = threadIdx.x & 31;
+    const long long G = K / 128;
+    const long long nw = (long long)gridDim.x * kWarpsPerBlock;
+    for (long long u = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); u < (long long)M * G; u += nw) {
+        const long long off = (u / G) * K + (u % G) * 128 + 4 * lane;
+        float v[4];
+        load4_bf16(x + off, v);
+        if (rotate) fwht128_warp(v, lane);
+        float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+        amax = warp_max(amax);
+        uint32_t packed = 0;
+        float s = 0.0f;
+        if (amax > 0.0f) {
+            s = __fdiv_rn(amax, 127.0f);
+            const float inv = __fdiv_rn(127.0f, amax);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int c = __float2int_rn(__fmul_rn(v[i], inv));
+                c = max(-127, min(127, c));
+                packed |= (uint32_t)(c & 0xFF) << (8 * i);
+            }
+        }
+        *reinterpret_cast<uint32_t*>(q + off) = packed;
+        if (lane == 0) sx[u] = s;  // [M][G] row-major: u = m * G + g
+    }
+}
+
+// One CTA per token.  The (optionally rotated and bf16-rounded) row is kept in
+// shared memory as fp32; its max |x| picks a power of two f with
+// max|x| * f in [2^14, 2^15), and xs = f16(x * f) is written in the element
+// order of the format (within each 8-block [0,4,1,5,2,6,3,7] for int4, within
+// each 4-block [0,3,1,2] for int5, natural otherwise).  xf = 1 / f.
+// f16 holds every bf16 value of the scaled row exactly down to 2^-14 (its
+// normal range); below that the rounding error is under 2^-39 of the row's
+// max, far beneath the fp32 accumulation error of the GEMM.
+__global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K, int rotate, int order, __half* xs,
+                                                  float* xf, float* yz, long long nz) {
+    extern __shared__ float row[];
+    zero_fill(yz, nz);  // the GEMM that follows accumulates into y
+    __shared__ float red[8];
+    const int t = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const __nv_bfloat16* xr = x + (long long)t * K;
+    float amax = 0.0f;
+    for (int g = warp; g < K / 128; g += 8) {
+        float v[4];
+        load4_bf16(xr + g * 128 + 4 * lane, v);
+        if (rotate) {
+            fwht128_warp(v, lane);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            row[g * 128 + 4 * lane + i] = v[i];
+            amax = fmaxf(amax, fabsf(v[i]));
+        }
+    }
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = red[0];
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+        int e = 0;
+        if (m > 0.0f && m <= 3.4e38f) frexpf(m, &e);
+        e = max(-100, min(128, e));
+        red[0] = ldexpf(1.0f, 15 - e);
+        xf[t] = ldexpf(1.0f, e - 15);
+    }
+    __syncthreads();
+    const float f = red[0];
+    __half* out = xs + (long long)t * K;
+    for (int k = threadIdx.x; k < K; k += 256) {
+        int src = k;
+        if (order == XORD_I4) {
+            const int p = k & 7;
+            src = (k & ~7) + ((p & 1) ? 4 + (p >> 1) : (p >> 1));
+        } else if (order == XORD_I5) {
+            const int p = k & 3;
+            src = (k & ~3) + (p == 0 ? 0 : (p == 1 ? 3 : p - 1));
+        }
+        out[k] = __float2half_rn(__fmul_rn(row[src], f));
+    }
+}
+
+int grid_for(long long warps, int sm_count) {
+    long long blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    long long cap = (long long)sm_count * 16;
+    return (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_rotate_bf16(const void* x, int M, int K, void* y, cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    k_rotate_bf16<<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), M, K, static_cast<__nv_bfloat16*>(y));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* yz, long long nz,
+                             cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    k_act_quant<<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, yz, nz);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
+                            long long nz, cudaStream_t s) {
+    const size_t smem = (size_t)K * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_prep_a16<<<M, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, order, xs, xf, yz, nz);
+    return cudaGetLastError();
+}
+
+}  // namespace ql

@@ -1,0 +1,454 @@
+// ql_api.cu -- the C ABI of libqlinear.so (declared in include/qlinear.h):
+// argument validation on the host, workspace carving, and the launch order
+// of the kernels of each call.  Every check happens before the first launch;
+// a rejected call enqueues nothing.
+#include <cstring>
+#include <new>
+
+#include "ql_internal.h"
+
+namespace ql {
+
+// The per-process device error word (one per device context).
+__device__ unsigned g_ql_err;
+
+void packed_sizes(int fmt, size_t N, size_t K, size_t* codes, size_t* scales, size_t* zeros) {
+    *codes = N * fmt_row_bytes(fmt, K);
+    *zeros = fmt == QL_I5Z_G128_F16 ? N * (K / 128) : 0;
+    if (fmt == QL_FP8_B128_BF16) *scales = ((N + 127) / 128) * (K / 128) * 2;
+    else *scales = N * (K / fmt_group(fmt)) * 2;
+}
+
+cudaError_t device_info(DeviceInfo* out) {
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && have[dev]) {
+        *out = cache[dev];
+        return cudaSuccess;
+    }
+    DeviceInfo d;
+    int v = 0;
+    if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    d.sm_count = v;
+    if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+    d.smem_optin = (size_t)v;
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_ql_err)) != cudaSuccess) return e;
+    d.err_word = static_cast<unsigned*>(p);
+    if (dev < 64) {
+        cache[dev] = d;
+        have[dev] = true;
+    }
+    *out = d;
+    return cudaSuccess;
+}
+
+// ---- launch trace -------------------------------------------------------------------
+namespace {
+struct TraceSlot {
+    int kind;
+    cudaEvent_t start, stop;
+};
+TraceSlot* g_slots = nullptr;
+int g_capacity = 0, g_used = 0;
+
+void trace_free() {
+    for (int i = 0; i < g_capacity; ++i) {
+        cudaEventDestroy(g_slots[i].start);
+        cudaEventDestroy(g_slots[i].stop);
+    }
+    delete[] g_slots;
+    g_slots = nullptr;
+    g_capacity = g_used = 0;
+}
+}  // namespace
+
+int trace_begin(int kind, cudaStream_t s) {
+    if (g_used >= g_capacity) return -1;
+    const int slot = g_used++;
+    g_slots[slot].kind = kind;
+    cudaEventRecord(g_slots[slot].start, s);
+    return slot;
+}
+
+void trace_end(int slot, cudaStream_t s) {
+    if (slot >= 0) cudaEventRecord(g_slots[slot].stop, s);
+}
+
+}  // namespace ql
+
+using namespace ql;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? QL_OK : QL_ECUDA; }
+
+// Activations prepared for the skinny GEMM: f16 [M][K] + factors [M] (A16), or
+// int8 [M][K] + fp32 scales [M][K/128] (W8A8).
+struct FwdWs {
+    size_t x_bytes, f_bytes;
+    size_t total() const { return x_bytes + f_bytes; }
+};
+FwdWs forward_ws(int fmt, size_t M, size_t K) {
+    FwdWs w;
+    if (fmt == QL_I8A8_G128_BF16) {
+        w.x_bytes = align_up(M * K, 256);
+        w.f_bytes = align_up(M * (K / 128) * 4, 256);
+    } else {
+        w.x_bytes = align_up(M * K * 2, 256);
+        w.f_bytes = align_up(M * 4, 256);
+    }
+    return w;
+}
+
+int x_order(int fmt) {
+    return fmt == QL_I4_G64_BF16 ? XORD_I4 : (fmt == QL_I5Z_G128_F16 ? XORD_I5 : XORD_NATURAL);
+}
+
+struct MoeWs {
+    size_t xs, xf, counts, offsets, perm, chunks, nch;
+    size_t total;
+};
+MoeWs moe_ws(const ql_experts* ex, int T, int topk) {
+    MoeWs w;
+    size_t o = 0;
+    w.xs = o; o += align_up((size_t)T * ex->K * 2, 256);
+    w.xf = o; o += align_up((size_t)T * 4, 256);
+    w.counts = o; o += align_up((size_t)ex->E * 4, 256);
+    w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
+    w.perm = o; o += align_up((size_t)T * topk * 4, 256);
+    w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
+    w.nch = o; o += 256;
+    w.total = o;
+    return w;
+}
+
+int check_experts(const ql_experts* ex) {
+    if (!ex) return QL_EINVAL;
+    if (ex->E < 1 || ex->E > 1024 || ex->N < 1 || ex->K < 128 || ex->K % 128) return QL_EINVAL;
+    if (ex->flags & ~QL_HADAMARD) return QL_EINVAL;
+    if (!fmt_valid(ex->fmt)) return QL_EINVAL;
+    if (ex->fmt != QL_I8_G128_BF16 && ex->fmt != QL_I8_G128_F16 && ex->fmt != QL_FP8_B128_BF16) return QL_EUNSUPPORTED;
+    if (!ex->codes || !ex->scales) return QL_EINVAL;
+    if (!aligned16(ex->codes) || !aligned16(ex->scales)) return QL_EALIGN;
+    return QL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ql_status_string(int status) {
+    switch (status) {
+    case QL_OK: return "ok";
+    case QL_EINVAL: return "invalid argument";
+    case QL_EUNSUPPORTED: return "unsupported format or mode";
+    case QL_EALIGN: return "device pointer not 16-byte aligned";
+    case QL_EWORKSPACE: return "workspace missing or too small";
+    case QL_ECUDA: return "CUDA runtime error";
+    case QL_EDEVICE: return "device error word set";
+    }
+    return "unknown status";
+}
+
+int qlinear_packed_sizes(int fmt, int N, int K, size_t* codes_bytes, size_t* scales_bytes, size_t* zeros_bytes) {
+    if (!fmt_valid(fmt) || N < 1 || K < 128 || K % 128 || !codes_bytes || !scales_bytes || !zeros_bytes)
+        return QL_EINVAL;
+    packed_sizes(fmt, (size_t)N, (size_t)K, codes_bytes, scales_bytes, zeros_bytes);
+    return QL_OK;
+}
+
+int qlinear_pack(const float* W, const void* codes_in, const void* scales_in, const uint8_t* zeros_in, int fmt,
+                 int flags, int N, int K, void* codes_out, void* scales_out, uint8_t* zeros_out, void* stream) {
+    if (!fmt_valid(fmt) || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
+    if (!codes_out || !scales_out) return QL_EINVAL;
+    if ((W == nullptr) == (codes_in == nullptr)) return QL_EINVAL;  // exactly one source
+    if (!aligned16(codes_out) || !aligned16(scales_out)) return QL_EALIGN;
+    if (fmt == QL_I5Z_G128_F16) {
+        if (!zeros_out) return QL_EINVAL;
+        if (!aligned16(zeros_out)) return QL_EALIGN;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    size_t cb, sb, zb;
+    packed_sizes(fmt, N, K, &cb, &sb, &zb);
+    if (W) {
+        if (!aligned16(W)) return QL_EALIGN;
+        if (fmt == QL_I5Z_G128_F16) return QL_EUNSUPPORTED;
+        const int t = trace_begin(QL_KIND_PACK, s);
+        const cudaError_t e = launch_pack_rtn(W, fmt, flags, N, K, codes_out, scales_out, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
+    if (!scales_in) return QL_EINVAL;
+    if (!aligned16(codes_in) || !aligned16(scales_in)) return QL_EALIGN;
+    if (fmt == QL_I5Z_G128_F16) {
+        if (!zeros_in) return QL_EINVAL;
+        if (!aligned16(zeros_in)) return QL_EALIGN;
+    }
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return QL_ECUDA;
+    int t = trace_begin(QL_KIND_PACK, s);
+    e = launch_pack_codes(codes_in, fmt, N, K, codes_out, di.err_word, s);
+    trace_end(t, s);
+    if (e != cudaSuccess) return QL_ECUDA;
+    if ((e = cudaMemcpyAsync(scales_out, scales_in, sb, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return QL_ECUDA;
+    if (fmt == QL_I5Z_G128_F16) {
+        t = trace_begin(QL_KIND_PACK, s);
+        e = launch_check_zeros(zeros_in, zb, zeros_out, di.err_word, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
+    return QL_OK;
+}
+
+int qlinear_workspace_size(int fmt, int flags, int M, int N, int K, size_t* bytes) {
+    if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD) || !bytes)
+        return QL_EINVAL;
+    *bytes = forward_ws(fmt, M, K).total();
+    return QL_OK;
+}
+
+int qlinear_forward(const void* x, const void* W_packed, const void* scales, const uint8_t* zeros, int fmt,
+                    int flags, int M, int N, int K, float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
+    if (!x || !W_packed || !scales || !y) return QL_EINVAL;
+    if (fmt == QL_I5Z_G128_F16 && !zeros) return QL_EINVAL;
+    if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y) ||
+        (zeros && !aligned16(zeros)))
+        return QL_EALIGN;
+    const FwdWs w = forward_ws(fmt, M, K);
+    if (!ws || ws_bytes < w.total()) return QL_EWORKSPACE;
+    if (!aligned16(ws)) return QL_EALIGN;
+    const int kmax = skinny_max_k(fmt);
+    if (kmax < 128) return QL_ECUDA;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int G = K / 128;
+    const int rot = (flags & QL_HADAMARD) ? 1 : 0;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    void* xs = wsb;
+    float* xf = reinterpret_cast<float*>(wsb + w.x_bytes);
+    cudaError_t e;
+    const long long ny = (long long)M * N;  // the prologue zeroes y for the accumulating GEMM
+    if (fmt == QL_I8A8_G128_BF16) {
+        const int t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, y, ny, s);
+        trace_end(t, s);
+    } else {
+        const int t = trace_begin(QL_KIND_PREP_A16, s);
+        e = launch_prep_a16(x, M, K, rot, x_order(fmt), static_cast<__half*>(xs), xf, y, ny, s);
+        trace_end(t, s);
+    }
+    if (e != cudaSuccess) return QL_ECUDA;
+
+    const size_t xelem = fmt == QL_I8A8_G128_BF16 ? 1 : 2;
+    for (int m0 = 0; m0 < M; m0 += 16) {
+        for (int k0 = 0; k0 < K; k0 += kmax) {
+            const int kc = K - k0 < kmax ? K - k0 : kmax;
+            SkinnyArgs a;
+            a.W = static_cast<const uint8_t*>(W_packed) + fmt_row_bytes(fmt, k0);
+            a.scales = scales;
+            a.zeros = zeros;
+            a.xs = static_cast<const uint8_t*>(xs) + ((size_t)m0 * K + k0) * xelem;
+            a.xf = fmt == QL_I8A8_G128_BF16 ? xf + (size_t)m0 * G : xf + m0;
+            a.y = y + (size_t)m0 * N;
+            a.acc = nullptr;
+            a.M = M - m0 < 16 ? M - m0 : 16;
+            a.N = N;
+            a.G = kc / 128;
+            a.g0 = k0 / 128;
+            a.Gtot = G;
+            a.ldw = (long long)fmt_row_bytes(fmt, K);
+            a.ldx = K;
+            a.ldy = N;
+            const int t = trace_begin(QL_KIND_SKINNY, s);
+            e = launch_skinny(fmt, a, s);
+            trace_end(t, s);
+            if (e != cudaSuccess) return QL_ECUDA;
+        }
+    }
+    return QL_OK;
+}
+
+int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int K, int32_t* acc, void* stream) {
+    if (M < 1 || N < 1 || K < 128 || K % 128 || !qx || !qw || !acc) return QL_EINVAL;
+    if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return QL_EALIGN;
+    const int kmax = skinny_max_k(QL_I8A8_G128_BF16);
+    if (kmax < 128) return QL_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int G = K / 128;
+    for (int m0 = 0; m0 < M; m0 += 16) {
+        for (int k0 = 0; k0 < K; k0 += kmax) {
+            const int kc = K - k0 < kmax ? K - k0 : kmax;
+            SkinnyArgs a;
+            std::memset(&a, 0, sizeof a);
+            a.W = reinterpret_cast<const uint8_t*>(qw) + k0;
+            a.xs = qx + (size_t)m0 * K + k0;
+            a.xf = nullptr;
+            a.acc = acc + (size_t)m0 * N * G;
+            a.M = M - m0 < 16 ? M - m0 : 16;
+            a.N = N;
+            a.G = kc / 128;
+            a.g0 = k0 / 128;
+            a.Gtot = G;
+            a.ldw = K;
+            a.ldx = K;
+            a.ldy = N;
+            const int t = trace_begin(QL_KIND_SKINNY, s);
+            cudaError_t e = launch_skinny(QL_I8A8_G128_BF16, a, s);
+            trace_end(t, s);
+            if (e != cudaSuccess) return QL_ECUDA;
+        }
+    }
+    return QL_OK;
+}
+
+int act_quant_i8_g128(const void* x, int M, int K, int rotate, int8_t* q, float* s, void* stream) {
+    if (M < 1 || K < 128 || K % 128 || !x || !q || !s) return QL_EINVAL;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return QL_EALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int t = trace_begin(QL_KIND_ACT_QUANT, st);
+    const cudaError_t e = launch_act_quant(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, st);
+    trace_end(t, st);
+    return from_cuda(e);
+}
+
+int hadamard128_rotate(const void* x, int M, int K, void* y, void* stream) {
+    if (M < 1 || K < 128 || K % 128 || !x || !y) return QL_EINVAL;
+    if (!aligned16(x) || !aligned16(y)) return QL_EALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int t = trace_begin(QL_KIND_ROTATE, st);
+    const cudaError_t e = launch_rotate_bf16(x, M, K, y, st);
+    trace_end(t, st);
+    return from_cuda(e);
+}
+
+int moe_permute(const int32_t* topk_ids, int T, int topk, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
+                void* stream) {
+    if (T < 1 || topk < 1 || topk > 64 || E < 1 || E > 1024 || !topk_ids || !counts || !offsets || !perm)
+        return QL_EINVAL;
+    if (!aligned16(topk_ids) || !aligned16(counts) || !aligned16(offsets) || !aligned16(perm)) return QL_EALIGN;
+    // Standalone permutation: the chunk table the grouped GEMM uses is not requested.
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return QL_ECUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int t = trace_begin(QL_KIND_MOE_PERMUTE, st);
+    const cudaError_t e = launch_moe_permute(topk_ids, T, topk, E, counts, offsets, perm, nullptr, nullptr, di.err_word, st);
+    trace_end(t, st);
+    return from_cuda(e);
+}
+
+int moe_workspace_size(const ql_experts* experts, int T, int topk, size_t* bytes) {
+    int st = check_experts(experts);
+    if (st != QL_OK) return st;
+    if (T < 1 || topk < 1 || topk > 64 || !bytes) return QL_EINVAL;
+    *bytes = moe_ws(experts, T, topk).total;
+    return QL_OK;
+}
+
+int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weights, const ql_experts* experts, int T,
+                int topk, float* y, void* ws, size_t ws_bytes, void* stream) {
+    (void)topk_weights;  // applied after the down projection, not here
+    int st = check_experts(experts);
+    if (st != QL_OK) return st;
+    if (T < 1 || topk < 1 || topk > 64 || !x || !topk_ids || !y) return QL_EINVAL;
+    if (!aligned16(x) || !aligned16(topk_ids) || !aligned16(y)) return QL_EALIGN;
+    const MoeWs w = moe_ws(experts, T, topk);
+    if (!ws || ws_bytes < w.total) return QL_EWORKSPACE;
+    if (!aligned16(ws)) return QL_EALIGN;
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return QL_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    __half* xs = reinterpret_cast<__half*>(b + w.xs);
+    float* xf = reinterpret_cast<float*>(b + w.xf);
+    int32_t* counts = reinterpret_cast<int32_t*>(b + w.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(b + w.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + w.perm);
+    MoeChunk* chunks = reinterpret_cast<MoeChunk*>(b + w.chunks);
+    int* nch = reinterpret_cast<int*>(b + w.nch);
+    const int K = experts->K, N = experts->N;
+    cudaError_t e;
+    int t = trace_begin(QL_KIND_PREP_A16, s);  // rotation, f16 staging, and the zeroing of y
+    e = launch_prep_a16(x, T, K, (experts->flags & QL_HADAMARD) ? 1 : 0, XORD_NATURAL, xs, xf, y,
+                        (long long)T * topk * N, s);
+    trace_end(t, s);
+    if (e != cudaSuccess) return QL_ECUDA;
+    t = trace_begin(QL_KIND_MOE_PERMUTE, s);
+    e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, chunks, nch, di.err_word, s);
+    trace_end(t, s);
+    if (e != cudaSuccess) return QL_ECUDA;
+    MoeArgs a;
+    a.codes = static_cast<const uint8_t*>(experts->codes);
+    a.scales = experts->scales;
+    a.xs = xs;
+    a.xf = xf;
+    a.perm = perm;
+    a.chunks = chunks;
+    a.n_chunks = nch;
+    a.y = y;
+    a.fmt = experts->fmt;
+    a.T = T;
+    a.topk = topk;
+    a.E = experts->E;
+    a.N = N;
+    a.K = K;
+    a.max_chunks = (long long)moe_max_chunks(T, topk, experts->E);
+    t = trace_begin(QL_KIND_MOE_GEMM, s);
+    e = launch_moe_skinny(a, s);
+    trace_end(t, s);
+    return from_cuda(e);
+}
+
+int ql_trace_enable(int capacity) {
+    if (capacity < 0 || capacity > (1 << 20)) return QL_EINVAL;
+    trace_free();
+    if (capacity == 0) return QL_OK;
+    g_slots = new (std::nothrow) TraceSlot[capacity];
+    if (!g_slots) return QL_EINVAL;
+    for (int i = 0; i < capacity; ++i) {
+        if (cudaEventCreate(&g_slots[i].start) != cudaSuccess || cudaEventCreate(&g_slots[i].stop) != cudaSuccess) {
+            g_capacity = i;
+            trace_free();
+            return QL_ECUDA;
+        }
+    }
+    g_capacity = capacity;
+    g_used = 0;
+    return QL_OK;
+}
+
+int ql_trace_read(int* kinds, float* ms, int max, int* count) {
+    if (!count || max < 0 || (max > 0 && (!kinds || !ms))) return QL_EINVAL;
+    const int n = g_used < max ? g_used : max;
+    for (int i = 0; i < n; ++i) {
+        if (cudaEventSynchronize(g_slots[i].stop) != cudaSuccess) return QL_ECUDA;
+        float t = 0.0f;
+        if (cudaEventElapsedTime(&t, g_slots[i].start, g_slots[i].stop) != cudaSuccess) return QL_ECUDA;
+        kinds[i] = g_slots[i].kind;
+        ms[i] = t;
+    }
+    *count = g_used;
+    return QL_OK;
+}
+
+int ql_get_device_error(void* stream, unsigned* bits) {
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return QL_ECUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QL_ECUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, di.err_word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return QL_ECUDA;
+    if (v) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(di.err_word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return QL_ECUDA;
+    }
+    if (bits) *bits = v;
+    return v ? QL_EDEVICE : QL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// ql_internal.h -- host-side interface between the C-ABI layer (ql_api.cu)
+// and the kernel translation units.  Nothing here is exported.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+// ---- format arithmetic -------------------------------------------------------
+inline bool fmt_valid(int f) { return f >= QL_I8_G128_BF16 && f <= QL_FP8_B128_BF16; }
+inline bool fmt_scale_f16(int f) { return f == QL_I8_G128_F16 || f == QL_I5Z_G128_F16; }
+inline int fmt_group(int f) { return f == QL_I4_G64_BF16 ? 64 : 128; }
+// Bytes of one packed row of K codes.
+inline size_t fmt_row_bytes(int f, size_t K) {
+    switch (f) {
+    case QL_I4_G64_BF16: return K / 2;
+    case QL_I5Z_G128_F16: return K * 5 / 8;
+    default: return K;
+    }
+}
+void packed_sizes(int fmt, size_t N, size_t K, size_t* codes, size_t* scales, size_t* zeros);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Per-device facts, cached on first use.
+struct DeviceInfo {
+    int sm_count;
+    size_t smem_optin;   // max dynamic shared memory per block (opt-in)
+    unsigned* err_word;  // device address of the error word
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// ---- activations ---------------------------------------------------------------
+// Prepared activations for the weight-only (A16) skinny GEMM: f16 copy of x
+// scaled per token by a power of two, in the element order the format's MMA
+// fragments want; xf[t] = the inverse power of two.
+enum XOrder { XORD_NATURAL = 0, XORD_I4 = 1, XORD_I5 = 2 };
+cudaError_t launch_rotate_bf16(const void* x, int M, int K, void* y, cudaStream_t s);
+// The act-quant and prep kernels also zero y[0 .. nz) (yz may be null), so the
+// skinny GEMM that follows can accumulate into it without a separate launch.
+cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* yz, long long nz,
+                             cudaStream_t s);
+cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
+                            long long nz, cudaStream_t s);
+
+// ---- packing ---------------------------------------------------------------------
+cudaError_t launch_pack_rtn(const float* W, int fmt, int flags, int N, int K, void* codes, void* scales,
+                            cudaStream_t s);
+cudaError_t launch_pack_codes(const void* codes_in, int fmt, int N, int K, void* codes_out, unsigned* err,
+                              cudaStream_t s);
+cudaError_t launch_check_zeros(const uint8_t* z_in, size_t n, uint8_t* z_out, unsigned* err, cudaStream_t s);
+
+// ---- skinny GEMM (M <= 16 per launch) -----------------------------------------------
+struct SkinnyArgs {
+    const uint8_t* W;      // packed codes, row stride ldw bytes; already offset to group g0
+    const void* scales;    // [N][Gtot] (fp8: [N/128][Gtot]); indexed with g0 + g
+    const uint8_t* zeros;  // int5: [N][Gtot]
+    const void* xs;        // prepared activations, row stride ldx elements; offset to group g0
+    const float* xf;       // A16: [M] inverse token factors; W8A8: sx [M][Gtot]
+    float* y;              // [M][ldy]
+    int32_t* acc;          // optional W8A8 group sums [M][N][Gtot]
+    int M, N, G, g0, Gtot;
+    long long ldw, ldx, ldy;
+};
+cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s);
+// Largest K (multiple of 128) one skinny launch stages in shared memory.
+int skinny_max_k(int fmt);
+
+// ---- MoE -----------------------------------------------------------------------------------
+struct MoeChunk {
+    int expert, start, count;  // rows perm[start .. start+count) of the permuted order
+};
+size_t moe_max_chunks(int T, int topk, int E);
+cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,
+                               int32_t* perm, MoeChunk* chunks, int* n_chunks, unsigned* err, cudaStream_t s);
+struct MoeArgs {
+    const uint8_t* codes;  // [E][N][K]
+    const void* scales;    // [E][...] per the format
+    const __half* xs;      // prepared activations [T][K] (natural order)
+    const float* xf;       // [T]
+    const int32_t* perm;   // [T*topk]
+    const MoeChunk* chunks;
+    const int* n_chunks;
+    float* y;              // [T*topk][N]
+    int fmt, T, topk, E, N, K;
+    long long max_chunks;
+};
+cudaError_t launch_moe_skinny(const MoeArgs& a, cudaStream_t s);
+
+// ---- launch trace (ql_trace_enable / ql_trace_read) --------------------------------------
+// trace_begin records a start event for one library launch when tracing is on
+// and returns its slot (or -1); trace_end records the matching stop event.
+int trace_begin(int kind, cudaStream_t s);
+void trace_end(int slot, cudaStream_t s);
+
+}  // namespace ql

@@ -5,15 +5,15 @@ layer's arithmetic (no transform, no quantiser, no packing, no matmul).  Both
 the CUDA path and the CPU oracle consume exactly the arrays it returns, so
 both sides see identical inputs.
 
-Generator: a counter-based splitmix64.  Value i of stream `name` under seed
-`seed` is mix64(key(seed, name) + (i + 1) * 0x9E3779B97F4A7C15), where mix64
-is the splitmix64 output function (Steele, Lea and Flood, "Fast splittable
-pseudorandom number generators", OOPSLA 2014).  Uniform doubles take the top
-53 bits; normals come from the Box-Muller transform of the uniform pair
-(2p, 2p+1): value 2p is the cosine branch, value 2p+1 the sine branch.
-Because every value is a function of its index, any slice of any tensor can
-be regenerated on its own (the parity tests use this to regenerate sampled
-weight rows at full size without drawing the whole matrix).
+Generator: a counter-based splitmix64 (synth_rng.c, compiled with gcc on first
+use).  Value i of stream `name` under seed `seed` is mix64(key + (i + 1) *
+0x9E3779B97F4A7C15), with key = mix64(FNV-1a(name) ^ seed * 0x9E37...) and
+mix64 the splitmix64 output function.  Uniform doubles take the top 53 bits;
+normals come from the Box-Muller transform of the uniform pair (2p, 2p+1):
+value 2p is the cosine branch, value 2p+1 the sine branch.  Because every
+value is a function of its index, computed with scalar libm calls, any slice of
+any tensor can be regenerated on its own, bit for bit (the parity tests use
+this to regenerate sampled weight rows at full size).
 
 Arrays come back as numpy: fp32 weights, and bf16 / f16 values as their
 uint16 bit patterns (rounded from the fp64 draw by torch / numpy casts, which
@@ -21,66 +21,77 @@ are input plumbing, not the method).
 """
 from __future__ import annotations
 
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
 import numpy as np
 import torch
 
-_GOLDEN = np.uint64(0x9E3779B97F4A7C15)
-_M1 = np.uint64(0xBF58476D1CE4E5B9)
-_M2 = np.uint64(0x94D049BB133111EB)
-_CHUNK = 1 << 22
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "synth_rng.c"
+_LIB = _HERE / "libsynth_rng.so"
+_rng = None
 
 
-def _mix(z: np.ndarray) -> np.ndarray:
-    z = (z ^ (z >> np.uint64(30))) * _M1
-    z = (z ^ (z >> np.uint64(27))) * _M2
-    return z ^ (z >> np.uint64(31))
+def build(force: bool = False) -> Path:
+    """Compile the generator (plain C, scalar libm, OpenMP over elements)."""
+    if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB.with_name(f"libsynth_rng.so.tmp{os.getpid()}")
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fno-fast-math", "-fPIC", "-shared", "-o", str(tmp),
+                               str(_SRC), "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
 
 
-def _key(seed: int, name: str) -> np.uint64:
+def _lib():
+    global _rng
+    if _rng is None:
+        build()
+        L = ctypes.CDLL(str(_LIB))
+        L.synth_mix64.restype = ctypes.c_uint64
+        L.synth_mix64.argtypes = [ctypes.c_uint64]
+        for name in ("synth_uniform01", "synth_normal"):
+            getattr(L, name).restype = None
+            getattr(L, name).argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
+        L.synth_uniform_int8.restype = None
+        L.synth_uniform_int8.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_void_p]
+        L.synth_normal_f32.restype = None
+        L.synth_normal_f32.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                                       ctypes.c_void_p]
+        _rng = L
+    return _rng
+
+
+def _key(seed: int, name: str) -> int:
     h = 0xCBF29CE484222325  # FNV-1a 64 of the stream name, mixed with the seed
     for ch in name.encode():
         h = ((h ^ ch) * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
-    with np.errstate(over="ignore"):
-        k = _mix(np.array([h ^ ((seed * 0x9E3779B97F4A7C15) & 0xFFFFFFFFFFFFFFFF)], np.uint64))
-    return k[0]
-
-
-def uniform_u64(seed: int, name: str, start: int, count: int) -> np.ndarray:
-    key = _key(seed, name)
-    out = np.empty(count, np.uint64)
-    with np.errstate(over="ignore"):
-        for a in range(0, count, _CHUNK):
-            b = min(count, a + _CHUNK)
-            ctr = np.arange(start + a + 1, start + b + 1, dtype=np.uint64)
-            out[a:b] = _mix(key + ctr * _GOLDEN)
-    return out
+    return _lib().synth_mix64(h ^ ((seed * 0x9E3779B97F4A7C15) & 0xFFFFFFFFFFFFFFFF))
 
 
 def uniform01(seed: int, name: str, start: int, count: int) -> np.ndarray:
-    u = uniform_u64(seed, name, start, count)
-    return (u >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
+    out = np.empty(count, np.float64)
+    _lib().synth_uniform01(_key(seed, name), start, count, out.ctypes.data)
+    return out
 
 
 def normal(seed: int, name: str, start: int, count: int) -> np.ndarray:
     """Standard normals with indices [start, start + count) of the stream."""
-    if count == 0:
-        return np.empty(0, np.float64)
-    p0 = start // 2
-    p1 = (start + count + 1) // 2
-    u = uniform01(seed, name, 2 * p0, 2 * (p1 - p0)).reshape(-1, 2)
-    r = np.sqrt(-2.0 * np.log1p(-u[:, 0]))
-    th = 2.0 * np.pi * u[:, 1]
-    z = np.empty((p1 - p0) * 2, np.float64)
-    z[0::2] = r * np.cos(th)
-    z[1::2] = r * np.sin(th)
-    off = start - 2 * p0
-    return z[off:off + count]
+    out = np.empty(count, np.float64)
+    _lib().synth_normal(_key(seed, name), start, count, out.ctypes.data)
+    return out
 
 
 def uniform_int(seed: int, name: str, lo: int, hi: int, shape) -> np.ndarray:
-    n = int(np.prod(shape))
-    u = uniform01(seed, name, 0, n)
-    return (lo + np.floor(u * (hi - lo + 1))).astype(np.int64).reshape(shape)
+    """Integers uniform in [lo, hi] (a range inside [-128, 127]) as int8:
+    lo + floor(u * (hi - lo + 1)) for the stream's uniforms u."""
+    assert -128 <= lo <= hi <= 127
+    out = np.empty(int(np.prod(shape)), np.int8)
+    _lib().synth_uniform_int8(_key(seed, name), 0, out.size, lo, hi, out.ctypes.data)
+    return out.reshape(shape)
 
 
 def to_bf16_bits(v: np.ndarray) -> np.ndarray:
@@ -94,9 +105,10 @@ def to_f16_bits(v: np.ndarray) -> np.ndarray:
 
 # ---- tensors of the workloads ----------------------------------------------
 def weight_rows(seed: int, name: str, K: int, row0: int, rows: int, std: float = 0.02) -> np.ndarray:
-    """Rows [row0, row0 + rows) of an fp32 weight W ~ N(0, std^2) of width K."""
-    z = normal(seed, name, row0 * K, rows * K)
-    return (std * z).astype(np.float32).reshape(rows, K)
+    """Rows [row0, row0 + rows) of an fp32 weight W = fp32(std * N(0, 1)) of width K."""
+    out = np.empty((rows, K), np.float32)
+    _lib().synth_normal_f32(_key(seed, name), row0 * K, rows * K, std, out.ctypes.data)
+    return out
 
 
 def activations(seed: int, name: str, M: int, K: int, outlier_frac: float = 0.0, outlier_gain: float = 20.0):

@@ -1,0 +1,235 @@
+"""GPU parity: every C-ABI call of libqlinear.so against the fp64 CPU oracle on
+the same seeded inputs.  Bit-exact for packed codes, scales, activation codes,
+W8A8 int32 group sums and the MoE permutation; rel-L2 <= 1e-5 and max-abs <=
+1e-3 * max|oracle| for fp32 outputs."""
+import numpy as np
+import pytest
+import torch
+
+from moe_hadamard128_act_b200 import synth
+from oracle import oracle as O
+from tests.gpu_util import assert_close, dev, dev_bf16, host_u16, host_u8
+
+pytestmark = pytest.mark.gpu
+
+Q = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def qlib():
+    global Q
+    from moe_hadamard128_act_b200 import build as qbuild
+    qbuild.build()
+    from moe_hadamard128_act_b200 import qlinear
+    Q = qlinear
+    Q.lib()
+    yield
+    st, bits = Q.ql_get_device_error()
+    assert st == 0 and bits == 0, f"device error word left set: {bits}"
+
+
+def x_bits(M, K, seed=0, name="x", outliers=0.0):
+    return synth.activations(seed, name, M, K, outlier_frac=outliers)
+
+
+# --------------------------------------------------------------------------
+# Activation kernels
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 256), (16, 5376), (7, 2816), (33, 640)])
+def test_hadamard128_rotate_bitexact(M, K):
+    x = x_bits(M, K, outliers=0.01)
+    ref = O.hadamard128_rotate(x)
+    xd = dev_bf16(x)
+    got = host_u16(Q.hadamard128_rotate(xd))
+    assert np.array_equal(got, ref)
+    Q.hadamard128_rotate(xd, out=xd)  # in place
+    assert np.array_equal(host_u16(xd), ref)
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+@pytest.mark.parametrize("M,K", [(1, 128), (4, 384), (16, 5376), (2048, 256)])
+def test_act_quant_bitexact(M, K, rotate):
+    x = x_bits(M, K, outliers=0.01)
+    x[0, :128] = 0  # an all-zero group
+    if K >= 256:
+        x[-1, 128:256] = O.bf16_encode(np.r_[127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, np.zeros(121)])  # ties
+    q_ref, s_ref = O.act_quant_i8_g128(x, rotate)
+    q, s = Q.act_quant_i8_g128(dev_bf16(x), rotate)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# Packing
+# --------------------------------------------------------------------------
+def oracle_pack_rtn(fmt, W, had):
+    if fmt in (Q.I8_G128_BF16, Q.I8A8_G128_BF16, Q.I8_G128_F16):
+        q, s = O.quant_i8_g128(W, hadamard=had, scale_f16=fmt == Q.I8_G128_F16)
+        return q.view(np.uint8), s, None
+    if fmt == Q.I4_G64_BF16:
+        q, s = O.quant_i4_g64(W, hadamard=had)
+        return O.pack_i4(q), s, None
+    if fmt == Q.FP8_B128_BF16:
+        q, s = O.quant_fp8_b128(W, hadamard=had)
+        return q, s, None
+    raise ValueError(fmt)
+
+
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 6])
+@pytest.mark.parametrize("N,K", [(64, 256), (200, 384), (130, 1024)])
+def test_pack_rtn_bitexact(fmt, had, N, K):
+    W = synth.weight_rows(3, f"Wp{N}", K, 0, N)
+    W[1, :128] = 0.0  # a zero group
+    codes, scales, _ = Q.qlinear_pack(fmt, N, K, W=dev(W), flags=had)
+    c_ref, s_ref, _ = oracle_pack_rtn(fmt, W, bool(had))
+    assert np.array_equal(host_u8(codes), c_ref.ravel())
+    assert np.array_equal(host_u8(scales).view(np.uint16), s_ref.ravel())
+
+
+def test_pack_given_codes_bitexact_and_range_flag():
+    N, K = 96, 256
+    rng = np.random.default_rng(7)
+    q4 = rng.integers(-8, 8, (N, K)).astype(np.int8)
+    s4 = O.bf16_encode(np.exp(rng.normal(-4, 0.5, (N, K // 64))))
+    c, s, _ = Q.qlinear_pack(Q.I4_G64_BF16, N, K, codes=dev(q4), scales=dev(s4))
+    assert np.array_equal(host_u8(c), O.pack_i4(q4).ravel())
+    assert np.array_equal(host_u8(s).view(np.uint16), s4.ravel())
+    q5 = rng.integers(0, 32, (N, K)).astype(np.uint8)
+    z5 = rng.integers(0, 32, (N, K // 128)).astype(np.uint8)
+    s5 = O.f16_encode(np.exp(rng.normal(-4, 0.5, (N, K // 128))))
+    c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N, K, codes=dev(q5), scales=dev(s5), zeros=dev(z5))
+    assert np.array_equal(host_u8(c), O.pack_i5(q5).ravel())
+    assert np.array_equal(host_u8(z), z5.ravel())
+    q8 = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    c, s, _ = Q.qlinear_pack(Q.I8_G128_BF16, N, K, codes=dev(q8), scales=dev(s4[:, ::2].copy()))
+    assert np.array_equal(host_u8(c), q8.view(np.uint8).ravel())
+    st, bits = Q.ql_get_device_error()
+    assert st == 0 and bits == 0
+    q4[3, 5] = 9  # out of the int4 range: packed as 0 and flagged, no fault
+    c, s, _ = Q.qlinear_pack(Q.I4_G64_BF16, N, K, codes=dev(q4), scales=dev(s4))
+    st, bits = Q.ql_get_device_error()
+    assert st == 6 and bits & Q.DEVERR_CODE_RANGE
+    q4[3, 5] = 0
+    assert np.array_equal(host_u8(c), O.pack_i4(q4).ravel())
+
+
+# --------------------------------------------------------------------------
+# Linear layer
+# --------------------------------------------------------------------------
+def make_weights(fmt, N, K, had, seed=5):
+    """Packed weights on the device plus the same bytes on the host."""
+    if fmt == Q.I5Z_G128_F16:
+        rng = np.random.default_rng(seed)
+        q5 = synth.uniform_int(seed, "i5", 0, 31, (N, K)).astype(np.uint8)
+        z5 = synth.uniform_int(seed, "i5z", 0, 31, (N, K // 128)).astype(np.uint8)
+        s5 = synth.lognormal_scales(seed, "i5s", (N, K // 128), f16=True)
+        c, s, z = Q.qlinear_pack(fmt, N, K, codes=dev(q5), scales=dev(s5), zeros=dev(z5))
+        del rng
+    else:
+        W = synth.weight_rows(seed, f"W{N}x{K}", K, 0, N)
+        c, s, z = Q.qlinear_pack(fmt, N, K, W=dev(W), flags=had)
+    return (c, s, z), (host_u8(c), host_u8(s).view(np.uint16), None if z is None else host_u8(z))
+
+
+SHAPES = [(1, 512, 256), (4, 200, 384), (5, 1000, 1024), (8, 64, 128), (9, 130, 256), (16, 333, 640),
+          (17, 64, 256), (33, 48, 128)]
+
+
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_forward_parity(fmt, had, M, N, K):
+    (c, s, z), (ch, sh, zh) = make_weights(fmt, N, K, had)
+    x = x_bits(M, K, seed=11, outliers=0.01)
+    y = Q.qlinear_forward(dev_bf16(x), c, s, z, fmt, N, flags=had)
+    ref = O.forward(x, ch, sh, zh, fmt, had, N)
+    assert_close(y.cpu().numpy(), ref, f"fmt {fmt} had {had} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 64, 128), (5, 200, 384), (16, 130, 1024), (20, 48, 256)])
+def test_w8a8_group_sums_bitexact(M, N, K):
+    x = x_bits(M, K, seed=2, outliers=0.01)
+    W = synth.weight_rows(2, "Wacc", K, 0, N)
+    qw, sw = O.quant_i8_g128(W, hadamard=True)
+    y_ref, acc_ref = O.forward(x, qw.view(np.uint8), sw, None, Q.I8A8_G128_BF16, Q.HADAMARD, N, want_acc=True)
+    qx, _ = O.act_quant_i8_g128(x, rotate=True)
+    acc = Q.qlinear_forward_i8_acc(dev(qx), dev(qw))
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    # full path on the same weights, extreme group: every code +-127
+    qw[0, :128] = 127
+    y = Q.qlinear_forward(dev_bf16(x), dev(qw), dev(sw), None, Q.I8A8_G128_BF16, N, flags=Q.HADAMARD)
+    assert_close(y.cpu().numpy(), O.forward(x, qw.view(np.uint8), sw, None, Q.I8A8_G128_BF16, Q.HADAMARD, N))
+
+
+def test_forward_zero_and_constant_inputs():
+    N, K = 64, 256
+    (c, s, z), (ch, sh, zh) = make_weights(Q.I8_G128_BF16, N, K, 0)
+    x = np.zeros((3, K), np.uint16)
+    y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.I8_G128_BF16, N)
+    assert not y.abs().sum().item()
+    x = O.bf16_encode(np.full((2, K), 3.0e4))  # large tokens: the per-token power-of-two keeps f16 in range
+    y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.I8_G128_BF16, N)
+    assert_close(y.cpu().numpy(), O.forward(x, ch, sh, None, Q.I8_G128_BF16, 0, N))
+
+
+# --------------------------------------------------------------------------
+# MoE
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("T,E,topk", [(1, 8, 2), (16, 128, 8), (40, 16, 4), (300, 32, 8), (2048, 128, 8)])
+def test_moe_permute_bitexact(T, E, topk):
+    ids, _ = synth.routing(4, T, E, topk)
+    counts, offsets, perm = Q.moe_permute(dev(ids), E)
+    c_ref, o_ref, p_ref, bad = O.moe_permute(ids, E)
+    assert bad == 0
+    assert np.array_equal(counts.cpu().numpy(), c_ref)
+    assert np.array_equal(offsets.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy(), p_ref)
+
+
+def test_moe_permute_degenerate_and_invalid():
+    ids = np.zeros((5, 8), np.int32)  # every pair on expert 0
+    counts, offsets, perm = Q.moe_permute(dev(ids), 4)
+    assert np.array_equal(perm.cpu().numpy(), np.arange(40))
+    ids[2, 3] = 77  # invalid id: dropped, flagged, no fault
+    counts, offsets, perm = Q.moe_permute(dev(ids), 4)
+    c_ref, o_ref, p_ref, bad = O.moe_permute(ids, 4)
+    assert np.array_equal(perm.cpu().numpy()[:39], p_ref[:39]) and perm[39].item() == -1
+    st, bits = Q.ql_get_device_error()
+    assert st == 6 and bits & Q.DEVERR_EXPERT_ID
+
+
+def moe_weights(E, N, K, fmt, seed=9):
+    qs, ss = [], []
+    for e in range(E):
+        W = synth.weight_rows(seed, f"moeW{e}", K, 0, N)
+        if fmt == Q.FP8_B128_BF16:
+            q, s = O.quant_fp8_b128(W, hadamard=True)
+        else:
+            q, s = O.quant_i8_g128(W, hadamard=True, scale_f16=fmt == Q.I8_G128_F16)
+            q = q.view(np.uint8)
+        qs.append(q)
+        ss.append(s)
+    return np.stack(qs), np.stack(ss)
+
+
+@pytest.mark.parametrize("fmt", [1, 2, 6])
+@pytest.mark.parametrize("T,E,topk,N,K", [(1, 8, 2, 96, 256), (8, 16, 4, 64, 384), (16, 32, 8, 130, 256),
+                                          (40, 8, 3, 48, 128)])
+def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
+    codes, scales = moe_weights(E, N, K, fmt)
+    ids, w = synth.routing(6, T, E, topk)
+    x = x_bits(T, K, seed=13)
+    y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N, fmt=fmt, flags=Q.HADAMARD,
+                      topk_weights=dev(w))
+    ref = O.moe_gate_up(x, ids, codes, scales, fmt, O.HADAMARD, E, N)
+    assert_close(y.cpu().numpy(), ref, f"moe fmt {fmt} T{T}")
+
+
+def test_moe_duplicate_expert_in_token():
+    E, N, K, T = 4, 64, 128, 3
+    codes, scales = moe_weights(E, N, K, Q.I8_G128_BF16)
+    ids = np.array([[1, 1, 2], [1, 3, 1], [0, 0, 0]], np.int32)
+    x = x_bits(T, K, seed=1)
+    y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N)
+    assert_close(y.cpu().numpy(), O.moe_gate_up(x, ids, codes, scales, 1, 1, E, N))
