@@ -191,8 +191,9 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
  * earlier trace is dropped); 0 stops tracing and destroys the events.  Once
  * all slots are used, further launches go unrecorded.  ql_trace_read waits
  * for the recorded stop events and returns, per slot in launch order, the
- * kind of launch (QL_KIND_*) and its duration in milliseconds; *count is the
- * number of slots used.  Host-side state only: not thread safe. */
+ * kind of launch (QL_KIND_*) and its duration in milliseconds (-1 if its
+ * events could not be recorded); *count is the number of slots used.
+ * Host-side state only: not thread safe. */
 enum {
     QL_KIND_ROTATE = 1,      /* hadamard128_rotate                              */
     QL_KIND_ACT_QUANT = 2,   /* activation quantiser (also zeroes y for W8A8)   */

@@ -128,8 +128,8 @@ __device__ __forceinline__ void load_unit(Regs<FMT>& r, const uint8_t* wbase, lo
                 r.w[h][1] = ldg_stream128(p + 16);
                 if constexpr (FMT == QL_FP8_B128_BF16)
                     r.s[h] = load_scale<FMT>(scales, (long long)(n >> 7) * Gtot + gabs);
-                else
-                    r.s[h] = load_scale<FMT>(scales, (long long)n * Gtot + gabs);
+                else  // the integer-only W8A8 check path has no scales
+                    r.s[h] = scales ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
             } else {
                 r.w[h][0] = r.w[h][1] = make_uint4(0, 0, 0, 0);
                 r.s[h] = 0.0f;
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny(SkinnyArgs a) {
         if constexpr (FMT == QL_I8A8_G128_BF16) {
             for (int i = threadIdx.x; i < 16 * G; i += kThreads) {
                 const int t = i / G, gg = i % G;
-                fac[i] = t < a.M ? a.xf[(long long)t * a.Gtot + a.g0 + gg] : 0.0f;
+                fac[i] = (t < a.M && a.xf) ? a.xf[(long long)t * a.Gtot + a.g0 + gg] : 0.0f;
             }
         } else {
             if (threadIdx.x < 16) fac[threadIdx.x] = threadIdx.x < a.M ? a.xf[threadIdx.x] : 0.0f;

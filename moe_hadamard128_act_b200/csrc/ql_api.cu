@@ -50,6 +50,7 @@ cudaError_t device_info(DeviceInfo* out) {
 namespace {
 struct TraceSlot {
     int kind;
+    bool ok;  // both events recorded
     cudaEvent_t start, stop;
 };
 TraceSlot* g_slots = nullptr;
@@ -66,16 +67,34 @@ void trace_free() {
 }
 }  // namespace
 
+namespace {
+// Under stream capture the record must be an external event node of the graph;
+// outside capture it is a plain record.  A failed record is cleared (so it
+// cannot surface at the next launch check) and reported as false.
+bool trace_record(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        cs = cudaStreamCaptureStatusNone;
+    }
+    const cudaError_t e = cs == cudaStreamCaptureStatusActive
+                              ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                              : cudaEventRecord(ev, s);
+    if (e != cudaSuccess) cudaGetLastError();
+    return e == cudaSuccess;
+}
+}  // namespace
+
 int trace_begin(int kind, cudaStream_t s) {
     if (g_used >= g_capacity) return -1;
     const int slot = g_used++;
     g_slots[slot].kind = kind;
-    cudaEventRecord(g_slots[slot].start, s);
+    g_slots[slot].ok = trace_record(g_slots[slot].start, s);
     return slot;
 }
 
 void trace_end(int slot, cudaStream_t s) {
-    if (slot >= 0) cudaEventRecord(g_slots[slot].stop, s);
+    if (slot >= 0) g_slots[slot].ok = trace_record(g_slots[slot].stop, s) && g_slots[slot].ok;
 }
 
 }  // namespace ql
@@ -427,9 +446,11 @@ int ql_trace_read(int* kinds, float* ms, int max, int* count) {
     if (!count || max < 0 || (max > 0 && (!kinds || !ms))) return QL_EINVAL;
     const int n = g_used < max ? g_used : max;
     for (int i = 0; i < n; ++i) {
-        if (cudaEventSynchronize(g_slots[i].stop) != cudaSuccess) return QL_ECUDA;
-        float t = 0.0f;
-        if (cudaEventElapsedTime(&t, g_slots[i].start, g_slots[i].stop) != cudaSuccess) return QL_ECUDA;
+        float t = -1.0f;  // -1: the slot's events were not recorded
+        if (g_slots[i].ok) {
+            if (cudaEventSynchronize(g_slots[i].stop) != cudaSuccess) return QL_ECUDA;
+            if (cudaEventElapsedTime(&t, g_slots[i].start, g_slots[i].stop) != cudaSuccess) return QL_ECUDA;
+        }
         kinds[i] = g_slots[i].kind;
         ms[i] = t;
     }
