@@ -184,6 +184,29 @@ int moe_workspace_size(const ql_experts* experts, int T, int topk, size_t* bytes
 int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weights, const ql_experts* experts,
                 int T, int topk, float* y, void* ws, size_t ws_bytes, void* stream);
 
+/* qlinear_forward_w8a8_noalloc -- the W8A8 forward of qlinear_forward
+ * (fmt QL_I8A8_G128_BF16) for callers that cannot allocate device memory,
+ * such as a plugin inside a host engine that owns all device memory and
+ * forbids cudaMalloc, or a latency-critical loop that must avoid cudaMalloc's
+ * implicit synchronisation.  The model cards have no counterpart: this is an
+ * interface choice of this library.
+ *
+ * Same arguments and result as qlinear_forward with fmt = QL_I8A8_G128_BF16,
+ * minus the workspace: the int8 activations and their scales go to a fixed
+ * array inside the library's device memory, sized for M <= QL_NOALLOC_MAX_M
+ * and K <= QL_NOALLOC_MAX_K (270,336 bytes, held on every GPU that loads the
+ * library until the process exits).  Larger M or K return QL_EUNSUPPORTED
+ * before anything is launched.  The call allocates nothing.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array: calls whose kernels may overlap on the GPU
+ * (other streams, other host threads) race on it and must be serialised by
+ * the caller.  Nothing in the array needs to start at zero; each call
+ * rewrites what it reads. */
+enum { QL_NOALLOC_MAX_M = 16, QL_NOALLOC_MAX_K = 16384 };
+int qlinear_forward_w8a8_noalloc(const void* x, const void* W_packed, const void* scales, int flags, int M, int N,
+                                 int K, float* y, void* stream);
+
 /* Launch trace.  Every kernel the library launches can be bracketed by a pair
  * of CUDA events recorded on the caller's stream (also inside stream capture,
  * where they become event nodes of the graph).  ql_trace_enable(capacity)

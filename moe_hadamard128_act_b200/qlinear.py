@@ -63,6 +63,7 @@ _SIGS = {
     "moe_workspace_size": (_I, [ctypes.POINTER(ql_experts), _I, _I, _PSZ]),
     "moe_gate_up": (_I, [_P, _P, _P, ctypes.POINTER(ql_experts), _I, _I, _P, _P, _SZ, _P]),
     "ql_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "qlinear_forward_w8a8_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "ql_trace_enable": (_I, [_I]),
     "ql_trace_read": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), _I,
                            ctypes.POINTER(ctypes.c_int)]),
@@ -171,6 +172,20 @@ def qlinear_forward(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, 
     st = lib().qlinear_forward(_ptr(x), _ptr(codes), _ptr(scales), _ptr(zeros), fmt, flags, M, N, K, _ptr(y),
                                _ptr(ws), ws.numel(), _stream(stream))
     _check("qlinear_forward", st)
+    return y
+
+
+def qlinear_forward_w8a8_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, N: int,
+                                 flags: int = 0, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """W8A8 forward without a workspace, for callers that cannot allocate
+    device memory (M <= 16, K <= 16384): the activation scratch lives in a fixed
+    array inside the library.  Calls that may overlap on the GPU race on it."""
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    st = lib().qlinear_forward_w8a8_noalloc(_ptr(x), _ptr(codes), _ptr(scales), flags, M, N, K, _ptr(y),
+                                            _stream(stream))
+    _check("qlinear_forward_w8a8_noalloc", st)
     return y
 
 
