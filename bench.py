@@ -12,9 +12,10 @@ Timing: W eager warm-up steps, then the K timed steps replayed from a CUDA
 graph, bracketed by a barrier and device synchronisation, measured with CUDA
 events on the launching stream; max over ranks.  Four packed copies of the
 weight (470 MB, more than the 126 MB L2) rotate between the forward calls, so
-no call finds its weight in L2.  The library's own launch trace (CUDA events
-around each of its kernels, captured into the graph) gives the per-kernel
-durations of the last timed graph replay for the roofline.
+no call finds its weight in L2.  The timed graph holds only the library's
+kernels; the per-kernel durations for the roofline come from one more replay
+of the same steps with the library's launch trace (CUDA events around each of
+its kernels, on the launching stream) captured into the graph.
 Multi-GPU: replicas only -- the layer does not shard in this workload, every
 rank runs the same step on its own GPU and value sums the ranks' bytes.
 """
@@ -374,21 +375,25 @@ def main():
             step()
     stream.synchronize()
 
-    # ---- graph of S steps with the launch trace captured in it ----
+    # ---- timed region: a graph of S steps, replayed R times (no trace nodes) ----
     S = max(d for d in range(1, min(args.steps, 50) + 1) if args.steps % d == 0)
     R = args.steps // S
     launches_per_step = 2 * len(MS)
-    Q.ql_trace_enable(S * launches_per_step)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(S):
-                step()
-    g.replay()  # untimed graph warm-up
-    stream.synchronize()
 
+    def capture(trace: bool):
+        if trace:
+            Q.ql_trace_enable(S * launches_per_step)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gr, stream=stream):
+                for _ in range(S):
+                    step()
+        gr.replay()  # untimed graph warm-up
+        stream.synchronize()
+        return gr
+
+    g = capture(trace=False)
     # clocks pre-roll: about a second of the same load while nvidia-smi samples
-    per_replay = None
     with ClockSampler(local) as clk:
         t0 = time.perf_counter()
         n = 0
@@ -398,7 +403,6 @@ def main():
             if n % 10 == 0:
                 stream.synchronize()
         stream.synchronize()
-        per_replay = (time.perf_counter() - t0) / n
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
         if world > 1:
@@ -412,13 +416,21 @@ def main():
         if world > 1:
             dist.barrier()
     ms = ev0.elapsed_time(ev1)
-    trace = Q.ql_trace_read(S * launches_per_step)
-    Q.ql_trace_enable(0)
     if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = t.item()
     value = world * args.steps * step_bytes() / (ms * 1e-3) / 1e9
+
+    # ---- per-kernel durations: the same S steps replayed once more with the
+    # library's launch trace (CUDA events around each of its kernels, recorded
+    # on the launching stream) captured into the graph ----
+    gt = capture(trace=True)
+    gt.replay()
+    stream.synchronize()
+    trace = Q.ql_trace_read(S * launches_per_step)
+    Q.ql_trace_enable(0)
+    del gt
 
     # ---- roofline of the dominant kernel (the skinny GEMM) from the trace ----
     hbm, bf16_tf, peak_src = peaks()
@@ -430,7 +442,8 @@ def main():
     traffic = kernel_traffic("skinny_w8a8_decode", ROOT / "moe_hadamard128_act_b200" / "csrc" / "k_skinny.cu")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm if achieved else None, "traffic": traffic,
-                "kernel": "k_skinny<W8A8>", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "kernel": "k_skinny_tma<W8A8>", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "timing": f"CUDA events around each launch, a traced replay of {S} timed steps (events included)",
                 "share_of_traced_time": share,
                 "per_m_us": {str(m): 1e3 * float(np.mean(sk[i::len(MS)])) for i, m in enumerate(MS)}}
 

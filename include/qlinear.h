@@ -45,9 +45,11 @@
  *   - K must be a multiple of 128, M, N, T >= 1, every device pointer 16-byte
  *     aligned.  Violations return a status before anything is launched.
  *   - Errors found on the device (an expert id outside [0, E), a code out of
- *     its range given to the packer) never trap: the offending item is skipped
- *     and a bit is set in a per-process device error word that
- *     ql_get_device_error reads and clears.
+ *     its range given to the packer, a copy into shared memory that did not
+ *     complete within 200 ms) never trap: the offending item is skipped (a
+ *     timed-out kernel stops early, leaving its output incomplete) and a bit is
+ *     set in a per-process device error word that ql_get_device_error reads and
+ *     clears.
  *   - No C++ exception crosses this interface.
  */
 #ifndef QLINEAR_H
@@ -82,7 +84,7 @@ typedef enum {
 enum { QL_HADAMARD = 1 };
 
 /* Bits of the device error word. */
-enum { QL_DEVERR_EXPERT_ID = 1, QL_DEVERR_CODE_RANGE = 2 };
+enum { QL_DEVERR_EXPERT_ID = 1, QL_DEVERR_CODE_RANGE = 2, QL_DEVERR_TIMEOUT = 4 };
 
 /* Human-readable name of a status. Never NULL. */
 const char* ql_status_string(int status);

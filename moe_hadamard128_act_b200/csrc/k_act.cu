@@ -57,6 +57,7 @@ __device__ __forceinline__ void zero_fill(float* y, long long n) {
 // s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127).
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bfloat16* x, int M, int K, int rotate,
                                                                    int8_t* q, float* sx, float* yz, long long nz) {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
     const int lane = threadIdx.x & 31;
     const long long G = K / 128;
@@ -89,13 +90,16 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // shared memory as fp32; its max |x| picks a power of two f with
 // max|x| * f in [2^14, 2^15), and xs = f16(x * f) is written in the element
 // order of the format (within each 8-block [0,4,1,5,2,6,3,7] for int4, within
-// each 4-block [0,3,1,2] for int5, natural otherwise).  xf = 1 / f.
+// each 4-block [0,3,1,2] for int5, natural otherwise; for int5 the 16-byte
+// pieces of each 128-group are also swapped pairwise in their upper half, the
+// shared-memory layout the GEMM reads without bank conflicts).  xf = 1 / f.
 // f16 holds every bf16 value of the scaled row exactly down to 2^-14 (its
 // normal range); below that the rounding error is under 2^-39 of the row's
 // max, far beneath the fp32 accumulation error of the GEMM.
 __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K, int rotate, int order, __half* xs,
                                                   float* xf, float* yz, long long nz) {
     extern __shared__ float row[];
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
     __shared__ float red[8];
     const int t = blockIdx.x;
@@ -140,8 +144,25 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K,
             const int p = k & 3;
             src = (k & ~3) + (p == 0 ? 0 : (p == 1 ? 3 : p - 1));
         }
-        out[k] = __float2half_rn(__fmul_rn(row[src], f));
+        int dst = k;
+        if (order == XORD_I5) dst = k ^ (((k >> 6) & 1) << 3);  // piece j -> j ^ bit3(j): conflict-free staging
+        out[dst] = __float2half_rn(__fmul_rn(row[src], f));
     }
+}
+
+// The GEMM that follows these kernels runs with (nearly) all of the SM's
+// shared memory; asking for the same L1/shared split here avoids an SM
+// reconfiguration between the two launches.
+template <typename F>
+cudaError_t prefer_max_shared(F* kernel) {
+    static bool done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && done[dev]) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess && dev < 64) done[dev] = true;
+    return e;
 }
 
 int grid_for(long long warps, int sm_count) {
@@ -166,6 +187,7 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
+    if ((e = prefer_max_shared(k_act_quant)) != cudaSuccess) return e;
     k_act_quant<<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, yz, nz);
     return cudaGetLastError();
@@ -174,8 +196,10 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s) {
     const size_t smem = (size_t)K * sizeof(float);
+    cudaError_t e = prefer_max_shared(k_prep_a16);
+    if (e != cudaSuccess) return e;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     k_prep_a16<<<M, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, order, xs, xf, yz, nz);

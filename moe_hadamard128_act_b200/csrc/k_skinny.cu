@@ -30,13 +30,24 @@
 //    dot product unchanged.
 //  * Partial sums leave through fp32 atomic adds only when a warp's range
 //    leaves a 16-row slab (about twice per warp), into a y the caller zeroed.
+#include <algorithm>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
 #include "ql_device.cuh"
 #include "ql_internal.h"
 
 namespace ql {
 namespace {
 
-constexpr int kThreads = 512;
+#ifndef QL_SKINNY_THREADS
+#define QL_SKINNY_THREADS 512
+#endif
+#ifndef QL_SKINNY_STAGES
+#define QL_SKINNY_STAGES 4
+#endif
+constexpr int kThreads = QL_SKINNY_THREADS;
 constexpr int kWarps = kThreads / 32;
 
 // Register image of one unit's weights, for one lane.
@@ -267,69 +278,380 @@ __device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX
     }
 }
 
+// ---------------------------------------------------------------------------
+// Dense skinny GEMM, TMA-fed.
+//
+// Every warp owns a ring of kStages shared-memory slots, one unit (16 rows of
+// the packed weight x one 128-K group) per slot.  Lane 0 keeps kStages units
+// in flight with cp.async.bulk.tensor (2-D tile [16 rows][unit bytes],
+// zero-filled past row N) completing on a per-slot mbarrier; the whole warp
+// waits on the slot, pulls its fragments out of shared memory, refills the
+// slot with the unit kStages ahead and computes.  With 16 warps x 4 slots x
+// 2 KB the SM keeps up to 128 KB of weight in flight without holding it in
+// registers.  Waits are bounded: a slot that never fills sets
+// QL_DEVERR_TIMEOUT in the device error word and the CTA drains and returns.
+//
+// Units are numbered (K part, row slab, group within the part): a CTA's
+// contiguous range touches at most two K parts, so it stages only those parts
+// of the activations.
+// ---------------------------------------------------------------------------
+constexpr int kStages = QL_SKINNY_STAGES;
+
 template <int FMT>
-constexpr size_t skinny_smem(int NT, int G) {
-    return (size_t)NT * 8 * ((size_t)G * x_group_bytes<FMT>() + x_row_pad<FMT>()) +
-           (FMT == QL_I8A8_G128_BF16 ? (size_t)16 * G * 4 : 16 * 4);
+__host__ __device__ constexpr int unit_row_bytes() {
+    return FMT == QL_I4_G64_BF16 ? 64 : (FMT == QL_I5Z_G128_F16 ? 80 : 128);
+}
+template <int FMT>
+__host__ __device__ constexpr int stage_bytes() { return 16 * unit_row_bytes<FMT>(); }
+template <int FMT>
+__host__ __device__ constexpr int stage_align() {
+    return FMT == QL_I4_G64_BF16 ? 512 : (FMT == QL_I5Z_G128_F16 ? 128 : 1024);
+}
+// Activation staging: bytes per token per group and the row padding that keeps
+// the fragment loads conflict-free (see the piece index in tma_getx).
+template <int FMT>
+__host__ __device__ constexpr int tx_group_bytes() { return FMT == QL_I8A8_G128_BF16 ? 128 : 256; }
+template <int FMT>
+__host__ __device__ constexpr int tx_row_pad() {
+    return FMT == QL_I8A8_G128_BF16 ? 64 : (FMT == QL_I5Z_G128_F16 ? 32 : 16);
 }
 
-// Dense skinny GEMM over one (token chunk, K chunk).
-template <int FMT, int NT, bool ACC>
-__global__ void __launch_bounds__(kThreads, 1) k_skinny(SkinnyArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    constexpr int XGB = x_group_bytes<FMT>();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, c = lane & 3;
-    const int G = a.G;
-    const long long R = (long long)G * XGB + x_row_pad<FMT>();
-    float* fac = reinterpret_cast<float*>(smem + NT * 8 * R);
+template <int FMT>
+__host__ __device__ constexpr size_t ring_bytes() {
+    return (size_t)kWarps * kStages * stage_bytes<FMT>();
+}
+template <int FMT>
+__host__ __device__ constexpr size_t tma_smem(int NT, int XG) {
+    return 1024 /* alignment slack */ + ring_bytes<FMT>() + (size_t)kWarps * kStages * 8 + 16 +
+           (size_t)NT * 8 * ((size_t)XG * tx_group_bytes<FMT>() + tx_row_pad<FMT>());
+}
 
-    const int slabs = (a.N + 15) / 16;
-    const long long units = (long long)slabs * G;
-    const long long wid = (long long)blockIdx.x * kWarps + warp, nw = (long long)gridDim.x * kWarps;
-    const long long u0 = units * wid / nw, u1 = units * (wid + 1) / nw;
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
+    return t;
+}
+// Wait for phase `phase` of the mbarrier; false after ~kWaitNs without it.
+constexpr unsigned long long kWaitNs = 200ull * 1000 * 1000;
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned phase) {
+    if (mbar_try_wait(bar, phase)) return true;
+    const unsigned long long t0 = global_ns();
+    for (unsigned it = 0;; ++it) {
+        if (mbar_try_wait(bar, phase)) return true;
+        if ((it & 255u) == 255u && global_ns() - t0 > kWaitNs) return false;
+    }
+}
+// One contiguous global -> shared copy, completing on an mbarrier (16-byte
+// aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, unsigned bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+            dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
 
-    Regs<FMT> r0, r1, r2;
-    auto load = [&](Regs<FMT>& r, long long u) {
-        const int slab = (int)(u / G), grp = (int)(u % G);
-        load_unit<FMT>(r, a.W, a.ldw, a.scales, a.zeros, a.N, a.Gtot, a.g0 + grp, slab, grp, g, c);
-    };
-    // Start the weight stream before staging the activations.
-    if (u0 < u1) load(r0, u0);
-    if (u0 + 1 < u1) load(r1, u0 + 1);
-
-    // Stage activations: token rows [0, NT*8), zero beyond M.
-    {
-        const int pieces_per_row = G * XGB / 16;
-        const int total = NT * 8 * pieces_per_row;
-        const uint8_t* xsrc = static_cast<const uint8_t*>(a.xs);
-        const long long ldx_b = a.ldx * (FMT == QL_I8A8_G128_BF16 ? 1 : 2);
-        for (int i = threadIdx.x; i < total; i += kThreads) {
-            const int t = i / pieces_per_row, j = i % pieces_per_row;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (t < a.M) v = *reinterpret_cast<const uint4*>(xsrc + t * ldx_b + 16LL * j);
-            *reinterpret_cast<uint4*>(smem + t * R + 16LL * swz<FMT>(j)) = v;
-        }
-        if constexpr (FMT == QL_I8A8_G128_BF16) {
-            for (int i = threadIdx.x; i < 16 * G; i += kThreads) {
-                const int t = i / G, gg = i % G;
-                fac[i] = (t < a.M && a.xf) ? a.xf[(long long)t * a.Gtot + a.g0 + gg] : 0.0f;
+// Position in the unit stream: K part, row slab, group within the part.
+struct UnitPos {
+    int part, slab, gi, gp;  // gp = groups in this part
+    __device__ __forceinline__ void init(unsigned u, int slabs, int GP, int G) {
+        const unsigned per_full = (unsigned)slabs * GP;
+        part = (int)(u / per_full);
+        const unsigned rem = u - (unsigned)part * per_full;
+        gp = min(GP, G - part * GP);
+        slab = (int)(rem / gp);
+        gi = (int)(rem % gp);
+    }
+    __device__ __forceinline__ void next(int slabs, int GP, int G) {
+        if (++gi == gp) {
+            gi = 0;
+            if (++slab == slabs) {
+                slab = 0;
+                ++part;
+                gp = min(GP, G - part * GP);
             }
-        } else {
-            if (threadIdx.x < 16) fac[threadIdx.x] = threadIdx.x < a.M ? a.xf[threadIdx.x] : 0.0f;
         }
     }
-    __syncthreads();
-    if (u0 >= u1) return;
+    __device__ __forceinline__ int grp(int GP) const { return part * GP + gi; }
+};
 
-    const uint32_t xs_base = smem_u32(smem);
+template <int FMT>
+__device__ __forceinline__ void load_unit_scales(Regs<FMT>& r, const void* scales, const uint8_t* zeros, int N,
+                                                 int Gtot, int gabs, int slab, int g) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int n = slab * 16 + g + 8 * h;
+        const bool ok = n < N;
+        if constexpr (FMT == QL_I4_G64_BF16) {
+            r.s[h][0] = ok ? load_scale<FMT>(scales, (long long)n * (2 * Gtot) + 2 * gabs) : 0.0f;
+            r.s[h][1] = ok ? load_scale<FMT>(scales, (long long)n * (2 * Gtot) + 2 * gabs + 1) : 0.0f;
+        } else if constexpr (FMT == QL_I5Z_G128_F16) {
+            r.s[h] = ok ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
+            const float z = ok ? (float)__ldg(zeros + (long long)n * Gtot + gabs) : 0.0f;
+            r.nz[h] = (uint32_t)__half_as_ushort(__float2half_rn(-(1024.0f + z))) * 0x10001u;
+        } else if constexpr (FMT == QL_FP8_B128_BF16) {
+            r.s[h] = ok ? load_scale<FMT>(scales, (long long)(n >> 7) * Gtot + gabs) : 0.0f;
+        } else {
+            r.s[h] = (ok && scales) ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
+        }
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void copy_scales(Regs<FMT>& d, const Regs<FMT>& s) {
+    if constexpr (FMT == QL_I4_G64_BF16) {
+        d.s[0][0] = s.s[0][0]; d.s[0][1] = s.s[0][1]; d.s[1][0] = s.s[1][0]; d.s[1][1] = s.s[1][1];
+    } else if constexpr (FMT == QL_I5Z_G128_F16) {
+        d.s[0] = s.s[0]; d.s[1] = s.s[1]; d.nz[0] = s.nz[0]; d.nz[1] = s.nz[1];
+    } else {
+        d.s[0] = s.s[0]; d.s[1] = s.s[1];
+    }
+}
+
+// The lane's weight fragments of one unit, out of its ring slot.
+template <int FMT>
+__device__ __forceinline__ void read_unit_smem(Regs<FMT>& r, uint32_t st, int g, int c) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = g + 8 * h;
+        if constexpr (FMT == QL_I4_G64_BF16) {
+            // 64-byte rows, 64B swizzle: 16-byte chunk j lands at j ^ ((row >> 1) & 3).
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int j = 2 * half + (c >> 1);
+                const uint32_t a = st + row * 64 + ((j ^ ((row >> 1) & 3)) << 4) + 8 * (c & 1);
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(r.w[h][half].x), "=r"(r.w[h][half].y) : "r"(a));
+            }
+        } else if constexpr (FMT == QL_I5Z_G128_F16) {
+            const uint32_t a = st + row * 80 + 20 * c;
+#pragma unroll
+            for (int i = 0; i < 5; ++i) asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(r.w[h][i]) : "r"(a + 4 * i));
+        } else {
+            // 128-byte rows, 128B swizzle: chunk j lands at j ^ (row & 7).  The lane
+            // holds chunks c and 4 + c; odd rows read them in the other order so each
+            // quarter-warp touches eight distinct 16-byte bank groups.
+            const bool odd = (g & 1) != 0;
+            const int j0 = odd ? 4 + c : c, j1 = odd ? c : 4 + c;
+            const uint4 v0 = lds128(st + row * 128 + ((j0 ^ (row & 7)) << 4));
+            const uint4 v1 = lds128(st + row * 128 + ((j1 ^ (row & 7)) << 4));
+            r.w[h][0] = odd ? v1 : v0;
+            r.w[h][1] = odd ? v0 : v1;
+        }
+    }
+}
+
+#ifdef QL_SKINNY_PROFILE
+__device__ unsigned long long g_skinny_prof[148 * 16];
+#define QL_PROF(slot)                                                                        \
+    if (threadIdx.x == 0 && blockIdx.x < 148)                                                  \
+        g_skinny_prof[blockIdx.x * 16 + (slot)] = (slot) == 0 ? global_ns() : clock64() - prof_c0;
+#else
+#define QL_PROF(slot)
+#endif
+
+// Per-unit side data, fetched kStages units ahead of use together with the
+// weight tile: raw scale bits (converted only when the unit is computed, so
+// the loads never stall the issuing loop), int5 zero points, and for W8A8 the
+// activation scales of the lane's output tokens.
+template <int FMT, int NT>
+struct Side {
+    uint32_t sw[2][2];  // weight scale bits [row g / g+8][int4 half]
+    uint32_t z[2];      // int5 zero points
+    float sx[NT][2];    // W8A8: activation scales of tokens 8nt + 2c + {0, 1}
+};
+
+template <int FMT, int NT>
+__device__ __forceinline__ void load_side_w(Side<FMT, NT>& d, const void* scales, const uint8_t* zeros, int N,
+                                            int Gtot, int gabs, int slab, int g) {
+    const uint16_t* sc = static_cast<const uint16_t*>(scales);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int n = slab * 16 + g + 8 * h;
+        const bool ok = n < N && sc;
+        if constexpr (FMT == QL_I4_G64_BF16) {
+            d.sw[h][0] = ok ? __ldg(sc + (long long)n * (2 * Gtot) + 2 * gabs) : 0u;
+            d.sw[h][1] = ok ? __ldg(sc + (long long)n * (2 * Gtot) + 2 * gabs + 1) : 0u;
+        } else if constexpr (FMT == QL_FP8_B128_BF16) {
+            d.sw[h][0] = ok ? __ldg(sc + (long long)(n >> 7) * Gtot + gabs) : 0u;
+        } else {
+            d.sw[h][0] = ok ? __ldg(sc + (long long)n * Gtot + gabs) : 0u;
+        }
+        if constexpr (FMT == QL_I5Z_G128_F16) d.z[h] = ok ? __ldg(zeros + (long long)n * Gtot + gabs) : 0u;
+    }
+}
+
+template <int FMT, int NT>
+__device__ __forceinline__ void load_side_x(Side<FMT, NT>& d, const float* sx, int M, int Gtot, int gabs, int c) {
+    if constexpr (FMT == QL_I8A8_G128_BF16) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int t = 8 * nt + 2 * c + i;
+                d.sx[nt][i] = (t < M && sx) ? __ldg(sx + (long long)t * Gtot + gabs) : 0.0f;
+            }
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ float scale_value(uint32_t bits) {
+    return (FMT == QL_I8_G128_F16 || FMT == QL_I5Z_G128_F16) ? __half2float(__ushort_as_half((unsigned short)bits))
+                                                             : __uint_as_float(bits << 16);
+}
+
+template <int FMT, int NT>
+__device__ __forceinline__ void side_to_regs(Regs<FMT>& r, const Side<FMT, NT>& d) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if constexpr (FMT == QL_I4_G64_BF16) {
+            r.s[h][0] = scale_value<FMT>(d.sw[h][0]);
+            r.s[h][1] = scale_value<FMT>(d.sw[h][1]);
+        } else {
+            r.s[h] = scale_value<FMT>(d.sw[h][0]);
+        }
+        if constexpr (FMT == QL_I5Z_G128_F16)
+            r.nz[h] = (uint32_t)__half_as_ushort(__float2half_rn(-(1024.0f + (float)d.z[h]))) * 0x10001u;
+    }
+}
+
+template <int FMT, int NT, bool ACC>
+__global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constant__ SkinnyArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+#ifdef QL_SKINNY_PROFILE
+    const long long prof_c0 = clock64();
+    if (threadIdx.x == 0 && blockIdx.x < 148) g_skinny_prof[blockIdx.x * 16 + 15] = 0;
+#endif
+    QL_PROF(0)
+    constexpr int XGB = tx_group_bytes<FMT>();
+    constexpr int SB = stage_bytes<FMT>();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    const int G = a.G, GP = a.GP, slabs = (a.N + 15) / 16;
+    if (lane == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmap) : "memory");
+
+    // Shared memory: [rings][mbarriers][activation barrier][activations], 1024-aligned base.
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const gbase = smem_raw + (base - raw);
+    const uint32_t ring = base + (uint32_t)(warp * kStages * SB);
+    const uint32_t bars = base + (uint32_t)ring_bytes<FMT>() + (uint32_t)(warp * kStages * 8);
+    const uint32_t xbar = base + (uint32_t)ring_bytes<FMT>() + kWarps * kStages * 8;
+    const uint32_t xs_off = (uint32_t)ring_bytes<FMT>() + kWarps * kStages * 8 + 16;
+    const int R = a.XG * XGB + tx_row_pad<FMT>();
+    uint8_t* const xs = gbase + xs_off;
+    const uint32_t xs_base = base + xs_off;
+
+    // Work: the CTA's contiguous unit range, split contiguously over its warps
+    // (32-bit: the host keeps units * gridDim below 2^31).
+    const unsigned units = (unsigned)slabs * G;
+    const unsigned cu0 = units * blockIdx.x / gridDim.x, cu1 = units * (blockIdx.x + 1) / gridDim.x;
+    const unsigned u0 = cu0 + (cu1 - cu0) * warp / kWarps, u1 = cu0 + (cu1 - cu0) * (warp + 1) / kWarps;
+
+    UnitPos cp;  // unit being computed
+    if (u0 < u1) cp.init(u0, slabs, GP, G);
+    UnitPos ip = cp;  // next unit to issue
+    Side<FMT, NT> sd[kStages];
+    unsigned issued = u0;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) mbar_init(bars + 8 * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncwarp();
+    QL_PROF(7)
+    // Start the weight stream first: it never depends on the kernel before.
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+        if (issued < u1) {
+            if (lane == 0) {
+                mbar_expect_tx(bars + 8 * s, SB);
+                tma_load_2d(ring + s * SB, &a.tmap, ip.grp(GP) * unit_row_bytes<FMT>(), ip.slab * 16, bars + 8 * s);
+            }
+            load_side_w<FMT, NT>(sd[s], a.scales, a.zeros, a.N, a.Gtot, a.g0 + ip.grp(GP), ip.slab, g);
+            ip.next(slabs, GP, G);
+            ++issued;
+        }
+    }
+    QL_PROF(8)
+
+    // The activations (and the zeroed y) come from the kernel launched just
+    // before this one: wait for it (a no-op without a programmatic dependency).
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    QL_PROF(2)
+
+    // Stage the activations of the K parts this CTA touches, one bulk copy per
+    // token row, while the weight stream runs; rows beyond M are zeroed.
+    int gs0 = 0, ngs = 0;
+    if (cu1 > cu0) {
+        UnitPos p0, p1;
+        p0.init(cu0, slabs, GP, G);
+        p1.init(cu1 - 1, slabs, GP, G);
+        gs0 = p0.part * GP;
+        ngs = min(G, (p1.part + 1) * GP) - gs0;
+    }
+    const int rows_x = ngs > 0 ? min(a.M, NT * 8) : 0;
+    if (threadIdx.x == 0) {
+        mbar_init(xbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        if (rows_x > 0) {
+            const unsigned row_bytes = (unsigned)(ngs * XGB);
+            mbar_expect_tx(xbar, row_bytes * rows_x);
+            const uint8_t* xsrc = static_cast<const uint8_t*>(a.xs);
+            const long long ldx_b = a.ldx * (FMT == QL_I8A8_G128_BF16 ? 1 : 2);
+            for (int t = 0; t < rows_x; ++t)
+                bulk_load(xs_base + (uint32_t)(t * R), xsrc + t * ldx_b + (long long)gs0 * XGB, row_bytes, xbar);
+        }
+    }
+    {
+        const int pieces = ngs * XGB / 16;
+        for (int i = threadIdx.x; i < (NT * 8 - rows_x) * pieces; i += kThreads) {
+            const int t = rows_x + i / pieces, j = i % pieces;
+            *reinterpret_cast<uint4*>(xs + t * R + 16 * j) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    if constexpr (FMT == QL_I8A8_G128_BF16) {  // activation scales of the units already in flight
+        UnitPos q = cp;
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) {
+            if (u0 + s < issued) load_side_x<FMT, NT>(sd[s], a.xf, a.M, a.Gtot, a.g0 + q.grp(GP), c);
+            q.next(slabs, GP, G);
+        }
+    }
+    QL_PROF(4)
+    __syncthreads();
+    QL_PROF(5)
+    if (u0 >= u1) return;
+    bool timed_out = rows_x > 0 && !mbar_wait(xbar, 0);
+    QL_PROF(1)
+
     const bool nt1_live = NT > 1 && a.M > 8;
     float yacc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = yacc[nt][2] = yacc[nt][3] = 0.0f;
-    int cur_slab = (int)(u0 / G);
+    int cur_key = cp.part * slabs + cp.slab;
 
-    auto flush = [&](int slab) {
+    auto flush = [&](int key) {
+        const int slab = key % slabs;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -337,64 +659,100 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny(SkinnyArgs a) {
                 const int t = 8 * nt + 2 * c + (i & 1);
                 const int n = slab * 16 + g + 8 * (i >> 1);
                 if (t < a.M && n < a.N) {
-                    const float f = (FMT == QL_I8A8_G128_BF16) ? 1.0f : fac[t];
+                    const float f = (FMT == QL_I8A8_G128_BF16) ? 1.0f : __ldg(a.xf + t);
                     atomicAdd(a.y + (long long)t * a.ldy + n, yacc[nt][i] * f);
                 }
                 yacc[nt][i] = 0.0f;
             }
     };
 
-    auto process = [&](const Regs<FMT>& r, long long u) {
-        const int slab = (int)(u / G), grp = (int)(u % G);
-        if (!ACC && slab != cur_slab) {
-            flush(cur_slab);
-            cur_slab = slab;
-        }
-        auto getx = [&](int nt, int p) -> uint4 {
-            // p: piece of the lane's chunk; for int4 bit 3 of p selects the 64-wide half
-            int j;
-            if constexpr (FMT == QL_I8A8_G128_BF16)
-                j = grp * 8 + 2 * c + p;
-            else if constexpr (FMT == QL_I4_G64_BF16)
-                j = grp * 16 + (p & 8) + 2 * c + (p & 1);
-            else
-                j = grp * 16 + 4 * c + p;
-            return lds128(xs_base + (uint32_t)((8 * nt + g) * R + 16 * swz<FMT>(j)));
-        };
-        if constexpr (FMT == QL_I8A8_G128_BF16) {
-            int acc[NT][4];
-            unit_w8a8<NT>(r, getx, acc);
+    unsigned phase = 0;
+    unsigned u = u0;
+    while (u < u1 && !timed_out) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+        for (int s = 0; s < kStages; ++s) {
+            if (u >= u1) break;
+            const int key = cp.part * slabs + cp.slab;
+            if (!ACC && key != cur_key) {
+                flush(cur_key);
+                cur_key = key;
+            }
+            if (!mbar_wait(bars + 8 * s, phase)) {
+                timed_out = true;
+                break;
+            }
+            Regs<FMT> r;
+            side_to_regs<FMT, NT>(r, sd[s]);
+            read_unit_smem<FMT>(r, ring + s * SB, g, c);
+            const int grp = cp.grp(GP);
+            const int lg = grp - gs0;  // group index in the staged activations
+            auto getx = [&](int nt, int p) -> uint4 {
+                int j;
+                if constexpr (FMT == QL_I8A8_G128_BF16)
+                    j = lg * 8 + 4 * p + c;
+                else if constexpr (FMT == QL_I4_G64_BF16)
+                    j = lg * 16 + (p & 8) + 2 * c + (p & 1);
+                else if constexpr (FMT == QL_I5Z_G128_F16) {
+                    j = lg * 16 + 4 * c + p;
+                    j ^= (j >> 3) & 1;
+                } else
+                    j = lg * 16 + (p >> 1) * 8 + 2 * c + (p & 1);
+                return lds128(xs_base + (uint32_t)((8 * nt + g) * R + 16 * j));
+            };
+            if constexpr (FMT == QL_I8A8_G128_BF16) {
+                int acc[NT][4];
+                unit_w8a8<NT>(r, getx, acc);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = 8 * nt + 2 * c + (i & 1);
-                    const int n = slab * 16 + g + 8 * (i >> 1);
-                    if (ACC) {
-                        if (t < a.M && n < a.N) a.acc[((long long)t * a.N + n) * a.Gtot + a.g0 + grp] = acc[nt][i];
-                    } else {
-                        const float sc = r.s[i >> 1] * fac[t * G + grp];
-                        yacc[nt][i] = fmaf(sc, __int2float_rn(acc[nt][i]), yacc[nt][i]);
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int t = 8 * nt + 2 * c + (i & 1);
+                        const int n = cp.slab * 16 + g + 8 * (i >> 1);
+                        if (ACC) {
+                            if (t < a.M && n < a.N)
+                                a.acc[((long long)t * a.N + n) * a.Gtot + a.g0 + grp] = acc[nt][i];
+                        } else {
+                            // |acc| <= 128 * 127^2 < 2^22: the magic-number conversion is exact.
+                            const float fa = __int_as_float(0x4B400000 + acc[nt][i]) - 12582912.0f;
+                            yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s].sx[nt][i & 1], fa, yacc[nt][i]);
+                        }
                     }
+            } else {
+                unit_a16<FMT, NT>(r, getx, nt1_live, yacc);
+            }
+            __syncwarp();
+            if (issued < u1) {  // refill this slot with the unit kStages ahead
+                if (lane == 0) {
+                    mbar_expect_tx(bars + 8 * s, SB);
+                    tma_load_2d(ring + s * SB, &a.tmap, ip.grp(GP) * unit_row_bytes<FMT>(), ip.slab * 16,
+                                bars + 8 * s);
                 }
-        } else {
-            unit_a16<FMT, NT>(r, getx, nt1_live, yacc);
+                load_side_w<FMT, NT>(sd[s], a.scales, a.zeros, a.N, a.Gtot, a.g0 + ip.grp(GP), ip.slab, g);
+                load_side_x<FMT, NT>(sd[s], a.xf, a.M, a.Gtot, a.g0 + ip.grp(GP), c);
+                ip.next(slabs, GP, G);
+                ++issued;
+            }
+            cp.next(slabs, GP, G);
+            ++u;
         }
-    };
-
-    long long u = u0;
-    while (u < u1) {
-        if (u + 2 < u1) load(r2, u + 2);
-        process(r0, u);
-        if (++u >= u1) break;
-        if (u + 2 < u1) load(r0, u + 2);
-        process(r1, u);
-        if (++u >= u1) break;
-        if (u + 2 < u1) load(r1, u + 2);
-        process(r2, u);
-        ++u;
+        phase ^= 1u;
     }
-    if (!ACC) flush(cur_slab);
+    if (timed_out) {
+        if (lane == 0) atomicOr(a.err, (unsigned)QL_DEVERR_TIMEOUT);
+        if (rows_x > 0) mbar_wait(xbar, 0);
+        // Let the copies still in flight land before the CTA's memory is released.
+        for (unsigned v = u; v < issued; ++v) {
+            const int s = (int)((v - u0) % kStages);
+            const unsigned ph = ((v - u0) / kStages) & 1u;
+            if (!mbar_wait(bars + 8 * s, ph)) break;
+        }
+        return;
+    }
+    if (!ACC) flush(cur_key);
+#ifdef QL_SKINNY_PROFILE
+    if (lane == 0 && blockIdx.x < 148) atomicMax(&g_skinny_prof[blockIdx.x * 16 + 15], (unsigned long long)(clock64() - prof_c0));
+    if (threadIdx.x == 0 && blockIdx.x < 148) g_skinny_prof[blockIdx.x * 16 + 6] = clock64() - prof_c0;
+#endif
 }
 
 // Grouped (MoE) skinny GEMM: units are (row chunk of one expert, slab, group);
@@ -487,20 +845,131 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_skinny(MoeArgs a) {
     flush(cur_key);
 }
 
+// ---- host side of the dense kernel -------------------------------------------------
+
+// Tensor maps of the packed weights, cached by (address, shape, format): the
+// encoding is host work that repeats for every call on the same weight.
+struct TmapKey {
+    const void* ptr;
+    long long rows, width, ldw;
+    int box_x, swz;
+    bool operator==(const TmapKey& o) const {
+        return ptr == o.ptr && rows == o.rows && width == o.width && ldw == o.ldw && box_x == o.box_x && swz == o.swz;
+    }
+};
+std::mutex g_tmap_mu;
+TmapKey g_tmap_keys[64];
+CUtensorMap g_tmap_vals[64];
+int g_tmap_n = 0, g_tmap_next = 0;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+cudaError_t weight_tmap(const void* W, long long rows, long long width, long long ldw, int box_x, int swz,
+                        CUtensorMap* out) {
+    std::lock_guard<std::mutex> lock(g_tmap_mu);
+    const TmapKey key{W, rows, width, ldw, box_x, swz};
+    for (int i = 0; i < g_tmap_n; ++i)
+        if (g_tmap_keys[i] == key) {
+            *out = g_tmap_vals[i];
+            return cudaSuccess;
+        }
+    if (!g_encode) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+            cudaGetLastError();
+            return cudaErrorNotSupported;
+        }
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldw};
+    const cuuint32_t box[2] = {(cuuint32_t)box_x, 16u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUtensorMap m;
+    const CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(W), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, static_cast<CUtensorMapSwizzle>(swz),
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const int slot = g_tmap_n < 64 ? g_tmap_n++ : (g_tmap_next++ & 63);
+    g_tmap_keys[slot] = key;
+    g_tmap_vals[slot] = m;
+    *out = m;
+    return cudaSuccess;
+}
+
+template <int FMT>
+int swizzle_mode() {
+    return FMT == QL_I4_G64_BF16 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : (FMT == QL_I5Z_G128_F16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Groups of activations one CTA can stage next to its rings.
+template <int FMT>
+int max_staged_groups(int NT, size_t smem_optin) {
+    for (int xg = 256; xg >= 1; --xg)
+        if (tma_smem<FMT>(NT, xg) <= smem_optin) return xg;
+    return 0;
+}
+
+// Largest K-part size GP whose parts, as the CTAs' contiguous unit ranges cut
+// them, never need more than XG staged groups in one CTA.
+int plan_parts(int G, int slabs, int ctas, int XG) {
+    for (int GP = G; GP >= 1; --GP) {
+        const long long units = (long long)slabs * G, per = (long long)slabs * GP;
+        int worst = 0;
+        for (int b = 0; b < ctas; ++b) {
+            const long long cu0 = units * b / ctas, cu1 = units * (b + 1) / ctas;
+            if (cu1 <= cu0) continue;
+            const long long p0 = cu0 / per, p1 = (cu1 - 1) / per;
+            const int ngs = (int)(std::min<long long>(G, (p1 + 1) * GP) - p0 * GP);
+            worst = std::max(worst, ngs);
+        }
+        if (worst <= XG) return GP;
+    }
+    return 0;
+}
+
 template <int FMT, int NT, bool ACC>
-cudaError_t run_skinny(const SkinnyArgs& a, cudaStream_t s, const DeviceInfo& di) {
-    const size_t smem = skinny_smem<FMT>(NT, a.G);
-    if (smem > di.smem_optin) return cudaErrorInvalidValue;
+cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& di) {
+    SkinnyArgs a = in;
+    const int XG = max_staged_groups<FMT>(NT, di.smem_optin);
+    if (XG < 1) return cudaErrorInvalidValue;
+    a.XG = XG;
+    a.GP = plan_parts(a.G, (a.N + 15) / 16, di.sm_count, XG);
+    if (a.GP < 1) return cudaErrorInvalidValue;
+    if ((long long)((a.N + 15) / 16) * a.G * (di.sm_count + 1) >= (1LL << 31)) return cudaErrorInvalidValue;
+    a.err = di.err_word;
+    cudaError_t e = weight_tmap(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw, unit_row_bytes<FMT>(),
+                                swizzle_mode<FMT>(), &a.tmap);
+    if (e != cudaSuccess) return e;
+    const size_t smem = tma_smem<FMT>(NT, XG);
     static bool attr_set[64] = {};  // per device ordinal
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_skinny<FMT, NT, ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)di.smem_optin);
+        e = cudaFuncSetAttribute(k_skinny_tma<FMT, NT, ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)di.smem_optin);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(k_skinny_tma<FMT, NT, ACC>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_set[dev] = true;
     }
-    k_skinny<FMT, NT, ACC><<<di.sm_count, kThreads, smem, s>>>(a);
+    // Programmatic dependent launch: the kernel may start while the kernel before
+    // it (the activation prologue) finishes; it waits for it before touching x.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(di.sm_count);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_skinny_tma<FMT, NT, ACC>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -515,13 +984,29 @@ cudaError_t run_skinny_fmt(const SkinnyArgs& a, cudaStream_t s, const DeviceInfo
 int skinny_max_k(int fmt) {
     DeviceInfo di;
     if (device_info(&di) != cudaSuccess) return 0;
-    for (int G = 256; G >= 1; --G) {
-        size_t need = fmt == QL_I8A8_G128_BF16 ? skinny_smem<QL_I8A8_G128_BF16>(2, G)
-                                                : skinny_smem<QL_I8_G128_BF16>(2, G);
-        if (need <= di.smem_optin) return G * 128;
+    int xg = 0;
+    switch (fmt) {
+    case QL_I8A8_G128_BF16: xg = max_staged_groups<QL_I8A8_G128_BF16>(2, di.smem_optin); break;
+    case QL_I4_G64_BF16: xg = max_staged_groups<QL_I4_G64_BF16>(2, di.smem_optin); break;
+    case QL_I5Z_G128_F16: xg = max_staged_groups<QL_I5Z_G128_F16>(2, di.smem_optin); break;
+    default: xg = max_staged_groups<QL_I8_G128_BF16>(2, di.smem_optin); break;
     }
-    return 0;
+    return xg * 128;  // with G <= XG a single part always fits
 }
+
+#ifdef QL_SKINNY_PROFILE
+__global__ void k_empty_bigsmem() { extern __shared__ uint8_t sm[]; if (threadIdx.x == 9999) sm[0] = 1; }
+extern "C" int ql_prof_empty_launch(void* stream) {
+    DeviceInfo di;
+    device_info(&di);
+    cudaFuncSetAttribute(k_empty_bigsmem, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)di.smem_optin);
+    k_empty_bigsmem<<<di.sm_count, kThreads, di.smem_optin - 1024, (cudaStream_t)stream>>>();
+    return cudaGetLastError() == cudaSuccess ? 0 : 5;
+}
+extern "C" int ql_skinny_prof_read(unsigned long long* out, int n) {
+    return cudaMemcpyFromSymbol(out, g_skinny_prof, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : 5;
+}
+#endif
 
 cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     DeviceInfo di;

@@ -285,6 +285,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
             a.ldw = (long long)fmt_row_bytes(fmt, K);
             a.ldx = K;
             a.ldy = N;
+            a.pdl = 1;  // preceded by this call's prologue (or the previous K chunk)
             const int t = trace_begin(QL_KIND_SKINNY, s);
             e = launch_skinny(fmt, a, s);
             trace_end(t, s);

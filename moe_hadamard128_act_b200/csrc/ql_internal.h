@@ -2,6 +2,7 @@
 // and the kernel translation units.  Nothing here is exported.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -57,6 +58,7 @@ cudaError_t launch_check_zeros(const uint8_t* z_in, size_t n, uint8_t* z_out, un
 
 // ---- skinny GEMM (M <= 16 per launch) -----------------------------------------------
 struct SkinnyArgs {
+    CUtensorMap tmap;      // filled by launch_skinny: W as [N rows][G units], box [16][unit bytes]
     const uint8_t* W;      // packed codes, row stride ldw bytes; already offset to group g0
     const void* scales;    // [N][Gtot] (fp8: [N/128][Gtot]); indexed with g0 + g
     const uint8_t* zeros;  // int5: [N][Gtot]
@@ -64,7 +66,10 @@ struct SkinnyArgs {
     const float* xf;       // A16: [M] inverse token factors; W8A8: sx [M][Gtot]
     float* y;              // [M][ldy]
     int32_t* acc;          // optional W8A8 group sums [M][N][Gtot]
+    unsigned* err;         // device error word (filled by launch_skinny)
     int M, N, G, g0, Gtot;
+    int GP, XG;            // K-part size and staged groups (filled by launch_skinny)
+    int pdl;               // launched right after this library's activation prologue: may overlap it
     long long ldw, ldx, ldy;
 };
 cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s);

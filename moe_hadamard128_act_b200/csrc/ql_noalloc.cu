@@ -91,6 +91,7 @@ extern "C" int qlinear_forward_w8a8_noalloc(const void* x, const void* W_packed,
         a.ldw = K;
         a.ldx = K;
         a.ldy = N;
+        a.pdl = 1;
         if ((e = launch_skinny(QL_I8A8_G128_BF16, a, s)) != cudaSuccess) return QL_ECUDA;
     }
     return QL_OK;
