@@ -388,13 +388,13 @@ def main():
             with torch.cuda.graph(gr, stream=stream):
                 for _ in range(S):
                     step()
-        gr.replay()  # untimed graph warm-up
+            gr.replay()  # untimed graph warm-up, on the launching stream
         stream.synchronize()
         return gr
 
     g = capture(trace=False)
     # clocks pre-roll: about a second of the same load while nvidia-smi samples
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):  # every replay goes to `stream`
         t0 = time.perf_counter()
         n = 0
         while time.perf_counter() - t0 < 1.0:
@@ -426,7 +426,8 @@ def main():
     # library's launch trace (CUDA events around each of its kernels, recorded
     # on the launching stream) captured into the graph ----
     gt = capture(trace=True)
-    gt.replay()
+    with torch.cuda.stream(stream):
+        gt.replay()
     stream.synchronize()
     trace = Q.ql_trace_read(S * launches_per_step)
     Q.ql_trace_enable(0)
