@@ -282,6 +282,26 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                            "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per}
         out["moe_gate_up_decode"] = res
         del codes, scales
+        # prefill W8A8 at M = 2048 (tcgen05 kind::i8 GEMM with per-group fp32 promotion)
+        M = 2048
+        d = synth.prefill(M=M)
+        c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+        x = bf(d["x"])
+        y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+        ws = torch.empty(Q.qlinear_workspace_size(Q.I8A8_G128_BF16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
+                         device=dev)
+        run = lambda i: Q.qlinear_forward(x, c, s, None, Q.I8A8_G128_BF16, N_FULL, y=y, ws=ws,  # noqa: E731
+                                          stream=stream)
+        for i in range(3):
+            run(i)
+        t, _ = _traced(Q, run, 10, "prefill")
+        tq, _ = _traced(Q, run, 10, "act_quant")
+        ops = 2.0 * M * N_FULL * K_FULL
+        peak_i8 = 2.0 * peaks()[1]  # measured bf16 dense burst x the nominal int8 / bf16 ratio of 2
+        out["prefill_w8a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq, "TOPS": ops / (t * 1e-3) / 1e12,
+                               "peak_TOPS": peak_i8, "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
+                               "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
+        del c, s, y, ws
     torch.cuda.synchronize()
     return out
 

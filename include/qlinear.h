@@ -232,6 +232,10 @@ enum {
 int ql_trace_enable(int capacity);
 int ql_trace_read(int* kinds, float* ms, int max, int* count);
 
+/* Text of the last CUDA runtime error behind a QL_ECUDA status returned to
+ * this host thread ("no error" if there was none).  Never NULL. */
+const char* ql_last_cuda_error(void);
+
 /* Synchronise `stream`, then read and clear the device error word.
  * Returns QL_OK when it was clear, QL_EDEVICE otherwise (with *bits, if not
  * NULL, set to its QL_DEVERR_* bits), QL_ECUDA if a CUDA call failed. */

@@ -31,9 +31,6 @@
 //  * Partial sums leave through fp32 atomic adds only when a warp's range
 //    leaves a 16-row slab (about twice per warp), into a y the caller zeroed.
 #include <algorithm>
-#include <mutex>
-
-#include <cudaTypedefs.h>
 
 #include "ql_device.cuh"
 #include "ql_internal.h"
@@ -324,51 +321,6 @@ template <int FMT>
 __host__ __device__ constexpr size_t tma_smem(int NT, int XG) {
     return 1024 /* alignment slack */ + ring_bytes<FMT>() + (size_t)kWarps * kStages * 8 + 16 +
            (size_t)NT * 8 * ((size_t)XG * tx_group_bytes<FMT>() + tx_row_pad<FMT>());
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned phase) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(phase)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
-    return t;
-}
-// Wait for phase `phase` of the mbarrier; false after ~kWaitNs without it.
-constexpr unsigned long long kWaitNs = 200ull * 1000 * 1000;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned phase) {
-    if (mbar_try_wait(bar, phase)) return true;
-    const unsigned long long t0 = global_ns();
-    for (unsigned it = 0;; ++it) {
-        if (mbar_try_wait(bar, phase)) return true;
-        if ((it & 255u) == 255u && global_ns() - t0 > kWaitNs) return false;
-    }
-}
-// One contiguous global -> shared copy, completing on an mbarrier (16-byte
-// aligned addresses, size a multiple of 16).
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, unsigned bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-            dst),
-        "l"(tmap), "r"(x), "r"(y), "r"(bar)
-        : "memory");
 }
 
 // Position in the unit stream: K part, row slab, group within the part.
@@ -847,57 +799,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_skinny(MoeArgs a) {
 
 // ---- host side of the dense kernel -------------------------------------------------
 
-// Tensor maps of the packed weights, cached by (address, shape, format): the
-// encoding is host work that repeats for every call on the same weight.
-struct TmapKey {
-    const void* ptr;
-    long long rows, width, ldw;
-    int box_x, swz;
-    bool operator==(const TmapKey& o) const {
-        return ptr == o.ptr && rows == o.rows && width == o.width && ldw == o.ldw && box_x == o.box_x && swz == o.swz;
-    }
-};
-std::mutex g_tmap_mu;
-TmapKey g_tmap_keys[64];
-CUtensorMap g_tmap_vals[64];
-int g_tmap_n = 0, g_tmap_next = 0;
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-cudaError_t weight_tmap(const void* W, long long rows, long long width, long long ldw, int box_x, int swz,
-                        CUtensorMap* out) {
-    std::lock_guard<std::mutex> lock(g_tmap_mu);
-    const TmapKey key{W, rows, width, ldw, box_x, swz};
-    for (int i = 0; i < g_tmap_n; ++i)
-        if (g_tmap_keys[i] == key) {
-            *out = g_tmap_vals[i];
-            return cudaSuccess;
-        }
-    if (!g_encode) {
-        cudaDriverEntryPointQueryResult q;
-        void* fn = nullptr;
-        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
-            cudaGetLastError();
-            return cudaErrorNotSupported;
-        }
-        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    }
-    const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)ldw};
-    const cuuint32_t box[2] = {(cuuint32_t)box_x, 16u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    CUtensorMap m;
-    const CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(W), dims, strides, box, estr,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, static_cast<CUtensorMapSwizzle>(swz),
-                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    const int slot = g_tmap_n < 64 ? g_tmap_n++ : (g_tmap_next++ & 63);
-    g_tmap_keys[slot] = key;
-    g_tmap_vals[slot] = m;
-    *out = m;
-    return cudaSuccess;
-}
-
 template <int FMT>
 int swizzle_mode() {
     return FMT == QL_I4_G64_BF16 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -940,8 +841,8 @@ cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& d
     if (a.GP < 1) return cudaErrorInvalidValue;
     if ((long long)((a.N + 15) / 16) * a.G * (di.sm_count + 1) >= (1LL << 31)) return cudaErrorInvalidValue;
     a.err = di.err_word;
-    cudaError_t e = weight_tmap(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw, unit_row_bytes<FMT>(),
-                                swizzle_mode<FMT>(), &a.tmap);
+    cudaError_t e = make_tmap_2d(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw, unit_row_bytes<FMT>(), 16,
+                                 swizzle_mode<FMT>(), &a.tmap);
     if (e != cudaSuccess) return e;
     const size_t smem = tma_smem<FMT>(NT, XG);
     static bool attr_set[64] = {};  // per device ordinal

@@ -104,7 +104,12 @@ using namespace ql;
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? QL_OK : QL_ECUDA; }
+thread_local cudaError_t g_last_cuda = cudaSuccess;  // reported by ql_last_cuda_error
+int from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return QL_OK;
+    g_last_cuda = e;
+    return QL_ECUDA;
+}
 
 // Activations prepared for the skinny GEMM: f16 [M][K] + factors [M] (A16), or
 // int8 [M][K] + fp32 scales [M][K/128] (W8A8).
@@ -210,12 +215,13 @@ int qlinear_pack(const float* W, const void* codes_in, const void* scales_in, co
     }
     DeviceInfo di;
     cudaError_t e = device_info(&di);
-    if (e != cudaSuccess) return QL_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     int t = trace_begin(QL_KIND_PACK, s);
     e = launch_pack_codes(codes_in, fmt, N, K, codes_out, di.err_word, s);
     trace_end(t, s);
-    if (e != cudaSuccess) return QL_ECUDA;
-    if ((e = cudaMemcpyAsync(scales_out, scales_in, sb, cudaMemcpyDeviceToDevice, s)) != cudaSuccess) return QL_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
+    if ((e = cudaMemcpyAsync(scales_out, scales_in, sb, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+        return from_cuda(e);
     if (fmt == QL_I5Z_G128_F16) {
         t = trace_begin(QL_KIND_PACK, s);
         e = launch_check_zeros(zeros_in, zb, zeros_out, di.err_word, s);
@@ -253,6 +259,17 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     void* xs = wsb;
     float* xf = reinterpret_cast<float*>(wsb + w.x_bytes);
     cudaError_t e;
+    if (fmt == QL_I8A8_G128_BF16 && M >= kPrefillMinM) {  // tensor-core GEMM, y written directly
+        int t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, nullptr, 0, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_PREFILL, s);
+        e = launch_prefill_w8a8(static_cast<const int8_t*>(xs), xf, static_cast<const int8_t*>(W_packed),
+                                static_cast<const uint16_t*>(scales), M, N, K, y, N, nullptr, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     const long long ny = (long long)M * N;  // the prologue zeroes y for the accumulating GEMM
     if (fmt == QL_I8A8_G128_BF16) {
         const int t = trace_begin(QL_KIND_ACT_QUANT, s);
@@ -263,7 +280,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         e = launch_prep_a16(x, M, K, rot, x_order(fmt), static_cast<__half*>(xs), xf, y, ny, s);
         trace_end(t, s);
     }
-    if (e != cudaSuccess) return QL_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
 
     const size_t xelem = fmt == QL_I8A8_G128_BF16 ? 1 : 2;
     for (int m0 = 0; m0 < M; m0 += 16) {
@@ -289,7 +306,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
             const int t = trace_begin(QL_KIND_SKINNY, s);
             e = launch_skinny(fmt, a, s);
             trace_end(t, s);
-            if (e != cudaSuccess) return QL_ECUDA;
+            if (e != cudaSuccess) return from_cuda(e);
         }
     }
     return QL_OK;
@@ -302,6 +319,12 @@ int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int
     if (kmax < 128) return QL_ECUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int G = K / 128;
+    if (M >= kPrefillMinM) {  // the same tensor-core GEMM qlinear_forward runs at this M
+        const int t = trace_begin(QL_KIND_PREFILL, s);
+        const cudaError_t e = launch_prefill_w8a8(qx, nullptr, qw, nullptr, M, N, K, nullptr, N, acc, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     for (int m0 = 0; m0 < M; m0 += 16) {
         for (int k0 = 0; k0 < K; k0 += kmax) {
             const int kc = K - k0 < kmax ? K - k0 : kmax;
@@ -322,7 +345,7 @@ int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int
             const int t = trace_begin(QL_KIND_SKINNY, s);
             cudaError_t e = launch_skinny(QL_I8A8_G128_BF16, a, s);
             trace_end(t, s);
-            if (e != cudaSuccess) return QL_ECUDA;
+            if (e != cudaSuccess) return from_cuda(e);
         }
     }
     return QL_OK;
@@ -398,11 +421,11 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     e = launch_prep_a16(x, T, K, (experts->flags & QL_HADAMARD) ? 1 : 0, XORD_NATURAL, xs, xf, y,
                         (long long)T * topk * N, s);
     trace_end(t, s);
-    if (e != cudaSuccess) return QL_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     t = trace_begin(QL_KIND_MOE_PERMUTE, s);
     e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, chunks, nch, di.err_word, s);
     trace_end(t, s);
-    if (e != cudaSuccess) return QL_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     MoeArgs a;
     a.codes = static_cast<const uint8_t*>(experts->codes);
     a.scales = experts->scales;
@@ -458,6 +481,8 @@ int ql_trace_read(int* kinds, float* ms, int max, int* count) {
     *count = g_used;
     return QL_OK;
 }
+
+const char* ql_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 
 int ql_get_device_error(void* stream, unsigned* bits) {
     DeviceInfo di;

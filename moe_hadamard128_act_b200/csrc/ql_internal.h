@@ -28,6 +28,11 @@ void packed_sizes(int fmt, size_t N, size_t K, size_t* codes, size_t* scales, si
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// A TMA tensor map over a 2-D byte matrix: `rows` rows of `width_bytes` bytes,
+// `ld_bytes` apart, box [box_y rows][box_x bytes], swizzle as CUtensorMapSwizzle.
+cudaError_t make_tmap_2d(const void* base, long long rows, long long width_bytes, long long ld_bytes, int box_x,
+                         int box_y, int swz, CUtensorMap* out);
+
 // Per-device facts, cached on first use.
 struct DeviceInfo {
     int sm_count;
@@ -75,6 +80,14 @@ struct SkinnyArgs {
 cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s);
 // Largest K (multiple of 128) one skinny launch stages in shared memory.
 int skinny_max_k(int fmt);
+
+// ---- prefill GEMM (tcgen05) ----------------------------------------------------------------
+// y[M][ldy] (fp32, overwritten) = W8A8 product of int8 activations qx [M][K] with
+// scales sx [M][K/128] and int8 weights qw [N][K] with bf16 scales sw [N][K/128].
+// With acc != null, writes the int32 group sums [M][N][K/128] instead of y.
+cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sx, const int8_t* qw, const uint16_t* sw, int M,
+                                int N, int K, float* y, long long ldy, int32_t* acc, cudaStream_t s);
+constexpr int kPrefillMinM = 17;  // from this many tokens on, W8A8 runs on the tcgen05 GEMM
 
 // ---- MoE -----------------------------------------------------------------------------------
 struct MoeChunk {

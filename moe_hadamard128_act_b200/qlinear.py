@@ -37,7 +37,10 @@ STATUS = {0: "QL_OK", 1: "QL_EINVAL", 2: "QL_EUNSUPPORTED", 3: "QL_EALIGN", 4: "
 class QLError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({lib().ql_status_string(status).decode()})")
+        detail = lib().ql_status_string(status).decode()
+        if status == 5:
+            detail += ": " + lib().ql_last_cuda_error().decode()
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({detail})")
 
 
 class ql_experts(ctypes.Structure):
@@ -52,6 +55,7 @@ _PSZ = ctypes.POINTER(ctypes.c_size_t)
 
 _SIGS = {
     "ql_status_string": (ctypes.c_char_p, [_I]),
+    "ql_last_cuda_error": (ctypes.c_char_p, []),
     "qlinear_packed_sizes": (_I, [_I, _I, _I, _PSZ, _PSZ, _PSZ]),
     "qlinear_pack": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P]),
     "qlinear_workspace_size": (_I, [_I, _I, _I, _I, _I, _PSZ]),

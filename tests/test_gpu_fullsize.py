@@ -109,3 +109,17 @@ def test_moe_gate_up_full(Q, T):
         qr, sr = O.quant_i8_g128(d["W"][e], hadamard=True)
         ref = O.forward(d["x"][t:t + 1], qr.view(np.uint8), sr, None, Q.I8_G128_BF16, Q.HADAMARD, N)
         assert_close(y[t, j][None], ref, f"moe T={T} pair {p}")
+
+
+def test_prefill_w8a8_full(Q):
+    """W8A8 prefill at M=2048, N=21504, K=5376 (no Hadamard transform)."""
+    d = synth.prefill()
+    c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N_FULL, K_FULL, W=dev(d["W"]))
+    del d["W"]
+    y = Q.qlinear_forward(dev_bf16(d["x"]), c, s, None, Q.I8A8_G128_BF16, N_FULL).cpu().numpy()
+    rows = sample_rows(N_FULL, seed=55, n_rand=8)
+    Wr = np.concatenate([synth.weight_rows(0, "W", K_FULL, int(n), 1) for n in rows])
+    qr, sr = O.quant_i8_g128(Wr)
+    assert np.array_equal(host_u8(c).reshape(N_FULL, K_FULL)[rows], qr.view(np.uint8))
+    ref = O.forward(d["x"], qr.view(np.uint8), sr, None, Q.I8A8_G128_BF16, 0, len(rows))
+    assert_close(y[:, rows], ref, "prefill W8A8 full")

@@ -233,3 +233,50 @@ def test_moe_duplicate_expert_in_token():
     x = x_bits(T, K, seed=1)
     y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N)
     assert_close(y.cpu().numpy(), O.moe_gate_up(x, ids, codes, scales, 1, 1, E, N))
+
+
+# --------------------------------------------------------------------------
+# Prefill (tcgen05) path: M >= 17 for W8A8
+# --------------------------------------------------------------------------
+PREFILL_SHAPES = [(17, 64, 128), (128, 128, 256), (200, 384, 512), (300, 130, 1024), (129, 257, 384)]
+
+
+@pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
+def test_prefill_group_sums_bitexact(M, N, K):
+    x = x_bits(M, K, seed=31, outliers=0.01)
+    W = synth.weight_rows(31, f"Wpf{N}x{K}", K, 0, N)
+    qw, sw = O.quant_i8_g128(W, hadamard=True)
+    _, acc_ref = O.forward(x, qw.view(np.uint8), sw, None, Q.I8A8_G128_BF16, Q.HADAMARD, N, want_acc=True)
+    qx, _ = O.act_quant_i8_g128(x, rotate=True)
+    qx[0, :128] = 127  # extreme groups: +-127 against +-127
+    qw_ext = qw.copy()
+    qw_ext[0, :128] = -127
+    acc = Q.qlinear_forward_i8_acc(dev(qx), dev(qw_ext))
+    ref = np.einsum("mgk,ngk->mng", qx.reshape(M, K // 128, 128).astype(np.int64),
+                    qw_ext.reshape(N, K // 128, 128).astype(np.int64))
+    assert np.array_equal(acc.cpu().numpy(), ref)
+    assert ref[0, 0, 0] == -128 * 127 * 127
+    del acc_ref
+
+
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
+def test_prefill_forward_parity(M, N, K, had):
+    x = x_bits(M, K, seed=37, outliers=0.01)
+    W = synth.weight_rows(37, f"Wpf{N}x{K}", K, 0, N)
+    c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N, K, W=dev(W), flags=had)
+    y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.I8A8_G128_BF16, N, flags=had)
+    ref = O.forward(x, host_u8(c), host_u8(s).view(np.uint16), None, Q.I8A8_G128_BF16, had, N)
+    assert_close(y.cpu().numpy(), ref, f"prefill {M}x{N}x{K} had {had}")
+
+
+def test_prefill_large_tile_count_and_repeat():
+    # more tiles than SMs (persistent CTAs walk several tiles), called twice
+    M, N, K = 512, 1280, 768
+    x = x_bits(M, K, seed=41)
+    W = synth.weight_rows(41, "Wpf_big", K, 0, N)
+    c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N, K, W=dev(W))
+    ref = O.forward(x, host_u8(c), host_u8(s).view(np.uint16), None, Q.I8A8_G128_BF16, 0, N)
+    for _ in range(2):
+        y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.I8A8_G128_BF16, N)
+        assert_close(y.cpu().numpy(), ref, "prefill 512x1280x768")
