@@ -19,11 +19,13 @@
 //    s_x[m, g] * s_w[n, g] * acc into fp32 running sums held in registers, and
 //    hands the accumulator back.
 // The per-group promotion is the cost centre: both scales change every 128 K,
-// so every output element is touched once per group.  To keep it to three
-// fp32 operations per element, the epilogue re-initialises each accumulator
-// to the bit pattern of 1.5 * 2^23 instead of zero: the MMAs add the group's
-// integer sum to it (|sum| <= 128 * 127^2 < 2^22), so the accumulator read as
-// an fp32 is exactly 12582912 + sum, and one subtraction recovers the sum.
+// so every output element is touched once per group.  To keep it to two fp32
+// FMAs per element, the epilogue re-initialises each accumulator to the bit
+// pattern of 1.5 * 2^23 instead of zero: the MMAs add the group's integer sum
+// to it (|sum| <= 128 * 127^2 < 2^22), so the accumulator read as an fp32 is
+// exactly 12582912 + sum; with the row's activation scale cut to 22
+// significant bits, s_x * 12582912 is exact and one FMA yields s_x * sum
+// rounded once, a second adds s_w * that to the running sum.
 //
 // All waits are bounded (200 ms); a role that gives up sets
 // QL_DEVERR_TIMEOUT and the CTA winds down without leaving tensor memory
@@ -234,23 +236,29 @@ __global__ void __maxnreg__(168) k_prefill_w8a8(const __grid_constant__ PrefillA
         if (lane == 0)
             for (int b = 0; b < NBUF; ++b) mbar_arrive(bars + 8 * (2 * PSTAGES + NBUF + b));
 
-        // Scales of step q (tile, group) for this thread: its row's activation
-        // scale and its column's weight scale (bits), fetched two steps ahead.
-        auto fetch = [&](int q, float& sxv, uint32_t& swv) {
+        // Scales of the steps (tile, group) for this thread, fetched three steps
+        // ahead: its row's activation scale and its column's weight scale bits.
+        int f_tl = 0, f_g = 0;  // position of the next step to fetch
+        auto fetch_next = [&](float& sxv, uint32_t& swv) {
             sxv = 0.0f;
             swv = 0u;
-            if (q >= total) return;
-            const int tl = q / G, g = q - tl * G;
-            const int t = blockIdx.x + tl * gridDim.x;
-            const int m = (t % MB) * PM + row, n = (t / MB) * PN + wg * WGC + ti;
-            if (m < a.M && a.sx) sxv = __ldg(a.sx + (long long)m * G + g);
-            if (ti < WGC && n < a.N && a.sw) swv = __ldg(a.sw + (long long)n * G + g);
+            if (f_tl < my_tiles) {
+                const int t = blockIdx.x + f_tl * gridDim.x;
+                const int mb = t % MB;
+                const int m = mb * PM + row, n = (t - mb) / MB * PN + wg * WGC + ti;
+                if (m < a.M && a.sx) sxv = __ldg(a.sx + (long long)m * G + f_g);
+                if (ti < WGC && n < a.N && a.sw) swv = __ldg(a.sw + (long long)n * G + f_g);
+            }
+            if (++f_g == G) {
+                f_g = 0;
+                ++f_tl;
+            }
         };
         float sx_cur, sx_n1, sx_n2;
         uint32_t sw0, sw_n1, sw_n2;
-        fetch(0, sx_cur, sw0);
-        fetch(1, sx_n1, sw_n1);
-        fetch(2, sx_n2, sw_n2);
+        fetch_next(sx_cur, sw0);
+        fetch_next(sx_n1, sw_n1);
+        fetch_next(sx_n2, sw_n2);
         if (ti < WGC) sw_s[(wg * 2 + 0) * WGC + ti] = __uint_as_float(sw0 << 16);
         wg_sync();
 
@@ -271,29 +279,34 @@ __global__ void __maxnreg__(168) k_prefill_w8a8(const __grid_constant__ PrefillA
             if (!dead) {
                 tc_fence_after();
                 const float* swp = sw_s + (wg * 2 + (k & 1)) * WGC;
+                // s_x truncated to 22 significant bits makes s_x' * 12582912 exact, so
+                // fma(s_x', acc_bits, -s_x' * 12582912) = round(s_x' * sum): one rounding, and
+                // the promotion costs two FMAs per element (relative change of s_x <= 2^-22).
+                const float sxr = __int_as_float(__float_as_int(sx_cur) & ~3);
+                const float kbias = -sxr * 12582912.0f;
 #pragma unroll
-                for (int j = 0; j < WGC / 16; ++j) {
-                    uint32_t v[16];
-                    QL_TMEM_LD16(tmem + tlane + buf * PN + wg * WGC + 16 * j, v);
+                for (int j = 0; j < WGC / 32; ++j) {
+                    uint32_t v[32];
+                    QL_TMEM_LD16(tmem + tlane + buf * PN + wg * WGC + 32 * j, v);
+                    QL_TMEM_LD16(tmem + tlane + buf * PN + wg * WGC + 32 * j + 16, (v + 16));
                     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
                     if constexpr (ACC) {
                         const int m = m0 + row;
                         if (m < a.M)
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int n = n0 + 16 * j + i;
+                            for (int i = 0; i < 32; ++i) {
+                                const int n = n0 + 32 * j + i;
                                 if (n < a.N) a.acc[((long long)m * a.N + n) * G + g] = (int)(v[i] - kMagic);
                             }
                     } else {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 c4 = *reinterpret_cast<const float4*>(swp + 16 * j + 4 * q);
-                            const int e = 16 * j + 4 * q;
-                            // acc read as fp32 is 12582912 + the exact group sum
-                            yr[e + 0] = fmaf(sx_cur * c4.x, __uint_as_float(v[4 * q + 0]) - 12582912.0f, yr[e + 0]);
-                            yr[e + 1] = fmaf(sx_cur * c4.y, __uint_as_float(v[4 * q + 1]) - 12582912.0f, yr[e + 1]);
-                            yr[e + 2] = fmaf(sx_cur * c4.z, __uint_as_float(v[4 * q + 2]) - 12582912.0f, yr[e + 2]);
-                            yr[e + 3] = fmaf(sx_cur * c4.w, __uint_as_float(v[4 * q + 3]) - 12582912.0f, yr[e + 3]);
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 c4 = *reinterpret_cast<const float4*>(swp + 32 * j + 4 * q);
+                            const int e = 32 * j + 4 * q;
+                            yr[e + 0] = fmaf(c4.x, fmaf(sxr, __uint_as_float(v[4 * q + 0]), kbias), yr[e + 0]);
+                            yr[e + 1] = fmaf(c4.y, fmaf(sxr, __uint_as_float(v[4 * q + 1]), kbias), yr[e + 1]);
+                            yr[e + 2] = fmaf(c4.z, fmaf(sxr, __uint_as_float(v[4 * q + 2]), kbias), yr[e + 2]);
+                            yr[e + 3] = fmaf(c4.w, fmaf(sxr, __uint_as_float(v[4 * q + 3]), kbias), yr[e + 3]);
                         }
                     }
                 }
@@ -309,7 +322,7 @@ __global__ void __maxnreg__(168) k_prefill_w8a8(const __grid_constant__ PrefillA
             sx_cur = sx_n1;
             sx_n1 = sx_n2;
             sw_n1 = sw_n2;
-            fetch(k + 3, sx_n2, sw_n2);
+            fetch_next(sx_n2, sw_n2);
             wg_sync();
 
             if (++g == G) {  // tile done: write the warpgroup's 128 x 64 block of y
