@@ -227,7 +227,8 @@ enum {
     QL_KIND_MOE_PERMUTE = 5, /* expert permutation and chunk table              */
     QL_KIND_MOE_GEMM = 6,    /* grouped expert GEMM with fused un-permute        */
     QL_KIND_PACK = 7,        /* weight packing                                  */
-    QL_KIND_PREFILL = 8      /* tensor-core prefill GEMM                        */
+    QL_KIND_PREFILL = 8,     /* tensor-core prefill GEMM                        */
+    QL_KIND_PREFILL_PREP = 9 /* weight scales transposed for the prefill GEMM   */
 };
 int ql_trace_enable(int capacity);
 int ql_trace_read(int* kinds, float* ms, int max, int* count);

@@ -56,7 +56,8 @@ __device__ __forceinline__ void zero_fill(float* y, long long n) {
 
 // s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127).
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bfloat16* x, int M, int K, int rotate,
-                                                                   int8_t* q, float* sx, float* yz, long long nz) {
+                                                                   int8_t* q, float* sx, float* sxT, int Mp,
+                                                                   float* yz, long long nz) {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
     const int lane = threadIdx.x & 31;
@@ -82,7 +83,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
             }
         }
         *reinterpret_cast<uint32_t*>(q + off) = packed;
-        if (lane == 0) sx[u] = s;  // [M][G] row-major: u = m * G + g
+        if (lane == 0) {
+            if (sx) sx[u] = s;                                 // [M][G] row-major: u = m * G + g
+            if (sxT) sxT[(u % G) * Mp + u / G] = s;            // [G][Mp], the prefill GEMM's layout
+        }
     }
 }
 
@@ -182,14 +186,14 @@ cudaError_t launch_rotate_bf16(const void* x, int M, int K, void* y, cudaStream_
     return cudaGetLastError();
 }
 
-cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* yz, long long nz,
-                             cudaStream_t s) {
+cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* sxT, int Mp,
+                             float* yz, long long nz, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
     if ((e = prefer_max_shared(k_act_quant)) != cudaSuccess) return e;
     k_act_quant<<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, yz, nz);
+        static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, sxT, Mp, yz, nz);
     return cudaGetLastError();
 }
 

@@ -111,17 +111,25 @@ int from_cuda(cudaError_t e) {
     return QL_ECUDA;
 }
 
-// Activations prepared for the skinny GEMM: f16 [M][K] + factors [M] (A16), or
-// int8 [M][K] + fp32 scales [M][K/128] (W8A8).
+// Activations prepared for the GEMM: f16 [M][K] + factors [M] (A16), or
+// int8 [M][K] + fp32 scales [M][K/128] (W8A8); for the tensor-core W8A8 GEMM
+// the scales are stored transposed, [K/128][M padded to the tile], followed by
+// the GEMM's own scratch.
 struct FwdWs {
-    size_t x_bytes, f_bytes;
-    size_t total() const { return x_bytes + f_bytes; }
+    size_t x_bytes, f_bytes, g_bytes;
+    size_t total() const { return x_bytes + f_bytes + g_bytes; }
 };
-FwdWs forward_ws(int fmt, size_t M, size_t K) {
+FwdWs forward_ws(int fmt, size_t M, size_t N, size_t K) {
     FwdWs w;
+    w.g_bytes = 0;
     if (fmt == QL_I8A8_G128_BF16) {
         w.x_bytes = align_up(M * K, 256);
-        w.f_bytes = align_up(M * (K / 128) * 4, 256);
+        if (M >= (size_t)kPrefillMinM) {
+            w.f_bytes = align_up((K / 128) * prefill_pad_m((int)M) * 4, 256);
+            w.g_bytes = prefill_scratch_bytes((int)N, (int)K);
+        } else {
+            w.f_bytes = align_up(M * (K / 128) * 4, 256);
+        }
     } else {
         w.x_bytes = align_up(M * K * 2, 256);
         w.f_bytes = align_up(M * 4, 256);
@@ -234,7 +242,7 @@ int qlinear_pack(const float* W, const void* codes_in, const void* scales_in, co
 int qlinear_workspace_size(int fmt, int flags, int M, int N, int K, size_t* bytes) {
     if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD) || !bytes)
         return QL_EINVAL;
-    *bytes = forward_ws(fmt, M, K).total();
+    *bytes = forward_ws(fmt, M, N, K).total();
     return QL_OK;
 }
 
@@ -246,7 +254,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y) ||
         (zeros && !aligned16(zeros)))
         return QL_EALIGN;
-    const FwdWs w = forward_ws(fmt, M, K);
+    const FwdWs w = forward_ws(fmt, M, N, K);
     if (!ws || ws_bytes < w.total()) return QL_EWORKSPACE;
     if (!aligned16(ws)) return QL_EALIGN;
     const int kmax = skinny_max_k(fmt);
@@ -261,19 +269,24 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     cudaError_t e;
     if (fmt == QL_I8A8_G128_BF16 && M >= kPrefillMinM) {  // tensor-core GEMM, y written directly
         int t = trace_begin(QL_KIND_ACT_QUANT, s);
-        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, nullptr, 0, s);
+        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), nullptr, xf, prefill_pad_m(M), nullptr, 0, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        uint8_t* const gs = wsb + w.x_bytes + w.f_bytes;
+        t = trace_begin(QL_KIND_PREFILL_PREP, s);
+        e = launch_prefill_prep(static_cast<const uint16_t*>(scales), N, K, gs, s);
         trace_end(t, s);
         if (e != cudaSuccess) return from_cuda(e);
         t = trace_begin(QL_KIND_PREFILL, s);
-        e = launch_prefill_w8a8(static_cast<const int8_t*>(xs), xf, static_cast<const int8_t*>(W_packed),
-                                static_cast<const uint16_t*>(scales), M, N, K, y, N, nullptr, s);
+        e = launch_prefill_w8a8(static_cast<const int8_t*>(xs), xf, static_cast<const int8_t*>(W_packed), M, N, K, y,
+                                N, nullptr, gs, s);
         trace_end(t, s);
         return from_cuda(e);
     }
     const long long ny = (long long)M * N;  // the prologue zeroes y for the accumulating GEMM
     if (fmt == QL_I8A8_G128_BF16) {
         const int t = trace_begin(QL_KIND_ACT_QUANT, s);
-        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, y, ny, s);
+        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, nullptr, 0, y, ny, s);
         trace_end(t, s);
     } else {
         const int t = trace_begin(QL_KIND_PREP_A16, s);
@@ -321,7 +334,7 @@ int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int
     const int G = K / 128;
     if (M >= kPrefillMinM) {  // the same tensor-core GEMM qlinear_forward runs at this M
         const int t = trace_begin(QL_KIND_PREFILL, s);
-        const cudaError_t e = launch_prefill_w8a8(qx, nullptr, qw, nullptr, M, N, K, nullptr, N, acc, s);
+        const cudaError_t e = launch_prefill_w8a8(qx, nullptr, qw, M, N, K, nullptr, N, acc, nullptr, s);
         trace_end(t, s);
         return from_cuda(e);
     }
@@ -356,7 +369,7 @@ int act_quant_i8_g128(const void* x, int M, int K, int rotate, int8_t* q, float*
     if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return QL_EALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int t = trace_begin(QL_KIND_ACT_QUANT, st);
-    const cudaError_t e = launch_act_quant(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, st);
+    const cudaError_t e = launch_act_quant(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, nullptr, 0, st);
     trace_end(t, st);
     return from_cuda(e);
 }

@@ -49,8 +49,10 @@ enum XOrder { XORD_NATURAL = 0, XORD_I4 = 1, XORD_I5 = 2 };
 cudaError_t launch_rotate_bf16(const void* x, int M, int K, void* y, cudaStream_t s);
 // The act-quant and prep kernels also zero y[0 .. nz) (yz may be null), so the
 // skinny GEMM that follows can accumulate into it without a separate launch.
-cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* yz, long long nz,
-                             cudaStream_t s);
+// act quant writes the scales [M][K/128] to sx and/or transposed, [K/128][Mp],
+// to sxT (either may be null).
+cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* sxT, int Mp,
+                             float* yz, long long nz, cudaStream_t s);
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s);
 
@@ -83,10 +85,19 @@ int skinny_max_k(int fmt);
 
 // ---- prefill GEMM (tcgen05) ----------------------------------------------------------------
 // y[M][ldy] (fp32, overwritten) = W8A8 product of int8 activations qx [M][K] with
-// scales sx [M][K/128] and int8 weights qw [N][K] with bf16 scales sw [N][K/128].
-// With acc != null, writes the int32 group sums [M][N][K/128] instead of y.
-cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sx, const int8_t* qw, const uint16_t* sw, int M,
-                                int N, int K, float* y, long long ldy, int32_t* acc, cudaStream_t s);
+// scales sxT [K/128][Mp] (transposed, Mp = prefill_pad_m(M)) and int8
+// weights qw [N][K] with bf16 scales sw [N][K/128].  `scratch` holds
+// prefill_scratch_bytes(N, K) bytes (the weight scales, transposed to fp32).
+// With acc != null, writes the int32 group sums [M][N][K/128] instead of y;
+// then sxT, sw and scratch are not used.
+constexpr int kPrefillTileM = 128, kPrefillTileN = 256;  // scale arrays are padded to these
+inline int prefill_pad_m(int v) { return (v + kPrefillTileM - 1) / kPrefillTileM * kPrefillTileM; }
+inline int prefill_pad_n(int v) { return (v + kPrefillTileN - 1) / kPrefillTileN * kPrefillTileN; }
+inline size_t prefill_scratch_bytes(int N, int K) { return align_up((size_t)(K / 128) * prefill_pad_n(N) * 4, 256); }
+cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t* qw, int M, int N, int K,
+                                float* y, long long ldy, int32_t* acc, const void* scratch, cudaStream_t s);
+// Fills the scratch: bf16 weight scales [N][K/128] -> fp32 [K/128][pad(N)].
+cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
 constexpr int kPrefillMinM = 17;  // from this many tokens on, W8A8 runs on the tcgen05 GEMM
 
 // ---- MoE -----------------------------------------------------------------------------------

@@ -71,7 +71,8 @@ extern "C" int qlinear_forward_w8a8_noalloc(const void* x, const void* W_packed,
     int8_t* qx = reinterpret_cast<int8_t*>(scratch);
     float* sx = reinterpret_cast<float*>(scratch + kQxBytes);
     // The quantiser also zeroes y, which the GEMM then accumulates into.
-    cudaError_t e = launch_act_quant(x, M, K, (flags & QL_HADAMARD) ? 1 : 0, qx, sx, y, (long long)M * N, s);
+    cudaError_t e = launch_act_quant(x, M, K, (flags & QL_HADAMARD) ? 1 : 0, qx, sx, nullptr, 0, y, (long long)M * N,
+                                     s);
     if (e != cudaSuccess) return QL_ECUDA;
     for (int k0 = 0; k0 < K; k0 += kmax) {
         const int kc = K - k0 < kmax ? K - k0 : kmax;

@@ -74,7 +74,7 @@ _SIGS = {
 }
 
 KIND_NAMES = {1: "rotate", 2: "act_quant", 3: "prep_a16", 4: "skinny", 5: "moe_permute", 6: "moe_gemm", 7: "pack",
-              8: "prefill"}
+              8: "prefill", 9: "prefill_prep"}
 
 _lib = None
 

@@ -271,12 +271,17 @@ def test_prefill_forward_parity(M, N, K, had):
 
 
 def test_prefill_large_tile_count_and_repeat():
-    # more tiles than SMs (persistent CTAs walk several tiles), called twice
-    M, N, K = 512, 1280, 768
+    # 11 x 16 = 176 output tiles of 128 x 256, more than the 148 SMs, so
+    # persistent CTAs walk two tiles each; ragged in both M and N; called twice
+    M, N, K = 1290, 3980, 256
     x = x_bits(M, K, seed=41)
     W = synth.weight_rows(41, "Wpf_big", K, 0, N)
     c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N, K, W=dev(W))
-    ref = O.forward(x, host_u8(c), host_u8(s).view(np.uint16), None, Q.I8A8_G128_BF16, 0, N)
+    ref, acc_ref = O.forward(x, host_u8(c), host_u8(s).view(np.uint16), None, Q.I8A8_G128_BF16, 0, N,
+                             want_acc=True)
     for _ in range(2):
         y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.I8A8_G128_BF16, N)
-        assert_close(y.cpu().numpy(), ref, "prefill 512x1280x768")
+        assert_close(y.cpu().numpy(), ref, f"prefill {M}x{N}x{K}")
+    qx, _ = O.act_quant_i8_g128(x, rotate=False)
+    acc = Q.qlinear_forward_i8_acc(dev(qx), c.view(torch.int8).reshape(N, K))
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
