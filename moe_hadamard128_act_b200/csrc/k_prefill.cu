@@ -4,39 +4,36 @@
 // 128-wide group's integer dot product exact, both scales applied in fp32
 // ("keptn/gemma4-12b-i8g", table "Format").
 //
-// Persistent CTAs, one per SM, walk 128 (tokens) x 256 (weight rows) output
+// Persistent CTAs, one per SM, walk 128 (tokens) x PN (weight rows) output
 // tiles, weight-tile-major so the token blocks that share a weight tile run at
 // the same time and read it from L2.  A step is one (tile, 128-K group): four
-// tcgen05.mma kind::i8 of M = 128, N = 256, K = 32 into one of two 256-column
-// int32 accumulators in tensor memory.  An M = 128 MMA takes about as long at
-// N = 128 as at N = 256, so the full width is what keeps the tensor core busy.
+// tcgen05.mma kind::i8 of M = 128, N = PN, K = 32 into one of 512 / PN int32
+// accumulators in tensor memory, the first of the four overwriting it.  An
+// M = 128 MMA takes about as long at N = 64 as at N = 256, so wide tiles keep
+// the tensor core busy; PN = 192 balances that against the epilogue's
+// registers (it divides the 21504 weight rows of the dense layer, too).
 //
-// All 16 warps run the epilogue; thread i of warp w owns tile row
-// 32 * (w % 4) + i (its tensor-memory lane) and columns 64 * (w / 4) ..
-// + 63.  Per step it reads its 64 accumulators (tcgen05.ld 32x32b, 8
-// columns at a time, the next read in flight while the last is used), resets
-// them, folds s_x[m, g] * s_w[n, g] * sum into 64 fp32 running sums held in
-// registers, and hands the accumulator and the step's scales back.  With 16
-// warps every thread may hold 128 registers; a separate producer or MMA warp
-// would put a fifth warp on one SM sub-partition and cut that to 96.  So lane
-// 0 of warp 0 also drives the pipeline, never blocking on it: between its
-// epilogue steps, and while it waits for its next accumulator, it issues the
-// TMA loads of the activation tile [128][128 B] and the weight tile
-// [256][128 B] (128-byte swizzle) into a 4-slot operand ring, bulk-copies each
-// step's 128 activation scales and 256 weight scales (fp32, transposed
-// beforehand into contiguous runs) into an 8-slot scale ring, and issues a
-// step's MMAs once its operands have landed and its accumulator is free.
+// Warpgroup 0 drives the pipeline and then holds only 24 registers per
+// thread: lane 0 of warp 0 issues the TMA loads of the activation tile
+// [128][128 B] and the weight tile [PN][128 B] (128-byte swizzle) into a
+// 4-slot operand ring and bulk-copies each step's 128 activation scales and
+// PN weight scales (fp32, transposed beforehand into contiguous runs) into an
+// 8-slot scale ring; lane 0 of warp 1 issues the MMAs.  Warps 4..19 (112
+// registers each) are the epilogue: thread i of warp w owns tile row
+// 32 * (w % 4) + i (its tensor-memory lane) and PN / 4 columns.  Per step it
+// reads its accumulators (tcgen05.ld 32x32b, 16 columns at a time, the next
+// read in flight while the last is used), folds s_x[m, g] * s_w[n, g] * sum
+// into fp32 running sums held in registers, and hands the accumulator and the
+// step's scales back.
 //
 // The per-group promotion is the epilogue's cost: both scales change every
 // 128 K, so every output element takes two fp32 FMAs per group.  Two is the
-// least: each accumulator is re-initialised to the bit pattern of 1.5 * 2^23
-// instead of zero, the MMAs add the group's integer sum to it (|sum| <=
-// 128 * 127^2 < 2^22), so the accumulator read as fp32 is exactly 12582912 +
-// sum; with the row's activation scale cut to 22 significant bits (relative
-// change <= 2^-22), s_x * 12582912 is exact, one FMA yields s_x * sum rounded
-// once, a second adds s_w times that to the running sum.  The first runs as
-// packed two-lane FMAs (FFMA2, heavy FMA pipe only), the second as scalar
-// FMAs, so both FMA pipes are busy.
+// least: the integer sum plus 0x4B400000 (|sum| <= 128 * 127^2 < 2^22), read
+// as fp32, is exactly 12582912 + sum; with the row's activation scale cut to
+// 22 significant bits (relative change <= 2^-22), s_x * 12582912 is exact, so
+// one FMA yields s_x * sum rounded once and a second adds s_w times that to
+// the running sum.  The first runs as packed two-lane FMAs (FFMA2, heavy FMA
+// pipe only), the second as scalar FMAs, so both FMA pipes are busy.
 //
 // All waits are bounded (200 ms); on a timeout the CTA sets
 // QL_DEVERR_TIMEOUT and winds down without leaving tensor memory allocated,
@@ -61,12 +58,14 @@ constexpr int SC_BYTES = (PM + PN) * 4;   // s_x of the tile's rows, then s_w of
 constexpr int kEpiWarps = 16;             // warps 4..19; warps 0..3 (warpgroup 0) drive the pipeline
 constexpr int kPThreads = 32 * (4 + kEpiWarps);
 constexpr int WGC = PN / 4;               // columns per thread (per warp column quarter)
-constexpr int CW = 8;                     // columns per tensor-memory read
+constexpr int CW = 16;                    // columns per tensor-memory read
 constexpr int NCH = WGC / CW;             // reads per step
 constexpr uint32_t kMagic = 0x4B400000u;  // 12582912.0f
-static_assert(PN == 256 && NBUF == 2, "one MMA per K chunk covers the tile; two accumulators fill tensor memory");
+static_assert(PN % 32 == 0 && PN >= 128 && PN <= 256 && NBUF >= 2, "one MMA per K chunk covers the tile; 2+ accumulators");
+static_assert(WGC % CW == 0, "whole tensor-memory reads per thread");
+static_assert(PN % 64 == 0 || PN == 160, "tile widths whose column quarters are whole reads");
 static_assert(SCB >= PSTAGES + NBUF, "the scale ring must not throttle the operand ring");
-static_assert((PSTAGES & (PSTAGES - 1)) == 0 && (SCB & (SCB - 1)) == 0, "ring slots from step counters");
+static_assert((PSTAGES & (PSTAGES - 1)) == 0 && (SCB & (SCB - 1)) == 0, "operand and scale slots from step counters");
 
 // Shared memory (from a 1024-aligned base):
 //   [operand ring][scale ring][mbarriers][tmem address]
@@ -85,15 +84,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// kind::i8, D s32, A s8, B s8, both K-major, N = 256, M = 128.
+// kind::i8, D s32, A s8, B s8, both K-major, N = PN, M = 128.
 constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PN >> 3) << 17) |
                               ((uint32_t)(PM >> 4) << 24);
 
-__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc) {
+// D (+)= A * B^T; acc_in = 0 overwrites D.
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc_in) {
     asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, 1, 0;\n"
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdescI8));
+        "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(acc_in));
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
@@ -104,17 +104,6 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
-// Non-blocking: has the phase of the given parity completed?
-__device__ __forceinline__ bool mbar_test(uint32_t bar, unsigned phase) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(phase)
-        : "memory");
-    return ok != 0;
-}
-
 #define QL_TMEM_LD16(addr, v)                                                                                   \
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}," \
                  " [%16];\n"                                                                                    \
@@ -122,15 +111,6 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, unsigned phase) {
                    "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),     \
                    "=r"(v[14]), "=r"(v[15])                                                                    \
                  : "r"(addr))
-#define QL_TMEM_LD8(addr, v)                                                                                  \
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"                      \
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]) \
-                 : "r"(addr))
-#define QL_TMEM_WAIT8(v)                                                                                      \
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n"                                                          \
-                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]) \
-                 :                                                                                           \
-                 : "memory")
 // Waits for this thread's tensor-memory reads; naming the registers of the last
 // read ties their uses to after the wait.
 #define QL_TMEM_WAIT16(v)                                                                                     \
@@ -140,15 +120,6 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, unsigned phase) {
                    "+r"(v[14]), "+r"(v[15])                                                                  \
                  :                                                                                           \
                  : "memory")
-
-__device__ __forceinline__ void tmem_fill_magic32(uint32_t addr) {
-    const uint32_t m = kMagic;
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
-        "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};\n" ::"r"(addr),
-        "r"(m)
-        : "memory");
-}
 
 struct PrefillArgs {
     CUtensorMap tmA;    // int8 activations [M][K], box [128 rows][128 B]
@@ -254,7 +225,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             // K = 32 chunk 2 further.
             const uint64_t da0 = smem_desc_sw128(base), db0 = smem_desc_sw128(base + A_BYTES);
             for (int k = 0; k < total; ++k) {
-                const int s = k & (PSTAGES - 1), b = k & (NBUF - 1);
+                const int s = k & (PSTAGES - 1), b = k % NBUF;
                 if (!mbar_wait(bar(BAR_FULL + s), (k / PSTAGES) & 1) || !mbar_wait(bar(BAR_ACCE + b), (k / NBUF) & 1)) {
                     dead = true;
                     break;
@@ -263,7 +234,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 const uint64_t so = (uint64_t)(s * (STAGE_BYTES >> 4));
                 const uint32_t d = tmem + b * PN;
 #pragma unroll
-                for (int kk = 0; kk < PKB / 32; ++kk) mma_i8(d, da0 + so + 2 * kk, db0 + so + 2 * kk);
+                for (int kk = 0; kk < PKB / 32; ++kk) mma_i8(d, da0 + so + 2 * kk, db0 + so + 2 * kk, kk ? 1u : 0u);
                 mma_commit(bar(BAR_EMPTY + s));  // operand slot free once these MMAs are done
                 mma_commit(bar(BAR_ACCF + b));   // accumulator ready for the epilogue
             }
@@ -280,14 +251,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
         const int tcol = wq * WGC;
         const bool vec_ok = (a.ldy & 3) == 0;
 
-        // Every accumulator starts at the magic value.
-#pragma unroll
-        for (int b = 0; b < NBUF; ++b)
-#pragma unroll
-            for (int j = 0; j < WGC / 32; ++j) tmem_fill_magic32(tmem + tlane + b * PN + tcol + 32 * j);
-        asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
-        tc_fence_before();
-        __syncwarp();
+        // Every accumulator starts free.
         if (lane == 0)
             for (int b = 0; b < NBUF; ++b) mbar_arrive(bar(BAR_ACCE + b));
 
@@ -296,7 +260,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
         for (int i = 0; i < WGC; ++i) yr[i] = 0.0f;
         int t = blockIdx.x, g = 0;
         for (int k = 0; k < total; ++k) {
-            const int b = k & (NBUF - 1), c = k & (SCB - 1);
+            const int b = k % NBUF, c = k & (SCB - 1);
             if (!mbar_wait(bar(BAR_ACCF + b), (k / NBUF) & 1) ||
                 (!ACC && !mbar_wait(bar(BAR_SCF + c), (k / SCB) & 1))) {
                 dead = true;
@@ -314,23 +278,18 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             }
             const float2 sx2 = make_float2(sxr, sxr), kb2 = make_float2(kb, kb);
             uint32_t v[2][CW];
-            QL_TMEM_LD8(taddr, v[0]);
-            QL_TMEM_WAIT8(v[0]);
+            QL_TMEM_LD16(taddr, v[0]);
+            QL_TMEM_WAIT16(v[0]);
 #pragma unroll
             for (int h = 0; h < NCH; ++h) {
                 uint32_t* const cur = v[h & 1];
-                if (h + 1 < NCH) {
-                    QL_TMEM_LD8(taddr + (h + 1) * CW, v[(h + 1) & 1]);  // next read in flight during this one's math
-                } else {
-#pragma unroll
-                    for (int j = 0; j < WGC / 32; ++j) tmem_fill_magic32(taddr + 32 * j);  // all read: reset
-                }
+                if (h + 1 < NCH) QL_TMEM_LD16(taddr + (h + 1) * CW, v[(h + 1) & 1]);  // in flight during this math
                 if constexpr (ACC) {
                     const int m = (t % MB) * PM + row, n0 = (t / MB) * PN + tcol + h * CW;
                     if (m < a.M)
 #pragma unroll
                         for (int i = 0; i < CW; ++i)
-                            if (n0 + i < a.N) a.acc[((long long)m * a.N + n0 + i) * G + g] = (int)(cur[i] - kMagic);
+                            if (n0 + i < a.N) a.acc[((long long)m * a.N + n0 + i) * G + g] = (int)cur[i];
                 } else {
                     // Weight scales read in place (volatile loads stay in their chunk instead of being
                     // hoisted, which would cost registers).
@@ -340,10 +299,11 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                         const uint4 cu = lds128(swa + 16 * q);
                         const float4 cs = make_float4(__uint_as_float(cu.x), __uint_as_float(cu.y),
                                                       __uint_as_float(cu.z), __uint_as_float(cu.w));
-                        const float2 t0 = __ffma2_rn(
-                            sx2, make_float2(__uint_as_float(cur[4 * q]), __uint_as_float(cur[4 * q + 1])), kb2);
-                        const float2 t1 = __ffma2_rn(
-                            sx2, make_float2(__uint_as_float(cur[4 * q + 2]), __uint_as_float(cur[4 * q + 3])), kb2);
+                        // sum + 0x4B400000, read as fp32, is exactly 12582912 + sum
+                        const float2 t0 = __ffma2_rn(sx2, make_float2(__uint_as_float(cur[4 * q] + kMagic),
+                                                                      __uint_as_float(cur[4 * q + 1] + kMagic)), kb2);
+                        const float2 t1 = __ffma2_rn(sx2, make_float2(__uint_as_float(cur[4 * q + 2] + kMagic),
+                                                                      __uint_as_float(cur[4 * q + 3] + kMagic)), kb2);
                         float* const yq = yr + h * CW + 4 * q;
                         yq[0] = fmaf(cs.x, t0.x, yq[0]);
                         yq[1] = fmaf(cs.y, t0.y, yq[1]);
@@ -351,9 +311,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                         yq[3] = fmaf(cs.w, t1.y, yq[3]);
                     }
                 }
-                if (h + 1 < NCH) QL_TMEM_WAIT8(v[(h + 1) & 1]);
+                if (h + 1 < NCH) QL_TMEM_WAIT16(v[(h + 1) & 1]);
             }
-            asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -361,7 +320,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 if (!ACC) mbar_arrive(bar(BAR_SCE + c));
             }
 
-            if (++g == G) {  // tile done: this thread's 64 columns of its row of y
+            if (++g == G) {  // tile done: this thread's WGC columns of its row of y
                 if (!ACC) {
                     const int m = (t % MB) * PM + row, n0 = (t / MB) * PN + tcol;
                     if (m < a.M) {

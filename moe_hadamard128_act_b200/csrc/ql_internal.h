@@ -90,9 +90,13 @@ int skinny_max_k(int fmt);
 // prefill_scratch_bytes(N, K) bytes (the weight scales, transposed to fp32).
 // With acc != null, writes the int32 group sums [M][N][K/128] instead of y;
 // then sxT, sw and scratch are not used.
-constexpr int kPrefillTileM = 128, kPrefillTileN = 256;  // scale arrays are padded to these
+#ifndef QL_PF_N
+#define QL_PF_N 192
+#endif
+constexpr int kPrefillTileM = 128, kPrefillTileN = QL_PF_N;  // output tile; scale arrays are padded to it
 inline int prefill_pad_m(int v) { return (v + kPrefillTileM - 1) / kPrefillTileM * kPrefillTileM; }
 inline int prefill_pad_n(int v) { return (v + kPrefillTileN - 1) / kPrefillTileN * kPrefillTileN; }
+static_assert(kPrefillTileN % 32 == 0, "weight-scale padding is a whole number of 32-wide transpose tiles");
 inline size_t prefill_scratch_bytes(int N, int K) { return align_up((size_t)(K / 128) * prefill_pad_n(N) * 4, 256); }
 cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t* qw, int M, int N, int K,
                                 float* y, long long ldy, int32_t* acc, const void* scratch, cudaStream_t s);
