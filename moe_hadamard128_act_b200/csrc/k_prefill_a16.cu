@@ -1,0 +1,411 @@
+// k_prefill_a16.cu -- the prefill-shaped GEMM (M >= 17 tokens) for the
+// formats whose activations stay 16-bit: int8 codes with a bf16 or f16 scale
+// per row per 128 of K ("gemma4-26b-a4b-dflash-i8" README, table "Weights")
+// and FP8 E4M3 codes with a bf16 scale per 128 x 128 block
+// ("gemma4-26b-a4b-dflash-fp8" README, table "Weights").
+//
+// The tensor cores run kind::f16 (f16 x f16, fp32 accumulation) with the
+// roles turned around: the MMA's M = 128 rows are weight rows, its N = 192
+// columns are tokens.  Both operands are exact:
+//  * the codes are converted to f16 exactly (every int8 and every e4m3 value
+//    is an f16) by a converter warpgroup, which writes them straight into
+//    tensor memory as the MMA's A operand -- no shared-memory round trip for
+//    the widened weights;
+//  * the activations are the f16 copy of x scaled per token by a power of two
+//    (prepared by the activation prologue), loaded by TMA into shared memory
+//    as the B operand.
+// One step is one 128-K group: eight MMAs with K = 16 into one of two fp32
+// accumulators [128 weight rows x 192 tokens].  The epilogue thread that owns
+// a weight row (its tensor-memory lane) folds the group's weight scale, a
+// scalar for that thread, into fp32 running sums: one FMA per element per
+// group.  At the end of a tile each sum is multiplied by its token's inverse
+// factor and written to y (32 lanes of a warp write 32 consecutive y values).
+//
+// Warp roles: warpgroup 0 (24 registers per thread after setmaxnreg): lane 0
+// of warp 0 issues the TMA loads (code tile [128 rows][128 B] into a 4-slot
+// ring, activation tile [192 rows][2 x 128 B] into a 3-slot ring), lane 0 of
+// warp 1 issues the MMAs.  Warpgroup 1 (56 registers) converts: thread i of
+// warp 4 + q converts weight row 32 q + i.  Warpgroups 2..5 (96 registers)
+// are the epilogue: warp w owns rows 32 (w % 4) .. + 31 and tokens
+// 48 ((w - 8) / 4) .. + 47.
+//
+// All waits are bounded (200 ms); on a timeout the CTA sets QL_DEVERR_TIMEOUT
+// and winds down without leaving tensor memory allocated, MMAs running or
+// copies in flight.
+#include "ql_device.cuh"
+#include "ql_internal.h"
+
+namespace ql {
+namespace {
+
+constexpr int TM = 128;                   // weight rows per tile (MMA M)
+constexpr int TN = kPrefillA16Tokens;     // tokens per tile (MMA N)
+constexpr int GK = 128;                   // K per step (one group)
+constexpr int CODE_BYTES = TM * GK;       // one code tile (1-byte codes), 16 KB
+constexpr int XATOM = TN * 128;           // one activation box: [TN rows][64 f16 = 128 B]
+constexpr int X_BYTES = 2 * XATOM;        // the step's activations, 48 KB
+constexpr int CS = 4, XS = 3;             // ring slots
+constexpr int NACC = (512 - 128) / TN;    // fp32 accumulators [128 x TN] in tensor memory (A tiles take 128 columns)
+constexpr int ACOLS = GK / 2;             // tensor-memory columns of one converted A tile (f16 pairs)
+constexpr int A_COL0 = NACC * TN;         // A tiles follow the accumulators
+constexpr uint32_t kTmemCols = 512;
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = 32 * (8 + kEpiWarps);
+constexpr int EPC = TN / 4;               // tokens per epilogue thread
+constexpr int CW = 16;                    // columns per tensor-memory read
+static_assert(A_COL0 + 2 * ACOLS <= (int)kTmemCols, "tensor memory budget");
+static_assert(EPC % CW == 0 && TN % 16 == 0 && TN <= 256, "token tile");
+static_assert(XATOM % 1024 == 0, "activation boxes stay 1024-byte aligned for the 128-byte swizzle");
+
+// Shared memory (from a 1024-aligned base): [code ring][activation ring][mbarriers][tmem address]
+constexpr int X_OFF = CS * CODE_BYTES;
+constexpr int BAR_OFF = X_OFF + XS * X_BYTES;
+constexpr int B_CFULL = 0, B_CEMPTY = CS, B_XFULL = 2 * CS, B_XEMPTY = 2 * CS + XS, B_AFULL = 2 * CS + 2 * XS,
+              B_AEMPTY = B_AFULL + 2, B_DFULL = B_AEMPTY + 2, B_DEMPTY = B_DFULL + NACC, B_DRAIN = B_DEMPTY + NACC,
+              NBARS = B_DRAIN + 1;
+constexpr int MISC_OFF = (BAR_OFF + 8 * NBARS + 15) / 16 * 16;
+constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+
+// Registers: 768 threads launch with 80 each (61440).  Warpgroup 0 drops to
+// 24, the converters to 56, the epilogue rises to 96: 128 * (24 + 56) +
+// 512 * 96 = 59392.  Per SM sub-partition: 32 * (24 + 56 + 4 * 96) = 14848.
+constexpr int kRegsDriver = 24, kRegsConv = 56, kRegsEpi = 96;
+static_assert(128 * (kRegsDriver + kRegsConv) + 32 * kEpiWarps * kRegsEpi <= kThreads * 80, "register split");
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    // K-major, 128-byte swizzle: 8-row atoms 1024 bytes apart (SBO), version 1.
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+// kind::f16: D f32, A f16, B f16, both K-major, N = TN, M = 128.
+constexpr uint32_t kIdescF16 = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(TN >> 3) << 17) |
+                               ((uint32_t)(TM >> 4) << 24);
+
+// D (+)= A * B^T with A in tensor memory; acc_in = 0 overwrites D.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t acc_in) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+        "r"(a_tmem), "l"(bdesc), "r"(kIdescF16), "r"(acc_in));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
+#define QL_TMEM_LD16(addr, v)                                                                                   \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}," \
+                 " [%16];\n"                                                                                    \
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),         \
+                   "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),     \
+                   "=r"(v[14]), "=r"(v[15])                                                                    \
+                 : "r"(addr))
+// Waits for this thread's tensor-memory reads; naming the registers of the last
+// read ties their uses to after the wait.
+#define QL_TMEM_WAIT16(v)                                                                                     \
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"                                                          \
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),       \
+                   "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]),   \
+                   "+r"(v[14]), "+r"(v[15])                                                                  \
+                 :                                                                                           \
+                 : "memory")
+#define QL_TMEM_ST16(addr, w)                                                                                   \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+                 "%15,%16};\n" ::"r"(addr),                                                                     \
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),       \
+                 "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])  \
+                 : "memory")
+
+struct A16Args {
+    CUtensorMap tmW;      // codes [N][K] bytes, box [128 rows][128 B]
+    CUtensorMap tmX;      // f16 activations [M][K] as bytes, box [TN rows][128 B]
+    const uint16_t* sw;   // scales: [N][G] (int8 formats) or [ceil(N/128)][G] (fp8), bf16 or f16 bits
+    const float* xf;      // [M] inverse token factors
+    float* y;             // [M][ldy]
+    unsigned* err;
+    int M, N, G;
+    long long ldy;
+};
+
+template <int FMT>
+__device__ __forceinline__ float scale_of(const A16Args& a, int n, int g) {
+    if (FMT == QL_FP8_B128_BF16) return bf16_bits_to_float(a.sw[(long long)(n / 128) * a.G + g]);
+    if (n >= a.N) return 0.0f;
+    const uint16_t b = a.sw[(long long)n * a.G + g];
+    return FMT == QL_I8_G128_F16 ? f16_bits_to_float(b) : bf16_bits_to_float(b);
+}
+
+// 16 codes (bytes of u) -> 8 f16 pairs, element order kept (low half = lower k).
+template <int FMT>
+__device__ __forceinline__ void convert16(const uint4 u, uint32_t* w) {
+    const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (FMT == QL_FP8_B128_BF16) {
+            w[2 * i] = e4m3x2_to_f16x2(q[i] & 0xFFFFu);
+            w[2 * i + 1] = e4m3x2_to_f16x2(q[i] >> 16);
+        } else {
+            i8x4_to_f16(q[i], w[2 * i], w[2 * i + 1]);
+        }
+    }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_constant__ A16Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const gb = smem_raw + (base - raw);
+    auto bar = [&](int i) { return base + BAR_OFF + 8u * (uint32_t)i; };
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gb + MISC_OFF);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int WB = (a.N + TM - 1) / TM, TB = (a.M + TN - 1) / TN;
+    const int tiles = WB * TB;  // weight-block-major: t -> (wb = t / TB, tb = t % TB)
+    const int my_tiles = (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int G = a.G;
+    const int total = my_tiles * G;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < CS; ++s) {
+            mbar_init(bar(B_CFULL + s), 1);  // expect_tx
+            mbar_init(bar(B_CEMPTY + s), 4);  // one arrive per converter warp
+        }
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(bar(B_XFULL + s), 1);   // expect_tx
+            mbar_init(bar(B_XEMPTY + s), 1);  // MMA commit
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_AFULL + s), 4);   // one arrive per converter warp
+            mbar_init(bar(B_AEMPTY + s), 1);  // MMA commit
+        }
+        for (int s = 0; s < NACC; ++s) {
+            mbar_init(bar(B_DFULL + s), 1);          // MMA commit
+            mbar_init(bar(B_DEMPTY + s), kEpiWarps);  // one arrive per epilogue warp
+        }
+        mbar_init(bar(B_DRAIN), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool dead = false;
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsDriver));
+        if (warp == 0 && lane == 0) {  // ---- producer ----
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmW) : "memory");
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmX) : "memory");
+            int g = 0, t = blockIdx.x, kc = 0, kx = 0;  // code / activation copies issued
+            int n0 = (t / TB) * TM, m0 = (t % TB) * TN;
+            for (int k = 0; k < total; ++k) {
+                const int c = k % CS, x = k % XS;
+                if (!mbar_wait(bar(B_CEMPTY + c), ((k / CS) & 1) ^ 1)) {
+                    dead = true;
+                    break;
+                }
+                const uint32_t cb = bar(B_CFULL + c);
+                mbar_expect_tx(cb, CODE_BYTES);
+                tma_load_2d(base + c * CODE_BYTES, &a.tmW, g * GK, n0, cb);
+                ++kc;
+                if (!mbar_wait(bar(B_XEMPTY + x), ((k / XS) & 1) ^ 1)) {
+                    dead = true;
+                    break;
+                }
+                const uint32_t xb = bar(B_XFULL + x), xd = base + X_OFF + x * X_BYTES;
+                mbar_expect_tx(xb, X_BYTES);
+                tma_load_2d(xd, &a.tmX, g * GK * 2, m0, xb);
+                tma_load_2d(xd + XATOM, &a.tmX, g * GK * 2 + 128, m0, xb);
+                ++kx;
+                if (++g == G) {
+                    g = 0;
+                    t += gridDim.x;
+                    n0 = (t / TB) * TM;
+                    m0 = (t % TB) * TN;
+                }
+            }
+            // Copies still in flight must land before the CTA's shared memory is released.
+            for (int j = kc > CS ? kc - CS : 0; j < kc; ++j)
+                if (!mbar_wait(bar(B_CFULL + j % CS), (j / CS) & 1)) break;
+            for (int j = kx > XS ? kx - XS : 0; j < kx; ++j)
+                if (!mbar_wait(bar(B_XFULL + j % XS), (j / XS) & 1)) break;
+        } else if (warp == 1 && lane == 0) {  // ---- MMA issuer ----
+            const uint64_t xd0 = smem_desc_sw128(base + X_OFF);
+            for (int k = 0; k < total; ++k) {
+                const int x = k % XS, ab = k & 1, db = k % NACC;
+                if (!mbar_wait(bar(B_XFULL + x), (k / XS) & 1) || !mbar_wait(bar(B_AFULL + ab), (k / 2) & 1) ||
+                    !mbar_wait(bar(B_DEMPTY + db), ((k / NACC) & 1) ^ 1)) {
+                    dead = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + db * TN, at = tmem + A_COL0 + ab * ACOLS;
+                const uint64_t xo = (uint64_t)((x * X_BYTES) >> 4);
+#pragma unroll
+                for (int j = 0; j < GK / 16; ++j)
+                    mma_f16_ts(d, at + 8 * j, xd0 + xo + (uint64_t)((j / 4) * (XATOM >> 4) + (j % 4) * 2),
+                               j ? 1u : 0u);
+                mma_commit(bar(B_XEMPTY + x));   // activation slot free once these MMAs are done
+                mma_commit(bar(B_AEMPTY + ab));  // converted weights free
+                mma_commit(bar(B_DFULL + db));   // accumulator ready for the epilogue
+            }
+            // Every MMA issued must finish before tensor memory is freed.
+            mma_commit(bar(B_DRAIN));
+            mbar_wait(bar(B_DRAIN), 0);
+        }
+    } else if (warp < 8) {  // ---- converters ----
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsConv));
+        const int q = warp & 3, r = 32 * q + lane;  // weight row within the tile
+        const uint32_t tl = (uint32_t)(32 * q) << 16;
+        for (int k = 0; k < total; ++k) {
+            const int c = k % CS, ab = k & 1;
+            if (!mbar_wait(bar(B_CFULL + c), (k / CS) & 1) || !mbar_wait(bar(B_AEMPTY + ab), ((k / 2) & 1) ^ 1)) {
+                dead = true;
+                break;
+            }
+            tc_fence_after();
+            // Row r of the code tile: 16-byte chunk j sits at chunk j ^ (r & 7) (128-byte swizzle).
+            const uint32_t rowp = base + c * CODE_BYTES + r * 128;
+            const uint32_t at = tmem + tl + A_COL0 + ab * ACOLS;
+#pragma unroll
+            for (int j = 0; j < GK / 32; ++j) {
+                uint32_t w[16];
+                convert16<FMT>(lds128(rowp + (((2 * j) ^ (r & 7)) << 4)), w);
+                convert16<FMT>(lds128(rowp + (((2 * j + 1) ^ (r & 7)) << 4)), w + 8);
+                QL_TMEM_ST16(at + 16 * j, w);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(B_AFULL + ab));
+                mbar_arrive(bar(B_CEMPTY + c));
+            }
+        }
+    } else {  // ---- epilogue ----
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsEpi));
+        const int q = warp & 3, cg = (warp - 8) >> 2;
+        const uint32_t tl = (uint32_t)(32 * q) << 16;
+        float yacc[EPC];
+#pragma unroll
+        for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
+        int t = blockIdx.x, g = 0;
+        int n = (t / TB) * TM + 32 * q + lane;
+        float s_next = my_tiles > 0 ? scale_of<FMT>(a, n, 0) : 0.0f;
+        for (int k = 0; k < total; ++k) {
+            const int db = k % NACC;
+            const float s = s_next;
+            {  // the next step's scale, one step ahead
+                int gn = g + 1, tn = t;
+                if (gn == G) {
+                    gn = 0;
+                    tn += gridDim.x;
+                }
+                if (k + 1 < total) s_next = scale_of<FMT>(a, (tn / TB) * TM + 32 * q + lane, gn);
+            }
+            if (!mbar_wait(bar(B_DFULL + db), (k / NACC) & 1)) {
+                dead = true;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dt = tmem + tl + db * TN + cg * EPC;
+#pragma unroll
+            for (int h = 0; h < EPC / CW; ++h) {
+                uint32_t v[CW];
+                QL_TMEM_LD16(dt + h * CW, v);
+                QL_TMEM_WAIT16(v);
+#pragma unroll
+                for (int i = 0; i < CW; ++i) yacc[h * CW + i] = fmaf(s, __uint_as_float(v[i]), yacc[h * CW + i]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
+
+            if (++g == G) {  // tile done: tokens m0 + cg * EPC .. of weight row n
+                const int m0 = (t % TB) * TN + cg * EPC;
+                if (n < a.N) {
+#pragma unroll
+                    for (int i = 0; i < EPC; ++i) {
+                        const int m = m0 + i;
+                        if (m < a.M) a.y[(long long)m * a.ldy + n] = yacc[i] * __ldg(a.xf + m);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
+                g = 0;
+                t += gridDim.x;
+                n = (t / TB) * TM + 32 * q + lane;
+            }
+        }
+    }
+    if (dead) atomicOr(a.err, (unsigned)QL_DEVERR_TIMEOUT);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const A16Args& a, int grid, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(k_prefill_a16<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    k_prefill_a16<FMT><<<grid, kThreads, SMEM_BYTES, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_a16_supported(int fmt) {
+    return fmt == QL_I8_G128_BF16 || fmt == QL_I8_G128_F16 || fmt == QL_FP8_B128_BF16;
+}
+
+cudaError_t launch_prefill_a16(int fmt, const __half* xs, const float* xf, const uint8_t* codes, const void* scales,
+                               int M, int N, int K, float* y, long long ldy, cudaStream_t s) {
+    if (!prefill_a16_supported(fmt)) return cudaErrorInvalidValue;
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
+    A16Args a;
+    if ((e = make_tmap_2d(codes, N, K, K, GK, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d(xs, M, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) != cudaSuccess)
+        return e;
+    a.sw = static_cast<const uint16_t*>(scales);
+    a.xf = xf;
+    a.y = y;
+    a.err = di.err_word;
+    a.M = M;
+    a.N = N;
+    a.G = K / GK;
+    a.ldy = ldy;
+    const int tiles = ((N + TM - 1) / TM) * ((M + TN - 1) / TN);
+    const int grid = tiles < di.sm_count ? tiles : di.sm_count;
+    switch (fmt) {
+    case QL_I8_G128_BF16: return launch_fmt<QL_I8_G128_BF16>(a, grid, s);
+    case QL_I8_G128_F16: return launch_fmt<QL_I8_G128_F16>(a, grid, s);
+    default: return launch_fmt<QL_FP8_B128_BF16>(a, grid, s);
+    }
+}
+
+}  // namespace ql

@@ -283,6 +283,17 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         trace_end(t, s);
         return from_cuda(e);
     }
+    if (M >= kPrefillMinM && prefill_a16_supported(fmt)) {  // tensor-core GEMM, y written directly
+        int t = trace_begin(QL_KIND_PREP_A16, s);
+        e = launch_prep_a16(x, M, K, rot, XORD_NATURAL, static_cast<__half*>(xs), xf, nullptr, 0, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_PREFILL, s);
+        e = launch_prefill_a16(fmt, static_cast<const __half*>(xs), xf, static_cast<const uint8_t*>(W_packed), scales,
+                               M, N, K, y, N, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     const long long ny = (long long)M * N;  // the prologue zeroes y for the accumulating GEMM
     if (fmt == QL_I8A8_G128_BF16) {
         const int t = trace_begin(QL_KIND_ACT_QUANT, s);

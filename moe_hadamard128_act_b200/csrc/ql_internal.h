@@ -104,6 +104,19 @@ cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t
 cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
 constexpr int kPrefillMinM = 17;  // from this many tokens on, W8A8 runs on the tcgen05 GEMM
 
+// The same for the formats with 16-bit activations (int8 g128 with bf16 or f16
+// scales, fp8 128x128): y[M][ldy] (fp32, overwritten) from the f16 activations
+// xs [M][K] (natural order, token factors xf [M], as launch_prep_a16 makes
+// them) and the packed codes and scales.  Weight rows are the MMA's M, tokens
+// its N (kPrefillA16Tokens per tile).
+#ifndef QL_A16_TN
+#define QL_A16_TN 192
+#endif
+constexpr int kPrefillA16Tokens = QL_A16_TN;
+bool prefill_a16_supported(int fmt);
+cudaError_t launch_prefill_a16(int fmt, const __half* xs, const float* xf, const uint8_t* codes, const void* scales,
+                               int M, int N, int K, float* y, long long ldy, cudaStream_t s);
+
 // ---- MoE -----------------------------------------------------------------------------------
 struct MoeChunk {
     int expert, start, count;  // rows perm[start .. start+count) of the permuted order

@@ -285,3 +285,23 @@ def test_prefill_large_tile_count_and_repeat():
     qx, _ = O.act_quant_i8_g128(x, rotate=False)
     acc = Q.qlinear_forward_i8_acc(dev(qx), c.view(torch.int8).reshape(N, K))
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+# --------------------------------------------------------------------------
+# Prefill (tcgen05 kind::f16) path: M >= 17 for the 16-bit-activation formats
+# with one-byte codes (int8 + bf16 / f16 scales, fp8 128x128 blocks)
+# --------------------------------------------------------------------------
+A16_PREFILL_SHAPES = [(17, 64, 128), (191, 128, 256), (193, 129, 384), (300, 130, 1024), (400, 6500, 256)]
+
+
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("fmt", [1, 2, 6])  # int8 g128 bf16, int8 g128 f16, fp8 128x128
+@pytest.mark.parametrize("M,N,K", A16_PREFILL_SHAPES)
+def test_prefill_a16_parity(fmt, had, M, N, K):
+    # (400, 6500, 256): 51 x 3 = 153 tiles of 128 weight rows x 192 tokens, more than the SMs
+    (c, s, z), (ch, sh, zh) = make_weights(fmt, N, K, had)
+    x = x_bits(M, K, seed=53, outliers=0.01)
+    for _ in range(2):
+        y = Q.qlinear_forward(dev_bf16(x), c, s, z, fmt, N, flags=had)
+        ref = O.forward(x, ch, sh, zh, fmt, had, N)
+        assert_close(y.cpu().numpy(), ref, f"a16 prefill fmt {fmt} had {had} {M}x{N}x{K}")
