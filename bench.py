@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    p.add_argument("--ncu-case", choices=["skinny_w8a8"], default=None,
+    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8"], default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
 
@@ -281,7 +281,26 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
             res[str(T)] = {"us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
                            "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per}
         out["moe_gate_up_decode"] = res
-        del codes, scales
+        # the same experts at prefill size, T = 2048 (every expert touched)
+        T = 2048
+        ids, _ = synth.routing(200, T, E, topk)
+        xT = bf(synth.activations(0, "x_T2048", T, Ke))
+        idsT = torch.from_numpy(ids).to(dev)
+        yT = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+        run = lambda i: Q.moe_gate_up(xT, idsT, codes, scales, E, Ne, y=yT, stream=stream)  # noqa: E731
+        for i in range(2):
+            run(i)
+        t, per = _traced(Q, run, 5, "moe_gemm")
+        touched = len(set(ids.ravel().tolist()))
+        byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
+        flops = 2.0 * T * topk * Ne * Ke
+        bf16_peak = peaks()[1]
+        t_roof = max(byts / (hbm * 1e9), flops / (bf16_peak * 1e12))
+        out["moe_gate_up_prefill"] = {"T": T, "us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
+                                      "TFLOPS": flops / (t * 1e-3) / 1e12, "roofline_us": 1e6 * t_roof,
+                                      "frac": 1e6 * t_roof / (1e3 * t), "launches_per_call": per,
+                                      "roofline": "max(bytes / measured HBM, flops / measured bf16 peak)"}
+        del codes, scales, xT, idsT, yT
         # prefill W8A8 at M = 2048 (tcgen05 kind::i8 GEMM with per-group fp32 promotion)
         M = 2048
         d = synth.prefill(M=M)
@@ -303,20 +322,53 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                                "peak_TOPS": peak_i8, "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
                                "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
         del c, s, y, ws
+        # prefill with 16-bit activations: fp8 128x128 and int8 g128 bf16 weights (tcgen05 kind::f16)
+        for name, fmt in (("prefill_fp8", Q.FP8_B128_BF16), ("prefill_w8a16", Q.I8_G128_BF16)):
+            c, s, _ = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+            y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+            ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, M, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
+            run = lambda i: Q.qlinear_forward(x, c, s, None, fmt, N_FULL, y=y, ws=ws, stream=stream)  # noqa: E731
+            for i in range(3):
+                run(i)
+            t, _ = _traced(Q, run, 10, "prefill")
+            tq, _ = _traced(Q, run, 10, "prep_a16")
+            tf = ops / (t * 1e-3) / 1e12
+            out[name] = {"M": M, "us_gemm": 1e3 * t, "us_prep_a16": 1e3 * tq, "TFLOPS": tf,
+                         "frac_of_fp8_peak": tf / peak_i8, "frac_of_bf16_peak": tf / peaks()[1],
+                         "peak_source": "MEASURED_PEAKS.json bf16_tflops (x 2 for fp8, nominal ratio)",
+                         "mma": "kind::f16 (exact f16 codes x token-scaled f16 activations)"}
+            del c, s, y, ws
     torch.cuda.synchronize()
     return out
 
 
 def ncu_case(name):
-    """A small, fixed launch sequence for one ncu capture: the W8A8 weight at
-    full size (117 MB codes, two copies so each launch misses L2), M = 16, two
-    warm-up forwards then two more; the skinny GEMM is launch 1..4 of its name."""
+    """A small, fixed launch sequence for one ncu capture.
+    skinny_w8a8: the W8A8 weight at full size (117 MB codes, two copies so each
+    launch misses L2), M = 16, two warm-up forwards then two more; the skinny
+    GEMM is launch 1..4 of its name.
+    prefill_w8a8 / prefill_fp8: the prefill workload (M = 2048, N = 21504,
+    K = 5376; about 0.6 GB on the device), four forwards; the tcgen05 GEMM
+    (k_prefill_w8a8 / k_prefill_a16) is launch 1..4 of its name."""
     import torch
 
     from moe_hadamard128_act_b200 import qlinear as Q
     from moe_hadamard128_act_b200 import synth
 
     dev = torch.device("cuda", 0)
+    if name.startswith("prefill"):
+        fmt = Q.I8A8_G128_BF16 if name == "prefill_w8a8" else Q.FP8_B128_BF16
+        d = synth.prefill(M=2048)
+        c, s, _ = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+        x = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((2048, N_FULL), dtype=torch.float32, device=dev)
+        for i in range(4):
+            Q.qlinear_forward(x, c, s, None, fmt, N_FULL, y=y)
+        torch.cuda.synchronize()
+        st, bits = Q.ql_get_device_error()
+        assert st == 0, bits
+        print(f"ncu case {name} done")
+        return
     W = torch.from_numpy(synth.weight_rows(0, "W", K_FULL, 0, N_FULL)).to(dev)
     c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N_FULL, K_FULL, W=W, flags=Q.HADAMARD)
     del W
