@@ -24,8 +24,8 @@
 // Warp roles: warpgroup 0 (24 registers per thread after setmaxnreg): lane 0
 // of warp 0 issues the TMA loads (code tile [128 rows][128 B] into a 4-slot
 // ring, activation tile [192 rows][2 x 128 B] into a 3-slot ring), lane 0 of
-// warp 1 issues the MMAs.  Warpgroup 1 (56 registers) converts: thread i of
-// warp 4 + q converts weight row 32 q + i.  Warpgroups 2..5 (96 registers)
+// warp 1 issues the MMAs.  Warpgroup 1 (40 registers) converts: thread i of
+// warp 4 + q converts weight row 32 q + i.  Warpgroups 2..5 (104 registers)
 // are the epilogue: warp w owns rows 32 (w % 4) .. + 31 and tokens
 // 48 ((w - 8) / 4) .. + 47.
 //
@@ -68,9 +68,9 @@ constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
 // Registers: 768 threads launch with 80 each (61440).  Warpgroup 0 drops to
-// 24, the converters to 56, the epilogue rises to 96: 128 * (24 + 56) +
-// 512 * 96 = 59392.  Per SM sub-partition: 32 * (24 + 56 + 4 * 96) = 14848.
-constexpr int kRegsDriver = 24, kRegsConv = 56, kRegsEpi = 96;
+// 24, the converters to 40, the epilogue rises to 104: 128 * (24 + 40) +
+// 512 * 104 = 61440.  Per SM sub-partition: 32 * (24 + 40 + 4 * 104) = 15360.
+constexpr int kRegsDriver = 24, kRegsConv = 40, kRegsEpi = 104;
 static_assert(128 * (kRegsDriver + kRegsConv) + 32 * kEpiWarps * kRegsEpi <= kThreads * 80, "register split");
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
@@ -131,14 +131,6 @@ struct A16Args {
     int M, N, G;
     long long ldy;
 };
-
-template <int FMT>
-__device__ __forceinline__ float scale_of(const A16Args& a, int n, int g) {
-    if (FMT == QL_FP8_B128_BF16) return bf16_bits_to_float(a.sw[(long long)(n / 128) * a.G + g]);
-    if (n >= a.N) return 0.0f;
-    const uint16_t b = a.sw[(long long)n * a.G + g];
-    return FMT == QL_I8_G128_F16 ? f16_bits_to_float(b) : bf16_bits_to_float(b);
-}
 
 // 16 codes (bytes of u) -> 8 f16 pairs, element order kept (low half = lower k).
 template <int FMT>
@@ -301,19 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
 #pragma unroll
         for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
         int t = blockIdx.x, g = 0;
-        int n = (t / TB) * TM + 32 * q + lane;
-        float s_next = my_tiles > 0 ? scale_of<FMT>(a, n, 0) : 0.0f;
+        // This thread's weight row and its scale row for the current tile: one scale per
+        // group, read one step ahead (fp8: the row's 128-row block; rows past N scale 0).
+        auto scale_row = [&](int tt, int& row) -> const uint16_t* {
+            row = (tt / TB) * TM + 32 * q + lane;
+            if (FMT == QL_FP8_B128_BF16) return a.sw + (long long)(row / 128) * G;
+            return row < a.N ? a.sw + (long long)row * G : nullptr;
+        };
+        auto scale_at = [&](const uint16_t* sp, int gg) -> float {
+            if (!sp) return 0.0f;
+            const uint16_t b = __ldg(sp + gg);
+            return FMT == QL_I8_G128_F16 ? f16_bits_to_float(b) : bf16_bits_to_float(b);
+        };
+        int n;
+        const uint16_t* sp = scale_row(t, n);
+        float s_next = my_tiles > 0 ? scale_at(sp, 0) : 0.0f;
         for (int k = 0; k < total; ++k) {
             const int db = k % NACC;
             const float s = s_next;
-            {  // the next step's scale, one step ahead
-                int gn = g + 1, tn = t;
-                if (gn == G) {
-                    gn = 0;
-                    tn += gridDim.x;
-                }
-                if (k + 1 < total) s_next = scale_of<FMT>(a, (tn / TB) * TM + 32 * q + lane, gn);
-            }
+            if (g + 1 < G) s_next = scale_at(sp, g + 1);
             if (!mbar_wait(bar(B_DFULL + db), (k / NACC) & 1)) {
                 dead = true;
                 break;
@@ -332,20 +330,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
 
-            if (++g == G) {  // tile done: tokens m0 + cg * EPC .. of weight row n
+            if (++g == G) {  // tile done: tokens m0 .. m0 + EPC - 1 of weight row n
                 const int m0 = (t % TB) * TN + cg * EPC;
                 if (n < a.N) {
+                    float* yp = a.y + (long long)m0 * a.ldy + n;
+                    const float* xp = a.xf + m0;
+                    const int mcount = a.M - m0;
 #pragma unroll
                     for (int i = 0; i < EPC; ++i) {
-                        const int m = m0 + i;
-                        if (m < a.M) a.y[(long long)m * a.ldy + n] = yacc[i] * __ldg(a.xf + m);
+                        if (i < mcount) *yp = yacc[i] * __ldg(xp + i);
+                        yp += a.ldy;
                     }
                 }
 #pragma unroll
                 for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
                 g = 0;
                 t += gridDim.x;
-                n = (t / TB) * TM + 32 * q + lane;
+                sp = scale_row(t, n);
+                if (k + 1 < total) s_next = scale_at(sp, 0);
             }
         }
     }
