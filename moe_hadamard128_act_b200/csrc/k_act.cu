@@ -100,8 +100,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // f16 holds every bf16 value of the scaled row exactly down to 2^-14 (its
 // normal range); below that the rounding error is under 2^-39 of the row's
 // max, far beneath the fp32 accumulation error of the GEMM.
+// With inv != null the row is written to rows inv[t * topk + j] (j < topk,
+// negative entries skipped) instead of row t: the permuted order of the
+// grouped expert GEMM.
 __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K, int rotate, int order, __half* xs,
-                                                  float* xf, float* yz, long long nz) {
+                                                  float* xf, float* yz, long long nz, const int32_t* inv, int topk) {
     extern __shared__ float row[];
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
@@ -138,6 +141,26 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K,
     }
     __syncthreads();
     const float f = red[0];
+    if (order == XORD_NATURAL) {  // 8 values per 16-byte store
+        const int nrep = inv ? topk : 1;
+        for (int j = 0; j < nrep; ++j) {
+            const long long orow = inv ? (long long)inv[(long long)t * topk + j] : (long long)t;
+            if (orow < 0) continue;
+            uint4* out = reinterpret_cast<uint4*>(xs + orow * K);
+            for (int c = threadIdx.x; c < K / 8; c += 256) {
+                const float* r = row + 8 * c;
+                uint32_t h[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __half2 p = __halves2half2(__float2half_rn(__fmul_rn(r[2 * i], f)),
+                                                     __float2half_rn(__fmul_rn(r[2 * i + 1], f)));
+                    h[i] = *reinterpret_cast<const uint32_t*>(&p);
+                }
+                out[c] = make_uint4(h[0], h[1], h[2], h[3]);
+            }
+        }
+        return;
+    }
     __half* out = xs + (long long)t * K;
     for (int k = threadIdx.x; k < K; k += 256) {
         int src = k;
@@ -206,7 +229,22 @@ cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, 
         e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_prep_a16<<<M, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, order, xs, xf, yz, nz);
+    k_prep_a16<<<M, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, order, xs, xf, yz, nz, nullptr,
+                                    1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, const int32_t* inv, int topk, __half* xs,
+                                    float* xf, cudaStream_t s) {
+    const size_t smem = (size_t)K * sizeof(float);
+    cudaError_t e = prefer_max_shared(k_prep_a16);
+    if (e != cudaSuccess) return e;
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_prep_a16<<<T, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, XORD_NATURAL, xs, xf, nullptr, 0,
+                                    inv, topk);
     return cudaGetLastError();
 }
 

@@ -122,15 +122,27 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
                  : "memory")
 
 struct A16Args {
-    CUtensorMap tmW;      // codes [N][K] bytes, box [128 rows][128 B]
-    CUtensorMap tmX;      // f16 activations [M][K] as bytes, box [TN rows][128 B]
-    const uint16_t* sw;   // scales: [N][G] (int8 formats) or [ceil(N/128)][G] (fp8), bf16 or f16 bits
-    const float* xf;      // [M] inverse token factors
-    float* y;             // [M][ldy]
+    CUtensorMap tmW;       // codes [E * N][K] bytes (E = 1 when dense), box [128 rows][128 B]
+    CUtensorMap tmX;       // f16 activations [M][K] as bytes, box [TN rows][128 B]
+    const uint16_t* sw;    // scales per expert: [N][G] (int8 formats) or [ceil(N/128)][G] (fp8), bf16 or f16 bits
+    const float* xf;       // inverse token factors: [M] (dense) or [T] (grouped, token of pair p = p / topk)
+    float* y;              // dense: [M][ldy]; grouped: [T * topk][N]
     unsigned* err;
     int M, N, G;
     long long ldy;
+    const MoeTile* tiles;  // grouped: the tile table and its length on the device
+    const int* n_tiles;
+    const int32_t* perm;   // grouped: permuted row -> pair index t * topk + j
+    int topk;
 };
+
+// The tile a CTA works on: expert, first activation row, rows, weight block.
+template <bool GRP>
+__device__ __forceinline__ MoeTile tile_at(const A16Args& a, int t, int TB) {
+    if (GRP) return a.tiles[t];
+    const int row0 = (t % TB) * kPrefillA16Tokens;
+    return MoeTile{0, row0, min(kPrefillA16Tokens, a.M - row0), t / TB};
+}
 
 // 16 codes (bytes of u) -> 8 f16 pairs, element order kept (low half = lower k).
 template <int FMT>
@@ -147,7 +159,7 @@ __device__ __forceinline__ void convert16(const uint4 u, uint32_t* w) {
     }
 }
 
-template <int FMT>
+template <int FMT, bool GRP>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_constant__ A16Args a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -158,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int WB = (a.N + TM - 1) / TM, TB = (a.M + TN - 1) / TN;
-    const int tiles = WB * TB;  // weight-block-major: t -> (wb = t / TB, tb = t % TB)
+    // dense: weight-block-major, t -> (wb = t / TB, tb = t % TB); grouped: the permute's table
+    const int tiles = GRP ? *a.n_tiles : WB * TB;
     const int my_tiles = (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int G = a.G;
     const int total = my_tiles * G;
@@ -200,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmW) : "memory");
             asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmX) : "memory");
             int g = 0, t = blockIdx.x, kc = 0, kx = 0;  // code / activation copies issued
-            int n0 = (t / TB) * TM, m0 = (t % TB) * TN;
+            MoeTile ti = my_tiles > 0 ? tile_at<GRP>(a, t, TB) : MoeTile{0, 0, 0, 0};
+            int n0 = ti.expert * a.N + ti.wb * TM, m0 = ti.row0;  // code row in the stacked experts, activation row
             for (int k = 0; k < total; ++k) {
                 const int c = k % CS, x = k % XS;
                 if (!mbar_wait(bar(B_CEMPTY + c), ((k / CS) & 1) ^ 1)) {
@@ -223,8 +237,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 if (++g == G) {
                     g = 0;
                     t += gridDim.x;
-                    n0 = (t / TB) * TM;
-                    m0 = (t % TB) * TN;
+                    if (k + 1 < total) {
+                        ti = tile_at<GRP>(a, t, TB);
+                        n0 = ti.expert * a.N + ti.wb * TM;
+                        m0 = ti.row0;
+                    }
                 }
             }
             // Copies still in flight must land before the CTA's shared memory is released.
@@ -293,20 +310,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
 #pragma unroll
         for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
         int t = blockIdx.x, g = 0;
-        // This thread's weight row and its scale row for the current tile: one scale per
+        // This thread's weight row of the current tile and its scale row: one scale per
         // group, read one step ahead (fp8: the row's 128-row block; rows past N scale 0).
-        auto scale_row = [&](int tt, int& row) -> const uint16_t* {
-            row = (tt / TB) * TM + 32 * q + lane;
-            if (FMT == QL_FP8_B128_BF16) return a.sw + (long long)(row / 128) * G;
-            return row < a.N ? a.sw + (long long)row * G : nullptr;
+        const int NBk = (a.N + TM - 1) / TM;
+        int n = 0, row0 = 0, rows = 0;
+        auto start_tile = [&](int tt) -> const uint16_t* {
+            const MoeTile ti = tile_at<GRP>(a, tt, TB);
+            n = ti.wb * TM + 32 * q + lane;
+            row0 = ti.row0 + cg * EPC;
+            rows = ti.rows - cg * EPC;
+            if (FMT == QL_FP8_B128_BF16) return a.sw + ((long long)ti.expert * NBk + n / 128) * G;
+            return n < a.N ? a.sw + ((long long)ti.expert * a.N + n) * G : nullptr;
         };
         auto scale_at = [&](const uint16_t* sp, int gg) -> float {
             if (!sp) return 0.0f;
             const uint16_t b = __ldg(sp + gg);
             return FMT == QL_I8_G128_F16 ? f16_bits_to_float(b) : bf16_bits_to_float(b);
         };
-        int n;
-        const uint16_t* sp = scale_row(t, n);
+        const uint16_t* sp = my_tiles > 0 ? start_tile(t) : nullptr;
         float s_next = my_tiles > 0 ? scale_at(sp, 0) : 0.0f;
         for (int k = 0; k < total; ++k) {
             const int db = k % NACC;
@@ -330,24 +351,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
 
-            if (++g == G) {  // tile done: tokens m0 .. m0 + EPC - 1 of weight row n
-                const int m0 = (t % TB) * TN + cg * EPC;
+            if (++g == G) {  // tile done: activation rows row0 .. row0 + EPC - 1 against weight row n
                 if (n < a.N) {
-                    float* yp = a.y + (long long)m0 * a.ldy + n;
-                    const float* xp = a.xf + m0;
-                    const int mcount = a.M - m0;
+                    if (GRP) {  // un-permute: row r is the pair perm[r] = t * topk + j
 #pragma unroll
-                    for (int i = 0; i < EPC; ++i) {
-                        if (i < mcount) *yp = yacc[i] * __ldg(xp + i);
-                        yp += a.ldy;
+                        for (int i = 0; i < EPC; ++i)
+                            if (i < rows) {
+                                const int pr = __ldg(a.perm + row0 + i);
+                                a.y[(long long)pr * a.N + n] = yacc[i] * __ldg(a.xf + pr / a.topk);
+                            }
+                    } else {
+                        float* yp = a.y + (long long)row0 * a.ldy + n;
+                        const float* xp = a.xf + row0;
+#pragma unroll
+                        for (int i = 0; i < EPC; ++i) {
+                            if (i < rows) *yp = yacc[i] * __ldg(xp + i);
+                            yp += a.ldy;
+                        }
                     }
                 }
 #pragma unroll
                 for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
                 g = 0;
                 t += gridDim.x;
-                sp = scale_row(t, n);
-                if (k + 1 < total) s_next = scale_at(sp, 0);
+                if (k + 1 < total) {
+                    sp = start_tile(t);
+                    s_next = scale_at(sp, 0);
+                }
             }
         }
     }
@@ -361,19 +391,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
     }
 }
 
-template <int FMT>
+template <int FMT, bool GRP>
 cudaError_t launch_fmt(const A16Args& a, int grid, cudaStream_t s) {
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
         const cudaError_t e =
-            cudaFuncSetAttribute(k_prefill_a16<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            cudaFuncSetAttribute(k_prefill_a16<FMT, GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_set[dev] = true;
     }
-    k_prefill_a16<FMT><<<grid, kThreads, SMEM_BYTES, s>>>(a);
+    k_prefill_a16<FMT, GRP><<<grid, kThreads, SMEM_BYTES, s>>>(a);
     return cudaGetLastError();
+}
+
+template <bool GRP>
+cudaError_t launch_any(int fmt, const A16Args& a, int grid, cudaStream_t s) {
+    switch (fmt) {
+    case QL_I8_G128_BF16: return launch_fmt<QL_I8_G128_BF16, GRP>(a, grid, s);
+    case QL_I8_G128_F16: return launch_fmt<QL_I8_G128_F16, GRP>(a, grid, s);
+    default: return launch_fmt<QL_FP8_B128_BF16, GRP>(a, grid, s);
+    }
 }
 
 }  // namespace
@@ -389,7 +428,7 @@ cudaError_t launch_prefill_a16(int fmt, const __half* xs, const float* xf, const
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
     if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
-    A16Args a;
+    A16Args a{};
     if ((e = make_tmap_2d(codes, N, K, K, GK, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(xs, M, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) != cudaSuccess)
         return e;
@@ -403,11 +442,38 @@ cudaError_t launch_prefill_a16(int fmt, const __half* xs, const float* xf, const
     a.ldy = ldy;
     const int tiles = ((N + TM - 1) / TM) * ((M + TN - 1) / TN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
-    switch (fmt) {
-    case QL_I8_G128_BF16: return launch_fmt<QL_I8_G128_BF16>(a, grid, s);
-    case QL_I8_G128_F16: return launch_fmt<QL_I8_G128_F16>(a, grid, s);
-    default: return launch_fmt<QL_FP8_B128_BF16>(a, grid, s);
-    }
+    return launch_any<false>(fmt, a, grid, s);
+}
+
+cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* xf, const uint8_t* codes,
+                                       const void* scales, int E, int N, int K, int rows_total, const MoeTile* tiles,
+                                       const int* n_tiles, int max_tiles, const int32_t* perm, int topk, float* y,
+                                       cudaStream_t s) {
+    if (!prefill_a16_supported(fmt)) return cudaErrorInvalidValue;
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
+    A16Args a{};
+    if ((e = make_tmap_2d(codes, (long long)E * N, K, K, GK, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) != cudaSuccess)
+        return e;
+    if ((e = make_tmap_2d(xs, rows_total, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) !=
+        cudaSuccess)
+        return e;
+    a.sw = static_cast<const uint16_t*>(scales);
+    a.xf = xf;
+    a.y = y;
+    a.err = di.err_word;
+    a.M = rows_total;
+    a.N = N;
+    a.G = K / GK;
+    a.ldy = N;
+    a.tiles = tiles;
+    a.n_tiles = n_tiles;
+    a.perm = perm;
+    a.topk = topk;
+    const int grid = max_tiles < di.sm_count ? max_tiles : di.sm_count;
+    return launch_any<true>(fmt, a, grid, s);
 }
 
 }  // namespace ql

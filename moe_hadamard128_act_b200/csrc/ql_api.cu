@@ -141,19 +141,34 @@ int x_order(int fmt) {
     return fmt == QL_I4_G64_BF16 ? XORD_I4 : (fmt == QL_I5Z_G128_F16 ? XORD_I5 : XORD_NATURAL);
 }
 
+// The grouped tensor-core GEMM takes over once experts average this many rows.
+bool moe_grouped(const ql_experts* ex, int T, int topk) {
+    return (long long)T * topk >= (long long)kMoePrefillMinRowsPerExpert * ex->E;
+}
 struct MoeWs {
-    size_t xs, xf, counts, offsets, perm, chunks, nch;
+    size_t xs, xf, counts, offsets, perm, chunks, nch, inv, tiles;
+    size_t max_tiles;
     size_t total;
 };
 MoeWs moe_ws(const ql_experts* ex, int T, int topk) {
     MoeWs w;
     size_t o = 0;
-    w.xs = o; o += align_up((size_t)T * ex->K * 2, 256);
+    const bool grp = moe_grouped(ex, T, topk);
+    // f16 activations: one row per token (skinny GEMM) or one per (token, slot) in permuted order
+    w.xs = o; o += align_up((size_t)(grp ? T * topk : T) * ex->K * 2, 256);
     w.xf = o; o += align_up((size_t)T * 4, 256);
     w.counts = o; o += align_up((size_t)ex->E * 4, 256);
     w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
     w.perm = o; o += align_up((size_t)T * topk * 4, 256);
-    w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
+    w.max_tiles = grp ? moe_max_tiles(T, topk, ex->E, kPrefillA16Tokens, (ex->N + 127) / 128) : 0;
+    if (grp) {
+        w.inv = o; o += align_up((size_t)T * topk * 4, 256);
+        w.tiles = o; o += align_up(w.max_tiles * sizeof(MoeTile), 256);
+        w.chunks = 0;
+    } else {
+        w.inv = w.tiles = 0;
+        w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
+    }
     w.nch = o; o += 256;
     w.total = o;
     return w;
@@ -405,7 +420,7 @@ int moe_permute(const int32_t* topk_ids, int T, int topk, int E, int32_t* counts
     if (device_info(&di) != cudaSuccess) return QL_ECUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int t = trace_begin(QL_KIND_MOE_PERMUTE, st);
-    const cudaError_t e = launch_moe_permute(topk_ids, T, topk, E, counts, offsets, perm, nullptr, nullptr, di.err_word, st);
+    const cudaError_t e = launch_moe_permute(topk_ids, T, topk, E, counts, offsets, perm, MoePermuteOut{}, di.err_word, st);
     trace_end(t, st);
     return from_cuda(e);
 }
@@ -440,14 +455,42 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     MoeChunk* chunks = reinterpret_cast<MoeChunk*>(b + w.chunks);
     int* nch = reinterpret_cast<int*>(b + w.nch);
     const int K = experts->K, N = experts->N;
+    const int rot = (experts->flags & QL_HADAMARD) ? 1 : 0;
     cudaError_t e;
+    if (moe_grouped(experts, T, topk)) {  // permute, stage x in permuted order, grouped tensor-core GEMM
+        MoePermuteOut po;
+        po.inv = reinterpret_cast<int32_t*>(b + w.inv);
+        po.tiles = reinterpret_cast<MoeTile*>(b + w.tiles);
+        po.n_tiles = nch;
+        po.tile_rows = kPrefillA16Tokens;
+        po.wblocks = (N + 127) / 128;
+        po.yz = y;  // rows of pairs with a bad expert id are zeroed
+        po.N = N;
+        int t = trace_begin(QL_KIND_MOE_PERMUTE, s);
+        e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_PREP_A16, s);
+        e = launch_prep_a16_scatter(x, T, K, rot, po.inv, topk, xs, xf, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_MOE_GEMM, s);
+        e = launch_prefill_a16_grouped(experts->fmt, xs, xf, static_cast<const uint8_t*>(experts->codes),
+                                       experts->scales, experts->E, N, K, T * topk, po.tiles, nch, (int)w.max_tiles,
+                                       perm, topk, y, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     int t = trace_begin(QL_KIND_PREP_A16, s);  // rotation, f16 staging, and the zeroing of y
-    e = launch_prep_a16(x, T, K, (experts->flags & QL_HADAMARD) ? 1 : 0, XORD_NATURAL, xs, xf, y,
+    e = launch_prep_a16(x, T, K, rot, XORD_NATURAL, xs, xf, y,
                         (long long)T * topk * N, s);
     trace_end(t, s);
     if (e != cudaSuccess) return from_cuda(e);
     t = trace_begin(QL_KIND_MOE_PERMUTE, s);
-    e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, chunks, nch, di.err_word, s);
+    MoePermuteOut po;
+    po.chunks = chunks;
+    po.n_chunks = nch;
+    e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
     trace_end(t, s);
     if (e != cudaSuccess) return from_cuda(e);
     MoeArgs a;

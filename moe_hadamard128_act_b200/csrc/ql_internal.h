@@ -55,6 +55,10 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
                              float* yz, long long nz, cudaStream_t s);
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s);
+// The same for the grouped expert GEMM: token t's f16 row goes to rows
+// inv[t * topk + j] of xs (j < topk, rows < 0 skipped); xf stays per token.
+cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, const int32_t* inv, int topk, __half* xs,
+                                    float* xf, cudaStream_t s);
 
 // ---- packing ---------------------------------------------------------------------
 cudaError_t launch_pack_rtn(const float* W, int fmt, int flags, int N, int K, void* codes, void* scales,
@@ -122,8 +126,38 @@ struct MoeChunk {
     int expert, start, count;  // rows perm[start .. start+count) of the permuted order
 };
 size_t moe_max_chunks(int T, int topk, int E);
+// One tile of the grouped expert GEMM: `rows` permuted rows from `row0` (all
+// of one expert) against weight rows wb * 128 .. + 127 of that expert.
+struct MoeTile {
+    int expert, row0, rows, wb;
+};
+// Optional outputs beyond counts/offsets/perm (each may be null):
+//   chunks / n_chunks: segments cut into <= 16-row chunks (the skinny GEMM's unit);
+//   inv: inv[t * topk + j] = position of the pair in perm, -1 for a bad id;
+//   tiles / n_tiles: segments cut into tile_rows-row blocks x wblocks weight blocks;
+//   yz: the rows y[t * topk + j][0 .. N) of pairs with a bad id are zeroed.
+struct MoePermuteOut {
+    MoeChunk* chunks = nullptr;
+    int* n_chunks = nullptr;
+    int32_t* inv = nullptr;
+    MoeTile* tiles = nullptr;
+    int* n_tiles = nullptr;
+    int tile_rows = 0, wblocks = 0;
+    float* yz = nullptr;
+    int N = 0;
+};
+size_t moe_max_tiles(int T, int topk, int E, int tile_rows, int wblocks);
+// Grouped over experts: codes [E][N][K] and scales stacked per expert, xs the
+// permuted rows (launch_prep_a16_scatter), tiles / n_tiles from the permute;
+// row r of a tile lands in y[perm[r]][0 .. N) scaled by xf[perm[r] / topk].
+cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* xf, const uint8_t* codes,
+                                       const void* scales, int E, int N, int K, int rows_total, const MoeTile* tiles,
+                                       const int* n_tiles, int max_tiles, const int32_t* perm, int topk, float* y,
+                                       cudaStream_t s);
+// From this many (token, slot) pairs per expert on average, moe_gate_up runs the grouped tensor-core GEMM.
+constexpr int kMoePrefillMinRowsPerExpert = 8;
 cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,
-                               int32_t* perm, MoeChunk* chunks, int* n_chunks, unsigned* err, cudaStream_t s);
+                               int32_t* perm, const MoePermuteOut& out, unsigned* err, cudaStream_t s);
 struct MoeArgs {
     const uint8_t* codes;  // [E][N][K]
     const void* scales;    // [E][...] per the format

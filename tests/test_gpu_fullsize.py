@@ -88,7 +88,7 @@ def test_w5a16_full(Q, M):
     assert_close(y[:, rows], ref, f"W5A16 M={M}")
 
 
-@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("T", [1, 16, 2048])
 def test_moe_gate_up_full(Q, T):
     E, topk, K, N = 128, 8, 2816, 1408
     ids, w = synth.routing(0, T, E, topk)

@@ -226,6 +226,39 @@ def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
     assert_close(y.cpu().numpy(), ref, f"moe fmt {fmt} T{T}")
 
 
+@pytest.mark.parametrize("fmt", [1, 2, 6])
+@pytest.mark.parametrize("T,E,topk,N,K", [(64, 8, 4, 130, 384), (300, 16, 8, 200, 256), (50, 64, 8, 128, 128)])
+def test_moe_gate_up_grouped_parity(fmt, T, E, topk, N, K):
+    # T * topk >= 8 E: the grouped tensor-core GEMM. (300, 16, 8): ~150 rows per expert, some over one
+    # 192-row block; N = 200: a ragged second weight block. (50, 64, 8): some experts get no rows.
+    codes, scales = moe_weights(E, N, K, fmt)
+    ids, w = synth.routing(7, T, E, topk)
+    x = x_bits(T, K, seed=17)
+    ref = O.moe_gate_up(x, ids, codes, scales, fmt, O.HADAMARD, E, N)
+    for _ in range(2):
+        y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N, fmt=fmt, flags=Q.HADAMARD,
+                          topk_weights=dev(w))
+        assert_close(y.cpu().numpy(), ref, f"moe grouped fmt {fmt} T{T} E{E}")
+
+
+def test_moe_gate_up_grouped_bad_id():
+    E, N, K, T, topk = 8, 64, 128, 40, 4
+    codes, scales = moe_weights(E, N, K, Q.I8_G128_BF16)
+    ids, _ = synth.routing(8, T, E, topk)
+    ids[5, 2] = 99  # skipped: flagged, its output row zero, every other pair exact
+    x = x_bits(T, K, seed=19)
+    Q.ql_get_device_error()
+    y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N).cpu().numpy()
+    st, bits = Q.ql_get_device_error()
+    assert st == 6 and bits & Q.DEVERR_EXPERT_ID
+    assert np.all(y[5, 2] == 0.0)
+    ids_ok = ids.copy()
+    ids_ok[5, 2] = 0
+    ref = O.moe_gate_up(x, ids_ok, codes, scales, 1, 1, E, N)
+    ref[5, 2] = 0.0
+    assert_close(y, ref, "moe grouped, one bad id")
+
+
 def test_moe_duplicate_expert_in_token():
     E, N, K, T = 4, 64, 128, 3
     codes, scales = moe_weights(E, N, K, Q.I8_G128_BF16)
