@@ -707,94 +707,158 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
 #endif
 }
 
-// Grouped (MoE) skinny GEMM: units are (row chunk of one expert, slab, group);
-// the activations of a chunk's tokens are gathered from the prepared [T, K]
-// buffer (L2-resident) and results are scattered to y[(t, j), :] rows.
+// Grouped (MoE) skinny GEMM: units are (row chunk of one expert, slab, group),
+// in that order.  Every warp streams its contiguous unit range through its own
+// ring of TMA copies, as the dense kernel does, from one tensor map over the
+// stacked experts' codes [E * N][K] (a unit is the box at row expert * N +
+// 16 * slab, byte 128 * group).  The activations of a chunk's (at most 16)
+// tokens are read from the prepared [T, K] buffer, which stays in L2, and the
+// results are added into y[(t, j), :] (zeroed by the prologue).
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, 1) k_moe_skinny(MoeArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__ MoeArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    constexpr int SB = stage_bytes<FMT>();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int G = a.K / 128;
     const int slabs = (a.N + 15) / 16;
     const long long per_chunk = (long long)slabs * G;
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the chunk table comes from the permute kernel
     const long long nch = min((long long)*a.n_chunks, a.max_chunks);
     const long long units = nch * per_chunk;
     const long long wid = (long long)blockIdx.x * kWarps + warp, nw = (long long)gridDim.x * kWarps;
     const long long u0 = units * wid / nw, u1 = units * (wid + 1) / nw;
-    if (u0 >= u1) return;
-    const long long ldw = a.K;  // int8 / fp8 rows
-    const long long expert_codes = (long long)a.N * a.K;
-    const long long expert_scales = FMT == QL_FP8_B128_BF16 ? (long long)((a.N + 127) / 128) * G : (long long)a.N * G;
+    if (lane == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmap) : "memory");
 
-    Regs<FMT> r0, r1, r2;
-    auto load = [&](Regs<FMT>& r, long long u) {
-        const MoeChunk ch = a.chunks[u / per_chunk];
-        const long long rem = u % per_chunk;
-        const int slab = (int)(rem / G), grp = (int)(rem % G);
-        const uint8_t* wb = a.codes + (long long)ch.expert * expert_codes;
-        const void* sb = static_cast<const uint16_t*>(a.scales) + (long long)ch.expert * expert_scales;
-        load_unit<FMT>(r, wb, ldw, sb, nullptr, a.N, G, grp, slab, grp, g, c);
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t ring = base + (uint32_t)(warp * kStages * SB);
+    const uint32_t bars = base + (uint32_t)ring_bytes<FMT>() + (uint32_t)(warp * kStages * 8);
+    if (u0 >= u1) return;
+    const long long expert_scales =
+        FMT == QL_FP8_B128_BF16 ? (long long)((a.N + 127) / 128) * G : (long long)a.N * G;
+    const uint16_t* const sc0 = static_cast<const uint16_t*>(a.scales);
+
+    // Unit position, stepped without divisions: chunk, slab, group.
+    struct Pos {
+        int ch, slab, grp;
+        __device__ void next(int slabs, int G) {
+            if (++grp == G) {
+                grp = 0;
+                if (++slab == slabs) {
+                    slab = 0;
+                    ++ch;
+                }
+            }
+        }
     };
-    if (u0 < u1) load(r0, u0);
-    if (u0 + 1 < u1) load(r1, u0 + 1);
+    Pos cp;
+    cp.ch = (int)(u0 / per_chunk);
+    cp.slab = (int)((u0 % per_chunk) / G);
+    cp.grp = (int)(u0 % G);
+    Pos ip = cp;
+    Side<FMT, NT> sd[kStages];
+    long long issued = u0;
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) mbar_init(bars + 8 * st, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncwarp();
+    auto issue = [&](int st) {
+        const MoeChunk ch = a.chunks[ip.ch];
+        if (lane == 0) {
+            mbar_expect_tx(bars + 8 * st, SB);
+            tma_load_2d(ring + st * SB, &a.tmap, ip.grp * 128, ch.expert * a.N + ip.slab * 16, bars + 8 * st);
+        }
+        load_side_w<FMT, NT>(sd[st], sc0 + (long long)ch.expert * expert_scales, nullptr, a.N, G, ip.grp, ip.slab, g);
+        ip.next(slabs, G);
+        ++issued;
+    };
+#pragma unroll
+    for (int st = 0; st < kStages; ++st)
+        if (issued < u1) issue(st);
 
     float yacc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = yacc[nt][2] = yacc[nt][3] = 0.0f;
-    long long cur_key = u0 / G;  // (chunk, slab)
+    MoeChunk chc = a.chunks[cp.ch];  // the chunk being computed
+    int tok[NT];                     // this lane's tokens in it (-1: none)
+    auto load_tokens = [&]() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int slot = 8 * nt + g;
+            tok[nt] = slot < chc.count ? __ldg(a.perm + chc.start + slot) / a.topk : -1;
+        }
+    };
+    load_tokens();
+    int cur_ch = cp.ch, cur_slab = cp.slab;
 
-    auto flush = [&](long long key) {
-        const MoeChunk ch = a.chunks[key / slabs];
-        const int slab = (int)(key % slabs);
+    auto flush = [&]() {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int slot = 8 * nt + 2 * c + (i & 1);
-                const int n = slab * 16 + g + 8 * (i >> 1);
-                if (slot < ch.count && n < a.N) {
-                    const int pair = a.perm[ch.start + slot];
-                    const float f = a.xf[pair / a.topk];
-                    atomicAdd(a.y + (long long)pair * a.N + n, yacc[nt][i] * f);
+                const int n = cur_slab * 16 + g + 8 * (i >> 1);
+                if (slot < chc.count && n < a.N) {
+                    const int pair = __ldg(a.perm + chc.start + slot);
+                    atomicAdd(a.y + (long long)pair * a.N + n, yacc[nt][i] * __ldg(a.xf + pair / a.topk));
                 }
                 yacc[nt][i] = 0.0f;
             }
     };
 
-    auto process = [&](const Regs<FMT>& r, long long u) {
-        const long long key = u / G;
-        const int grp = (int)(u % G);
-        if (key != cur_key) {
-            flush(cur_key);
-            cur_key = key;
-        }
-        const MoeChunk ch = a.chunks[key / slabs];
-        int tok[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int slot = 8 * nt + g;
-            tok[nt] = slot < ch.count ? a.perm[ch.start + slot] / a.topk : -1;
-        }
-        auto getx = [&](int nt, int p) -> uint4 {
-            if (tok[nt] < 0) return make_uint4(0, 0, 0, 0);
-            return __ldg(reinterpret_cast<const uint4*>(a.xs + (long long)tok[nt] * a.K + grp * 128 + 32 * c + 8 * p));
-        };
-        unit_a16<FMT, NT>(r, getx, ch.count > 8, yacc);
-    };
-
+    bool timed_out = false;
+    unsigned phase = 0;
     long long u = u0;
-    while (u < u1) {
-        if (u + 2 < u1) load(r2, u + 2);
-        process(r0, u);
-        if (++u >= u1) break;
-        if (u + 2 < u1) load(r0, u + 2);
-        process(r1, u);
-        if (++u >= u1) break;
-        if (u + 2 < u1) load(r1, u + 2);
-        process(r2, u);
-        ++u;
+    while (u < u1 && !timed_out) {
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) {
+            if (u >= u1) break;
+            if (cp.ch != cur_ch || cp.slab != cur_slab) {
+                flush();
+                if (cp.ch != cur_ch) {
+                    chc = a.chunks[cp.ch];
+                    load_tokens();
+                }
+                cur_ch = cp.ch;
+                cur_slab = cp.slab;
+            }
+            if (!mbar_wait(bars + 8 * st, phase)) {
+                timed_out = true;
+                break;
+            }
+            Regs<FMT> r;
+            side_to_regs<FMT, NT>(r, sd[st]);
+            read_unit_smem<FMT>(r, ring + st * SB, g, c);
+            const int grp = cp.grp;
+            // The fragments read_unit_smem hands out pair with these 16-byte x pieces of the group
+            // (the same order as the dense kernel's staged activations).
+            auto getx = [&](int nt, int p) -> uint4 {
+                if (tok[nt] < 0) return make_uint4(0, 0, 0, 0);
+                const int j = (p >> 1) * 8 + 2 * c + (p & 1);
+                return __ldg(reinterpret_cast<const uint4*>(a.xs + (long long)tok[nt] * a.K + grp * 128 + 8 * j));
+            };
+            unit_a16<FMT, NT>(r, getx, chc.count > 8, yacc);
+            __syncwarp();
+            if (issued < u1) issue(st);  // refill this slot with the unit kStages ahead
+            cp.next(slabs, G);
+            ++u;
+        }
+        phase ^= 1u;
     }
-    flush(cur_key);
+    if (timed_out) {
+        if (lane == 0) atomicOr(a.err, (unsigned)QL_DEVERR_TIMEOUT);
+        // Let the copies still in flight land before the CTA's memory is released.
+        for (long long v = u; v < issued; ++v) {
+            const int st = (int)((v - u0) % kStages);
+            const unsigned ph = (unsigned)(((v - u0) / kStages) & 1);
+            if (!mbar_wait(bars + 8 * st, ph)) break;
+        }
+        return;
+    }
+    flush();
 }
 
 // ---- host side of the dense kernel -------------------------------------------------
@@ -929,17 +993,45 @@ cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_moe_skinny(const MoeArgs& a, cudaStream_t s) {
+cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
+    MoeArgs a = in;
+    a.err = di.err_word;
+    if ((e = make_tmap_2d(a.codes, (long long)a.E * a.N, a.K, a.K, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmap)) !=
+        cudaSuccess)
+        return e;
+    const size_t smem = 1024 + ring_bytes<QL_I8_G128_BF16>() + (size_t)kWarps * kStages * 8;
+    static bool attr_set[64] = {};  // per device ordinal, for all three instantiations at once
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        for (auto kern : {k_moe_tma<QL_I8_G128_BF16, 2>, k_moe_tma<QL_I8_G128_F16, 2>, k_moe_tma<QL_FP8_B128_BF16, 2>})
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    auto run = [&](auto kern) -> cudaError_t {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(di.sm_count);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 0;  // everything depends on the permute
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t r = cudaLaunchKernelEx(&cfg, kern, a);
+        return r != cudaSuccess ? r : cudaGetLastError();
+    };
     switch (a.fmt) {
-    case QL_I8_G128_BF16: k_moe_skinny<QL_I8_G128_BF16, 2><<<di.sm_count, kThreads, 0, s>>>(a); break;
-    case QL_I8_G128_F16: k_moe_skinny<QL_I8_G128_F16, 2><<<di.sm_count, kThreads, 0, s>>>(a); break;
-    case QL_FP8_B128_BF16: k_moe_skinny<QL_FP8_B128_BF16, 2><<<di.sm_count, kThreads, 0, s>>>(a); break;
+    case QL_I8_G128_BF16: return run(k_moe_tma<QL_I8_G128_BF16, 2>);
+    case QL_I8_G128_F16: return run(k_moe_tma<QL_I8_G128_F16, 2>);
+    case QL_FP8_B128_BF16: return run(k_moe_tma<QL_FP8_B128_BF16, 2>);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace ql

@@ -159,6 +159,8 @@ constexpr int kMoePrefillMinRowsPerExpert = 8;
 cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,
                                int32_t* perm, const MoePermuteOut& out, unsigned* err, cudaStream_t s);
 struct MoeArgs {
+    CUtensorMap tmap;      // filled by launch_moe_skinny: codes as [E * N rows][K bytes], box [16][128 B]
+    unsigned* err;         // device error word (filled by launch_moe_skinny)
     const uint8_t* codes;  // [E][N][K]
     const void* scales;    // [E][...] per the format
     const __half* xs;      // prepared activations [T][K] (natural order)
