@@ -175,13 +175,15 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
                     if (nt == 0 || nt1_live) xv[nt] = getx(nt, 8 * h + p);
 #pragma unroll
                 for (int sub = 0; sub < 2; ++sub) {
-                    const int j = 2 * sub;
-                    const uint32_t w0 = p == 0 ? r.w[0][h].x : r.w[0][h].y;
-                    const uint32_t w1 = p == 0 ? r.w[1][h].x : r.w[1][h].y;
-                    const uint32_t a0 = hadd2_u32(((w0 >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
-                    const uint32_t a2 = hadd2_u32(((w0 >> (4 * j + 4)) & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
-                    const uint32_t a1 = hadd2_u32(((w1 >> (4 * j)) & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
-                    const uint32_t a3 = hadd2_u32(((w1 >> (4 * j + 4)) & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
+                    // Nibble pairs at bits (8 sub, 8 sub + 16) and (8 sub + 4, 8 sub + 20): the low
+                    // nibble of each byte becomes 1024 + u and -1032 leaves q = u - 8; the high nibble,
+                    // masked in place, becomes 1024 + 16 u and one exact FMA (x / 16 - 72) leaves q.
+                    const uint32_t w0 = (p == 0 ? r.w[0][h].x : r.w[0][h].y) >> (8 * sub);
+                    const uint32_t w1 = (p == 0 ? r.w[1][h].x : r.w[1][h].y) >> (8 * sub);
+                    const uint32_t a0 = hadd2_u32((w0 & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
+                    const uint32_t a2 = hfma2_u32((w0 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
+                    const uint32_t a1 = hadd2_u32((w1 & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
+                    const uint32_t a3 = hfma2_u32((w1 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
                         if (nt == 1 && !nt1_live) continue;

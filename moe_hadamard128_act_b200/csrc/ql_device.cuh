@@ -56,6 +56,11 @@ __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+    __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b), *reinterpret_cast<__half2*>(&c));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
 // Four int8 codes (bytes 0..3 of w) -> f16x2 pairs lo = (c0, c1), hi = (c2, c3).
 // Biasing to unsigned u = c + 128 and placing u in the low mantissa byte of
 // 1024.0 gives 1024 + u exactly; adding -1152 leaves c, exact in f16.
