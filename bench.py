@@ -69,6 +69,23 @@ def skinny_bytes(m):
     return N_FULL * K_FULL + N_FULL * G * 2 + m * K_FULL + m * G * 4 + m * N_FULL * 4
 
 
+def replicas_time(ms_local: float, world: int, device) -> float:
+    """The job's time for a replicated step: the slowest rank's (max over ranks)."""
+    if world <= 1:
+        return ms_local
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replicas_value(ms_job: float, world: int, steps: int, bytes_per_step: int) -> float:
+    """Whole-job GB/s of N replicas: every rank moved bytes_per_step per step."""
+    return world * steps * bytes_per_step / (ms_job * 1e-3) / 1e9
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -488,12 +505,8 @@ def main():
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    value = world * args.steps * step_bytes() / (ms * 1e-3) / 1e9
+    ms = replicas_time(ev0.elapsed_time(ev1), world, dev)
+    value = replicas_value(ms, world, args.steps, step_bytes())
 
     # ---- per-kernel durations: the same S steps replayed once more with the
     # library's launch trace (CUDA events around each of its kernels, recorded
@@ -541,12 +554,8 @@ def main():
                 yh[m].copy_(ys[m], non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e = {"value": world * e2e_steps * step_bytes() / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+    e2e_ms = replicas_time(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": replicas_value(e2e_ms, world, e2e_steps, step_bytes()), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     extras = None
