@@ -32,9 +32,9 @@ def _rank(rank: int, world: int, port: int, times, out):
 @pytest.mark.parametrize("times", [(2.0, 3.5), (4.0, 1.0)])
 def test_replicas_max_over_ranks_gloo(times):
     world = 2
-    mgr = mp.Manager()
-    out = mgr.dict()
     ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
     port = _free_port()
     procs = [ctx.Process(target=_rank, args=(r, world, port, list(times), out))
              for r in range(world)]
