@@ -17,14 +17,6 @@ namespace {
 
 constexpr int kWarpsPerBlock = 8;
 
-__device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float v[4]) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(p);
-    v[0] = __uint_as_float(raw.x << 16);
-    v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(raw.y << 16);
-    v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-}
-
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_rotate_bf16(const __nv_bfloat16* x, int M, int K,
                                                                      __nv_bfloat16* y) {
     const int lane = threadIdx.x & 31;
@@ -68,20 +60,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
         float v[4];
         load4_bf16(x + off, v);
         if (rotate) fwht128_warp(v, lane);
-        float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-        amax = warp_max(amax);
-        uint32_t packed = 0;
-        float s = 0.0f;
-        if (amax > 0.0f) {
-            s = __fdiv_rn(amax, 127.0f);
-            const float inv = __fdiv_rn(127.0f, amax);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int c = __float2int_rn(__fmul_rn(v[i], inv));
-                c = max(-127, min(127, c));
-                packed |= (uint32_t)(c & 0xFF) << (8 * i);
-            }
-        }
+        float s;
+        const uint32_t packed = quant_i8_group_warp(v, &s);
         *reinterpret_cast<uint32_t*>(q + off) = packed;
         if (lane == 0) {
             if (sx) sx[u] = s;                                 // [M][G] row-major: u = m * G + g

@@ -49,6 +49,38 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Four consecutive bf16 values (8-byte aligned) as fp32.
+__device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float v[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(raw.x << 16);
+    v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(raw.y << 16);
+    v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+}
+
+// The int8 quantiser of one 128-group held 4 values per lane by a warp:
+// s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127);
+// amax = 0 gives s = 0 and q = 0.  Returns the lane's 4 codes packed low byte
+// first; *s is the group's scale in every lane.
+__device__ __forceinline__ uint32_t quant_i8_group_warp(const float v[4], float* s_out) {
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    amax = warp_max(amax);
+    uint32_t packed = 0;
+    float s = 0.0f;
+    if (amax > 0.0f) {
+        s = __fdiv_rn(amax, 127.0f);
+        const float inv = __fdiv_rn(127.0f, amax);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int c = __float2int_rn(__fmul_rn(v[i], inv));
+            c = max(-127, min(127, c));
+            packed |= (uint32_t)(c & 0xFF) << (8 * i);
+        }
+    }
+    *s_out = s;
+    return packed;
+}
 __device__ __forceinline__ float f16_bits_to_float(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
