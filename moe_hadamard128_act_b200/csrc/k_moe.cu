@@ -1,115 +1,146 @@
 // k_moe.cu -- MoE token permutation for the routed experts' gate_up
 // projection ("gemma4-26b-a4b-dflash-i8", table "Weights").
 //
-// One CTA of 1024 threads groups the T*topk (token, slot) pairs by expert,
-// stably (expert, t, j): a shared-memory histogram and scan give the segment
-// offsets; then the pairs are placed tile by tile (1024 per tile, in input
-// order): inside a warp the peers with the same expert are found with
-// __match_any_sync and ranked by lane, the per-warp counts of each expert are
-// prefix-summed across the 32 warps, and a running per-expert base carries
-// over between tiles.  The same kernel cuts every expert's segment into
-// chunks of at most 16 rows, the unit the grouped skinny GEMM consumes, or
-// into the (row block, weight block) tiles of the grouped tensor-core GEMM,
-// and records each pair's position (the inverse permutation) so that the
-// activation staging can write rows straight into permuted order.
-// Everything stays on the device: the GEMM reads the chunk count itself, so
-// no host round trip sits between routing and the expert GEMM.
+// The T*topk (token, slot) pairs are grouped by expert, stably in (expert, t,
+// j) order, by one CTA per expert, so no CTA waits for another.  Every CTA
+// reads all pair ids once (they stay in L2), with each thread owning a
+// contiguous span: a shared-memory histogram of all experts gives the CTA its
+// segment offset and its first chunk and tile, and the thread's own count of
+// the CTA's expert, scanned across the block, gives where its pairs go.  The
+// threads that hold such pairs read their span again to write them.
+// Each CTA also writes its expert's count and offset, its entries of the
+// inverse permutation, and its chunks of at most 16 rows (the unit of the
+// grouped skinny GEMM) or its (row block, weight block) tiles (the grouped
+// tensor-core GEMM).  One more CTA takes the pairs whose id is outside
+// [0, E): it flags them, marks them in the inverse permutation, zeroes their
+// output rows when asked, fills the tail of perm with -1, and writes the
+// totals.  Everything stays on the device: the GEMMs read the chunk or tile
+// count themselves, so no host round trip sits between routing and the
+// expert GEMM.
 #include "ql_device.cuh"
 #include "ql_internal.h"
 
 namespace ql {
 namespace {
 
-constexpr int kPermThreads = 1024;
+constexpr int kPermThreads = 512;
+
+// Sum of v over the block; every thread gets the result.  red holds a slot per warp.
+__device__ __forceinline__ int block_sum(int v, int* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    int t = 0;
+    for (int w = 0; w < kPermThreads / 32; ++w) t += red[w];
+    return t;
+}
 
 __global__ void __launch_bounds__(kPermThreads) k_moe_permute(const int32_t* ids, int T, int topk, int E,
                                                               int32_t* counts, int32_t* offsets, int32_t* perm,
                                                               const MoePermuteOut o, unsigned* err) {
-    extern __shared__ int sm[];
-    int* cnt = sm;                // [E]
-    int* off = cnt + E;           // [E + 1]
-    int* run = off + E + 1;       // [E]
-    int* whist = run + E;         // [32][E]
-    int* coff = whist + 32 * E;   // [E] first chunk of each expert
-    int* toff = coff + E;         // [E] first tile of each expert
+    extern __shared__ int hist[];  // [E]
+    __shared__ int s_red[kPermThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int P = T * topk;
+    const int e = blockIdx.x;  // this CTA's expert; e == E: the bad ids and the totals
 
-    for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+    for (int x = tid; x < E; x += kPermThreads) hist[x] = 0;
     __syncthreads();
-    int bad = 0;
-    for (int i = tid; i < P; i += kPermThreads) {
-        const int e = ids[i];
-        if (e < 0 || e >= E) {
-            ++bad;
-            if (o.inv) o.inv[i] = -1;
-            if (o.yz)  // the pair is skipped: its output row is zero
-                for (int n = 0; n < o.N; ++n) o.yz[(long long)i * o.N + n] = 0.0f;
+
+    // Each thread owns a contiguous span of ids (a multiple of 4 long, so the
+    // 16-byte loads stay aligned), which keeps the compaction in input order
+    // with a single scan of per-thread counts.
+    const int S = ((P + kPermThreads - 1) / kPermThreads + 3) & ~3;
+    const int b0 = tid * S, b1 = min(P, b0 + S);
+    const bool vec = (P & 3) == 0;  // ids are 16-byte aligned (checked on the host)
+    int mine = 0;
+#pragma unroll 4
+    for (int i = b0; i < b1; i += 4) {
+        int xs[4];
+        if (vec) {
+            const int4 q = __ldg(reinterpret_cast<const int4*>(ids + i));
+            xs[0] = q.x; xs[1] = q.y; xs[2] = q.z; xs[3] = q.w;
         } else {
-            atomicAdd(&cnt[e], 1);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xs[j] = i + j < b1 ? __ldg(ids + i + j) : 0;
         }
-    }
-    if (__syncthreads_or(bad) && tid == 0) atomicOr(err, (unsigned)QL_DEVERR_EXPERT_ID);
-    if (tid == 0) {  // exclusive scans over experts: rows, chunks, tiles
-        int acc = 0, ch = 0, nt = 0;
-        for (int e = 0; e < E; ++e) {
-            const int c = cnt[e];
-            off[e] = acc;
-            run[e] = 0;
-            coff[e] = ch;
-            toff[e] = nt;
-            acc += c;
-            ch += (c + 15) / 16;
-            if (o.tiles) nt += (c + o.tile_rows - 1) / o.tile_rows * o.wblocks;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (i + j >= b1) break;
+            const int x = xs[j];
+            if (x >= 0 && x < E) {
+                atomicAdd(&hist[x], 1);
+                mine += x == e;
+            } else if (e == E) {  // a pair routed to no expert: flagged, its output row zero
+                ++mine;
+                if (o.inv) o.inv[i + j] = -1;
+                if (o.yz)
+                    for (int n = 0; n < o.N; ++n) o.yz[(long long)(i + j) * o.N + n] = 0.0f;
+            }
         }
-        off[E] = acc;
-        if (o.n_chunks) *o.n_chunks = ch;
-        if (o.n_tiles) *o.n_tiles = nt;
     }
     __syncthreads();
-    for (int e = tid; e < E; e += kPermThreads) {  // each expert's chunks and tiles, in parallel
-        const int c = cnt[e], r0 = off[e];
-        if (o.chunks)
-            for (int s = 0, ch = coff[e]; s < c; s += 16, ++ch) o.chunks[ch] = MoeChunk{e, r0 + s, min(16, c - s)};
-        if (o.tiles) {  // weight-block-major within the expert: its row blocks share each weight block
-            int nt = toff[e];
-            for (int wb = 0; wb < o.wblocks; ++wb)
-                for (int s = 0; s < c; s += o.tile_rows, ++nt) o.tiles[nt] = MoeTile{e, r0 + s, min(o.tile_rows, c - s), wb};
-        }
-    }
-    for (int e = tid; e < E; e += kPermThreads) counts[e] = cnt[e];
-    for (int e = tid; e <= E; e += kPermThreads) offsets[e] = off[e];
-    const int valid = off[E];
-    for (int i = valid + tid; i < P; i += kPermThreads) perm[i] = -1;
 
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = 0; base < P; base += kPermThreads) {
-        for (int i = tid; i < 32 * E; i += kPermThreads) whist[i] = 0;
-        __syncthreads();
-        const int i = base + tid;
-        int e = (i < P) ? ids[i] : -1;
-        if (e >= E) e = -1;
-        const unsigned peers = __match_any_sync(kFull, e);
-        const int rank = __popc(peers & lt);
-        if (e >= 0 && rank == 0) whist[warp * E + e] = __popc(peers);
-        __syncthreads();
-        // Exclusive prefix over warps, per expert; whist becomes the warp's base.
-        for (int x = tid; x < E; x += kPermThreads) {
-            int r = run[x];
-            for (int w = 0; w < 32; ++w) {
-                const int c = whist[w * E + x];
-                whist[w * E + x] = r;
-                r += c;
+    // Exclusive sums over the experts before e of rows, chunks and tiles (for
+    // e == E: the totals), each thread taking every 512th expert.
+    int r = 0, ch = 0, nt = 0;
+    for (int x = tid; x < e; x += kPermThreads) {
+        const int c = hist[x];
+        r += c;
+        ch += (c + 15) >> 4;
+        if (o.tiles) nt += (c + o.tile_rows - 1) / o.tile_rows * o.wblocks;
+    }
+    const int r0 = block_sum(r, s_red);
+    const int coff = block_sum(ch, s_red);
+    const int toff = block_sum(nt, s_red);
+
+    if (e == E) {  // ---- bad ids, the tail of perm, the totals ----
+        if (__syncthreads_or(mine) && tid == 0) atomicOr(err, (unsigned)QL_DEVERR_EXPERT_ID);
+        for (int i = r0 + tid; i < P; i += kPermThreads) perm[i] = -1;
+        if (tid == 0) {
+            offsets[E] = r0;
+            if (o.n_chunks) *o.n_chunks = coff;
+            if (o.n_tiles) *o.n_tiles = toff;
+        }
+        return;
+    }
+
+    const int c = hist[e];
+    if (tid == 0) {
+        counts[e] = c;
+        offsets[e] = r0;
+    }
+    // Exclusive scan of the per-thread counts: shuffles within the warp, warp totals across.
+    int incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int up = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += up;
+    }
+    __syncthreads();
+    if (lane == 31) s_red[warp] = incl;
+    __syncthreads();
+    int pos = r0 + incl - mine;
+    for (int w = 0; w < warp; ++w) pos += s_red[w];
+    if (mine > 0)  // second read of the span, now in L1/L2
+        for (int i = b0; i < b1; ++i)
+            if (__ldg(ids + i) == e) {
+                perm[pos] = i;
+                if (o.inv) o.inv[i] = pos;
+                ++pos;
             }
-            run[x] = r;
+
+    if (o.chunks)
+        for (int k = tid; 16 * k < c; k += kPermThreads) o.chunks[coff + k] = MoeChunk{e, r0 + 16 * k, min(16, c - 16 * k)};
+    if (o.tiles) {  // weight-block-major within the expert: its row blocks share each weight block
+        const int nrb = (c + o.tile_rows - 1) / o.tile_rows;
+        for (int k = tid; k < nrb * o.wblocks; k += kPermThreads) {
+            const int wb = k / nrb, rb = k - wb * nrb;
+            o.tiles[toff + k] = MoeTile{e, r0 + rb * o.tile_rows, min(o.tile_rows, c - rb * o.tile_rows), wb};
         }
-        __syncthreads();
-        if (e >= 0) {
-            const int pos = off[e] + whist[warp * E + e] + rank;
-            perm[pos] = i;
-            if (o.inv) o.inv[i] = pos;
-        }
-        __syncthreads();
     }
 }
 
@@ -122,12 +153,9 @@ size_t moe_max_tiles(int T, int topk, int E, int tile_rows, int wblocks) {
 
 cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,
                                int32_t* perm, const MoePermuteOut& out, unsigned* err, cudaStream_t s) {
-    const size_t smem = (size_t)(5 * E + 1 + 32 * E) * sizeof(int);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k_moe_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    k_moe_permute<<<1, kPermThreads, smem, s>>>(ids, T, topk, E, counts, offsets, perm, out, err);
+    const size_t smem = (size_t)E * sizeof(int);
+    if (smem > 48 * 1024) return cudaErrorInvalidValue;  // E <= 1024 (checked by the caller)
+    k_moe_permute<<<E + 1, kPermThreads, smem, s>>>(ids, T, topk, E, counts, offsets, perm, out, err);
     return cudaGetLastError();
 }
 

@@ -54,7 +54,7 @@ constexpr int kThreads = 32 * (8 + kEpiWarps);
 constexpr int EPC = TN / 4;               // tokens per epilogue thread
 constexpr int CW = 16;                    // columns per tensor-memory read
 static_assert(A_COL0 + 2 * ACOLS <= (int)kTmemCols, "tensor memory budget");
-static_assert(EPC % CW == 0 && TN % 16 == 0 && TN <= 256, "token tile");
+static_assert(EPC % CW == 0 && EPC <= 64 && TN % 16 == 0 && TN <= 256, "token tile");
 static_assert(XATOM % 1024 == 0, "activation boxes stay 1024-byte aligned for the 128-byte swizzle");
 
 // Shared memory (from a 1024-aligned base): [code ring][activation ring][mbarriers][tmem address]
@@ -126,7 +126,7 @@ struct A16Args {
     CUtensorMap tmX;       // f16 activations [M][K] as bytes, box [TN rows][128 B]
     const uint16_t* sw;    // scales per expert: [N][G] (int8 formats) or [ceil(N/128)][G] (fp8), bf16 or f16 bits
     const float* xf;       // inverse token factors: [M] (dense) or [T] (grouped, token of pair p = p / topk)
-    float* y;              // dense: [M][ldy]; grouped: [T * topk][N]
+    float* y;              // dense: [M][ldy]; grouped: [T * topk][ldy = N]
     unsigned* err;
     int M, N, G;
     long long ldy;
@@ -352,23 +352,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
 
             if (++g == G) {  // tile done: activation rows row0 .. row0 + EPC - 1 against weight row n
-                if (n < a.N) {
-                    if (GRP) {  // un-permute: row r is the pair perm[r] = t * topk + j
+                // Lane l fetches the output row and the token factor of activation rows
+                // l and 32 + l; the stores take them by shuffle, so no load waits behind a store.
+                int pr0 = 0, pr1 = 0;
+                float f0 = 0.0f, f1 = 0.0f;
+                if (GRP) {  // un-permute: row r is the pair perm[r] = t * topk + j
+                    if (lane < rows) pr0 = __ldg(a.perm + row0 + lane);
+                    if (32 + lane < min(rows, EPC)) pr1 = __ldg(a.perm + row0 + 32 + lane);
+                    if (lane < rows) f0 = __ldg(a.xf + pr0 / a.topk);
+                    if (32 + lane < min(rows, EPC)) f1 = __ldg(a.xf + pr1 / a.topk);
+                } else {
+                    if (lane < rows) f0 = __ldg(a.xf + row0 + lane);
+                    if (32 + lane < min(rows, EPC)) f1 = __ldg(a.xf + row0 + 32 + lane);
+                }
 #pragma unroll
-                        for (int i = 0; i < EPC; ++i)
-                            if (i < rows) {
-                                const int pr = __ldg(a.perm + row0 + i);
-                                a.y[(long long)pr * a.N + n] = yacc[i] * __ldg(a.xf + pr / a.topk);
-                            }
-                    } else {
-                        float* yp = a.y + (long long)row0 * a.ldy + n;
-                        const float* xp = a.xf + row0;
-#pragma unroll
-                        for (int i = 0; i < EPC; ++i) {
-                            if (i < rows) *yp = yacc[i] * __ldg(xp + i);
-                            yp += a.ldy;
-                        }
-                    }
+                for (int i = 0; i < EPC; ++i) {
+                    const float f = __shfl_sync(kFull, i < 32 ? f0 : f1, i & 31);
+                    const long long orow = GRP ? (long long)__shfl_sync(kFull, i < 32 ? pr0 : pr1, i & 31)
+                                               : (long long)(row0 + i);
+                    if (i < rows && n < a.N) a.y[orow * a.ldy + n] = yacc[i] * f;
                 }
 #pragma unroll
                 for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
