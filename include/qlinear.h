@@ -129,7 +129,11 @@ int qlinear_workspace_size(int fmt, int flags, int M, int N, int K, size_t* byte
  *   W_packed, scales, zeros: the packed weight (zeros only for int5).
  *   ws, ws_bytes: caller's device workspace, at least qlinear_workspace_size.
  * y is overwritten.  The floating-point sums may be accumulated in any order;
- * they are not bit-reproducible across calls. */
+ * they are not bit-reproducible across calls.
+ * Formats whose activations stay 16-bit (all but QL_I8A8_G128_BF16) stage one
+ * token row, in fp32 and f16, in shared memory: they take K <= QL_A16_MAX_K
+ * and return QL_EUNSUPPORTED above it (moe_gate_up likewise). */
+enum { QL_A16_MAX_K = 32768 };
 int qlinear_forward(const void* x, const void* W_packed, const void* scales, const uint8_t* zeros, int fmt,
                     int flags, int M, int N, int K, float* y, void* ws, size_t ws_bytes, void* stream);
 

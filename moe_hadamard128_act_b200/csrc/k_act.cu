@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // grouped expert GEMM.
 __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K, int rotate, int order, __half* xs,
                                                   float* xf, float* yz, long long nz, const int32_t* inv, int topk) {
-    extern __shared__ float row[];
+    extern __shared__ float row[];  // [K] fp32, then (natural order) [K] f16
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
     __shared__ float red[8];
@@ -121,23 +121,26 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K,
     }
     __syncthreads();
     const float f = red[0];
-    if (order == XORD_NATURAL) {  // 8 values per 16-byte store
-        const int nrep = inv ? topk : 1;
-        for (int j = 0; j < nrep; ++j) {
-            const long long orow = inv ? (long long)inv[(long long)t * topk + j] : (long long)t;
-            if (orow < 0) continue;
-            uint4* out = reinterpret_cast<uint4*>(xs + orow * K);
-            for (int c = threadIdx.x; c < K / 8; c += 256) {
-                const float* r = row + 8 * c;
-                uint32_t h[4];
+    if (order == XORD_NATURAL) {  // converted once into shared memory, then 16-byte copies per output row
+        uint4* const hrow = reinterpret_cast<uint4*>(row + K);  // [K / 8] x 8 f16
+        const int K8 = K / 8;
+        for (int c = threadIdx.x; c < K8; c += 256) {
+            const float* r = row + 8 * c;
+            uint32_t h[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __half2 p = __halves2half2(__float2half_rn(__fmul_rn(r[2 * i], f)),
-                                                     __float2half_rn(__fmul_rn(r[2 * i + 1], f)));
-                    h[i] = *reinterpret_cast<const uint32_t*>(&p);
-                }
-                out[c] = make_uint4(h[0], h[1], h[2], h[3]);
+            for (int i = 0; i < 4; ++i) {
+                const __half2 p = __halves2half2(__float2half_rn(__fmul_rn(r[2 * i], f)),
+                                                 __float2half_rn(__fmul_rn(r[2 * i + 1], f)));
+                h[i] = *reinterpret_cast<const uint32_t*>(&p);
             }
+            hrow[c] = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+        __syncthreads();
+        const int nrep = inv ? topk : 1;
+        for (int idx = threadIdx.x; idx < nrep * K8; idx += 256) {
+            const int j = idx / K8, c = idx - j * K8;
+            const long long orow = inv ? (long long)__ldg(inv + (long long)t * topk + j) : (long long)t;
+            if (orow >= 0) reinterpret_cast<uint4*>(xs + orow * K)[c] = hrow[c];
         }
         return;
     }
@@ -202,7 +205,7 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
 
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s) {
-    const size_t smem = (size_t)K * sizeof(float);
+    const size_t smem = (size_t)K * (sizeof(float) + sizeof(__half));  // the fp32 row and its f16 copy
     cudaError_t e = prefer_max_shared(k_prep_a16);
     if (e != cudaSuccess) return e;
     if (smem > 48 * 1024) {
@@ -216,7 +219,7 @@ cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, 
 
 cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, const int32_t* inv, int topk, __half* xs,
                                     float* xf, cudaStream_t s) {
-    const size_t smem = (size_t)K * sizeof(float);
+    const size_t smem = (size_t)K * (sizeof(float) + sizeof(__half));  // the fp32 row and its f16 copy
     cudaError_t e = prefer_max_shared(k_prep_a16);
     if (e != cudaSuccess) return e;
     if (smem > 48 * 1024) {

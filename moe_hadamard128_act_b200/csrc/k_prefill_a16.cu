@@ -5,8 +5,8 @@
 // ("gemma4-26b-a4b-dflash-fp8" README, table "Weights").
 //
 // The tensor cores run kind::f16 (f16 x f16, fp32 accumulation) with the
-// roles turned around: the MMA's M = 128 rows are weight rows, its N = 192
-// columns are tokens.  Both operands are exact:
+// roles turned around: the MMA's M = 128 rows are weight rows, its N = TN
+// columns are tokens (192 by default).  Both operands are exact:
 //  * the codes are converted to f16 exactly (every int8 and every e4m3 value
 //    is an f16) by a converter warpgroup, which writes them straight into
 //    tensor memory as the MMA's A operand -- no shared-memory round trip for
@@ -14,20 +14,33 @@
 //  * the activations are the f16 copy of x scaled per token by a power of two
 //    (prepared by the activation prologue), loaded by TMA into shared memory
 //    as the B operand.
-// One step is one 128-K group: eight MMAs with K = 16 into one of two fp32
-// accumulators [128 weight rows x 192 tokens].  The epilogue thread that owns
+// One step is one 128-K group: eight MMAs with K = 16 into one of the fp32
+// accumulators [128 weight rows x TN tokens] (two at TN = 192, three at
+// TN = 128, as tensor memory allows next to two A tiles).  The epilogue thread that owns
 // a weight row (its tensor-memory lane) folds the group's weight scale, a
 // scalar for that thread, into fp32 running sums: one FMA per element per
 // group.  At the end of a tile each sum is multiplied by its token's inverse
 // factor and written to y (32 lanes of a warp write 32 consecutive y values).
 //
 // Warp roles: warpgroup 0 (24 registers per thread after setmaxnreg): lane 0
-// of warp 0 issues the TMA loads (code tile [128 rows][128 B] into a 4-slot
-// ring, activation tile [192 rows][2 x 128 B] into a 3-slot ring), lane 0 of
-// warp 1 issues the MMAs.  Warpgroup 1 (40 registers) converts: thread i of
-// warp 4 + q converts weight row 32 q + i.  Warpgroups 2..5 (104 registers)
-// are the epilogue: warp w owns rows 32 (w % 4) .. + 31 and tokens
-// 48 ((w - 8) / 4) .. + 47.
+// of warp 0 issues the TMA loads (code tile [128 rows][128 B] into a 4- or
+// 6-slot ring, activation tile [TN rows][2 x 128 B] into a 3-slot ring), lane 0 of
+// warps 1 and 2 issue the MMAs of the even and the odd steps.  The next one
+// or two warpgroups (40 registers) convert: thread i of warp 4 + 4 h + q
+// converts part h of weight row 32 q + i (the whole row with one warpgroup,
+// halves with two).  The last four warpgroups (96 or 104 registers) are the
+// epilogue: warp w owns rows 32 (w % 4) .. + 31 and TN / 4 of the tokens.
+//
+// The tensor pipe must never wait for its issuer: a tcgen05.mma is accepted
+// only about one MMA ahead of the one executing, so every cycle an issuing
+// thread spends on barriers and commits would leave the pipe idle.  Hence two
+// issuing threads taking alternate steps (the steps are independent: each has
+// its own accumulator, A tile and activation slot, so their MMAs may
+// interleave), whose waits hide behind each other's MMAs, and a single commit
+// per step: the consumers of a step (the epilogue reading its accumulator, the
+// converters and the producer reusing its A tile and activation slot) all
+// wait on that one commit, on a ring of 6 mbarriers (a multiple of the
+// activation, A-tile and accumulator ring depths).
 //
 // All waits are bounded (200 ms); on a timeout the CTA sets QL_DEVERR_TIMEOUT
 // and winds down without leaving tensor memory allocated, MMAs running or
@@ -44,34 +57,44 @@ constexpr int GK = 128;                   // K per step (one group)
 constexpr int CODE_BYTES = TM * GK;       // one code tile (1-byte codes), 16 KB
 constexpr int XATOM = TN * 128;           // one activation box: [TN rows][64 f16 = 128 B]
 constexpr int X_BYTES = 2 * XATOM;        // the step's activations, 48 KB
-constexpr int CS = 4, XS = 3;             // ring slots
-constexpr int NACC = (512 - 128) / TN;    // fp32 accumulators [128 x TN] in tensor memory (A tiles take 128 columns)
+constexpr int CS = TN > 128 ? 4 : 6, XS = 3;  // ring slots (codes, activations)
+constexpr int AS = 2;                     // converted A tiles in tensor memory
+constexpr int NACC = (512 - AS * 64) / TN;  // fp32 accumulators [128 x TN] in tensor memory
+constexpr int SR = 6;                     // step-commit ring: a multiple of XS, AS and NACC
 constexpr int ACOLS = GK / 2;             // tensor-memory columns of one converted A tile (f16 pairs)
 constexpr int A_COL0 = NACC * TN;         // A tiles follow the accumulators
 constexpr uint32_t kTmemCols = 512;
+constexpr int kConvWarps = TN > 128 ? 4 : 8;  // one or two per sub-partition (a row or half a row each)
+constexpr int kRowParts = kConvWarps / 4;     // converter warps per weight row
+constexpr int CPW = 8 / kRowParts;            // 16-byte code chunks per converter thread
 constexpr int kEpiWarps = 16;
-constexpr int kThreads = 32 * (8 + kEpiWarps);
+constexpr int kEpiWarp0 = 4 + kConvWarps;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int EPC = TN / 4;               // tokens per epilogue thread
 constexpr int CW = 16;                    // columns per tensor-memory read
-static_assert(A_COL0 + 2 * ACOLS <= (int)kTmemCols, "tensor memory budget");
+static_assert(A_COL0 + AS * ACOLS <= (int)kTmemCols, "tensor memory budget");
+static_assert(SR % XS == 0 && SR % AS == 0 && SR % NACC == 0, "one commit ring serves every per-step resource");
 static_assert(EPC % CW == 0 && EPC <= 64 && TN % 16 == 0 && TN <= 256, "token tile");
 static_assert(XATOM % 1024 == 0, "activation boxes stay 1024-byte aligned for the 128-byte swizzle");
 
 // Shared memory (from a 1024-aligned base): [code ring][activation ring][mbarriers][tmem address]
 constexpr int X_OFF = CS * CODE_BYTES;
 constexpr int BAR_OFF = X_OFF + XS * X_BYTES;
-constexpr int B_CFULL = 0, B_CEMPTY = CS, B_XFULL = 2 * CS, B_XEMPTY = 2 * CS + XS, B_AFULL = 2 * CS + 2 * XS,
-              B_AEMPTY = B_AFULL + 2, B_DFULL = B_AEMPTY + 2, B_DEMPTY = B_DFULL + NACC, B_DRAIN = B_DEMPTY + NACC,
-              NBARS = B_DRAIN + 1;
+constexpr int B_CFULL = 0, B_CEMPTY = CS, B_XFULL = 2 * CS, B_AFULL = 2 * CS + XS, B_STEP = B_AFULL + AS,
+              B_DEMPTY = B_STEP + SR, B_DRAIN = B_DEMPTY + NACC, NBARS = B_DRAIN + 1;
 constexpr int MISC_OFF = (BAR_OFF + 8 * NBARS + 15) / 16 * 16;
 constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
-// Registers: 768 threads launch with 80 each (61440).  Warpgroup 0 drops to
-// 24, the converters to 40, the epilogue rises to 104: 128 * (24 + 40) +
-// 512 * 104 = 61440.  Per SM sub-partition: 32 * (24 + 40 + 4 * 104) = 15360.
-constexpr int kRegsDriver = 24, kRegsConv = 40, kRegsEpi = 104;
-static_assert(128 * (kRegsDriver + kRegsConv) + 32 * kEpiWarps * kRegsEpi <= kThreads * 80, "register split");
+// Registers: 896 threads (128-token tiles) launch with 72 each, 768 threads
+// (wider tiles) with 80.  Warpgroup 0 drops to 24, the converters to 40, the
+// epilogue (32 or 48 running sums per thread) rises to 96 or 104:
+// 128 * 24 + 256 * 40 + 512 * 96 = 62464 <= 896 * 72, and
+// 128 * 24 + 128 * 40 + 512 * 104 = 61440 <= 768 * 80.
+constexpr int kRegsLaunch = (65536 / kThreads) & ~7, kRegsDriver = 24, kRegsConv = 40, kRegsEpi = TN > 128 ? 104 : 96;
+static_assert(128 * kRegsDriver + 32 * kConvWarps * kRegsConv + 32 * kEpiWarps * kRegsEpi <= kThreads * kRegsLaunch,
+              "register split");
+static_assert(32 * (kRegsDriver + kRowParts * kRegsConv + 4 * kRegsEpi) <= 16384, "registers per sub-partition");
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     // K-major, 128-byte swizzle: 8-row atoms 1024 bytes apart (SBO), version 1.
@@ -178,22 +201,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < CS; ++s) {
-            mbar_init(bar(B_CFULL + s), 1);  // expect_tx
-            mbar_init(bar(B_CEMPTY + s), 4);  // one arrive per converter warp
+            mbar_init(bar(B_CFULL + s), 1);           // expect_tx
+            mbar_init(bar(B_CEMPTY + s), kConvWarps);  // one arrive per converter warp
         }
-        for (int s = 0; s < XS; ++s) {
-            mbar_init(bar(B_XFULL + s), 1);   // expect_tx
-            mbar_init(bar(B_XEMPTY + s), 1);  // MMA commit
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(B_AFULL + s), 4);   // one arrive per converter warp
-            mbar_init(bar(B_AEMPTY + s), 1);  // MMA commit
-        }
-        for (int s = 0; s < NACC; ++s) {
-            mbar_init(bar(B_DFULL + s), 1);          // MMA commit
-            mbar_init(bar(B_DEMPTY + s), kEpiWarps);  // one arrive per epilogue warp
-        }
-        mbar_init(bar(B_DRAIN), 1);
+        for (int s = 0; s < XS; ++s) mbar_init(bar(B_XFULL + s), 1);           // expect_tx
+        for (int s = 0; s < AS; ++s) mbar_init(bar(B_AFULL + s), kConvWarps);  // one arrive per converter warp
+        for (int s = 0; s < SR; ++s) mbar_init(bar(B_STEP + s), 1);            // the step's MMA commit
+        for (int s = 0; s < NACC; ++s) mbar_init(bar(B_DEMPTY + s), kEpiWarps);  // one arrive per epilogue warp
+        mbar_init(bar(B_DRAIN), 2);  // one commit per issuing thread
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     if (warp == 1) {
@@ -225,8 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 mbar_expect_tx(cb, CODE_BYTES);
                 tma_load_2d(base + c * CODE_BYTES, &a.tmW, g * GK, n0, cb);
                 ++kc;
-                if (!mbar_wait(bar(B_XEMPTY + x), ((k / XS) & 1) ^ 1)) {
-                    dead = true;
+                if (k >= XS && !mbar_wait(bar(B_STEP + (k - XS) % SR), ((k - XS) / SR) & 1)) {
+                    dead = true;  // the slot's previous activations are still in use
                     break;
                 }
                 const uint32_t xb = bar(B_XFULL + x), xd = base + X_OFF + x * X_BYTES;
@@ -249,11 +264,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 if (!mbar_wait(bar(B_CFULL + j % CS), (j / CS) & 1)) break;
             for (int j = kx > XS ? kx - XS : 0; j < kx; ++j)
                 if (!mbar_wait(bar(B_XFULL + j % XS), (j / XS) & 1)) break;
-        } else if (warp == 1 && lane == 0) {  // ---- MMA issuer ----
+        } else if ((warp == 1 || warp == 2) && lane == 0) {  // ---- MMA issuers: even / odd steps ----
             const uint64_t xd0 = smem_desc_sw128(base + X_OFF);
-            for (int k = 0; k < total; ++k) {
-                const int x = k % XS, ab = k & 1, db = k % NACC;
-                if (!mbar_wait(bar(B_XFULL + x), (k / XS) & 1) || !mbar_wait(bar(B_AFULL + ab), (k / 2) & 1) ||
+            for (int k = warp - 1; k < total; k += 2) {
+                const int x = k % XS, ab = k % AS, db = k % NACC;
+                if (!mbar_wait(bar(B_XFULL + x), (k / XS) & 1) || !mbar_wait(bar(B_AFULL + ab), (k / AS) & 1) ||
                     !mbar_wait(bar(B_DEMPTY + db), ((k / NACC) & 1) ^ 1)) {
                     dead = true;
                     break;
@@ -265,33 +280,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 for (int j = 0; j < GK / 16; ++j)
                     mma_f16_ts(d, at + 8 * j, xd0 + xo + (uint64_t)((j / 4) * (XATOM >> 4) + (j % 4) * 2),
                                j ? 1u : 0u);
-                mma_commit(bar(B_XEMPTY + x));   // activation slot free once these MMAs are done
-                mma_commit(bar(B_AEMPTY + ab));  // converted weights free
-                mma_commit(bar(B_DFULL + db));   // accumulator ready for the epilogue
+                // One commit per step: its accumulator is ready for the epilogue, and its
+                // A tile and activation slot may be refilled.  A waiter for step j checks
+                // the parity of its completion on slot j % SR, and the slot cannot
+                // complete again before that check: step j + SR needs the waiter to have
+                // moved on first (the producer's activations for it, the converters' A
+                // tile for it, or the epilogue freeing its accumulator after step
+                // j + SR - NACC).
+                mma_commit(bar(B_STEP + k % SR));
             }
-            // Every MMA issued must finish before tensor memory is freed.
+            // Every MMA issued (by both threads) must finish before tensor memory is freed.
             mma_commit(bar(B_DRAIN));
             mbar_wait(bar(B_DRAIN), 0);
         }
-    } else if (warp < 8) {  // ---- converters ----
+    } else if (warp < kEpiWarp0) {  // ---- converters ----
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsConv));
-        const int q = warp & 3, r = 32 * q + lane;  // weight row within the tile
+        const int q = warp & 3, h = (warp - 4) >> 2, r = 32 * q + lane;  // weight row, part of its 128 codes
         const uint32_t tl = (uint32_t)(32 * q) << 16;
         for (int k = 0; k < total; ++k) {
-            const int c = k % CS, ab = k & 1;
-            if (!mbar_wait(bar(B_CFULL + c), (k / CS) & 1) || !mbar_wait(bar(B_AEMPTY + ab), ((k / 2) & 1) ^ 1)) {
-                dead = true;
+            const int c = k % CS, ab = k % AS;
+            if (!mbar_wait(bar(B_CFULL + c), (k / CS) & 1) ||
+                (k >= AS && !mbar_wait(bar(B_STEP + (k - AS) % SR), ((k - AS) / SR) & 1))) {
+                dead = true;  // no codes, or the A tile's previous MMAs are still running
                 break;
             }
             tc_fence_after();
             // Row r of the code tile: 16-byte chunk j sits at chunk j ^ (r & 7) (128-byte swizzle).
             const uint32_t rowp = base + c * CODE_BYTES + r * 128;
-            const uint32_t at = tmem + tl + A_COL0 + ab * ACOLS;
+            const uint32_t at = tmem + tl + A_COL0 + ab * ACOLS + 8 * CPW * h;
 #pragma unroll
-            for (int j = 0; j < GK / 32; ++j) {
+            for (int j = 0; j < CPW / 2; ++j) {
+                const int ch = CPW * h + 2 * j;  // 16-byte chunks ch, ch + 1: codes 16 ch .. 16 ch + 31
                 uint32_t w[16];
-                convert16<FMT>(lds128(rowp + (((2 * j) ^ (r & 7)) << 4)), w);
-                convert16<FMT>(lds128(rowp + (((2 * j + 1) ^ (r & 7)) << 4)), w + 8);
+                convert16<FMT>(lds128(rowp + ((ch ^ (r & 7)) << 4)), w);
+                convert16<FMT>(lds128(rowp + (((ch + 1) ^ (r & 7)) << 4)), w + 8);
                 QL_TMEM_ST16(at + 16 * j, w);
             }
             asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
@@ -304,36 +326,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
         }
     } else {  // ---- epilogue ----
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsEpi));
-        const int q = warp & 3, cg = (warp - 8) >> 2;
+        const int q = warp & 3, cg = (warp - kEpiWarp0) >> 2;
         const uint32_t tl = (uint32_t)(32 * q) << 16;
         float yacc[EPC];
 #pragma unroll
         for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
         int t = blockIdx.x, g = 0;
-        // This thread's weight row of the current tile and its scale row: one scale per
-        // group, read one step ahead (fp8: the row's 128-row block; rows past N scale 0).
         const int NBk = (a.N + TM - 1) / TM;
-        int n = 0, row0 = 0, rows = 0;
-        auto start_tile = [&](int tt) -> const uint16_t* {
-            const MoeTile ti = tile_at<GRP>(a, tt, TB);
+        // Everything a step or a tile end needs from global memory is requested well
+        // before it is used, so no load latency sits between the tensor-memory reads:
+        //  * the group scale (raw 16 bits) one step ahead, converted only at its use;
+        //  * the next tile's descriptor one tile ahead;
+        //  * the output rows and token factors of this thread's activation rows
+        //    during the tile's first steps (lane l: rows l and 32 + l).
+        int n = 0, row0 = 0, rows = 0, pr0 = 0, pr1 = 0;
+        float f0 = 0.0f, f1 = 0.0f;
+        const uint16_t* sp = nullptr;
+        MoeTile nt = my_tiles > 0 ? tile_at<GRP>(a, t, TB) : MoeTile{0, 0, 0, 0};
+        auto start_tile = [&](int tt) {
+            const MoeTile ti = nt;
+            if (tt + (int)gridDim.x < tiles) nt = tile_at<GRP>(a, tt + (int)gridDim.x, TB);
             n = ti.wb * TM + 32 * q + lane;
             row0 = ti.row0 + cg * EPC;
             rows = ti.rows - cg * EPC;
-            if (FMT == QL_FP8_B128_BF16) return a.sw + ((long long)ti.expert * NBk + n / 128) * G;
-            return n < a.N ? a.sw + ((long long)ti.expert * a.N + n) * G : nullptr;
+            if (FMT == QL_FP8_B128_BF16) sp = a.sw + ((long long)ti.expert * NBk + n / 128) * G;
+            else sp = n < a.N ? a.sw + ((long long)ti.expert * a.N + n) * G : nullptr;  // rows past N: scale 0
+            pr0 = pr1 = 0;
+            if (GRP) {  // row r of the permuted activations is the pair perm[r] = t * topk + j
+                if (lane < rows) pr0 = __ldg(a.perm + row0 + lane);
+                if (32 + lane < min(rows, EPC)) pr1 = __ldg(a.perm + row0 + 32 + lane);
+            } else {
+                pr0 = row0 + lane;
+                pr1 = row0 + 32 + lane;
+            }
         };
-        auto scale_at = [&](const uint16_t* sp, int gg) -> float {
-            if (!sp) return 0.0f;
-            const uint16_t b = __ldg(sp + gg);
-            return FMT == QL_I8_G128_F16 ? f16_bits_to_float(b) : bf16_bits_to_float(b);
-        };
-        const uint16_t* sp = my_tiles > 0 ? start_tile(t) : nullptr;
-        float s_next = my_tiles > 0 ? scale_at(sp, 0) : 0.0f;
+        auto scale_raw = [&](int gg) -> uint32_t { return sp ? (uint32_t)__ldg(sp + gg) : 0u; };
+        uint32_t sb_next = 0;
+        if (my_tiles > 0) {
+            start_tile(t);
+            sb_next = scale_raw(0);
+        }
         for (int k = 0; k < total; ++k) {
             const int db = k % NACC;
-            const float s = s_next;
-            if (g + 1 < G) s_next = scale_at(sp, g + 1);
-            if (!mbar_wait(bar(B_DFULL + db), (k / NACC) & 1)) {
+            const float s = FMT == QL_I8_G128_F16 ? f16_bits_to_float((uint16_t)sb_next)
+                                                  : bf16_bits_to_float((uint16_t)sb_next);
+            if (g + 1 < G) sb_next = scale_raw(g + 1);
+            if (!mbar_wait(bar(B_STEP + k % SR), (k / SR) & 1)) {
                 dead = true;
                 break;
             }
@@ -351,25 +389,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
 
+            if (g == min(1, G - 1)) {  // the token factors, once the output rows have arrived
+                f0 = lane < rows ? __ldg(a.xf + (GRP ? pr0 / a.topk : pr0)) : 0.0f;
+                f1 = 32 + lane < min(rows, EPC) ? __ldg(a.xf + (GRP ? pr1 / a.topk : pr1)) : 0.0f;
+            }
             if (++g == G) {  // tile done: activation rows row0 .. row0 + EPC - 1 against weight row n
-                // Lane l fetches the output row and the token factor of activation rows
-                // l and 32 + l; the stores take them by shuffle, so no load waits behind a store.
-                int pr0 = 0, pr1 = 0;
-                float f0 = 0.0f, f1 = 0.0f;
-                if (GRP) {  // un-permute: row r is the pair perm[r] = t * topk + j
-                    if (lane < rows) pr0 = __ldg(a.perm + row0 + lane);
-                    if (32 + lane < min(rows, EPC)) pr1 = __ldg(a.perm + row0 + 32 + lane);
-                    if (lane < rows) f0 = __ldg(a.xf + pr0 / a.topk);
-                    if (32 + lane < min(rows, EPC)) f1 = __ldg(a.xf + pr1 / a.topk);
-                } else {
-                    if (lane < rows) f0 = __ldg(a.xf + row0 + lane);
-                    if (32 + lane < min(rows, EPC)) f1 = __ldg(a.xf + row0 + 32 + lane);
-                }
 #pragma unroll
                 for (int i = 0; i < EPC; ++i) {
                     const float f = __shfl_sync(kFull, i < 32 ? f0 : f1, i & 31);
-                    const long long orow = GRP ? (long long)__shfl_sync(kFull, i < 32 ? pr0 : pr1, i & 31)
-                                               : (long long)(row0 + i);
+                    const long long orow = __shfl_sync(kFull, i < 32 ? pr0 : pr1, i & 31);
                     if (i < rows && n < a.N) a.y[orow * a.ldy + n] = yacc[i] * f;
                 }
 #pragma unroll
@@ -377,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 g = 0;
                 t += gridDim.x;
                 if (k + 1 < total) {
-                    sp = start_tile(t);
-                    s_next = scale_at(sp, 0);
+                    start_tile(t);
+                    sb_next = scale_raw(0);
                 }
             }
         }

@@ -180,6 +180,7 @@ int check_experts(const ql_experts* ex) {
     if (ex->flags & ~QL_HADAMARD) return QL_EINVAL;
     if (!fmt_valid(ex->fmt)) return QL_EINVAL;
     if (ex->fmt != QL_I8_G128_BF16 && ex->fmt != QL_I8_G128_F16 && ex->fmt != QL_FP8_B128_BF16) return QL_EUNSUPPORTED;
+    if (ex->K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
     if (!ex->codes || !ex->scales) return QL_EINVAL;
     if (!aligned16(ex->codes) || !aligned16(ex->scales)) return QL_EALIGN;
     return QL_OK;
@@ -266,6 +267,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
     if (!x || !W_packed || !scales || !y) return QL_EINVAL;
     if (fmt == QL_I5Z_G128_F16 && !zeros) return QL_EINVAL;
+    if (fmt != QL_I8A8_G128_BF16 && K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
     if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y) ||
         (zeros && !aligned16(zeros)))
         return QL_EALIGN;

@@ -80,6 +80,7 @@ def test_forward_validation_statuses(L):
     assert call(flags=4) == 1
     assert call(x=None) == 1
     assert call(fmt=5) == 1  # int5 needs zeros
+    assert call(K=32768 + 128) == 2  # a 16-bit activation row no longer fits in shared memory
     assert call(x=P(A + 8)) == 3
     assert call(y=P(A + 4)) == 3
     assert call(ws=None) == 4
@@ -115,5 +116,7 @@ def test_moe_validation_statuses(L):
     bad = Q.ql_experts(128, 1408, 2816, 1, 0, A + 8, A)
     assert g(P(A), P(A), None, ctypes.byref(bad), 4, 8, P(A), P(A), 1 << 30, None) == 3
     assert g(P(A), P(A), None, None, 4, 8, P(A), P(A), 1 << 30, None) == 1
+    big = Q.ql_experts(8, 256, 32768 + 128, 1, 0, A, A)
+    assert g(P(A), P(A), None, ctypes.byref(big), 4, 8, P(A), P(A), 1 << 40, None) == 2
     assert L.moe_permute(P(A), 4, 8, 0, P(A), P(A), P(A), None) == 1
     assert Q.moe_workspace_size(128, 1408, 2816, 1, 1, 2048, 8) > 2048 * 2816 * 2
