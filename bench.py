@@ -51,7 +51,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8"], default=None,
+    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "moe_decode", "moe_prefill"],
+                   default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
 
@@ -366,13 +367,39 @@ def ncu_case(name):
     GEMM is launch 1..4 of its name.
     prefill_w8a8 / prefill_fp8: the prefill workload (M = 2048, N = 21504,
     K = 5376; about 0.6 GB on the device), four forwards; the tcgen05 GEMM
-    (k_prefill_w8a8 / k_prefill_a16) is launch 1..4 of its name."""
+    (k_prefill_w8a8 / k_prefill_a16) is launch 1..4 of its name.
+    moe_decode / moe_prefill: the MoE gate_up experts (128 x [1408, 2816] int8
+    g128 bf16, Hadamard domain; about 0.5 GB), top-8 routing of T = 16 / 2048
+    tokens, four calls of moe_gate_up (permute, activation prologue, expert
+    GEMM per call)."""
     import torch
 
     from moe_hadamard128_act_b200 import qlinear as Q
     from moe_hadamard128_act_b200 import synth
 
     dev = torch.device("cuda", 0)
+    if name.startswith("moe"):
+        E, topk, Ke, Ne = 128, 8, 2816, 1408
+        T = 16 if name == "moe_decode" else 2048
+        Ws = synth.moe_gate_up(1, experts=range(E))["W"]
+        codes = torch.empty((E, Ne, Ke), dtype=torch.int8, device=dev)
+        scales = torch.empty((E, Ne, Ke // 128), dtype=torch.int16, device=dev)
+        for e in range(E):
+            c, s, _ = Q.qlinear_pack(Q.I8_G128_BF16, Ne, Ke, W=torch.from_numpy(Ws[e]).to(dev), flags=Q.HADAMARD)
+            codes[e] = c.view(torch.int8).reshape(Ne, Ke)
+            scales[e] = s.view(torch.int16).reshape(Ne, Ke // 128)
+        del Ws
+        ids, _ = synth.routing(200, T, E, topk)
+        x = torch.from_numpy(synth.activations(0, f"x_T{T}", T, Ke).view(np.int16)).view(torch.bfloat16).to(dev)
+        idt = torch.from_numpy(ids).to(dev)
+        y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+        for i in range(4):
+            Q.moe_gate_up(x, idt, codes, scales, E, Ne, y=y)
+        torch.cuda.synchronize()
+        st, bits = Q.ql_get_device_error()
+        assert st == 0, bits
+        print(f"ncu case {name} done")
+        return
     if name.startswith("prefill"):
         fmt = Q.I8A8_G128_BF16 if name == "prefill_w8a8" else Q.FP8_B128_BF16
         d = synth.prefill(M=2048)
