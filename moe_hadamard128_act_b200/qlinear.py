@@ -30,6 +30,8 @@ FORMATS = (I8_G128_BF16, I8_G128_F16, I8A8_G128_BF16, I4_G64_BF16, I5Z_G128_F16,
 DEVERR_EXPERT_ID = 1
 DEVERR_CODE_RANGE = 2
 
+A16_MAX_K = 32768  # QL_A16_MAX_K: largest K for the formats whose activations stay 16-bit
+
 STATUS = {0: "QL_OK", 1: "QL_EINVAL", 2: "QL_EUNSUPPORTED", 3: "QL_EALIGN", 4: "QL_EWORKSPACE", 5: "QL_ECUDA",
           6: "QL_EDEVICE"}
 

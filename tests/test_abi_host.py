@@ -34,6 +34,14 @@ def test_exports_every_declared_function(L):
         assert hasattr(L, n), n
 
 
+def test_binding_constants_match_header():
+    from moe_hadamard128_act_b200 import qlinear as Q
+    text = (ROOT / "include" / "qlinear.h").read_text()
+    assert int(re.search(r"QL_A16_MAX_K\s*=\s*(\d+)", text).group(1)) == Q.A16_MAX_K
+    for name in ("I8_G128_BF16", "I8_G128_F16", "I8A8_G128_BF16", "I4_G64_BF16", "I5Z_G128_F16", "FP8_B128_BF16"):
+        assert int(re.search(rf"QL_{name}\s*=\s*(\d+)", text).group(1)) == getattr(Q, name), name
+
+
 def test_status_strings(L):
     for st in range(7):
         assert L.ql_status_string(st)
