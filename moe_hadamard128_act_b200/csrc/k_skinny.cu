@@ -716,6 +716,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
 // 16 * slab, byte 128 * group).  The activations of a chunk's (at most 16)
 // tokens are read from the prepared [T, K] buffer, which stays in L2, and the
 // results are added into y[(t, j), :] (zeroed by the prologue).
+//
+// Small batches (T * topk <= kMoeFusedMaxPairs) skip the permute kernel: every
+// CTA ranks the routing ids itself in shared memory -- the position of pair i
+// is the number of valid ids below its expert plus the number of equal ids
+// before it, which is the stable (expert, t, j) order -- and cuts each expert's
+// segment into chunks of 16.  It then starts its weight stream at once and
+// waits for the activation prologue (programmatic dependent launch) only before
+// it reads the activations or adds into y.
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__ MoeArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -725,15 +733,71 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     const int G = a.K / 128;
     const int slabs = (a.N + 15) / 16;
     const long long per_chunk = (long long)slabs * G;
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the chunk table comes from the permute kernel
-    const long long nch = min((long long)*a.n_chunks, a.max_chunks);
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const bool fused = a.ids != nullptr;
+    // Routing state of the fused mode, after the rings and barriers.
+    int* const s_ids = reinterpret_cast<int*>(smem_raw + (base - raw) + ring_bytes<FMT>() + kWarps * kStages * 8);
+    int* const s_perm = s_ids + kMoeFusedMaxPairs;   // permuted position -> pair index t * topk + j
+    int* const s_bef = s_perm + kMoeFusedMaxPairs;   // per position: pairs of the same expert before it
+    int* const s_cnt = s_bef + kMoeFusedMaxPairs;    // per position: pairs of its expert
+    int* const s_exp = s_cnt + kMoeFusedMaxPairs;    // per position: its expert
+    MoeChunk* const s_ch = reinterpret_cast<MoeChunk*>(s_exp + kMoeFusedMaxPairs);
+    int* const s_nch = reinterpret_cast<int*>(s_ch + kMoeFusedMaxPairs);
+    long long nch;
+    if (fused) {
+        // The ids are complete: the activation prologue this grid depends on is an
+        // ordinary launch, so it started only after all earlier work on the stream
+        // (the router included), and this grid starts no earlier than it.
+        const int P = a.T * a.topk;
+        for (int i = threadIdx.x; i < P; i += kThreads) s_ids[i] = a.ids[i];
+        __syncthreads();
+        for (int i = threadIdx.x; i < P; i += kThreads) {
+            const int e = s_ids[i];
+            int less = 0, before = 0, same = 0;
+            for (int j = 0; j < P; ++j) {
+                const int f = s_ids[j];
+                less += f >= 0 && f < e;
+                same += f == e;
+                before += f == e && j < i;
+            }
+            if (e < 0 || e >= a.E) {  // routed to no expert: flagged, its output row stays zero
+                if (blockIdx.x == 0) atomicOr(a.err, (unsigned)QL_DEVERR_EXPERT_ID);
+                continue;
+            }
+            const int pos = less + before;
+            s_perm[pos] = i;
+            s_bef[pos] = before;
+            s_cnt[pos] = same;
+            s_exp[pos] = e;
+        }
+        __syncthreads();
+        int nv = 0;  // valid pairs: positions 0 .. nv - 1
+        for (int j = 0; j < P; ++j) nv += s_ids[j] >= 0 && s_ids[j] < a.E;
+        for (int p = threadIdx.x; p < nv; p += kThreads) {
+            if (s_bef[p] % 16) continue;  // a chunk starts at every 16th row of an expert's segment
+            int idx = 0;
+            for (int q = 0; q < p; ++q) idx += s_bef[q] % 16 == 0;
+            s_ch[idx] = MoeChunk{s_exp[p], p, min(16, s_cnt[p] - s_bef[p])};
+        }
+        if (threadIdx.x == 0) {
+            int n = 0;
+            for (int q = 0; q < nv; ++q) n += s_bef[q] % 16 == 0;
+            *s_nch = n;
+        }
+        __syncthreads();
+        nch = *s_nch;
+    } else {
+        asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the chunk table comes from the permute kernel
+        nch = min((long long)*a.n_chunks, a.max_chunks);
+    }
+    const MoeChunk* const chunks = fused ? s_ch : a.chunks;
+    const int* const perm = fused ? s_perm : a.perm;
     const long long units = nch * per_chunk;
     const long long wid = (long long)blockIdx.x * kWarps + warp, nw = (long long)gridDim.x * kWarps;
     const long long u0 = units * wid / nw, u1 = units * (wid + 1) / nw;
     if (lane == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmap) : "memory");
 
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t ring = base + (uint32_t)(warp * kStages * SB);
     const uint32_t bars = base + (uint32_t)ring_bytes<FMT>() + (uint32_t)(warp * kStages * 8);
     if (u0 >= u1) return;
@@ -768,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     }
     __syncwarp();
     auto issue = [&](int st) {
-        const MoeChunk ch = a.chunks[ip.ch];
+        const MoeChunk ch = chunks[ip.ch];
         if (lane == 0) {
             mbar_expect_tx(bars + 8 * st, SB);
             tma_load_2d(ring + st * SB, &a.tmap, ip.grp * 128, ch.expert * a.N + ip.slab * 16, bars + 8 * st);
@@ -784,13 +848,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     float yacc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = yacc[nt][2] = yacc[nt][3] = 0.0f;
-    MoeChunk chc = a.chunks[cp.ch];  // the chunk being computed
+    // The weight stream is running; the activations and the zeroed y come from the prologue.
+    if (fused) asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    MoeChunk chc = chunks[cp.ch];  // the chunk being computed
     int tok[NT];                     // this lane's tokens in it (-1: none)
     auto load_tokens = [&]() {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int slot = 8 * nt + g;
-            tok[nt] = slot < chc.count ? __ldg(a.perm + chc.start + slot) / a.topk : -1;
+            tok[nt] = slot < chc.count ? perm[chc.start + slot] / a.topk : -1;
         }
     };
     load_tokens();
@@ -804,7 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 const int slot = 8 * nt + 2 * c + (i & 1);
                 const int n = cur_slab * 16 + g + 8 * (i >> 1);
                 if (slot < chc.count && n < a.N) {
-                    const int pair = __ldg(a.perm + chc.start + slot);
+                    const int pair = perm[chc.start + slot];
                     atomicAdd(a.y + (long long)pair * a.N + n, yacc[nt][i] * __ldg(a.xf + pair / a.topk));
                 }
                 yacc[nt][i] = 0.0f;
@@ -821,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
             if (cp.ch != cur_ch || cp.slab != cur_slab) {
                 flush();
                 if (cp.ch != cur_ch) {
-                    chc = a.chunks[cp.ch];
+                    chc = chunks[cp.ch];
                     load_tokens();
                 }
                 cur_ch = cp.ch;
@@ -1004,7 +1070,9 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     if ((e = make_tmap_2d(a.codes, (long long)a.E * a.N, a.K, a.K, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmap)) !=
         cudaSuccess)
         return e;
-    const size_t smem = 1024 + ring_bytes<QL_I8_G128_BF16>() + (size_t)kWarps * kStages * 8;
+    // rings, their mbarriers, and the routing state of the fused small-batch mode
+    const size_t smem = 1024 + ring_bytes<QL_I8_G128_BF16>() + (size_t)kWarps * kStages * 8 +
+                        (5 * sizeof(int) + sizeof(MoeChunk)) * kMoeFusedMaxPairs + 16;
     static bool attr_set[64] = {};  // per device ordinal, for all three instantiations at once
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1022,7 +1090,9 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 0;  // everything depends on the permute
+        // With the permute kernel before it everything depends on its table; in the
+        // fused mode only the activations and y do, so the weight stream may start early.
+        attr[0].val.programmaticStreamSerializationAllowed = a.ids ? 1 : 0;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         cudaError_t r = cudaLaunchKernelEx(&cfg, kern, a);

@@ -488,13 +488,17 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
                         (long long)T * topk * N, s);
     trace_end(t, s);
     if (e != cudaSuccess) return from_cuda(e);
-    t = trace_begin(QL_KIND_MOE_PERMUTE, s);
-    MoePermuteOut po;
-    po.chunks = chunks;
-    po.n_chunks = nch;
-    e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
-    trace_end(t, s);
-    if (e != cudaSuccess) return from_cuda(e);
+    // Small batches: the expert GEMM ranks the ids itself (no permute launch).
+    const bool fused = (long long)T * topk <= kMoeFusedMaxPairs;
+    if (!fused) {
+        t = trace_begin(QL_KIND_MOE_PERMUTE, s);
+        MoePermuteOut po;
+        po.chunks = chunks;
+        po.n_chunks = nch;
+        e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
     MoeArgs a;
     a.codes = static_cast<const uint8_t*>(experts->codes);
     a.scales = experts->scales;
@@ -503,6 +507,7 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     a.perm = perm;
     a.chunks = chunks;
     a.n_chunks = nch;
+    a.ids = fused ? topk_ids : nullptr;
     a.y = y;
     a.fmt = experts->fmt;
     a.T = T;

@@ -168,10 +168,13 @@ struct MoeArgs {
     const int32_t* perm;   // [T*topk]
     const MoeChunk* chunks;
     const int* n_chunks;
+    const int32_t* ids = nullptr;  // [T*topk] routing ids: when set (T*topk <= kMoeFusedMaxPairs), every CTA
+                           // builds the permutation and chunk table itself and perm / chunks are unused
     float* y;              // [T*topk][N]
     int fmt, T, topk, E, N, K;
     long long max_chunks;
 };
+constexpr int kMoeFusedMaxPairs = 128;
 cudaError_t launch_moe_skinny(const MoeArgs& a, cudaStream_t s);
 
 // ---- launch trace (ql_trace_enable / ql_trace_read) --------------------------------------

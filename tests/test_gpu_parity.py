@@ -215,8 +215,10 @@ def moe_weights(E, N, K, fmt, seed=9):
 
 @pytest.mark.parametrize("fmt", [1, 2, 6])
 @pytest.mark.parametrize("T,E,topk,N,K", [(1, 8, 2, 96, 256), (8, 16, 4, 64, 384), (16, 32, 8, 130, 256),
-                                          (40, 8, 3, 48, 128)])
+                                          (20, 32, 8, 130, 256), (40, 8, 3, 48, 128)])
 def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
+    # T * topk <= 128: the expert GEMM ranks the ids itself; (20, 32, 8): 160 pairs, the
+    # permute kernel's chunk table; (40, 8, 3): the grouped tensor-core GEMM.
     codes, scales = moe_weights(E, N, K, fmt)
     ids, w = synth.routing(6, T, E, topk)
     x = x_bits(T, K, seed=13)
@@ -257,6 +259,26 @@ def test_moe_gate_up_grouped_bad_id():
     ref = O.moe_gate_up(x, ids_ok, codes, scales, 1, 1, E, N)
     ref[5, 2] = 0.0
     assert_close(y, ref, "moe grouped, one bad id")
+
+
+@pytest.mark.parametrize("T,E,topk", [(4, 8, 2), (20, 32, 8)])  # skinny modes: in-kernel ranking, permute kernel
+def test_moe_gate_up_skinny_bad_ids(T, E, topk):
+    N, K = 64, 128
+    codes, scales = moe_weights(E, N, K, Q.I8_G128_BF16)
+    ids, _ = synth.routing(8, T, E, topk)
+    ids[1, 0] = E + 5  # skipped: flagged, their output rows zero, every other pair exact
+    ids[2, topk - 1] = -1
+    x = x_bits(T, K, seed=19)
+    Q.ql_get_device_error()
+    y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N).cpu().numpy()
+    st, bits = Q.ql_get_device_error()
+    assert st == 6 and bits & Q.DEVERR_EXPERT_ID
+    assert np.all(y[1, 0] == 0.0) and np.all(y[2, topk - 1] == 0.0)
+    ids_ok = ids.copy()
+    ids_ok[1, 0] = ids_ok[2, topk - 1] = 0
+    ref = O.moe_gate_up(x, ids_ok, codes, scales, 1, 1, E, N)
+    ref[1, 0] = ref[2, topk - 1] = 0.0
+    assert_close(y, ref, "moe skinny, bad ids")
 
 
 def test_moe_duplicate_expert_in_token():
