@@ -233,6 +233,26 @@ def run_reference(args, rank, world):
 # --------------------------------------------------------------------------
 # Secondary workloads (reported under "extras"; the headline is the W8A8 step)
 # --------------------------------------------------------------------------
+def _graph_call_us(torch, fn, stream, calls=64, reps=10):
+    """Mean us per fn(i) call, fn(0 .. calls-1) captured once in a CUDA graph and
+    replayed reps times on `stream` (CUDA events on that stream)."""
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gr, stream=stream):
+            for i in range(calls):
+                fn(i)
+        gr.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            gr.replay()
+        e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / (reps * calls) * 1e3
+
+
 def _traced(Q, fn, iters, kind):
     """Run fn(i) iters times with the library trace on; mean ms of `kind` launches."""
     Q.ql_trace_enable(64 * iters)
@@ -289,15 +309,19 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                 batches.append((bf(synth.activations(b, f"x_T{T}", T, Ke)), torch.from_numpy(ids).to(dev),
                                 len(set(ids.ravel().tolist()))))
             y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+            wsm = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.I8_G128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
+                              device=dev)
             run = lambda i: Q.moe_gate_up(batches[i % 8][0], batches[i % 8][1], codes, scales, E, Ne, y=y,  # noqa
-                                          stream=stream)
+                                          ws=wsm, stream=stream)
             for i in range(8):
                 run(i)
             t, per = _traced(Q, run, 40, "moe_gemm")
+            us_call = _graph_call_us(torch, run, stream)
             touched = float(np.mean([b[2] for b in batches]))
             byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
             res[str(T)] = {"us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
-                           "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per}
+                           "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per,
+                           "us_call_graph": us_call, "GB/s_call": byts / (us_call * 1e-6) / 1e9}
         out["moe_gate_up_decode"] = res
         # the same experts at prefill size, T = 2048 (every expert touched)
         T = 2048
@@ -305,10 +329,13 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
         xT = bf(synth.activations(0, "x_T2048", T, Ke))
         idsT = torch.from_numpy(ids).to(dev)
         yT = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
-        run = lambda i: Q.moe_gate_up(xT, idsT, codes, scales, E, Ne, y=yT, stream=stream)  # noqa: E731
+        wsT = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.I8_G128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
+                          device=dev)
+        run = lambda i: Q.moe_gate_up(xT, idsT, codes, scales, E, Ne, y=yT, ws=wsT, stream=stream)  # noqa: E731
         for i in range(2):
             run(i)
         t, per = _traced(Q, run, 5, "moe_gemm")
+        us_call = _graph_call_us(torch, run, stream, calls=8, reps=3)
         touched = len(set(ids.ravel().tolist()))
         byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
         flops = 2.0 * T * topk * Ne * Ke
@@ -317,6 +344,7 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
         out["moe_gate_up_prefill"] = {"T": T, "us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
                                       "TFLOPS": flops / (t * 1e-3) / 1e12, "roofline_us": 1e6 * t_roof,
                                       "frac": 1e6 * t_roof / (1e3 * t), "launches_per_call": per,
+                                      "us_call_graph": us_call,
                                       "roofline": "max(bytes / measured HBM, flops / measured bf16 peak)"}
         del codes, scales, xT, idsT, yT
         # prefill W8A8 at M = 2048 (tcgen05 kind::i8 GEMM with per-group fp32 promotion)
