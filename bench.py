@@ -51,7 +51,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "moe_decode", "moe_prefill"],
+    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "moe_decode", "moe_decode_t1",
+                                             "moe_prefill"],
                    default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
@@ -396,10 +397,10 @@ def ncu_case(name):
     prefill_w8a8 / prefill_fp8: the prefill workload (M = 2048, N = 21504,
     K = 5376; about 0.6 GB on the device), four forwards; the tcgen05 GEMM
     (k_prefill_w8a8 / k_prefill_a16) is launch 1..4 of its name.
-    moe_decode / moe_prefill: the MoE gate_up experts (128 x [1408, 2816] int8
-    g128 bf16, Hadamard domain; about 0.5 GB), top-8 routing of T = 16 / 2048
-    tokens, four calls of moe_gate_up (permute, activation prologue, expert
-    GEMM per call)."""
+    moe_decode / moe_decode_t1 / moe_prefill: the MoE gate_up experts (128 x
+    [1408, 2816] int8 g128 bf16, Hadamard domain; about 0.5 GB), top-8 routing
+    of T = 16 / 1 / 2048 tokens, four calls of moe_gate_up (activation
+    prologue and expert GEMM; the permute too at T = 2048)."""
     import torch
 
     from moe_hadamard128_act_b200 import qlinear as Q
@@ -408,7 +409,7 @@ def ncu_case(name):
     dev = torch.device("cuda", 0)
     if name.startswith("moe"):
         E, topk, Ke, Ne = 128, 8, 2816, 1408
-        T = 16 if name == "moe_decode" else 2048
+        T = {"moe_decode": 16, "moe_decode_t1": 1}.get(name, 2048)
         Ws = synth.moe_gate_up(1, experts=range(E))["W"]
         codes = torch.empty((E, Ne, Ke), dtype=torch.int8, device=dev)
         scales = torch.empty((E, Ne, Ke // 128), dtype=torch.int16, device=dev)

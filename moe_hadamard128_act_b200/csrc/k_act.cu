@@ -83,13 +83,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // With inv != null the row is written to rows inv[t * topk + j] (j < topk,
 // negative entries skipped) instead of row t: the permuted order of the
 // grouped expert GEMM.
-__global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int K, int rotate, int order, __half* xs,
-                                                  float* xf, float* yz, long long nz, const int32_t* inv, int topk) {
+__global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M, int K, int rotate, int order,
+                                                  __half* xs, float* xf, float* yz, long long nz, const int32_t* inv,
+                                                  int topk) {
     extern __shared__ float row[];  // [K] fp32, then (natural order) [K] f16
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
-    zero_fill(yz, nz);  // the GEMM that follows accumulates into y
-    __shared__ float red[8];
+    zero_fill(yz, nz);  // the GEMM that follows accumulates into y (CTAs past M only help with this)
     const int t = blockIdx.x;
+    if (t >= M) return;
+    __shared__ float red[8];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const __nv_bfloat16* xr = x + (long long)t * K;
     float amax = 0.0f;
@@ -212,8 +214,14 @@ cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, 
         e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_prep_a16<<<M, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, order, xs, xf, yz, nz, nullptr,
-                                    1);
+    DeviceInfo di;
+    if ((e = device_info(&di)) != cudaSuccess) return e;
+    // Small M: extra CTAs (no row work) share the zeroing of y, about 8 KB each.
+    const long long zb = yz ? (nz * 4 + 8191) / 8192 : 0;
+    const long long zc = zb < 2LL * di.sm_count ? zb : 2LL * di.sm_count;
+    const int grid = (int)(M > zc ? M : zc);
+    k_prep_a16<<<grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), M, K, rotate, order, xs, xf, yz, nz,
+                                       nullptr, 1);
     return cudaGetLastError();
 }
 
@@ -226,7 +234,7 @@ cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, con
         e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_prep_a16<<<T, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), K, rotate, XORD_NATURAL, xs, xf, nullptr, 0,
+    k_prep_a16<<<T, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), T, K, rotate, XORD_NATURAL, xs, xf, nullptr, 0,
                                     inv, topk);
     return cudaGetLastError();
 }
