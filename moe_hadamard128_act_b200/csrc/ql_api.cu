@@ -274,8 +274,10 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     const FwdWs w = forward_ws(fmt, M, N, K);
     if (!ws || ws_bytes < w.total()) return QL_EWORKSPACE;
     if (!aligned16(ws)) return QL_EALIGN;
-    const int kmax = skinny_max_k(fmt);
-    if (kmax < 128) return QL_ECUDA;
+    if (skinny_max_k(fmt) < 128) return QL_ECUDA;
+    // One decode launch per 16-row block covers the whole K: the kernel orders its
+    // units by K part and each CTA stages only the parts its unit range touches.
+    const int kmax = K;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int G = K / 128;
@@ -356,8 +358,8 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
 int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int K, int32_t* acc, void* stream) {
     if (M < 1 || N < 1 || K < 128 || K % 128 || !qx || !qw || !acc) return QL_EINVAL;
     if (!aligned16(qx) || !aligned16(qw) || !aligned16(acc)) return QL_EALIGN;
-    const int kmax = skinny_max_k(QL_I8A8_G128_BF16);
-    if (kmax < 128) return QL_ECUDA;
+    if (skinny_max_k(QL_I8A8_G128_BF16) < 128) return QL_ECUDA;
+    const int kmax = K;  // one launch per 16-row block (see qlinear_forward)
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int G = K / 128;
     if (M >= kPrefillMinM) {  // the same tensor-core GEMM qlinear_forward runs at this M
