@@ -270,12 +270,22 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
     G = K_FULL // 128
     bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     with torch.cuda.stream(stream):
-        # weight-only decode, int4 g64 and int5 + zero point g128
-        for name, fmt in (("w4a16_decode", Q.I4_G64_BF16), ("w5a16_decode", Q.I5Z_G128_F16)):
-            d = synth.w4a16(16) if fmt == Q.I4_G64_BF16 else synth.w5a16(16)
-            z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None
-            c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
-                                      scales=torch.from_numpy(d["scales"].view(np.int16)).to(dev), zeros=z)
+        # weight-only decode: int4 g64, int5 + zero point g128, int8 g128 bf16, fp8 128x128.
+        # "us" is the whole forward (activation prologue + decode GEMM) replayed from a
+        # CUDA graph, the rate it gives is over the forward's bytes; "us_gemm" is the
+        # traced decode kernel alone.
+        Wd = None
+        for name, fmt in (("w4a16_decode", Q.I4_G64_BF16), ("w5a16_decode", Q.I5Z_G128_F16),
+                          ("w8a16_decode", Q.I8_G128_BF16), ("fp8_decode", Q.FP8_B128_BF16)):
+            if fmt in (Q.I4_G64_BF16, Q.I5Z_G128_F16):
+                d = synth.w4a16(16) if fmt == Q.I4_G64_BF16 else synth.w5a16(16)
+                z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None
+                c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
+                                          scales=torch.from_numpy(d["scales"].view(np.int16)).to(dev), zeros=z)
+            else:
+                if Wd is None:
+                    Wd = torch.from_numpy(synth.weight_rows(0, "W", K_FULL, 0, N_FULL)).to(dev)
+                c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=Wd)
             cp = [(c, s, zz)] + [(c.clone(), s.clone(), None if zz is None else zz.clone()) for _ in range(3)]
             res = {}
             for m in (1, 5, 16) if fmt == Q.I4_G64_BF16 else (1, 4, 16):
@@ -286,12 +296,15 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                                                   y=y, ws=ws, stream=stream)
                 for i in range(8):
                     run(i)
-                t, _ = _traced(Q, run, 40, "skinny")
+                t, per = _traced(Q, run, 40, "skinny")
+                us = _graph_call_us(torch, run, stream)
                 cb, sb, zb = Q.qlinear_packed_sizes(fmt, N_FULL, K_FULL)
                 byts = cb + sb + zb + m * K_FULL * 2 + m * N_FULL * 4
-                res[str(m)] = {"us": 1e3 * t, "GB/s": byts / (t * 1e-3) / 1e9, "frac": byts / (t * 1e-3) / 1e9 / hbm}
+                res[str(m)] = {"us": us, "GB/s": byts / (us * 1e-6) / 1e9, "frac": byts / (us * 1e-6) / 1e9 / hbm,
+                               "us_gemm": 1e3 * t, "launches_per_call": per}
             out[name] = res
             del cp, c, s, zz
+        del Wd
         # MoE gate_up, int8 Hadamard-domain experts, decode batches
         E, topk, Ke, Ne = 128, 8, 2816, 1408
         Ws = synth.moe_gate_up(1, experts=range(E))["W"]
