@@ -32,6 +32,7 @@ I8A8_G128_BF16 = 3
 I4_G64_BF16 = 4
 I5Z_G128_F16 = 5
 FP8_B128_BF16 = 6
+FP8A8_B128_BF16 = 7
 HADAMARD = 1
 
 _c_p = ctypes.c_void_p
@@ -75,6 +76,8 @@ def lib():
             "qo_hadamard128_rotate": [_c_p, _c_i, _c_i, _c_p],
             "qo_act_quant_i8_g128": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
             "qo_act_quant_group": [_c_p, _c_p, _c_p],
+            "qo_act_quant_e4m3_g128": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
+            "qo_act_quant_e4m3_group": [_c_p, _c_p, _c_p],
             "qo_quant_i8_g128": [_c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p],
             "qo_quant_i4_g64": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
             "qo_quant_fp8_b128": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
@@ -170,6 +173,25 @@ def act_quant_i8_g128(x_bits: np.ndarray, rotate: bool):
     s = np.empty((M, K // 128), np.float32)
     lib().qo_act_quant_i8_g128(_p(x), M, K, int(rotate), _p(q), _p(s))
     return q, s
+
+
+def act_quant_e4m3_g128(x_bits: np.ndarray, rotate: bool):
+    """E4M3 codes (uint8) and fp32 scales per token per 128 (format 7's activations)."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), np.uint8)
+    s = np.empty((M, K // 128), np.float32)
+    lib().qo_act_quant_e4m3_g128(_p(x), M, K, int(rotate), _p(q), _p(s))
+    return q, s
+
+
+def act_quant_e4m3_group(v) -> tuple[np.ndarray, np.float32]:
+    """Quantise one fp32 group of 128 values to E4M3 (no rotation)."""
+    v = _c(v, np.float32)
+    q = np.empty(128, np.uint8)
+    s = np.empty(1, np.float32)
+    lib().qo_act_quant_e4m3_group(_p(v), _p(q), _p(s))
+    return q, s[0]
 
 
 def act_quant_group(v) -> tuple[np.ndarray, np.float32]:

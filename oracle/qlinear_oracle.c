@@ -19,6 +19,10 @@
  *     int5 codes with a u8 zero point and one f16 scale per 128 weights.
  *   "keptn/gemma4-12b-i8g", table "Format": int8 weights with a bf16 scale
  *     per 128, activations int8 with one scale per token and 128 values.
+ *   The FP8-activation variant of the fp8 container (format 7) takes the
+ *     weights of "gemma4-26b-a4b-dflash-fp8" unchanged and quantises the
+ *     activations as the int8 cards do -- one fp32 scale per token and 128
+ *     values -- but to E4M3 codes: a reading of this build, not a card's.
  *
  * Where the cards leave the arithmetic open, the oracle takes one plain
  * reading and states it at the function that implements it.  Everything is
@@ -40,7 +44,8 @@ enum {
     QO_I8A8_G128_BF16 = 3, /* int8 weights and int8 activations (W8A8)    */
     QO_I4_G64_BF16 = 4,    /* int4 [-8,7], bf16 scale per row per 64 K    */
     QO_I5Z_G128_F16 = 5,   /* int5 [0,31], u8 zero + f16 scale per 128 K  */
-    QO_FP8_B128_BF16 = 6   /* e4m3, bf16 scale per 128x128 block          */
+    QO_FP8_B128_BF16 = 6,  /* e4m3, bf16 scale per 128x128 block          */
+    QO_FP8A8_B128_BF16 = 7 /* the same weights, e4m3 activations          */
 };
 enum { QO_HADAMARD = 1 };
 
@@ -261,6 +266,45 @@ void qo_act_quant_group(const float* v, int8_t* q, float* s)
     }
 }
 
+/* E4M3 activations, per token per 128 values, in the same steps as the int8
+ * quantiser with 448 (the largest finite E4M3 value) in place of 127:
+ *   amax = max |v|;  s = fp32(amax / 448);  inv = fp32(448 / amax);
+ *   q[i] = e4m3_rne_satfinite(fp32(v[i] * inv)).
+ *   amax == 0 gives s = 0 and q = 0.  The scale is kept in fp32. */
+void qo_act_quant_e4m3_group(const float* v, uint8_t* q, float* s)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 128; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *s = 0.0f;
+        for (int i = 0; i < 128; ++i) q[i] = 0;
+        return;
+    }
+    volatile float sv = amax / 448.0f;
+    volatile float inv = 448.0f / amax;
+    *s = sv;
+    for (int i = 0; i < 128; ++i) {
+        volatile float p = v[i] * inv;
+        q[i] = qo_e4m3_encode((double)p);
+    }
+}
+
+void qo_act_quant_e4m3_g128(const uint16_t* x, int M, int K, int rotate, uint8_t* q, float* s)
+{
+    float v[128], r[128];
+    for (int m = 0; m < M; ++m)
+        for (int g = 0; g < K / 128; ++g) {
+            const uint16_t* src = x + (size_t)m * K + (size_t)g * 128;
+            for (int i = 0; i < 128; ++i) v[i] = (float)qo_bf16_decode(src[i]);
+            if (rotate) qo_fwht128_spec_f32(v, r);
+            else memcpy(r, v, sizeof r);
+            qo_act_quant_e4m3_group(r, q + (size_t)m * K + (size_t)g * 128, s + (size_t)m * (K / 128) + g);
+        }
+}
+
 void qo_act_quant_i8_g128(const uint16_t* x, int M, int K, int rotate, int8_t* q, float* s)
 {
     float v[128], r[128];
@@ -469,6 +513,7 @@ int qo_packed_sizes(int fmt, int N, int K, size_t* codes, size_t* scales, size_t
         *zeros = n * (k / 128);
         return 0;
     case QO_FP8_B128_BF16:
+    case QO_FP8A8_B128_BF16:
         *codes = n * k;
         *scales = ((n + 127) / 128) * (k / 128) * 2;
         return 0;
@@ -521,6 +566,7 @@ static void dequant_row(int fmt, const uint8_t* codes, const uint16_t* s, const 
         break;
     }
     case QO_FP8_B128_BF16:
+    case QO_FP8A8_B128_BF16:
         for (int k = 0; k < K; ++k)
             out[k] = scale_of(fmt, s, (N0 / 128) * (K / 128) + k / 128) * qo_e4m3_decode(codes[N0 * K + k]);
         break;
@@ -550,8 +596,32 @@ void qo_dequant(int fmt, const uint8_t* codes, const uint16_t* scales, const uin
 int qo_forward(const uint16_t* x, int M, int K, const uint8_t* codes, const uint16_t* scales,
                const uint8_t* zeros, int fmt, int flags, int N, double* y, int32_t* acc_out)
 {
-    if (fmt < QO_I8_G128_BF16 || fmt > QO_FP8_B128_BF16) return 1;
+    if (fmt < QO_I8_G128_BF16 || fmt > QO_FP8A8_B128_BF16) return 1;
     int G = K / 128;
+    if (fmt == QO_FP8A8_B128_BF16) {
+        /* E4M3 activations: y = sum_g sx[m,g] * sw[n/128,g] * sum_{k in g} e4m3(qx) * e4m3(qw).
+         * Every product of two E4M3 values and every partial sum here is exact in fp64. */
+        uint8_t* qx = (uint8_t*)malloc((size_t)M * K);
+        float* sx = (float*)malloc(sizeof(float) * (size_t)M * G);
+        qo_act_quant_e4m3_g128(x, M, K, flags & QO_HADAMARD, qx, sx);
+#pragma omp parallel for schedule(static)
+        for (int n = 0; n < N; ++n) {
+            const uint8_t* qw = codes + (size_t)n * K;
+            for (int m = 0; m < M; ++m) {
+                double sum = 0.0;
+                for (int g = 0; g < G; ++g) {
+                    double part = 0.0;
+                    for (int i = 0; i < 128; ++i)
+                        part += qo_e4m3_decode(qx[(size_t)m * K + g * 128 + i]) * qo_e4m3_decode(qw[g * 128 + i]);
+                    sum += (double)sx[(size_t)m * G + g] * qo_bf16_decode(scales[(size_t)(n / 128) * G + g]) * part;
+                }
+                y[(size_t)m * N + n] = sum;
+            }
+        }
+        free(qx);
+        free(sx);
+        return 0;
+    }
     if (fmt == QO_I8A8_G128_BF16) {
         int8_t* qx = (int8_t*)malloc((size_t)M * K);
         float* sx = (float*)malloc(sizeof(float) * (size_t)M * G);

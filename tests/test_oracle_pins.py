@@ -185,6 +185,49 @@ def test_act_quant_rotate_is_spec_transform_then_quant():
         assert np.max(np.abs(deq - rot)) <= 0.5 * float(s[0, g]) * (1 + 1e-4) + 1e-5 * np.abs(rot).max()
 
 
+def _torch_e4m3(vals32: np.ndarray) -> np.ndarray:
+    """E4M3 codes of fp32 values by torch's own conversion (round to nearest even)."""
+    return torch.from_numpy(np.ascontiguousarray(vals32, np.float32)).to(torch.float8_e4m3fn).view(
+        torch.uint8).numpy()
+
+
+def test_act_quant_e4m3_hand_example_and_zero():
+    # amax 448: s = 1 and the codes are torch's E4M3 conversion of the values themselves
+    v = np.zeros(128, np.float32)
+    v[:8] = [448.0, 1.0625, 1.1875, -3.3, 0.001, -448.0, 240.0, 2.0 ** -9]
+    q, s = O.act_quant_e4m3_group(v)
+    assert s == np.float32(1.0)
+    assert np.array_equal(q, _torch_e4m3(v))
+    assert list(q[:3]) == [0x7E, 0x38, 0x3A] and q[5] == 0xFE and q[7] == 0x01  # ties to even; a subnormal
+    q, s = O.act_quant_e4m3_group(np.zeros(128, np.float32))
+    assert s == 0 and not q.any()
+
+
+def test_act_quant_e4m3_rule_and_error_bound():
+    for _ in range(50):
+        v = (RNG.standard_normal(128) * RNG.uniform(1e-3, 1e3)).astype(np.float32)
+        q, s = O.act_quant_e4m3_group(v)
+        amax = np.max(np.abs(v))
+        assert s == np.float32(amax / np.float32(448))
+        inv = np.float32(np.float32(448) / amax)
+        assert np.array_equal(q, _torch_e4m3((v * inv).astype(np.float32)))  # fp32 product, then RNE
+        assert np.max(np.abs(O.e4m3_decode(q))) == 448.0
+        d = torch.from_numpy(q).view(torch.float8_e4m3fn).double().numpy() * float(s)
+        # half an E4M3 step: 2^-4 relative (3 mantissa bits), 2^-10 * s absolute in the subnormal range
+        assert np.all(np.abs(d - v) <= 2.0 ** -4 * np.abs(v) * (1 + 1e-6) + 2.0 ** -10 * float(s) * (1 + 1e-6))
+
+
+def test_act_quant_e4m3_rotate_is_spec_transform_then_quant():
+    x = O.bf16_encode(RNG.standard_normal(256) * 3)[None, :]
+    q, s = O.act_quant_e4m3_g128(x, rotate=True)
+    c = 1.0 / np.sqrt(128.0)
+    xv = O.bf16_decode(x)[0]
+    for g in range(2):
+        rot = O.fwht128_f64(xv[g * 128:(g + 1) * 128]) * c  # exact rotation
+        deq = float(s[0, g]) * O.e4m3_decode(q[0, g * 128:(g + 1) * 128])
+        assert np.all(np.abs(deq - rot) <= 2.0 ** -4 * np.abs(rot) + 2.0 ** -10 * float(s[0, g]) + 1e-5 * np.abs(rot).max())
+
+
 # --------------------------------------------------------------------------
 # Weight quantisers
 # --------------------------------------------------------------------------
@@ -295,7 +338,7 @@ def test_pack_i5_layout_and_roundtrip():
 
 @pytest.mark.parametrize("fmt,bpw", [(O.I4_G64_BF16, 4.25), (O.I8_G128_BF16, 8.125), (O.I8_G128_F16, 8.125),
                                      (O.I8A8_G128_BF16, 8.125), (O.I5Z_G128_F16, 5.1875),
-                                     (O.FP8_B128_BF16, 8 + 16 / 16384)])
+                                     (O.FP8_B128_BF16, 8 + 16 / 16384), (O.FP8A8_B128_BF16, 8 + 16 / 16384)])
 def test_packed_sizes_bits_per_weight(fmt, bpw):
     N, K = 21504, 5376
     c, s, z = O.packed_sizes(fmt, N, K)
@@ -365,6 +408,41 @@ def test_forward_brute_force_random_scales():
         torch.from_numpy(s8.view(np.int16)).view(torch.bfloat16).double().numpy(), 128, axis=1)
     y8 = O.forward(x, c8, s8, None, O.FP8_B128_BF16, 0, N)
     assert np.allclose(y8, xd @ W8.T, rtol=1e-12, atol=1e-14)
+
+
+def test_forward_fp8a8_equals_fp8_when_activations_are_exact():
+    # Every 128-group has amax 448 * 2^j and values that are E4M3 values times 2^j: the E4M3
+    # activation codes then represent x exactly, so format 7 must equal format 6 on the same x.
+    M, N, K = 3, 5, 384
+    fin = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    fin = fin[np.isfinite(fin)]
+    xv = np.empty((M, K))
+    for m in range(M):
+        for g in range(K // 128):
+            j = int(RNG.integers(-6, 4))
+            blk = RNG.choice(fin, 128) * RNG.choice([-1.0, 1.0], 128)
+            blk[int(RNG.integers(128))] = 448.0
+            xv[m, g * 128:(g + 1) * 128] = blk * 2.0 ** j
+    x = O.bf16_encode(xv)
+    assert np.array_equal(O.bf16_decode(x), xv)  # representable in bf16 too
+    codes, scales = O.quant_fp8_b128((RNG.standard_normal((N, K)) * 0.02).astype(np.float32))
+    y7 = O.forward(x, codes, scales, None, O.FP8A8_B128_BF16, 0, N)
+    y6 = O.forward(x, codes, scales, None, O.FP8_B128_BF16, 0, N)
+    assert np.allclose(y7, y6, rtol=1e-12, atol=1e-14)
+
+
+def test_forward_fp8a8_brute_force():
+    # explicit fp64 sum from torch-decoded activation and weight codes and scales
+    M, N, K = 3, 130, 256
+    x = O.bf16_encode(RNG.standard_normal((M, K)))
+    codes, scales = O.quant_fp8_b128((RNG.standard_normal((N, K)) * 0.02).astype(np.float32))
+    qx, sx = O.act_quant_e4m3_g128(x, rotate=False)
+    xd = torch.from_numpy(qx).view(torch.float8_e4m3fn).double().numpy() * np.repeat(sx.astype(np.float64), 128, axis=1)
+    sw = torch.from_numpy(scales.view(np.int16)).view(torch.bfloat16).double().numpy()
+    Wd = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy() * np.repeat(
+        np.repeat(sw, 128, axis=1), 128, axis=0)[:N]
+    y = O.forward(x, codes, scales, None, O.FP8A8_B128_BF16, 0, N)
+    assert np.allclose(y, xd @ Wd.T, rtol=1e-12, atol=1e-14)
 
 
 def test_w8a8_int32_accumulators_and_combination():
