@@ -21,13 +21,20 @@
  *   QL_FP8_B128_BF16  FP8 E4M3 codes with one bf16 scale per 128 (rows) x 128
  *                     (K) block ("gemma4-26b-a4b-dflash-fp8" README, table
  *                     "Weights" and its recipe); x is bf16.
+ *   QL_FP8A8_B128_BF16  the same packed weights with E4M3 activations: x is
+ *                     quantised per token per 128 values as
+ *                     act_quant_e4m3_g128 does (the int8 activation rule of
+ *                     "keptn/gemma4-12b-i8g" with E4M3 codes; a reading, no card
+ *                     ships it), and every 128-group's products are summed
+ *                     before both scales are applied.  All M run the
+ *                     tensor-core E4M3 GEMM.
  * Flag QL_HADAMARD: the weights live in the 128-wide Walsh-Hadamard domain
  * ("transform=fwht128" in the recipe of "gemma4-26b-a4b-dflash-i8"); the
  * forward pass rotates each 128-block of x by the same orthonormal transform
  * first, so that (H x) . (H w) = x . w.
  *
  * Packed layouts (all row-major, W is [N, K] with K contiguous):
- *   int8 / fp8 codes: one byte per code, [N][K].
+ *   int8 / fp8 codes: one byte per code, [N][K] (formats 6 and 7 pack alike).
  *   int4 codes: [N][K/2] bytes, code k of a row in byte k/2, low nibble for
  *     even k, stored offset-binary (q + 8).
  *   int5 codes: [N][5K/8] bytes, each row a least-significant-bit-first bit
@@ -78,7 +85,8 @@ typedef enum {
     QL_I8A8_G128_BF16 = 3,
     QL_I4_G64_BF16 = 4,
     QL_I5Z_G128_F16 = 5,
-    QL_FP8_B128_BF16 = 6
+    QL_FP8_B128_BF16 = 6,
+    QL_FP8A8_B128_BF16 = 7
 } ql_fmt;
 
 enum { QL_HADAMARD = 1 };
@@ -148,6 +156,13 @@ int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int
  * q = clamp(rne(fp32(v * fp32(127/amax))), -127, 127); amax = 0 gives s = 0,
  * q = 0.  x bf16 [M, K]; q int8 [M, K]; s fp32 [M, K/128]. */
 int act_quant_i8_g128(const void* x, int M, int K, int rotate, int8_t* q, float* s, void* stream);
+
+/* act_quant_e4m3_g128 -- the same rule with E4M3 codes (QL_FP8A8_B128_BF16's
+ * activations): s = fp32(amax/448), q = e4m3(fp32(v * fp32(448/amax))) rounded
+ * to nearest even and saturated to +-448 (448 is the largest finite E4M3
+ * value); amax = 0 gives s = 0, q = 0.  x bf16 [M, K]; q E4M3 bytes [M, K];
+ * s fp32 [M, K/128]. */
+int act_quant_e4m3_g128(const void* x, int M, int K, int rotate, uint8_t* q, float* s, void* stream);
 
 /* hadamard128_rotate -- y = per-128-block orthonormal Walsh-Hadamard
  * transform of x along K, Sylvester order (the "attention join" of

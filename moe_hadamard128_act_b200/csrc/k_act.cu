@@ -46,7 +46,9 @@ __device__ __forceinline__ void zero_fill(float* y, long long n) {
     for (long long i = (n & ~3LL) + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) y[i] = 0.f;
 }
 
-// s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127).
+// s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127);
+// with E4M3 set, the E4M3 rule (448 for 127, codes by the hardware conversion).
+template <bool E4M3>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bfloat16* x, int M, int K, int rotate,
                                                                    int8_t* q, float* sx, float* sxT, int Mp,
                                                                    float* yz, long long nz) {
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
         load4_bf16(x + off, v);
         if (rotate) fwht128_warp(v, lane);
         float s;
-        const uint32_t packed = quant_i8_group_warp(v, &s);
+        const uint32_t packed = E4M3 ? quant_e4m3_group_warp(v, &s) : quant_i8_group_warp(v, &s);
         *reinterpret_cast<uint32_t*>(q + off) = packed;
         if (lane == 0) {
             if (sx) sx[u] = s;                                 // [M][G] row-major: u = m * G + g
@@ -165,15 +167,23 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
 // The GEMM that follows these kernels runs with (nearly) all of the SM's
 // shared memory; asking for the same L1/shared split here avoids an SM
 // reconfiguration between the two launches.
+// Once per kernel and device (kernels of one signature share F, so the flag is
+// kept per kernel address).
 template <typename F>
 cudaError_t prefer_max_shared(F* kernel) {
-    static bool done[64] = {};
+    struct Done {
+        const void* k;
+        int dev;
+    };
+    static Done done[64];
+    static int n = 0;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && done[dev]) return cudaSuccess;
+    for (int i = 0; i < n; ++i)
+        if (done[i].k == (const void*)kernel && done[i].dev == dev) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          (int)cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess && dev < 64) done[dev] = true;
+    if (e == cudaSuccess && n < 64) done[n++] = Done{(const void*)kernel, dev};
     return e;
 }
 
@@ -199,9 +209,20 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
-    if ((e = prefer_max_shared(k_act_quant)) != cudaSuccess) return e;
-    k_act_quant<<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
+    if ((e = prefer_max_shared(k_act_quant<false>)) != cudaSuccess) return e;
+    k_act_quant<false><<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, sxT, Mp, yz, nz);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
+                                  cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    if ((e = prefer_max_shared(k_act_quant<true>)) != cudaSuccess) return e;
+    k_act_quant<true><<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), M, K, rotate, reinterpret_cast<int8_t*>(q), sx, sxT, Mp, nullptr, 0);
     return cudaGetLastError();
 }
 

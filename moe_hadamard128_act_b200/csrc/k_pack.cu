@@ -217,7 +217,8 @@ cudaError_t launch_pack_rtn(const float* W, int fmt, int flags, int N, int K, vo
     case QL_I4_G64_BF16:
         k_rtn_i4<<<grid, 256, 0, s>>>(W, N, K, had, static_cast<uint8_t*>(codes), static_cast<uint16_t*>(scales));
         break;
-    case QL_FP8_B128_BF16: {
+    case QL_FP8_B128_BF16:
+    case QL_FP8A8_B128_BF16: {
         const int smem = 128 * 128 * sizeof(float);
         e = cudaFuncSetAttribute(k_rtn_fp8, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
@@ -243,7 +244,8 @@ cudaError_t launch_pack_codes(const void* codes_in, int fmt, int N, int K, void*
     switch (fmt) {
     case QL_I4_G64_BF16: k_pack_codes<QL_I4_G64_BF16><<<grid, 256, 0, s>>>(in, n8, out, err); break;
     case QL_I5Z_G128_F16: k_pack_codes<QL_I5Z_G128_F16><<<grid, 256, 0, s>>>(in, n8, out, err); break;
-    case QL_FP8_B128_BF16: k_pack_codes<QL_FP8_B128_BF16><<<grid, 256, 0, s>>>(in, n8, out, err); break;
+    case QL_FP8_B128_BF16:
+    case QL_FP8A8_B128_BF16: k_pack_codes<QL_FP8_B128_BF16><<<grid, 256, 0, s>>>(in, n8, out, err); break;
     default: k_pack_codes<QL_I8_G128_BF16><<<grid, 256, 0, s>>>(in, n8, out, err); break;
     }
     return cudaGetLastError();

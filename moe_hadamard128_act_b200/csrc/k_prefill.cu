@@ -35,6 +35,13 @@
 // the running sum.  The first runs as packed two-lane FMAs (FFMA2, heavy FMA
 // pipe only), the second as scalar FMAs, so both FMA pipes are busy.
 //
+// The same kernel runs format 7 (E4M3 weights and E4M3 activations, an fp32
+// scale per token per 128 and a bf16 scale per 128 x 128 weight block) with
+// tcgen05.mma kind::f8f6f4 at the same rate: the tiles are bytes either way,
+// the accumulators hold fp32 group sums, and since a weight scale covers a
+// whole 128-row block the promotion is one FMA per element with s_x * s_w taken
+// once per 16 columns.
+//
 // All waits are bounded (200 ms); on a timeout the CTA sets
 // QL_DEVERR_TIMEOUT and winds down without leaving tensor memory allocated,
 // MMAs running or copies in flight.
@@ -63,6 +70,8 @@ constexpr int NCH = WGC / CW;             // reads per step
 constexpr uint32_t kMagic = 0x4B400000u;  // 12582912.0f
 static_assert(PN % 32 == 0 && PN >= 128 && PN <= 256 && NBUF >= 2, "one MMA per K chunk covers the tile; 2+ accumulators");
 static_assert(WGC % CW == 0, "whole tensor-memory reads per thread");
+static_assert(PN % CW == 0 && WGC % CW == 0 && 128 % CW == 0,
+              "column chunks start on multiples of CW, so none crosses a 128-row weight block");
 static_assert(PN % 64 == 0 || PN == 160, "tile widths whose column quarters are whole reads");
 static_assert(SCB >= PSTAGES + NBUF, "the scale ring must not throttle the operand ring");
 static_assert((PSTAGES & (PSTAGES - 1)) == 0 && (SCB & (SCB - 1)) == 0, "operand and scale slots from step counters");
@@ -84,16 +93,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// MMA kinds of this kernel: int8 x int8 -> s32, and E4M3 x E4M3 -> f32.
+enum { kKindI8 = 0, kKindE4M3 = 1 };
 // kind::i8, D s32, A s8, B s8, both K-major, N = PN, M = 128.
 constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PN >> 3) << 17) |
                               ((uint32_t)(PM >> 4) << 24);
+// kind::f8f6f4, D f32, A e4m3 (0), B e4m3 (0), both K-major, N = PN, M = 128.
+constexpr uint32_t kIdescE4M3 = (1u << 4) | ((uint32_t)(PN >> 3) << 17) | ((uint32_t)(PM >> 4) << 24);
 
-// D (+)= A * B^T; acc_in = 0 overwrites D.
-__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc_in) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(acc_in));
+// D (+)= A * B^T with K = 32 bytes; acc_in = 0 overwrites D.
+template <int KIND>
+__device__ __forceinline__ void mma_k32(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc_in) {
+    if (KIND == kKindI8)
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(acc_in));
+    else
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+            "l"(adesc), "l"(bdesc), "r"(kIdescE4M3), "r"(acc_in));
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
@@ -139,8 +159,9 @@ struct PrefillArgs {
 constexpr int kRegsDriver = 24, kRegsEpi = 112;
 static_assert(128 * kRegsDriver + 32 * kEpiWarps * kRegsEpi <= kPThreads * 96, "register split");
 
-template <bool ACC>
+template <bool ACC, int KIND>
 __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_constant__ PrefillArgs a) {
+    static_assert(!ACC || KIND == kKindI8, "the integer group sums exist for int8 only");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -234,7 +255,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 const uint64_t so = (uint64_t)(s * (STAGE_BYTES >> 4));
                 const uint32_t d = tmem + b * PN;
 #pragma unroll
-                for (int kk = 0; kk < PKB / 32; ++kk) mma_i8(d, da0 + so + 2 * kk, db0 + so + 2 * kk, kk ? 1u : 0u);
+                for (int kk = 0; kk < PKB / 32; ++kk)
+                    mma_k32<KIND>(d, da0 + so + 2 * kk, db0 + so + 2 * kk, kk ? 1u : 0u);
                 mma_commit(bar(BAR_EMPTY + s));  // operand slot free once these MMAs are done
                 mma_commit(bar(BAR_ACCF + b));   // accumulator ready for the epilogue
             }
@@ -270,12 +292,15 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             const uint32_t taddr = tmem + tlane + b * PN + tcol;
             const float* scp = reinterpret_cast<const float*>(gb + SC_OFF + c * SC_BYTES);
             float sxr = 0.0f, kb = 0.0f;
-            if (!ACC) {
+            if (!ACC && KIND == kKindE4M3) {
+                sxr = scp[row];  // fp32 group sums: t = s_x * sum, no bias
+            } else if (!ACC) {
                 // s_x cut to 22 significant bits: s_x * 12582912 is exact, so the first FMA is
                 // round(s_x * sum) (the accumulator bits read as fp32 are 12582912 + sum).
                 sxr = __int_as_float(__float_as_int(scp[row]) & ~3);
                 kb = -sxr * 12582912.0f;
             }
+            const uint32_t mg = KIND == kKindE4M3 ? 0u : kMagic;
             const float2 sx2 = make_float2(sxr, sxr), kb2 = make_float2(kb, kb);
             uint32_t v[2][CW];
             QL_TMEM_LD16(taddr, v[0]);
@@ -290,6 +315,23 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
 #pragma unroll
                         for (int i = 0; i < CW; ++i)
                             if (n0 + i < a.N) a.acc[((long long)m * a.N + n0 + i) * G + g] = (int)cur[i];
+                } else if constexpr (KIND == kKindE4M3) {
+                    // fp8 weights scale whole 128-row blocks, and a 16-column chunk starts on a
+                    // multiple of 16 weight rows, so it never crosses a block: one s_x * s_w per
+                    // chunk, then one FMA per element (half packed, half scalar: both FMA pipes).
+                    const float p = sxr * scp[PM + tcol + h * CW];
+                    const float2 p2 = make_float2(p, p);
+#pragma unroll
+                    for (int q = 0; q < CW / 4; ++q) {
+                        float* const yq = yr + h * CW + 4 * q;
+                        const float2 u = __ffma2_rn(p2, make_float2(__uint_as_float(cur[4 * q]),
+                                                                    __uint_as_float(cur[4 * q + 1])),
+                                                    make_float2(yq[0], yq[1]));
+                        yq[0] = u.x;
+                        yq[1] = u.y;
+                        yq[2] = fmaf(p, __uint_as_float(cur[4 * q + 2]), yq[2]);
+                        yq[3] = fmaf(p, __uint_as_float(cur[4 * q + 3]), yq[3]);
+                    }
                 } else {
                     // Weight scales read in place (volatile loads stay in their chunk instead of being
                     // hoisted, which would cost registers).
@@ -300,10 +342,10 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                         const float4 cs = make_float4(__uint_as_float(cu.x), __uint_as_float(cu.y),
                                                       __uint_as_float(cu.z), __uint_as_float(cu.w));
                         // sum + 0x4B400000, read as fp32, is exactly 12582912 + sum
-                        const float2 t0 = __ffma2_rn(sx2, make_float2(__uint_as_float(cur[4 * q] + kMagic),
-                                                                      __uint_as_float(cur[4 * q + 1] + kMagic)), kb2);
-                        const float2 t1 = __ffma2_rn(sx2, make_float2(__uint_as_float(cur[4 * q + 2] + kMagic),
-                                                                      __uint_as_float(cur[4 * q + 3] + kMagic)), kb2);
+                        const float2 t0 = __ffma2_rn(sx2, make_float2(__uint_as_float(cur[4 * q] + mg),
+                                                                      __uint_as_float(cur[4 * q + 1] + mg)), kb2);
+                        const float2 t1 = __ffma2_rn(sx2, make_float2(__uint_as_float(cur[4 * q + 2] + mg),
+                                                                      __uint_as_float(cur[4 * q + 3] + mg)), kb2);
                         float* const yq = yr + h * CW + 4 * q;
                         yq[0] = fmaf(cs.x, t0.x, yq[0]);
                         yq[1] = fmaf(cs.y, t0.y, yq[1]);
@@ -373,7 +415,23 @@ __global__ void __launch_bounds__(256) k_prefill_prep(const uint16_t* sw, int N,
     }
 }
 
+// bf16 block scales [ceil(N/128)][G] -> fp32 [G][Np], each row's block scale
+// repeated for the 128 rows of its block; columns n >= N zero.
+__global__ void __launch_bounds__(256) k_prefill_prep_blk(const uint16_t* sw, int N, int G, int Np, float* swT) {
+    const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (i >= (long long)G * Np) return;
+    const int g = (int)(i / Np), n = (int)(i - (long long)g * Np);
+    swT[i] = n < N ? __uint_as_float((uint32_t)sw[(long long)(n >> 7) * G + g] << 16) : 0.0f;
+}
+
 }  // namespace
+
+cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s) {
+    const int G = K / 128, Np = prefill_pad_n(N);
+    const long long n = (long long)G * Np;
+    k_prefill_prep_blk<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sw, N, G, Np, static_cast<float*>(scratch));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s) {
     const int G = K / 128, Np = prefill_pad_n(N);
@@ -383,7 +441,7 @@ cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch,
 }
 
 cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t* qw, int M, int N, int K, float* y,
-                                long long ldy, int32_t* acc, const void* scratch, cudaStream_t s) {
+                                long long ldy, int32_t* acc, const void* scratch, cudaStream_t s, bool e4m3) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
@@ -409,14 +467,17 @@ cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        for (auto fn : {k_prefill_w8a8<false>, k_prefill_w8a8<true>}) {
+        for (auto fn : {k_prefill_w8a8<false, kKindI8>, k_prefill_w8a8<true, kKindI8>,
+                        k_prefill_w8a8<false, kKindE4M3>}) {
             if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
                 return e;
         }
         if (dev < 64) attr_set[dev] = true;
     }
-    if (acc) k_prefill_w8a8<true><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
-    else k_prefill_w8a8<false><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
+    if (acc && e4m3) return cudaErrorInvalidValue;
+    if (acc) k_prefill_w8a8<true, kKindI8><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
+    else if (e4m3) k_prefill_w8a8<false, kKindE4M3><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
+    else k_prefill_w8a8<false, kKindI8><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -15,7 +15,7 @@ __device__ unsigned g_ql_err;
 void packed_sizes(int fmt, size_t N, size_t K, size_t* codes, size_t* scales, size_t* zeros) {
     *codes = N * fmt_row_bytes(fmt, K);
     *zeros = fmt == QL_I5Z_G128_F16 ? N * (K / 128) : 0;
-    if (fmt == QL_FP8_B128_BF16) *scales = ((N + 127) / 128) * (K / 128) * 2;
+    if (fmt_fp8_weights(fmt)) *scales = ((N + 127) / 128) * (K / 128) * 2;
     else *scales = N * (K / fmt_group(fmt)) * 2;
 }
 
@@ -122,7 +122,11 @@ struct FwdWs {
 FwdWs forward_ws(int fmt, size_t M, size_t N, size_t K) {
     FwdWs w;
     w.g_bytes = 0;
-    if (fmt == QL_I8A8_G128_BF16) {
+    if (fmt == QL_FP8A8_B128_BF16) {  // E4M3 codes, transposed scales, the GEMM's weight scales (every M)
+        w.x_bytes = align_up(M * K, 256);
+        w.f_bytes = align_up((K / 128) * prefill_pad_m((int)M) * 4, 256);
+        w.g_bytes = prefill_scratch_bytes((int)N, (int)K);
+    } else if (fmt == QL_I8A8_G128_BF16) {
         w.x_bytes = align_up(M * K, 256);
         if (M >= (size_t)kPrefillMinM) {
             w.f_bytes = align_up((K / 128) * prefill_pad_m((int)M) * 4, 256);
@@ -267,7 +271,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
     if (!x || !W_packed || !scales || !y) return QL_EINVAL;
     if (fmt == QL_I5Z_G128_F16 && !zeros) return QL_EINVAL;
-    if (fmt != QL_I8A8_G128_BF16 && K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
+    if (fmt != QL_I8A8_G128_BF16 && fmt != QL_FP8A8_B128_BF16 && K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
     if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y) ||
         (zeros && !aligned16(zeros)))
         return QL_EALIGN;
@@ -286,6 +290,22 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     void* xs = wsb;
     float* xf = reinterpret_cast<float*>(wsb + w.x_bytes);
     cudaError_t e;
+    if (fmt == QL_FP8A8_B128_BF16) {  // E4M3 activations, the tensor-core E4M3 GEMM for every M
+        int t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant_e4m3(x, M, K, rot, static_cast<uint8_t*>(xs), nullptr, xf, prefill_pad_m(M), s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        uint8_t* const gs = wsb + w.x_bytes + w.f_bytes;
+        t = trace_begin(QL_KIND_PREFILL_PREP, s);
+        e = launch_prefill_prep_blk(static_cast<const uint16_t*>(scales), N, K, gs, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_PREFILL, s);
+        e = launch_prefill_w8a8(static_cast<const int8_t*>(xs), xf, static_cast<const int8_t*>(W_packed), M, N, K, y,
+                                N, nullptr, gs, s, true);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     if (fmt == QL_I8A8_G128_BF16 && M >= kPrefillMinM) {  // tensor-core GEMM, y written directly
         int t = trace_begin(QL_KIND_ACT_QUANT, s);
         e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), nullptr, xf, prefill_pad_m(M), nullptr, 0, s);
@@ -400,6 +420,16 @@ int act_quant_i8_g128(const void* x, int M, int K, int rotate, int8_t* q, float*
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int t = trace_begin(QL_KIND_ACT_QUANT, st);
     const cudaError_t e = launch_act_quant(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, nullptr, 0, st);
+    trace_end(t, st);
+    return from_cuda(e);
+}
+
+int act_quant_e4m3_g128(const void* x, int M, int K, int rotate, uint8_t* q, float* s, void* stream) {
+    if (M < 1 || K < 128 || K % 128 || !x || !q || !s) return QL_EINVAL;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return QL_EALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int t = trace_begin(QL_KIND_ACT_QUANT, st);
+    const cudaError_t e = launch_act_quant_e4m3(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, st);
     trace_end(t, st);
     return from_cuda(e);
 }

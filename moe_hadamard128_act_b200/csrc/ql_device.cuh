@@ -81,6 +81,32 @@ __device__ __forceinline__ uint32_t quant_i8_group_warp(const float v[4], float*
     *s_out = s;
     return packed;
 }
+// Two fp32 values to E4M3 by the hardware conversion (round to nearest even,
+// saturating to +-448): the low byte holds `lo`, the high byte `hi`.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
+    uint16_t r;
+    asm("{\n .reg .b16 t;\n cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n mov.b16 %0, t;\n}\n" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// The E4M3 quantiser of one 128-group held 4 values per lane by a warp: the
+// int8 rule with 448, the largest finite E4M3 value, in place of 127:
+// s = fp32(amax / 448), q = e4m3(fp32(v * fp32(448 / amax))); amax = 0 gives
+// s = 0 and q = 0.  Returns the lane's 4 codes packed low byte first.
+__device__ __forceinline__ uint32_t quant_e4m3_group_warp(const float v[4], float* s_out) {
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    amax = warp_max(amax);
+    uint32_t packed = 0;
+    float s = 0.0f;
+    if (amax > 0.0f) {
+        s = __fdiv_rn(amax, 448.0f);
+        const float inv = __fdiv_rn(448.0f, amax);
+        const uint32_t lo = cvt_e4m3x2(__fmul_rn(v[1], inv), __fmul_rn(v[0], inv));
+        const uint32_t hi = cvt_e4m3x2(__fmul_rn(v[3], inv), __fmul_rn(v[2], inv));
+        packed = lo | (hi << 16);
+    }
+    *s_out = s;
+    return packed;
+}
 __device__ __forceinline__ float f16_bits_to_float(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {

@@ -13,7 +13,9 @@
 namespace ql {
 
 // ---- format arithmetic -------------------------------------------------------
-inline bool fmt_valid(int f) { return f >= QL_I8_G128_BF16 && f <= QL_FP8_B128_BF16; }
+inline bool fmt_valid(int f) { return f >= QL_I8_G128_BF16 && f <= QL_FP8A8_B128_BF16; }
+// FP8 E4M3 weights with 128 x 128 block scales (formats 6 and 7 pack alike).
+inline bool fmt_fp8_weights(int f) { return f == QL_FP8_B128_BF16 || f == QL_FP8A8_B128_BF16; }
 inline bool fmt_scale_f16(int f) { return f == QL_I8_G128_F16 || f == QL_I5Z_G128_F16; }
 inline int fmt_group(int f) { return f == QL_I4_G64_BF16 ? 64 : 128; }
 // Bytes of one packed row of K codes.
@@ -53,6 +55,9 @@ cudaError_t launch_rotate_bf16(const void* x, int M, int K, void* y, cudaStream_
 // to sxT (either may be null).
 cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* sxT, int Mp,
                              float* yz, long long nz, cudaStream_t s);
+// The same rule with E4M3 codes (448 for 127), written as bytes.
+cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
+                                  cudaStream_t s);
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s);
 // The same for the grouped expert GEMM: token t's f16 row goes to rows
@@ -102,10 +107,14 @@ inline int prefill_pad_m(int v) { return (v + kPrefillTileM - 1) / kPrefillTileM
 inline int prefill_pad_n(int v) { return (v + kPrefillTileN - 1) / kPrefillTileN * kPrefillTileN; }
 static_assert(kPrefillTileN % 32 == 0, "weight-scale padding is a whole number of 32-wide transpose tiles");
 inline size_t prefill_scratch_bytes(int N, int K) { return align_up((size_t)(K / 128) * prefill_pad_n(N) * 4, 256); }
+// e4m3: qx and qw hold E4M3 codes (format 7), the MMAs run kind::f8f6f4.
 cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t* qw, int M, int N, int K,
-                                float* y, long long ldy, int32_t* acc, const void* scratch, cudaStream_t s);
+                                float* y, long long ldy, int32_t* acc, const void* scratch, cudaStream_t s,
+                                bool e4m3 = false);
 // Fills the scratch: bf16 weight scales [N][K/128] -> fp32 [K/128][pad(N)].
 cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
+// The same from bf16 block scales [ceil(N/128)][K/128] (each row takes its block's scale).
+cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
 constexpr int kPrefillMinM = 17;  // from this many tokens on, W8A8 runs on the tcgen05 GEMM
 
 // The same for the formats with 16-bit activations (int8 g128 with bf16 or f16

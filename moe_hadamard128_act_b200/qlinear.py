@@ -24,8 +24,9 @@ I8A8_G128_BF16 = 3
 I4_G64_BF16 = 4
 I5Z_G128_F16 = 5
 FP8_B128_BF16 = 6
+FP8A8_B128_BF16 = 7  # the fp8 weights with E4M3 activations
 HADAMARD = 1
-FORMATS = (I8_G128_BF16, I8_G128_F16, I8A8_G128_BF16, I4_G64_BF16, I5Z_G128_F16, FP8_B128_BF16)
+FORMATS = (I8_G128_BF16, I8_G128_F16, I8A8_G128_BF16, I4_G64_BF16, I5Z_G128_F16, FP8_B128_BF16, FP8A8_B128_BF16)
 
 DEVERR_EXPERT_ID = 1
 DEVERR_CODE_RANGE = 2
@@ -211,6 +212,16 @@ def act_quant_i8_g128(x: torch.Tensor, rotate: bool = False, stream=None):
     s = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
     _check("act_quant_i8_g128", lib().act_quant_i8_g128(_ptr(x), M, K, int(rotate), _ptr(q), _ptr(s),
                                                         _stream(stream)))
+    return q, s
+
+
+def act_quant_e4m3_g128(x: torch.Tensor, rotate: bool = False, stream=None):
+    """E4M3 codes (uint8 [M, K]) and fp32 scales [M, K/128] per token per 128."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _check("act_quant_e4m3_g128", lib().act_quant_e4m3_g128(_ptr(x), M, K, int(rotate), _ptr(q), _ptr(s),
+                                                            _stream(stream)))
     return q, s
 
 

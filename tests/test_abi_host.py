@@ -38,7 +38,8 @@ def test_binding_constants_match_header():
     from moe_hadamard128_act_b200 import qlinear as Q
     text = (ROOT / "include" / "qlinear.h").read_text()
     assert int(re.search(r"QL_A16_MAX_K\s*=\s*(\d+)", text).group(1)) == Q.A16_MAX_K
-    for name in ("I8_G128_BF16", "I8_G128_F16", "I8A8_G128_BF16", "I4_G64_BF16", "I5Z_G128_F16", "FP8_B128_BF16"):
+    for name in ("I8_G128_BF16", "I8_G128_F16", "I8A8_G128_BF16", "I4_G64_BF16", "I5Z_G128_F16", "FP8_B128_BF16",
+                 "FP8A8_B128_BF16"):
         assert int(re.search(rf"QL_{name}\s*=\s*(\d+)", text).group(1)) == getattr(Q, name), name
 
 
@@ -48,7 +49,7 @@ def test_status_strings(L):
     assert L.ql_status_string(99) == b"unknown status"
 
 
-@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 5, 6, 7])
 @pytest.mark.parametrize("N,K", [(1, 128), (200, 384), (21504, 5376), (1408, 2816)])
 def test_packed_sizes_match_oracle(L, fmt, N, K):
     from moe_hadamard128_act_b200 import qlinear as Q
@@ -57,7 +58,7 @@ def test_packed_sizes_match_oracle(L, fmt, N, K):
 
 def test_packed_sizes_and_workspace_reject_bad_args(L):
     from moe_hadamard128_act_b200 import qlinear as Q
-    for fmt, N, K in ((0, 8, 128), (7, 8, 128), (1, 0, 128), (1, 8, 64), (1, 8, 200)):
+    for fmt, N, K in ((0, 8, 128), (8, 8, 128), (1, 0, 128), (1, 8, 64), (1, 8, 200)):
         with pytest.raises(Q.QLError) as e:
             Q.qlinear_packed_sizes(fmt, N, K)
         assert e.value.status == 1
@@ -65,6 +66,7 @@ def test_packed_sizes_and_workspace_reject_bad_args(L):
         Q.qlinear_workspace_size(1, 2, 1, 8, 128)  # unknown flag
     assert Q.qlinear_workspace_size(1, 0, 16, 21504, 5376) >= 16 * 5376 * 2
     assert Q.qlinear_workspace_size(3, 1, 16, 21504, 5376) >= 16 * 5376 + 16 * 42 * 4
+    assert Q.qlinear_workspace_size(7, 1, 1, 21504, 5376) >= 5376 + 42 * 128 * 4 + 42 * 21504 * 4
 
 
 A = 1 << 20  # an aligned fake address: every call below fails validation first
@@ -105,6 +107,8 @@ def test_pack_and_act_validation_statuses(L):
     assert p(None, P(A), None, None, 4, 0, 8, 128, P(A), P(A), None, None) == 1  # codes without scales
     assert p(None, P(A), P(A), None, 5, 0, 8, 128, P(A), P(A), P(A), None) == 1  # int5 codes without zeros
     assert L.act_quant_i8_g128(P(A), 4, 100, 0, P(A), P(A), None) == 1
+    assert L.act_quant_e4m3_g128(P(A), 4, 100, 0, P(A), P(A), None) == 1
+    assert L.act_quant_e4m3_g128(P(A), 4, 128, 0, P(A + 4), P(A), None) == 3
     assert L.act_quant_i8_g128(P(A + 2), 4, 128, 0, P(A), P(A), None) == 3
     assert L.hadamard128_rotate(P(A), 0, 128, P(A), None) == 1
     assert L.hadamard128_rotate(P(A), 1, 128, P(A + 1), None) == 3

@@ -59,6 +59,19 @@ def test_act_quant_bitexact(M, K, rotate):
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("rotate", [False, True])
+@pytest.mark.parametrize("M,K", [(1, 128), (4, 384), (16, 5376), (2048, 256)])
+def test_act_quant_e4m3_bitexact(M, K, rotate):
+    x = x_bits(M, K, outliers=0.01)
+    x[0, :128] = 0  # an all-zero group
+    if K >= 256:  # amax 448: ties between E4M3 neighbours, a subnormal, a value that rounds to zero
+        x[-1, 128:256] = O.bf16_encode(np.r_[448.0, 1.0625, 1.1875, -2.0 ** -9, 2.0 ** -12, 240.0, np.zeros(122)])
+    q_ref, s_ref = O.act_quant_e4m3_g128(x, rotate)
+    q, s = Q.act_quant_e4m3_g128(dev_bf16(x), rotate)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
 # --------------------------------------------------------------------------
 # Packing
 # --------------------------------------------------------------------------
@@ -69,14 +82,14 @@ def oracle_pack_rtn(fmt, W, had):
     if fmt == Q.I4_G64_BF16:
         q, s = O.quant_i4_g64(W, hadamard=had)
         return O.pack_i4(q), s, None
-    if fmt == Q.FP8_B128_BF16:
+    if fmt in (Q.FP8_B128_BF16, Q.FP8A8_B128_BF16):
         q, s = O.quant_fp8_b128(W, hadamard=had)
         return q, s, None
     raise ValueError(fmt)
 
 
 @pytest.mark.parametrize("had", [0, 1])
-@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 6])
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 6, 7])
 @pytest.mark.parametrize("N,K", [(64, 256), (200, 384), (130, 1024)])
 def test_pack_rtn_bitexact(fmt, had, N, K):
     W = synth.weight_rows(3, f"Wp{N}", K, 0, N)
@@ -340,6 +353,33 @@ def test_prefill_large_tile_count_and_repeat():
     qx, _ = O.act_quant_i8_g128(x, rotate=False)
     acc = Q.qlinear_forward_i8_acc(dev(qx), c.view(torch.int8).reshape(N, K))
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+# --------------------------------------------------------------------------
+# Format 7: E4M3 activations x fp8 weights on the tcgen05 kind::f8f6f4 GEMM (every M)
+# --------------------------------------------------------------------------
+FP8A8_SHAPES = [(1, 64, 128), (5, 130, 256), (16, 333, 640), (17, 64, 256), (129, 257, 384), (200, 384, 512),
+                (300, 130, 1024)]
+
+
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("M,N,K", FP8A8_SHAPES)
+def test_fp8a8_forward_parity(M, N, K, had):
+    (c, s, z), (ch, sh, zh) = make_weights(Q.FP8A8_B128_BF16, N, K, had)
+    x = x_bits(M, K, seed=43, outliers=0.01)
+    y = Q.qlinear_forward(dev_bf16(x), c, s, z, Q.FP8A8_B128_BF16, N, flags=had)
+    ref = O.forward(x, ch, sh, zh, O.FP8A8_B128_BF16, had, N)
+    assert_close(y.cpu().numpy(), ref, f"fp8a8 had {had} {M}x{N}x{K}")
+
+
+def test_fp8a8_large_tile_count_and_repeat():
+    M, N, K = 1290, 3980, 256  # more tiles than SMs, ragged in M and N, called twice
+    (c, s, z), (ch, sh, zh) = make_weights(Q.FP8A8_B128_BF16, N, K, 0, seed=47)
+    x = x_bits(M, K, seed=47)
+    ref = O.forward(x, ch, sh, zh, O.FP8A8_B128_BF16, 0, N)
+    for _ in range(2):
+        y = Q.qlinear_forward(dev_bf16(x), c, s, z, Q.FP8A8_B128_BF16, N)
+        assert_close(y.cpu().numpy(), ref, f"fp8a8 {M}x{N}x{K}")
 
 
 # --------------------------------------------------------------------------
