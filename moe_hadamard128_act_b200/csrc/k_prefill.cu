@@ -18,7 +18,10 @@
 // [128][128 B] and the weight tile [PN][128 B] (128-byte swizzle) into a
 // 4-slot operand ring and bulk-copies each step's 128 activation scales and
 // PN weight scales (fp32, transposed beforehand into contiguous runs) into an
-// 8-slot scale ring; lane 0 of warp 1 issues the MMAs.  Warps 4..19 (112
+// 8-slot scale ring; lane 0 of warp 1 issues the MMAs (for E4M3, lane 0 of warps
+// 1 and 2 issue the even and the odd steps, one accumulator each, so that one
+// thread's barrier waits and its single commit per step hide behind the other's
+// MMAs).  Warps 4..19 (112
 // registers each) are the epilogue: thread i of warp w owns tile row
 // 32 * (w % 4) + i (its tensor-memory lane) and PN / 4 columns.  Per step it
 // reads its accumulators (tcgen05.ld 32x32b, 16 columns at a time, the next
@@ -61,6 +64,7 @@ constexpr int PSTAGES = 4;                // operand ring slots
 constexpr uint32_t kTmemCols = 512;
 constexpr int NBUF = kTmemCols / PN;      // int32 accumulators in tensor memory
 constexpr int SCB = 8;                    // scale ring slots
+constexpr int SR = PSTAGES;               // step-commit ring: a multiple of the operand and accumulator rings
 constexpr int SC_BYTES = (PM + PN) * 4;   // s_x of the tile's rows, then s_w of its columns
 constexpr int kEpiWarps = 16;             // warps 4..19; warps 0..3 (warpgroup 0) drive the pipeline
 constexpr int kPThreads = 32 * (4 + kEpiWarps);
@@ -74,14 +78,15 @@ static_assert(PN % CW == 0 && WGC % CW == 0 && 128 % CW == 0,
               "column chunks start on multiples of CW, so none crosses a 128-row weight block");
 static_assert(PN % 64 == 0 || PN == 160, "tile widths whose column quarters are whole reads");
 static_assert(SCB >= PSTAGES + NBUF, "the scale ring must not throttle the operand ring");
+static_assert(SR % PSTAGES == 0 && SR % NBUF == 0 && NBUF == 2, "one commit per step serves both rings; one accumulator per issuer");
 static_assert((PSTAGES & (PSTAGES - 1)) == 0 && (SCB & (SCB - 1)) == 0, "operand and scale slots from step counters");
 
 // Shared memory (from a 1024-aligned base):
 //   [operand ring][scale ring][mbarriers][tmem address]
 constexpr int SC_OFF = PSTAGES * STAGE_BYTES;
 constexpr int BAR_OFF = SC_OFF + SCB * SC_BYTES;
-constexpr int BAR_FULL = 0, BAR_EMPTY = PSTAGES, BAR_ACCF = 2 * PSTAGES, BAR_ACCE = BAR_ACCF + NBUF,
-              BAR_SCF = BAR_ACCE + NBUF, BAR_SCE = BAR_SCF + SCB, BAR_DRAIN = BAR_SCE + SCB, NBARS = BAR_DRAIN + 1;
+constexpr int BAR_FULL = 0, BAR_STEP = PSTAGES, BAR_ACCE = BAR_STEP + SR, BAR_SCF = BAR_ACCE + NBUF,
+              BAR_SCE = BAR_SCF + SCB, BAR_DRAIN = BAR_SCE + SCB, NBARS = BAR_DRAIN + 1;
 constexpr int MISC_OFF = (BAR_OFF + 8 * NBARS + 15) / 16 * 16;  // tmem address
 constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
 static_assert(STAGE_BYTES % 1024 == 0, "operand slots must stay 1024-byte aligned for the 128-byte swizzle");
@@ -162,6 +167,9 @@ static_assert(128 * kRegsDriver + 32 * kEpiWarps * kRegsEpi <= kPThreads * 96, "
 template <bool ACC, int KIND>
 __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_constant__ PrefillArgs a) {
     static_assert(!ACC || KIND == kKindI8, "the integer group sums exist for int8 only");
+    // Two MMA-issuing threads for E4M3, whose light epilogue leaves the issue as the
+    // limit; one for int8, whose heavier epilogue needs the issue slots instead.
+    constexpr int kIssuers = KIND == kKindE4M3 ? 2 : 1;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -177,19 +185,14 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
     const int total = my_tiles * G;  // steps of this CTA
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < PSTAGES; ++s) {
-            mbar_init(bar(BAR_FULL + s), 1);   // expect_tx
-            mbar_init(bar(BAR_EMPTY + s), 1);  // MMA commit
-        }
-        for (int b = 0; b < NBUF; ++b) {
-            mbar_init(bar(BAR_ACCF + b), 1);          // MMA commit
-            mbar_init(bar(BAR_ACCE + b), kEpiWarps);  // one arrive per epilogue warp
-        }
+        for (int s = 0; s < PSTAGES; ++s) mbar_init(bar(BAR_FULL + s), 1);  // expect_tx
+        for (int s = 0; s < SR; ++s) mbar_init(bar(BAR_STEP + s), 1);       // the step's MMA commit
+        for (int b = 0; b < NBUF; ++b) mbar_init(bar(BAR_ACCE + b), kEpiWarps);  // one arrive per epilogue warp
         for (int b = 0; b < SCB; ++b) {
             mbar_init(bar(BAR_SCF + b), 1);          // expect_tx
             mbar_init(bar(BAR_SCE + b), kEpiWarps);  // one arrive per epilogue warp
         }
-        mbar_init(bar(BAR_DRAIN), 1);
+        mbar_init(bar(BAR_DRAIN), kIssuers);  // one commit per issuing thread
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     if (warp == 1) {
@@ -212,7 +215,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             int m0 = (t % MB) * PM, n0 = (t / MB) * PN;  // tile origin
             for (; k < total; ++k) {
                 const int s = k & (PSTAGES - 1), c = k & (SCB - 1);
-                if (!mbar_wait(bar(BAR_EMPTY + s), ((k / PSTAGES) & 1) ^ 1) ||
+                // the slot's previous operands (step k - PSTAGES) are free once that step's MMAs are done
+                if ((k >= PSTAGES && !mbar_wait(bar(BAR_STEP + (k - PSTAGES) % SR), ((k - PSTAGES) / SR) & 1)) ||
                     (!ACC && !mbar_wait(bar(BAR_SCE + c), ((k / SCB) & 1) ^ 1))) {
                     dead = true;
                     break;
@@ -240,12 +244,12 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             if (!ACC)
                 for (int j = k > SCB ? k - SCB : 0; j < k; ++j)
                     if (!mbar_wait(bar(BAR_SCF + (j & (SCB - 1))), (j / SCB) & 1)) break;
-        } else if (warp == 1 && lane == 0) {  // ---- MMA issuer ----
+        } else if ((warp == 1 || (kIssuers == 2 && warp == 2)) && lane == 0) {  // ---- MMA issuer(s) ----
             // The descriptors of slot s are those of slot 0 plus s * STAGE_BYTES / 16 (the
             // start-address field cannot carry: shared addresses are below 2^18), each
             // K = 32 chunk 2 further.
             const uint64_t da0 = smem_desc_sw128(base), db0 = smem_desc_sw128(base + A_BYTES);
-            for (int k = 0; k < total; ++k) {
+            for (int k = warp - 1; k < total; k += kIssuers) {  // two issuers: b = k % NBUF is this thread's
                 const int s = k & (PSTAGES - 1), b = k % NBUF;
                 if (!mbar_wait(bar(BAR_FULL + s), (k / PSTAGES) & 1) || !mbar_wait(bar(BAR_ACCE + b), (k / NBUF) & 1)) {
                     dead = true;
@@ -257,10 +261,13 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
 #pragma unroll
                 for (int kk = 0; kk < PKB / 32; ++kk)
                     mma_k32<KIND>(d, da0 + so + 2 * kk, db0 + so + 2 * kk, kk ? 1u : 0u);
-                mma_commit(bar(BAR_EMPTY + s));  // operand slot free once these MMAs are done
-                mma_commit(bar(BAR_ACCF + b));   // accumulator ready for the epilogue
+                // One commit per step: its accumulator is ready and its operand slot free.  A
+                // waiter for step j cannot see slot j % SR complete again first: step j + SR
+                // needs that waiter to have moved on (the producer's operands for it, or the
+                // epilogue freeing the accumulator after step j + SR - NBUF).
+                mma_commit(bar(BAR_STEP + k % SR));
             }
-            // Every MMA issued must finish before tensor memory is freed.
+            // Every MMA issued (by both threads) must finish before tensor memory is freed.
             mma_commit(bar(BAR_DRAIN));
             mbar_wait(bar(BAR_DRAIN), 0);
         }
@@ -283,7 +290,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
         int t = blockIdx.x, g = 0;
         for (int k = 0; k < total; ++k) {
             const int b = k % NBUF, c = k & (SCB - 1);
-            if (!mbar_wait(bar(BAR_ACCF + b), (k / NBUF) & 1) ||
+            if (!mbar_wait(bar(BAR_STEP + k % SR), (k / SR) & 1) ||
                 (!ACC && !mbar_wait(bar(BAR_SCF + c), (k / SCB) & 1))) {
                 dead = true;
                 break;
