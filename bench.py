@@ -51,8 +51,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "moe_decode", "moe_decode_t1",
-                                             "moe_prefill"],
+    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "moe_decode",
+                                             "moe_decode_t1", "moe_prefill"],
                    default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
@@ -398,6 +398,24 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                          "peak_source": "MEASURED_PEAKS.json bf16_tflops (x 2 for fp8, nominal ratio)",
                          "mma": "kind::f16 (exact f16 codes x token-scaled f16 activations)"}
             del c, s, y, ws
+        # format 7: the fp8 weights with E4M3 activations (tcgen05 kind::f8f6f4, fp8 rate)
+        c, s, _ = Q.qlinear_pack(Q.FP8A8_B128_BF16, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+        y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+        ws = torch.empty(Q.qlinear_workspace_size(Q.FP8A8_B128_BF16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
+                         device=dev)
+        run = lambda i: Q.qlinear_forward(x, c, s, None, Q.FP8A8_B128_BF16, N_FULL, y=y, ws=ws,  # noqa: E731
+                                          stream=stream)
+        for i in range(3):
+            run(i)
+        t, _ = _traced(Q, run, 10, "prefill")
+        tq, _ = _traced(Q, run, 10, "act_quant")
+        tp, _ = _traced(Q, run, 10, "prefill_prep")
+        tf = ops / (t * 1e-3) / 1e12
+        out["prefill_fp8a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq, "us_scale_prep": 1e3 * tp,
+                                "TFLOPS": tf, "frac_of_fp8_peak": tf / peak_i8,
+                                "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal fp8/bf16 ratio)",
+                                "mma": "kind::f8f6f4 (E4M3 x E4M3, fp32 group sums)"}
+        del c, s, y, ws
     torch.cuda.synchronize()
     return out
 
@@ -407,9 +425,10 @@ def ncu_case(name):
     skinny_w8a8: the W8A8 weight at full size (117 MB codes, two copies so each
     launch misses L2), M = 16, two warm-up forwards then two more; the skinny
     GEMM is launch 1..4 of its name.
-    prefill_w8a8 / prefill_fp8: the prefill workload (M = 2048, N = 21504,
-    K = 5376; about 0.6 GB on the device), four forwards; the tcgen05 GEMM
-    (k_prefill_w8a8 / k_prefill_a16) is launch 1..4 of its name.
+    prefill_w8a8 / prefill_fp8 / prefill_fp8a8: the prefill workload (M = 2048,
+    N = 21504, K = 5376; about 0.6 GB on the device), four forwards; the tcgen05
+    GEMM (k_prefill_w8a8, which also runs format 7, / k_prefill_a16) is launch
+    1..4 of its name.
     moe_decode / moe_decode_t1 / moe_prefill: the MoE gate_up experts (128 x
     [1408, 2816] int8 g128 bf16, Hadamard domain; about 0.5 GB), top-8 routing
     of T = 16 / 1 / 2048 tokens, four calls of moe_gate_up (activation
@@ -443,7 +462,7 @@ def ncu_case(name):
         print(f"ncu case {name} done")
         return
     if name.startswith("prefill"):
-        fmt = Q.I8A8_G128_BF16 if name == "prefill_w8a8" else Q.FP8_B128_BF16
+        fmt = {"prefill_w8a8": Q.I8A8_G128_BF16, "prefill_fp8a8": Q.FP8A8_B128_BF16}.get(name, Q.FP8_B128_BF16)
         d = synth.prefill(M=2048)
         c, s, _ = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
         x = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).to(dev)
