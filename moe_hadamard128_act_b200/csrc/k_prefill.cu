@@ -45,6 +45,14 @@
 // whole 128-row block the promotion is one FMA per element with s_x * s_w taken
 // once per 16 columns.
 //
+// A finished tile leaves through shared memory: each epilogue warp stages its
+// 32 rows x PN / 4 columns in two halves in a private 3 KB buffer and one lane
+// writes each half with a TMA tensor store (rows and columns past the matrix are
+// clipped by the store).  Stored straight from registers, every warp store
+// instruction would touch 32 rows, 16 bytes each, and at this tile rate those
+// scattered writes cost about a sixth of the kernel's time.  Rows of y that are
+// not 16-byte multiples (N % 4 != 0) take plain stores.
+//
 // All waits are bounded (200 ms); on a timeout the CTA sets
 // QL_DEVERR_TIMEOUT and winds down without leaving tensor memory allocated,
 // MMAs running or copies in flight.
@@ -60,11 +68,14 @@ constexpr int PKB = 128;                  // K bytes per group
 constexpr int A_BYTES = PM * PKB;         // 16 KB
 constexpr int B_BYTES = PN * PKB;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int PSTAGES = 4;                // operand ring slots
+#ifndef QL_PF_STAGES
+#define QL_PF_STAGES 4
+#endif
+constexpr int PSTAGES = QL_PF_STAGES;     // operand ring slots
 constexpr uint32_t kTmemCols = 512;
 constexpr int NBUF = kTmemCols / PN;      // int32 accumulators in tensor memory
 constexpr int SCB = 8;                    // scale ring slots
-constexpr int SR = PSTAGES;               // step-commit ring: a multiple of the operand and accumulator rings
+constexpr int SR = PSTAGES;               // step-commit ring: at least as long as the operand and accumulator rings
 constexpr int SC_BYTES = (PM + PN) * 4;   // s_x of the tile's rows, then s_w of its columns
 constexpr int kEpiWarps = 16;             // warps 4..19; warps 0..3 (warpgroup 0) drive the pipeline
 constexpr int kPThreads = 32 * (4 + kEpiWarps);
@@ -78,8 +89,8 @@ static_assert(PN % CW == 0 && WGC % CW == 0 && 128 % CW == 0,
               "column chunks start on multiples of CW, so none crosses a 128-row weight block");
 static_assert(PN % 64 == 0 || PN == 160, "tile widths whose column quarters are whole reads");
 static_assert(SCB >= PSTAGES + NBUF, "the scale ring must not throttle the operand ring");
-static_assert(SR % PSTAGES == 0 && SR % NBUF == 0 && NBUF == 2, "one commit per step serves both rings; one accumulator per issuer");
-static_assert((PSTAGES & (PSTAGES - 1)) == 0 && (SCB & (SCB - 1)) == 0, "operand and scale slots from step counters");
+static_assert(SR >= PSTAGES && SR >= NBUF && NBUF % 2 == 0, "one commit per step serves both rings; each issuer its own accumulators");
+static_assert((SCB & (SCB - 1)) == 0, "scale slots from step counters");
 
 // Shared memory (from a 1024-aligned base):
 //   [operand ring][scale ring][mbarriers][tmem address]
@@ -88,10 +99,19 @@ constexpr int BAR_OFF = SC_OFF + SCB * SC_BYTES;
 constexpr int BAR_FULL = 0, BAR_STEP = PSTAGES, BAR_ACCE = BAR_STEP + SR, BAR_SCF = BAR_ACCE + NBUF,
               BAR_SCE = BAR_SCF + SCB, BAR_DRAIN = BAR_SCE + SCB, NBARS = BAR_DRAIN + 1;
 constexpr int MISC_OFF = (BAR_OFF + 8 * NBARS + 15) / 16 * 16;  // tmem address
-constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+// Output staging: each epilogue warp writes its 32 rows x WGC columns of a
+// finished tile in two halves of YH columns through a private buffer, and one
+// lane stores each half with a TMA tensor store.
+constexpr int YH = WGC / 2;
+constexpr int Y_WARP_BYTES = 32 * YH * 4;
+constexpr int Y_OFF = (MISC_OFF + 16 + 1023) / 1024 * 1024;
+constexpr int SMEM_BYTES = Y_OFF + kEpiWarps * Y_WARP_BYTES + 1024;
+static_assert((YH * 4) % 16 == 0 && YH % 4 == 0 && Y_WARP_BYTES % 128 == 0,
+              "TMA store boxes: 16-byte rows, 128-byte aligned staging");
 static_assert(STAGE_BYTES % 1024 == 0, "operand slots must stay 1024-byte aligned for the 128-byte swizzle");
 static_assert(SC_OFF % 16 == 0 && SC_BYTES % 16 == 0, "scale slots take 16-byte bulk copies and loads");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+static_assert(Y_OFF >= MISC_OFF + 16, "staging after the tensor-memory address");
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     // K-major, 128-byte swizzle: 8-row atoms 1024 bytes apart (SBO), version 1.
@@ -126,6 +146,22 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+// Bulk tensor store of a staged box (global <- shared), tracked by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(tmap), "r"(x),
+                 "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// This thread's committed stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// ... and have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+// Makes this thread's shared-memory writes visible to the TMA (async proxy).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void sts128(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
@@ -146,15 +182,25 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
                  :                                                                                           \
                  : "memory")
 
+// The registers of a read issued before the last wait: ties their uses to after it
+// (volatile asm statements keep their order).
+#define QL_TMEM_AFTER_WAIT16(v)                                                                          \
+    asm volatile(""                                                                                     \
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),  \
+                   "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), \
+                   "+r"(v[14]), "+r"(v[15]))
+
 struct PrefillArgs {
     CUtensorMap tmA;    // int8 activations [M][K], box [128 rows][128 B]
-    CUtensorMap tmB;    // int8 weights [N][K], box [256 rows][128 B]
+    CUtensorMap tmB;    // int8 weights [N][K], box [PN rows][128 B]
+    CUtensorMap tmY;    // y as bytes [M][4 N], row pitch 4 ldy, box [32 rows][4 YH B] (when ytma)
     const float* sxT;   // [G][Mp] activation scales (ACC: unused)
     const float* swT;   // [G][Np] weight scales as fp32 (ACC: unused)
     float* y;           // [M][ldy]
     int32_t* acc;       // group sums [M][N][G] (check path only)
     unsigned* err;
     int M, N, G, Mp, Np;
+    int ytma;           // y is written by TMA stores (16-byte aligned rows)
     long long ldy;
 };
 
@@ -214,7 +260,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             int g = 0, t = blockIdx.x, k = 0;
             int m0 = (t % MB) * PM, n0 = (t / MB) * PN;  // tile origin
             for (; k < total; ++k) {
-                const int s = k & (PSTAGES - 1), c = k & (SCB - 1);
+                const int s = k % PSTAGES, c = k & (SCB - 1);
                 // the slot's previous operands (step k - PSTAGES) are free once that step's MMAs are done
                 if ((k >= PSTAGES && !mbar_wait(bar(BAR_STEP + (k - PSTAGES) % SR), ((k - PSTAGES) / SR) & 1)) ||
                     (!ACC && !mbar_wait(bar(BAR_SCE + c), ((k / SCB) & 1) ^ 1))) {
@@ -240,7 +286,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             }
             // Copies still in flight must land before the CTA's shared memory is released.
             for (int j = k > PSTAGES ? k - PSTAGES : 0; j < k; ++j)
-                if (!mbar_wait(bar(BAR_FULL + (j & (PSTAGES - 1))), (j / PSTAGES) & 1)) break;
+                if (!mbar_wait(bar(BAR_FULL + j % PSTAGES), (j / PSTAGES) & 1)) break;
             if (!ACC)
                 for (int j = k > SCB ? k - SCB : 0; j < k; ++j)
                     if (!mbar_wait(bar(BAR_SCF + (j & (SCB - 1))), (j / SCB) & 1)) break;
@@ -250,7 +296,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             // K = 32 chunk 2 further.
             const uint64_t da0 = smem_desc_sw128(base), db0 = smem_desc_sw128(base + A_BYTES);
             for (int k = warp - 1; k < total; k += kIssuers) {  // two issuers: b = k % NBUF is this thread's
-                const int s = k & (PSTAGES - 1), b = k % NBUF;
+                const int s = k % PSTAGES, b = k % NBUF;
                 if (!mbar_wait(bar(BAR_FULL + s), (k / PSTAGES) & 1) || !mbar_wait(bar(BAR_ACCE + b), (k / NBUF) & 1)) {
                     dead = true;
                     break;
@@ -307,6 +353,41 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 sxr = __int_as_float(__float_as_int(scp[row]) & ~3);
                 kb = -sxr * 12582912.0f;
             }
+            if constexpr (!ACC && KIND == kKindE4M3) {
+                // All of this thread's columns are read at once and the accumulator goes
+                // back to the MMAs before the math: a light promotion leaves the read
+                // latency, not the arithmetic, on the accumulator's round trip.
+                uint32_t v[WGC];
+#pragma unroll
+                for (int h = 0; h < NCH; ++h) QL_TMEM_LD16(taddr + h * CW, (v + h * CW));
+                QL_TMEM_WAIT16(v);
+#pragma unroll
+                for (int h = 1; h < NCH; ++h) QL_TMEM_AFTER_WAIT16((v + h * CW));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_ACCE + b));
+                // fp8 weights scale whole 128-row blocks, and a 16-column chunk starts on a
+                // multiple of 16 weight rows, so it never crosses a block: one s_x * s_w per
+                // chunk, then one FMA per element (half packed, half scalar: both FMA pipes).
+#pragma unroll
+                for (int h = 0; h < NCH; ++h) {
+                    const float p = sxr * scp[PM + tcol + h * CW];
+                    const float2 p2 = make_float2(p, p);
+#pragma unroll
+                    for (int q = 0; q < CW / 4; ++q) {
+                        const uint32_t* const cu = v + h * CW + 4 * q;
+                        float* const yq = yr + h * CW + 4 * q;
+                        const float2 u = __ffma2_rn(p2, make_float2(__uint_as_float(cu[0]), __uint_as_float(cu[1])),
+                                                    make_float2(yq[0], yq[1]));
+                        yq[0] = u.x;
+                        yq[1] = u.y;
+                        yq[2] = fmaf(p, __uint_as_float(cu[2]), yq[2]);
+                        yq[3] = fmaf(p, __uint_as_float(cu[3]), yq[3]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_SCE + c));
+            } else {
             const uint32_t mg = KIND == kKindE4M3 ? 0u : kMagic;
             const float2 sx2 = make_float2(sxr, sxr), kb2 = make_float2(kb, kb);
             uint32_t v[2][CW];
@@ -322,23 +403,6 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
 #pragma unroll
                         for (int i = 0; i < CW; ++i)
                             if (n0 + i < a.N) a.acc[((long long)m * a.N + n0 + i) * G + g] = (int)cur[i];
-                } else if constexpr (KIND == kKindE4M3) {
-                    // fp8 weights scale whole 128-row blocks, and a 16-column chunk starts on a
-                    // multiple of 16 weight rows, so it never crosses a block: one s_x * s_w per
-                    // chunk, then one FMA per element (half packed, half scalar: both FMA pipes).
-                    const float p = sxr * scp[PM + tcol + h * CW];
-                    const float2 p2 = make_float2(p, p);
-#pragma unroll
-                    for (int q = 0; q < CW / 4; ++q) {
-                        float* const yq = yr + h * CW + 4 * q;
-                        const float2 u = __ffma2_rn(p2, make_float2(__uint_as_float(cur[4 * q]),
-                                                                    __uint_as_float(cur[4 * q + 1])),
-                                                    make_float2(yq[0], yq[1]));
-                        yq[0] = u.x;
-                        yq[1] = u.y;
-                        yq[2] = fmaf(p, __uint_as_float(cur[4 * q + 2]), yq[2]);
-                        yq[3] = fmaf(p, __uint_as_float(cur[4 * q + 3]), yq[3]);
-                    }
                 } else {
                     // Weight scales read in place (volatile loads stay in their chunk instead of being
                     // hoisted, which would cost registers).
@@ -368,9 +432,31 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 mbar_arrive(bar(BAR_ACCE + b));
                 if (!ACC) mbar_arrive(bar(BAR_SCE + c));
             }
+            }
 
             if (++g == G) {  // tile done: this thread's WGC columns of its row of y
-                if (!ACC) {
+                if (!ACC && a.ytma) {
+                    const int r0 = (t % MB) * PM + sub * 32, n0 = (t / MB) * PN + tcol;
+                    const uint32_t yb = base + Y_OFF + (uint32_t)(warp - 4) * Y_WARP_BYTES;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (lane == 0) bulk_wait_read();  // the buffer's previous store has read it
+                        __syncwarp();
+#pragma unroll
+                        for (int q = 0; q < YH / 4; ++q)
+                            sts128(yb + (uint32_t)lane * (YH * 4) + 16 * q, yr[hh * YH + 4 * q], yr[hh * YH + 4 * q + 1],
+                                   yr[hh * YH + 4 * q + 2], yr[hh * YH + 4 * q + 3]);
+                        fence_async_smem();
+                        __syncwarp();
+                        // Rows past M and columns past N are clipped by the store; boxes wholly outside are skipped.
+                        if (lane == 0 && r0 < a.M && n0 + hh * YH < a.N) {
+                            tma_store_2d(&a.tmY, yb, (n0 + hh * YH) * 4, r0);
+                            bulk_commit();
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < WGC; ++i) yr[i] = 0.0f;
+                } else if (!ACC) {
                     const int m = (t % MB) * PM + row, n0 = (t / MB) * PN + tcol;
                     if (m < a.M) {
                         float* yrow = a.y + (long long)m * a.ldy + n0;
@@ -394,6 +480,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
         }
     }
     if (dead) atomicOr(a.err, (unsigned)QL_DEVERR_TIMEOUT);
+    // Outstanding output stores finish before the CTA (and its staging buffers) goes.
+    if (!ACC && a.ytma && warp >= 4 && lane == 0) bulk_wait_all();
 
     tc_fence_before();
     __syncthreads();
@@ -468,6 +556,12 @@ cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t
     a.Mp = prefill_pad_m(M);
     a.Np = prefill_pad_n(N);
     a.ldy = ldy;
+    a.ytma = 0;
+    if (!acc && ldy % 4 == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0) {
+        if ((e = make_tmap_2d(y, M, 4LL * N, 4 * ldy, YH * 4, 32, CU_TENSOR_MAP_SWIZZLE_NONE, &a.tmY)) != cudaSuccess)
+            return e;
+        a.ytma = 1;
+    }
     const int tiles = ((M + PM - 1) / PM) * ((N + PN - 1) / PN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
     static bool attr_set[64] = {};

@@ -306,7 +306,9 @@ def test_moe_duplicate_expert_in_token():
 # --------------------------------------------------------------------------
 # Prefill (tcgen05) path: M >= 17 for W8A8
 # --------------------------------------------------------------------------
-PREFILL_SHAPES = [(17, 64, 128), (128, 128, 256), (200, 384, 512), (300, 130, 1024), (129, 257, 384)]
+# N % 4 == 0: y is written by TMA stores (N = 388: a ragged last tile, boxes clipped or skipped);
+# N = 130 / 257: plain stores
+PREFILL_SHAPES = [(17, 64, 128), (128, 128, 256), (200, 384, 512), (300, 130, 1024), (129, 257, 384), (150, 388, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
@@ -339,7 +341,7 @@ def test_prefill_forward_parity(M, N, K, had):
 
 
 def test_prefill_large_tile_count_and_repeat():
-    # 11 x 16 = 176 output tiles of 128 x 256, more than the 148 SMs, so
+    # 11 x 21 = 231 output tiles of 128 x 192, more than the 148 SMs, so
     # persistent CTAs walk two tiles each; ragged in both M and N; called twice
     M, N, K = 1290, 3980, 256
     x = x_bits(M, K, seed=41)
@@ -359,7 +361,7 @@ def test_prefill_large_tile_count_and_repeat():
 # Format 7: E4M3 activations x fp8 weights on the tcgen05 kind::f8f6f4 GEMM (every M)
 # --------------------------------------------------------------------------
 FP8A8_SHAPES = [(1, 64, 128), (5, 130, 256), (16, 333, 640), (17, 64, 256), (129, 257, 384), (200, 384, 512),
-                (300, 130, 1024)]
+                (300, 130, 1024), (150, 388, 256)]
 
 
 @pytest.mark.parametrize("had", [0, 1])
