@@ -69,7 +69,7 @@ constexpr int A_BYTES = PM * PKB;         // 16 KB
 constexpr int B_BYTES = PN * PKB;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 #ifndef QL_PF_STAGES
-#define QL_PF_STAGES 4
+#define QL_PF_STAGES (QL_PF_N > 192 ? 3 : 4)
 #endif
 constexpr int PSTAGES = QL_PF_STAGES;     // operand ring slots
 constexpr uint32_t kTmemCols = 512;
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 sxr = __int_as_float(__float_as_int(scp[row]) & ~3);
                 kb = -sxr * 12582912.0f;
             }
-            if constexpr (!ACC && KIND == kKindE4M3) {
+            if constexpr (!ACC && KIND == kKindE4M3 && WGC <= 48) {
                 // All of this thread's columns are read at once and the accumulator goes
                 // back to the MMAs before the math: a light promotion leaves the read
                 // latency, not the arithmetic, on the accumulator's round trip.
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(BAR_SCE + c));
             } else {
-            const uint32_t mg = KIND == kKindE4M3 ? 0u : kMagic;
+            const uint32_t mg = kMagic;
             const float2 sx2 = make_float2(sxr, sxr), kb2 = make_float2(kb, kb);
             uint32_t v[2][CW];
             QL_TMEM_LD16(taddr, v[0]);
@@ -403,6 +403,20 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
 #pragma unroll
                         for (int i = 0; i < CW; ++i)
                             if (n0 + i < a.N) a.acc[((long long)m * a.N + n0 + i) * G + g] = (int)cur[i];
+                } else if constexpr (KIND == kKindE4M3) {  // wide tiles: one s_x * s_w per chunk, as above
+                    const float p = sxr * scp[PM + tcol + h * CW];
+                    const float2 p2 = make_float2(p, p);
+#pragma unroll
+                    for (int q = 0; q < CW / 4; ++q) {
+                        float* const yq = yr + h * CW + 4 * q;
+                        const float2 u = __ffma2_rn(p2, make_float2(__uint_as_float(cur[4 * q]),
+                                                                    __uint_as_float(cur[4 * q + 1])),
+                                                    make_float2(yq[0], yq[1]));
+                        yq[0] = u.x;
+                        yq[1] = u.y;
+                        yq[2] = fmaf(p, __uint_as_float(cur[4 * q + 2]), yq[2]);
+                        yq[3] = fmaf(p, __uint_as_float(cur[4 * q + 3]), yq[3]);
+                    }
                 } else {
                     // Weight scales read in place (volatile loads stay in their chunk instead of being
                     // hoisted, which would cost registers).
