@@ -79,6 +79,8 @@ def lib():
             "qo_act_quant_e4m3_g128": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
             "qo_act_quant_e4m3_group": [_c_p, _c_p, _c_p],
             "qo_quant_i8_g128": [_c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p],
+            "qo_scale_search_group": [_c_p, _c_i, _c_p, _c_p, _c_p],
+            "qo_quant_i8_g128_search": [_c_p, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p],
             "qo_quant_i4_g64": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
             "qo_quant_fp8_b128": [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p],
             "qo_pack_i4": [_c_p, _c_i, _c_i, _c_p],
@@ -210,6 +212,27 @@ def quant_i8_g128(W: np.ndarray, hadamard: bool = False, scale_f16: bool = False
     s = np.empty((N, K // 128), np.uint16)
     lib().qo_quant_i8_g128(_p(W), N, K, HADAMARD if hadamard else 0, int(scale_f16), _p(q), _p(s))
     return q, s
+
+
+def scale_search_group(v, scale_f16: bool = False):
+    """One fp32 group of 128 through the scale search: (codes, scale bits, chosen candidate i)."""
+    v = _c(v, np.float32)
+    q = np.empty(128, np.int8)
+    s = np.empty(1, np.uint16)
+    i = np.empty(1, np.int32)
+    lib().qo_scale_search_group(_p(v), int(scale_f16), _p(q), _p(s), _p(i))
+    return q, s[0], int(i[0])
+
+
+def quant_i8_g128_search(W: np.ndarray, hadamard: bool = False, scale_f16: bool = False):
+    """int8 g128 with the scale search: (codes [N, K], scale bits [N, K/128], chosen i [N, K/128])."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    q = np.empty((N, K), np.int8)
+    s = np.empty((N, K // 128), np.uint16)
+    ci = np.empty((N, K // 128), np.int32)
+    lib().qo_quant_i8_g128_search(_p(W), N, K, HADAMARD if hadamard else 0, int(scale_f16), _p(q), _p(s), _p(ci))
+    return q, s, ci
 
 
 def quant_i4_g64(W: np.ndarray, hadamard: bool = False):

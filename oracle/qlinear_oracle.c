@@ -366,6 +366,83 @@ void qo_quant_i8_g128(const float* W, int N, int K, int flags, int scale_f16, in
     }
 }
 
+/* int8 group 128 with a scale search ("round to nearest with a scale search",
+ * rule=search, in the "gemma4-26b-a4b-dflash-i8" README's "Weights" table and
+ * recipe).  The card names the search but not its candidates or its measure;
+ * the reading taken here:
+ *   r = fp32(amax / 127) (the round-to-nearest scale before rounding);
+ *   candidate i = 0..20: raw_i = fp32(r * c_i), c_i = fp32((100 - i) / 100),
+ *     s_i = scale_fmt(raw_i), codes q = clamp(rne(fp32(w / s_i)), -127, 127)
+ *     (s_i == 0: every code 0), exactly as round to nearest does with s_i;
+ *   error_i = sum over the group, k = 0..127 in order, of (w_k - s_i * q_k)^2,
+ *     each product, difference and sum rounded to fp64 (no fused operations);
+ *   the group keeps the candidate with the smallest error, the smaller i on a tie.
+ * c_0 = 1, so candidate 0 is the round-to-nearest result and the search never
+ * does worse than it.  v is the group as the quantiser sees it (rotated when
+ * the weights live in the Hadamard domain); *i_out (may be NULL) gets the
+ * chosen i. */
+void qo_scale_search_group(const float* v, int scale_f16, int8_t* q, uint16_t* s_out, int* i_out)
+{
+    float amax = 0.0f;
+    for (int k = 0; k < 128; ++k)
+        if (fabsf(v[k]) > amax) amax = fabsf(v[k]);
+    volatile float r = amax / 127.0f;
+    int best = 0;
+    double best_err = 0.0;
+    uint16_t best_s = 0;
+    for (int i = 0; i <= 20; ++i) {
+        volatile float c = (float)(100 - i) / 100.0f;
+        volatile float raw = r * c;
+        uint16_t sb = scale_f16 ? qo_f16_encode(raw) : qo_bf16_encode(raw);
+        float sf = (float)(scale_f16 ? qo_f16_decode(sb) : qo_bf16_decode(sb));
+        double err = 0.0;
+        for (int k = 0; k < 128; ++k) {
+            int code = 0;
+            if (sf != 0.0f) {
+                volatile float t = v[k] / sf;
+                code = clampi(rint_even_f32(t), -127, 127);
+            }
+            double d = (double)v[k] - (double)sf * (double)code;
+            err = err + d * d;
+        }
+        if (i == 0 || err < best_err) {
+            best = i;
+            best_err = err;
+            best_s = sb;
+        }
+    }
+    float sf = (float)(scale_f16 ? qo_f16_decode(best_s) : qo_bf16_decode(best_s));
+    for (int k = 0; k < 128; ++k) {
+        int code = 0;
+        if (sf != 0.0f) {
+            volatile float t = v[k] / sf;
+            code = clampi(rint_even_f32(t), -127, 127);
+        }
+        q[k] = (int8_t)code;
+    }
+    *s_out = best_s;
+    if (i_out) *i_out = best;
+}
+
+/* The scale search over a whole [N, K] weight (rows rotated first when
+ * QO_HADAMARD is set); chosen (may be NULL) gets each group's i, [N][K/128]. */
+void qo_quant_i8_g128_search(const float* W, int N, int K, int flags, int scale_f16, int8_t* q, uint16_t* s,
+                             int32_t* chosen)
+{
+    int G = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        float* row = (float*)malloc(sizeof(float) * (size_t)K);
+        weight_row(W, K, n, flags, row);
+        for (int g = 0; g < G; ++g) {
+            int ci;
+            qo_scale_search_group(row + g * 128, scale_f16, q + (size_t)n * K + g * 128, s + (size_t)n * G + g, &ci);
+            if (chosen) chosen[(size_t)n * G + g] = ci;
+        }
+        free(row);
+    }
+}
+
 /* Symmetric int4, group 64: s = bf16(fp32(amax / 7)),
  * q = clamp(round_half_even(fp32(w / s)), -8, 7); s == 0 gives q = 0. */
 void qo_quant_i4_g64(const float* W, int N, int K, int flags, int8_t* q, uint16_t* s)

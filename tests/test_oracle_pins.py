@@ -278,6 +278,117 @@ def test_quant_i8_hadamard_domain_reproduces_product():
     assert np.max(np.abs(back - W)) < 0.02 * 4 / 127 * 4
 
 
+# --------------------------------------------------------------------------
+# Scale search (rule=search): candidates s_i from fp32(amax/127) * (100 - i)/100,
+# i = 0..20, the smallest squared error wins, the smaller i on a tie
+# --------------------------------------------------------------------------
+def _torch_scale(vals32: np.ndarray, f16: bool) -> np.ndarray:
+    """scale_fmt round-to-nearest-even by torch / numpy, independent of the oracle's codecs."""
+    if f16:
+        return vals32.astype(np.float16).astype(np.float64)
+    return torch.from_numpy(vals32.astype(np.float32)).to(torch.bfloat16).float().numpy().astype(np.float64)
+
+
+def _exact_err(v: np.ndarray, sf: float, q: np.ndarray):
+    from fractions import Fraction
+    fs = Fraction(sf)
+    return sum((Fraction(float(w)) - fs * int(c)) ** 2 for w, c in zip(v, q))
+
+
+def _search_groups():
+    rng = np.random.default_rng(7)  # its own stream: the picks below do not depend on test order
+    groups = []
+    for _ in range(20):
+        groups.append((rng.standard_normal(128) * 0.02).astype(np.float32))
+        groups.append((rng.laplace(size=128) * 0.03).astype(np.float32))
+        groups.append((rng.standard_t(3, size=128) * 0.01).astype(np.float32))
+    return groups
+
+
+@pytest.mark.parametrize("f16", [False, True])
+def test_scale_search_brute_force_exact_errors(f16):
+    # every candidate rebuilt here (numpy fp32 arithmetic, torch / numpy scale rounding) and its
+    # squared error summed exactly in rationals: the oracle's pick has the least error, the
+    # smaller i on a tie, and its codes and scale are that candidate's
+    picked_nonzero = 0
+    for v in _search_groups():
+        q, sb, i = O.scale_search_group(v, f16)
+        amax = np.float32(np.max(np.abs(v)))
+        r = np.float32(amax / np.float32(127))
+        errs, cands = [], []
+        for c in range(21):
+            ci = np.float32(np.float32(100 - c) / np.float32(100))
+            sf = float(_torch_scale(np.array([np.float32(r * ci)]), f16)[0])
+            qc = (np.zeros(128, np.int64) if sf == 0 else
+                  np.clip(np.rint((v / np.float32(sf)).astype(np.float32)), -127, 127).astype(np.int64))
+            errs.append(_exact_err(v, sf, qc))
+            cands.append((sf, qc))
+        best = min(errs)
+        want = errs.index(best)
+        got_err = errs[i]
+        # the oracle sums in fp64: it may only differ from the exact pick on a near-tie
+        assert got_err <= best * (1 + 1e-12) + 0
+        if got_err != best:
+            assert i > want
+        sd = float(O.f16_decode(np.array([sb]))[0] if f16 else O.bf16_decode(np.array([sb]))[0])
+        assert sd == cands[i][0]
+        assert np.array_equal(q.astype(np.int64), cands[i][1])
+        picked_nonzero += i > 0
+    assert picked_nonzero >= 2  # some groups do take a smaller scale
+
+
+def test_scale_search_never_worse_than_rtn_and_candidate_zero_is_rtn():
+    W = np.stack(_search_groups()).astype(np.float32)
+    for f16 in (False, True):
+        q0, s0 = O.quant_i8_g128(W, scale_f16=f16)
+        dec0 = O.f16_decode(s0) if f16 else O.bf16_decode(s0)
+        for n, v in enumerate(W):
+            q, sb, i = O.scale_search_group(v, f16)
+            sd = float(O.f16_decode(np.array([sb]))[0] if f16 else O.bf16_decode(np.array([sb]))[0])
+            e_search = _exact_err(v, sd, q)
+            e_rtn = _exact_err(v, float(dec0[n, 0]), q0[n])
+            assert e_search <= e_rtn * (1 + 1e-12)
+            if i == 0:
+                assert sb == s0[n, 0] and np.array_equal(q, q0[n])
+
+
+def test_scale_search_closed_forms_and_invariances():
+    # all-zero group: scale 0, codes 0, candidate 0
+    q, sb, i = O.scale_search_group(np.zeros(128, np.float32))
+    assert sb == 0 and not q.any() and i == 0
+    # a group already on the round-to-nearest grid (s = 2^-10 exactly, codes up to 127): zero error
+    # at candidate 0, while every smaller scale clips the 127s
+    n = RNG.integers(-127, 128, 128)
+    n[5] = 127
+    v = (n * 2.0 ** -10).astype(np.float32)
+    q, sb, i = O.scale_search_group(v)
+    assert i == 0 and float(O.bf16_decode(np.array([sb]))[0]) == 2.0 ** -10 and np.array_equal(q, n)
+    # sign and power-of-two scaling change nothing but the sign of the codes and the scale's exponent
+    for v in _search_groups()[:8]:
+        q, sb, i = O.scale_search_group(v)
+        sd = float(O.bf16_decode(np.array([sb]))[0])
+        qn, sbn, iN = O.scale_search_group(-v)
+        assert iN == i and sbn == sb and np.array_equal(qn, -q)
+        for e in (-3, 5):
+            q2, sb2, i2 = O.scale_search_group((v * np.float32(2.0 ** e)).astype(np.float32))
+            assert i2 == i and np.array_equal(q2, q)
+            assert float(O.bf16_decode(np.array([sb2]))[0]) == sd * 2.0 ** e
+
+
+def test_quant_i8_search_matrix_is_groupwise_on_rotated_rows():
+    W = (RNG.standard_normal((3, 384)) * 0.02).astype(np.float32)
+    W[1, 200] = 0.5  # an outlier in one group
+    for had in (False, True):
+        q, s, ci = O.quant_i8_g128_search(W, hadamard=had)
+        for n in range(3):
+            for g in range(3):
+                v = W[n, g * 128:(g + 1) * 128]
+                if had:
+                    v = O.fwht128_spec_f32(v)
+                qg, sg, ig = O.scale_search_group(v)
+                assert np.array_equal(q[n, g * 128:(g + 1) * 128], qg) and s[n, g] == sg and ci[n, g] == ig
+
+
 def test_quant_fp8_block_rule():
     N, K = 200, 256  # a ragged last row block (72 rows)
     W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
