@@ -89,7 +89,10 @@ typedef enum {
     QL_FP8A8_B128_BF16 = 7
 } ql_fmt;
 
-enum { QL_HADAMARD = 1 };
+/* QL_SCALE_SEARCH: a rule for qlinear_pack's mode (a), int8 formats (1, 2, 3)
+ * only -- see qlinear_pack.  The packed result has the same layout, so other
+ * calls accept the flag and ignore it. */
+enum { QL_HADAMARD = 1, QL_SCALE_SEARCH = 2 };
 
 /* Bits of the device error word. */
 enum { QL_DEVERR_EXPERT_ID = 1, QL_DEVERR_CODE_RANGE = 2, QL_DEVERR_TIMEOUT = 4 };
@@ -116,10 +119,20 @@ int qlinear_packed_sizes(int fmt, int N, int K, size_t* codes_bytes, size_t* sca
  *      128x128 block, s = bf16(fp32(amax/448)), q = e4m3_rne_satfinite(w/s).
  *      An all-zero group gets s = 0 and q = 0.  int5 is rejected
  *      (QL_EUNSUPPORTED): its codes come from a calibrated quantiser.
+ *      With QL_SCALE_SEARCH (int8 formats; others QL_EUNSUPPORTED) each group
+ *      takes the best of 21 scales instead ("round to nearest with a scale
+ *      search", rule=search, in the "gemma4-26b-a4b-dflash-i8" README; the
+ *      card names the search, the candidates and measure are a reading):
+ *      r = fp32(amax/127); for i = 0..20, s_i = scale_fmt(fp32(r *
+ *      fp32((100 - i)/100))), codes by the round-to-nearest rule with s_i, and
+ *      the squared error sum_k (w_k - s_i q_k)^2 over k = 0..127 in order, each
+ *      operation rounded to fp64; the least error wins, the smaller i on a
+ *      tie (i = 0 is the plain round-to-nearest result).
  *  (b) codes_in != NULL: pack given codes.  codes_in is int8 [N, K] (uint8 for
  *      int5, e4m3 bytes for fp8), scales_in the scales in the output layout,
  *      zeros_in the int5 zero points; they are copied / bit-packed.  A code
  *      outside its format's range is packed as 0 and flags QL_DEVERR_CODE_RANGE.
+ *      QL_SCALE_SEARCH with given codes is QL_EINVAL.
  * Outputs: codes_out, scales_out and (int5) zeros_out, sized by
  * qlinear_packed_sizes. */
 int qlinear_pack(const float* W, const void* codes_in, const void* scales_in, const uint8_t* zeros_in, int fmt,

@@ -5,7 +5,8 @@
 //
 // Round-to-nearest quantisers: one warp per (row, 128 columns), 4 fp32 per
 // lane (16-byte loads), optional in-register Walsh-Hadamard transform, the
-// group max by shuffles.  FP8 takes one CTA per 128x128 block, whose rotated
+// group max by shuffles; the int8 scale search scores its 21 candidate scales
+// on 21 lanes of the same warp.  FP8 takes one CTA per 128x128 block, whose rotated
 // values are staged in shared memory for the block max.  Packers of given
 // codes run one thread per 8 codes.
 #include "ql_device.cuh"
@@ -56,6 +57,83 @@ __global__ void __launch_bounds__(256) k_rtn_i8(const float* W, int N, int K, in
         }
         *reinterpret_cast<uint32_t*>(q + off) = packed;
         if (lane == 0) s[u] = sb;
+    }
+}
+
+// int8, group 128, with the scale search of the int8 experts' recipe (rule=search, "round to
+// nearest with a scale search"): candidate i = 0..20 quantises the group by round to nearest
+// with s_i = scale_fmt(fp32(fp32(amax / 127) * fp32((100 - i) / 100))) and scores it by its
+// squared error, summed over k = 0..127 in order in fp64 with every product, difference and sum
+// rounded on its own; the least error wins, the smaller i on a tie.  One warp per group: lane i
+// scores candidate i over the group staged in shared memory (its sum is sequential, so the
+// result does not depend on how the work is split), then every lane writes its four codes.
+template <bool kF16Scale>
+__global__ void __launch_bounds__(256) k_search_i8(const float* W, int N, int K, int hadamard, int8_t* q,
+                                                   uint16_t* s) {
+    __shared__ float grp[8][128];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const long long G = K / 128;
+    const long long nw = (long long)gridDim.x * 8;
+    for (long long u = (long long)blockIdx.x * 8 + wib; u < (long long)N * G; u += nw) {
+        const long long off = (u / G) * K + (u % G) * 128 + 4 * lane;
+        float v[4];
+        load4_f32(W + off, v);
+        if (hadamard) fwht128_warp(v, lane);
+        float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+        amax = warp_max(amax);
+        *reinterpret_cast<float4*>(&grp[wib][4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
+        __syncwarp();
+        const float r = __fdiv_rn(amax, 127.0f);
+        double err = INFINITY;
+        float sf_i = 0.0f;
+        uint32_t sb_i = 0;
+        if (lane <= 20) {
+            const float raw = __fmul_rn(r, __fdiv_rn((float)(100 - lane), 100.0f));
+            if (kF16Scale) {
+                const __half h = __float2half_rn(raw);
+                sb_i = __half_as_ushort(h);
+                sf_i = __half2float(h);
+            } else {
+                const __nv_bfloat16 b = __float2bfloat16_rn(raw);
+                sb_i = __bfloat16_as_ushort(b);
+                sf_i = __bfloat162float(b);
+            }
+            const double sd = (double)sf_i;
+            double e = 0.0;
+            for (int k = 0; k < 128; ++k) {
+                const float w = grp[wib][k];
+                const int c = sf_i != 0.0f ? max(-127, min(127, __float2int_rn(__fdiv_rn(w, sf_i)))) : 0;
+                const double d = __dsub_rn((double)w, __dmul_rn(sd, (double)c));
+                e = __dadd_rn(e, __dmul_rn(d, d));
+            }
+            // A NaN score (a scale that overflowed f16) never wins, except at candidate 0,
+            // which a sequential scan starts from and only a smaller score replaces.
+            err = isnan(e) ? (lane == 0 ? -INFINITY : INFINITY) : e;
+        }
+        int best = lane;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            const double oe = __shfl_xor_sync(kFull, err, m);
+            const int ob = __shfl_xor_sync(kFull, best, m);
+            if (oe < err || (oe == err && ob < best)) {
+                err = oe;
+                best = ob;
+            }
+        }
+        const float sf = __shfl_sync(kFull, sf_i, best);
+        const uint32_t sb = __shfl_sync(kFull, sb_i, best);
+        uint32_t packed = 0;
+        if (sf != 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int c = __float2int_rn(__fdiv_rn(v[i], sf));
+                c = max(-127, min(127, c));
+                packed |= (uint32_t)(c & 0xFF) << (8 * i);
+            }
+        }
+        *reinterpret_cast<uint32_t*>(q + off) = packed;
+        if (lane == 0) s[u] = (uint16_t)sb;
+        __syncwarp();  // the group's shared-memory copy is read before the next one lands
     }
 }
 
@@ -206,6 +284,21 @@ cudaError_t launch_pack_rtn(const float* W, int fmt, int flags, int N, int K, vo
     const int had = (flags & QL_HADAMARD) ? 1 : 0;
     const long long warps = (long long)N * (K / 128);
     const int grid = blocks_for(warps * 32, 256, di.sm_count);
+    if (flags & QL_SCALE_SEARCH) {
+        switch (fmt) {
+        case QL_I8_G128_BF16:
+        case QL_I8A8_G128_BF16:
+            k_search_i8<false><<<grid, 256, 0, s>>>(W, N, K, had, static_cast<int8_t*>(codes),
+                                                    static_cast<uint16_t*>(scales));
+            return cudaGetLastError();
+        case QL_I8_G128_F16:
+            k_search_i8<true><<<grid, 256, 0, s>>>(W, N, K, had, static_cast<int8_t*>(codes),
+                                                   static_cast<uint16_t*>(scales));
+            return cudaGetLastError();
+        default:
+            return cudaErrorNotSupported;
+        }
+    }
     switch (fmt) {
     case QL_I8_G128_BF16:
     case QL_I8A8_G128_BF16:

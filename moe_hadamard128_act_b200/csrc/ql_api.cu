@@ -181,7 +181,7 @@ MoeWs moe_ws(const ql_experts* ex, int T, int topk) {
 int check_experts(const ql_experts* ex) {
     if (!ex) return QL_EINVAL;
     if (ex->E < 1 || ex->E > 1024 || ex->N < 1 || ex->K < 128 || ex->K % 128) return QL_EINVAL;
-    if (ex->flags & ~QL_HADAMARD) return QL_EINVAL;
+    if (ex->flags & ~(QL_HADAMARD | QL_SCALE_SEARCH)) return QL_EINVAL;
     if (!fmt_valid(ex->fmt)) return QL_EINVAL;
     if (ex->fmt != QL_I8_G128_BF16 && ex->fmt != QL_I8_G128_F16 && ex->fmt != QL_FP8_B128_BF16) return QL_EUNSUPPORTED;
     if (ex->K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
@@ -216,9 +216,14 @@ int qlinear_packed_sizes(int fmt, int N, int K, size_t* codes_bytes, size_t* sca
 
 int qlinear_pack(const float* W, const void* codes_in, const void* scales_in, const uint8_t* zeros_in, int fmt,
                  int flags, int N, int K, void* codes_out, void* scales_out, uint8_t* zeros_out, void* stream) {
-    if (!fmt_valid(fmt) || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
+    if (!fmt_valid(fmt) || N < 1 || K < 128 || K % 128 || (flags & ~(QL_HADAMARD | QL_SCALE_SEARCH)))
+        return QL_EINVAL;
     if (!codes_out || !scales_out) return QL_EINVAL;
     if ((W == nullptr) == (codes_in == nullptr)) return QL_EINVAL;  // exactly one source
+    if (flags & QL_SCALE_SEARCH) {  // a rule for quantising W, int8 formats only
+        if (!W) return QL_EINVAL;
+        if (fmt != QL_I8_G128_BF16 && fmt != QL_I8_G128_F16 && fmt != QL_I8A8_G128_BF16) return QL_EUNSUPPORTED;
+    }
     if (!aligned16(codes_out) || !aligned16(scales_out)) return QL_EALIGN;
     if (fmt == QL_I5Z_G128_F16) {
         if (!zeros_out) return QL_EINVAL;
@@ -260,7 +265,8 @@ int qlinear_pack(const float* W, const void* codes_in, const void* scales_in, co
 }
 
 int qlinear_workspace_size(int fmt, int flags, int M, int N, int K, size_t* bytes) {
-    if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD) || !bytes)
+    if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~(QL_HADAMARD | QL_SCALE_SEARCH)) ||
+        !bytes)
         return QL_EINVAL;
     *bytes = forward_ws(fmt, M, N, K).total();
     return QL_OK;
@@ -268,7 +274,8 @@ int qlinear_workspace_size(int fmt, int flags, int M, int N, int K, size_t* byte
 
 int qlinear_forward(const void* x, const void* W_packed, const void* scales, const uint8_t* zeros, int fmt,
                     int flags, int M, int N, int K, float* y, void* ws, size_t ws_bytes, void* stream) {
-    if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
+    if (!fmt_valid(fmt) || M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~(QL_HADAMARD | QL_SCALE_SEARCH)))
+        return QL_EINVAL;
     if (!x || !W_packed || !scales || !y) return QL_EINVAL;
     if (fmt == QL_I5Z_G128_F16 && !zeros) return QL_EINVAL;
     if (fmt != QL_I8A8_G128_BF16 && fmt != QL_FP8A8_B128_BF16 && K > QL_A16_MAX_K) return QL_EUNSUPPORTED;

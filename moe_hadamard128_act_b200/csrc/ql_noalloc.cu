@@ -57,7 +57,7 @@ using namespace ql;
 
 extern "C" int qlinear_forward_w8a8_noalloc(const void* x, const void* W_packed, const void* scales, int flags, int M,
                                             int N, int K, float* y, void* stream) {
-    if (M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~QL_HADAMARD)) return QL_EINVAL;
+    if (M < 1 || N < 1 || K < 128 || K % 128 || (flags & ~(QL_HADAMARD | QL_SCALE_SEARCH))) return QL_EINVAL;
     if (M > kMaxM || K > kMaxK) return QL_EUNSUPPORTED;  // larger than the fixed scratch
     if (!x || !W_packed || !scales || !y) return QL_EINVAL;
     if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y)) return QL_EALIGN;

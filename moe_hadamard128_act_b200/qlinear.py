@@ -26,6 +26,7 @@ I5Z_G128_F16 = 5
 FP8_B128_BF16 = 6
 FP8A8_B128_BF16 = 7  # the fp8 weights with E4M3 activations
 HADAMARD = 1
+SCALE_SEARCH = 2  # qlinear_pack of an fp32 W, int8 formats: the best of 21 scales per group
 FORMATS = (I8_G128_BF16, I8_G128_F16, I8A8_G128_BF16, I4_G64_BF16, I5Z_G128_F16, FP8_B128_BF16, FP8A8_B128_BF16)
 
 DEVERR_EXPERT_ID = 1

@@ -38,6 +38,8 @@ def test_binding_constants_match_header():
     from moe_hadamard128_act_b200 import qlinear as Q
     text = (ROOT / "include" / "qlinear.h").read_text()
     assert int(re.search(r"QL_A16_MAX_K\s*=\s*(\d+)", text).group(1)) == Q.A16_MAX_K
+    assert int(re.search(r"QL_HADAMARD\s*=\s*(\d+)", text).group(1)) == Q.HADAMARD
+    assert int(re.search(r"QL_SCALE_SEARCH\s*=\s*(\d+)", text).group(1)) == Q.SCALE_SEARCH
     for name in ("I8_G128_BF16", "I8_G128_F16", "I8A8_G128_BF16", "I4_G64_BF16", "I5Z_G128_F16", "FP8_B128_BF16",
                  "FP8A8_B128_BF16"):
         assert int(re.search(rf"QL_{name}\s*=\s*(\d+)", text).group(1)) == getattr(Q, name), name
@@ -63,7 +65,9 @@ def test_packed_sizes_and_workspace_reject_bad_args(L):
             Q.qlinear_packed_sizes(fmt, N, K)
         assert e.value.status == 1
     with pytest.raises(Q.QLError):
-        Q.qlinear_workspace_size(1, 2, 1, 8, 128)  # unknown flag
+        Q.qlinear_workspace_size(1, 4, 1, 8, 128)  # unknown flag
+    # the scale-search bit describes how W was packed, not its layout: accepted and ignored
+    assert Q.qlinear_workspace_size(3, 2 | 1, 16, 21504, 5376) == Q.qlinear_workspace_size(3, 1, 16, 21504, 5376)
     assert Q.qlinear_workspace_size(1, 0, 16, 21504, 5376) >= 16 * 5376 * 2
     assert Q.qlinear_workspace_size(3, 1, 16, 21504, 5376) >= 16 * 5376 + 16 * 42 * 4
     assert Q.qlinear_workspace_size(7, 1, 1, 21504, 5376) >= 5376 + 42 * 128 * 4 + 42 * 21504 * 4
@@ -106,6 +110,10 @@ def test_pack_and_act_validation_statuses(L):
     assert p(P(A + 4), None, None, None, 1, 0, 8, 128, P(A), P(A), None, None) == 3
     assert p(None, P(A), None, None, 4, 0, 8, 128, P(A), P(A), None, None) == 1  # codes without scales
     assert p(None, P(A), P(A), None, 5, 0, 8, 128, P(A), P(A), P(A), None) == 1  # int5 codes without zeros
+    assert p(P(A), None, None, None, 4, 2, 8, 128, P(A), P(A), None, None) == 2  # scale search: int8 only
+    assert p(P(A), None, None, None, 6, 3, 8, 128, P(A), P(A), None, None) == 2
+    assert p(None, P(A), P(A), None, 1, 2, 8, 128, P(A), P(A), None, None) == 1  # a rule for W, not for codes
+    assert p(P(A), None, None, None, 1, 4, 8, 128, P(A), P(A), None, None) == 1  # unknown flag bit
     assert L.act_quant_i8_g128(P(A), 4, 100, 0, P(A), P(A), None) == 1
     assert L.act_quant_e4m3_g128(P(A), 4, 100, 0, P(A), P(A), None) == 1
     assert L.act_quant_e4m3_g128(P(A), 4, 128, 0, P(A + 4), P(A), None) == 3

@@ -100,6 +100,39 @@ def test_pack_rtn_bitexact(fmt, had, N, K):
     assert np.array_equal(host_u8(scales).view(np.uint16), s_ref.ravel())
 
 
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("fmt", [1, 2, 3])
+@pytest.mark.parametrize("N,K", [(40, 384), (300, 1024)])
+def test_pack_scale_search_bitexact(fmt, had, N, K):
+    # codes, scales and (through them) every group's pick among the 21 candidates, bit for bit;
+    # heavy-tailed rows make some groups pick a smaller scale, and a zero group keeps s = 0
+    rng = np.random.default_rng(61 + N)
+    W = synth.weight_rows(61, f"Ws{N}", K, 0, N)
+    W[::3] = (rng.standard_t(3, size=W[::3].shape) * 0.01).astype(np.float32)
+    W[1, :128] = 0.0
+    codes, scales, _ = Q.qlinear_pack(fmt, N, K, W=dev(W), flags=had | Q.SCALE_SEARCH)
+    q_ref, s_ref, picks = O.quant_i8_g128_search(W, hadamard=bool(had), scale_f16=(fmt == Q.I8_G128_F16))
+    assert np.array_equal(host_u8(codes), q_ref.view(np.uint8).ravel())
+    assert np.array_equal(host_u8(scales).view(np.uint16), s_ref.ravel())
+    assert (picks > 0).any() and s_ref[1, 0] == 0
+    # and it is a different packing from round to nearest on those groups
+    c_rtn, s_rtn, _ = Q.qlinear_pack(fmt, N, K, W=dev(W), flags=had)
+    assert not np.array_equal(host_u8(scales), host_u8(s_rtn))
+
+
+def test_pack_scale_search_then_forward():
+    # the searched weights through the W8A8 forward, decode and prefill sizes, against the oracle
+    N, K = 320, 512
+    W = synth.weight_rows(67, "Wsf", K, 0, N)
+    c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N, K, W=dev(W), flags=Q.HADAMARD | Q.SCALE_SEARCH)
+    q_ref, s_ref, _ = O.quant_i8_g128_search(W, hadamard=True)
+    for M in (3, 40):
+        x = x_bits(M, K, seed=67)
+        y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.I8A8_G128_BF16, N, flags=Q.HADAMARD | Q.SCALE_SEARCH)
+        ref = O.forward(x, q_ref.view(np.uint8), s_ref, None, Q.I8A8_G128_BF16, Q.HADAMARD, N)
+        assert_close(y.cpu().numpy(), ref, f"searched W8A8 M={M}")
+
+
 def test_pack_given_codes_bitexact_and_range_flag():
     N, K = 96, 256
     rng = np.random.default_rng(7)
