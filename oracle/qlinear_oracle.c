@@ -668,7 +668,12 @@ void qo_dequant(int fmt, const uint8_t* codes, const uint16_t* scales, const uin
 /* QO_HADAMARD); each group's integer dot product                            */
 /*   acc[m,n,g] = sum_{k in g} qx[m,k] * qw[n,k]                             */
 /* is kept exactly (int32), and y = sum_g sx[m,g] * sw[n,g] * acc[m,n,g].    */
+/* The int5 format does the same above 64 rows ("keptn/gemma4-31b-w5",      */
+/* table "Format": activations up to 64 rows f16, above that int8 with one  */
+/* scale per token and 128 values), with qw = q - z, the zero-point-        */
+/* corrected code, and its f16 scale for sw.                                 */
 /* ------------------------------------------------------------------------ */
+enum { QO_W5A8_MIN_M = 65 };
 
 int qo_forward(const uint16_t* x, int M, int K, const uint8_t* codes, const uint16_t* scales,
                const uint8_t* zeros, int fmt, int flags, int N, double* y, int32_t* acc_out)
@@ -694,6 +699,38 @@ int qo_forward(const uint16_t* x, int M, int K, const uint8_t* codes, const uint
                 }
                 y[(size_t)m * N + n] = sum;
             }
+        }
+        free(qx);
+        free(sx);
+        return 0;
+    }
+    if (fmt == QO_I5Z_G128_F16 && M >= QO_W5A8_MIN_M) {
+        int8_t* qx = (int8_t*)malloc((size_t)M * K);
+        float* sx = (float*)malloc(sizeof(float) * (size_t)M * G);
+        qo_act_quant_i8_g128(x, M, K, flags & QO_HADAMARD, qx, sx);
+        size_t rb = (size_t)K * 5 / 8;
+#pragma omp parallel for schedule(static)
+        for (int n = 0; n < N; ++n) {
+            int32_t* qw = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+            for (int k = 0; k < K; ++k) {
+                unsigned v = 0;
+                for (int bit = 0; bit < 5; ++bit) {
+                    size_t b = (size_t)k * 5 + bit;
+                    v |= (unsigned)((codes[(size_t)n * rb + b / 8] >> (b % 8)) & 1) << bit;
+                }
+                qw[k] = (int32_t)v - (int32_t)zeros[(size_t)n * G + k / 128];
+            }
+            for (int m = 0; m < M; ++m) {
+                double sum = 0.0;
+                for (int g = 0; g < G; ++g) {
+                    int32_t acc = 0;
+                    for (int i = 0; i < 128; ++i) acc += (int32_t)qx[(size_t)m * K + g * 128 + i] * qw[g * 128 + i];
+                    if (acc_out) acc_out[((size_t)m * N + n) * G + g] = acc;
+                    sum += (double)sx[(size_t)m * G + g] * qo_f16_decode(scales[(size_t)n * G + g]) * (double)acc;
+                }
+                y[(size_t)m * N + n] = sum;
+            }
+            free(qw);
         }
         free(qx);
         free(sx);

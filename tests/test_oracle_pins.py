@@ -556,6 +556,42 @@ def test_forward_fp8a8_brute_force():
     assert np.allclose(y, xd @ Wd.T, rtol=1e-12, atol=1e-14)
 
 
+@pytest.mark.parametrize("had", [0, 1])
+def test_forward_int5_switches_to_w5a8_above_64_rows(had):
+    # "keptn/gemma4-31b-w5", table "Format": activations up to 64 rows f16, above that int8 per token
+    # per 128.  Above 64 rows the int5 forward must equal the (separately pinned) W8A8 forward of the
+    # zero-point-corrected codes q - z with the same scales; at 64 rows it is the weight-only product.
+    rng = np.random.default_rng(71)
+    N, K = 6, 256
+    q5 = rng.integers(0, 32, (N, K)).astype(np.uint8)
+    z5 = rng.integers(0, 32, (N, K // 128)).astype(np.uint8)
+    # scales with 8 significant bits inside the f16 range: exact in f16 and in bf16 alike
+    sval = (1 + rng.integers(0, 128, (N, K // 128)) / 128.0) * 2.0 ** rng.integers(-9, -3, (N, K // 128))
+    s_f16 = O.f16_encode(sval)
+    s_bf16 = O.bf16_encode(sval)
+    assert np.array_equal(O.f16_decode(s_f16), sval) and np.array_equal(O.bf16_decode(s_bf16), sval)
+    q8 = (q5.astype(np.int16) - np.repeat(z5, 128, axis=1)).astype(np.int8)
+    packed = O.pack_i5(q5)
+    for M in (65, 130):
+        x = O.bf16_encode(rng.standard_normal((M, K)))
+        y5, acc5 = O.forward(x, packed, s_f16, z5, O.I5Z_G128_F16, had, N, want_acc=True)
+        y8, acc8 = O.forward(x, q8.view(np.uint8), s_bf16, None, O.I8A8_G128_BF16, had, N, want_acc=True)
+        assert np.array_equal(acc5, acc8) and np.array_equal(y5, y8)
+        assert np.abs(acc5).max() <= 128 * 127 * 31
+    # at 64 rows: bf16 x (rotated with the flag) times the dequantised weight, no activation codes
+    x = O.bf16_encode(rng.standard_normal((65, K)))
+    xr = O.hadamard128_rotate(x) if had else x
+    W = O.dequant(O.I5Z_G128_F16, packed, s_f16, z5, N, K)
+    y64 = O.forward(x[:64], packed, s_f16, z5, O.I5Z_G128_F16, had, N)
+    exact = O.bf16_decode(xr[:64]) @ W.T
+    assert np.allclose(y64, exact, rtol=1e-12, atol=1e-12 * np.abs(exact).max())
+    # one row more switches the whole call to int8 activations: close to, but not, the weight-only product
+    y65 = O.forward(x, packed, s_f16, z5, O.I5Z_G128_F16, had, N)
+    exact65 = O.bf16_decode(xr) @ W.T
+    rel = np.linalg.norm(y65 - exact65) / np.linalg.norm(exact65)
+    assert 1e-5 < rel < 2e-2
+
+
 def test_w8a8_int32_accumulators_and_combination():
     M, N, K = 3, 4, 384
     q = RNG.integers(-127, 128, (N, K)).astype(np.int8)
