@@ -416,6 +416,28 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                                 "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal fp8/bf16 ratio)",
                                 "mma": "kind::f8f6f4 (E4M3 x E4M3, fp32 group sums)"}
         del c, s, y, ws
+        # int5 with a zero point from 65 rows on (W5A8): int8 activations, the codes converted to
+        # int8 q - z in the workspace, the W8A8 tensor-core GEMM
+        d5 = synth.w5a16(M)
+        c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N_FULL, K_FULL, codes=torch.from_numpy(d5["codes"]).to(dev),
+                                 scales=torch.from_numpy(d5["scales"]).to(dev),
+                                 zeros=torch.from_numpy(d5["zeros"]).to(dev))
+        x5 = bf(d5["x"])
+        y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+        ws = torch.empty(Q.qlinear_workspace_size(Q.I5Z_G128_F16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
+                         device=dev)
+        run = lambda i: Q.qlinear_forward(x5, c, s, z, Q.I5Z_G128_F16, N_FULL, y=y, ws=ws,  # noqa: E731
+                                          stream=stream)
+        for i in range(3):
+            run(i)
+        t, _ = _traced(Q, run, 10, "prefill")
+        tq, _ = _traced(Q, run, 10, "act_quant")
+        tp, _ = _traced(Q, run, 10, "prefill_prep")
+        out["prefill_w5a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq,
+                               "us_scale_prep_and_code_conversion": 1e3 * tp, "TOPS": ops / (t * 1e-3) / 1e12,
+                               "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
+                               "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
+        del c, s, z, y, ws, d5
     torch.cuda.synchronize()
     return out
 

@@ -17,7 +17,11 @@
  *                     release"); x is bf16.
  *   QL_I5Z_G128_F16   int5 codes [0,31] with a u8 zero point and one f16 scale
  *                     per row per 128 of K: w = s * (q - z) ("keptn/gemma4-31b-w5",
- *                     table "Format"); x is bf16.
+ *                     table "Format"); x is bf16 up to 64 rows (M <= 64).  From
+ *                     65 rows on, as that card's activations do, x is quantised
+ *                     to int8 per token per 128 like W8A8's and each group's
+ *                     integer dot product sum qx * (q - z) is exact before s_x * s
+ *                     is applied (W5A8).
  *   QL_FP8_B128_BF16  FP8 E4M3 codes with one bf16 scale per 128 (rows) x 128
  *                     (K) block ("gemma4-26b-a4b-dflash-fp8" README, table
  *                     "Weights" and its recipe); x is bf16.
@@ -146,14 +150,16 @@ int qlinear_workspace_size(int fmt, int flags, int M, int N, int K, size_t* byte
  *      rotation rounded to bf16 (as hadamard128_rotate); for W8A8, x~ is the
  *      int8 quantisation of (rotated) x, one fp32 scale per token per 128
  *      (as act_quant_i8_g128), and each 128-group's integer dot product is
- *      exact in int32 before its two scales are applied.
+ *      exact in int32 before its two scales are applied; the same for int5
+ *      with M >= 65 (W5A8, codes q - z).
  *   W_packed, scales, zeros: the packed weight (zeros only for int5).
  *   ws, ws_bytes: caller's device workspace, at least qlinear_workspace_size.
  * y is overwritten.  The floating-point sums may be accumulated in any order;
  * they are not bit-reproducible across calls.
- * Formats whose activations stay 16-bit (all but QL_I8A8_G128_BF16) stage one
- * token row, in fp32 and f16, in shared memory: they take K <= QL_A16_MAX_K
- * and return QL_EUNSUPPORTED above it (moe_gate_up likewise). */
+ * Calls whose activations stay 16-bit (all formats but W8A8 and format 7, and
+ * int5 up to 64 rows) stage one token row, in fp32 and f16, in shared memory:
+ * they take K <= QL_A16_MAX_K and return QL_EUNSUPPORTED above it
+ * (moe_gate_up likewise). */
 enum { QL_A16_MAX_K = 32768 };
 int qlinear_forward(const void* x, const void* W_packed, const void* scales, const uint8_t* zeros, int fmt,
                     int flags, int M, int N, int K, float* y, void* ws, size_t ws_bytes, void* stream);

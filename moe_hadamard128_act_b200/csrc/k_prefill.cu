@@ -505,8 +505,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
     }
 }
 
-// bf16 weight scales [N][G] -> fp32 [G][Np], columns n >= N zero.  32 x 32
+// bf16 (or f16) weight scales [N][G] -> fp32 [G][Np], columns n >= N zero.  32 x 32
 // tiles through shared memory, so reads and writes are both coalesced.
+template <bool kF16>
 __global__ void __launch_bounds__(256) k_prefill_prep(const uint16_t* sw, int N, int G, int Np, float* swT) {
     __shared__ float tile[32][33];
     const int g0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
@@ -514,7 +515,8 @@ __global__ void __launch_bounds__(256) k_prefill_prep(const uint16_t* sw, int N,
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = ty + 8 * i, n = n0 + r, g = g0 + tx;
-        tile[r][tx] = (n < N && g < G) ? __uint_as_float((uint32_t)sw[(long long)n * G + g] << 16) : 0.0f;
+        const uint16_t b = (n < N && g < G) ? sw[(long long)n * G + g] : 0;
+        tile[r][tx] = kF16 ? __half2float(__ushort_as_half(b)) : __uint_as_float((uint32_t)b << 16);
     }
     __syncthreads();
 #pragma unroll
@@ -522,6 +524,38 @@ __global__ void __launch_bounds__(256) k_prefill_prep(const uint16_t* sw, int N,
         const int gg = ty + 8 * i, g = g0 + gg;
         if (g < G) swT[(long long)g * Np + n0 + tx] = tile[tx][gg];
     }
+}
+
+// int5 codes with zero points -> the int8 codes q - z in [-31, 31] that the W8A8
+// GEMM multiplies, [N][K].  One thread per 32 codes: 20 bytes of the row's
+// least-significant-bit-first stream (code k at bits 5k .. 5k+4) in five
+// 32-bit words, out as two 16-byte stores.  A row is K * 5 / 8 bytes, a
+// multiple of 80, so every 32-code run starts on a 4-byte boundary.
+__global__ void __launch_bounds__(256) k_prefill_i5_codes(const uint8_t* codes, const uint8_t* zeros, int N, int K,
+                                                          int8_t* out) {
+    const long long u = (long long)blockIdx.x * 256 + threadIdx.x;
+    const int per_row = K / 32;
+    if (u >= (long long)N * per_row) return;
+    const long long n = u / per_row;
+    const int j = (int)(u - n * per_row);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(codes + n * ((long long)K * 5 / 8) + (long long)j * 20);
+    uint32_t w[6];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) w[i] = src[i];
+    w[5] = 0;
+    const int z = zeros[n * (K / 128) + (j * 32) / 128];
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = 0;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const int bit = 5 * c, wi = bit >> 5, sh = bit & 31;
+        const uint32_t v = (sh <= 27 ? (w[wi] >> sh) : ((w[wi] >> sh) | (w[wi + 1] << (32 - sh)))) & 31u;
+        o[c >> 2] |= (uint32_t)(((int)v - z) & 0xFF) << (8 * (c & 3));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + n * (long long)K + (long long)j * 32);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // bf16 block scales [ceil(N/128)][G] -> fp32 [G][Np], each row's block scale
@@ -542,10 +576,19 @@ cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scra
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s) {
+cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s, bool f16) {
     const int G = K / 128, Np = prefill_pad_n(N);
     const dim3 grid((G + 31) / 32, Np / 32);
-    k_prefill_prep<<<grid, 256, 0, s>>>(sw, N, G, Np, static_cast<float*>(scratch));
+    if (f16) k_prefill_prep<true><<<grid, 256, 0, s>>>(sw, N, G, Np, static_cast<float*>(scratch));
+    else k_prefill_prep<false><<<grid, 256, 0, s>>>(sw, N, G, Np, static_cast<float*>(scratch));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_i5_codes(const uint8_t* codes, const uint8_t* zeros, int N, int K, int8_t* out,
+                                    cudaStream_t s) {
+    const long long units = (long long)N * (K / 32);
+    const long long blocks = (units + 255) / 256;
+    k_prefill_i5_codes<<<(unsigned)blocks, 256, 0, s>>>(codes, zeros, N, K, out);
     return cudaGetLastError();
 }
 

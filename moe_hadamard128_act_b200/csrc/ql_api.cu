@@ -126,6 +126,12 @@ FwdWs forward_ws(int fmt, size_t M, size_t N, size_t K) {
         w.x_bytes = align_up(M * K, 256);
         w.f_bytes = align_up((K / 128) * prefill_pad_m((int)M) * 4, 256);
         w.g_bytes = prefill_scratch_bytes((int)N, (int)K);
+    } else if (fmt == QL_I5Z_G128_F16 && M >= (size_t)kW5A8MinM) {
+        // int8 activation codes, transposed scales, then the GEMM's weight scales and the
+        // weight codes converted to int8 (q - z)
+        w.x_bytes = align_up(M * K, 256);
+        w.f_bytes = align_up((K / 128) * prefill_pad_m((int)M) * 4, 256);
+        w.g_bytes = prefill_scratch_bytes((int)N, (int)K) + align_up(N * K, 256);
     } else if (fmt == QL_I8A8_G128_BF16) {
         w.x_bytes = align_up(M * K, 256);
         if (M >= (size_t)kPrefillMinM) {
@@ -278,7 +284,8 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         return QL_EINVAL;
     if (!x || !W_packed || !scales || !y) return QL_EINVAL;
     if (fmt == QL_I5Z_G128_F16 && !zeros) return QL_EINVAL;
-    if (fmt != QL_I8A8_G128_BF16 && fmt != QL_FP8A8_B128_BF16 && K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
+    const bool a8 = fmt == QL_I8A8_G128_BF16 || fmt == QL_FP8A8_B128_BF16 || (fmt == QL_I5Z_G128_F16 && M >= kW5A8MinM);
+    if (!a8 && K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
     if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y) ||
         (zeros && !aligned16(zeros)))
         return QL_EALIGN;
@@ -310,6 +317,23 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         t = trace_begin(QL_KIND_PREFILL, s);
         e = launch_prefill_w8a8(static_cast<const int8_t*>(xs), xf, static_cast<const int8_t*>(W_packed), M, N, K, y,
                                 N, nullptr, gs, s, true);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
+    if (fmt == QL_I5Z_G128_F16 && M >= kW5A8MinM) {  // W5A8: int8 activations, the W8A8 tensor-core GEMM
+        int t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), nullptr, xf, prefill_pad_m(M), nullptr, 0, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        uint8_t* const gs = wsb + w.x_bytes + w.f_bytes;
+        int8_t* const q8 = reinterpret_cast<int8_t*>(gs + prefill_scratch_bytes(N, K));
+        t = trace_begin(QL_KIND_PREFILL_PREP, s);
+        e = launch_prefill_prep(static_cast<const uint16_t*>(scales), N, K, gs, s, true);
+        if (e == cudaSuccess) e = launch_prefill_i5_codes(static_cast<const uint8_t*>(W_packed), zeros, N, K, q8, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_PREFILL, s);
+        e = launch_prefill_w8a8(static_cast<const int8_t*>(xs), xf, q8, M, N, K, y, N, nullptr, gs, s);
         trace_end(t, s);
         return from_cuda(e);
     }

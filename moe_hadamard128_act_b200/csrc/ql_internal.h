@@ -111,8 +111,14 @@ inline size_t prefill_scratch_bytes(int N, int K) { return align_up((size_t)(K /
 cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t* qw, int M, int N, int K,
                                 float* y, long long ldy, int32_t* acc, const void* scratch, cudaStream_t s,
                                 bool e4m3 = false);
-// Fills the scratch: bf16 weight scales [N][K/128] -> fp32 [K/128][pad(N)].
-cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
+// Fills the scratch: bf16 (f16) weight scales [N][K/128] -> fp32 [K/128][pad(N)].
+cudaError_t launch_prefill_prep(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s, bool f16 = false);
+// int5 codes [N][5K/8] and zero points [N][K/128] -> int8 q - z [N][K] (for the W5A8 path).
+cudaError_t launch_prefill_i5_codes(const uint8_t* codes, const uint8_t* zeros, int N, int K, int8_t* out,
+                                    cudaStream_t s);
+// From this many rows on, the int5 format takes int8 activations ("keptn/gemma4-31b-w5",
+// table "Format": f16 activations up to 64 rows, int8 per token per 128 above).
+constexpr int kW5A8MinM = 65;
 // The same from bf16 block scales [ceil(N/128)][K/128] (each row takes its block's scale).
 cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
 constexpr int kPrefillMinM = 17;  // from this many tokens on, W8A8 runs on the tcgen05 GEMM

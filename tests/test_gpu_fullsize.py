@@ -75,6 +75,19 @@ def test_w4a16_full(Q, M):
     assert_close(y[:, rows], ref, f"W4A16 M={M}")
 
 
+def test_w5a8_prefill_full(Q):
+    # the int5 weight at full size with 2048 tokens: int8 activations (W5A8), sampled rows
+    M = 2048
+    d = synth.w5a16(M)
+    c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N_FULL, K_FULL, codes=dev(d["codes"]), scales=dev(d["scales"]),
+                             zeros=dev(d["zeros"]))
+    y = Q.qlinear_forward(dev_bf16(d["x"]), c, s, z, Q.I5Z_G128_F16, N_FULL).cpu().numpy()
+    rows = sample_rows(N_FULL, seed=29)
+    ref = O.forward(d["x"], O.pack_i5(d["codes"][rows]), d["scales"][rows], d["zeros"][rows], Q.I5Z_G128_F16, 0,
+                    len(rows))
+    assert_close(y[:, rows], ref, "W5A8 M=2048")
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_w5a16_full(Q, M):
     d = synth.w5a16(M)

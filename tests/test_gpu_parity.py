@@ -407,6 +407,31 @@ def test_fp8a8_forward_parity(M, N, K, had):
     assert_close(y.cpu().numpy(), ref, f"fp8a8 had {had} {M}x{N}x{K}")
 
 
+# --------------------------------------------------------------------------
+# int5 from 65 rows on: int8 activations on the W8A8 tensor-core GEMM (W5A8)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("had", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(64, 130, 256), (65, 130, 256), (65, 64, 128), (130, 388, 512),
+                                   (300, 200, 384)])
+def test_w5a8_forward_parity(M, N, K, had):
+    # M = 64 is the last weight-only call, M = 65 the first W5A8 one; the oracle switches alike
+    (c, s, z), (ch, sh, zh) = make_weights(Q.I5Z_G128_F16, N, K, had, seed=73)
+    x = x_bits(M, K, seed=73, outliers=0.01)
+    y = Q.qlinear_forward(dev_bf16(x), c, s, z, Q.I5Z_G128_F16, N, flags=had)
+    ref = O.forward(x, ch, sh, zh, Q.I5Z_G128_F16, had, N)
+    assert_close(y.cpu().numpy(), ref, f"int5 had {had} {M}x{N}x{K}")
+
+
+def test_w5a8_large_tile_count_and_repeat():
+    M, N, K = 1290, 3980, 256  # more tiles than SMs, ragged in M and N, called twice
+    (c, s, z), (ch, sh, zh) = make_weights(Q.I5Z_G128_F16, N, K, 0, seed=79)
+    x = x_bits(M, K, seed=79)
+    ref = O.forward(x, ch, sh, zh, Q.I5Z_G128_F16, 0, N)
+    for _ in range(2):
+        y = Q.qlinear_forward(dev_bf16(x), c, s, z, Q.I5Z_G128_F16, N)
+        assert_close(y.cpu().numpy(), ref, f"w5a8 {M}x{N}x{K}")
+
+
 def test_fp8a8_large_tile_count_and_repeat():
     M, N, K = 1290, 3980, 256  # more tiles than SMs, ragged in M and N, called twice
     (c, s, z), (ch, sh, zh) = make_weights(Q.FP8A8_B128_BF16, N, K, 0, seed=47)
