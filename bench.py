@@ -270,13 +270,15 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
     G = K_FULL // 128
     bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     with torch.cuda.stream(stream):
-        # weight-only decode: int4 g64, int5 + zero point g128, int8 g128 bf16, fp8 128x128.
+        # weight-only decode: int4 g64, int5 + zero point g128, int8 g128 bf16, fp8 128x128; and
+        # format 7 (the fp8 weight with E4M3 activations) on the same decode kernel.
         # "us" is the whole forward (activation prologue + decode GEMM) replayed from a
         # CUDA graph, the rate it gives is over the forward's bytes; "us_gemm" is the
         # traced decode kernel alone.
         Wd = None
         for name, fmt in (("w4a16_decode", Q.I4_G64_BF16), ("w5a16_decode", Q.I5Z_G128_F16),
-                          ("w8a16_decode", Q.I8_G128_BF16), ("fp8_decode", Q.FP8_B128_BF16)):
+                          ("w8a16_decode", Q.I8_G128_BF16), ("fp8_decode", Q.FP8_B128_BF16),
+                          ("fp8a8_decode", Q.FP8A8_B128_BF16)):
             if fmt in (Q.I4_G64_BF16, Q.I5Z_G128_F16):
                 d = synth.w4a16(16) if fmt == Q.I4_G64_BF16 else synth.w5a16(16)
                 z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None

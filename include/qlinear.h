@@ -30,8 +30,9 @@
  *                     act_quant_e4m3_g128 does (the int8 activation rule of
  *                     "keptn/gemma4-12b-i8g" with E4M3 codes; a reading, no card
  *                     ships it), and every 128-group's products are summed
- *                     before both scales are applied.  All M run the
- *                     tensor-core E4M3 GEMM.
+ *                     before both scales are applied.  M <= 16 runs
+ *                     the weight-streaming decode kernel on E4M3 mma.sync,
+ *                     M >= 17 the tensor-core E4M3 GEMM.
  * Flag QL_HADAMARD: the weights live in the 128-wide Walsh-Hadamard domain
  * ("transform=fwht128" in the recipe of "gemma4-26b-a4b-dflash-i8"); the
  * forward pass rotates each 128-block of x by the same orthonormal transform

@@ -216,13 +216,13 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
 }
 
 cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
-                                  cudaStream_t s) {
+                                  float* yz, long long nz, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
     if ((e = prefer_max_shared(k_act_quant<true>)) != cudaSuccess) return e;
     k_act_quant<true><<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), M, K, rotate, reinterpret_cast<int8_t*>(q), sx, sxT, Mp, nullptr, 0);
+        static_cast<const __nv_bfloat16*>(x), M, K, rotate, reinterpret_cast<int8_t*>(q), sx, sxT, Mp, yz, nz);
     return cudaGetLastError();
 }
 

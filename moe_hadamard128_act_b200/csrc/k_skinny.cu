@@ -62,6 +62,16 @@ struct Regs<QL_I8A8_G128_BF16> : Regs<QL_I8_G128_BF16> {};
 template <>
 struct Regs<QL_FP8_B128_BF16> : Regs<QL_I8_G128_BF16> {};
 template <>
+struct Regs<QL_FP8A8_B128_BF16> : Regs<QL_I8_G128_BF16> {};
+
+// Formats whose activations are one-byte codes with an fp32 scale per token
+// per 128 (int8 for W8A8, E4M3 for format 7), multiplied on the byte MMAs.
+template <int FMT>
+__host__ __device__ constexpr bool act8() { return FMT == QL_I8A8_G128_BF16 || FMT == QL_FP8A8_B128_BF16; }
+// Weight scales per 128 x 128 block rather than per row.
+template <int FMT>
+__host__ __device__ constexpr bool block_scaled() { return FMT == QL_FP8_B128_BF16 || FMT == QL_FP8A8_B128_BF16; }
+template <>
 struct Regs<QL_I4_G64_BF16> {
     uint2 w[2][2];  // [row][64-wide half group]: 16 codes each
     float s[2][2];
@@ -76,11 +86,11 @@ struct Regs<QL_I5Z_G128_F16> {
 // Bytes of activations per token per 128-group in shared memory, and the
 // padding that makes the row stride an odd (1) or 2-mod-8 multiple of 16 B.
 template <int FMT>
-__host__ __device__ constexpr int x_group_bytes() { return FMT == QL_I8A8_G128_BF16 ? 128 : 256; }
+__host__ __device__ constexpr int x_group_bytes() { return act8<FMT>() ? 128 : 256; }
 template <int FMT>
-__host__ __device__ constexpr int x_row_pad() { return (FMT == QL_I8A8_G128_BF16 || FMT == QL_I4_G64_BF16) ? 16 : 32; }
+__host__ __device__ constexpr int x_row_pad() { return (act8<FMT>() || FMT == QL_I4_G64_BF16) ? 16 : 32; }
 template <int FMT>
-__host__ __device__ constexpr bool x_swizzled() { return !(FMT == QL_I8A8_G128_BF16 || FMT == QL_I4_G64_BF16); }
+__host__ __device__ constexpr bool x_swizzled() { return !(act8<FMT>() || FMT == QL_I4_G64_BF16); }
 
 template <int FMT>
 __device__ __forceinline__ int swz(int j) { return x_swizzled<FMT>() ? (j ^ ((j >> 3) & 1)) : j; }
@@ -134,7 +144,7 @@ __device__ __forceinline__ void load_unit(Regs<FMT>& r, const uint8_t* wbase, lo
                 const uint8_t* p = row + grp * 128 + 32 * c;
                 r.w[h][0] = ldg_stream128(p);
                 r.w[h][1] = ldg_stream128(p + 16);
-                if constexpr (FMT == QL_FP8_B128_BF16)
+                if constexpr (block_scaled<FMT>())
                     r.s[h] = load_scale<FMT>(scales, (long long)(n >> 7) * Gtot + gabs);
                 else  // the integer-only W8A8 check path has no scales
                     r.s[h] = scales ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
@@ -252,6 +262,16 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
     }
 }
 
+// E4M3 x E4M3 -> fp32 (format 7): the same fragments as the s8 MMA.
+__device__ __forceinline__ void mma_e4m3(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // W8A8: exact int32 sums of one group (4 k-steps of m16n8k32).
 template <int NT, typename GetX>
 __device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX getx, int (&acc)[NT][4]) {
@@ -272,6 +292,31 @@ __device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX
                 const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
                 const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
                 mma_s8(acc[nt], a0, a1, a2, a3, b0, b1);
+            }
+        }
+    }
+}
+
+// Format 7: fp32 sums of one group's E4M3 products, the same walk as unit_w8a8.
+template <int NT, typename GetX>
+__device__ __forceinline__ void unit_e4m3(const Regs<QL_FP8A8_B128_BF16>& r, GetX getx, float (&acc)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        uint4 xv[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) xv[nt] = getx(nt, p);
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+            const int s = 2 * p + sub;
+            const uint32_t a0 = word_of(r.w[0], 2 * s), a2 = word_of(r.w[0], 2 * s + 1);
+            const uint32_t a1 = word_of(r.w[1], 2 * s), a3 = word_of(r.w[1], 2 * s + 1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
+                const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
+                mma_e4m3(acc[nt], a0, a1, a2, a3, b0, b1);
             }
         }
     }
@@ -309,10 +354,10 @@ __host__ __device__ constexpr int stage_align() {
 // Activation staging: bytes per token per group and the row padding that keeps
 // the fragment loads conflict-free (see the piece index in tma_getx).
 template <int FMT>
-__host__ __device__ constexpr int tx_group_bytes() { return FMT == QL_I8A8_G128_BF16 ? 128 : 256; }
+__host__ __device__ constexpr int tx_group_bytes() { return act8<FMT>() ? 128 : 256; }
 template <int FMT>
 __host__ __device__ constexpr int tx_row_pad() {
-    return FMT == QL_I8A8_G128_BF16 ? 64 : (FMT == QL_I5Z_G128_F16 ? 32 : 16);
+    return act8<FMT>() ? 64 : (FMT == QL_I5Z_G128_F16 ? 32 : 16);
 }
 
 template <int FMT>
@@ -426,12 +471,12 @@ __device__ unsigned long long g_skinny_prof[148 * 16];
 // Per-unit side data, fetched kStages units ahead of use together with the
 // weight tile: raw scale bits (converted only when the unit is computed, so
 // the loads never stall the issuing loop), int5 zero points, and for W8A8 the
-// activation scales of the lane's output tokens.
+// activation scales of the lane's output tokens (W8A8 and format 7).
 template <int FMT, int NT>
 struct Side {
     uint32_t sw[2][2];  // weight scale bits [row g / g+8][int4 half]
     uint32_t z[2];      // int5 zero points
-    float sx[NT][2];    // W8A8: activation scales of tokens 8nt + 2c + {0, 1}
+    float sx[NT][2];    // byte activations: scales of tokens 8nt + 2c + {0, 1}
 };
 
 template <int FMT, int NT>
@@ -445,7 +490,7 @@ __device__ __forceinline__ void load_side_w(Side<FMT, NT>& d, const void* scales
         if constexpr (FMT == QL_I4_G64_BF16) {
             d.sw[h][0] = ok ? __ldg(sc + (long long)n * (2 * Gtot) + 2 * gabs) : 0u;
             d.sw[h][1] = ok ? __ldg(sc + (long long)n * (2 * Gtot) + 2 * gabs + 1) : 0u;
-        } else if constexpr (FMT == QL_FP8_B128_BF16) {
+        } else if constexpr (block_scaled<FMT>()) {
             d.sw[h][0] = ok ? __ldg(sc + (long long)(n >> 7) * Gtot + gabs) : 0u;
         } else {
             d.sw[h][0] = ok ? __ldg(sc + (long long)n * Gtot + gabs) : 0u;
@@ -456,7 +501,7 @@ __device__ __forceinline__ void load_side_w(Side<FMT, NT>& d, const void* scales
 
 template <int FMT, int NT>
 __device__ __forceinline__ void load_side_x(Side<FMT, NT>& d, const float* sx, int M, int Gtot, int gabs, int c) {
-    if constexpr (FMT == QL_I8A8_G128_BF16) {
+    if constexpr (act8<FMT>()) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -571,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
             const unsigned row_bytes = (unsigned)(ngs * XGB);
             mbar_expect_tx(xbar, row_bytes * rows_x);
             const uint8_t* xsrc = static_cast<const uint8_t*>(a.xs);
-            const long long ldx_b = a.ldx * (FMT == QL_I8A8_G128_BF16 ? 1 : 2);
+            const long long ldx_b = a.ldx * (act8<FMT>() ? 1 : 2);
             for (int t = 0; t < rows_x; ++t)
                 bulk_load(xs_base + (uint32_t)(t * R), xsrc + t * ldx_b + (long long)gs0 * XGB, row_bytes, xbar);
         }
@@ -583,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
             *reinterpret_cast<uint4*>(xs + t * R + 16 * j) = make_uint4(0, 0, 0, 0);
         }
     }
-    if constexpr (FMT == QL_I8A8_G128_BF16) {  // activation scales of the units already in flight
+    if constexpr (act8<FMT>()) {  // activation scales of the units already in flight
         UnitPos q = cp;
 #pragma unroll
         for (int s = 0; s < kStages; ++s) {
@@ -613,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 const int t = 8 * nt + 2 * c + (i & 1);
                 const int n = slab * 16 + g + 8 * (i >> 1);
                 if (t < a.M && n < a.N) {
-                    const float f = (FMT == QL_I8A8_G128_BF16) ? 1.0f : __ldg(a.xf + t);
+                    const float f = act8<FMT>() ? 1.0f : __ldg(a.xf + t);
                     atomicAdd(a.y + (long long)t * a.ldy + n, yacc[nt][i] * f);
                 }
                 yacc[nt][i] = 0.0f;
@@ -642,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
             const int lg = grp - gs0;  // group index in the staged activations
             auto getx = [&](int nt, int p) -> uint4 {
                 int j;
-                if constexpr (FMT == QL_I8A8_G128_BF16)
+                if constexpr (act8<FMT>())
                     j = lg * 8 + 4 * p + c;
                 else if constexpr (FMT == QL_I4_G64_BF16)
                     j = lg * 16 + (p & 8) + 2 * c + (p & 1);
@@ -671,6 +716,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                             yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s].sx[nt][i & 1], fa, yacc[nt][i]);
                         }
                     }
+            } else if constexpr (FMT == QL_FP8A8_B128_BF16) {
+                float acc[NT][4];
+                unit_e4m3<NT>(r, getx, acc);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s].sx[nt][i & 1], acc[nt][i], yacc[nt][i]);
             } else {
                 unit_a16<FMT, NT>(r, getx, nt1_live, yacc);
             }
@@ -1019,7 +1072,8 @@ int skinny_max_k(int fmt) {
     if (device_info(&di) != cudaSuccess) return 0;
     int xg = 0;
     switch (fmt) {
-    case QL_I8A8_G128_BF16: xg = max_staged_groups<QL_I8A8_G128_BF16>(2, di.smem_optin); break;
+    case QL_I8A8_G128_BF16:
+    case QL_FP8A8_B128_BF16: xg = max_staged_groups<QL_I8A8_G128_BF16>(2, di.smem_optin); break;
     case QL_I4_G64_BF16: xg = max_staged_groups<QL_I4_G64_BF16>(2, di.smem_optin); break;
     case QL_I5Z_G128_F16: xg = max_staged_groups<QL_I5Z_G128_F16>(2, di.smem_optin); break;
     default: xg = max_staged_groups<QL_I8_G128_BF16>(2, di.smem_optin); break;
@@ -1057,6 +1111,7 @@ cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     case QL_I4_G64_BF16: return run_skinny_fmt<QL_I4_G64_BF16>(a, s, di);
     case QL_I5Z_G128_F16: return run_skinny_fmt<QL_I5Z_G128_F16>(a, s, di);
     case QL_FP8_B128_BF16: return run_skinny_fmt<QL_FP8_B128_BF16>(a, s, di);
+    case QL_FP8A8_B128_BF16: return run_skinny_fmt<QL_FP8A8_B128_BF16>(a, s, di);
     }
     return cudaErrorInvalidValue;
 }

@@ -122,10 +122,14 @@ struct FwdWs {
 FwdWs forward_ws(int fmt, size_t M, size_t N, size_t K) {
     FwdWs w;
     w.g_bytes = 0;
-    if (fmt == QL_FP8A8_B128_BF16) {  // E4M3 codes, transposed scales, the GEMM's weight scales (every M)
+    if (fmt == QL_FP8A8_B128_BF16 && M >= (size_t)kPrefillMinM) {
+        // E4M3 codes, transposed scales, the GEMM's weight scales
         w.x_bytes = align_up(M * K, 256);
         w.f_bytes = align_up((K / 128) * prefill_pad_m((int)M) * 4, 256);
         w.g_bytes = prefill_scratch_bytes((int)N, (int)K);
+    } else if (fmt == QL_FP8A8_B128_BF16) {  // decode: E4M3 codes and their scales [M][K/128]
+        w.x_bytes = align_up(M * K, 256);
+        w.f_bytes = align_up(M * (K / 128) * 4, 256);
     } else if (fmt == QL_I5Z_G128_F16 && M >= (size_t)kW5A8MinM) {
         // int8 activation codes, transposed scales, then the GEMM's weight scales and the
         // weight codes converted to int8 (q - z)
@@ -304,9 +308,9 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     void* xs = wsb;
     float* xf = reinterpret_cast<float*>(wsb + w.x_bytes);
     cudaError_t e;
-    if (fmt == QL_FP8A8_B128_BF16) {  // E4M3 activations, the tensor-core E4M3 GEMM for every M
+    if (fmt == QL_FP8A8_B128_BF16 && M >= kPrefillMinM) {  // E4M3 activations, the tensor-core E4M3 GEMM
         int t = trace_begin(QL_KIND_ACT_QUANT, s);
-        e = launch_act_quant_e4m3(x, M, K, rot, static_cast<uint8_t*>(xs), nullptr, xf, prefill_pad_m(M), s);
+        e = launch_act_quant_e4m3(x, M, K, rot, static_cast<uint8_t*>(xs), nullptr, xf, prefill_pad_m(M), nullptr, 0, s);
         trace_end(t, s);
         if (e != cudaSuccess) return from_cuda(e);
         uint8_t* const gs = wsb + w.x_bytes + w.f_bytes;
@@ -369,6 +373,10 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         const int t = trace_begin(QL_KIND_ACT_QUANT, s);
         e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, nullptr, 0, y, ny, s);
         trace_end(t, s);
+    } else if (fmt == QL_FP8A8_B128_BF16) {
+        const int t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant_e4m3(x, M, K, rot, static_cast<uint8_t*>(xs), xf, nullptr, 0, y, ny, s);
+        trace_end(t, s);
     } else {
         const int t = trace_begin(QL_KIND_PREP_A16, s);
         e = launch_prep_a16(x, M, K, rot, x_order(fmt), static_cast<__half*>(xs), xf, y, ny, s);
@@ -376,7 +384,8 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
     }
     if (e != cudaSuccess) return from_cuda(e);
 
-    const size_t xelem = fmt == QL_I8A8_G128_BF16 ? 1 : 2;
+    const bool act8 = fmt == QL_I8A8_G128_BF16 || fmt == QL_FP8A8_B128_BF16;  // byte activations, scales [M][G]
+    const size_t xelem = act8 ? 1 : 2;
     for (int m0 = 0; m0 < M; m0 += 16) {
         for (int k0 = 0; k0 < K; k0 += kmax) {
             const int kc = K - k0 < kmax ? K - k0 : kmax;
@@ -385,7 +394,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
             a.scales = scales;
             a.zeros = zeros;
             a.xs = static_cast<const uint8_t*>(xs) + ((size_t)m0 * K + k0) * xelem;
-            a.xf = fmt == QL_I8A8_G128_BF16 ? xf + (size_t)m0 * G : xf + m0;
+            a.xf = act8 ? xf + (size_t)m0 * G : xf + m0;
             a.y = y + (size_t)m0 * N;
             a.acc = nullptr;
             a.M = M - m0 < 16 ? M - m0 : 16;
@@ -460,7 +469,7 @@ int act_quant_e4m3_g128(const void* x, int M, int K, int rotate, uint8_t* q, flo
     if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return QL_EALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int t = trace_begin(QL_KIND_ACT_QUANT, st);
-    const cudaError_t e = launch_act_quant_e4m3(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, st);
+    const cudaError_t e = launch_act_quant_e4m3(x, M, K, rotate ? 1 : 0, q, s, nullptr, 0, nullptr, 0, st);
     trace_end(t, st);
     return from_cuda(e);
 }

@@ -57,7 +57,7 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
                              float* yz, long long nz, cudaStream_t s);
 // The same rule with E4M3 codes (448 for 127), written as bytes.
 cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
-                                  cudaStream_t s);
+                                  float* yz, long long nz, cudaStream_t s);
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s);
 // The same for the grouped expert GEMM: token t's f16 row goes to rows

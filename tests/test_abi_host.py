@@ -70,7 +70,10 @@ def test_packed_sizes_and_workspace_reject_bad_args(L):
     assert Q.qlinear_workspace_size(3, 2 | 1, 16, 21504, 5376) == Q.qlinear_workspace_size(3, 1, 16, 21504, 5376)
     assert Q.qlinear_workspace_size(1, 0, 16, 21504, 5376) >= 16 * 5376 * 2
     assert Q.qlinear_workspace_size(3, 1, 16, 21504, 5376) >= 16 * 5376 + 16 * 42 * 4
-    assert Q.qlinear_workspace_size(7, 1, 1, 21504, 5376) >= 5376 + 42 * 128 * 4 + 42 * 21504 * 4
+    # format 7: E4M3 codes and their scales for the decode kernel (M <= 16); from 17 rows the tensor-core
+    # GEMM also takes transposed scales and its weight-scale scratch
+    assert 5376 + 42 * 4 <= Q.qlinear_workspace_size(7, 1, 1, 21504, 5376) < 42 * 21504 * 4
+    assert Q.qlinear_workspace_size(7, 1, 17, 21504, 5376) >= 17 * 5376 + 42 * 128 * 4 + 42 * 21504 * 4
     # int5 switches to int8 activations at 65 rows: the workspace then holds the activation codes, their
     # transposed scales, the GEMM's weight scales and the weight converted to int8 codes (N * K bytes)
     assert Q.qlinear_workspace_size(5, 0, 64, 21504, 5376) < 21504 * 5376
