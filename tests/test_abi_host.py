@@ -102,6 +102,14 @@ def test_forward_validation_statuses(L):
     assert call(x=None) == 1
     assert call(fmt=5) == 1  # int5 needs zeros
     assert call(K=32768 + 128) == 2  # a 16-bit activation row no longer fits in shared memory
+    # byte activations have no such limit: W8A8, format 7 (decode and prefill) and int5 from 65 rows on
+    # pass that check and stop at the (too small) workspace instead
+    big = 32768 + 128
+    assert call(fmt=3, K=big, wsb=16) == 4
+    assert call(fmt=7, K=big, M=1, wsb=16) == 4
+    assert call(fmt=7, K=big, M=17, wsb=16) == 4
+    assert call(fmt=5, z=P(A), K=big, M=64) == 2
+    assert call(fmt=5, z=P(A), K=big, M=65, wsb=16) == 4
     assert call(x=P(A + 8)) == 3
     assert call(y=P(A + 4)) == 3
     assert call(ws=None) == 4
