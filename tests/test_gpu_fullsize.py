@@ -136,3 +136,21 @@ def test_prefill_w8a8_full(Q):
     assert np.array_equal(host_u8(c).reshape(N_FULL, K_FULL)[rows], qr.view(np.uint8))
     ref = O.forward(d["x"], qr.view(np.uint8), sr, None, Q.I8A8_G128_BF16, 0, len(rows))
     assert_close(y[:, rows], ref, "prefill W8A8 full")
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_fp8a8_decode_full(Q, M):
+    """Format 7 (fp8 weights, E4M3 activations) at decode sizes, on the weight-streaming kernel.  A
+    weight block's scale depends on all of its 128 rows, so whole blocks are sampled."""
+    W = dev(synth.weight_rows(0, "W", K_FULL, 0, N_FULL))
+    c, s, _ = Q.qlinear_pack(Q.FP8A8_B128_BF16, N_FULL, K_FULL, W=W)
+    del W
+    x = synth.activations(0, f"x_M{M}", M, K_FULL)
+    y = Q.qlinear_forward(dev_bf16(x), c, s, None, Q.FP8A8_B128_BF16, N_FULL).cpu().numpy()
+    blocks = [0, 97, N_FULL // 128 - 1]
+    rows = np.concatenate([np.arange(128 * b, 128 * b + 128) for b in blocks])
+    qr, sr = O.quant_fp8_b128(np.concatenate([synth.weight_rows(0, "W", K_FULL, 128 * b, 128) for b in blocks]))
+    assert np.array_equal(host_u8(c).reshape(N_FULL, K_FULL)[rows], qr)
+    assert np.array_equal(host_u8(s).view(np.uint16).reshape(N_FULL // 128, K_FULL // 128)[blocks], sr)
+    ref = O.forward(x, qr, sr, None, Q.FP8A8_B128_BF16, 0, len(rows))
+    assert_close(y[:, rows], ref, f"format 7 decode M={M}")
