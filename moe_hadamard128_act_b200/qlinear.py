@@ -152,8 +152,10 @@ def qlinear_pack(fmt: int, N: int, K: int, W: torch.Tensor | None = None, codes:
                  scales: torch.Tensor | None = None, zeros: torch.Tensor | None = None, flags: int = 0,
                  stream=None):
     """Pack a weight: RTN-quantise fp32 W [N, K], or bit-pack given codes with
-    their scales (and int5 zeros).  Returns (codes, scales, zeros) as uint8
-    tensors of the packed byte sizes (zeros is None except for int5)."""
+    their scales (and int5 zeros).  flags: HADAMARD quantises in the rotated
+    domain; SCALE_SEARCH (int8 formats, from W) takes each group's best of 21
+    scales instead of round to nearest's.  Returns (codes, scales, zeros) as
+    uint8 tensors of the packed byte sizes (zeros is None except for int5)."""
     dev = (W if W is not None else codes).device
     cb, sb, zb = qlinear_packed_sizes(fmt, N, K)
     c_out, s_out = _empty(cb, dev), _empty(sb, dev)
