@@ -578,12 +578,14 @@ def test_forward_int5_switches_to_w5a8_above_64_rows(had):
         y8, acc8 = O.forward(x, q8.view(np.uint8), s_bf16, None, O.I8A8_G128_BF16, had, N, want_acc=True)
         assert np.array_equal(acc5, acc8) and np.array_equal(y5, y8)
         assert np.abs(acc5).max() <= 128 * 127 * 31
-    # at 64 rows: bf16 x (rotated with the flag) times the dequantised weight, no activation codes
-    x = O.bf16_encode(rng.standard_normal((65, K)))
+    # at the card's last f16 row count: bf16 x (rotated with the flag) times the dequantised weight
+    last = FACTS["int5_f16_activation_max_rows"]["value"]
+    assert last == 64
+    x = O.bf16_encode(rng.standard_normal((last + 1, K)))
     xr = O.hadamard128_rotate(x) if had else x
     W = O.dequant(O.I5Z_G128_F16, packed, s_f16, z5, N, K)
-    y64 = O.forward(x[:64], packed, s_f16, z5, O.I5Z_G128_F16, had, N)
-    exact = O.bf16_decode(xr[:64]) @ W.T
+    y64 = O.forward(x[:last], packed, s_f16, z5, O.I5Z_G128_F16, had, N)
+    exact = O.bf16_decode(xr[:last]) @ W.T
     assert np.allclose(y64, exact, rtol=1e-12, atol=1e-12 * np.abs(exact).max())
     # one row more switches the whole call to int8 activations: close to, but not, the weight-only product
     y65 = O.forward(x, packed, s_f16, z5, O.I5Z_G128_F16, had, N)
