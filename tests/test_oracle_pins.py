@@ -635,20 +635,28 @@ def test_moe_permute_brute_force():
     assert bad == 1 and counts[0] == 39 and offsets[1] == 39
 
 
-def test_moe_gate_up_reduces_to_dense():
-    T, E, N, K, topk = 5, 6, 48, 256, 3
-    ids = np.stack([RNG.permutation(E)[:topk] for _ in range(T)]).astype(np.int32)
-    x = O.bf16_encode(RNG.standard_normal((T, K)))
+@pytest.mark.parametrize("fmt,had", [(1, 1), (1, 0), (2, 1), (6, 0), (6, 1)])
+def test_moe_gate_up_reduces_to_dense(fmt, had):
+    # every expert format the grouped path takes: int8 with bf16 or f16 scales, fp8 128 x 128 blocks
+    # (N = 200: a ragged second block)
+    T, E, N, K, topk = 5, 6, 200 if fmt == 6 else 48, 256, 3
+    rng = np.random.default_rng(83 + fmt + 10 * had)
+    ids = np.stack([rng.permutation(E)[:topk] for _ in range(T)]).astype(np.int32)
+    x = O.bf16_encode(rng.standard_normal((T, K)))
     qs, ss = [], []
     for e in range(E):
-        q, s = O.quant_i8_g128((RNG.standard_normal((N, K)) * 0.02).astype(np.float32), hadamard=True)
+        W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        if fmt == 6:
+            q, s = O.quant_fp8_b128(W, hadamard=bool(had))
+        else:
+            q, s = O.quant_i8_g128(W, hadamard=bool(had), scale_f16=(fmt == 2))
         qs.append(q)
         ss.append(s)
     codes = np.stack(qs).view(np.uint8)
     scales = np.stack(ss)
-    out = O.moe_gate_up(x, ids, codes, scales, O.I8_G128_BF16, O.HADAMARD, E, N)
+    out = O.moe_gate_up(x, ids, codes, scales, fmt, had, E, N)
     for t in range(T):
         for j in range(topk):
             e = ids[t, j]
-            dense = O.forward(x[t:t + 1], codes[e], scales[e], None, O.I8_G128_BF16, O.HADAMARD, N)
+            dense = O.forward(x[t:t + 1], codes[e], scales[e], None, fmt, had, N)
             assert np.array_equal(out[t, j], dense[0])
