@@ -16,7 +16,11 @@
  *   "Gemma4-26B-CIRU-AMD-STRIX-vLLM", "What is in the release": symmetric
  *     int4, group 64, bf16 scales, 4.25 bits per quantized weight.
  *   "keptn/gemma4-31b-w5", table "Format" and "How it was made" step 4:
- *     int5 codes with a u8 zero point and one f16 scale per 128 weights.
+ *     int5 codes with a u8 zero point and one f16 scale per 128 weights;
+ *     activations 16-bit up to 64 rows, int8 per token and 128 above.
+ *   The i8 card's recipe marks the experts' quantiser "rule=search" (round to
+ *     nearest with a scale search); the candidates and the measure are a
+ *     reading of this build, stated at qo_scale_search_group.
  *   "keptn/gemma4-12b-i8g", table "Format": int8 weights with a bf16 scale
  *     per 128, activations int8 with one scale per token and 128 values.
  *   The FP8-activation variant of the fp8 container (format 7) takes the
