@@ -51,8 +51,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "moe_decode",
-                                             "moe_decode_t1", "moe_prefill"],
+    p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "prefill_w5a8",
+                                          "moe_decode", "moe_decode_t1", "moe_prefill"],
                    default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
@@ -453,6 +453,9 @@ def ncu_case(name):
     N = 21504, K = 5376; about 0.6 GB on the device), four forwards; the tcgen05
     GEMM (k_prefill_w8a8, which also runs format 7, / k_prefill_a16) is launch
     1..4 of its name.
+    prefill_w5a8: the int5 weight of the W5A16 workload with M = 2048 tokens
+    (int8 activations), four forwards: act quant, scale prep, int5 -> int8 code
+    conversion (k_prefill_i5_codes) and the W8A8 GEMM each launch four times.
     moe_decode / moe_decode_t1 / moe_prefill: the MoE gate_up experts (128 x
     [1408, 2816] int8 g128 bf16, Hadamard domain; about 0.5 GB), top-8 routing
     of T = 16 / 1 / 2048 tokens, four calls of moe_gate_up (activation
@@ -480,6 +483,19 @@ def ncu_case(name):
         y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
         for i in range(4):
             Q.moe_gate_up(x, idt, codes, scales, E, Ne, y=y)
+        torch.cuda.synchronize()
+        st, bits = Q.ql_get_device_error()
+        assert st == 0, bits
+        print(f"ncu case {name} done")
+        return
+    if name == "prefill_w5a8":
+        d = synth.w5a16(2048)
+        c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
+                                 scales=torch.from_numpy(d["scales"]).to(dev), zeros=torch.from_numpy(d["zeros"]).to(dev))
+        x = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((2048, N_FULL), dtype=torch.float32, device=dev)
+        for i in range(4):
+            Q.qlinear_forward(x, c, s, z, Q.I5Z_G128_F16, N_FULL, y=y)
         torch.cuda.synchronize()
         st, bits = Q.ql_get_device_error()
         assert st == 0, bits
