@@ -389,6 +389,24 @@ def test_quant_i8_search_matrix_is_groupwise_on_rotated_rows():
                 assert np.array_equal(q[n, g * 128:(g + 1) * 128], qg) and s[n, g] == sg and ci[n, g] == ig
 
 
+@pytest.mark.parametrize("which", ["fp8", "i4", "i8"])
+def test_quant_hadamard_flag_is_the_rotated_rows(which):
+    # with the flag, every quantiser sees each 128-block of each row through the (separately pinned)
+    # spec transform: the same as quantising the rotated rows without it
+    rng = np.random.default_rng(89)
+    N, K = 136, 384  # a ragged second fp8 row block
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[3, 10] = 0.4  # an outlier the rotation spreads over its block
+    R = np.concatenate([np.stack([O.fwht128_spec_f32(W[n, g * 128:(g + 1) * 128]) for g in range(K // 128)]).ravel()[None]
+                        for n in range(N)]).astype(np.float32)
+    quant = {"fp8": O.quant_fp8_b128, "i4": O.quant_i4_g64, "i8": O.quant_i8_g128}[which]
+    q1, s1 = quant(W, hadamard=True)
+    q2, s2 = quant(R)
+    assert np.array_equal(q1, q2) and np.array_equal(s1, s2)
+    q0, s0 = quant(W)
+    assert not np.array_equal(s0, s1)  # and the flag is not a no-op
+
+
 def test_quant_fp8_block_rule():
     N, K = 200, 256  # a ragged last row block (72 rows)
     W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
