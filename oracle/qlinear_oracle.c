@@ -820,13 +820,47 @@ int qo_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, 
  * x rotated once per token (bf16, as qo_hadamard128_rotate) when QO_HADAMARD
  * is set.  The routing weights are not applied: they belong after the down
  * projection, which this layer does not compute.  Pairs with an invalid id
- * leave their output row untouched. */
+ * leave their output row untouched.
+ * Format 7 experts (the fp8 container's E4M3 weights with E4M3 activations,
+ * "gemma4-26b-a4b-dflash-fp8" README, table "Weights", with the activation
+ * rule of "keptn/gemma4-12b-i8g" applied to E4M3 codes -- a reading of this
+ * build): each token is quantised once, per 128 values (rotated first with
+ * QO_HADAMARD), and every pair's output is the format-7 sum
+ * sum_g sx[t,g] * sw_e[n/128,g] * sum_{k in g} e4m3(qx) * e4m3(qw). */
 int qo_moe_gate_up(const uint16_t* x, const int32_t* ids, int T, int topk, int E, int N, int K, int fmt,
                    int flags, const uint8_t* codes, const uint16_t* scales, double* out)
 {
-    if (fmt != QO_I8_G128_BF16 && fmt != QO_I8_G128_F16 && fmt != QO_FP8_B128_BF16) return 1;
+    if (fmt != QO_I8_G128_BF16 && fmt != QO_I8_G128_F16 && fmt != QO_FP8_B128_BF16 && fmt != QO_FP8A8_B128_BF16)
+        return 1;
     size_t cs, ss, zs;
     qo_packed_sizes(fmt, N, K, &cs, &ss, &zs);
+    if (fmt == QO_FP8A8_B128_BF16) {
+        const int G = K / 128;
+        uint8_t* qx = (uint8_t*)malloc((size_t)T * K);
+        float* sx = (float*)malloc(sizeof(float) * (size_t)T * G);
+        qo_act_quant_e4m3_g128(x, T, K, flags & QO_HADAMARD, qx, sx);
+#pragma omp parallel for schedule(dynamic)
+        for (int p = 0; p < T * topk; ++p) {
+            const int e = ids[p], t = p / topk;
+            if (e < 0 || e >= E) continue;
+            const uint8_t* ce = codes + (size_t)e * cs;
+            const uint16_t* se = scales + (size_t)e * (ss / 2);
+            for (int n = 0; n < N; ++n) {
+                double sum = 0.0;
+                for (int g = 0; g < G; ++g) {
+                    double part = 0.0;
+                    for (int i = 0; i < 128; ++i)
+                        part += qo_e4m3_decode(qx[(size_t)t * K + g * 128 + i]) *
+                                qo_e4m3_decode(ce[(size_t)n * K + g * 128 + i]);
+                    sum += (double)sx[(size_t)t * G + g] * qo_bf16_decode(se[(size_t)(n / 128) * G + g]) * part;
+                }
+                out[(size_t)p * N + n] = sum;
+            }
+        }
+        free(qx);
+        free(sx);
+        return 0;
+    }
     double* xt = (double*)malloc(sizeof(double) * (size_t)T * K);
     uint16_t* xr = (uint16_t*)malloc(2 * (size_t)T * K);
     if (flags & QO_HADAMARD) qo_hadamard128_rotate(x, T, K, xr);

@@ -653,18 +653,18 @@ def test_moe_permute_brute_force():
     assert bad == 1 and counts[0] == 39 and offsets[1] == 39
 
 
-@pytest.mark.parametrize("fmt,had", [(1, 1), (1, 0), (2, 1), (6, 0), (6, 1)])
+@pytest.mark.parametrize("fmt,had", [(1, 1), (1, 0), (2, 1), (6, 0), (6, 1), (7, 0), (7, 1)])
 def test_moe_gate_up_reduces_to_dense(fmt, had):
     # every expert format the grouped path takes: int8 with bf16 or f16 scales, fp8 128 x 128 blocks
-    # (N = 200: a ragged second block)
-    T, E, N, K, topk = 5, 6, 200 if fmt == 6 else 48, 256, 3
+    # (N = 200: a ragged second block), and the fp8 blocks with E4M3 activations (format 7)
+    T, E, N, K, topk = 5, 6, 200 if fmt in (6, 7) else 48, 256, 3
     rng = np.random.default_rng(83 + fmt + 10 * had)
     ids = np.stack([rng.permutation(E)[:topk] for _ in range(T)]).astype(np.int32)
     x = O.bf16_encode(rng.standard_normal((T, K)))
     qs, ss = [], []
     for e in range(E):
         W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
-        if fmt == 6:
+        if fmt in (6, 7):
             q, s = O.quant_fp8_b128(W, hadamard=bool(had))
         else:
             q, s = O.quant_i8_g128(W, hadamard=bool(had), scale_f16=(fmt == 2))
