@@ -99,6 +99,10 @@ def lib():
         L.qo_moe_permute.argtypes = [_c_p, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]
         L.qo_moe_gate_up.restype = _c_i
         L.qo_moe_gate_up.argtypes = [_c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p, _c_p]
+        L.qo_gelu_tanh.restype = ctypes.c_double
+        L.qo_gelu_tanh.argtypes = [ctypes.c_double]
+        L.qo_moe_down_combine.restype = _c_i
+        L.qo_moe_down_combine.argtypes = [_c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_p, _c_p]
         _lib = L
     return _lib
 
@@ -339,4 +343,29 @@ def moe_gate_up(x_bits, ids, codes, scales, fmt: int, flags: int, E: int, N: int
     rc = lib().qo_moe_gate_up(_p(x), _p(ids), T, topk, E, N, K, fmt, flags, _p(codes), _p(scales), _p(out))
     if rc:
         raise ValueError(f"oracle moe_gate_up rejected format {fmt}")
+    return out
+
+
+def gelu_tanh(v) -> np.ndarray:
+    """The tanh form of GELU in fp64, element by element."""
+    v = np.ascontiguousarray(v, np.float64)
+    out = np.empty_like(v)
+    f = lib().qo_gelu_tanh
+    for i, x in enumerate(v.ravel()):
+        out.ravel()[i] = f(float(x))
+    return out
+
+
+def moe_down_combine(h, ids, weights, wd_bits, E: int):
+    """out [T, K] fp64: per pair gelu(gate) * up of its gate_up row h [T, topk, 2I] (fp32), through its
+    expert's bf16 down weight wd [E, K, I], summed over the slots with the routing weights."""
+    h = _c(h, np.float32)
+    ids = _c(ids, np.int32)
+    w = _c(weights, np.float32)
+    wd = _c(wd_bits, np.uint16)
+    T, topk = ids.shape
+    I = h.shape[-1] // 2
+    K = wd.shape[1]
+    out = np.empty((T, K), np.float64)
+    lib().qo_moe_down_combine(_p(h), _p(ids), _p(w), T, topk, E, I, K, _p(wd), _p(out))
     return out

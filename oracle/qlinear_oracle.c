@@ -27,6 +27,10 @@
  *     weights of "gemma4-26b-a4b-dflash-fp8" unchanged and quantises the
  *     activations as the int8 cards do -- one fp32 scale per token and 128
  *     values -- but to E4M3 codes: a reading of this build, not a card's.
+ *   The experts' down projections and the router stay bf16 ("gemma4-26b-
+ *     a4b-dflash-i8" README, table "Weights"); the activation between the
+ *     gate and up halves and the routing-weighted combine are not on the
+ *     cards: qo_moe_down_combine states the reading taken.
  *
  * Where the cards leave the arithmetic open, the oracle takes one plain
  * reading and states it at the function that implements it.  Everything is
@@ -888,5 +892,50 @@ int qo_moe_gate_up(const uint16_t* x, const int32_t* ids, int T, int topk, int E
         free(w);
     }
     free(xt);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MoE down projection and combine ("gemma4-26b-a4b-dflash-i8", Weights:     */
+/* the routed experts' down projections bf16 as the checkpoint ships them).  */
+/* ------------------------------------------------------------------------ */
+
+/* GELU with the tanh approximation, the activation of the Gemma family's
+ * gated MLP (the cards name no activation; this is the reading taken):
+ * gelu(v) = 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), in fp64. */
+double qo_gelu_tanh(double v)
+{
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    return 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+}
+
+/* For every (token, slot) pair p = t * topk + j routed to expert e = ids[p]:
+ * h[p] is its gate_up output (fp32, [2I]: the gate half first, then the up
+ * half, the row order of the packed experts), a_i = gelu(h[p][i]) * h[p][I + i]
+ * (fp64), d[n] = sum_i a_i * wd_e[n][i] with the expert's bf16 down weight
+ * wd_e [K][I] decoded exactly, and out[t][n] = sum_j w[t][j] * d_(t,j)[n],
+ * the routing weights as given (not renormalised), summed in slot order.
+ * Pairs with an id outside [0, E) add nothing.  out fp64 [T][K]. */
+int qo_moe_down_combine(const float* h, const int32_t* ids, const float* w, int T, int topk, int E, int I, int K,
+                        const uint16_t* wd, double* out)
+{
+#pragma omp parallel for schedule(dynamic)
+    for (int t = 0; t < T; ++t) {
+        double* a = (double*)malloc(sizeof(double) * (size_t)I);
+        for (int n = 0; n < K; ++n) out[(size_t)t * K + n] = 0.0;
+        for (int j = 0; j < topk; ++j) {
+            const int p = t * topk + j, e = ids[p];
+            if (e < 0 || e >= E) continue;
+            const float* hp = h + (size_t)p * 2 * I;
+            for (int i = 0; i < I; ++i) a[i] = qo_gelu_tanh((double)hp[i]) * (double)hp[I + i];
+            const uint16_t* we = wd + (size_t)e * K * I;
+            for (int n = 0; n < K; ++n) {
+                double d = 0.0;
+                for (int i = 0; i < I; ++i) d += a[i] * qo_bf16_decode(we[(size_t)n * I + i]);
+                out[(size_t)t * K + n] += (double)w[p] * d;
+            }
+        }
+        free(a);
+    }
     return 0;
 }

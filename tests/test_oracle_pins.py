@@ -678,3 +678,64 @@ def test_moe_gate_up_reduces_to_dense(fmt, had):
             e = ids[t, j]
             dense = O.forward(x[t:t + 1], codes[e], scales[e], None, fmt, had, N)
             assert np.array_equal(out[t, j], dense[0])
+
+
+# --------------------------------------------------------------------------
+# MoE down projection and combine (reading: GeGLU with the tanh form of GELU,
+# the gate half first; bf16 down weights; routing weights applied as given)
+# --------------------------------------------------------------------------
+def test_gelu_tanh_against_torch_and_identities():
+    import torch
+    v = np.concatenate([np.linspace(-12, 12, 401), RNG.standard_normal(300) * 3, [0.0, 1e-30, -1e-30, 40.0, -40.0]])
+    ours = O.gelu_tanh(v)
+    ref = torch.nn.functional.gelu(torch.from_numpy(v), approximate="tanh").numpy()
+    # 1 + tanh(u) cancels for negative v, so both forms agree to a few ulp of |v|, not of the result
+    assert np.all(np.abs(ours - ref) <= 1e-14 * np.maximum(np.abs(v), np.abs(ref)))
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert np.allclose(ours - O.gelu_tanh(-v), v, rtol=1e-14, atol=1e-14)  # gelu(x) - gelu(-x) = x
+    assert O.gelu_tanh(np.array([40.0]))[0] == 40.0 and O.gelu_tanh(np.array([-40.0]))[0] == 0.0
+
+
+def _down_case(T, topk, E, I, K, seed):
+    rng = np.random.default_rng(seed)
+    ids = np.stack([rng.permutation(E)[:topk] for _ in range(T)]).astype(np.int32)
+    w = rng.random((T, topk)).astype(np.float32)
+    h = (rng.standard_normal((T, topk, 2 * I)) * 2).astype(np.float32)
+    wd = O.bf16_encode(rng.standard_normal((E, K, I)) * 0.02)
+    return ids, w, h, wd
+
+
+def test_moe_down_combine_brute_force():
+    import torch
+    T, topk, E, I, K = 3, 4, 6, 64, 48
+    ids, w, h, wd = _down_case(T, topk, E, I, K, 5)
+    out = O.moe_down_combine(h, ids, w, wd, E)
+    hd = torch.from_numpy(h.astype(np.float64))
+    a = (torch.nn.functional.gelu(hd[..., :I], approximate="tanh") * hd[..., I:]).numpy()  # [T, topk, I]
+    wdec = torch.from_numpy(wd.view(np.int16)).view(torch.bfloat16).double().numpy()        # [E, K, I]
+    ref = np.zeros((T, K))
+    for t in range(T):
+        for j in range(topk):
+            ref[t] += float(w[t, j]) * (wdec[ids[t, j]] @ a[t, j])
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_moe_down_combine_invariants():
+    T, topk, E, I, K = 2, 3, 5, 32, 40
+    ids, w, h, wd = _down_case(T, topk, E, I, K, 6)
+    base = O.moe_down_combine(h, ids, w, wd, E)
+    # linear in the routing weights: scaling them by a power of two scales the output exactly
+    assert np.array_equal(O.moe_down_combine(h, ids, w * 4, wd, E), base * 4)
+    # one-hot weights pick one slot: the sum of the one-hot outputs is the output
+    parts = []
+    for j in range(topk):
+        oh = np.zeros_like(w)
+        oh[:, j] = w[:, j]
+        parts.append(O.moe_down_combine(h, ids, oh, wd, E))
+    assert np.allclose(sum(parts), base, rtol=1e-13, atol=1e-15)
+    # a pair routed to no expert adds nothing; an up half of zeros silences its slot
+    bad = ids.copy()
+    bad[0, 1] = E + 3
+    hz = h.copy()
+    hz[0, 1, I:] = 0.0
+    assert np.array_equal(O.moe_down_combine(h, bad, w, wd, E), O.moe_down_combine(hz, ids, w, wd, E))
