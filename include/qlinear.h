@@ -170,6 +170,20 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
  * [N, K] (device).  Runs the same integer MMA path as qlinear_forward. */
 int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int K, int32_t* acc, void* stream);
 
+/* qlinear_gemm_a8 -- the decode GEMM alone, on activations that are already
+ * quantised per token per 128 values ("keptn/gemma4-12b-i8g", table "Format":
+ * int8 activations with one scale per token per 128), for callers whose
+ * previous kernel emits them:
+ *   y[m, n] (+)= sum_g sx[m, g] * s_w[n, g] * sum_{k in g} qx[m, k] * qw[n, k].
+ * fmt QL_I8A8_G128_BF16: qx int8 [M, K] as act_quant_i8_g128 makes it, each
+ * group's integer sum exact; fmt QL_FP8A8_B128_BF16: qx E4M3 bytes [M, K] as
+ * act_quant_e4m3_g128 makes it, s_w the weight's 128 x 128 block scale.  sx
+ * fp32 [M, K/128].  W_packed, scales: the packed weight.  M <= 16 (the decode
+ * shapes; larger M returns QL_EUNSUPPORTED).  accumulate != 0 adds the product
+ * to y; accumulate == 0 overwrites y.  No workspace; y fp32 [M, N]. */
+int qlinear_gemm_a8(const void* qx, const float* sx, const void* W_packed, const void* scales, int fmt, int M, int N,
+                    int K, float* y, int accumulate, void* stream);
+
 /* act_quant_i8_g128 -- per token per 128 values ("keptn/gemma4-12b-i8g",
  * table "Format"): on the fp32 group v (rotated as hadamard128_rotate but
  * NOT rounded to bf16 when rotate != 0), amax = max|v|, s = fp32(amax/127),
@@ -196,7 +210,9 @@ typedef struct {
     int E;              /* number of experts                                    */
     int N;              /* output rows per expert (gate and up halves together) */
     int K;              /* hidden size, multiple of 128                          */
-    int fmt;            /* QL_I8_G128_BF16, QL_I8_G128_F16 or QL_FP8_B128_BF16   */
+    int fmt;            /* QL_I8_G128_BF16, QL_I8_G128_F16, QL_FP8_B128_BF16 or
+                           QL_FP8A8_B128_BF16 (the fp8 experts with E4M3
+                           activations, quantised once per token)            */
     int flags;          /* QL_HADAMARD when the experts are in the rotated domain */
     const void* codes;  /* device, [E] consecutive packed weights of [N, K]      */
     const void* scales; /* device, [E] consecutive scale arrays                  */
@@ -216,7 +232,11 @@ int moe_workspace_size(const ql_experts* experts, int T, int topk, size_t* bytes
 /* moe_gate_up -- the routed experts' gate_up projection
  * ("gemma4-26b-a4b-dflash-i8", table "Weights"): for every pair (t, j),
  * y[t, j, :] = x~[t, :] . dequant(W_{topk_ids[t, j]})^T, where x~ is x
- * rotated once per token (bf16) when the experts carry QL_HADAMARD.
+ * rotated once per token (bf16) when the experts carry QL_HADAMARD.  With
+ * QL_FP8A8_B128_BF16 experts ("gemma4-26b-a4b-dflash-fp8" README, table
+ * "Weights", with E4M3 activations) x~ is instead each token quantised once
+ * as act_quant_e4m3_g128 does (rotated first with QL_HADAMARD), and
+ * y[t, j, n] = sum_g sx[t, g] * s_w[n / 128, g] * sum_{k in g} qx * qw.
  * x bf16 [T, K]; topk_ids int32 [T, topk]; y fp32 [T, topk, N], overwritten.
  * topk_weights (fp32 [T, topk], may be NULL) is accepted but not applied:
  * the routing weight belongs after the down projection.  Internally:
@@ -224,6 +244,36 @@ int moe_workspace_size(const ql_experts* experts, int T, int topk, size_t* bytes
  * output stores.  `experts` is a host pointer. */
 int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weights, const ql_experts* experts,
                 int T, int topk, float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Stacked bf16 down-projection weights of the routed experts. */
+typedef struct {
+    int E;               /* number of experts                                  */
+    int K;               /* hidden size: output rows of each down weight       */
+    int I;               /* intermediate size: the gate and up halves' width,  */
+                         /* multiple of 64                                      */
+    const void* weights; /* device, bf16 [E][K][I] (row-major, I contiguous)    */
+} ql_down_experts;
+
+/* Workspace bytes moe_down_combine needs. */
+int moe_down_workspace_size(const ql_down_experts* experts, int T, int topk, size_t* bytes);
+
+/* moe_down_combine -- the step after moe_gate_up: the routed experts' down
+ * projections, bf16 as the checkpoint ships them ("gemma4-26b-a4b-dflash-i8"
+ * README, table "Weights"), and the routing-weighted sum over each token's
+ * slots.  The cards give neither the activation nor the combine; this library
+ * takes the Gemma family's gated MLP:
+ *   a[t, j, i] = gelu(h[t, j, i]) * h[t, j, I + i],
+ *     gelu(v) = 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))),
+ *   out[t, n]  = sum_j topk_weights[t, j] * sum_i a[t, j, i] * W_{topk_ids[t, j]}[n, i].
+ * h fp32 [T, topk, 2I]: the gate_up output (gate half first, as moe_gate_up
+ * writes it); topk_ids int32 [T, topk]; topk_weights fp32 [T, topk], applied
+ * as given; out fp32 [T, K], overwritten.  a is formed in fp32 and the products
+ * keep fp32 precision (the bf16 tensor cores see a as three bf16 parts); the
+ * sums are accumulated in any order.  Pairs with an id outside [0, E) add
+ * nothing and set QL_DEVERR_EXPERT_ID.  `experts` is a host pointer. */
+int moe_down_combine(const float* h, const int32_t* topk_ids, const float* topk_weights,
+                     const ql_down_experts* experts, int T, int topk, float* out, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /* qlinear_forward_w8a8_noalloc -- the W8A8 forward of qlinear_forward
  * (fmt QL_I8A8_G128_BF16) for callers that cannot allocate device memory,
@@ -238,8 +288,10 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
  * and K <= QL_NOALLOC_MAX_K (270,336 bytes, held on every GPU that loads the
  * library until the process exits).  Larger M or K return QL_EUNSUPPORTED
  * before anything is launched.  The call allocates nothing.
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, which allocates nothing).  The first call on each
+ * device also sets the decode kernel's launch attributes once; make that first
+ * call before any stream capture.
  * All calls share the array: calls whose kernels may overlap on the GPU
  * (other streams, other host threads) race on it and must be serialised by
  * the caller.  Nothing in the array needs to start at zero; each call
@@ -267,7 +319,9 @@ enum {
     QL_KIND_MOE_GEMM = 6,    /* grouped expert GEMM with fused un-permute        */
     QL_KIND_PACK = 7,        /* weight packing                                  */
     QL_KIND_PREFILL = 8,     /* tensor-core prefill GEMM                        */
-    QL_KIND_PREFILL_PREP = 9 /* weight scales transposed for the prefill GEMM   */
+    QL_KIND_PREFILL_PREP = 9, /* weight scales transposed for the prefill GEMM  */
+    QL_KIND_MOE_ACT = 10,     /* gelu(gate) * up ahead of the down projection   */
+    QL_KIND_MOE_DOWN = 11     /* experts' down projection with the combine       */
 };
 int ql_trace_enable(int capacity);
 int ql_trace_read(int* kinds, float* ms, int max, int* count);

@@ -48,10 +48,14 @@ __device__ __forceinline__ void zero_fill(float* y, long long n) {
 
 // s = fp32(amax / 127), q = clamp(rne(fp32(v * fp32(127 / amax))), -127, 127);
 // with E4M3 set, the E4M3 rule (448 for 127, codes by the hardware conversion).
+// With inv != null (the grouped expert GEMM) token t's codes and scales go to
+// rows inv[t * topk + j] of q and sxT (j < topk, negative entries skipped)
+// instead of row t: the permuted order.
 template <bool E4M3>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bfloat16* x, int M, int K, int rotate,
                                                                    int8_t* q, float* sx, float* sxT, int Mp,
-                                                                   float* yz, long long nz) {
+                                                                   float* yz, long long nz, const int32_t* inv,
+                                                                   int topk) {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
     const int lane = threadIdx.x & 31;
@@ -64,6 +68,16 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
         if (rotate) fwht128_warp(v, lane);
         float s;
         const uint32_t packed = E4M3 ? quant_e4m3_group_warp(v, &s) : quant_i8_group_warp(v, &s);
+        if (inv) {
+            const long long t = u / G, g = u % G;
+            for (int j = 0; j < topk; ++j) {
+                const int r = __ldg(inv + t * topk + j);
+                if (r < 0) continue;
+                *reinterpret_cast<uint32_t*>(q + (long long)r * K + g * 128 + 4 * lane) = packed;
+                if (lane == 0) sxT[g * Mp + r] = s;
+            }
+            continue;
+        }
         *reinterpret_cast<uint32_t*>(q + off) = packed;
         if (lane == 0) {
             if (sx) sx[u] = s;                                 // [M][G] row-major: u = m * G + g
@@ -164,6 +178,59 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
     }
 }
 
+// The activation between the experts' gate_up and down projections: for each
+// (token, slot) pair p routed to an expert, a_i = gelu(h[p][i]) * h[p][I + i]
+// in fp32, where h is the pair's gate_up output (gate half first) and gelu is
+// the tanh form v * sigmoid(2 sqrt(2/pi) (v + 0.044715 v^3)), written with the
+// logistic function so that nothing cancels for negative v.  a is stored as
+// three bf16 planes a0 = bf16(a), a1 = bf16(a - a0), a2 = bf16(a - a0 - a1)
+// (each difference exact in fp32), whose sum is a to within 2^-24 |a|, so the
+// bf16 tensor-core products of the down projection keep fp32 precision.  One
+// thread per 8 values (two 32-byte loads, three 16-byte stores).  Also zeroes
+// out[0 .. nz), which the down projection accumulates into.
+__device__ __forceinline__ float gelu_tanh_f32(float v) {
+    const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);  // sqrt(2 / pi) (v + 0.044715 v^3)
+    return v / (1.0f + expf(-2.0f * u));
+}
+
+__global__ void __launch_bounds__(256) k_moe_act(const float* h, const int32_t* ids, int P, int E, int I,
+                                                 __nv_bfloat16* act, float* out, long long nz) {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the down GEMM start its weight stream
+    zero_fill(out, nz);
+    const int I8 = I / 8;
+    const long long n = (long long)P * I8;
+    for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < n; u += (long long)gridDim.x * blockDim.x) {
+        const long long p = u / I8;
+        const int i0 = (int)(u - p * I8) * 8;
+        const int e = __ldg(ids + p);
+        if (e < 0 || e >= E) continue;
+        const float* hp = h + p * 2 * I;
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(hp + i0));
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(hp + i0 + 4));
+        const float4 u0 = __ldg(reinterpret_cast<const float4*>(hp + I + i0));
+        const float4 u1 = __ldg(reinterpret_cast<const float4*>(hp + I + i0 + 4));
+        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        uint32_t pl[3][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float r[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) r[k] = __fmul_rn(gelu_tanh_f32(gv[2 * q + k]), uv[2 * q + k]);
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(r[0], r[1]);
+                pl[l][q] = *reinterpret_cast<const uint32_t*>(&b);
+                r[0] = __fsub_rn(r[0], __low2float(b));
+                r[1] = __fsub_rn(r[1], __high2float(b));
+            }
+        }
+#pragma unroll
+        for (int l = 0; l < 3; ++l)
+            *reinterpret_cast<uint4*>(act + (p * 3 + l) * I + i0) = make_uint4(pl[l][0], pl[l][1], pl[l][2], pl[l][3]);
+    }
+}
+
 // The GEMM that follows these kernels runs with (nearly) all of the SM's
 // shared memory; asking for the same L1/shared split here avoids an SM
 // reconfiguration between the two launches.
@@ -211,18 +278,19 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
     if (e != cudaSuccess) return e;
     if ((e = prefer_max_shared(k_act_quant<false>)) != cudaSuccess) return e;
     k_act_quant<false><<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, sxT, Mp, yz, nz);
+        static_cast<const __nv_bfloat16*>(x), M, K, rotate, q, sx, sxT, Mp, yz, nz, nullptr, 0);
     return cudaGetLastError();
 }
 
 cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
-                                  float* yz, long long nz, cudaStream_t s) {
+                                  float* yz, long long nz, cudaStream_t s, const int32_t* inv, int topk) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
     if ((e = prefer_max_shared(k_act_quant<true>)) != cudaSuccess) return e;
     k_act_quant<true><<<grid_for((long long)M * (K / 128), di.sm_count), kWarpsPerBlock * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), M, K, rotate, reinterpret_cast<int8_t*>(q), sx, sxT, Mp, yz, nz);
+        static_cast<const __nv_bfloat16*>(x), M, K, rotate, reinterpret_cast<int8_t*>(q), sx, sxT, Mp, yz, nz, inv,
+        topk);
     return cudaGetLastError();
 }
 
@@ -260,4 +328,21 @@ cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, con
     return cudaGetLastError();
 }
 
+}  // namespace ql
+
+namespace ql {
+cudaError_t launch_moe_act(const float* h, const int32_t* ids, int P, int E, int I, __nv_bfloat16* act, float* out,
+                           long long nz, cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    if ((e = prefer_max_shared(k_moe_act)) != cudaSuccess) return e;
+    const long long work = (long long)P * (I / 8);
+    const long long zb = (nz + 1023) / 1024;
+    long long blocks = ((work > zb * 256 ? work : zb * 256) + 255) / 256;
+    if (blocks > 8LL * di.sm_count) blocks = 8LL * di.sm_count;
+    if (blocks < 1) blocks = 1;
+    k_moe_act<<<(unsigned)blocks, 256, 0, s>>>(h, ids, P, E, I, act, out, nz);
+    return cudaGetLastError();
+}
 }  // namespace ql

@@ -76,7 +76,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int NBUF = kTmemCols / PN;      // int32 accumulators in tensor memory
 constexpr int SCB = 8;                    // scale ring slots
 constexpr int SR = PSTAGES;               // step-commit ring: at least as long as the operand and accumulator rings
-constexpr int SC_BYTES = (PM + PN) * 4;   // s_x of the tile's rows, then s_w of its columns
+constexpr int SXS = PM + 4;               // s_x span of a scale slot: grouped tiles start on any row, so
+                                          // their copy starts at the 16-byte boundary below it
+constexpr int SC_BYTES = (SXS + PN) * 4;  // s_x of the tile's rows, then s_w of its columns
 constexpr int kEpiWarps = 16;             // warps 4..19; warps 0..3 (warpgroup 0) drive the pipeline
 constexpr int kPThreads = 32 * (4 + kEpiWarps);
 constexpr int WGC = PN / 4;               // columns per thread (per warp column quarter)
@@ -191,8 +193,8 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
                    "+r"(v[14]), "+r"(v[15]))
 
 struct PrefillArgs {
-    CUtensorMap tmA;    // int8 activations [M][K], box [128 rows][128 B]
-    CUtensorMap tmB;    // int8 weights [N][K], box [PN rows][128 B]
+    CUtensorMap tmA;    // int8 activations [M][K], box [128 rows][128 B] (grouped: [P permuted rows][K])
+    CUtensorMap tmB;    // int8 weights [N][K], box [PN rows][128 B] (grouped: the stacked experts [E * N][K])
     CUtensorMap tmY;    // y as bytes [M][4 N], row pitch 4 ldy, box [32 rows][4 YH B] (when ytma)
     const float* sxT;   // [G][Mp] activation scales (ACC: unused)
     const float* swT;   // [G][Np] weight scales as fp32 (ACC: unused)
@@ -202,7 +204,30 @@ struct PrefillArgs {
     int M, N, G, Mp, Np;
     int ytma;           // y is written by TMA stores (16-byte aligned rows)
     long long ldy;
+    // Grouped over experts (format 7 MoE): tiles (expert, first permuted row, rows, weight block
+    // of PN rows) from the permute, its count on the device; sxT [G][Mp] holds the permuted rows'
+    // scales, swT [E][G][Np] each expert's weight scales; row r of a tile goes to y[perm[r]][..N).
+    const MoeTile* tiles;
+    const int* n_tiles;
+    int max_tiles;
+    const int32_t* perm;
 };
+
+// Where tile t of the CTA's walk sits: activation rows m0 .. m0 + rows, weight
+// rows wrow .. + PN of the (stacked) weight matrix, the tile's weight block wb
+// and expert.  Dense tiles go weight-tile-major.
+struct TilePos {
+    int m0, rows, wrow, wb, expert;
+};
+template <bool GRP>
+__device__ __forceinline__ TilePos tile_pos(const PrefillArgs& a, int t, int MB) {
+    if (GRP) {
+        const MoeTile ti = a.tiles[t];
+        return TilePos{ti.row0, ti.rows, ti.expert * a.N + ti.wb * PN, ti.wb, ti.expert};
+    }
+    const int m0 = (t % MB) * PM;
+    return TilePos{m0, min(PM, a.M - m0), (t / MB) * PN, t / MB, 0};
+}
 
 // Registers: 640 threads launch with 96 each (61440).  Warpgroup 0 drops to
 // 24 (3072) and the four epilogue warpgroups rise to 112 (57344): 60416 in
@@ -210,9 +235,10 @@ struct PrefillArgs {
 constexpr int kRegsDriver = 24, kRegsEpi = 112;
 static_assert(128 * kRegsDriver + 32 * kEpiWarps * kRegsEpi <= kPThreads * 96, "register split");
 
-template <bool ACC, int KIND>
+template <bool ACC, int KIND, bool GRP = false>
 __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_constant__ PrefillArgs a) {
     static_assert(!ACC || KIND == kKindI8, "the integer group sums exist for int8 only");
+    static_assert(!GRP || (KIND == kKindE4M3 && !ACC), "the grouped mode runs the E4M3 experts");
     // Two MMA-issuing threads for E4M3, whose light epilogue leaves the issue as the
     // limit; one for int8, whose heavier epilogue needs the issue slots instead.
     constexpr int kIssuers = KIND == kKindE4M3 ? 2 : 1;
@@ -225,7 +251,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int MB = (a.M + PM - 1) / PM, NB = (a.N + PN - 1) / PN;
-    const int tiles = MB * NB;
+    const int tiles = GRP ? min(*a.n_tiles, a.max_tiles) : MB * NB;
     const int my_tiles = (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int G = a.G;
     const int total = my_tiles * G;  // steps of this CTA
@@ -258,7 +284,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmA) : "memory");
             asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmB) : "memory");
             int g = 0, t = blockIdx.x, k = 0;
-            int m0 = (t % MB) * PM, n0 = (t / MB) * PN;  // tile origin
+            TilePos tp = total > 0 ? tile_pos<GRP>(a, t, MB) : TilePos{0, 0, 0, 0, 0};
             for (; k < total; ++k) {
                 const int s = k % PSTAGES, c = k & (SCB - 1);
                 // the slot's previous operands (step k - PSTAGES) are free once that step's MMAs are done
@@ -269,19 +295,22 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 }
                 const uint32_t st = base + s * STAGE_BYTES, fb = bar(BAR_FULL + s);
                 mbar_expect_tx(fb, STAGE_BYTES);
-                tma_load_2d(st, &a.tmA, g * PKB, m0, fb);
-                tma_load_2d(st + A_BYTES, &a.tmB, g * PKB, n0, fb);
+                tma_load_2d(st, &a.tmA, g * PKB, tp.m0, fb);
+                tma_load_2d(st + A_BYTES, &a.tmB, g * PKB, tp.wrow, fb);
                 if (!ACC) {
                     const uint32_t ss = base + SC_OFF + c * SC_BYTES, sb = bar(BAR_SCF + c);
-                    mbar_expect_tx(sb, SC_BYTES);
-                    bulk_load(ss, a.sxT + (long long)g * a.Mp + m0, PM * 4, sb);
-                    bulk_load(ss + PM * 4, a.swT + (long long)g * a.Np + n0, PN * 4, sb);
+                    const int sx0 = GRP ? (tp.m0 & ~3) : tp.m0;  // 16-byte aligned start of the s_x copy
+                    const int sxn = GRP ? SXS : PM;
+                    const long long sw0 = GRP ? ((long long)tp.expert * G + g) * a.Np + (long long)tp.wb * PN
+                                              : (long long)g * a.Np + tp.wrow;
+                    mbar_expect_tx(sb, (unsigned)(sxn + PN) * 4);
+                    bulk_load(ss, a.sxT + (long long)g * a.Mp + sx0, sxn * 4, sb);
+                    bulk_load(ss + SXS * 4, a.swT + sw0, PN * 4, sb);
                 }
                 if (++g == G) {
                     g = 0;
                     t += gridDim.x;
-                    m0 = (t % MB) * PM;
-                    n0 = (t / MB) * PN;
+                    if (k + 1 < total) tp = tile_pos<GRP>(a, t, MB);
                 }
             }
             // Copies still in flight must land before the CTA's shared memory is released.
@@ -334,6 +363,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
 #pragma unroll
         for (int i = 0; i < WGC; ++i) yr[i] = 0.0f;
         int t = blockIdx.x, g = 0;
+        TilePos tp = total > 0 ? tile_pos<GRP>(a, t, MB) : TilePos{0, 0, 0, 0, 0};
         for (int k = 0; k < total; ++k) {
             const int b = k % NBUF, c = k & (SCB - 1);
             if (!mbar_wait(bar(BAR_STEP + k % SR), (k / SR) & 1) ||
@@ -346,7 +376,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             const float* scp = reinterpret_cast<const float*>(gb + SC_OFF + c * SC_BYTES);
             float sxr = 0.0f, kb = 0.0f;
             if (!ACC && KIND == kKindE4M3) {
-                sxr = scp[row];  // fp32 group sums: t = s_x * sum, no bias
+                sxr = scp[(GRP ? (tp.m0 & 3) : 0) + row];  // fp32 group sums: t = s_x * sum, no bias
             } else if (!ACC) {
                 // s_x cut to 22 significant bits: s_x * 12582912 is exact, so the first FMA is
                 // round(s_x * sum) (the accumulator bits read as fp32 are 12582912 + sum).
@@ -371,7 +401,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 // chunk, then one FMA per element (half packed, half scalar: both FMA pipes).
 #pragma unroll
                 for (int h = 0; h < NCH; ++h) {
-                    const float p = sxr * scp[PM + tcol + h * CW];
+                    const float p = sxr * scp[SXS + tcol + h * CW];
                     const float2 p2 = make_float2(p, p);
 #pragma unroll
                     for (int q = 0; q < CW / 4; ++q) {
@@ -404,7 +434,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                         for (int i = 0; i < CW; ++i)
                             if (n0 + i < a.N) a.acc[((long long)m * a.N + n0 + i) * G + g] = (int)cur[i];
                 } else if constexpr (KIND == kKindE4M3) {  // wide tiles: one s_x * s_w per chunk, as above
-                    const float p = sxr * scp[PM + tcol + h * CW];
+                    const float p = sxr * scp[SXS + tcol + h * CW];
                     const float2 p2 = make_float2(p, p);
 #pragma unroll
                     for (int q = 0; q < CW / 4; ++q) {
@@ -420,7 +450,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 } else {
                     // Weight scales read in place (volatile loads stay in their chunk instead of being
                     // hoisted, which would cost registers).
-                    const uint32_t swa = smem_u32(scp + PM + tcol + h * CW);
+                    const uint32_t swa = smem_u32(scp + SXS + tcol + h * CW);
 #pragma unroll
                     for (int q = 0; q < CW / 4; ++q) {
                         const uint4 cu = lds128(swa + 16 * q);
@@ -449,7 +479,25 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             }
 
             if (++g == G) {  // tile done: this thread's WGC columns of its row of y
-                if (!ACC && a.ytma) {
+                if constexpr (GRP) {  // row of the permuted order -> its (token, slot) row of y
+                    const int n0 = tp.wb * PN + tcol;
+                    if (row < tp.rows && n0 < a.N) {
+                        const int pair = __ldg(a.perm + tp.m0 + row);
+                        float* yrow = a.y + (long long)pair * a.ldy + n0;
+                        if (vec_ok && n0 + WGC <= a.N) {
+#pragma unroll
+                            for (int q = 0; q < WGC / 4; ++q)
+                                *reinterpret_cast<float4*>(yrow + 4 * q) =
+                                    make_float4(yr[4 * q], yr[4 * q + 1], yr[4 * q + 2], yr[4 * q + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < WGC; ++i)
+                                if (n0 + i < a.N) yrow[i] = yr[i];
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < WGC; ++i) yr[i] = 0.0f;
+                } else if (!ACC && a.ytma) {
                     const int r0 = (t % MB) * PM + sub * 32, n0 = (t / MB) * PN + tcol;
                     const uint32_t yb = base + Y_OFF + (uint32_t)(warp - 4) * Y_WARP_BYTES;
 #pragma unroll
@@ -490,6 +538,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
                 }
                 g = 0;
                 t += gridDim.x;
+                if (k + 1 < total) tp = tile_pos<GRP>(a, t, MB);
             }
         }
     }
@@ -559,20 +608,25 @@ __global__ void __launch_bounds__(256) k_prefill_i5_codes(const uint8_t* codes, 
 }
 
 // bf16 block scales [ceil(N/128)][G] -> fp32 [G][Np], each row's block scale
-// repeated for the 128 rows of its block; columns n >= N zero.
+// repeated for the 128 rows of its block; columns n >= N zero.  Expert e
+// (blockIdx.y) reads its scales at sw + e * ceil(N/128) * G and writes
+// swT + e * G * Np.
 __global__ void __launch_bounds__(256) k_prefill_prep_blk(const uint16_t* sw, int N, int G, int Np, float* swT) {
     const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
     if (i >= (long long)G * Np) return;
     const int g = (int)(i / Np), n = (int)(i - (long long)g * Np);
+    sw += (long long)blockIdx.y * ((N + 127) / 128) * G;
+    swT += (long long)blockIdx.y * G * Np;
     swT[i] = n < N ? __uint_as_float((uint32_t)sw[(long long)(n >> 7) * G + g] << 16) : 0.0f;
 }
 
 }  // namespace
 
-cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s) {
+cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s, int E) {
     const int G = K / 128, Np = prefill_pad_n(N);
     const long long n = (long long)G * Np;
-    k_prefill_prep_blk<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sw, N, G, Np, static_cast<float*>(scratch));
+    k_prefill_prep_blk<<<dim3((unsigned)((n + 255) / 256), (unsigned)E), 256, 0, s>>>(sw, N, G, Np,
+                                                                                      static_cast<float*>(scratch));
     return cudaGetLastError();
 }
 
@@ -636,6 +690,49 @@ cudaError_t launch_prefill_w8a8(const int8_t* qx, const float* sxT, const int8_t
     if (acc) k_prefill_w8a8<true, kKindI8><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
     else if (e4m3) k_prefill_w8a8<false, kKindE4M3><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
     else k_prefill_w8a8<false, kKindI8><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_e4m3_grouped(const uint8_t* qx, const float* sxT, int Mp, const uint8_t* codes,
+                                        const float* swT, int E, int N, int K, int rows_total, const MoeTile* tiles,
+                                        const int* n_tiles, int max_tiles, const int32_t* perm, float* y,
+                                        cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
+    if (Mp % 4 || (reinterpret_cast<uintptr_t>(sxT) & 15)) return cudaErrorInvalidValue;
+    PrefillArgs a;
+    if ((e = make_tmap_2d(qx, rows_total, K, K, PKB, PM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmA)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d(codes, (long long)E * N, K, K, PKB, PN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmB)) != cudaSuccess)
+        return e;
+    a.sxT = sxT;
+    a.swT = swT;
+    a.y = y;
+    a.acc = nullptr;
+    a.err = di.err_word;
+    a.M = rows_total;
+    a.N = N;
+    a.G = K / 128;
+    a.Mp = Mp;
+    a.Np = prefill_pad_n(N);
+    a.ldy = N;
+    a.ytma = 0;
+    a.tiles = tiles;
+    a.n_tiles = n_tiles;
+    a.max_tiles = max_tiles;
+    a.perm = perm;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        if ((e = cudaFuncSetAttribute(k_prefill_w8a8<false, kKindE4M3, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
+            return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    const int grid = max_tiles < di.sm_count ? max_tiles : di.sm_count;
+    k_prefill_w8a8<false, kKindE4M3, true><<<grid, kPThreads, SMEM_BYTES, s>>>(a);
     return cudaGetLastError();
 }
 

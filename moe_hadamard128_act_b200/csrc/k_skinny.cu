@@ -64,6 +64,12 @@ struct Regs<QL_FP8_B128_BF16> : Regs<QL_I8_G128_BF16> {};
 template <>
 struct Regs<QL_FP8A8_B128_BF16> : Regs<QL_I8_G128_BF16> {};
 
+// The experts' bf16 down projection (not a packed format of the ABI): units of
+// 16 rows x 64 bf16 weights, the same 128-byte rows as the int8 formats.
+constexpr int kFmtDown = 16;
+template <>
+struct Regs<kFmtDown> : Regs<QL_I8_G128_BF16> {};
+
 // Formats whose activations are one-byte codes with an fp32 scale per token
 // per 128 (int8 for W8A8, E4M3 for format 7), multiplied on the byte MMAs.
 template <int FMT>
@@ -317,6 +323,45 @@ __device__ __forceinline__ void unit_e4m3(const Regs<QL_FP8A8_B128_BF16>& r, Get
                 const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
                 const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
                 mma_e4m3(acc[nt], a0, a1, a2, a3, b0, b1);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void mma_bf16(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The bf16 down projection of one unit (16 rows x 64 K): the weights are MMA
+// operands as they are; the activation is three bf16 planes whose sum is the
+// fp32 value, so the three products summed in fp32 carry its full precision.
+// getx(nt, piece, plane) returns the lane's 16-byte piece (chunk c, or 4 + c)
+// of a plane.  No scale: the sums go straight into yacc.
+template <int NT, typename GetX>
+__device__ __forceinline__ void unit_down(const Regs<kFmtDown>& r, GetX getx, bool nt1_live, float (&yacc)[NT][4]) {
+#pragma unroll
+    for (int piece = 0; piece < 2; ++piece) {
+#pragma unroll
+        for (int pl = 0; pl < 3; ++pl) {
+            uint4 xv[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                if (nt == 0 || nt1_live) xv[nt] = getx(nt, piece, pl);
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const int s = 2 * piece + s2;
+                const uint32_t a0 = word_of(r.w[0], 2 * s), a2 = word_of(r.w[0], 2 * s + 1);
+                const uint32_t a1 = word_of(r.w[1], 2 * s), a3 = word_of(r.w[1], 2 * s + 1);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (nt == 1 && !nt1_live) continue;
+                    mma_bf16(yacc[nt], a0, a1, a2, a3, s2 == 0 ? xv[nt].x : xv[nt].z, s2 == 0 ? xv[nt].y : xv[nt].w);
+                }
             }
         }
     }
@@ -777,13 +822,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
 // segment into chunks of 16.  It then starts its weight stream at once and
 // waits for the activation prologue (programmatic dependent launch) only before
 // it reads the activations or adds into y.
+//
+// With FMT == kFmtDown the same walk runs the experts' bf16 down projection:
+// K is the intermediate size (units of 64 bf16), xs the activation of every
+// pair as three bf16 planes [pairs][3][K], and each chunk row, a pair (t, j),
+// is added into y[t][:] (zeroed by the prologue) scaled by its routing weight.
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__ MoeArgs a) {
     extern __shared__ uint8_t smem_raw[];
+    constexpr bool DOWN = FMT == kFmtDown;
     constexpr int SB = stage_bytes<FMT>();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int G = a.K / 128;
+    const int G = DOWN ? a.K / 64 : a.K / 128;
     const int slabs = (a.N + 15) / 16;
     const long long per_chunk = (long long)slabs * G;
     const uint32_t raw = smem_u32(smem_raw);
@@ -854,8 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     const uint32_t ring = base + (uint32_t)(warp * kStages * SB);
     const uint32_t bars = base + (uint32_t)ring_bytes<FMT>() + (uint32_t)(warp * kStages * 8);
     if (u0 >= u1) return;
-    const long long expert_scales =
-        FMT == QL_FP8_B128_BF16 ? (long long)((a.N + 127) / 128) * G : (long long)a.N * G;
+    const long long expert_scales = block_scaled<FMT>() ? (long long)((a.N + 127) / 128) * G : (long long)a.N * G;
     const uint16_t* const sc0 = static_cast<const uint16_t*>(a.scales);
 
     // Unit position, stepped without divisions: chunk, slab, group.
@@ -890,7 +940,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
             mbar_expect_tx(bars + 8 * st, SB);
             tma_load_2d(ring + st * SB, &a.tmap, ip.grp * 128, ch.expert * a.N + ip.slab * 16, bars + 8 * st);
         }
-        load_side_w<FMT, NT>(sd[st], sc0 + (long long)ch.expert * expert_scales, nullptr, a.N, G, ip.grp, ip.slab, g);
+        if constexpr (!DOWN)
+            load_side_w<FMT, NT>(sd[st], sc0 + (long long)ch.expert * expert_scales, nullptr, a.N, G, ip.grp, ip.slab,
+                                 g);
         ip.next(slabs, G);
         ++issued;
     };
@@ -904,12 +956,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     // The weight stream is running; the activations and the zeroed y come from the prologue.
     if (fused) asm volatile("griddepcontrol.wait;\n" ::: "memory");
     MoeChunk chc = chunks[cp.ch];  // the chunk being computed
-    int tok[NT];                     // this lane's tokens in it (-1: none)
+    int tok[NT];                     // this lane's tokens in it (-1: none): the MMA's B columns it loads
+    int ctok[NT][2];                 // format 7: the tokens of this lane's accumulator columns
     auto load_tokens = [&]() {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int slot = 8 * nt + g;
-            tok[nt] = slot < chc.count ? perm[chc.start + slot] / a.topk : -1;
+            const int slot = 8 * nt + g;  // (the down projection's activations are per pair)
+            tok[nt] = slot < chc.count ? perm[chc.start + slot] / (DOWN ? 1 : a.topk) : -1;
+            if constexpr (act8<FMT>()) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int cs = 8 * nt + 2 * c + i;
+                    ctok[nt][i] = cs < chc.count ? perm[chc.start + cs] / a.topk : -1;
+                }
+            }
         }
     };
     load_tokens();
@@ -924,7 +984,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 const int n = cur_slab * 16 + g + 8 * (i >> 1);
                 if (slot < chc.count && n < a.N) {
                     const int pair = perm[chc.start + slot];
-                    atomicAdd(a.y + (long long)pair * a.N + n, yacc[nt][i] * __ldg(a.xf + pair / a.topk));
+                    if constexpr (DOWN) {  // the routing-weighted sum over the token's slots
+                        atomicAdd(a.y + (long long)(pair / a.topk) * a.N + n, yacc[nt][i] * __ldg(a.wts + pair));
+                    } else {
+                        const float f = act8<FMT>() ? 1.0f : __ldg(a.xf + pair / a.topk);
+                        atomicAdd(a.y + (long long)pair * a.N + n, yacc[nt][i] * f);
+                    }
                 }
                 yacc[nt][i] = 0.0f;
             }
@@ -951,17 +1016,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 break;
             }
             Regs<FMT> r;
-            side_to_regs<FMT, NT>(r, sd[st]);
+            if constexpr (!DOWN) side_to_regs<FMT, NT>(r, sd[st]);
             read_unit_smem<FMT>(r, ring + st * SB, g, c);
             const int grp = cp.grp;
             // The fragments read_unit_smem hands out pair with these 16-byte x pieces of the group
             // (the same order as the dense kernel's staged activations).
             auto getx = [&](int nt, int p) -> uint4 {
                 if (tok[nt] < 0) return make_uint4(0, 0, 0, 0);
-                const int j = (p >> 1) * 8 + 2 * c + (p & 1);
-                return __ldg(reinterpret_cast<const uint4*>(a.xs + (long long)tok[nt] * a.K + grp * 128 + 8 * j));
+                if constexpr (act8<FMT>()) {  // E4M3 codes: the dense kernel's piece order, 16 B each
+                    const int j = 4 * p + c;
+                    return __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.xs) +
+                                                                (long long)tok[nt] * a.K + grp * 128 + 16 * j));
+                } else {
+                    const int j = (p >> 1) * 8 + 2 * c + (p & 1);
+                    return __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(a.xs) +
+                                                                (long long)tok[nt] * a.K + grp * 128 + 8 * j));
+                }
             };
-            unit_a16<FMT, NT>(r, getx, chc.count > 8, yacc);
+            if constexpr (DOWN) {
+                auto getx3 = [&](int nt, int piece, int pl) -> uint4 {
+                    if (tok[nt] < 0) return make_uint4(0, 0, 0, 0);
+                    const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(a.xs) +
+                                              ((long long)tok[nt] * 3 + pl) * a.K + grp * 64 + 8 * (piece ? 4 + c : c);
+                    return __ldg(reinterpret_cast<const uint4*>(xr));
+                };
+                unit_down<NT>(r, getx3, chc.count > 8, yacc);
+            } else if constexpr (act8<FMT>()) {
+                // fp32 sums of the group's E4M3 products, then both scales: the block's weight
+                // scale and the scale of the column's token for this group.
+                float acc[NT][4];
+                unit_e4m3<NT>(r, getx, acc);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const float sx = ctok[nt][i] >= 0 ? __ldg(a.xf + (long long)ctok[nt][i] * G + grp) : 0.0f;
+                        yacc[nt][i] = fmaf(r.s[0] * sx, acc[nt][i], yacc[nt][i]);
+                        yacc[nt][2 + i] = fmaf(r.s[1] * sx, acc[nt][2 + i], yacc[nt][2 + i]);
+                    }
+            } else {
+                unit_a16<FMT, NT>(r, getx, chc.count > 8, yacc);
+            }
             __syncwarp();
             if (issued < u1) issue(st);  // refill this slot with the unit kStages ahead
             cp.next(slabs, G);
@@ -1116,6 +1211,41 @@ cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    MoeArgs a = in;
+    a.err = di.err_word;
+    // the stacked bf16 weights as bytes: [E * N rows][2 K bytes], units of 16 rows x 128 B
+    if ((e = make_tmap_2d(a.codes, (long long)a.E * a.N, 2LL * a.K, 2LL * a.K, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B,
+                          &a.tmap)) != cudaSuccess)
+        return e;
+    const size_t smem = 1024 + ring_bytes<kFmtDown>() + (size_t)kWarps * kStages * 8 +
+                        (5 * sizeof(int) + sizeof(MoeChunk)) * kMoeFusedMaxPairs + 16;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        if ((e = cudaFuncSetAttribute(k_moe_tma<kFmtDown, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(di.sm_count);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = a.ids ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_moe_tma<kFmtDown, 2>, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
@@ -1128,11 +1258,12 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     // rings, their mbarriers, and the routing state of the fused small-batch mode
     const size_t smem = 1024 + ring_bytes<QL_I8_G128_BF16>() + (size_t)kWarps * kStages * 8 +
                         (5 * sizeof(int) + sizeof(MoeChunk)) * kMoeFusedMaxPairs + 16;
-    static bool attr_set[64] = {};  // per device ordinal, for all three instantiations at once
+    static bool attr_set[64] = {};  // per device ordinal, for all four instantiations at once
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        for (auto kern : {k_moe_tma<QL_I8_G128_BF16, 2>, k_moe_tma<QL_I8_G128_F16, 2>, k_moe_tma<QL_FP8_B128_BF16, 2>})
+        for (auto kern : {k_moe_tma<QL_I8_G128_BF16, 2>, k_moe_tma<QL_I8_G128_F16, 2>, k_moe_tma<QL_FP8_B128_BF16, 2>,
+                          k_moe_tma<QL_FP8A8_B128_BF16, 2>})
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
                 return e;
         if (dev < 64) attr_set[dev] = true;
@@ -1157,6 +1288,7 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     case QL_I8_G128_BF16: return run(k_moe_tma<QL_I8_G128_BF16, 2>);
     case QL_I8_G128_F16: return run(k_moe_tma<QL_I8_G128_F16, 2>);
     case QL_FP8_B128_BF16: return run(k_moe_tma<QL_FP8_B128_BF16, 2>);
+    case QL_FP8A8_B128_BF16: return run(k_moe_tma<QL_FP8A8_B128_BF16, 2>);
     default: return cudaErrorInvalidValue;
     }
 }

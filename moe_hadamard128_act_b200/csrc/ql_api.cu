@@ -159,8 +159,11 @@ int x_order(int fmt) {
 bool moe_grouped(const ql_experts* ex, int T, int topk) {
     return (long long)T * topk >= (long long)kMoePrefillMinRowsPerExpert * ex->E;
 }
+// Format 7 experts, grouped: the permuted rows' scales [K/128][Mp], with the 132 columns past the last
+// row that a tile's 16-byte aligned scale copy may read.
+int moe_e4m3_mp(int T, int topk) { return (int)align_up((size_t)T * topk + 132, 4); }
 struct MoeWs {
-    size_t xs, xf, counts, offsets, perm, chunks, nch, inv, tiles;
+    size_t xs, xf, counts, offsets, perm, chunks, nch, inv, tiles, sw;
     size_t max_tiles;
     size_t total;
 };
@@ -168,17 +171,26 @@ MoeWs moe_ws(const ql_experts* ex, int T, int topk) {
     MoeWs w;
     size_t o = 0;
     const bool grp = moe_grouped(ex, T, topk);
-    // f16 activations: one row per token (skinny GEMM) or one per (token, slot) in permuted order
-    w.xs = o; o += align_up((size_t)(grp ? T * topk : T) * ex->K * 2, 256);
-    w.xf = o; o += align_up((size_t)T * 4, 256);
+    // f16 activations: one row per token (skinny GEMM) or one per (token, slot) in permuted order;
+    // format 7: E4M3 codes per token and their scales [T][K/128]
+    // (grouped: the permuted rows' scales transposed, [K/128][moe_e4m3_mp]; then the experts' weight
+    // scales as fp32 [E][K/128][pad(N)] for the tensor-core GEMM)
+    const bool e4 = ex->fmt == QL_FP8A8_B128_BF16;
+    const size_t G = (size_t)ex->K / 128;
+    w.xs = o; o += align_up((size_t)(grp ? T * topk : T) * ex->K * (e4 ? 1 : 2), 256);
+    w.xf = o; o += align_up(e4 ? (grp ? G * moe_e4m3_mp(T, topk) * 4 : (size_t)T * G * 4) : (size_t)T * 4, 256);
     w.counts = o; o += align_up((size_t)ex->E * 4, 256);
     w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
     w.perm = o; o += align_up((size_t)T * topk * 4, 256);
-    w.max_tiles = grp ? moe_max_tiles(T, topk, ex->E, kPrefillA16Tokens, (ex->N + 127) / 128) : 0;
+    w.max_tiles = !grp ? 0
+                  : e4 ? moe_max_tiles(T, topk, ex->E, kPrefillTileM, (ex->N + kPrefillTileN - 1) / kPrefillTileN)
+                       : moe_max_tiles(T, topk, ex->E, kPrefillA16Tokens, (ex->N + 127) / 128);
+    w.sw = 0;
     if (grp) {
         w.inv = o; o += align_up((size_t)T * topk * 4, 256);
         w.tiles = o; o += align_up(w.max_tiles * sizeof(MoeTile), 256);
         w.chunks = 0;
+        if (e4) { w.sw = o; o += align_up((size_t)ex->E * G * prefill_pad_n(ex->N) * 4, 256); }
     } else {
         w.inv = w.tiles = 0;
         w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
@@ -193,10 +205,38 @@ int check_experts(const ql_experts* ex) {
     if (ex->E < 1 || ex->E > 1024 || ex->N < 1 || ex->K < 128 || ex->K % 128) return QL_EINVAL;
     if (ex->flags & ~(QL_HADAMARD | QL_SCALE_SEARCH)) return QL_EINVAL;
     if (!fmt_valid(ex->fmt)) return QL_EINVAL;
-    if (ex->fmt != QL_I8_G128_BF16 && ex->fmt != QL_I8_G128_F16 && ex->fmt != QL_FP8_B128_BF16) return QL_EUNSUPPORTED;
+    if (ex->fmt != QL_I8_G128_BF16 && ex->fmt != QL_I8_G128_F16 && ex->fmt != QL_FP8_B128_BF16 &&
+        ex->fmt != QL_FP8A8_B128_BF16)
+        return QL_EUNSUPPORTED;
     if (ex->K > QL_A16_MAX_K) return QL_EUNSUPPORTED;
     if (!ex->codes || !ex->scales) return QL_EINVAL;
     if (!aligned16(ex->codes) || !aligned16(ex->scales)) return QL_EALIGN;
+    return QL_OK;
+}
+
+// moe_down_combine's workspace: the activation planes, then the permutation.
+struct DownWs {
+    size_t act, counts, offsets, perm, chunks, nch, total;
+};
+DownWs down_ws(const ql_down_experts* ex, int T, int topk) {
+    DownWs w;
+    size_t o = 0;
+    const size_t P = (size_t)T * topk;
+    w.act = o; o += align_up(P * 3 * ex->I * 2, 256);
+    w.counts = o; o += align_up((size_t)ex->E * 4, 256);
+    w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
+    w.perm = o; o += align_up(P * 4, 256);
+    w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
+    w.nch = o; o += 256;
+    w.total = o;
+    return w;
+}
+
+int check_down_experts(const ql_down_experts* ex) {
+    if (!ex) return QL_EINVAL;
+    if (ex->E < 1 || ex->E > 1024 || ex->K < 1 || ex->I < 64 || ex->I % 64) return QL_EINVAL;
+    if (!ex->weights) return QL_EINVAL;
+    if (!aligned16(ex->weights)) return QL_EALIGN;
     return QL_OK;
 }
 
@@ -454,6 +494,44 @@ int qlinear_forward_i8_acc(const int8_t* qx, const int8_t* qw, int M, int N, int
     return QL_OK;
 }
 
+int qlinear_gemm_a8(const void* qx, const float* sx, const void* W_packed, const void* scales, int fmt, int M, int N,
+                    int K, float* y, int accumulate, void* stream) {
+    if ((fmt != QL_I8A8_G128_BF16 && fmt != QL_FP8A8_B128_BF16) || M < 1 || N < 1 || K < 128 || K % 128)
+        return QL_EINVAL;
+    if (!qx || !sx || !W_packed || !scales || !y) return QL_EINVAL;
+    if (M > 16) return QL_EUNSUPPORTED;
+    if (!aligned16(qx) || !aligned16(sx) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y))
+        return QL_EALIGN;
+    if (skinny_max_k(fmt) < 128) return QL_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!accumulate) {
+        const cudaError_t e = cudaMemsetAsync(y, 0, (size_t)M * N * sizeof(float), s);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    const int G = K / 128;
+    SkinnyArgs a;
+    a.W = static_cast<const uint8_t*>(W_packed);
+    a.scales = scales;
+    a.zeros = nullptr;
+    a.xs = qx;
+    a.xf = sx;
+    a.y = y;
+    a.acc = nullptr;
+    a.M = M;
+    a.N = N;
+    a.G = G;
+    a.g0 = 0;
+    a.Gtot = G;
+    a.ldw = K;
+    a.ldx = K;
+    a.ldy = N;
+    a.pdl = 1;  // waits for the kernel before it before reading qx, sx or y
+    const int t = trace_begin(QL_KIND_SKINNY, s);
+    const cudaError_t e = launch_skinny(fmt, a, s);
+    trace_end(t, s);
+    return from_cuda(e);
+}
+
 int act_quant_i8_g128(const void* x, int M, int K, int rotate, int8_t* q, float* s, void* stream) {
     if (M < 1 || K < 128 || K % 128 || !x || !q || !s) return QL_EINVAL;
     if (!aligned16(x) || !aligned16(q) || !aligned16(s)) return QL_EALIGN;
@@ -531,6 +609,39 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     const int K = experts->K, N = experts->N;
     const int rot = (experts->flags & QL_HADAMARD) ? 1 : 0;
     cudaError_t e;
+    if (moe_grouped(experts, T, topk) && experts->fmt == QL_FP8A8_B128_BF16) {
+        // permute; E4M3 codes and scales straight into permuted order; the experts' weight scales
+        // as fp32; the grouped E4M3 tensor-core GEMM with the un-permute in its stores
+        MoePermuteOut po;
+        po.inv = reinterpret_cast<int32_t*>(b + w.inv);
+        po.tiles = reinterpret_cast<MoeTile*>(b + w.tiles);
+        po.n_tiles = nch;
+        po.tile_rows = kPrefillTileM;
+        po.wblocks = (N + kPrefillTileN - 1) / kPrefillTileN;
+        po.yz = y;  // rows of pairs with a bad expert id are zeroed
+        po.N = N;
+        int t = trace_begin(QL_KIND_MOE_PERMUTE, s);
+        e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        const int Mp = moe_e4m3_mp(T, topk);
+        t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant_e4m3(x, T, K, rot, reinterpret_cast<uint8_t*>(xs), nullptr, xf, Mp, nullptr, 0, s,
+                                  po.inv, topk);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        float* swT = reinterpret_cast<float*>(b + w.sw);
+        t = trace_begin(QL_KIND_PREFILL_PREP, s);
+        e = launch_prefill_prep_blk(static_cast<const uint16_t*>(experts->scales), N, K, swT, s, experts->E);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_MOE_GEMM, s);
+        e = launch_prefill_e4m3_grouped(reinterpret_cast<const uint8_t*>(xs), xf, Mp,
+                                        static_cast<const uint8_t*>(experts->codes), swT, experts->E, N, K, T * topk,
+                                        po.tiles, nch, (int)w.max_tiles, perm, y, s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     if (moe_grouped(experts, T, topk)) {  // permute, stage x in permuted order, grouped tensor-core GEMM
         MoePermuteOut po;
         po.inv = reinterpret_cast<int32_t*>(b + w.inv);
@@ -555,9 +666,15 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
         trace_end(t, s);
         return from_cuda(e);
     }
-    int t = trace_begin(QL_KIND_PREP_A16, s);  // rotation, f16 staging, and the zeroing of y
-    e = launch_prep_a16(x, T, K, rot, XORD_NATURAL, xs, xf, y,
-                        (long long)T * topk * N, s);
+    int t;
+    if (experts->fmt == QL_FP8A8_B128_BF16) {  // rotation, E4M3 codes and scales per token, the zeroing of y
+        t = trace_begin(QL_KIND_ACT_QUANT, s);
+        e = launch_act_quant_e4m3(x, T, K, rot, reinterpret_cast<uint8_t*>(xs), xf, nullptr, 0, y,
+                                  (long long)T * topk * N, s);
+    } else {  // rotation, f16 staging, and the zeroing of y
+        t = trace_begin(QL_KIND_PREP_A16, s);
+        e = launch_prep_a16(x, T, K, rot, XORD_NATURAL, xs, xf, y, (long long)T * topk * N, s);
+    }
     trace_end(t, s);
     if (e != cudaSuccess) return from_cuda(e);
     // Small batches: the expert GEMM ranks the ids itself (no permute launch).
@@ -590,6 +707,75 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     a.max_chunks = (long long)moe_max_chunks(T, topk, experts->E);
     t = trace_begin(QL_KIND_MOE_GEMM, s);
     e = launch_moe_skinny(a, s);
+    trace_end(t, s);
+    return from_cuda(e);
+}
+
+int moe_down_workspace_size(const ql_down_experts* experts, int T, int topk, size_t* bytes) {
+    const int st = check_down_experts(experts);
+    if (st != QL_OK) return st;
+    if (T < 1 || topk < 1 || topk > 64 || !bytes) return QL_EINVAL;
+    *bytes = down_ws(experts, T, topk).total;
+    return QL_OK;
+}
+
+int moe_down_combine(const float* h, const int32_t* topk_ids, const float* topk_weights,
+                     const ql_down_experts* experts, int T, int topk, float* out, void* ws, size_t ws_bytes,
+                     void* stream) {
+    int st = check_down_experts(experts);
+    if (st != QL_OK) return st;
+    if (T < 1 || topk < 1 || topk > 64 || !h || !topk_ids || !topk_weights || !out) return QL_EINVAL;
+    if (!aligned16(h) || !aligned16(topk_ids) || !aligned16(topk_weights) || !aligned16(out)) return QL_EALIGN;
+    const DownWs w = down_ws(experts, T, topk);
+    if (!ws || ws_bytes < w.total) return QL_EWORKSPACE;
+    if (!aligned16(ws)) return QL_EALIGN;
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return QL_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(b + w.act);
+    int32_t* counts = reinterpret_cast<int32_t*>(b + w.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(b + w.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + w.perm);
+    MoeChunk* chunks = reinterpret_cast<MoeChunk*>(b + w.chunks);
+    int* nch = reinterpret_cast<int*>(b + w.nch);
+    const int P = T * topk;
+    // gelu(gate) * up as three bf16 planes, and the zeroing of out
+    int t = trace_begin(QL_KIND_MOE_ACT, s);
+    cudaError_t e = launch_moe_act(h, topk_ids, P, experts->E, experts->I, act, out, (long long)T * experts->K, s);
+    trace_end(t, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    // Small batches: the expert GEMM ranks the ids itself (no permute launch).
+    const bool fused = P <= kMoeFusedMaxPairs;
+    if (!fused) {
+        MoePermuteOut po;
+        po.chunks = chunks;
+        po.n_chunks = nch;
+        t = trace_begin(QL_KIND_MOE_PERMUTE, s);
+        e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    MoeArgs a;
+    a.codes = static_cast<const uint8_t*>(experts->weights);
+    a.scales = nullptr;
+    a.xs = act;
+    a.xf = nullptr;
+    a.perm = perm;
+    a.chunks = chunks;
+    a.n_chunks = nch;
+    a.ids = fused ? topk_ids : nullptr;
+    a.y = out;
+    a.wts = topk_weights;
+    a.fmt = 0;
+    a.T = T;
+    a.topk = topk;
+    a.E = experts->E;
+    a.N = experts->K;
+    a.K = experts->I;
+    a.max_chunks = (long long)moe_max_chunks(T, topk, experts->E);
+    t = trace_begin(QL_KIND_MOE_DOWN, s);
+    e = launch_moe_down(a, s);
     trace_end(t, s);
     return from_cuda(e);
 }

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -55,9 +56,11 @@ cudaError_t launch_rotate_bf16(const void* x, int M, int K, void* y, cudaStream_
 // to sxT (either may be null).
 cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q, float* sx, float* sxT, int Mp,
                              float* yz, long long nz, cudaStream_t s);
-// The same rule with E4M3 codes (448 for 127), written as bytes.
+// The same rule with E4M3 codes (448 for 127), written as bytes.  With inv != null, token t's codes
+// and scales go to rows inv[t * topk + j] of q and sxT (the permuted order of the grouped expert GEMM).
 cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
-                                  float* yz, long long nz, cudaStream_t s);
+                                  float* yz, long long nz, cudaStream_t s, const int32_t* inv = nullptr,
+                                  int topk = 0);
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s);
 // The same for the grouped expert GEMM: token t's f16 row goes to rows
@@ -119,8 +122,9 @@ cudaError_t launch_prefill_i5_codes(const uint8_t* codes, const uint8_t* zeros, 
 // From this many rows on, the int5 format takes int8 activations ("keptn/gemma4-31b-w5",
 // table "Format": f16 activations up to 64 rows, int8 per token per 128 above).
 constexpr int kW5A8MinM = 65;
-// The same from bf16 block scales [ceil(N/128)][K/128] (each row takes its block's scale).
-cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s);
+// The same from bf16 block scales [ceil(N/128)][K/128] (each row takes its block's scale); for E
+// stacked experts, E consecutive scale arrays in, E consecutive [K/128][pad(N)] blocks out.
+cudaError_t launch_prefill_prep_blk(const uint16_t* sw, int N, int K, void* scratch, cudaStream_t s, int E = 1);
 constexpr int kPrefillMinM = 17;  // from this many tokens on, W8A8 runs on the tcgen05 GEMM
 
 // The same for the formats with 16-bit activations (int8 g128 with bf16 or f16
@@ -169,6 +173,14 @@ cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* x
                                        const void* scales, int E, int N, int K, int rows_total, const MoeTile* tiles,
                                        const int* n_tiles, int max_tiles, const int32_t* perm, int topk, float* y,
                                        cudaStream_t s);
+// Format 7 experts on the E4M3 tensor-core GEMM, grouped: qx the E4M3 codes of the permuted rows
+// [rows_total][K] with their scales sxT [K/128][Mp] (Mp % 4 == 0, at least 132 columns past the last
+// row), swT the experts' weight scales from launch_prefill_prep_blk (E blocks), tiles of
+// kPrefillTileM permuted rows x kPrefillTileN weight rows from the permute.
+cudaError_t launch_prefill_e4m3_grouped(const uint8_t* qx, const float* sxT, int Mp, const uint8_t* codes,
+                                        const float* swT, int E, int N, int K, int rows_total, const MoeTile* tiles,
+                                        const int* n_tiles, int max_tiles, const int32_t* perm, float* y,
+                                        cudaStream_t s);
 // From this many (token, slot) pairs per expert on average, moe_gate_up runs the grouped tensor-core GEMM.
 constexpr int kMoePrefillMinRowsPerExpert = 8;
 cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,
@@ -178,19 +190,30 @@ struct MoeArgs {
     unsigned* err;         // device error word (filled by launch_moe_skinny)
     const uint8_t* codes;  // [E][N][K]
     const void* scales;    // [E][...] per the format
-    const __half* xs;      // prepared activations [T][K] (natural order)
-    const float* xf;       // [T]
+    const void* xs;        // prepared activations [T][K]: f16 in natural order, or E4M3 codes (format 7)
+    const float* xf;       // [T] inverse token factors, or (format 7) activation scales [T][K/128]
     const int32_t* perm;   // [T*topk]
     const MoeChunk* chunks;
     const int* n_chunks;
     const int32_t* ids = nullptr;  // [T*topk] routing ids: when set (T*topk <= kMoeFusedMaxPairs), every CTA
                            // builds the permutation and chunk table itself and perm / chunks are unused
-    float* y;              // [T*topk][N]
+    float* y;              // [T*topk][N] (down projection: [T][N])
+    const float* wts = nullptr;  // down projection: routing weights [T*topk]
     int fmt, T, topk, E, N, K;
     long long max_chunks;
 };
 constexpr int kMoeFusedMaxPairs = 128;
 cudaError_t launch_moe_skinny(const MoeArgs& a, cudaStream_t s);
+// The experts' bf16 down projection with the routing-weighted combine: codes are the stacked bf16
+// weights [E][N][K] (N = hidden size, K = intermediate size, K % 64 == 0), xs the pairs'
+// activations as three bf16 planes [T*topk][3][K]; y [T][N] (zeroed before) gets
+// sum_j wts[t*topk+j] * (act of (t, j)) . W_e^T.  Chunks / fused ranking as launch_moe_skinny.
+cudaError_t launch_moe_down(const MoeArgs& a, cudaStream_t s);
+// gelu(gate) * up of each pair's gate_up row h [P][2 I] (fp32), split into three bf16 planes
+// act [P][3][I] whose sum is the fp32 value; pairs with an id outside [0, E) are skipped.  Also
+// zeroes out[0 .. nz).
+cudaError_t launch_moe_act(const float* h, const int32_t* ids, int P, int E, int I, __nv_bfloat16* act, float* out,
+                           long long nz, cudaStream_t s);
 
 // ---- launch trace (ql_trace_enable / ql_trace_read) --------------------------------------
 // trace_begin records a start event for one library launch when tracing is on

@@ -28,23 +28,16 @@ constexpr size_t kScratchBytes = kQxBytes + kSxBytes;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-// Device address of the scratch array, looked up once per device.  In host
-// code the symbol g_noalloc_scratch is only a host-side stand-in, so the
-// kernels must be given this address instead.
-unsigned char* g_scratch_ptr[64] = {};
-
+// Device address of the scratch array on the current device.  In host code
+// the symbol g_noalloc_scratch is only a host-side stand-in, so the kernels
+// must be given this address instead.  It is looked up on every call (the
+// lookup allocates nothing), so no address outlives a device reset and
+// concurrent first calls from several host threads need no lock.
 cudaError_t scratch_for_current_device(unsigned char** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
-    }
-    *out = g_scratch_ptr[dev];
+    *out = static_cast<unsigned char*>(p);
     return cudaSuccess;
 }
 
@@ -63,37 +56,38 @@ extern "C" int qlinear_forward_w8a8_noalloc(const void* x, const void* W_packed,
     if (!aligned16(x) || !aligned16(W_packed) || !aligned16(scales) || !aligned16(y)) return QL_EALIGN;
     unsigned char* scratch = nullptr;
     if (scratch_for_current_device(&scratch) != cudaSuccess) return QL_ECUDA;
-    const int kmax = skinny_max_k(QL_I8A8_G128_BF16);
-    if (kmax < 128) return QL_ECUDA;
+    if (skinny_max_k(QL_I8A8_G128_BF16) < 128) return QL_ECUDA;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int G = K / 128;
     int8_t* qx = reinterpret_cast<int8_t*>(scratch);
     float* sx = reinterpret_cast<float*>(scratch + kQxBytes);
     // The quantiser also zeroes y, which the GEMM then accumulates into.
+    int t = trace_begin(QL_KIND_ACT_QUANT, s);
     cudaError_t e = launch_act_quant(x, M, K, (flags & QL_HADAMARD) ? 1 : 0, qx, sx, nullptr, 0, y, (long long)M * N,
                                      s);
+    trace_end(t, s);
     if (e != cudaSuccess) return QL_ECUDA;
-    for (int k0 = 0; k0 < K; k0 += kmax) {
-        const int kc = K - k0 < kmax ? K - k0 : kmax;
-        SkinnyArgs a{};
-        a.W = static_cast<const uint8_t*>(W_packed) + k0;
-        a.scales = scales;
-        a.zeros = nullptr;
-        a.xs = qx + k0;
-        a.xf = sx;
-        a.y = y;
-        a.acc = nullptr;
-        a.M = M;
-        a.N = N;
-        a.G = kc / 128;
-        a.g0 = k0 / 128;
-        a.Gtot = G;
-        a.ldw = K;
-        a.ldx = K;
-        a.ldy = N;
-        a.pdl = 1;
-        if ((e = launch_skinny(QL_I8A8_G128_BF16, a, s)) != cudaSuccess) return QL_ECUDA;
-    }
-    return QL_OK;
+    // One decode launch over the whole K, as qlinear_forward makes it.
+    SkinnyArgs a{};
+    a.W = static_cast<const uint8_t*>(W_packed);
+    a.scales = scales;
+    a.zeros = nullptr;
+    a.xs = qx;
+    a.xf = sx;
+    a.y = y;
+    a.acc = nullptr;
+    a.M = M;
+    a.N = N;
+    a.G = G;
+    a.g0 = 0;
+    a.Gtot = G;
+    a.ldw = K;
+    a.ldx = K;
+    a.ldy = N;
+    a.pdl = 1;
+    t = trace_begin(QL_KIND_SKINNY, s);
+    e = launch_skinny(QL_I8A8_G128_BF16, a, s);
+    trace_end(t, s);
+    return e == cudaSuccess ? QL_OK : QL_ECUDA;
 }

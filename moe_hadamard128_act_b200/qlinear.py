@@ -52,6 +52,10 @@ class ql_experts(ctypes.Structure):
                 ("flags", ctypes.c_int), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
+class ql_down_experts(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("K", ctypes.c_int), ("I", ctypes.c_int), ("weights", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.c_size_t
@@ -65,11 +69,15 @@ _SIGS = {
     "qlinear_workspace_size": (_I, [_I, _I, _I, _I, _I, _PSZ]),
     "qlinear_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "qlinear_forward_i8_acc": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+    "qlinear_gemm_a8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
     "act_quant_i8_g128": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "act_quant_e4m3_g128": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "hadamard128_rotate": (_I, [_P, _I, _I, _P, _P]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_workspace_size": (_I, [ctypes.POINTER(ql_experts), _I, _I, _PSZ]),
     "moe_gate_up": (_I, [_P, _P, _P, ctypes.POINTER(ql_experts), _I, _I, _P, _P, _SZ, _P]),
+    "moe_down_workspace_size": (_I, [ctypes.POINTER(ql_down_experts), _I, _I, _PSZ]),
+    "moe_down_combine": (_I, [_P, _P, _P, ctypes.POINTER(ql_down_experts), _I, _I, _P, _P, _SZ, _P]),
     "ql_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "qlinear_forward_w8a8_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "ql_trace_enable": (_I, [_I]),
@@ -78,7 +86,7 @@ _SIGS = {
 }
 
 KIND_NAMES = {1: "rotate", 2: "act_quant", 3: "prep_a16", 4: "skinny", 5: "moe_permute", 6: "moe_gemm", 7: "pack",
-              8: "prefill", 9: "prefill_prep"}
+              8: "prefill", 9: "prefill_prep", 10: "moe_act", 11: "moe_down"}
 
 _lib = None
 
@@ -190,9 +198,13 @@ def qlinear_forward_w8a8_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: t
     """W8A8 forward without a workspace, for callers that cannot allocate
     device memory (M <= 16, K <= 16384): the activation scratch lives in a fixed
     array inside the library.  Calls that may overlap on the GPU race on it."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bf16 tensor")
     M, K = x.shape
     if y is None:
         y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    elif y.dtype != torch.float32 or tuple(y.shape) != (M, N):
+        raise ValueError(f"y must be an fp32 tensor of shape ({M}, {N})")
     st = lib().qlinear_forward_w8a8_noalloc(_ptr(x), _ptr(codes), _ptr(scales), flags, M, N, K, _ptr(y),
                                             _stream(stream))
     _check("qlinear_forward_w8a8_noalloc", st)
@@ -207,6 +219,28 @@ def qlinear_forward_i8_acc(qx: torch.Tensor, qw: torch.Tensor, stream=None) -> t
     _check("qlinear_forward_i8_acc", lib().qlinear_forward_i8_acc(_ptr(qx), _ptr(qw), M, N, K, _ptr(acc),
                                                                   _stream(stream)))
     return acc
+
+
+def qlinear_gemm_a8(qx: torch.Tensor, sx: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, fmt: int, N: int,
+                    y: torch.Tensor | None = None, accumulate: bool = False, stream=None) -> torch.Tensor:
+    """The decode GEMM on quantised activations (M <= 16): qx [M, K] int8
+    (W8A8) or E4M3 bytes (format 7) with fp32 scales sx [M, K/128], as the
+    act_quant_* calls make them.  y [M, N] fp32 is overwritten, or added to
+    with accumulate=True."""
+    if qx.dim() != 2 or qx.element_size() != 1:
+        raise ValueError("qx must be a 2-D one-byte tensor")
+    M, K = qx.shape
+    if sx.dtype != torch.float32 or tuple(sx.shape) != (M, K // 128):
+        raise ValueError(f"sx must be an fp32 tensor of shape ({M}, {K // 128})")
+    if y is None:
+        if accumulate:
+            raise ValueError("accumulate needs y")
+        y = torch.empty((M, N), dtype=torch.float32, device=qx.device)
+    elif y.dtype != torch.float32 or tuple(y.shape) != (M, N):
+        raise ValueError(f"y must be an fp32 tensor of shape ({M}, {N})")
+    _check("qlinear_gemm_a8", lib().qlinear_gemm_a8(_ptr(qx), _ptr(sx), _ptr(codes), _ptr(scales), fmt, M, N, K,
+                                                    _ptr(y), int(accumulate), _stream(stream)))
+    return y
 
 
 def act_quant_i8_g128(x: torch.Tensor, rotate: bool = False, stream=None):
@@ -264,6 +298,37 @@ def moe_gate_up(x: torch.Tensor, topk_ids: torch.Tensor, codes: torch.Tensor, sc
                            _ptr(ws), ws.numel(), _stream(stream))
     _check("moe_gate_up", st)
     return y
+
+
+def moe_down_workspace_size(E: int, K: int, I: int, T: int, topk: int) -> int:
+    ex = ql_down_experts(E, K, I, 16)  # placeholder aligned pointer: only sizes are read
+    b = ctypes.c_size_t()
+    _check("moe_down_workspace_size", lib().moe_down_workspace_size(ctypes.byref(ex), T, topk, ctypes.byref(b)))
+    return b.value
+
+
+def moe_down_combine(h: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor, wd: torch.Tensor, E: int,
+                     out: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out [T, K] fp32: the experts' bf16 down projections of gelu(gate) * up of the gate_up output
+    h [T, topk, 2I] (fp32), summed over each token's slots with the routing weights.  wd: the stacked
+    bf16 weights [E, K, I] (any 2-byte dtype, viewed as bits)."""
+    if h.dtype != torch.float32 or h.dim() != 3:
+        raise ValueError("h must be an fp32 tensor [T, topk, 2I]")
+    T, topk, I2 = h.shape
+    if wd.element_size() != 2 or wd.dim() != 3 or wd.shape[0] != E or wd.shape[2] * 2 != I2:
+        raise ValueError("wd must be a 2-byte tensor [E, K, I] with 2I = h.shape[-1]")
+    K = wd.shape[1]
+    ex = ql_down_experts(E, K, I2 // 2, wd.data_ptr())
+    b = ctypes.c_size_t()
+    _check("moe_down_workspace_size", lib().moe_down_workspace_size(ctypes.byref(ex), T, topk, ctypes.byref(b)))
+    if ws is None or ws.numel() < b.value:
+        ws = _empty(b.value, h.device)
+    if out is None:
+        out = torch.empty((T, K), dtype=torch.float32, device=h.device)
+    st = lib().moe_down_combine(_ptr(h), _ptr(topk_ids), _ptr(topk_weights), ctypes.byref(ex), T, topk, _ptr(out),
+                                _ptr(ws), ws.numel(), _stream(stream))
+    _check("moe_down_combine", st)
+    return out
 
 
 def ql_trace_enable(capacity: int):

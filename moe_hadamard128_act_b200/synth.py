@@ -195,3 +195,14 @@ def prefill(seed: int = 0, M: int = 2048, K: int = 5376, N: int = 21504, rows=No
     W = weight_rows(seed, "W", K, r0, nr)
     x = activations(seed, "x_prefill", M, K)
     return dict(W=W, x=x, M=M, N=N, K=K)
+
+
+def moe_down(T: int, seed: int = 0, E: int = 128, topk: int = 8, K: int = 2816, I: int = 704, experts=None):
+    """The down projection's inputs: routing as moe_gate_up's workload (same seed, so the same ids and
+    weights), the gate_up output h ~ N(0, 1) as fp32 [T, topk, 2I], and per expert a bf16 down weight
+    [K, I] ~ N(0, 0.02^2) (expert e is stream "Wd_e<e>"; `experts` limits which are drawn)."""
+    ids, w = routing(seed, T, E, topk)
+    h = normal(seed, f"h_T{T}", 0, T * topk * 2 * I).astype(np.float32).reshape(T, topk, 2 * I)
+    which = range(E) if experts is None else experts
+    Wd = {e: to_bf16_bits(weight_rows(seed, f"Wd_e{e}", I, 0, K)) for e in which}
+    return dict(ids=ids, weights=w, h=h, Wd=Wd, T=T, E=E, topk=topk, K=K, I=I)

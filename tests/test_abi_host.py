@@ -136,6 +136,12 @@ def test_pack_and_act_validation_statuses(L):
     assert L.hadamard128_rotate(P(A), 0, 128, P(A), None) == 1
     assert L.hadamard128_rotate(P(A), 1, 128, P(A + 1), None) == 3
     assert L.qlinear_forward_i8_acc(P(A), P(A), 1, 1, 64, P(A), None) == 1
+    g = L.qlinear_gemm_a8  # (qx, sx, W, scales, fmt, M, N, K, y, accumulate, stream)
+    assert g(P(A), P(A), P(A), P(A), 1, 4, 64, 256, P(A), 0, None) == 1  # weight-only formats take bf16 x
+    assert g(P(A), P(A), P(A), P(A), 3, 4, 64, 200, P(A), 0, None) == 1
+    assert g(P(A), None, P(A), P(A), 3, 4, 64, 256, P(A), 0, None) == 1
+    assert g(P(A), P(A), P(A), P(A), 3, 17, 64, 256, P(A), 0, None) == 2  # decode shapes only
+    assert g(P(A), P(A), P(A), P(A), 7, 4, 64, 256, P(A + 4), 1, None) == 3
 
 
 def test_moe_validation_statuses(L):

@@ -63,7 +63,7 @@ def test_dense_w8a8_hadamard_full(Q, dense_w8a8, M):
     assert_close(y[:, rows], ref, f"W8A8 M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("M", [1, 4, 5, 16])
 def test_w4a16_full(Q, M):
     d = synth.w4a16(M)
     c, s, _ = Q.qlinear_pack(Q.I4_G64_BF16, N_FULL, K_FULL, codes=dev(d["codes"]), scales=dev(d["scales"]))
@@ -88,7 +88,7 @@ def test_w5a8_prefill_full(Q):
     assert_close(y[:, rows], ref, "W5A8 M=2048")
 
 
-@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("M", [1, 4, 5, 16])
 def test_w5a16_full(Q, M):
     d = synth.w5a16(M)
     c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N_FULL, K_FULL, codes=dev(d["codes"]), scales=dev(d["scales"]),
@@ -101,7 +101,7 @@ def test_w5a16_full(Q, M):
     assert_close(y[:, rows], ref, f"W5A16 M={M}")
 
 
-@pytest.mark.parametrize("T", [1, 16, 2048])
+@pytest.mark.parametrize("T", [1, 8, 16, 2048])
 def test_moe_gate_up_full(Q, T):
     E, topk, K, N = 128, 8, 2816, 1408
     ids, w = synth.routing(0, T, E, topk)
@@ -122,6 +122,57 @@ def test_moe_gate_up_full(Q, T):
         qr, sr = O.quant_i8_g128(d["W"][e], hadamard=True)
         ref = O.forward(d["x"][t:t + 1], qr.view(np.uint8), sr, None, Q.I8_G128_BF16, Q.HADAMARD, N)
         assert_close(y[t, j][None], ref, f"moe T={T} pair {p}")
+
+
+@pytest.mark.parametrize("T", [1, 16, 2048])
+def test_moe_gate_up_fp8a8_full(Q, T):
+    """The fp8 experts ("gemma4-26b-a4b-dflash-fp8" README, table "Weights") with E4M3 activations at
+    the MoE workload's sizes: 128 experts of [1408, 2816], top-8 routing, the weights packed on the GPU
+    in the rotated domain.  T = 1 and 16 run the weight-streaming kernel, T = 2048 the grouped E4M3
+    tensor-core GEMM.  Sampled pairs against the oracle's dense format-7 forward of their expert."""
+    E, topk, K, N = 128, 8, 2816, 1408
+    ids, w = synth.routing(0, T, E, topk)
+    touched = sorted(set(ids.ravel().tolist()))
+    d = synth.moe_gate_up(T, experts=touched)
+    codes = dev(np.zeros((E, N, K), np.uint8))
+    sb = (N + 127) // 128 * (K // 128)
+    scales = dev(np.zeros((E, sb), np.int16))
+    for e in touched:
+        c, s, _ = Q.qlinear_pack(Q.FP8A8_B128_BF16, N, K, W=dev(d["W"][e]), flags=Q.HADAMARD)
+        codes[e] = c.reshape(N, K)
+        scales[e] = s.view(torch.int16)
+    y = Q.moe_gate_up(dev_bf16(d["x"]), dev(ids), codes, scales, E, N, fmt=Q.FP8A8_B128_BF16, flags=Q.HADAMARD,
+                      topk_weights=dev(w)).cpu().numpy()
+    rng = np.random.default_rng(100 + T)
+    pairs = rng.choice(T * topk, min(T * topk, 12), replace=False)
+    for p in pairs:
+        t, j = divmod(int(p), topk)
+        e = ids[t, j]
+        qr, sr = O.quant_fp8_b128(d["W"][e], hadamard=True)
+        ref = O.forward(d["x"][t:t + 1], qr, sr, None, Q.FP8A8_B128_BF16, Q.HADAMARD, N)
+        assert_close(y[t, j][None], ref, f"moe format 7 T={T} pair {p}")
+
+
+@pytest.mark.parametrize("T", [1, 16, 2048])
+def test_moe_down_combine_full(Q, T):
+    """The experts' bf16 down projections (128 x [2816, 704], "gemma4-26b-a4b-dflash-i8" README, table
+    "Weights") and the routing-weighted combine at the MoE workload's sizes, top-8 routing; sampled
+    tokens against the oracle (only the experts they touch, renumbered)."""
+    E, topk, K, I = 128, 8, 2816, 704
+    ids, _ = synth.routing(0, T, E, topk)
+    touched = sorted(set(ids.ravel().tolist()))
+    d = synth.moe_down(T, experts=touched)
+    wd = torch.zeros((E, K, I), dtype=torch.int16, device="cuda")
+    for e in touched:
+        wd[e] = dev(d["Wd"][e].view(np.int16))
+    out = Q.moe_down_combine(dev(d["h"]), dev(d["ids"]), dev(d["weights"]), wd, E).cpu().numpy()
+    rng = np.random.default_rng(200 + T)
+    for t in rng.choice(T, min(T, 6), replace=False):
+        es = sorted(set(d["ids"][t].tolist()))
+        local = np.array([[es.index(e) for e in d["ids"][t]]], np.int32)
+        ref = O.moe_down_combine(d["h"][t:t + 1], local, d["weights"][t:t + 1], np.stack([d["Wd"][e] for e in es]),
+                                 len(es))
+        assert_close(out[t:t + 1], ref, f"down T={T} token {t}")
 
 
 def test_prefill_w8a8_full(Q):
@@ -154,3 +205,22 @@ def test_fp8a8_decode_full(Q, M):
     assert np.array_equal(host_u8(s).view(np.uint16).reshape(N_FULL // 128, K_FULL // 128)[blocks], sr)
     ref = O.forward(x, qr, sr, None, Q.FP8A8_B128_BF16, 0, len(rows))
     assert_close(y[:, rows], ref, f"format 7 decode M={M}")
+
+
+def test_prefill_fp8_full(Q):
+    """FP8 E4M3 weights per 128 x 128 block with bf16 block scales and bf16 activations
+    ("gemma4-26b-a4b-dflash-fp8" README, table "Weights") at M=2048, N=21504, K=5376: the weight
+    packed on the GPU from the seeded fp32 draw, the tensor-core prefill GEMM over all 1232
+    persistent tiles.  A block scale depends on all 128 rows of its block, so whole blocks are
+    sampled: their codes and scales bit-exact, their outputs against the oracle."""
+    d = synth.prefill()
+    c, s, _ = Q.qlinear_pack(Q.FP8_B128_BF16, N_FULL, K_FULL, W=dev(d["W"]))
+    del d["W"]
+    y = Q.qlinear_forward(dev_bf16(d["x"]), c, s, None, Q.FP8_B128_BF16, N_FULL).cpu().numpy()
+    blocks = [0, 61, N_FULL // 128 - 1]
+    rows = np.concatenate([np.arange(128 * b, 128 * b + 128) for b in blocks])
+    qr, sr = O.quant_fp8_b128(np.concatenate([synth.weight_rows(0, "W", K_FULL, 128 * b, 128) for b in blocks]))
+    assert np.array_equal(host_u8(c).reshape(N_FULL, K_FULL)[rows], qr)
+    assert np.array_equal(host_u8(s).view(np.uint16).reshape(N_FULL // 128, K_FULL // 128)[blocks], sr)
+    ref = O.forward(d["x"], qr, sr, None, Q.FP8_B128_BF16, 0, len(rows))
+    assert_close(y[:, rows], ref, "prefill fp8 full")

@@ -208,6 +208,26 @@ def test_w8a8_group_sums_bitexact(M, N, K):
     assert_close(y.cpu().numpy(), O.forward(x, qw.view(np.uint8), sw, None, Q.I8A8_G128_BF16, Q.HADAMARD, N))
 
 
+@pytest.mark.parametrize("fmt", [3, 7])
+@pytest.mark.parametrize("M,N,K", [(1, 512, 256), (5, 1000, 1024), (9, 130, 256), (16, 333, 640), (16, 4000, 5376)])
+def test_gemm_a8_parity(fmt, M, N, K):
+    """The decode GEMM on activations quantised beforehand: the act_quant call's codes (bit-exact
+    against the oracle's quantiser) into qlinear_gemm_a8, against the oracle's forward of the bf16 x,
+    overwriting y and then adding to a y that already holds values."""
+    had = 1
+    (c, s, z), (ch, sh, zh) = make_weights(fmt, N, K, had)
+    x = x_bits(M, K, seed=13, outliers=0.01)
+    quant = Q.act_quant_i8_g128 if fmt == Q.I8A8_G128_BF16 else Q.act_quant_e4m3_g128
+    qx, sx = quant(dev_bf16(x), rotate=True)
+    ref = O.forward(x, ch, sh, zh, fmt, had, N)
+    y = Q.qlinear_gemm_a8(qx, sx, c, s, fmt, N)
+    assert_close(y.cpu().numpy(), ref, f"fmt {fmt} {M}x{N}x{K}")
+    y0 = np.linspace(-1.0, 1.0, M * N, dtype=np.float32).reshape(M, N)
+    y = dev(y0)
+    Q.qlinear_gemm_a8(qx, sx, c, s, fmt, N, y=y, accumulate=True)
+    assert_close(y.cpu().numpy(), ref + y0.astype(np.float64), f"fmt {fmt} {M}x{N}x{K} accumulate")
+
+
 def test_forward_zero_and_constant_inputs():
     N, K = 64, 256
     (c, s, z), (ch, sh, zh) = make_weights(Q.I8_G128_BF16, N, K, 0)
@@ -249,7 +269,7 @@ def moe_weights(E, N, K, fmt, seed=9):
     qs, ss = [], []
     for e in range(E):
         W = synth.weight_rows(seed, f"moeW{e}", K, 0, N)
-        if fmt == Q.FP8_B128_BF16:
+        if fmt in (Q.FP8_B128_BF16, Q.FP8A8_B128_BF16):
             q, s = O.quant_fp8_b128(W, hadamard=True)
         else:
             q, s = O.quant_i8_g128(W, hadamard=True, scale_f16=fmt == Q.I8_G128_F16)
@@ -259,7 +279,7 @@ def moe_weights(E, N, K, fmt, seed=9):
     return np.stack(qs), np.stack(ss)
 
 
-@pytest.mark.parametrize("fmt", [1, 2, 6])
+@pytest.mark.parametrize("fmt", [1, 2, 6, 7])
 @pytest.mark.parametrize("T,E,topk,N,K", [(1, 8, 2, 96, 256), (8, 16, 4, 64, 384), (16, 32, 8, 130, 256),
                                           (20, 32, 8, 130, 256), (40, 8, 3, 48, 128)])
 def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
@@ -274,11 +294,14 @@ def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
     assert_close(y.cpu().numpy(), ref, f"moe fmt {fmt} T{T}")
 
 
-@pytest.mark.parametrize("fmt", [1, 2, 6])
-@pytest.mark.parametrize("T,E,topk,N,K", [(64, 8, 4, 130, 384), (300, 16, 8, 200, 256), (50, 64, 8, 128, 128)])
+@pytest.mark.parametrize("fmt", [1, 2, 6, 7])
+@pytest.mark.parametrize("T,E,topk,N,K", [(64, 8, 4, 130, 384), (300, 16, 8, 200, 256), (50, 64, 8, 128, 128),
+                                          (600, 8, 2, 400, 256)])
 def test_moe_gate_up_grouped_parity(fmt, T, E, topk, N, K):
     # T * topk >= 8 E: the grouped tensor-core GEMM. (300, 16, 8): ~150 rows per expert, some over one
     # 192-row block; N = 200: a ragged second weight block. (50, 64, 8): some experts get no rows.
+    # (600, 8, 2): ~150 rows per expert, several 128-row tiles each; N = 400: three weight tiles of the
+    # E4M3 GEMM (192 rows each), the last one ragged.
     codes, scales = moe_weights(E, N, K, fmt)
     ids, w = synth.routing(7, T, E, topk)
     x = x_bits(T, K, seed=17)
@@ -287,6 +310,50 @@ def test_moe_gate_up_grouped_parity(fmt, T, E, topk, N, K):
         y = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, N, fmt=fmt, flags=Q.HADAMARD,
                           topk_weights=dev(w))
         assert_close(y.cpu().numpy(), ref, f"moe grouped fmt {fmt} T{T} E{E}")
+
+
+@pytest.mark.parametrize("T,E,topk,K,I", [(1, 8, 2, 96, 64), (4, 16, 4, 130, 128), (16, 32, 8, 64, 192),
+                                          (20, 32, 8, 200, 64), (300, 16, 8, 48, 128)])
+def test_moe_down_combine_parity(T, E, topk, K, I):
+    # T * topk <= 128: the down GEMM ranks the ids itself; 160 and 2400 pairs: the permute kernel's
+    # chunks.  K = 130, 200: ragged 16-row slabs of the down weights.
+    d = synth.moe_down(T, seed=3, E=E, topk=topk, K=K, I=I)
+    wd = np.stack([d["Wd"][e] for e in range(E)])
+    ref = O.moe_down_combine(d["h"], d["ids"], d["weights"], wd, E)
+    for _ in range(2):
+        out = Q.moe_down_combine(dev(d["h"]), dev(d["ids"]), dev(d["weights"]), dev(wd.view(np.int16)), E)
+        assert_close(out.cpu().numpy(), ref, f"down T{T} E{E} K{K} I{I}")
+
+
+@pytest.mark.parametrize("T", [4, 20])
+def test_moe_down_combine_bad_id(T):
+    E, topk, K, I = 8, 8 if T == 20 else 2, 64, 64
+    d = synth.moe_down(T, seed=4, E=E, topk=topk, K=K, I=I)
+    wd = np.stack([d["Wd"][e] for e in range(E)])
+    ids = d["ids"].copy()
+    ids[1, 1] = E + 5  # adds nothing, flagged
+    Q.ql_get_device_error()
+    out = Q.moe_down_combine(dev(d["h"]), dev(ids), dev(d["weights"]), dev(wd.view(np.int16)), E).cpu().numpy()
+    st, bits = Q.ql_get_device_error()
+    assert st == 6 and bits & Q.DEVERR_EXPERT_ID
+    assert_close(out, O.moe_down_combine(d["h"], ids, d["weights"], wd, E), "down with a bad id")
+
+
+def test_moe_gate_up_then_down_combine():
+    """The whole routed-expert MLP: gate_up (int8 experts in the rotated domain) then the bf16 down
+    projection and the combine, against the oracle's two steps (its gate_up output rounded to fp32,
+    the input the down step takes)."""
+    T, E, topk, K, I = 12, 16, 4, 256, 128
+    codes, scales = moe_weights(E, 2 * I, K, Q.I8_G128_BF16)
+    dd = synth.moe_down(T, seed=5, E=E, topk=topk, K=K, I=I)
+    wd = np.stack([dd["Wd"][e] for e in range(E)])
+    ids, w = dd["ids"], dd["weights"]
+    x = x_bits(T, K, seed=23)
+    h = Q.moe_gate_up(dev_bf16(x), dev(ids), dev(codes), dev(scales), E, 2 * I, fmt=Q.I8_G128_BF16,
+                      flags=Q.HADAMARD)
+    out = Q.moe_down_combine(h, dev(ids), dev(w), dev(wd.view(np.int16)), E).cpu().numpy()
+    h_ref = O.moe_gate_up(x, ids, codes, scales, Q.I8_G128_BF16, O.HADAMARD, E, 2 * I).astype(np.float32)
+    assert_close(out, O.moe_down_combine(h_ref, ids, w, wd, E), "gate_up then down")
 
 
 def test_moe_gate_up_grouped_bad_id():
