@@ -52,7 +52,8 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "prefill_w5a8",
-                                          "moe_decode", "moe_decode_t1", "moe_prefill"],
+                                          "moe_decode", "moe_decode_t1", "moe_prefill", "act_quant", "decode_w4a16",
+                                          "decode_w5a16", "decode_w8a16", "decode_fp8"],
                    default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
@@ -363,6 +364,7 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
                                       "us_call_graph": us_call,
                                       "roofline": "max(bytes / measured HBM, flops / measured bf16 peak)"}
         del codes, scales, xT, idsT, yT
+        out.update(moe_extras(torch, Q, synth, dev, stream, hbm))
         # prefill W8A8 at M = 2048 (tcgen05 kind::i8 GEMM with per-group fp32 promotion)
         M = 2048
         d = synth.prefill(M=M)
@@ -444,6 +446,78 @@ def run_extras(torch, Q, synth, dev, stream, hbm):
     return out
 
 
+def moe_extras(torch, Q, synth, dev, stream, hbm):
+    """The fp8 experts with E4M3 activations (format 7) at the MoE workload's decode and prefill batch
+    sizes, and the bf16 down projection with its routing-weighted combine: whole calls replayed from a
+    CUDA graph, and the expert GEMM alone from the launch trace."""
+    out = {}
+    E, topk, Ke, Ne, I = 128, 8, 2816, 1408, 704
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    Ws = synth.moe_gate_up(1, experts=range(E))["W"]
+    sb = (Ne + 127) // 128 * (Ke // 128)
+    codes = torch.empty((E, Ne, Ke), dtype=torch.uint8, device=dev)
+    scales = torch.empty((E, sb), dtype=torch.int16, device=dev)
+    for e in range(E):
+        c, s, _ = Q.qlinear_pack(Q.FP8A8_B128_BF16, Ne, Ke, W=torch.from_numpy(Ws[e]).to(dev), flags=Q.HADAMARD)
+        codes[e] = c.reshape(Ne, Ke)
+        scales[e] = s.view(torch.int16)
+    del Ws
+    res = {}
+    for T in (1, 16, 2048):
+        ids, _ = synth.routing(300 + T, T, E, topk)
+        x = bf(synth.activations(0, f"x_T{T}", T, Ke))
+        idt = torch.from_numpy(ids).to(dev)
+        y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+        ws = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.FP8A8_B128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
+                         device=dev)
+        run = lambda i: Q.moe_gate_up(x, idt, codes, scales, E, Ne, fmt=Q.FP8A8_B128_BF16,  # noqa: E731
+                                      flags=Q.HADAMARD, y=y, ws=ws, stream=stream)
+        for i in range(3):
+            run(i)
+        t, per = _traced(Q, run, 10, "moe_gemm")
+        us_call = _graph_call_us(torch, run, stream, calls=16 if T == 2048 else 64, reps=3 if T == 2048 else 10)
+        touched = len(set(ids.ravel().tolist()))
+        byts = touched * (Ne * Ke + sb * 2) + T * Ke * 2 + T * topk * Ne * 4
+        flops = 2.0 * T * topk * Ne * Ke
+        r = {"us_gemm": 1e3 * t, "us_call_graph": us_call, "touched_experts": touched,
+             "GB/s": byts / (t * 1e-3) / 1e9, "frac_hbm": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per}
+        if T == 2048:
+            r["TFLOPS"] = flops / (t * 1e-3) / 1e12
+            r["frac_of_fp8_peak"] = r["TFLOPS"] / (2.0 * peaks()[1])
+        res[str(T)] = r
+    out["moe_gate_up_fp8a8"] = res
+    del codes, scales
+    # down projection: bf16 [128][2816][704] (507 MB), routing-weighted combine into [T, 2816]
+    wd = torch.empty((E, Ke, I), dtype=torch.int16, device=dev)
+    dd = synth.moe_down(1, experts=range(E))
+    for e in range(E):
+        wd[e] = torch.from_numpy(dd["Wd"][e].view(np.int16)).to(dev)
+    del dd
+    res = {}
+    for T in (1, 16, 2048):
+        d = synth.moe_down(T, experts=[])
+        h = torch.from_numpy(d["h"]).to(dev)
+        idt = torch.from_numpy(d["ids"]).to(dev)
+        wt = torch.from_numpy(d["weights"]).to(dev)
+        o = torch.empty((T, Ke), dtype=torch.float32, device=dev)
+        ws = torch.empty(Q.moe_down_workspace_size(E, Ke, I, T, topk), dtype=torch.uint8, device=dev)
+        run = lambda i: Q.moe_down_combine(h, idt, wt, wd, E, out=o, ws=ws, stream=stream)  # noqa: E731
+        for i in range(3):
+            run(i)
+        t, per = _traced(Q, run, 10 if T < 2048 else 3, "moe_down")
+        us_call = _graph_call_us(torch, run, stream, calls=16 if T == 2048 else 64, reps=2 if T == 2048 else 10)
+        touched = len(set(d["ids"].ravel().tolist()))
+        byts = touched * Ke * I * 2 + T * topk * 2 * I * 4 + T * Ke * 4
+        flops = 2.0 * T * topk * Ke * I
+        res[str(T)] = {"us_gemm": 1e3 * t, "us_call_graph": us_call, "touched_experts": touched,
+                       "GB/s": byts / (t * 1e-3) / 1e9, "frac_hbm": byts / (t * 1e-3) / 1e9 / hbm,
+                       "TFLOPS": flops / (t * 1e-3) / 1e12, "launches_per_call": per}
+    out["moe_down_combine"] = res
+    del wd
+    torch.cuda.synchronize()
+    return out
+
+
 def ncu_case(name):
     """A small, fixed launch sequence for one ncu capture.
     skinny_w8a8: the W8A8 weight at full size (117 MB codes, two copies so each
@@ -453,6 +527,12 @@ def ncu_case(name):
     N = 21504, K = 5376; about 0.6 GB on the device), four forwards; the tcgen05
     GEMM (k_prefill_w8a8, which also runs format 7, / k_prefill_a16) is launch
     1..4 of its name.
+    act_quant: the rotation + int8 quantiser on 16384 x 5376 bf16 (176 MB, more
+    than L2), four calls.
+    decode_w4a16 / decode_w5a16 / decode_w8a16 / decode_fp8: a weight-only
+    decode forward at M = 1 on the full 21504 x 5376 weight of that format (two
+    packed copies, alternating), four forwards; the decode GEMM is launch 1..4 of
+    k_skinny_tma.
     prefill_w5a8: the int5 weight of the W5A16 workload with M = 2048 tokens
     (int8 activations), four forwards: act quant, scale prep, int5 -> int8 code
     conversion (k_prefill_i5_codes) and the W8A8 GEMM each launch four times.
@@ -466,6 +546,42 @@ def ncu_case(name):
     from moe_hadamard128_act_b200 import synth
 
     dev = torch.device("cuda", 0)
+    if name.startswith("decode_"):
+        # a weight-only decode forward at M = 1 on the full 21504 x 5376 weight (two packed copies,
+        # so no launch finds its weight in L2): two warm-up forwards, then two more
+        fmt = {"decode_w4a16": Q.I4_G64_BF16, "decode_w5a16": Q.I5Z_G128_F16, "decode_w8a16": Q.I8_G128_BF16,
+               "decode_fp8": Q.FP8_B128_BF16}[name]
+        if fmt in (Q.I4_G64_BF16, Q.I5Z_G128_F16):
+            d = synth.w4a16(1) if fmt == Q.I4_G64_BF16 else synth.w5a16(1)
+            z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None
+            c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
+                                      scales=torch.from_numpy(d["scales"].view(np.int16)).to(dev), zeros=z)
+        else:
+            W = torch.from_numpy(synth.weight_rows(0, "W", K_FULL, 0, N_FULL)).to(dev)
+            c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=W)
+            del W
+        cp = [(c, s, zz), (c.clone(), s.clone(), None if zz is None else zz.clone())]
+        x = torch.from_numpy(synth.activations(0, "x_M1", 1, K_FULL).view(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((1, N_FULL), dtype=torch.float32, device=dev)
+        for i in range(4):
+            Q.qlinear_forward(x, cp[i % 2][0], cp[i % 2][1], cp[i % 2][2], fmt, N_FULL, y=y)
+        torch.cuda.synchronize()
+        st, bits = Q.ql_get_device_error()
+        assert st == 0, bits
+        print(f"ncu case {name} done")
+        return
+    if name == "act_quant":
+        # the fused rotation + int8 quantiser on 16384 tokens of K = 5376 (176 MB of bf16 in, more
+        # than L2), four calls
+        M = 16384
+        x = torch.from_numpy(synth.activations(0, "x_aq", M, K_FULL).view(np.int16)).view(torch.bfloat16).to(dev)
+        for i in range(4):
+            Q.act_quant_i8_g128(x, rotate=True)
+        torch.cuda.synchronize()
+        st, bits = Q.ql_get_device_error()
+        assert st == 0, bits
+        print(f"ncu case {name} done")
+        return
     if name.startswith("moe"):
         E, topk, Ke, Ne = 128, 8, 2816, 1408
         T = {"moe_decode": 16, "moe_decode_t1": 1}.get(name, 2048)

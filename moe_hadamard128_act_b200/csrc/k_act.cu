@@ -89,19 +89,37 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // One CTA per token.  The (optionally rotated and bf16-rounded) row is kept in
 // shared memory as fp32; its max |x| picks a power of two f with
 // max|x| * f in [2^14, 2^15), and xs = f16(x * f) is written in the element
-// order of the format (within each 8-block [0,4,1,5,2,6,3,7] for int4, within
-// each 4-block [0,3,1,2] for int5, natural otherwise; for int5 the 16-byte
-// pieces of each 128-group are also swapped pairwise in their upper half, the
-// shared-memory layout the GEMM reads without bank conflicts).  xf = 1 / f.
+// order of the format (within each 8-block [0,4,1,5,2,6,3,7] for int4,
+// natural otherwise), and xf = 1 / f.  For int5 each 32-element run of a
+// 128-group holds, in MMA slot order, the activations of the run's codes as
+// the decode GEMM extracts them (kI5Pairs), each divided by 2^o for its code's
+// offset o; the 16-byte pieces of each group are also swapped pairwise in
+// their upper half (the shared-memory layout the GEMM reads without bank
+// conflicts); xsum[t][g] = the group's sum of f16(x * f) (for the zero point),
+// and xf = 2^24 / f (the codes enter the MMAs as u * 2^-24).
 // f16 holds every bf16 value of the scaled row exactly down to 2^-14 (its
 // normal range); below that the rounding error is under 2^-39 of the row's
 // max, far beneath the fp32 accumulation error of the GEMM.
 // With inv != null the row is written to rows inv[t * topk + j] (j < topk,
 // negative entries skipped) instead of row t: the permuted order of the
 // grouped expert GEMM.
+// Slots SL .. 31 of one int5 lane run starting at element b: the f16 activation
+// of the slot's code (i5_slot_code), divided by 2^o (i5_slot_off), to its
+// place with the pairwise piece swap.
+template <int SL>
+__device__ __forceinline__ void i5_stage_run(const float* r, float f, __half* out, int b) {
+    if constexpr (SL < 32) {
+        constexpr int code = i5_slot_code(SL), off = i5_slot_off(SL);
+        const __half h = __float2half_rn(__fmul_rn(r[code], f));
+        const int k = b + SL;
+        out[k ^ (((k >> 6) & 1) << 3)] = __float2half_rn(__fmul_rn(__half2float(h), 1.0f / (float)(1 << off)));
+        i5_stage_run<SL + 1>(r, f, out, b);
+    }
+}
+
 __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M, int K, int rotate, int order,
                                                   __half* xs, float* xf, float* yz, long long nz, const int32_t* inv,
-                                                  int topk) {
+                                                  int topk, float* xsum) {
     extern __shared__ float row[];  // [K] fp32, then (natural order) [K] f16
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y (CTAs past M only help with this)
@@ -135,7 +153,7 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
         if (m > 0.0f && m <= 3.4e38f) frexpf(m, &e);
         e = max(-100, min(128, e));
         red[0] = ldexpf(1.0f, 15 - e);
-        xf[t] = ldexpf(1.0f, e - 15);
+        xf[t] = ldexpf(1.0f, e - 15 + (order == XORD_I5 ? 24 : 0));
     }
     __syncthreads();
     const float f = red[0];
@@ -163,18 +181,29 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
         return;
     }
     __half* out = xs + (long long)t * K;
+    if (order == XORD_I5) {
+        const int lane5 = threadIdx.x & 31, warp5 = threadIdx.x >> 5;
+        for (int g = warp5; g < K / 128; g += 8) {  // the groups' sums of the f16 activations
+            float sum = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sum += __half2float(__float2half_rn(__fmul_rn(row[g * 128 + 4 * lane5 + i], f)));
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
+            if (lane5 == 0) xsum[(long long)t * (K / 128) + g] = sum;
+        }
+    }
+    if (order == XORD_I5) {
+        for (int run = threadIdx.x; run < K / 32; run += 256)  // one lane's 32 codes of a group
+            i5_stage_run<0>(row + run * 32, f, out, run * 32);
+        return;
+    }
     for (int k = threadIdx.x; k < K; k += 256) {
         int src = k;
         if (order == XORD_I4) {
             const int p = k & 7;
             src = (k & ~7) + ((p & 1) ? 4 + (p >> 1) : (p >> 1));
-        } else if (order == XORD_I5) {
-            const int p = k & 3;
-            src = (k & ~3) + (p == 0 ? 0 : (p == 1 ? 3 : p - 1));
         }
-        int dst = k;
-        if (order == XORD_I5) dst = k ^ (((k >> 6) & 1) << 3);  // piece j -> j ^ bit3(j): conflict-free staging
-        out[dst] = __float2half_rn(__fmul_rn(row[src], f));
+        out[k] = __float2half_rn(__fmul_rn(row[src], f));
     }
 }
 
@@ -295,7 +324,8 @@ cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8
 }
 
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
-                            long long nz, cudaStream_t s) {
+                            long long nz, cudaStream_t s, float* xsum) {
+    if (order == XORD_I5 && !xsum) return cudaErrorInvalidValue;
     const size_t smem = (size_t)K * (sizeof(float) + sizeof(__half));  // the fp32 row and its f16 copy
     cudaError_t e = prefer_max_shared(k_prep_a16);
     if (e != cudaSuccess) return e;
@@ -310,7 +340,7 @@ cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, 
     const long long zc = zb < 2LL * di.sm_count ? zb : 2LL * di.sm_count;
     const int grid = (int)(M > zc ? M : zc);
     k_prep_a16<<<grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), M, K, rotate, order, xs, xf, yz, nz,
-                                       nullptr, 1);
+                                       nullptr, 1, xsum);
     return cudaGetLastError();
 }
 
@@ -324,7 +354,7 @@ cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, con
         if (e != cudaSuccess) return e;
     }
     k_prep_a16<<<T, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), T, K, rotate, XORD_NATURAL, xs, xf, nullptr, 0,
-                                    inv, topk);
+                                    inv, topk, nullptr);
     return cudaGetLastError();
 }
 

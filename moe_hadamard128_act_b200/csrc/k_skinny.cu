@@ -86,7 +86,7 @@ template <>
 struct Regs<QL_I5Z_G128_F16> {
     uint32_t w[2][5];  // [row][160-bit stream of 32 codes]
     float s[2];
-    uint32_t nz[2];  // f16x2 of -(1024 + zero point)
+    float zz[2];  // zero point * 2^-24 (the codes' unit in the MMAs)
 };
 
 // Bytes of activations per token per 128-group in shared memory, and the
@@ -105,61 +105,6 @@ template <int FMT>
 __device__ __forceinline__ float load_scale(const void* scales, long long idx) {
     const uint16_t b = __ldg(static_cast<const uint16_t*>(scales) + idx);
     return (FMT == QL_I8_G128_F16 || FMT == QL_I5Z_G128_F16) ? f16_bits_to_float(b) : bf16_bits_to_float(b);
-}
-
-// Load one unit (rows n0 = slab*16 + g and n0 + 8, group grp) for lane (g, c).
-// `wbase` points at the codes of row 0 of the matrix (group offset applied),
-// `sbase`/`zbase` index the scales and zeros with row stride Gtot.
-template <int FMT>
-__device__ __forceinline__ void load_unit(Regs<FMT>& r, const uint8_t* wbase, long long ldw, const void* scales,
-                                          const uint8_t* zeros, int N, int Gtot, int gabs, int slab, int grp, int g,
-                                          int c) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int n = slab * 16 + g + 8 * h;
-        const bool ok = n < N;
-        const uint8_t* row = wbase + (long long)n * ldw;
-        if constexpr (FMT == QL_I4_G64_BF16) {
-            if (ok) {
-                const uint8_t* p = row + grp * 64 + 8 * c;
-                r.w[h][0] = ldg_stream64(p);
-                r.w[h][1] = ldg_stream64(p + 32);
-                r.s[h][0] = load_scale<FMT>(scales, (long long)n * (2 * Gtot) + 2 * gabs);
-                r.s[h][1] = load_scale<FMT>(scales, (long long)n * (2 * Gtot) + 2 * gabs + 1);
-            } else {
-                r.w[h][0] = r.w[h][1] = make_uint2(0x88888888u, 0x88888888u);
-                r.s[h][0] = r.s[h][1] = 0.0f;
-            }
-        } else if constexpr (FMT == QL_I5Z_G128_F16) {
-            if (ok) {
-                const uint8_t* p = row + grp * 80 + 20 * c;
-#pragma unroll
-                for (int i = 0; i < 5; ++i) r.w[h][i] = ldg_stream32(p + 4 * i);
-                r.s[h] = load_scale<FMT>(scales, (long long)n * Gtot + gabs);
-                const float z = (float)__ldg(zeros + (long long)n * Gtot + gabs);
-                const __half nz = __float2half_rn(-(1024.0f + z));
-                r.nz[h] = (uint32_t)__half_as_ushort(nz) * 0x10001u;
-            } else {
-#pragma unroll
-                for (int i = 0; i < 5; ++i) r.w[h][i] = 0;
-                r.s[h] = 0.0f;
-                r.nz[h] = 0xE400E400u;  // -1024
-            }
-        } else {
-            if (ok) {
-                const uint8_t* p = row + grp * 128 + 32 * c;
-                r.w[h][0] = ldg_stream128(p);
-                r.w[h][1] = ldg_stream128(p + 16);
-                if constexpr (block_scaled<FMT>())
-                    r.s[h] = load_scale<FMT>(scales, (long long)(n >> 7) * Gtot + gabs);
-                else  // the integer-only W8A8 check path has no scales
-                    r.s[h] = scales ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
-            } else {
-                r.w[h][0] = r.w[h][1] = make_uint4(0, 0, 0, 0);
-                r.s[h] = 0.0f;
-            }
-        }
-    }
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 (&w)[2], int s) {
@@ -231,15 +176,7 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
             for (int sub = 0; sub < 2; ++sub) {
                 const int s = 2 * p + sub;
                 uint32_t a0, a1, a2, a3;
-                if constexpr (FMT == QL_I5Z_G128_F16) {
-                    const int bit = 20 * s, wi = bit >> 5, sh = bit & 31;
-                    const uint32_t t0 = __funnelshift_r(r.w[0][wi], wi < 4 ? r.w[0][wi + 1] : 0u, sh);
-                    const uint32_t t1 = __funnelshift_r(r.w[1][wi], wi < 4 ? r.w[1][wi + 1] : 0u, sh);
-                    a0 = hadd2_u32((t0 & 0x1Fu) | ((t0 << 1) & 0x1F0000u) | 0x64006400u, r.nz[0]);
-                    a2 = hadd2_u32(((t0 >> 5) & 0x1Fu) | ((t0 << 6) & 0x1F0000u) | 0x64006400u, r.nz[0]);
-                    a1 = hadd2_u32((t1 & 0x1Fu) | ((t1 << 1) & 0x1F0000u) | 0x64006400u, r.nz[1]);
-                    a3 = hadd2_u32(((t1 >> 5) & 0x1Fu) | ((t1 << 6) & 0x1F0000u) | 0x64006400u, r.nz[1]);
-                } else if constexpr (FMT == QL_FP8_B128_BF16) {
+                if constexpr (FMT == QL_FP8_B128_BF16) {
                     const uint32_t w0 = word_of(r.w[0], s), w1 = word_of(r.w[1], s);
                     a0 = e4m3x2_to_f16x2(w0);
                     a2 = e4m3x2_to_f16x2(w0 >> 16);
@@ -266,6 +203,64 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
             yacc[nt][3] = fmaf(r.s[1], acc[nt][3], yacc[nt][3]);
         }
     }
+}
+
+// int5 register pair Q of a row (kI5Pairs): the stream window at bit B masked to
+// its two codes, each an exact f16 subnormal u * 2^(o - 24).
+template <int Q>
+__device__ __forceinline__ uint32_t i5_pair(const uint32_t (&w)[5]) {
+    constexpr int B = kI5Pairs[Q].B, wi = B >> 5, sh = B & 31;
+    constexpr uint32_t mask = (0x1Fu << i5_off_lo(Q)) | ((0x1Fu << i5_off_hi(Q)) << 16);
+    uint32_t win;
+    if constexpr (sh == 0) win = w[wi];
+    else win = __funnelshift_r(w[wi], wi < 4 ? w[wi + 1] : 0u, sh);
+    return win & mask;
+}
+
+// One int5 unit (16 rows x 128 K): 28 integer instructions per row make the
+// 16 operand pairs, eight MMAs per n-tile sum u * x * 2^-24 over the group, and
+// the zero point comes off with the token's group sum X (same units after
+// zz = z * 2^-24) before the scale: y += s * (acc - zz * X).
+template <int NT, typename GetX>
+__device__ __forceinline__ void unit_i5(const Regs<QL_I5Z_G128_F16>& r, GetX getx, bool nt1_live,
+                                        const float (&X)[NT][2], float (&yacc)[NT][4]) {
+    uint32_t A[2][16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        A[h][0] = i5_pair<0>(r.w[h]);   A[h][1] = i5_pair<1>(r.w[h]);   A[h][2] = i5_pair<2>(r.w[h]);
+        A[h][3] = i5_pair<3>(r.w[h]);   A[h][4] = i5_pair<4>(r.w[h]);   A[h][5] = i5_pair<5>(r.w[h]);
+        A[h][6] = i5_pair<6>(r.w[h]);   A[h][7] = i5_pair<7>(r.w[h]);   A[h][8] = i5_pair<8>(r.w[h]);
+        A[h][9] = i5_pair<9>(r.w[h]);   A[h][10] = i5_pair<10>(r.w[h]); A[h][11] = i5_pair<11>(r.w[h]);
+        A[h][12] = i5_pair<12>(r.w[h]); A[h][13] = i5_pair<13>(r.w[h]); A[h][14] = i5_pair<14>(r.w[h]);
+        A[h][15] = i5_pair<15>(r.w[h]);
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {  // the lane's 16-byte activation piece p feeds MMAs 2p and 2p + 1
+        uint4 xv[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            if (nt == 0 || nt1_live) xv[nt] = getx(nt, p);
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+            const int m = 2 * p + sub;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                if (nt == 1 && !nt1_live) continue;
+                mma_f16(acc[nt], A[0][2 * m], A[1][2 * m], A[0][2 * m + 1], A[1][2 * m + 1],
+                        sub == 0 ? xv[nt].x : xv[nt].z, sub == 0 ? xv[nt].y : xv[nt].w);
+            }
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float t = fmaf(-r.zz[i >> 1], X[nt][i & 1], acc[nt][i]);
+            yacc[nt][i] = fmaf(r.s[i >> 1], t, yacc[nt][i]);
+        }
 }
 
 // E4M3 x E4M3 -> fp32 (format 7): the same fragments as the s8 MMA.
@@ -405,14 +400,23 @@ __host__ __device__ constexpr int tx_row_pad() {
     return act8<FMT>() ? 64 : (FMT == QL_I5Z_G128_F16 ? 32 : 16);
 }
 
-template <int FMT>
-__host__ __device__ constexpr size_t ring_bytes() {
-    return (size_t)kWarps * kStages * stage_bytes<FMT>();
+// The nibble formats put UPS = 2 consecutive units of a row slab in one ring
+// slot (two TMA boxes, one barrier): the per-slot waits, refills and
+// bookkeeping then cover 2 KB (int4) or 2.5 KB (int5) of weights instead of
+// half that.  The 2.5 KB int5 slots take three ring stages instead of four.
+template <int FMT, int UPS = 1>
+__host__ __device__ constexpr int stages_of() {
+    return (FMT == QL_I5Z_G128_F16 && UPS == 2) ? 3 : kStages;
 }
-template <int FMT>
-__host__ __device__ constexpr size_t tma_smem(int NT, int XG) {
-    return 1024 /* alignment slack */ + ring_bytes<FMT>() + (size_t)kWarps * kStages * 8 + 16 +
-           (size_t)NT * 8 * ((size_t)XG * tx_group_bytes<FMT>() + tx_row_pad<FMT>());
+template <int FMT, int UPS = 1>
+__host__ __device__ constexpr size_t ring_bytes() {
+    return (size_t)kWarps * stages_of<FMT, UPS>() * UPS * stage_bytes<FMT>();
+}
+// Shared memory of the dense kernel staging `rows` token rows of XG groups.
+template <int FMT, int UPS>
+__host__ __device__ constexpr size_t tma_smem(int rows, int XG) {
+    return 1024 /* alignment slack */ + ring_bytes<FMT, UPS>() + (size_t)kWarps * stages_of<FMT, UPS>() * 8 + 16 +
+           (size_t)rows * ((size_t)XG * tx_group_bytes<FMT>() + tx_row_pad<FMT>());
 }
 
 // Position in the unit stream: K part, row slab, group within the part.
@@ -438,39 +442,6 @@ struct UnitPos {
     }
     __device__ __forceinline__ int grp(int GP) const { return part * GP + gi; }
 };
-
-template <int FMT>
-__device__ __forceinline__ void load_unit_scales(Regs<FMT>& r, const void* scales, const uint8_t* zeros, int N,
-                                                 int Gtot, int gabs, int slab, int g) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int n = slab * 16 + g + 8 * h;
-        const bool ok = n < N;
-        if constexpr (FMT == QL_I4_G64_BF16) {
-            r.s[h][0] = ok ? load_scale<FMT>(scales, (long long)n * (2 * Gtot) + 2 * gabs) : 0.0f;
-            r.s[h][1] = ok ? load_scale<FMT>(scales, (long long)n * (2 * Gtot) + 2 * gabs + 1) : 0.0f;
-        } else if constexpr (FMT == QL_I5Z_G128_F16) {
-            r.s[h] = ok ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
-            const float z = ok ? (float)__ldg(zeros + (long long)n * Gtot + gabs) : 0.0f;
-            r.nz[h] = (uint32_t)__half_as_ushort(__float2half_rn(-(1024.0f + z))) * 0x10001u;
-        } else if constexpr (FMT == QL_FP8_B128_BF16) {
-            r.s[h] = ok ? load_scale<FMT>(scales, (long long)(n >> 7) * Gtot + gabs) : 0.0f;
-        } else {
-            r.s[h] = (ok && scales) ? load_scale<FMT>(scales, (long long)n * Gtot + gabs) : 0.0f;
-        }
-    }
-}
-
-template <int FMT>
-__device__ __forceinline__ void copy_scales(Regs<FMT>& d, const Regs<FMT>& s) {
-    if constexpr (FMT == QL_I4_G64_BF16) {
-        d.s[0][0] = s.s[0][0]; d.s[0][1] = s.s[0][1]; d.s[1][0] = s.s[1][0]; d.s[1][1] = s.s[1][1];
-    } else if constexpr (FMT == QL_I5Z_G128_F16) {
-        d.s[0] = s.s[0]; d.s[1] = s.s[1]; d.nz[0] = s.nz[0]; d.nz[1] = s.nz[1];
-    } else {
-        d.s[0] = s.s[0]; d.s[1] = s.s[1];
-    }
-}
 
 // The lane's weight fragments of one unit, out of its ring slot.
 template <int FMT>
@@ -519,9 +490,9 @@ __device__ unsigned long long g_skinny_prof[148 * 16];
 // activation scales of the lane's output tokens (W8A8 and format 7).
 template <int FMT, int NT>
 struct Side {
-    uint32_t sw[2][2];  // weight scale bits [row g / g+8][int4 half]
+    uint32_t sw[2][1];  // weight scale bits [row g / g+8] (int4: both 64-groups' bf16 scales in one word)
     uint32_t z[2];      // int5 zero points
-    float sx[NT][2];    // byte activations: scales of tokens 8nt + 2c + {0, 1}
+    float sx[NT][2];    // byte activations: scales of tokens 8nt + 2c + {0, 1}; int5: their group sums
 };
 
 template <int FMT, int NT>
@@ -532,9 +503,8 @@ __device__ __forceinline__ void load_side_w(Side<FMT, NT>& d, const void* scales
     for (int h = 0; h < 2; ++h) {
         const int n = slab * 16 + g + 8 * h;
         const bool ok = n < N && sc;
-        if constexpr (FMT == QL_I4_G64_BF16) {
-            d.sw[h][0] = ok ? __ldg(sc + (long long)n * (2 * Gtot) + 2 * gabs) : 0u;
-            d.sw[h][1] = ok ? __ldg(sc + (long long)n * (2 * Gtot) + 2 * gabs + 1) : 0u;
+        if constexpr (FMT == QL_I4_G64_BF16) {  // the unit's two bf16 scales, adjacent: one 32-bit load
+            d.sw[h][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(sc + (long long)n * (2 * Gtot) + 2 * gabs)) : 0u;
         } else if constexpr (block_scaled<FMT>()) {
             d.sw[h][0] = ok ? __ldg(sc + (long long)(n >> 7) * Gtot + gabs) : 0u;
         } else {
@@ -546,7 +516,7 @@ __device__ __forceinline__ void load_side_w(Side<FMT, NT>& d, const void* scales
 
 template <int FMT, int NT>
 __device__ __forceinline__ void load_side_x(Side<FMT, NT>& d, const float* sx, int M, int Gtot, int gabs, int c) {
-    if constexpr (act8<FMT>()) {
+    if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16) {  // int5: the tokens' group sums
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -568,17 +538,21 @@ __device__ __forceinline__ void side_to_regs(Regs<FMT>& r, const Side<FMT, NT>& 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         if constexpr (FMT == QL_I4_G64_BF16) {
-            r.s[h][0] = scale_value<FMT>(d.sw[h][0]);
-            r.s[h][1] = scale_value<FMT>(d.sw[h][1]);
+            r.s[h][0] = __uint_as_float(d.sw[h][0] << 16);
+            r.s[h][1] = __uint_as_float(d.sw[h][0] & 0xFFFF0000u);
         } else {
             r.s[h] = scale_value<FMT>(d.sw[h][0]);
         }
-        if constexpr (FMT == QL_I5Z_G128_F16)
-            r.nz[h] = (uint32_t)__half_as_ushort(__float2half_rn(-(1024.0f + (float)d.z[h]))) * 0x10001u;
+        if constexpr (FMT == QL_I5Z_G128_F16) r.zz[h] = (float)d.z[h] * 5.9604644775390625e-8f;  // z * 2^-24
     }
 }
 
-template <int FMT, int NT, bool ACC>
+//
+// Slot positions count in slots of UPS units (UPS consecutive groups of one
+// slab): G, GP and the unit positions below are in those, the activations'
+// staging and the scale indices in groups.  Only the token rows that exist
+// are staged; fragments of the others are zeros taken without a load.
+template <int FMT, int NT, bool ACC, int UPS>
 __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constant__ SkinnyArgs a) {
     extern __shared__ uint8_t smem_raw[];
 #ifdef QL_SKINNY_PROFILE
@@ -587,23 +561,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
 #endif
     QL_PROF(0)
     constexpr int XGB = tx_group_bytes<FMT>();
-    constexpr int SB = stage_bytes<FMT>();
+    constexpr int ST = stages_of<FMT, UPS>();
+    constexpr int SB1 = stage_bytes<FMT>();  // one unit
+    constexpr int SB = UPS * SB1;             // one ring slot
+    constexpr int URB = unit_row_bytes<FMT>();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
-    const int G = a.G, GP = a.GP, slabs = (a.N + 15) / 16;
+    const int G = a.G / UPS, GP = a.GP / UPS, slabs = (a.N + 15) / 16;
     if (lane == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmap) : "memory");
 
     // Shared memory: [rings][mbarriers][activation barrier][activations], 1024-aligned base.
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* const gbase = smem_raw + (base - raw);
-    const uint32_t ring = base + (uint32_t)(warp * kStages * SB);
-    const uint32_t bars = base + (uint32_t)ring_bytes<FMT>() + (uint32_t)(warp * kStages * 8);
-    const uint32_t xbar = base + (uint32_t)ring_bytes<FMT>() + kWarps * kStages * 8;
-    const uint32_t xs_off = (uint32_t)ring_bytes<FMT>() + kWarps * kStages * 8 + 16;
+    constexpr uint32_t RB = (uint32_t)ring_bytes<FMT, UPS>();
+    const uint32_t ring = base + (uint32_t)(warp * ST * SB);
+    const uint32_t bars = base + RB + (uint32_t)(warp * ST * 8);
+    const uint32_t xbar = base + RB + kWarps * ST * 8;
+    const uint32_t xs_off = RB + kWarps * ST * 8 + 16;
     const int R = a.XG * XGB + tx_row_pad<FMT>();
-    uint8_t* const xs = gbase + xs_off;
     const uint32_t xs_base = base + xs_off;
+    (void)gbase;
 
     // Work: the CTA's contiguous unit range, split contiguously over its warps
     // (32-bit: the host keeps units * gridDim below 2^31).
@@ -611,27 +589,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     const unsigned cu0 = units * blockIdx.x / gridDim.x, cu1 = units * (blockIdx.x + 1) / gridDim.x;
     const unsigned u0 = cu0 + (cu1 - cu0) * warp / kWarps, u1 = cu0 + (cu1 - cu0) * (warp + 1) / kWarps;
 
-    UnitPos cp;  // unit being computed
+    UnitPos cp;  // slot of units being computed
     if (u0 < u1) cp.init(u0, slabs, GP, G);
-    UnitPos ip = cp;  // next unit to issue
-    Side<FMT, NT> sd[kStages];
+    UnitPos ip = cp;  // next slot to issue
+    Side<FMT, NT> sd[ST][UPS];
     unsigned issued = u0;
     if (lane == 0) {
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) mbar_init(bars + 8 * s, 1);
+        for (int s = 0; s < ST; ++s) mbar_init(bars + 8 * s, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncwarp();
     QL_PROF(7)
+    // Issues slot s's TMA boxes (UPS consecutive groups of one slab) and fetches their side data.
+    auto issue = [&](int s) {
+        if (lane == 0) {
+            mbar_expect_tx(bars + 8 * s, SB);
+#pragma unroll
+            for (int i = 0; i < UPS; ++i)
+                tma_load_2d(ring + s * SB + i * SB1, &a.tmap, (UPS * ip.grp(GP) + i) * URB, ip.slab * 16,
+                            bars + 8 * s);
+        }
+#pragma unroll
+        for (int i = 0; i < UPS; ++i)
+            load_side_w<FMT, NT>(sd[s][i], a.scales, a.zeros, a.N, a.Gtot, a.g0 + UPS * ip.grp(GP) + i, ip.slab, g);
+    };
     // Start the weight stream first: it never depends on the kernel before.
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < ST; ++s) {
         if (issued < u1) {
-            if (lane == 0) {
-                mbar_expect_tx(bars + 8 * s, SB);
-                tma_load_2d(ring + s * SB, &a.tmap, ip.grp(GP) * unit_row_bytes<FMT>(), ip.slab * 16, bars + 8 * s);
-            }
-            load_side_w<FMT, NT>(sd[s], a.scales, a.zeros, a.N, a.Gtot, a.g0 + ip.grp(GP), ip.slab, g);
+            issue(s);
             ip.next(slabs, GP, G);
             ++issued;
         }
@@ -644,14 +631,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     QL_PROF(2)
 
     // Stage the activations of the K parts this CTA touches, one bulk copy per
-    // token row, while the weight stream runs; rows beyond M are zeroed.
+    // token row, while the weight stream runs (groups gs0 .. gs0 + ngs).
     int gs0 = 0, ngs = 0;
     if (cu1 > cu0) {
         UnitPos p0, p1;
         p0.init(cu0, slabs, GP, G);
         p1.init(cu1 - 1, slabs, GP, G);
-        gs0 = p0.part * GP;
-        ngs = min(G, (p1.part + 1) * GP) - gs0;
+        gs0 = p0.part * GP * UPS;
+        ngs = min(G, (p1.part + 1) * GP) * UPS - gs0;
     }
     const int rows_x = ngs > 0 ? min(a.M, NT * 8) : 0;
     if (threadIdx.x == 0) {
@@ -666,18 +653,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 bulk_load(xs_base + (uint32_t)(t * R), xsrc + t * ldx_b + (long long)gs0 * XGB, row_bytes, xbar);
         }
     }
-    {
-        const int pieces = ngs * XGB / 16;
-        for (int i = threadIdx.x; i < (NT * 8 - rows_x) * pieces; i += kThreads) {
-            const int t = rows_x + i / pieces, j = i % pieces;
-            *reinterpret_cast<uint4*>(xs + t * R + 16 * j) = make_uint4(0, 0, 0, 0);
-        }
-    }
-    if constexpr (act8<FMT>()) {  // activation scales of the units already in flight
+    // Per-token side data of the units already in flight: the activation scales (byte
+    // activations) or the group sums (int5), written by the kernel before this one.
+    const float* const xside = FMT == QL_I5Z_G128_F16 ? a.xsum : a.xf;
+    if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16) {
         UnitPos q = cp;
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) {
-            if (u0 + s < issued) load_side_x<FMT, NT>(sd[s], a.xf, a.M, a.Gtot, a.g0 + q.grp(GP), c);
+        for (int s = 0; s < ST; ++s) {
+            if (u0 + s < issued)
+#pragma unroll
+                for (int i = 0; i < UPS; ++i)
+                    load_side_x<FMT, NT>(sd[s][i], xside, a.M, a.Gtot, a.g0 + UPS * q.grp(GP) + i, c);
             q.next(slabs, GP, G);
         }
     }
@@ -714,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     unsigned u = u0;
     while (u < u1 && !timed_out) {
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < ST; ++s) {
             if (u >= u1) break;
             const int key = cp.part * slabs + cp.slab;
             if (!ACC && key != cur_key) {
@@ -725,62 +711,65 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 timed_out = true;
                 break;
             }
-            Regs<FMT> r;
-            side_to_regs<FMT, NT>(r, sd[s]);
-            read_unit_smem<FMT>(r, ring + s * SB, g, c);
-            const int grp = cp.grp(GP);
-            const int lg = grp - gs0;  // group index in the staged activations
-            auto getx = [&](int nt, int p) -> uint4 {
-                int j;
-                if constexpr (act8<FMT>())
-                    j = lg * 8 + 4 * p + c;
-                else if constexpr (FMT == QL_I4_G64_BF16)
-                    j = lg * 16 + (p & 8) + 2 * c + (p & 1);
-                else if constexpr (FMT == QL_I5Z_G128_F16) {
-                    j = lg * 16 + 4 * c + p;
-                    j ^= (j >> 3) & 1;
-                } else
-                    j = lg * 16 + (p >> 1) * 8 + 2 * c + (p & 1);
-                return lds128(xs_base + (uint32_t)((8 * nt + g) * R + 16 * j));
-            };
-            if constexpr (FMT == QL_I8A8_G128_BF16) {
-                int acc[NT][4];
-                unit_w8a8<NT>(r, getx, acc);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+            for (int ui = 0; ui < UPS; ++ui) {
+                Regs<FMT> r;
+                side_to_regs<FMT, NT>(r, sd[s][ui]);
+                read_unit_smem<FMT>(r, ring + s * SB + ui * SB1, g, c);
+                const int grp = UPS * cp.grp(GP) + ui;
+                const int lg = grp - gs0;  // group index in the staged activations
+                auto getx = [&](int nt, int p) -> uint4 {
+                    if (8 * nt + g >= rows_x) return make_uint4(0, 0, 0, 0);  // no such token
+                    int j;
+                    if constexpr (act8<FMT>())
+                        j = lg * 8 + 4 * p + c;
+                    else if constexpr (FMT == QL_I4_G64_BF16)
+                        j = lg * 16 + (p & 8) + 2 * c + (p & 1);
+                    else if constexpr (FMT == QL_I5Z_G128_F16) {
+                        j = lg * 16 + 4 * c + p;
+                        j ^= (j >> 3) & 1;
+                    } else
+                        j = lg * 16 + (p >> 1) * 8 + 2 * c + (p & 1);
+                    return lds128(xs_base + (uint32_t)((8 * nt + g) * R + 16 * j));
+                };
+                if constexpr (FMT == QL_I8A8_G128_BF16) {
+                    int acc[NT][4];
+                    unit_w8a8<NT>(r, getx, acc);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int t = 8 * nt + 2 * c + (i & 1);
-                        const int n = cp.slab * 16 + g + 8 * (i >> 1);
-                        if (ACC) {
-                            if (t < a.M && n < a.N)
-                                a.acc[((long long)t * a.N + n) * a.Gtot + a.g0 + grp] = acc[nt][i];
-                        } else {
-                            // |acc| <= 128 * 127^2 < 2^22: the magic-number conversion is exact.
-                            const float fa = __int_as_float(0x4B400000 + acc[nt][i]) - 12582912.0f;
-                            yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s].sx[nt][i & 1], fa, yacc[nt][i]);
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int t = 8 * nt + 2 * c + (i & 1);
+                            const int n = cp.slab * 16 + g + 8 * (i >> 1);
+                            if (ACC) {
+                                if (t < a.M && n < a.N)
+                                    a.acc[((long long)t * a.N + n) * a.Gtot + a.g0 + grp] = acc[nt][i];
+                            } else {
+                                // |acc| <= 128 * 127^2 < 2^22: the magic-number conversion is exact.
+                                const float fa = __int_as_float(0x4B400000 + acc[nt][i]) - 12582912.0f;
+                                yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s][ui].sx[nt][i & 1], fa, yacc[nt][i]);
+                            }
                         }
-                    }
-            } else if constexpr (FMT == QL_FP8A8_B128_BF16) {
-                float acc[NT][4];
-                unit_e4m3<NT>(r, getx, acc);
+                } else if constexpr (FMT == QL_FP8A8_B128_BF16) {
+                    float acc[NT][4];
+                    unit_e4m3<NT>(r, getx, acc);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s].sx[nt][i & 1], acc[nt][i], yacc[nt][i]);
-            } else {
-                unit_a16<FMT, NT>(r, getx, nt1_live, yacc);
+                        for (int i = 0; i < 4; ++i)
+                            yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s][ui].sx[nt][i & 1], acc[nt][i], yacc[nt][i]);
+                } else if constexpr (FMT == QL_I5Z_G128_F16) {
+                    unit_i5<NT>(r, getx, nt1_live, sd[s][ui].sx, yacc);
+                } else {
+                    unit_a16<FMT, NT>(r, getx, nt1_live, yacc);
+                }
             }
             __syncwarp();
-            if (issued < u1) {  // refill this slot with the unit kStages ahead
-                if (lane == 0) {
-                    mbar_expect_tx(bars + 8 * s, SB);
-                    tma_load_2d(ring + s * SB, &a.tmap, ip.grp(GP) * unit_row_bytes<FMT>(), ip.slab * 16,
-                                bars + 8 * s);
-                }
-                load_side_w<FMT, NT>(sd[s], a.scales, a.zeros, a.N, a.Gtot, a.g0 + ip.grp(GP), ip.slab, g);
-                load_side_x<FMT, NT>(sd[s], a.xf, a.M, a.Gtot, a.g0 + ip.grp(GP), c);
+            if (issued < u1) {  // refill this slot with the units ST slots ahead
+                issue(s);
+#pragma unroll
+                for (int i = 0; i < UPS; ++i)
+                    load_side_x<FMT, NT>(sd[s][i], xside, a.M, a.Gtot, a.g0 + UPS * ip.grp(GP) + i, c);
                 ip.next(slabs, GP, G);
                 ++issued;
             }
@@ -794,8 +783,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
         if (rows_x > 0) mbar_wait(xbar, 0);
         // Let the copies still in flight land before the CTA's memory is released.
         for (unsigned v = u; v < issued; ++v) {
-            const int s = (int)((v - u0) % kStages);
-            const unsigned ph = ((v - u0) / kStages) & 1u;
+            const int s = (int)((v - u0) % ST);
+            const unsigned ph = ((v - u0) / ST) & 1u;
             if (!mbar_wait(bars + 8 * s, ph)) break;
         }
         return;
@@ -1085,11 +1074,11 @@ int swizzle_mode() {
                                  : (FMT == QL_I5Z_G128_F16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Groups of activations one CTA can stage next to its rings.
-template <int FMT>
-int max_staged_groups(int NT, size_t smem_optin) {
+// Groups of activations one CTA can stage for `rows` tokens next to its rings.
+template <int FMT, int UPS = 1>
+int max_staged_groups(int rows, size_t smem_optin) {
     for (int xg = 256; xg >= 1; --xg)
-        if (tma_smem<FMT>(NT, xg) <= smem_optin) return xg;
+        if (tma_smem<FMT, UPS>(rows, xg) <= smem_optin) return xg;
     return 0;
 }
 
@@ -1111,28 +1100,31 @@ int plan_parts(int G, int slabs, int ctas, int XG) {
     return 0;
 }
 
-template <int FMT, int NT, bool ACC>
+template <int FMT, int NT, bool ACC, int UPS = 1>
 cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& di) {
     SkinnyArgs a = in;
-    const int XG = max_staged_groups<FMT>(NT, di.smem_optin);
-    if (XG < 1) return cudaErrorInvalidValue;
+    if (a.G % UPS) return cudaErrorInvalidValue;
+    const int rows = a.M < NT * 8 ? a.M : NT * 8;  // token rows staged
+    const int XG = max_staged_groups<FMT, UPS>(rows, di.smem_optin);
+    if (XG < UPS) return cudaErrorInvalidValue;
     a.XG = XG;
-    a.GP = plan_parts(a.G, (a.N + 15) / 16, di.sm_count, XG);
+    // K parts in whole slots, so a slot never straddles two parts
+    a.GP = UPS * plan_parts(a.G / UPS, (a.N + 15) / 16, di.sm_count, XG / UPS);
     if (a.GP < 1) return cudaErrorInvalidValue;
     if ((long long)((a.N + 15) / 16) * a.G * (di.sm_count + 1) >= (1LL << 31)) return cudaErrorInvalidValue;
     a.err = di.err_word;
     cudaError_t e = make_tmap_2d(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw, unit_row_bytes<FMT>(), 16,
                                  swizzle_mode<FMT>(), &a.tmap);
     if (e != cudaSuccess) return e;
-    const size_t smem = tma_smem<FMT>(NT, XG);
+    const size_t smem = tma_smem<FMT, UPS>(rows, XG);
     static bool attr_set[64] = {};  // per device ordinal
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(k_skinny_tma<FMT, NT, ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(k_skinny_tma<FMT, NT, ACC, UPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)di.smem_optin);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(k_skinny_tma<FMT, NT, ACC>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(k_skinny_tma<FMT, NT, ACC, UPS>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_set[dev] = true;
@@ -1149,13 +1141,19 @@ cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& d
     attr[0].val.programmaticStreamSerializationAllowed = a.pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k_skinny_tma<FMT, NT, ACC>, a);
+    e = cudaLaunchKernelEx(&cfg, k_skinny_tma<FMT, NT, ACC, UPS>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <int FMT>
 cudaError_t run_skinny_fmt(const SkinnyArgs& a, cudaStream_t s, const DeviceInfo& di) {
+    if constexpr (FMT == QL_I4_G64_BF16 || FMT == QL_I5Z_G128_F16) {
+        // Two units per ring slot up to 8 tokens.  With 16 the doubled ring leaves room for
+        // fewer staged activation groups, K splits into more parts, and that costs more than
+        // the slots save.
+        if (a.G % 2 == 0 && a.M <= 8) return run_skinny<FMT, 1, false, 2>(a, s, di);
+    }
     if (a.M > 8) return run_skinny<FMT, 2, false>(a, s, di);
     return run_skinny<FMT, 1, false>(a, s, di);
 }
@@ -1168,10 +1166,10 @@ int skinny_max_k(int fmt) {
     int xg = 0;
     switch (fmt) {
     case QL_I8A8_G128_BF16:
-    case QL_FP8A8_B128_BF16: xg = max_staged_groups<QL_I8A8_G128_BF16>(2, di.smem_optin); break;
-    case QL_I4_G64_BF16: xg = max_staged_groups<QL_I4_G64_BF16>(2, di.smem_optin); break;
-    case QL_I5Z_G128_F16: xg = max_staged_groups<QL_I5Z_G128_F16>(2, di.smem_optin); break;
-    default: xg = max_staged_groups<QL_I8_G128_BF16>(2, di.smem_optin); break;
+    case QL_FP8A8_B128_BF16: xg = max_staged_groups<QL_I8A8_G128_BF16>(16, di.smem_optin); break;
+    case QL_I4_G64_BF16: xg = max_staged_groups<QL_I4_G64_BF16, 2>(16, di.smem_optin); break;
+    case QL_I5Z_G128_F16: xg = max_staged_groups<QL_I5Z_G128_F16, 2>(16, di.smem_optin); break;
+    default: xg = max_staged_groups<QL_I8_G128_BF16>(16, di.smem_optin); break;
     }
     return xg * 128;  // with G <= XG a single part always fits
 }
@@ -1196,8 +1194,8 @@ cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     if (a.acc) {
         if (fmt != QL_I8A8_G128_BF16) return cudaErrorInvalidValue;
-        if (a.M > 8) return run_skinny<QL_I8A8_G128_BF16, 2, true>(a, s, di);
-        return run_skinny<QL_I8A8_G128_BF16, 1, true>(a, s, di);
+        if (a.M > 8) return run_skinny<QL_I8A8_G128_BF16, 2, true, 1>(a, s, di);
+        return run_skinny<QL_I8A8_G128_BF16, 1, true, 1>(a, s, di);
     }
     switch (fmt) {
     case QL_I8_G128_BF16: return run_skinny_fmt<QL_I8_G128_BF16>(a, s, di);

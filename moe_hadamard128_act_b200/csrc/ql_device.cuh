@@ -109,6 +109,34 @@ __device__ __forceinline__ uint32_t quant_e4m3_group_warp(const float v[4], floa
 }
 __device__ __forceinline__ float f16_bits_to_float(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
+// int5 codes straight into f16 MMA operands.  A lane holds 32 codes of a row
+// as a 160-bit stream (code k at bits 5k .. 5k+4).  A 32-bit window of the
+// stream starting at bit B, masked to one code inside the low half's mantissa
+// (bits 0..9) and one inside the high half's, is an f16x2 pair of exact
+// subnormals u * 2^(o - 24), o the code's offset inside its half.  The table
+// lists the 16 pairs (window start, low code, high code): 4 windows are whole
+// words, 12 take one funnel shift, so 32 codes cost 28 integer instructions.
+// The activation of each code's MMA slot is staged pre-divided by 2^o, so every
+// product is u * x * 2^-24; the zero point is taken off once per group with the
+// token's sum of that group's activations.  Register r holds the codes of MMA
+// slots (2c, 2c+1) of MMA r / 2 when r is even, (2c+8, 2c+9) when odd.
+struct I5Pair {
+    int B, klo, khi;
+};
+constexpr I5Pair kI5Pairs[16] = {{0, 0, 4},    {4, 1, 5},    {10, 2, 6},   {14, 3, 7},   {37, 8, 11},  {43, 9, 12},
+                                 {49, 10, 14}, {64, 13, 17}, {72, 15, 18}, {76, 16, 19}, {96, 20, 23}, {100, 21, 24},
+                                 {109, 22, 25}, {128, 26, 29}, {130, 27, 30}, {137, 28, 31}};
+__host__ __device__ constexpr int i5_off_lo(int r) { return 5 * kI5Pairs[r].klo - kI5Pairs[r].B; }
+__host__ __device__ constexpr int i5_off_hi(int r) { return 5 * kI5Pairs[r].khi - kI5Pairs[r].B - 16; }
+// Slot s (0..31) of a lane's 32 activation values: MMA s / 4, register 2 (s / 4) + ((s / 2) & 1),
+// its low half when s is even.  Returns the code index (0..31) it multiplies and its offset o.
+__host__ __device__ constexpr int i5_slot_code(int s) {
+    return (s & 1) ? kI5Pairs[2 * (s >> 2) + ((s >> 1) & 1)].khi : kI5Pairs[2 * (s >> 2) + ((s >> 1) & 1)].klo;
+}
+__host__ __device__ constexpr int i5_slot_off(int s) {
+    return (s & 1) ? i5_off_hi(2 * (s >> 2) + ((s >> 1) & 1)) : i5_off_lo(2 * (s >> 2) + ((s >> 1) & 1));
+}
+
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
     __half2 r = __hadd2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
     return *reinterpret_cast<uint32_t*>(&r);

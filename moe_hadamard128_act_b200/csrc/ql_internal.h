@@ -61,8 +61,10 @@ cudaError_t launch_act_quant(const void* x, int M, int K, int rotate, int8_t* q,
 cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8_t* q, float* sx, float* sxT, int Mp,
                                   float* yz, long long nz, cudaStream_t s, const int32_t* inv = nullptr,
                                   int topk = 0);
+// XORD_I5 also writes xsum [M][K/128] (each group's sum of the f16 activations, for the zero
+// point) and puts 2^24 into xf (the int5 codes enter the MMAs as exact subnormals u * 2^-24).
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
-                            long long nz, cudaStream_t s);
+                            long long nz, cudaStream_t s, float* xsum = nullptr);
 // The same for the grouped expert GEMM: token t's f16 row goes to rows
 // inv[t * topk + j] of xs (j < topk, rows < 0 skipped); xf stays per token.
 cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, const int32_t* inv, int topk, __half* xs,
@@ -83,6 +85,7 @@ struct SkinnyArgs {
     const uint8_t* zeros;  // int5: [N][Gtot]
     const void* xs;        // prepared activations, row stride ldx elements; offset to group g0
     const float* xf;       // A16: [M] inverse token factors; W8A8: sx [M][Gtot]
+    const float* xsum = nullptr;  // int5: each token's sums of its f16 activations per group [M][Gtot]
     float* y;              // [M][ldy]
     int32_t* acc;          // optional W8A8 group sums [M][N][Gtot]
     unsigned* err;         // device error word (filled by launch_skinny)
