@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--extras", default=None,
+                   help="comma-separated extras sections to run (decode, moe_decode, moe_prefill, moe_fp8a8_down, "
+                        "prefill); default all")
     p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "prefill_w5a8",
                                           "moe_decode", "moe_decode_t1", "moe_prefill", "act_quant", "decode_w4a16",
                                           "decode_w5a16", "decode_w8a16", "decode_fp8"],
@@ -266,182 +269,205 @@ def _traced(Q, fn, iters, kind):
     return float(np.mean(ks)) if ks else None, len(tr) / iters
 
 
-def run_extras(torch, Q, synth, dev, stream, hbm):
+def _mark(torch, section, stream):
+    """Synchronise after a section of the extras and say so on stderr, so that a device fault
+    is reported against the section that raised it."""
+    stream.synchronize()
+    torch.cuda.synchronize()
+    print(f"[bench] section done: {section}", file=sys.stderr, flush=True)
+
+
+def run_extras(torch, Q, synth, dev, stream, hbm, sections=None):
+    """The secondary workloads; `sections` (a set of names, None = all) limits which run:
+    decode, moe_decode, moe_prefill, moe_fp8a8_down, prefill."""
+    want = lambda name: sections is None or name in sections  # noqa: E731
     out = {}
     G = K_FULL // 128
     bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     with torch.cuda.stream(stream):
-        # weight-only decode: int4 g64, int5 + zero point g128, int8 g128 bf16, fp8 128x128; and
-        # format 7 (the fp8 weight with E4M3 activations) on the same decode kernel.
-        # "us" is the whole forward (activation prologue + decode GEMM) replayed from a
-        # CUDA graph, the rate it gives is over the forward's bytes; "us_gemm" is the
-        # traced decode kernel alone.
-        Wd = None
-        for name, fmt in (("w4a16_decode", Q.I4_G64_BF16), ("w5a16_decode", Q.I5Z_G128_F16),
-                          ("w8a16_decode", Q.I8_G128_BF16), ("fp8_decode", Q.FP8_B128_BF16),
-                          ("fp8a8_decode", Q.FP8A8_B128_BF16)):
-            if fmt in (Q.I4_G64_BF16, Q.I5Z_G128_F16):
-                d = synth.w4a16(16) if fmt == Q.I4_G64_BF16 else synth.w5a16(16)
-                z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None
-                c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
-                                          scales=torch.from_numpy(d["scales"].view(np.int16)).to(dev), zeros=z)
-            else:
-                if Wd is None:
-                    Wd = torch.from_numpy(synth.weight_rows(0, "W", K_FULL, 0, N_FULL)).to(dev)
-                c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=Wd)
-            cp = [(c, s, zz)] + [(c.clone(), s.clone(), None if zz is None else zz.clone()) for _ in range(3)]
+        if want("decode"):
+            # weight-only decode: int4 g64, int5 + zero point g128, int8 g128 bf16, fp8 128x128; and
+            # format 7 (the fp8 weight with E4M3 activations) on the same decode kernel.
+            # "us" is the whole forward (activation prologue + decode GEMM) replayed from a
+            # CUDA graph, the rate it gives is over the forward's bytes; "us_gemm" is the
+            # traced decode kernel alone.
+            Wd = None
+            for name, fmt in (("w4a16_decode", Q.I4_G64_BF16), ("w5a16_decode", Q.I5Z_G128_F16),
+                              ("w8a16_decode", Q.I8_G128_BF16), ("fp8_decode", Q.FP8_B128_BF16),
+                              ("fp8a8_decode", Q.FP8A8_B128_BF16)):
+                if fmt in (Q.I4_G64_BF16, Q.I5Z_G128_F16):
+                    d = synth.w4a16(16) if fmt == Q.I4_G64_BF16 else synth.w5a16(16)
+                    z = torch.from_numpy(d["zeros"]).to(dev) if "zeros" in d else None
+                    c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, codes=torch.from_numpy(d["codes"]).to(dev),
+                                              scales=torch.from_numpy(d["scales"].view(np.int16)).to(dev), zeros=z)
+                else:
+                    if Wd is None:
+                        Wd = torch.from_numpy(synth.weight_rows(0, "W", K_FULL, 0, N_FULL)).to(dev)
+                    c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=Wd)
+                cp = [(c, s, zz)] + [(c.clone(), s.clone(), None if zz is None else zz.clone()) for _ in range(3)]
+                res = {}
+                for m in (1, 5, 16) if fmt == Q.I4_G64_BF16 else (1, 4, 16):
+                    x = bf(synth.activations(0, f"x_M{m}", m, K_FULL))
+                    y = torch.empty((m, N_FULL), dtype=torch.float32, device=dev)
+                    ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, m, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
+                    run = lambda i: Q.qlinear_forward(x, cp[i % 4][0], cp[i % 4][1], cp[i % 4][2], fmt, N_FULL,  # noqa
+                                                      y=y, ws=ws, stream=stream)
+                    for i in range(8):
+                        run(i)
+                    t, per = _traced(Q, run, 40, "skinny")
+                    us = _graph_call_us(torch, run, stream)
+                    cb, sb, zb = Q.qlinear_packed_sizes(fmt, N_FULL, K_FULL)
+                    byts = cb + sb + zb + m * K_FULL * 2 + m * N_FULL * 4
+                    res[str(m)] = {"us": us, "GB/s": byts / (us * 1e-6) / 1e9, "frac": byts / (us * 1e-6) / 1e9 / hbm,
+                                   "us_gemm": 1e3 * t, "launches_per_call": per}
+                out[name] = res
+                del cp, c, s, zz
+            del Wd
+            _mark(torch, "decode", stream)
+        if want("moe_decode") or want("moe_prefill"):
+            # MoE gate_up, int8 Hadamard-domain experts, decode batches
+            E, topk, Ke, Ne = 128, 8, 2816, 1408
+            Ws = synth.moe_gate_up(1, experts=range(E))["W"]
+            codes = torch.empty((E, Ne, Ke), dtype=torch.int8, device=dev)
+            scales = torch.empty((E, Ne, Ke // 128), dtype=torch.int16, device=dev)
+            for e in range(E):
+                c, s, _ = Q.qlinear_pack(Q.I8_G128_BF16, Ne, Ke, W=torch.from_numpy(Ws[e]).to(dev), flags=Q.HADAMARD)
+                codes[e] = c.view(torch.int8).reshape(Ne, Ke)
+                scales[e] = s.view(torch.int16).reshape(Ne, Ke // 128)
+            del Ws
+        if want("moe_decode"):
             res = {}
-            for m in (1, 5, 16) if fmt == Q.I4_G64_BF16 else (1, 4, 16):
-                x = bf(synth.activations(0, f"x_M{m}", m, K_FULL))
-                y = torch.empty((m, N_FULL), dtype=torch.float32, device=dev)
-                ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, m, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
-                run = lambda i: Q.qlinear_forward(x, cp[i % 4][0], cp[i % 4][1], cp[i % 4][2], fmt, N_FULL,  # noqa
-                                                  y=y, ws=ws, stream=stream)
+            for T in (1, 8, 16):
+                batches = []
+                for b in range(8):
+                    ids, w = synth.routing(100 + b, T, E, topk)
+                    batches.append((bf(synth.activations(b, f"x_T{T}", T, Ke)), torch.from_numpy(ids).to(dev),
+                                    len(set(ids.ravel().tolist()))))
+                y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+                wsm = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.I8_G128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
+                                  device=dev)
+                run = lambda i: Q.moe_gate_up(batches[i % 8][0], batches[i % 8][1], codes, scales, E, Ne, y=y,  # noqa
+                                              ws=wsm, stream=stream)
                 for i in range(8):
                     run(i)
-                t, per = _traced(Q, run, 40, "skinny")
-                us = _graph_call_us(torch, run, stream)
-                cb, sb, zb = Q.qlinear_packed_sizes(fmt, N_FULL, K_FULL)
-                byts = cb + sb + zb + m * K_FULL * 2 + m * N_FULL * 4
-                res[str(m)] = {"us": us, "GB/s": byts / (us * 1e-6) / 1e9, "frac": byts / (us * 1e-6) / 1e9 / hbm,
-                               "us_gemm": 1e3 * t, "launches_per_call": per}
-            out[name] = res
-            del cp, c, s, zz
-        del Wd
-        # MoE gate_up, int8 Hadamard-domain experts, decode batches
-        E, topk, Ke, Ne = 128, 8, 2816, 1408
-        Ws = synth.moe_gate_up(1, experts=range(E))["W"]
-        codes = torch.empty((E, Ne, Ke), dtype=torch.int8, device=dev)
-        scales = torch.empty((E, Ne, Ke // 128), dtype=torch.int16, device=dev)
-        for e in range(E):
-            c, s, _ = Q.qlinear_pack(Q.I8_G128_BF16, Ne, Ke, W=torch.from_numpy(Ws[e]).to(dev), flags=Q.HADAMARD)
-            codes[e] = c.view(torch.int8).reshape(Ne, Ke)
-            scales[e] = s.view(torch.int16).reshape(Ne, Ke // 128)
-        del Ws
-        res = {}
-        for T in (1, 8, 16):
-            batches = []
-            for b in range(8):
-                ids, w = synth.routing(100 + b, T, E, topk)
-                batches.append((bf(synth.activations(b, f"x_T{T}", T, Ke)), torch.from_numpy(ids).to(dev),
-                                len(set(ids.ravel().tolist()))))
-            y = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
-            wsm = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.I8_G128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
+                t, per = _traced(Q, run, 40, "moe_gemm")
+                us_call = _graph_call_us(torch, run, stream)
+                touched = float(np.mean([b[2] for b in batches]))
+                byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
+                res[str(T)] = {"us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
+                               "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per,
+                               "us_call_graph": us_call, "GB/s_call": byts / (us_call * 1e-6) / 1e9}
+            out["moe_gate_up_decode"] = res
+            _mark(torch, "moe_decode", stream)
+        if want("moe_prefill"):
+            # the same experts at prefill size, T = 2048 (every expert touched)
+            T = 2048
+            ids, _ = synth.routing(200, T, E, topk)
+            xT = bf(synth.activations(0, "x_T2048", T, Ke))
+            idsT = torch.from_numpy(ids).to(dev)
+            yT = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
+            wsT = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.I8_G128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
                               device=dev)
-            run = lambda i: Q.moe_gate_up(batches[i % 8][0], batches[i % 8][1], codes, scales, E, Ne, y=y,  # noqa
-                                          ws=wsm, stream=stream)
-            for i in range(8):
+            run = lambda i: Q.moe_gate_up(xT, idsT, codes, scales, E, Ne, y=yT, ws=wsT, stream=stream)  # noqa: E731
+            for i in range(2):
                 run(i)
-            t, per = _traced(Q, run, 40, "moe_gemm")
-            us_call = _graph_call_us(torch, run, stream)
-            touched = float(np.mean([b[2] for b in batches]))
+            t, per = _traced(Q, run, 5, "moe_gemm")
+            us_call = _graph_call_us(torch, run, stream, calls=8, reps=3)
+            touched = len(set(ids.ravel().tolist()))
             byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
-            res[str(T)] = {"us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
-                           "frac": byts / (t * 1e-3) / 1e9 / hbm, "launches_per_call": per,
-                           "us_call_graph": us_call, "GB/s_call": byts / (us_call * 1e-6) / 1e9}
-        out["moe_gate_up_decode"] = res
-        # the same experts at prefill size, T = 2048 (every expert touched)
-        T = 2048
-        ids, _ = synth.routing(200, T, E, topk)
-        xT = bf(synth.activations(0, "x_T2048", T, Ke))
-        idsT = torch.from_numpy(ids).to(dev)
-        yT = torch.empty((T, topk, Ne), dtype=torch.float32, device=dev)
-        wsT = torch.empty(Q.moe_workspace_size(E, Ne, Ke, Q.I8_G128_BF16, Q.HADAMARD, T, topk), dtype=torch.uint8,
-                          device=dev)
-        run = lambda i: Q.moe_gate_up(xT, idsT, codes, scales, E, Ne, y=yT, ws=wsT, stream=stream)  # noqa: E731
-        for i in range(2):
-            run(i)
-        t, per = _traced(Q, run, 5, "moe_gemm")
-        us_call = _graph_call_us(torch, run, stream, calls=8, reps=3)
-        touched = len(set(ids.ravel().tolist()))
-        byts = touched * (Ne * Ke + Ne * (Ke // 128) * 2) + T * Ke * 2 + T * topk * Ne * 4
-        flops = 2.0 * T * topk * Ne * Ke
-        bf16_peak = peaks()[1]
-        t_roof = max(byts / (hbm * 1e9), flops / (bf16_peak * 1e12))
-        out["moe_gate_up_prefill"] = {"T": T, "us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
-                                      "TFLOPS": flops / (t * 1e-3) / 1e12, "roofline_us": 1e6 * t_roof,
-                                      "frac": 1e6 * t_roof / (1e3 * t), "launches_per_call": per,
-                                      "us_call_graph": us_call,
-                                      "roofline": "max(bytes / measured HBM, flops / measured bf16 peak)"}
-        del codes, scales, xT, idsT, yT
-        out.update(moe_extras(torch, Q, synth, dev, stream, hbm))
-        # prefill W8A8 at M = 2048 (tcgen05 kind::i8 GEMM with per-group fp32 promotion)
-        M = 2048
-        d = synth.prefill(M=M)
-        c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
-        x = bf(d["x"])
-        y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
-        ws = torch.empty(Q.qlinear_workspace_size(Q.I8A8_G128_BF16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
-                         device=dev)
-        run = lambda i: Q.qlinear_forward(x, c, s, None, Q.I8A8_G128_BF16, N_FULL, y=y, ws=ws,  # noqa: E731
-                                          stream=stream)
-        for i in range(3):
-            run(i)
-        t, _ = _traced(Q, run, 10, "prefill")
-        tq, _ = _traced(Q, run, 10, "act_quant")
-        tp, _ = _traced(Q, run, 10, "prefill_prep")
-        ops = 2.0 * M * N_FULL * K_FULL
-        peak_i8 = 2.0 * peaks()[1]  # measured bf16 dense burst x the nominal int8 / bf16 ratio of 2
-        out["prefill_w8a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq, "us_scale_prep": 1e3 * tp, "TOPS": ops / (t * 1e-3) / 1e12,
-                               "peak_TOPS": peak_i8, "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
-                               "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
-        del c, s, y, ws
-        # prefill with 16-bit activations: fp8 128x128 and int8 g128 bf16 weights (tcgen05 kind::f16)
-        for name, fmt in (("prefill_fp8", Q.FP8_B128_BF16), ("prefill_w8a16", Q.I8_G128_BF16)):
-            c, s, _ = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+            flops = 2.0 * T * topk * Ne * Ke
+            bf16_peak = peaks()[1]
+            t_roof = max(byts / (hbm * 1e9), flops / (bf16_peak * 1e12))
+            out["moe_gate_up_prefill"] = {"T": T, "us_gemm": 1e3 * t, "touched_experts": touched, "GB/s": byts / (t * 1e-3) / 1e9,
+                                          "TFLOPS": flops / (t * 1e-3) / 1e12, "roofline_us": 1e6 * t_roof,
+                                          "frac": 1e6 * t_roof / (1e3 * t), "launches_per_call": per,
+                                          "us_call_graph": us_call,
+                                          "roofline": "max(bytes / measured HBM, flops / measured bf16 peak)"}
+            _mark(torch, "moe_prefill", stream)
+        if want("moe_decode") or want("moe_prefill"):
+            del codes, scales
+        if want("moe_fp8a8_down"):
+            out.update(moe_extras(torch, Q, synth, dev, stream, hbm))
+            _mark(torch, "moe_fp8a8_down", stream)
+        if want("prefill"):
+            # prefill W8A8 at M = 2048 (tcgen05 kind::i8 GEMM with per-group fp32 promotion)
+            M = 2048
+            d = synth.prefill(M=M)
+            c, s, _ = Q.qlinear_pack(Q.I8A8_G128_BF16, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+            x = bf(d["x"])
             y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
-            ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, M, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
-            run = lambda i: Q.qlinear_forward(x, c, s, None, fmt, N_FULL, y=y, ws=ws, stream=stream)  # noqa: E731
+            ws = torch.empty(Q.qlinear_workspace_size(Q.I8A8_G128_BF16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
+                             device=dev)
+            run = lambda i: Q.qlinear_forward(x, c, s, None, Q.I8A8_G128_BF16, N_FULL, y=y, ws=ws,  # noqa: E731
+                                              stream=stream)
             for i in range(3):
                 run(i)
             t, _ = _traced(Q, run, 10, "prefill")
-            tq, _ = _traced(Q, run, 10, "prep_a16")
-            tf = ops / (t * 1e-3) / 1e12
-            out[name] = {"M": M, "us_gemm": 1e3 * t, "us_prep_a16": 1e3 * tq, "TFLOPS": tf,
-                         "frac_of_fp8_peak": tf / peak_i8, "frac_of_bf16_peak": tf / peaks()[1],
-                         "peak_source": "MEASURED_PEAKS.json bf16_tflops (x 2 for fp8, nominal ratio)",
-                         "mma": "kind::f16 (exact f16 codes x token-scaled f16 activations)"}
+            tq, _ = _traced(Q, run, 10, "act_quant")
+            tp, _ = _traced(Q, run, 10, "prefill_prep")
+            ops = 2.0 * M * N_FULL * K_FULL
+            peak_i8 = 2.0 * peaks()[1]  # measured bf16 dense burst x the nominal int8 / bf16 ratio of 2
+            out["prefill_w8a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq, "us_scale_prep": 1e3 * tp, "TOPS": ops / (t * 1e-3) / 1e12,
+                                   "peak_TOPS": peak_i8, "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
+                                   "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
             del c, s, y, ws
-        # format 7: the fp8 weights with E4M3 activations (tcgen05 kind::f8f6f4, fp8 rate)
-        c, s, _ = Q.qlinear_pack(Q.FP8A8_B128_BF16, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
-        y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
-        ws = torch.empty(Q.qlinear_workspace_size(Q.FP8A8_B128_BF16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
-                         device=dev)
-        run = lambda i: Q.qlinear_forward(x, c, s, None, Q.FP8A8_B128_BF16, N_FULL, y=y, ws=ws,  # noqa: E731
-                                          stream=stream)
-        for i in range(3):
-            run(i)
-        t, _ = _traced(Q, run, 10, "prefill")
-        tq, _ = _traced(Q, run, 10, "act_quant")
-        tp, _ = _traced(Q, run, 10, "prefill_prep")
-        tf = ops / (t * 1e-3) / 1e12
-        out["prefill_fp8a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq, "us_scale_prep": 1e3 * tp,
-                                "TFLOPS": tf, "frac_of_fp8_peak": tf / peak_i8,
-                                "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal fp8/bf16 ratio)",
-                                "mma": "kind::f8f6f4 (E4M3 x E4M3, fp32 group sums)"}
-        del c, s, y, ws
-        # int5 with a zero point from 65 rows on (W5A8): int8 activations, the codes converted to
-        # int8 q - z in the workspace, the W8A8 tensor-core GEMM
-        d5 = synth.w5a16(M)
-        c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N_FULL, K_FULL, codes=torch.from_numpy(d5["codes"]).to(dev),
-                                 scales=torch.from_numpy(d5["scales"]).to(dev),
-                                 zeros=torch.from_numpy(d5["zeros"]).to(dev))
-        x5 = bf(d5["x"])
-        y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
-        ws = torch.empty(Q.qlinear_workspace_size(Q.I5Z_G128_F16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
-                         device=dev)
-        run = lambda i: Q.qlinear_forward(x5, c, s, z, Q.I5Z_G128_F16, N_FULL, y=y, ws=ws,  # noqa: E731
-                                          stream=stream)
-        for i in range(3):
-            run(i)
-        t, _ = _traced(Q, run, 10, "prefill")
-        tq, _ = _traced(Q, run, 10, "act_quant")
-        tp, _ = _traced(Q, run, 10, "prefill_prep")
-        out["prefill_w5a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq,
-                               "us_scale_prep_and_code_conversion": 1e3 * tp, "TOPS": ops / (t * 1e-3) / 1e12,
-                               "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
-                               "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
-        del c, s, z, y, ws, d5
+            # prefill with 16-bit activations: fp8 128x128 and int8 g128 bf16 weights (tcgen05 kind::f16)
+            for name, fmt in (("prefill_fp8", Q.FP8_B128_BF16), ("prefill_w8a16", Q.I8_G128_BF16)):
+                c, s, _ = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+                y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+                ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, M, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
+                run = lambda i: Q.qlinear_forward(x, c, s, None, fmt, N_FULL, y=y, ws=ws, stream=stream)  # noqa: E731
+                for i in range(3):
+                    run(i)
+                t, _ = _traced(Q, run, 10, "prefill")
+                tq, _ = _traced(Q, run, 10, "prep_a16")
+                tf = ops / (t * 1e-3) / 1e12
+                out[name] = {"M": M, "us_gemm": 1e3 * t, "us_prep_a16": 1e3 * tq, "TFLOPS": tf,
+                             "frac_of_fp8_peak": tf / peak_i8, "frac_of_bf16_peak": tf / peaks()[1],
+                             "peak_source": "MEASURED_PEAKS.json bf16_tflops (x 2 for fp8, nominal ratio)",
+                             "mma": "kind::f16 (exact f16 codes x token-scaled f16 activations)"}
+                del c, s, y, ws
+            # format 7: the fp8 weights with E4M3 activations (tcgen05 kind::f8f6f4, fp8 rate)
+            c, s, _ = Q.qlinear_pack(Q.FP8A8_B128_BF16, N_FULL, K_FULL, W=torch.from_numpy(d["W"]).to(dev))
+            y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+            ws = torch.empty(Q.qlinear_workspace_size(Q.FP8A8_B128_BF16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
+                             device=dev)
+            run = lambda i: Q.qlinear_forward(x, c, s, None, Q.FP8A8_B128_BF16, N_FULL, y=y, ws=ws,  # noqa: E731
+                                              stream=stream)
+            for i in range(3):
+                run(i)
+            t, _ = _traced(Q, run, 10, "prefill")
+            tq, _ = _traced(Q, run, 10, "act_quant")
+            tp, _ = _traced(Q, run, 10, "prefill_prep")
+            tf = ops / (t * 1e-3) / 1e12
+            out["prefill_fp8a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq, "us_scale_prep": 1e3 * tp,
+                                    "TFLOPS": tf, "frac_of_fp8_peak": tf / peak_i8,
+                                    "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal fp8/bf16 ratio)",
+                                    "mma": "kind::f8f6f4 (E4M3 x E4M3, fp32 group sums)"}
+            del c, s, y, ws
+            # int5 with a zero point from 65 rows on (W5A8): int8 activations, the codes converted to
+            # int8 q - z in the workspace, the W8A8 tensor-core GEMM
+            d5 = synth.w5a16(M)
+            c, s, z = Q.qlinear_pack(Q.I5Z_G128_F16, N_FULL, K_FULL, codes=torch.from_numpy(d5["codes"]).to(dev),
+                                     scales=torch.from_numpy(d5["scales"]).to(dev),
+                                     zeros=torch.from_numpy(d5["zeros"]).to(dev))
+            x5 = bf(d5["x"])
+            y = torch.empty((M, N_FULL), dtype=torch.float32, device=dev)
+            ws = torch.empty(Q.qlinear_workspace_size(Q.I5Z_G128_F16, 0, M, N_FULL, K_FULL), dtype=torch.uint8,
+                             device=dev)
+            run = lambda i: Q.qlinear_forward(x5, c, s, z, Q.I5Z_G128_F16, N_FULL, y=y, ws=ws,  # noqa: E731
+                                              stream=stream)
+            for i in range(3):
+                run(i)
+            t, _ = _traced(Q, run, 10, "prefill")
+            tq, _ = _traced(Q, run, 10, "act_quant")
+            tp, _ = _traced(Q, run, 10, "prefill_prep")
+            out["prefill_w5a8"] = {"M": M, "us_gemm": 1e3 * t, "us_act_quant": 1e3 * tq,
+                                   "us_scale_prep_and_code_conversion": 1e3 * tp, "TOPS": ops / (t * 1e-3) / 1e12,
+                                   "frac": ops / (t * 1e-3) / 1e12 / peak_i8,
+                                   "peak_source": "MEASURED_PEAKS.json bf16_tflops x 2 (nominal int8/bf16 ratio)"}
+            del c, s, z, y, ws, d5
+            _mark(torch, "prefill", stream)
     torch.cuda.synchronize()
     return out
 
@@ -888,13 +914,16 @@ def main():
         del copies, codes0, scales0
         torch.cuda.empty_cache()
         try:
-            extras = run_extras(torch, Q, synth, dev, stream, hbm)
+            sections = None if args.extras is None else set(args.extras.split(","))
+            extras = run_extras(torch, Q, synth, dev, stream, hbm, sections)
         except Exception as ex:  # report, keep the headline line
             extras = {"error": f"{type(ex).__name__}: {ex}"}
+            print(f"[bench] extras failed: {extras['error']}", file=sys.stderr, flush=True)
 
     st, bits = Q.ql_get_device_error(stream)
     if st != 0:
-        raise RuntimeError(f"device error word set: {bits}")
+        raise RuntimeError(f"ql_get_device_error: status {st} ({Q.STATUS.get(st, st)}), bits {bits}, "
+                           f"last CUDA error: {Q.lib().ql_last_cuda_error().decode()}")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -59,29 +59,38 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y
     const int lane = threadIdx.x & 31;
-    const long long G = K / 128;
-    const long long nw = (long long)gridDim.x * kWarpsPerBlock;
-    for (long long u = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); u < (long long)M * G; u += nw) {
-        const long long off = (u / G) * K + (u % G) * 128 + 4 * lane;
+    const int G = K / 128;
+    // This warp's (token, group) units u = t * G + g, grid-strided by nw; the position is
+    // stepped by (nw / G, nw % G) with a carry instead of divided out every time.
+    const int nw = gridDim.x * kWarpsPerBlock, dt = nw / G, dg = nw % G;
+    const int u0 = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    int t = u0 / G, g = u0 % G;
+    for (; t < M; t += dt, g += dg) {
+        if (g >= G) {
+            g -= G;
+            ++t;
+            if (t >= M) break;
+        }
+        const long long u = (long long)t * G + g;
+        const long long off = (long long)t * K + g * 128 + 4 * lane;
         float v[4];
         load4_bf16(x + off, v);
         if (rotate) fwht128_warp(v, lane);
         float s;
         const uint32_t packed = E4M3 ? quant_e4m3_group_warp(v, &s) : quant_i8_group_warp(v, &s);
         if (inv) {
-            const long long t = u / G, g = u % G;
             for (int j = 0; j < topk; ++j) {
                 const int r = __ldg(inv + t * topk + j);
                 if (r < 0) continue;
                 *reinterpret_cast<uint32_t*>(q + (long long)r * K + g * 128 + 4 * lane) = packed;
-                if (lane == 0) sxT[g * Mp + r] = s;
+                if (lane == 0) sxT[(long long)g * Mp + r] = s;
             }
             continue;
         }
         *reinterpret_cast<uint32_t*>(q + off) = packed;
         if (lane == 0) {
             if (sx) sx[u] = s;                                 // [M][G] row-major: u = m * G + g
-            if (sxT) sxT[(u % G) * Mp + u / G] = s;            // [G][Mp], the prefill GEMM's layout
+            if (sxT) sxT[(long long)g * Mp + t] = s;           // [G][Mp], the prefill GEMM's layout
         }
     }
 }

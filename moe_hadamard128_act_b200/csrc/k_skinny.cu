@@ -141,10 +141,10 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
                     // masked in place, becomes 1024 + 16 u and one exact FMA (x / 16 - 72) leaves q.
                     const uint32_t w0 = (p == 0 ? r.w[0][h].x : r.w[0][h].y) >> (8 * sub);
                     const uint32_t w1 = (p == 0 ? r.w[1][h].x : r.w[1][h].y) >> (8 * sub);
-                    const uint32_t a0 = hadd2_u32((w0 & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
-                    const uint32_t a2 = hfma2_u32((w0 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
-                    const uint32_t a1 = hadd2_u32((w1 & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
-                    const uint32_t a3 = hfma2_u32((w1 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
+                    const uint32_t a0 = hadd2_u32(and_or(w0, 0x000F000Fu, 0x64006400u), 0xE408E408u);
+                    const uint32_t a2 = hfma2_u32(and_or(w0, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+                    const uint32_t a1 = hadd2_u32(and_or(w1, 0x000F000Fu, 0x64006400u), 0xE408E408u);
+                    const uint32_t a3 = hfma2_u32(and_or(w1, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
                         if (nt == 1 && !nt1_live) continue;
@@ -641,6 +641,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
         ngs = min(G, (p1.part + 1) * GP) * UPS - gs0;
     }
     const int rows_x = ngs > 0 ? min(a.M, NT * 8) : 0;
+    // Lanes whose token row does not exist read a row of zeros staged after the real ones, so
+    // the fragment loads need no test.
+    uint32_t xrow_off[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) xrow_off[nt] = (uint32_t)((8 * nt + g < rows_x ? 8 * nt + g : rows_x) * R);
+    if (rows_x < NT * 8) {
+        const int pieces = ngs * XGB / 16;
+        for (int i = threadIdx.x; i < pieces; i += kThreads)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(xs_base + (uint32_t)(rows_x * R + 16 * i)),
+                         "r"(0u)
+                         : "memory");
+    }
     if (threadIdx.x == 0) {
         mbar_init(xbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -719,7 +731,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 const int grp = UPS * cp.grp(GP) + ui;
                 const int lg = grp - gs0;  // group index in the staged activations
                 auto getx = [&](int nt, int p) -> uint4 {
-                    if (8 * nt + g >= rows_x) return make_uint4(0, 0, 0, 0);  // no such token
                     int j;
                     if constexpr (act8<FMT>())
                         j = lg * 8 + 4 * p + c;
@@ -730,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                         j ^= (j >> 3) & 1;
                     } else
                         j = lg * 16 + (p >> 1) * 8 + 2 * c + (p & 1);
-                    return lds128(xs_base + (uint32_t)((8 * nt + g) * R + 16 * j));
+                    return lds128(xs_base + xrow_off[nt] + (uint32_t)(16 * j));
                 };
                 if constexpr (FMT == QL_I8A8_G128_BF16) {
                     int acc[NT][4];
@@ -1104,7 +1115,8 @@ template <int FMT, int NT, bool ACC, int UPS = 1>
 cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& di) {
     SkinnyArgs a = in;
     if (a.G % UPS) return cudaErrorInvalidValue;
-    const int rows = a.M < NT * 8 ? a.M : NT * 8;  // token rows staged
+    // token rows staged, plus one row of zeros for the lanes of absent tokens
+    const int rows = a.M < NT * 8 ? a.M + 1 : NT * 8;
     const int XG = max_staged_groups<FMT, UPS>(rows, di.smem_optin);
     if (XG < UPS) return cudaErrorInvalidValue;
     a.XG = XG;

@@ -821,13 +821,15 @@ const char* ql_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 
 int ql_get_device_error(void* stream, unsigned* bits) {
     DeviceInfo di;
-    if (device_info(&di) != cudaSuccess) return QL_ECUDA;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QL_ECUDA;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return from_cuda(e);
+    if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) return from_cuda(e);
     unsigned v = 0;
-    if (cudaMemcpy(&v, di.err_word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return QL_ECUDA;
+    if ((e = cudaMemcpy(&v, di.err_word, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess) return from_cuda(e);
     if (v) {
         const unsigned zero = 0;
-        if (cudaMemcpy(di.err_word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return QL_ECUDA;
+        if ((e = cudaMemcpy(di.err_word, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
+            return from_cuda(e);
     }
     if (bits) *bits = v;
     return v ? QL_EDEVICE : QL_OK;

@@ -30,11 +30,13 @@ __device__ __forceinline__ void fwht128_warp(float v[4], int lane) {
     a = v[1]; b = v[3]; v[1] = __fadd_rn(a, b); v[3] = __fsub_rn(a, b);
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
-        const bool upper = (lane & m) != 0;
+        // lower lane: v + o; upper lane: o - v.  Both are o + sgn * v with sgn = +-1, one
+        // FMA whose product is exact, so the single rounding is that of the add or subtract.
+        const float sgn = (lane & m) ? -1.0f : 1.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float o = __shfl_xor_sync(kFull, v[i], m);
-            v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+            v[i] = __fmaf_rn(sgn, v[i], o);
         }
     }
     const float c = fwht_scale();
@@ -135,6 +137,13 @@ __host__ __device__ constexpr int i5_slot_code(int s) {
 }
 __host__ __device__ constexpr int i5_slot_off(int s) {
     return (s & 1) ? i5_off_hi(2 * (s >> 2) + ((s >> 1) & 1)) : i5_off_lo(2 * (s >> 2) + ((s >> 1) & 1));
+}
+
+// (a & b) | c in one LOP3 (truth table 0xEA).
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
