@@ -330,6 +330,16 @@ int ql_trace_read(int* kinds, float* ms, int max, int* count);
  * this host thread ("no error" if there was none).  Never NULL. */
 const char* ql_last_cuda_error(void);
 
+/* Bound every wait of the library's kernels for a copy, an MMA or another
+ * warp's work to `ns` nanoseconds on the current device (0 restores the
+ * default, 200 ms).  A wait that runs out sets QL_DEVERR_TIMEOUT, and its
+ * kernel stops early, letting the copies and MMAs it already started finish
+ * (those waits keep the default bound) and freeing its tensor memory; the
+ * call's output is then incomplete.  For testing that path: a limit of 1 makes
+ * nearly every pipeline wait run out.  Synchronises the device; host state
+ * only per device, not per stream. */
+int ql_set_wait_limit(unsigned long long ns);
+
 /* Synchronise `stream`, then read and clear the device error word.
  * Returns QL_OK when it was clear, QL_EDEVICE otherwise (with *bits, if not
  * NULL, set to its QL_DEVERR_* bits), QL_ECUDA if a CUDA call failed. */

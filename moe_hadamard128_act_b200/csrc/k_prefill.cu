@@ -277,6 +277,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool dead = false;
+    // Pipeline waits are bounded by lim; the waits that let started copies and MMAs
+    // finish before the CTA ends keep the default bound.
+    const unsigned long long lim = wait_limit(a.err);
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsDriver));
@@ -288,8 +291,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             for (; k < total; ++k) {
                 const int s = k % PSTAGES, c = k & (SCB - 1);
                 // the slot's previous operands (step k - PSTAGES) are free once that step's MMAs are done
-                if ((k >= PSTAGES && !mbar_wait(bar(BAR_STEP + (k - PSTAGES) % SR), ((k - PSTAGES) / SR) & 1)) ||
-                    (!ACC && !mbar_wait(bar(BAR_SCE + c), ((k / SCB) & 1) ^ 1))) {
+                if ((k >= PSTAGES && !mbar_wait(bar(BAR_STEP + (k - PSTAGES) % SR), ((k - PSTAGES) / SR) & 1, lim)) ||
+                    (!ACC && !mbar_wait(bar(BAR_SCE + c), ((k / SCB) & 1) ^ 1, lim))) {
                     dead = true;
                     break;
                 }
@@ -326,7 +329,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
             const uint64_t da0 = smem_desc_sw128(base), db0 = smem_desc_sw128(base + A_BYTES);
             for (int k = warp - 1; k < total; k += kIssuers) {  // two issuers: b = k % NBUF is this thread's
                 const int s = k % PSTAGES, b = k % NBUF;
-                if (!mbar_wait(bar(BAR_FULL + s), (k / PSTAGES) & 1) || !mbar_wait(bar(BAR_ACCE + b), (k / NBUF) & 1)) {
+                if (!mbar_wait(bar(BAR_FULL + s), (k / PSTAGES) & 1, lim) ||
+                    !mbar_wait(bar(BAR_ACCE + b), (k / NBUF) & 1, lim)) {
                     dead = true;
                     break;
                 }
@@ -366,8 +370,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_w8a8(const __grid_cons
         TilePos tp = total > 0 ? tile_pos<GRP>(a, t, MB) : TilePos{0, 0, 0, 0, 0};
         for (int k = 0; k < total; ++k) {
             const int b = k % NBUF, c = k & (SCB - 1);
-            if (!mbar_wait(bar(BAR_STEP + k % SR), (k / SR) & 1) ||
-                (!ACC && !mbar_wait(bar(BAR_SCF + c), (k / SCB) & 1))) {
+            const bool ok = mbar_wait(bar(BAR_STEP + k % SR), (k / SR) & 1, lim) &&
+                            (ACC || mbar_wait(bar(BAR_SCF + c), (k / SCB) & 1, lim));
+            if (!__all_sync(kFull, ok)) {  // the warp gives up together
                 dead = true;
                 break;
             }

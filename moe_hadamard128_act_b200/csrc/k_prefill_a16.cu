@@ -221,6 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool dead = false;
+    // Pipeline waits are bounded by lim; the waits that let started copies and MMAs
+    // finish before the CTA ends keep the default bound.
+    const unsigned long long lim = wait_limit(a.err);
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsDriver));
@@ -232,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             int n0 = ti.expert * a.N + ti.wb * TM, m0 = ti.row0;  // code row in the stacked experts, activation row
             for (int k = 0; k < total; ++k) {
                 const int c = k % CS, x = k % XS;
-                if (!mbar_wait(bar(B_CEMPTY + c), ((k / CS) & 1) ^ 1)) {
+                if (!mbar_wait(bar(B_CEMPTY + c), ((k / CS) & 1) ^ 1, lim)) {
                     dead = true;
                     break;
                 }
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 mbar_expect_tx(cb, CODE_BYTES);
                 tma_load_2d(base + c * CODE_BYTES, &a.tmW, g * GK, n0, cb);
                 ++kc;
-                if (k >= XS && !mbar_wait(bar(B_STEP + (k - XS) % SR), ((k - XS) / SR) & 1)) {
+                if (k >= XS && !mbar_wait(bar(B_STEP + (k - XS) % SR), ((k - XS) / SR) & 1, lim)) {
                     dead = true;  // the slot's previous activations are still in use
                     break;
                 }
@@ -268,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             const uint64_t xd0 = smem_desc_sw128(base + X_OFF);
             for (int k = warp - 1; k < total; k += 2) {
                 const int x = k % XS, ab = k % AS, db = k % NACC;
-                if (!mbar_wait(bar(B_XFULL + x), (k / XS) & 1) || !mbar_wait(bar(B_AFULL + ab), (k / AS) & 1) ||
-                    !mbar_wait(bar(B_DEMPTY + db), ((k / NACC) & 1) ^ 1)) {
+                if (!mbar_wait(bar(B_XFULL + x), (k / XS) & 1, lim) || !mbar_wait(bar(B_AFULL + ab), (k / AS) & 1, lim) ||
+                    !mbar_wait(bar(B_DEMPTY + db), ((k / NACC) & 1) ^ 1, lim)) {
                     dead = true;
                     break;
                 }
@@ -299,8 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
         const uint32_t tl = (uint32_t)(32 * q) << 16;
         for (int k = 0; k < total; ++k) {
             const int c = k % CS, ab = k % AS;
-            if (!mbar_wait(bar(B_CFULL + c), (k / CS) & 1) ||
-                (k >= AS && !mbar_wait(bar(B_STEP + (k - AS) % SR), ((k - AS) / SR) & 1))) {
+            const bool ok = mbar_wait(bar(B_CFULL + c), (k / CS) & 1, lim) &&
+                            (k < AS || mbar_wait(bar(B_STEP + (k - AS) % SR), ((k - AS) / SR) & 1, lim));
+            if (!__all_sync(kFull, ok)) {  // the warp gives up together
                 dead = true;  // no codes, or the A tile's previous MMAs are still running
                 break;
             }
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             const float s = FMT == QL_I8_G128_F16 ? f16_bits_to_float((uint16_t)sb_next)
                                                   : bf16_bits_to_float((uint16_t)sb_next);
             if (g + 1 < G) sb_next = scale_raw(g + 1);
-            if (!mbar_wait(bar(B_STEP + k % SR), (k / SR) & 1)) {
+            if (!__all_sync(kFull, mbar_wait(bar(B_STEP + k % SR), (k / SR) & 1, lim))) {  // together
                 dead = true;
                 break;
             }

@@ -117,17 +117,32 @@ __device__ __forceinline__ uint32_t word_of(const uint4 (&w)[2], int s) {
     }
 }
 
+// With a single n-tile the MMAs of a group would form one dependent chain; they
+// alternate between CH accumulators instead, summed here into chain 0.
+template <int CH, int NT, typename T>
+__device__ __forceinline__ void fold_chains(T (&acc)[CH][NT][4]) {
+#pragma unroll
+    for (int ch = 1; ch < CH; ++ch)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[0][nt][i] += acc[ch][nt][i];
+}
+
 // The per-group MMAs of one unit for the weight-only formats.
 // getx(nt, piece) returns the lane's 16-byte activation piece for n-tile nt.
 // yacc[nt][i] accumulates scale * partial; i = 0,1 row g, i = 2,3 row g + 8.
 template <int FMT, int NT, typename GetX>
 __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1_live, float (&yacc)[NT][4]) {
+    constexpr int CH = NT == 1 ? 2 : 1;  // independent accumulation chains per group (see fold_chains)
     if constexpr (FMT == QL_I4_G64_BF16) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float acc[NT][4];
+            float acc[CH][NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+            for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0.0f;
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
                 uint4 xv[NT];
@@ -150,22 +165,25 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
                         if (nt == 1 && !nt1_live) continue;
                         const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
                         const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
-                        mma_f16(acc[nt], a0, a1, a2, a3, b0, b1);
+                        mma_f16(acc[sub % CH][nt], a0, a1, a2, a3, b0, b1);
                     }
                 }
             }
+            fold_chains<CH, NT>(acc);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                yacc[nt][0] = fmaf(r.s[0][h], acc[nt][0], yacc[nt][0]);
-                yacc[nt][1] = fmaf(r.s[0][h], acc[nt][1], yacc[nt][1]);
-                yacc[nt][2] = fmaf(r.s[1][h], acc[nt][2], yacc[nt][2]);
-                yacc[nt][3] = fmaf(r.s[1][h], acc[nt][3], yacc[nt][3]);
+                yacc[nt][0] = fmaf(r.s[0][h], acc[0][nt][0], yacc[nt][0]);
+                yacc[nt][1] = fmaf(r.s[0][h], acc[0][nt][1], yacc[nt][1]);
+                yacc[nt][2] = fmaf(r.s[1][h], acc[0][nt][2], yacc[nt][2]);
+                yacc[nt][3] = fmaf(r.s[1][h], acc[0][nt][3], yacc[nt][3]);
             }
         }
     } else {
-        float acc[NT][4];
+        float acc[CH][NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+        for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0.0f;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             uint4 xv[NT];
@@ -191,16 +209,17 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
                     if (nt == 1 && !nt1_live) continue;
                     const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
                     const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
-                    mma_f16(acc[nt], a0, a1, a2, a3, b0, b1);
+                    mma_f16(acc[sub % CH][nt], a0, a1, a2, a3, b0, b1);
                 }
             }
         }
+        fold_chains<CH, NT>(acc);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            yacc[nt][0] = fmaf(r.s[0], acc[nt][0], yacc[nt][0]);
-            yacc[nt][1] = fmaf(r.s[0], acc[nt][1], yacc[nt][1]);
-            yacc[nt][2] = fmaf(r.s[1], acc[nt][2], yacc[nt][2]);
-            yacc[nt][3] = fmaf(r.s[1], acc[nt][3], yacc[nt][3]);
+            yacc[nt][0] = fmaf(r.s[0], acc[0][nt][0], yacc[nt][0]);
+            yacc[nt][1] = fmaf(r.s[0], acc[0][nt][1], yacc[nt][1]);
+            yacc[nt][2] = fmaf(r.s[1], acc[0][nt][2], yacc[nt][2]);
+            yacc[nt][3] = fmaf(r.s[1], acc[0][nt][3], yacc[nt][3]);
         }
     }
 }
@@ -234,9 +253,12 @@ __device__ __forceinline__ void unit_i5(const Regs<QL_I5Z_G128_F16>& r, GetX get
         A[h][12] = i5_pair<12>(r.w[h]); A[h][13] = i5_pair<13>(r.w[h]); A[h][14] = i5_pair<14>(r.w[h]);
         A[h][15] = i5_pair<15>(r.w[h]);
     }
-    float acc[NT][4];
+    constexpr int CH = NT == 1 ? 2 : 1;
+    float acc[CH][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+    for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0.0f;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {  // the lane's 16-byte activation piece p feeds MMAs 2p and 2p + 1
         uint4 xv[NT];
@@ -249,16 +271,17 @@ __device__ __forceinline__ void unit_i5(const Regs<QL_I5Z_G128_F16>& r, GetX get
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 if (nt == 1 && !nt1_live) continue;
-                mma_f16(acc[nt], A[0][2 * m], A[1][2 * m], A[0][2 * m + 1], A[1][2 * m + 1],
+                mma_f16(acc[sub % CH][nt], A[0][2 * m], A[1][2 * m], A[0][2 * m + 1], A[1][2 * m + 1],
                         sub == 0 ? xv[nt].x : xv[nt].z, sub == 0 ? xv[nt].y : xv[nt].w);
             }
         }
     }
+    fold_chains<CH, NT>(acc);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float t = fmaf(-r.zz[i >> 1], X[nt][i & 1], acc[nt][i]);
+            const float t = fmaf(-r.zz[i >> 1], X[nt][i & 1], acc[0][nt][i]);
             yacc[nt][i] = fmaf(r.s[i >> 1], t, yacc[nt][i]);
         }
 }
@@ -275,9 +298,13 @@ __device__ __forceinline__ void mma_e4m3(float d[4], uint32_t a0, uint32_t a1, u
 
 // W8A8: exact int32 sums of one group (4 k-steps of m16n8k32).
 template <int NT, typename GetX>
-__device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX getx, int (&acc)[NT][4]) {
+__device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX getx, int (&out)[NT][4]) {
+    constexpr int CH = NT == 1 ? 2 : 1;
+    int acc[CH][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+    for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0;
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
         uint4 xv[NT];
@@ -292,17 +319,26 @@ __device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
                 const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
-                mma_s8(acc[nt], a0, a1, a2, a3, b0, b1);
+                mma_s8(acc[sub % CH][nt], a0, a1, a2, a3, b0, b1);
             }
         }
     }
+    fold_chains<CH, NT>(acc);  // integer sums: exact in any order
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) out[nt][i] = acc[0][nt][i];
 }
 
 // Format 7: fp32 sums of one group's E4M3 products, the same walk as unit_w8a8.
 template <int NT, typename GetX>
-__device__ __forceinline__ void unit_e4m3(const Regs<QL_FP8A8_B128_BF16>& r, GetX getx, float (&acc)[NT][4]) {
+__device__ __forceinline__ void unit_e4m3(const Regs<QL_FP8A8_B128_BF16>& r, GetX getx, float (&out)[NT][4]) {
+    constexpr int CH = NT == 1 ? 2 : 1;
+    float acc[CH][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+    for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0.0f;
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
         uint4 xv[NT];
@@ -317,10 +353,15 @@ __device__ __forceinline__ void unit_e4m3(const Regs<QL_FP8A8_B128_BF16>& r, Get
             for (int nt = 0; nt < NT; ++nt) {
                 const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
                 const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
-                mma_e4m3(acc[nt], a0, a1, a2, a3, b0, b1);
+                mma_e4m3(acc[sub % CH][nt], a0, a1, a2, a3, b0, b1);
             }
         }
     }
+    fold_chains<CH, NT>(acc);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) out[nt][i] = acc[0][nt][i];
 }
 
 __device__ __forceinline__ void mma_bf16(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -412,6 +453,15 @@ template <int FMT, int UPS = 1>
 __host__ __device__ constexpr size_t ring_bytes() {
     return (size_t)kWarps * stages_of<FMT, UPS>() * UPS * stage_bytes<FMT>();
 }
+// The grouped (MoE) kernel stages nothing but its ring and the routing state, so
+// its rings are deeper: a small batch gives each warp only a few units, and all of
+// them should be in flight at once.
+constexpr int kMoeStages = 6;
+template <int FMT>
+__host__ __device__ constexpr size_t moe_ring_bytes() {
+    return (size_t)kWarps * kMoeStages * stage_bytes<FMT>();
+}
+
 // Shared memory of the dense kernel staging `rows` token rows of XG groups.
 template <int FMT, int UPS>
 __host__ __device__ constexpr size_t tma_smem(int rows, int XG) {
@@ -683,7 +733,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     __syncthreads();
     QL_PROF(5)
     if (u0 >= u1) return;
-    bool timed_out = rows_x > 0 && !mbar_wait(xbar, 0);
+    const unsigned long long lim = wait_limit(a.err);
+    bool timed_out = rows_x > 0 && !__all_sync(kFull, mbar_wait(xbar, 0, lim));
     QL_PROF(1)
 
     const bool nt1_live = NT > 1 && a.M > 8;
@@ -719,7 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 flush(cur_key);
                 cur_key = key;
             }
-            if (!mbar_wait(bars + 8 * s, phase)) {
+            if (!__all_sync(kFull, mbar_wait(bars + 8 * s, phase, lim))) {  // the warp gives up together
                 timed_out = true;
                 break;
             }
@@ -841,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     const uint32_t base = (raw + 1023u) & ~1023u;
     const bool fused = a.ids != nullptr;
     // Routing state of the fused mode, after the rings and barriers.
-    int* const s_ids = reinterpret_cast<int*>(smem_raw + (base - raw) + ring_bytes<FMT>() + kWarps * kStages * 8);
+    int* const s_ids = reinterpret_cast<int*>(smem_raw + (base - raw) + moe_ring_bytes<FMT>() + kWarps * kMoeStages * 8);
     int* const s_perm = s_ids + kMoeFusedMaxPairs;   // permuted position -> pair index t * topk + j
     int* const s_bef = s_perm + kMoeFusedMaxPairs;   // per position: pairs of the same expert before it
     int* const s_cnt = s_bef + kMoeFusedMaxPairs;    // per position: pairs of its expert
@@ -902,8 +953,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     const long long u0 = units * wid / nw, u1 = units * (wid + 1) / nw;
     if (lane == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmap) : "memory");
 
-    const uint32_t ring = base + (uint32_t)(warp * kStages * SB);
-    const uint32_t bars = base + (uint32_t)ring_bytes<FMT>() + (uint32_t)(warp * kStages * 8);
+    const uint32_t ring = base + (uint32_t)(warp * kMoeStages * SB);
+    const uint32_t bars = base + (uint32_t)moe_ring_bytes<FMT>() + (uint32_t)(warp * kMoeStages * 8);
     if (u0 >= u1) return;
     const long long expert_scales = block_scaled<FMT>() ? (long long)((a.N + 127) / 128) * G : (long long)a.N * G;
     const uint16_t* const sc0 = static_cast<const uint16_t*>(a.scales);
@@ -926,11 +977,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     cp.slab = (int)((u0 % per_chunk) / G);
     cp.grp = (int)(u0 % G);
     Pos ip = cp;
-    Side<FMT, NT> sd[kStages];
+    Side<FMT, NT> sd[kMoeStages];
     long long issued = u0;
     if (lane == 0) {
 #pragma unroll
-        for (int st = 0; st < kStages; ++st) mbar_init(bars + 8 * st, 1);
+        for (int st = 0; st < kMoeStages; ++st) mbar_init(bars + 8 * st, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncwarp();
@@ -947,7 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
         ++issued;
     };
 #pragma unroll
-    for (int st = 0; st < kStages; ++st)
+    for (int st = 0; st < kMoeStages; ++st)
         if (issued < u1) issue(st);
 
     float yacc[NT][4];
@@ -996,11 +1047,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     };
 
     bool timed_out = false;
+    const unsigned long long lim = wait_limit(a.err);
     unsigned phase = 0;
     long long u = u0;
     while (u < u1 && !timed_out) {
 #pragma unroll
-        for (int st = 0; st < kStages; ++st) {
+        for (int st = 0; st < kMoeStages; ++st) {
             if (u >= u1) break;
             if (cp.ch != cur_ch || cp.slab != cur_slab) {
                 flush();
@@ -1011,7 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 cur_ch = cp.ch;
                 cur_slab = cp.slab;
             }
-            if (!mbar_wait(bars + 8 * st, phase)) {
+            if (!__all_sync(kFull, mbar_wait(bars + 8 * st, phase, lim))) {  // the warp gives up together
                 timed_out = true;
                 break;
             }
@@ -1058,7 +1110,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 unit_a16<FMT, NT>(r, getx, chc.count > 8, yacc);
             }
             __syncwarp();
-            if (issued < u1) issue(st);  // refill this slot with the unit kStages ahead
+            if (issued < u1) issue(st);  // refill this slot with the unit kMoeStages ahead
             cp.next(slabs, G);
             ++u;
         }
@@ -1068,8 +1120,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
         if (lane == 0) atomicOr(a.err, (unsigned)QL_DEVERR_TIMEOUT);
         // Let the copies still in flight land before the CTA's memory is released.
         for (long long v = u; v < issued; ++v) {
-            const int st = (int)((v - u0) % kStages);
-            const unsigned ph = (unsigned)(((v - u0) / kStages) & 1);
+            const int st = (int)((v - u0) % kMoeStages);
+            const unsigned ph = (unsigned)(((v - u0) / kMoeStages) & 1);
             if (!mbar_wait(bars + 8 * st, ph)) break;
         }
         return;
@@ -1231,7 +1283,7 @@ cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     if ((e = make_tmap_2d(a.codes, (long long)a.E * a.N, 2LL * a.K, 2LL * a.K, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B,
                           &a.tmap)) != cudaSuccess)
         return e;
-    const size_t smem = 1024 + ring_bytes<kFmtDown>() + (size_t)kWarps * kStages * 8 +
+    const size_t smem = 1024 + moe_ring_bytes<kFmtDown>() + (size_t)kWarps * kMoeStages * 8 +
                         (5 * sizeof(int) + sizeof(MoeChunk)) * kMoeFusedMaxPairs + 16;
     static bool attr_set[64] = {};
     int dev = 0;
@@ -1266,7 +1318,7 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
         cudaSuccess)
         return e;
     // rings, their mbarriers, and the routing state of the fused small-batch mode
-    const size_t smem = 1024 + ring_bytes<QL_I8_G128_BF16>() + (size_t)kWarps * kStages * 8 +
+    const size_t smem = 1024 + moe_ring_bytes<QL_I8_G128_BF16>() + (size_t)kWarps * kMoeStages * 8 +
                         (5 * sizeof(int) + sizeof(MoeChunk)) * kMoeFusedMaxPairs + 16;
     static bool attr_set[64] = {};  // per device ordinal, for all four instantiations at once
     int dev = 0;

@@ -9,8 +9,9 @@
 
 namespace ql {
 
-// The per-process device error word (one per device context).
-__device__ unsigned g_ql_err;
+// The per-process device state (one per device context): [0] the error word,
+// [2..3] the pipeline wait limit in ns as a 64-bit value (0: the default).
+__device__ __align__(16) unsigned g_ql_state[4];
 
 void packed_sizes(int fmt, size_t N, size_t K, size_t* codes, size_t* scales, size_t* zeros) {
     *codes = N * fmt_row_bytes(fmt, K);
@@ -36,7 +37,7 @@ cudaError_t device_info(DeviceInfo* out) {
     if ((e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
     d.smem_optin = (size_t)v;
     void* p = nullptr;
-    if ((e = cudaGetSymbolAddress(&p, g_ql_err)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&p, g_ql_state)) != cudaSuccess) return e;
     d.err_word = static_cast<unsigned*>(p);
     if (dev < 64) {
         cache[dev] = d;
@@ -818,6 +819,15 @@ int ql_trace_read(int* kinds, float* ms, int max, int* count) {
 }
 
 const char* ql_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
+
+int ql_set_wait_limit(unsigned long long ns) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return from_cuda(e);
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return from_cuda(e);
+    if ((e = cudaMemcpy(di.err_word + 2, &ns, sizeof ns, cudaMemcpyHostToDevice)) != cudaSuccess) return from_cuda(e);
+    return QL_OK;
+}
 
 int ql_get_device_error(void* stream, unsigned* bits) {
     DeviceInfo di;

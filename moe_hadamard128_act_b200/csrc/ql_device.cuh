@@ -241,15 +241,24 @@ __device__ __forceinline__ unsigned long long global_ns() {
     asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
     return t;
 }
-// Wait for phase `phase` of the mbarrier; false after ~kWaitNs without it.
+// Wait for phase `phase` of the mbarrier; false after ~lim ns without it.  The
+// kernels bound their pipeline waits by wait_limit() and the waits that let
+// work already started finish (copies in flight, MMAs before tensor memory is
+// freed) by the default kWaitNs.
 constexpr unsigned long long kWaitNs = 200ull * 1000 * 1000;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned phase) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned phase, unsigned long long lim = kWaitNs) {
     if (mbar_try_wait(bar, phase)) return true;
     const unsigned long long t0 = global_ns();
     for (unsigned it = 0;; ++it) {
         if (mbar_try_wait(bar, phase)) return true;
-        if ((it & 255u) == 255u && global_ns() - t0 > kWaitNs) return false;
+        if (((it & 255u) == 255u || lim < kWaitNs) && global_ns() - t0 > lim) return false;
     }
+}
+// The pipeline wait limit: the override that ql_set_wait_limit stores next to
+// the device error word (err[2..3]), or kWaitNs when it is 0.
+__device__ __forceinline__ unsigned long long wait_limit(const unsigned* err) {
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(err + 2);
+    return v ? v : kWaitNs;
 }
 // One contiguous global -> shared copy, completing on an mbarrier (16-byte
 // aligned addresses, size a multiple of 16).

@@ -40,7 +40,7 @@ cudaError_t make_tmap_2d(const void* base, long long rows, long long width_bytes
 struct DeviceInfo {
     int sm_count;
     size_t smem_optin;   // max dynamic shared memory per block (opt-in)
-    unsigned* err_word;  // device address of the error word
+    unsigned* err_word;  // device address of the error word; the wait limit follows it (see wait_limit)
 };
 cudaError_t device_info(DeviceInfo* out);
 

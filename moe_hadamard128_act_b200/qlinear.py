@@ -31,6 +31,7 @@ FORMATS = (I8_G128_BF16, I8_G128_F16, I8A8_G128_BF16, I4_G64_BF16, I5Z_G128_F16,
 
 DEVERR_EXPERT_ID = 1
 DEVERR_CODE_RANGE = 2
+DEVERR_TIMEOUT = 4
 
 A16_MAX_K = 32768  # QL_A16_MAX_K: largest K for the formats whose activations stay 16-bit
 
@@ -79,6 +80,7 @@ _SIGS = {
     "moe_down_workspace_size": (_I, [ctypes.POINTER(ql_down_experts), _I, _I, _PSZ]),
     "moe_down_combine": (_I, [_P, _P, _P, ctypes.POINTER(ql_down_experts), _I, _I, _P, _P, _SZ, _P]),
     "ql_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "ql_set_wait_limit": (_I, [ctypes.c_ulonglong]),
     "qlinear_forward_w8a8_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "ql_trace_enable": (_I, [_I]),
     "ql_trace_read": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float), _I,
@@ -351,3 +353,8 @@ def ql_get_device_error(stream=None):
     bits = ctypes.c_uint()
     st = lib().ql_get_device_error(_stream(stream), ctypes.byref(bits))
     return st, bits.value
+
+
+def ql_set_wait_limit(ns: int):
+    """Bound the kernels' pipeline waits to ns nanoseconds on the current device (0: the default)."""
+    _check("ql_set_wait_limit", lib().ql_set_wait_limit(int(ns)))
