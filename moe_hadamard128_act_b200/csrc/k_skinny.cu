@@ -453,10 +453,11 @@ template <int FMT, int UPS = 1>
 __host__ __device__ constexpr size_t ring_bytes() {
     return (size_t)kWarps * stages_of<FMT, UPS>() * UPS * stage_bytes<FMT>();
 }
-// The grouped (MoE) kernel stages nothing but its ring and the routing state, so
-// its rings are deeper: a small batch gives each warp only a few units, and all of
-// them should be in flight at once.
-constexpr int kMoeStages = 6;
+// The grouped (MoE) kernel reads its activations through L1 (a chunk's tokens are
+// scattered rows of the prepared x), so it keeps the ring at four slots and asks
+// for no more shared memory than it uses: the rest of the SM's 256 KB stays L1.
+// (Six slots were measured slower at every decode batch size.)
+constexpr int kMoeStages = 4;
 template <int FMT>
 __host__ __device__ constexpr size_t moe_ring_bytes() {
     return (size_t)kWarps * kMoeStages * stage_bytes<FMT>();
@@ -1273,6 +1274,14 @@ cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
+// The smallest shared-memory carveout (percent of the most a CTA can take) that
+// holds `smem` bytes and the CTA's reserved kilobyte; the rest of the SM stays L1.
+int moe_carveout(size_t smem, size_t optin) {
+    const size_t need = smem + 1024;
+    const int pct = (int)((need * 100 + optin - 1) / optin);
+    return pct > 100 ? 100 : pct;
+}
+
 cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
@@ -1291,6 +1300,9 @@ cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     if (dev >= 64 || !attr_set[dev]) {
         if ((e = cudaFuncSetAttribute(k_moe_tma<kFmtDown, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
             cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(k_moe_tma<kFmtDown, 2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      moe_carveout(smem, di.smem_optin))) != cudaSuccess)
             return e;
         if (dev < 64) attr_set[dev] = true;
     }
@@ -1325,9 +1337,13 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
         for (auto kern : {k_moe_tma<QL_I8_G128_BF16, 2>, k_moe_tma<QL_I8_G128_F16, 2>, k_moe_tma<QL_FP8_B128_BF16, 2>,
-                          k_moe_tma<QL_FP8A8_B128_BF16, 2>})
+                          k_moe_tma<QL_FP8A8_B128_BF16, 2>}) {
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
                 return e;
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          moe_carveout(smem, di.smem_optin))) != cudaSuccess)
+                return e;
+        }
         if (dev < 64) attr_set[dev] = true;
     }
     auto run = [&](auto kern) -> cudaError_t {

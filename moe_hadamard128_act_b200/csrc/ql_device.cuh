@@ -246,7 +246,19 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // work already started finish (copies in flight, MMAs before tensor memory is
 // freed) by the default kWaitNs.
 constexpr unsigned long long kWaitNs = 200ull * 1000 * 1000;
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, unsigned phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned phase, unsigned long long lim = kWaitNs) {
+    // A bound of at most 1 ns: one probe that does not block (try_wait may suspend for
+    // a while, long enough for a copy to land), so the wait gives up unless done already.
+    if (lim <= 1) return mbar_test_wait(bar, phase);
     if (mbar_try_wait(bar, phase)) return true;
     const unsigned long long t0 = global_ns();
     for (unsigned it = 0;; ++it) {
