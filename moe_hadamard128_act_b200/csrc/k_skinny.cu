@@ -453,10 +453,9 @@ template <int FMT, int UPS = 1>
 __host__ __device__ constexpr size_t ring_bytes() {
     return (size_t)kWarps * stages_of<FMT, UPS>() * UPS * stage_bytes<FMT>();
 }
-// The grouped (MoE) kernel reads its activations through L1 (a chunk's tokens are
-// scattered rows of the prepared x), so it keeps the ring at four slots and asks
-// for no more shared memory than it uses: the rest of the SM's 256 KB stays L1.
-// (Six slots were measured slower at every decode batch size.)
+// The grouped (MoE) kernel's ring depth.  It reads its activations through L1 (a
+// chunk's tokens are scattered rows of the prepared x); six slots, which leave
+// less of the SM to L1, were measured slower at every decode batch size.
 constexpr int kMoeStages = 4;
 template <int FMT>
 __host__ __device__ constexpr size_t moe_ring_bytes() {
@@ -620,6 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     const int g = lane >> 2, c = lane & 3;
     const int G = a.G / UPS, GP = a.GP / UPS, slabs = (a.N + 15) / 16;
     if (lane == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmap) : "memory");
+    const unsigned long long lim = wait_limit(a.err);  // requested first: its latency hides behind the setup
 
     // Shared memory: [rings][mbarriers][activation barrier][activations], 1024-aligned base.
     const uint32_t raw = smem_u32(smem_raw);
@@ -734,7 +734,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     __syncthreads();
     QL_PROF(5)
     if (u0 >= u1) return;
-    const unsigned long long lim = wait_limit(a.err);
     bool timed_out = rows_x > 0 && !__all_sync(kFull, mbar_wait(xbar, 0, lim));
     QL_PROF(1)
 
@@ -884,6 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     constexpr bool DOWN = FMT == kFmtDown;
     constexpr int SB = stage_bytes<FMT>();
+    const unsigned long long lim = wait_limit(a.err);  // requested first: its latency hides behind the setup
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int G = DOWN ? a.K / 64 : a.K / 128;
@@ -1048,7 +1048,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     };
 
     bool timed_out = false;
-    const unsigned long long lim = wait_limit(a.err);
     unsigned phase = 0;
     long long u = u0;
     while (u < u1 && !timed_out) {
@@ -1274,14 +1273,6 @@ cudaError_t launch_skinny(int fmt, const SkinnyArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
-// The smallest shared-memory carveout (percent of the most a CTA can take) that
-// holds `smem` bytes and the CTA's reserved kilobyte; the rest of the SM stays L1.
-int moe_carveout(size_t smem, size_t optin) {
-    const size_t need = smem + 1024;
-    const int pct = (int)((need * 100 + optin - 1) / optin);
-    return pct > 100 ? 100 : pct;
-}
-
 cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
@@ -1300,9 +1291,6 @@ cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     if (dev >= 64 || !attr_set[dev]) {
         if ((e = cudaFuncSetAttribute(k_moe_tma<kFmtDown, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
             cudaSuccess)
-            return e;
-        if ((e = cudaFuncSetAttribute(k_moe_tma<kFmtDown, 2>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                      moe_carveout(smem, di.smem_optin))) != cudaSuccess)
             return e;
         if (dev < 64) attr_set[dev] = true;
     }
@@ -1339,9 +1327,6 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
         for (auto kern : {k_moe_tma<QL_I8_G128_BF16, 2>, k_moe_tma<QL_I8_G128_F16, 2>, k_moe_tma<QL_FP8_B128_BF16, 2>,
                           k_moe_tma<QL_FP8A8_B128_BF16, 2>}) {
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-                return e;
-            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                          moe_carveout(smem, di.smem_optin))) != cudaSuccess)
                 return e;
         }
         if (dev < 64) attr_set[dev] = true;

@@ -3,11 +3,14 @@
 Every wait of a kernel for a copy, an MMA or another warp's work gives up after
 a bound and sets QL_DEVERR_TIMEOUT instead of hanging; the kernel then lets the
 copies and MMAs it already started finish and frees its tensor memory.  Here the
-bound is set to 1 ns, so the decode GEMM's ring waits and the tcgen05 prefill
-GEMM's pipeline waits run out at once: the calls must return, the error word
-must report the timeout, and after the default bound is restored the same calls
-on the same process and GPU must match the oracle (nothing was left allocated
-or in flight)."""
+bound is set to 1 ns, which makes every pipeline wait a single probe that does
+not block.  The tcgen05 prefill GEMM's first waits (for its first operand tiles,
+its first MMAs) cannot be satisfied that early, so it must report the timeout,
+with copies in flight to drain and tensor memory to free.  The decode GEMM's
+ring runs several units ahead of its use, so its probes may all succeed; its
+call must return either way.  After the default bound is restored, both calls
+on the same process and GPU must match the oracle (nothing was left allocated or
+in flight)."""
 import numpy as np
 import pytest
 
@@ -40,7 +43,10 @@ def test_waits_run_out_then_recover(Q):
         for M, what in cases:
             Q.qlinear_forward(dev_bf16(xs[M]), c, s, None, Q.I8A8_G128_BF16, N, flags=Q.HADAMARD)
             st, bits = Q.ql_get_device_error()
-            assert st == 6 and bits & Q.DEVERR_TIMEOUT, (what, st, bits)
+            if what == "prefill":
+                assert st == 6 and bits & Q.DEVERR_TIMEOUT, (what, st, bits)
+            else:  # returned, and nothing but a timeout was flagged
+                assert st in (0, 6) and bits & ~Q.DEVERR_TIMEOUT == 0, (what, st, bits)
     finally:
         Q.ql_set_wait_limit(0)
     for M, what in cases:
