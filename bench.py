@@ -56,7 +56,7 @@ def parse():
                         "prefill); default all")
     p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "prefill_w5a8",
                                           "moe_decode", "moe_decode_t1", "moe_prefill", "act_quant", "decode_w4a16",
-                                          "decode_w5a16", "decode_w8a16", "decode_fp8"],
+                                          "decode_w5a16", "decode_w8a16", "decode_fp8", "moe_down"],
                    default=None,
                    help="run only a small fixed case for an ncu capture (2 warm-up + 2 profiled launches)")
     return p.parse_args()
@@ -565,7 +565,10 @@ def ncu_case(name):
     moe_decode / moe_decode_t1 / moe_prefill: the MoE gate_up experts (128 x
     [1408, 2816] int8 g128 bf16, Hadamard domain; about 0.5 GB), top-8 routing
     of T = 16 / 1 / 2048 tokens, four calls of moe_gate_up (activation
-    prologue and expert GEMM; the permute too at T = 2048)."""
+    prologue and expert GEMM; the permute too at T = 2048).
+    moe_down: the bf16 down projection (128 x [2816, 704], 507 MB) with its
+    routing-weighted combine for T = 2048 tokens, top-8, four calls of
+    moe_down_combine (permute, activation planes, grouped tensor-core GEMM)."""
     import torch
 
     from moe_hadamard128_act_b200 import qlinear as Q
@@ -603,6 +606,25 @@ def ncu_case(name):
         x = torch.from_numpy(synth.activations(0, "x_aq", M, K_FULL).view(np.int16)).view(torch.bfloat16).to(dev)
         for i in range(4):
             Q.act_quant_i8_g128(x, rotate=True)
+        torch.cuda.synchronize()
+        st, bits = Q.ql_get_device_error()
+        assert st == 0, bits
+        print(f"ncu case {name} done")
+        return
+    if name == "moe_down":
+        E, topk, Ke, I, T = 128, 8, 2816, 704, 2048
+        wd = torch.empty((E, Ke, I), dtype=torch.int16, device=dev)
+        dd = synth.moe_down(1, experts=range(E))
+        for e in range(E):
+            wd[e] = torch.from_numpy(dd["Wd"][e].view(np.int16)).to(dev)
+        del dd
+        d = synth.moe_down(T, experts=[])
+        h = torch.from_numpy(d["h"]).to(dev)
+        idt = torch.from_numpy(d["ids"]).to(dev)
+        wt = torch.from_numpy(d["weights"]).to(dev)
+        o = torch.empty((T, Ke), dtype=torch.float32, device=dev)
+        for i in range(4):
+            Q.moe_down_combine(h, idt, wt, wd, E, out=o)
         torch.cuda.synchronize()
         st, bits = Q.ql_get_device_error()
         assert st == 0, bits

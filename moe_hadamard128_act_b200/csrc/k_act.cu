@@ -232,7 +232,7 @@ __device__ __forceinline__ float gelu_tanh_f32(float v) {
 }
 
 __global__ void __launch_bounds__(256) k_moe_act(const float* h, const int32_t* ids, int P, int E, int I,
-                                                 __nv_bfloat16* act, float* out, long long nz) {
+                                                 __nv_bfloat16* act, float* out, long long nz, const int32_t* inv) {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the down GEMM start its weight stream
     zero_fill(out, nz);
     const int I8 = I / 8;
@@ -263,9 +263,10 @@ __global__ void __launch_bounds__(256) k_moe_act(const float* h, const int32_t* 
                 r[1] = __fsub_rn(r[1], __high2float(b));
             }
         }
+        const long long row = inv ? (long long)__ldg(inv + p) : p;
 #pragma unroll
         for (int l = 0; l < 3; ++l)
-            *reinterpret_cast<uint4*>(act + (p * 3 + l) * I + i0) = make_uint4(pl[l][0], pl[l][1], pl[l][2], pl[l][3]);
+            *reinterpret_cast<uint4*>(act + (row * 3 + l) * I + i0) = make_uint4(pl[l][0], pl[l][1], pl[l][2], pl[l][3]);
     }
 }
 
@@ -371,7 +372,7 @@ cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, con
 
 namespace ql {
 cudaError_t launch_moe_act(const float* h, const int32_t* ids, int P, int E, int I, __nv_bfloat16* act, float* out,
-                           long long nz, cudaStream_t s) {
+                           long long nz, cudaStream_t s, const int32_t* inv) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
@@ -381,7 +382,7 @@ cudaError_t launch_moe_act(const float* h, const int32_t* ids, int P, int E, int
     long long blocks = ((work > zb * 256 ? work : zb * 256) + 255) / 256;
     if (blocks > 8LL * di.sm_count) blocks = 8LL * di.sm_count;
     if (blocks < 1) blocks = 1;
-    k_moe_act<<<(unsigned)blocks, 256, 0, s>>>(h, ids, P, E, I, act, out, nz);
+    k_moe_act<<<(unsigned)blocks, 256, 0, s>>>(h, ids, P, E, I, act, out, nz, inv);
     return cudaGetLastError();
 }
 }  // namespace ql

@@ -216,19 +216,32 @@ int check_experts(const ql_experts* ex) {
     return QL_OK;
 }
 
-// moe_down_combine's workspace: the activation planes, then the permutation.
+// moe_down_combine's workspace: the activation planes, then the permutation and either the
+// weight-streaming kernel's chunks or (prefill batches) the grouped GEMM's tiles.
+bool down_grouped(const ql_down_experts* ex, int T, int topk) {
+    return (long long)T * topk >= (long long)kMoePrefillMinRowsPerExpert * ex->E;
+}
 struct DownWs {
-    size_t act, counts, offsets, perm, chunks, nch, total;
+    size_t act, counts, offsets, perm, chunks, inv, tiles, nch, max_tiles, total;
 };
 DownWs down_ws(const ql_down_experts* ex, int T, int topk) {
     DownWs w;
     size_t o = 0;
     const size_t P = (size_t)T * topk;
+    const bool grp = down_grouped(ex, T, topk);
     w.act = o; o += align_up(P * 3 * ex->I * 2, 256);
     w.counts = o; o += align_up((size_t)ex->E * 4, 256);
     w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
     w.perm = o; o += align_up(P * 4, 256);
-    w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
+    w.max_tiles = grp ? moe_max_tiles(T, topk, ex->E, kPrefillA16Tokens, (ex->K + 127) / 128) : 0;
+    if (grp) {
+        w.chunks = 0;
+        w.inv = o; o += align_up(P * 4, 256);
+        w.tiles = o; o += align_up(w.max_tiles * sizeof(MoeTile), 256);
+    } else {
+        w.inv = w.tiles = 0;
+        w.chunks = o; o += align_up(moe_max_chunks(T, topk, ex->E) * sizeof(MoeChunk), 256);
+    }
     w.nch = o; o += 256;
     w.total = o;
     return w;
@@ -744,6 +757,30 @@ int moe_down_combine(const float* h, const int32_t* topk_ids, const float* topk_
     MoeChunk* chunks = reinterpret_cast<MoeChunk*>(b + w.chunks);
     int* nch = reinterpret_cast<int*>(b + w.nch);
     const int P = T * topk;
+    if (down_grouped(experts, T, topk)) {
+        // permute into 192-row tiles; the planes straight into permuted order (and out zeroed);
+        // the grouped bf16 tensor-core GEMM adds each pair's share into its token's row
+        MoePermuteOut po;
+        po.inv = reinterpret_cast<int32_t*>(b + w.inv);
+        po.tiles = reinterpret_cast<MoeTile*>(b + w.tiles);
+        po.n_tiles = nch;
+        po.tile_rows = kPrefillA16Tokens;
+        po.wblocks = (experts->K + 127) / 128;
+        int t = trace_begin(QL_KIND_MOE_PERMUTE, s);
+        cudaError_t e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_MOE_ACT, s);
+        e = launch_moe_act(h, topk_ids, P, experts->E, experts->I, act, out, (long long)T * experts->K, s, po.inv);
+        trace_end(t, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        t = trace_begin(QL_KIND_MOE_DOWN, s);
+        e = launch_prefill_down_grouped(act, static_cast<const uint16_t*>(experts->weights), experts->E, experts->K,
+                                        experts->I, P, po.tiles, nch, (int)w.max_tiles, perm, topk, topk_weights, out,
+                                        s);
+        trace_end(t, s);
+        return from_cuda(e);
+    }
     // gelu(gate) * up as three bf16 planes, and the zeroing of out
     int t = trace_begin(QL_KIND_MOE_ACT, s);
     cudaError_t e = launch_moe_act(h, topk_ids, P, experts->E, experts->I, act, out, (long long)T * experts->K, s);

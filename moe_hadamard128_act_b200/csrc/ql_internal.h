@@ -184,6 +184,14 @@ cudaError_t launch_prefill_e4m3_grouped(const uint8_t* qx, const float* sxT, int
                                         const float* swT, int E, int N, int K, int rows_total, const MoeTile* tiles,
                                         const int* n_tiles, int max_tiles, const int32_t* perm, float* y,
                                         cudaStream_t s);
+// The experts' bf16 down projection on the grouped tensor-core GEMM (a mode of the A16 kernel):
+// act holds each pair's activation as three bf16 planes [rows_total][3 I] in permuted order, wd the
+// stacked bf16 weights [E * N][I]; tiles of kPrefillA16Tokens permuted rows x 128 weight rows from
+// the permute; row r of a tile is added into y[perm[r] / topk][0 .. N) scaled by wts[perm[r]].
+constexpr int kFmtDownA16 = 17;
+cudaError_t launch_prefill_down_grouped(const __nv_bfloat16* act, const uint16_t* wd, int E, int N, int I,
+                                        int rows_total, const MoeTile* tiles, const int* n_tiles, int max_tiles,
+                                        const int32_t* perm, int topk, const float* wts, float* y, cudaStream_t s);
 // From this many (token, slot) pairs per expert on average, moe_gate_up runs the grouped tensor-core GEMM.
 constexpr int kMoePrefillMinRowsPerExpert = 8;
 cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,
@@ -213,10 +221,10 @@ cudaError_t launch_moe_skinny(const MoeArgs& a, cudaStream_t s);
 // sum_j wts[t*topk+j] * (act of (t, j)) . W_e^T.  Chunks / fused ranking as launch_moe_skinny.
 cudaError_t launch_moe_down(const MoeArgs& a, cudaStream_t s);
 // gelu(gate) * up of each pair's gate_up row h [P][2 I] (fp32), split into three bf16 planes
-// act [P][3][I] whose sum is the fp32 value; pairs with an id outside [0, E) are skipped.  Also
-// zeroes out[0 .. nz).
+// act [P][3][I] whose sum is the fp32 value (pair p to row inv[p] when inv is given, the permuted
+// order); pairs with an id outside [0, E) are skipped.  Also zeroes out[0 .. nz).
 cudaError_t launch_moe_act(const float* h, const int32_t* ids, int P, int E, int I, __nv_bfloat16* act, float* out,
-                           long long nz, cudaStream_t s);
+                           long long nz, cudaStream_t s, const int32_t* inv = nullptr);
 
 // ---- launch trace (ql_trace_enable / ql_trace_read) --------------------------------------
 // trace_begin records a start event for one library launch when tracing is on
