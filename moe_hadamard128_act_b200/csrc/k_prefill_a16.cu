@@ -23,9 +23,11 @@
 // factor and written to y (32 lanes of a warp write 32 consecutive y values).
 //
 // Warp roles: warpgroup 0 (24 registers per thread after setmaxnreg): lane 0
-// of warp 0 issues the TMA loads (code tile [128 rows][128 B] into a 4- or
-// 6-slot ring, activation tile [TN rows][2 x 128 B] into a 3-slot ring), lane 0 of
-// warps 1 and 2 issue the MMAs of the even and the odd steps.  The next one
+// of warp 0 issues the TMA loads of the code tiles [128 rows][128 B] into a 4-
+// or 6-slot ring, lane 0 of warp 3 those of the activation tiles [TN rows][2 x
+// 128 B] into a 3-slot ring (two threads, so that neither ring waits for the
+// other and each loop fits the warpgroup's registers), lane 0 of warps 1 and 2
+// issue the MMAs of the even and the odd steps.  The next one
 // or two warpgroups (40 registers) convert: thread i of warp 4 + 4 h + q
 // converts part h of weight row 32 q + i (the whole row with one warpgroup,
 // halves with two).  The last four warpgroups (96 or 104 registers) are the
@@ -103,17 +105,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 // kind::f16: D f32, A f16, B f16, both K-major, N = TN, M = 128.
 constexpr uint32_t kIdescF16 = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(TN >> 3) << 17) |
                                ((uint32_t)(TM >> 4) << 24);
-// The same with A and B bf16 (the down projection: bf16 weights, bf16 activation planes).
-constexpr uint32_t kIdescBF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TN >> 3) << 17) |
-                                ((uint32_t)(TM >> 4) << 24);
 
 // D (+)= A * B^T with A in tensor memory; acc_in = 0 overwrites D.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t acc_in,
-                                           uint32_t idesc = kIdescF16) {
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t acc_in) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc_in));
+        "r"(a_tmem), "l"(bdesc), "r"(kIdescF16), "r"(acc_in));
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
@@ -161,12 +159,6 @@ struct A16Args {
     const int* n_tiles;
     const int32_t* perm;   // grouped: permuted row -> pair index t * topk + j
     int topk;
-    // Down projection (kFmtDownA16): the weights are bf16 [E * N][GW * 64]; a step is 64 K, the
-    // activation rows are the three bf16 planes of each pair [rows][3 * GW * 64], so step k takes
-    // weight columns (k % GW) * 64 and activation columns k * 64; finished rows are added into
-    // y[pair / topk] scaled by wts[pair].
-    const float* wts;
-    int GW;
 };
 
 // The tile a CTA works on: expert, first activation row, rows, weight block.
@@ -194,9 +186,6 @@ __device__ __forceinline__ void convert16(const uint4 u, uint32_t* w) {
 
 template <int FMT, bool GRP>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_constant__ A16Args a) {
-    constexpr bool DOWN = FMT == kFmtDownA16;
-    static_assert(!DOWN || GRP, "the down projection runs grouped");
-    constexpr int KSTEP = DOWN ? 64 : GK;  // K per step: 64 bf16 weights, or 128 one-byte codes
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -240,50 +229,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsDriver));
-        if (warp == 0 && lane == 0) {  // ---- producer ----
+        if (warp == 0 && lane == 0) {  // ---- producer of the code tiles ----
             asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmW) : "memory");
-            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmX) : "memory");
-            int g = 0, t = blockIdx.x, kc = 0, kx = 0;  // code / activation copies issued
-            MoeTile ti = my_tiles > 0 ? tile_at<GRP>(a, t, TB) : MoeTile{0, 0, 0, 0};
-            int n0 = ti.expert * a.N + ti.wb * TM, m0 = ti.row0;  // code row in the stacked experts, activation row
-            for (int k = 0; k < total; ++k) {
-                const int c = k % CS, x = k % XS;
+            int g = 0, t = blockIdx.x, k = 0;
+            int n0 = 0;  // code row of the tile in the stacked experts
+            for (; k < total; ++k) {
+                if (g == 0) {
+                    const MoeTile ti = tile_at<GRP>(a, t, TB);
+                    n0 = ti.expert * a.N + ti.wb * TM;
+                }
+                const int c = k % CS;
                 if (!mbar_wait(bar(B_CEMPTY + c), ((k / CS) & 1) ^ 1, lim)) {
                     dead = true;
                     break;
                 }
                 const uint32_t cb = bar(B_CFULL + c);
                 mbar_expect_tx(cb, CODE_BYTES);
-                tma_load_2d(base + c * CODE_BYTES, &a.tmW, DOWN ? (g % a.GW) * 128 : g * GK, n0, cb);
-                ++kc;
+                tma_load_2d(base + c * CODE_BYTES, &a.tmW, g * GK, n0, cb);
+                if (++g == G) {
+                    g = 0;
+                    t += gridDim.x;
+                }
+            }
+            // Copies still in flight must land before the CTA's shared memory is released.
+            for (int j = k > CS ? k - CS : 0; j < k; ++j)
+                if (!mbar_wait(bar(B_CFULL + j % CS), (j / CS) & 1)) break;
+        } else if (warp == 3 && lane == 0) {  // ---- producer of the activation tiles ----
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmX) : "memory");
+            int g = 0, t = blockIdx.x, k = 0;
+            int m0 = 0;  // first activation row of the tile
+            for (; k < total; ++k) {
+                if (g == 0) m0 = tile_at<GRP>(a, t, TB).row0;
+                const int x = k % XS;
                 if (k >= XS && !mbar_wait(bar(B_STEP + (k - XS) % SR), ((k - XS) / SR) & 1, lim)) {
                     dead = true;  // the slot's previous activations are still in use
                     break;
                 }
                 const uint32_t xb = bar(B_XFULL + x), xd = base + X_OFF + x * X_BYTES;
-                if (DOWN) {  // one 64-wide atom of the activation planes
-                    mbar_expect_tx(xb, XATOM);
-                    tma_load_2d(xd, &a.tmX, g * 128, m0, xb);
-                } else {
-                    mbar_expect_tx(xb, X_BYTES);
-                    tma_load_2d(xd, &a.tmX, g * GK * 2, m0, xb);
-                    tma_load_2d(xd + XATOM, &a.tmX, g * GK * 2 + 128, m0, xb);
-                }
-                ++kx;
+                mbar_expect_tx(xb, X_BYTES);
+                tma_load_2d(xd, &a.tmX, g * GK * 2, m0, xb);
+                tma_load_2d(xd + XATOM, &a.tmX, g * GK * 2 + 128, m0, xb);
                 if (++g == G) {
                     g = 0;
                     t += gridDim.x;
-                    if (k + 1 < total) {
-                        ti = tile_at<GRP>(a, t, TB);
-                        n0 = ti.expert * a.N + ti.wb * TM;
-                        m0 = ti.row0;
-                    }
                 }
             }
-            // Copies still in flight must land before the CTA's shared memory is released.
-            for (int j = kc > CS ? kc - CS : 0; j < kc; ++j)
-                if (!mbar_wait(bar(B_CFULL + j % CS), (j / CS) & 1)) break;
-            for (int j = kx > XS ? kx - XS : 0; j < kx; ++j)
+            for (int j = k > XS ? k - XS : 0; j < k; ++j)
                 if (!mbar_wait(bar(B_XFULL + j % XS), (j / XS) & 1)) break;
         } else if ((warp == 1 || warp == 2) && lane == 0) {  // ---- MMA issuers: even / odd steps ----
             const uint64_t xd0 = smem_desc_sw128(base + X_OFF);
@@ -298,9 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 const uint32_t d = tmem + db * TN, at = tmem + A_COL0 + ab * ACOLS;
                 const uint64_t xo = (uint64_t)((x * X_BYTES) >> 4);
 #pragma unroll
-                for (int j = 0; j < KSTEP / 16; ++j)
+                for (int j = 0; j < GK / 16; ++j)
                     mma_f16_ts(d, at + 8 * j, xd0 + xo + (uint64_t)((j / 4) * (XATOM >> 4) + (j % 4) * 2),
-                               j ? 1u : 0u, DOWN ? kIdescBF16 : kIdescF16);
+                               j ? 1u : 0u);
                 // One commit per step: its accumulator is ready for the epilogue, and its
                 // A tile and activation slot may be refilled.  A waiter for step j checks
                 // the parity of its completion on slot j % SR, and the slot cannot
@@ -330,31 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             // Row r of the code tile: 16-byte chunk j sits at chunk j ^ (r & 7) (128-byte swizzle).
             const uint32_t rowp = base + c * CODE_BYTES + r * 128;
             const uint32_t at = tmem + tl + A_COL0 + ab * ACOLS + 8 * CPW * h;
-            if constexpr (DOWN) {
-                // bf16 weights go to tensor memory as they are: 4 chunks (32 values) per 16 columns
-                static_assert(!DOWN || CPW == 8, "the down projection's converter takes whole rows");
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 u = lds128(rowp + (((4 * j + q4) ^ (r & 7)) << 4));
-                        w[4 * q4] = u.x;
-                        w[4 * q4 + 1] = u.y;
-                        w[4 * q4 + 2] = u.z;
-                        w[4 * q4 + 3] = u.w;
-                    }
-                    QL_TMEM_ST16(at + 16 * j, w);
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < CPW / 2; ++j) {
-                    const int ch = CPW * h + 2 * j;  // 16-byte chunks ch, ch + 1: codes 16 ch .. 16 ch + 31
-                    uint32_t w[16];
-                    convert16<FMT>(lds128(rowp + ((ch ^ (r & 7)) << 4)), w);
-                    convert16<FMT>(lds128(rowp + (((ch + 1) ^ (r & 7)) << 4)), w + 8);
-                    QL_TMEM_ST16(at + 16 * j, w);
-                }
+            for (int j = 0; j < CPW / 2; ++j) {
+                const int ch = CPW * h + 2 * j;  // 16-byte chunks ch, ch + 1: codes 16 ch .. 16 ch + 31
+                uint32_t w[16];
+                convert16<FMT>(lds128(rowp + ((ch ^ (r & 7)) << 4)), w);
+                convert16<FMT>(lds128(rowp + (((ch + 1) ^ (r & 7)) << 4)), w + 8);
+                QL_TMEM_ST16(at + 16 * j, w);
             }
             asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
             tc_fence_before();
@@ -389,8 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             n = ti.wb * TM + 32 * q + lane;
             row0 = ti.row0 + cg * EPC;
             rows = ti.rows - cg * EPC;
-            if (DOWN) sp = nullptr;  // no scales: the bf16 weights are the values
-            else if (FMT == QL_FP8_B128_BF16) sp = a.sw + ((long long)ti.expert * NBk + n / 128) * G;
+            if (FMT == QL_FP8_B128_BF16) sp = a.sw + ((long long)ti.expert * NBk + n / 128) * G;
             else sp = n < a.N ? a.sw + ((long long)ti.expert * a.N + n) * G : nullptr;  // rows past N: scale 0
             pr0 = pr1 = 0;
             if (GRP) {  // row r of the permuted activations is the pair perm[r] = t * topk + j
@@ -409,9 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
         }
         for (int k = 0; k < total; ++k) {
             const int db = k % NACC;
-            const float s = DOWN ? 1.0f
-                            : FMT == QL_I8_G128_F16 ? f16_bits_to_float((uint16_t)sb_next)
-                                                    : bf16_bits_to_float((uint16_t)sb_next);
+            const float s = FMT == QL_I8_G128_F16 ? f16_bits_to_float((uint16_t)sb_next)
+                                                  : bf16_bits_to_float((uint16_t)sb_next);
             if (g + 1 < G) sb_next = scale_raw(g + 1);
             if (!__all_sync(kFull, mbar_wait(bar(B_STEP + k % SR), (k / SR) & 1, lim))) {  // together
                 dead = true;
@@ -431,22 +402,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_DEMPTY + db));
 
-            if (g == min(1, G - 1)) {  // the token factors (down: routing weights), once the rows have arrived
-                const float* const fs = DOWN ? a.wts : a.xf;
-                const int dv = DOWN ? 1 : a.topk;
-                f0 = lane < rows ? __ldg(fs + (GRP ? pr0 / dv : pr0)) : 0.0f;
-                f1 = 32 + lane < min(rows, EPC) ? __ldg(fs + (GRP ? pr1 / dv : pr1)) : 0.0f;
+            if (g == min(1, G - 1)) {  // the token factors, once the output rows have arrived
+                f0 = lane < rows ? __ldg(a.xf + (GRP ? pr0 / a.topk : pr0)) : 0.0f;
+                f1 = 32 + lane < min(rows, EPC) ? __ldg(a.xf + (GRP ? pr1 / a.topk : pr1)) : 0.0f;
             }
             if (++g == G) {  // tile done: activation rows row0 .. row0 + EPC - 1 against weight row n
 #pragma unroll
                 for (int i = 0; i < EPC; ++i) {
                     const float f = __shfl_sync(kFull, i < 32 ? f0 : f1, i & 31);
                     const long long orow = __shfl_sync(kFull, i < 32 ? pr0 : pr1, i & 31);
-                    if (DOWN) {  // the pair's routing-weighted share of its token's output row
-                        if (i < rows && n < a.N) atomicAdd(a.y + (orow / a.topk) * a.ldy + n, yacc[i] * f);
-                    } else if (i < rows && n < a.N) {
-                        a.y[orow * a.ldy + n] = yacc[i] * f;
-                    }
+                    if (i < rows && n < a.N) a.y[orow * a.ldy + n] = yacc[i] * f;
                 }
 #pragma unroll
                 for (int i = 0; i < EPC; ++i) yacc[i] = 0.0f;
@@ -494,39 +459,6 @@ cudaError_t launch_any(int fmt, const A16Args& a, int grid, cudaStream_t s) {
 }
 
 }  // namespace
-
-cudaError_t launch_prefill_down_grouped(const __nv_bfloat16* act, const uint16_t* wd, int E, int N, int I,
-                                        int rows_total, const MoeTile* tiles, const int* n_tiles, int max_tiles,
-                                        const int32_t* perm, int topk, const float* wts, float* y, cudaStream_t s) {
-    if (I % 64) return cudaErrorInvalidValue;
-    DeviceInfo di;
-    cudaError_t e = device_info(&di);
-    if (e != cudaSuccess) return e;
-    if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
-    A16Args a{};
-    if ((e = make_tmap_2d(wd, (long long)E * N, 2LL * I, 2LL * I, 128, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) !=
-        cudaSuccess)
-        return e;
-    if ((e = make_tmap_2d(act, rows_total, 6LL * I, 6LL * I, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) !=
-        cudaSuccess)
-        return e;
-    a.sw = nullptr;
-    a.xf = nullptr;
-    a.y = y;
-    a.err = di.err_word;
-    a.M = rows_total;
-    a.N = N;
-    a.G = 3 * I / 64;  // steps per tile: the three planes' K
-    a.GW = I / 64;
-    a.ldy = N;
-    a.tiles = tiles;
-    a.n_tiles = n_tiles;
-    a.perm = perm;
-    a.topk = topk;
-    a.wts = wts;
-    const int grid = max_tiles < di.sm_count ? max_tiles : di.sm_count;
-    return launch_fmt<kFmtDownA16, true>(a, grid, s);
-}
 
 bool prefill_a16_supported(int fmt) {
     return fmt == QL_I8_G128_BF16 || fmt == QL_I8_G128_F16 || fmt == QL_FP8_B128_BF16;

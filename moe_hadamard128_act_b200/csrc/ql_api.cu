@@ -233,7 +233,7 @@ DownWs down_ws(const ql_down_experts* ex, int T, int topk) {
     w.counts = o; o += align_up((size_t)ex->E * 4, 256);
     w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
     w.perm = o; o += align_up(P * 4, 256);
-    w.max_tiles = grp ? moe_max_tiles(T, topk, ex->E, kPrefillA16Tokens, (ex->K + 127) / 128) : 0;
+    w.max_tiles = grp ? moe_max_tiles(T, topk, ex->E, kDownTileRows, (ex->K + 127) / 128) : 0;
     if (grp) {
         w.chunks = 0;
         w.inv = o; o += align_up(P * 4, 256);
@@ -758,13 +758,13 @@ int moe_down_combine(const float* h, const int32_t* topk_ids, const float* topk_
     int* nch = reinterpret_cast<int*>(b + w.nch);
     const int P = T * topk;
     if (down_grouped(experts, T, topk)) {
-        // permute into 192-row tiles; the planes straight into permuted order (and out zeroed);
-        // the grouped bf16 tensor-core GEMM adds each pair's share into its token's row
+        // permute into tiles of up to 160 rows; the planes straight into permuted order (and out
+        // zeroed); the grouped bf16 tensor-core GEMM adds each pair's share into its token's row
         MoePermuteOut po;
         po.inv = reinterpret_cast<int32_t*>(b + w.inv);
         po.tiles = reinterpret_cast<MoeTile*>(b + w.tiles);
         po.n_tiles = nch;
-        po.tile_rows = kPrefillA16Tokens;
+        po.tile_rows = kDownTileRows;
         po.wblocks = (experts->K + 127) / 128;
         int t = trace_begin(QL_KIND_MOE_PERMUTE, s);
         cudaError_t e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
@@ -775,9 +775,8 @@ int moe_down_combine(const float* h, const int32_t* topk_ids, const float* topk_
         trace_end(t, s);
         if (e != cudaSuccess) return from_cuda(e);
         t = trace_begin(QL_KIND_MOE_DOWN, s);
-        e = launch_prefill_down_grouped(act, static_cast<const uint16_t*>(experts->weights), experts->E, experts->K,
-                                        experts->I, P, po.tiles, nch, (int)w.max_tiles, perm, topk, topk_weights, out,
-                                        s);
+        e = launch_down_grouped(act, static_cast<const uint16_t*>(experts->weights), experts->E, experts->K,
+                                experts->I, P, po.tiles, nch, (int)w.max_tiles, perm, topk, topk_weights, out, s);
         trace_end(t, s);
         return from_cuda(e);
     }

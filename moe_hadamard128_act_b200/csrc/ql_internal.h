@@ -184,14 +184,15 @@ cudaError_t launch_prefill_e4m3_grouped(const uint8_t* qx, const float* sxT, int
                                         const float* swT, int E, int N, int K, int rows_total, const MoeTile* tiles,
                                         const int* n_tiles, int max_tiles, const int32_t* perm, float* y,
                                         cudaStream_t s);
-// The experts' bf16 down projection on the grouped tensor-core GEMM (a mode of the A16 kernel):
-// act holds each pair's activation as three bf16 planes [rows_total][3 I] in permuted order, wd the
-// stacked bf16 weights [E * N][I]; tiles of kPrefillA16Tokens permuted rows x 128 weight rows from
-// the permute; row r of a tile is added into y[perm[r] / topk][0 .. N) scaled by wts[perm[r]].
-constexpr int kFmtDownA16 = 17;
-cudaError_t launch_prefill_down_grouped(const __nv_bfloat16* act, const uint16_t* wd, int E, int N, int I,
-                                        int rows_total, const MoeTile* tiles, const int* n_tiles, int max_tiles,
-                                        const int32_t* perm, int topk, const float* wts, float* y, cudaStream_t s);
+// The experts' bf16 down projection on the grouped tensor-core GEMM (k_down.cu): act holds each
+// pair's activation as three bf16 planes [rows_total][3 I] in permuted order, wd the stacked bf16
+// weights [E * N][I]; tiles of at most kDownTileRows permuted rows x 128 weight rows from the
+// permute; row r of a tile is added into out[perm[r] / topk][0 .. N) scaled by wts[perm[r]], the
+// whole 3 I accumulated in tensor memory.
+constexpr int kDownTileRows = 160;
+cudaError_t launch_down_grouped(const __nv_bfloat16* act, const uint16_t* wd, int E, int N, int I, int rows_total,
+                                const MoeTile* tiles, const int* n_tiles, int max_tiles, const int32_t* perm,
+                                int topk, const float* wts, float* out, cudaStream_t s);
 // From this many (token, slot) pairs per expert on average, moe_gate_up runs the grouped tensor-core GEMM.
 constexpr int kMoePrefillMinRowsPerExpert = 8;
 cudaError_t launch_moe_permute(const int32_t* ids, int T, int topk, int E, int32_t* counts, int32_t* offsets,

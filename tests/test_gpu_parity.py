@@ -314,12 +314,13 @@ def test_moe_gate_up_grouped_parity(fmt, T, E, topk, N, K):
 
 @pytest.mark.parametrize("T,E,topk,K,I", [(1, 8, 2, 96, 64), (4, 16, 4, 130, 128), (16, 32, 8, 64, 192),
                                           (20, 32, 8, 200, 64), (300, 16, 8, 48, 128), (400, 8, 2, 200, 192),
-                                          (500, 64, 8, 256, 64)])
+                                          (500, 64, 8, 256, 64), (600, 4, 2, 136, 128)])
 def test_moe_down_combine_parity(T, E, topk, K, I):
     # T * topk <= 128: the weight-streaming kernel ranks the ids itself; 160 pairs: the permute
     # kernel's chunks; from 8 pairs per expert on (2400, 800 and 4000 pairs) the grouped bf16
-    # tensor-core GEMM over 192-row tiles.  K = 130, 200: ragged 16-row slabs and a ragged
-    # 128-row weight block; I = 192: three 64-wide steps per plane.
+    # tensor-core GEMM over tiles of up to 160 rows (600 x top-2 over 4 experts: two row tiles per
+    # expert, the second short).  K = 130, 136, 200: ragged 16-row slabs and ragged 128-row weight
+    # blocks; I = 192: three 64-wide steps per plane.
     d = synth.moe_down(T, seed=3, E=E, topk=topk, K=K, I=I)
     wd = np.stack([d["Wd"][e] for e in range(E)])
     ref = O.moe_down_combine(d["h"], d["ids"], d["weights"], wd, E)
