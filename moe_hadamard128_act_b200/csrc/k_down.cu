@@ -11,19 +11,20 @@
 //
 // A tile is 128 weight rows of one expert (the MMA's M, tensor-memory lanes)
 // by up to 160 of its pairs (the MMA's N: the tile's row count rounded up to
-// 16, so a short tile costs only its own rows).  A step is 64 of the 3 I: the
-// weight box [128 rows][128 B] and as many activation boxes [32 rows][128 B]
-// as the tile's rows need land in a 6-slot ring, and four MMAs (kind::f16,
-// bf16 x bf16, K = 16, both operands from shared memory) accumulate into the
-// tile's fp32 accumulator.  No scale changes along K, so the accumulator
-// holds the whole sum and is read once per tile; two of them let the
-// epilogue of one tile run under the MMAs of the next.
+// 16, so a short tile costs only its own rows).  A weight step is 64 of the
+// I: its weight box [128 rows][128 B] lands in a 3-slot ring and serves the
+// three planes, whose activation boxes land in an 8-slot ring; each plane
+// takes four MMAs (kind::f16, bf16 x bf16, K = 16, both operands from shared
+// memory) into the tile's fp32 accumulator.  No scale changes along K, so the
+// accumulator holds the whole sum and is read once per tile; two of them let
+// the epilogue of one tile run under the MMAs of the next.
 //
-// The step rate is set by how many bytes are in flight, not by the tensor
-// pipe: a copy takes a few thousand cycles to land under load, so the ring
-// must hold several steps' operands (up to 36 KB each).  The 160-row cap
-// (an expert's pairs at 2048 tokens x top-8 over 128 experts number about
-// 128) is what leaves room for six slots.
+// The kernel is bound by the operand stream from L2 into shared memory, not
+// by the tensor pipe, so it moves as few and as large boxes as it can: each
+// weight box once for its three planes, and a tile's activation rows in one
+// 128-row box plus 32-row boxes for what is left.  The 160-row cap (an
+// expert's pairs at 2048 tokens x top-8 over 128 experts number about 128)
+// keeps the activation slots small enough for eight of them.
 //
 // Warp roles: lane 0 of warp 0 issues the TMA loads, lane 0 of warp 1 the
 // MMAs, warp 2 owns the tensor-memory allocation.  Warps 4..11 are the
@@ -51,8 +52,8 @@ constexpr int XBOX = 32;                 // activation rows per small TMA box
 constexpr int XBIG = 128;                // activation rows per large TMA box
 constexpr int A_BYTES = DM * 128;        // weight box, 16 KB
 constexpr int B_BYTES = DN * 128;        // activation boxes, up to 20 KB
-constexpr int STAGE = A_BYTES + B_BYTES;
-constexpr int DS = 6;                    // ring slots
+constexpr int WS = 3;                    // weight ring slots
+constexpr int XS = 8;                    // activation ring slots
 constexpr int NACC = 2;                  // accumulators [128 x DN]
 constexpr uint32_t kTmemCols = 512;
 constexpr int kEpiWarp0 = 4, kEpiWarps = 8;
@@ -61,15 +62,16 @@ constexpr int HALF = DN / 2;             // pairs per epilogue warp
 constexpr int CW = 16;                   // columns per tensor-memory read
 static_assert(NACC * ACC_COLS <= (int)kTmemCols && DN % 32 == 0 && DN <= ACC_COLS, "tile width");
 static_assert(DN >= XBIG && (DN - XBIG) % XBOX == 0, "a large box and small ones cover any tile");
-static_assert(STAGE % 1024 == 0 && A_BYTES % 1024 == 0 && (XBOX * 128) % 1024 == 0,
+static_assert(B_BYTES % 1024 == 0 && A_BYTES % 1024 == 0 && (XBOX * 128) % 1024 == 0,
               "operand boxes stay 1024-byte aligned for the 128-byte swizzle");
 constexpr int NBAT = (HALF + 31) / 32;  // 32-pair batches per epilogue warp
 static_assert(HALF % CW == 0, "whole tensor-memory reads per warp");
 
-// Shared memory (from a 1024-aligned base): [ring][mbarriers][tmem address]
-constexpr int BAR_OFF = DS * STAGE;
-constexpr int B_FULL = 0, B_EMPTY = DS, B_ACCF = 2 * DS, B_ACCE = B_ACCF + NACC, B_DRAIN = B_ACCE + NACC,
-              NBARS = B_DRAIN + 1;
+// Shared memory (from a 1024-aligned base): [weight ring][activation ring][mbarriers][tmem address]
+constexpr int X_OFF = WS * A_BYTES;
+constexpr int BAR_OFF = X_OFF + XS * B_BYTES;
+constexpr int B_WFULL = 0, B_WEMPTY = WS, B_XFULL = 2 * WS, B_XEMPTY = B_XFULL + XS, B_ACCF = B_XEMPTY + XS,
+              B_ACCE = B_ACCF + NACC, B_DRAIN = B_ACCE + NACC, NBARS = B_DRAIN + 1;
 constexpr int MISC_OFF = (BAR_OFF + 8 * NBARS + 15) / 16 * 16;
 constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
@@ -122,7 +124,7 @@ struct DownArgs {
     const float* wts;      // routing weight of each pair
     float* out;            // [T][N], zeroed before
     unsigned* err;
-    int N, G, GW, topk;    // G = 3 I / 64 steps per tile, GW = I / 64 weight steps
+    int N, GW, topk;       // GW = I / 64 weight steps per tile
 };
 
 __global__ void __launch_bounds__(kThreads, 1) k_down_grouped(const __grid_constant__ DownArgs a) {
@@ -134,12 +136,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_grouped(const __grid_const
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gb + MISC_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles = *a.n_tiles;
-    const int G = a.G;
+    const int GW = a.GW;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DS; ++s) {
-            mbar_init(bar(B_FULL + s), 1);   // expect_tx
-            mbar_init(bar(B_EMPTY + s), 1);  // the step's MMA commit
+        for (int s = 0; s < WS; ++s) {
+            mbar_init(bar(B_WFULL + s), 1);   // expect_tx
+            mbar_init(bar(B_WEMPTY + s), 1);  // the MMA commit after the weight step's last plane
+        }
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(bar(B_XFULL + s), 1);   // expect_tx
+            mbar_init(bar(B_XEMPTY + s), 1);  // the plane's MMA commit
         }
         for (int b = 0; b < NACC; ++b) {
             mbar_init(bar(B_ACCF + b), 1);          // the tile's last commit
@@ -164,34 +170,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_grouped(const __grid_const
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmW) : "memory");
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmX) : "memory");
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmXb) : "memory");
-        int step = 0;
+        int wstep = 0, xstep = 0;
         for (int t = blockIdx.x; t < tiles && !dead; t += gridDim.x) {
             const MoeTile ti = a.tiles[t];
             // The tile's rows come in one 128-row box (from 96 rows on: large boxes stream faster than
             // small ones, worth the rows fetched past the tile) and 32-row boxes for the rest.
             const int big = ti.rows >= 96 ? 1 : 0;
             const int nb = (max(ti.rows - big * XBIG, 0) + XBOX - 1) / XBOX;
+            const unsigned xbytes = (big * XBIG + nb * XBOX) * 128;
             const int wrow = ti.expert * a.N + ti.wb * DM;
-            for (int g = 0; g < G; ++g, ++step) {
-                const int s = step % DS;
-                if (!mbar_wait(bar(B_EMPTY + s), ((step / DS) & 1) ^ 1, lim)) {
+            for (int w = 0; w < GW && !dead; ++w, ++wstep) {
+                const int ws = wstep % WS;
+                if (!mbar_wait(bar(B_WEMPTY + ws), ((wstep / WS) & 1) ^ 1, lim)) {
                     dead = true;
                     break;
                 }
-                const uint32_t fb = bar(B_FULL + s), dst = base + s * STAGE;
-                mbar_expect_tx(fb, A_BYTES + (big * XBIG + nb * XBOX) * 128);
-                tma_load_2d(dst, &a.tmW, (g % a.GW) * 128, wrow, fb);
-                if (big) tma_load_2d(dst + A_BYTES, &a.tmXb, g * 128, ti.row0, fb);
-                for (int b = 0; b < nb; ++b)
-                    tma_load_2d(dst + A_BYTES + (big * XBIG + b * XBOX) * 128, &a.tmX, g * 128,
-                                ti.row0 + big * XBIG + b * XBOX, fb);
+                mbar_expect_tx(bar(B_WFULL + ws), A_BYTES);
+                tma_load_2d(base + ws * A_BYTES, &a.tmW, w * 128, wrow, bar(B_WFULL + ws));
+                for (int pl = 0; pl < 3; ++pl, ++xstep) {  // plane pl: columns pl * I + 64 w
+                    const int xs = xstep % XS;
+                    if (!mbar_wait(bar(B_XEMPTY + xs), ((xstep / XS) & 1) ^ 1, lim)) {
+                        dead = true;
+                        break;
+                    }
+                    const uint32_t fb = bar(B_XFULL + xs), dst = base + X_OFF + xs * B_BYTES;
+                    const int x = (pl * GW + w) * 128;
+                    mbar_expect_tx(fb, xbytes);
+                    if (big) tma_load_2d(dst, &a.tmXb, x, ti.row0, fb);
+                    for (int b = 0; b < nb; ++b)
+                        tma_load_2d(dst + (big * XBIG + b * XBOX) * 128, &a.tmX, x, ti.row0 + big * XBIG + b * XBOX,
+                                    fb);
+                }
             }
         }
         // Copies still in flight must land before the CTA's shared memory is released.
-        for (int j = step > DS ? step - DS : 0; j < step; ++j)
-            if (!mbar_wait(bar(B_FULL + j % DS), (j / DS) & 1)) break;
+        for (int j = wstep > WS ? wstep - WS : 0; j < wstep; ++j)
+            if (!mbar_wait(bar(B_WFULL + j % WS), (j / WS) & 1)) break;
+        for (int j = xstep > XS ? xstep - XS : 0; j < xstep; ++j)
+            if (!mbar_wait(bar(B_XFULL + j % XS), (j / XS) & 1)) break;
     } else if (warp == 1 && lane == 0) {  // ---- MMA issuer ----
-        int step = 0, tl = 0;
+        int wstep = 0, xstep = 0, tl = 0;
         for (int t = blockIdx.x; t < tiles && !dead; t += gridDim.x, ++tl) {
             const MoeTile ti = a.tiles[t];
             const int b = tl % NACC;
@@ -201,18 +219,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_grouped(const __grid_const
             }
             fence_after();
             const uint32_t idesc = idesc_bf16((ti.rows + 15) & ~15), d = tmem + b * ACC_COLS;
-            for (int g = 0; g < G; ++g, ++step) {
-                const int s = step % DS;
-                if (!mbar_wait(bar(B_FULL + s), (step / DS) & 1, lim)) {
+            for (int w = 0; w < GW && !dead; ++w, ++wstep) {
+                const int ws = wstep % WS;
+                if (!mbar_wait(bar(B_WFULL + ws), (wstep / WS) & 1, lim)) {
                     dead = true;
                     break;
                 }
-                fence_after();
-                const uint64_t ad = desc_sw128(base + s * STAGE), bd = desc_sw128(base + s * STAGE + A_BYTES);
+                const uint64_t ad = desc_sw128(base + ws * A_BYTES);
+                for (int pl = 0; pl < 3; ++pl, ++xstep) {
+                    const int xs = xstep % XS;
+                    if (!mbar_wait(bar(B_XFULL + xs), (xstep / XS) & 1, lim)) {
+                        dead = true;
+                        break;
+                    }
+                    fence_after();
+                    const uint64_t bd = desc_sw128(base + X_OFF + xs * B_BYTES);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)  // K = 16 bf16 = 32 bytes: +2 in the descriptor's address field
-                    mma_ss(d, ad + 2 * j, bd + 2 * j, idesc, (g | j) ? 1u : 0u);
-                commit(bar(B_EMPTY + s));  // the slot may be refilled once these MMAs are done
+                    for (int j = 0; j < 4; ++j)  // K = 16 bf16 = 32 bytes: +2 in the descriptor's address field
+                        mma_ss(d, ad + 2 * j, bd + 2 * j, idesc, (w | pl | j) ? 1u : 0u);
+                    commit(bar(B_XEMPTY + xs));  // the activation slot may be refilled once these are done
+                }
+                commit(bar(B_WEMPTY + ws));  // and the weight slot after its three planes
             }
             if (dead) break;
             commit(bar(B_ACCF + b));  // the tile's sums are complete
@@ -304,7 +331,6 @@ cudaError_t launch_down_grouped(const __nv_bfloat16* act, const uint16_t* wd, in
     a.out = out;
     a.err = di.err_word;
     a.N = N;
-    a.G = 3 * I / 64;
     a.GW = I / 64;
     a.topk = topk;
     static bool attr_set[64] = {};
