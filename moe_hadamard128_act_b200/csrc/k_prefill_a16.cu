@@ -14,6 +14,10 @@
 //  * the activations are the f16 copy of x scaled per token by a power of two
 //    (prepared by the activation prologue), loaded by TMA into shared memory
 //    as the B operand.
+// A grouped tile holds one expert's rows, about 128 of 192 when 2048 tokens are
+// routed top-8 over 128 experts: its MMAs are as wide as its rows (rounded up
+// to 16), a tile of at most 128 rows loads 128-row activation boxes, and the
+// epilogue reads only the columns of its rows.
 // One step is one 128-K group: eight MMAs with K = 16 into one of the fp32
 // accumulators [128 weight rows x TN tokens] (two at TN = 192, three at
 // TN = 128, as tensor memory allows next to two A tiles).  The epilogue thread that owns
@@ -102,16 +106,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     // K-major, 128-byte swizzle: 8-row atoms 1024 bytes apart (SBO), version 1.
     return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
-// kind::f16: D f32, A f16, B f16, both K-major, N = TN, M = 128.
-constexpr uint32_t kIdescF16 = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(TN >> 3) << 17) |
-                               ((uint32_t)(TM >> 4) << 24);
+// kind::f16: D f32, A f16, B f16, both K-major, M = 128, N = n (a multiple of 16, at most TN).
+__device__ __forceinline__ uint32_t idesc_f16(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
+}
 
 // D (+)= A * B^T with A in tensor memory; acc_in = 0 overwrites D.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t acc_in) {
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t acc_in) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
-        "r"(a_tmem), "l"(bdesc), "r"(kIdescF16), "r"(acc_in));
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc_in));
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
@@ -149,6 +155,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 struct A16Args {
     CUtensorMap tmW;       // codes [E * N][K] bytes (E = 1 when dense), box [128 rows][128 B]
     CUtensorMap tmX;       // f16 activations [M][K] as bytes, box [TN rows][128 B]
+    CUtensorMap tmXb;      // the same, box [128 rows][128 B]
     const uint16_t* sw;    // scales per expert: [N][G] (int8 formats) or [ceil(N/128)][G] (fp8), bf16 or f16 bits
     const float* xf;       // inverse token factors: [M] (dense) or [T] (grouped, token of pair p = p / topk)
     float* y;              // dense: [M][ldy]; grouped: [T * topk][ldy = N]
@@ -256,19 +263,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 if (!mbar_wait(bar(B_CFULL + j % CS), (j / CS) & 1)) break;
         } else if (warp == 3 && lane == 0) {  // ---- producer of the activation tiles ----
             asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmX) : "memory");
+            asm volatile("prefetch.tensormap [%0];\n" ::"l"(&a.tmXb) : "memory");
             int g = 0, t = blockIdx.x, k = 0;
-            int m0 = 0;  // first activation row of the tile
+            int m0 = 0, rows = 0;  // first activation row of the tile, its rows
             for (; k < total; ++k) {
-                if (g == 0) m0 = tile_at<GRP>(a, t, TB).row0;
+                if (g == 0) {
+                    const MoeTile ti = tile_at<GRP>(a, t, TB);
+                    m0 = ti.row0;
+                    rows = ti.rows;
+                }
                 const int x = k % XS;
                 if (k >= XS && !mbar_wait(bar(B_STEP + (k - XS) % SR), ((k - XS) / SR) & 1, lim)) {
                     dead = true;  // the slot's previous activations are still in use
                     break;
                 }
                 const uint32_t xb = bar(B_XFULL + x), xd = base + X_OFF + x * X_BYTES;
-                mbar_expect_tx(xb, X_BYTES);
-                tma_load_2d(xd, &a.tmX, g * GK * 2, m0, xb);
-                tma_load_2d(xd + XATOM, &a.tmX, g * GK * 2 + 128, m0, xb);
+                // A grouped tile of at most 128 rows loads 128-row boxes, a wider one the TN-row boxes.
+                const bool narrow = GRP && rows <= 128;
+                const CUtensorMap* const tm = narrow ? &a.tmXb : &a.tmX;
+                mbar_expect_tx(xb, narrow ? 2 * 128 * 128 : X_BYTES);
+                tma_load_2d(xd, tm, g * GK * 2, m0, xb);
+                tma_load_2d(xd + XATOM, tm, g * GK * 2 + 128, m0, xb);
                 if (++g == G) {
                     g = 0;
                     t += gridDim.x;
@@ -278,8 +293,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 if (!mbar_wait(bar(B_XFULL + j % XS), (j / XS) & 1)) break;
         } else if ((warp == 1 || warp == 2) && lane == 0) {  // ---- MMA issuers: even / odd steps ----
             const uint64_t xd0 = smem_desc_sw128(base + X_OFF);
+            // The step's tile (its position tcur among this CTA's tiles, and gk, the step within
+            // it) advances by two steps per iteration without a division.
+            int tcur = 0, gk = warp - 1;
+            while (gk >= G) gk -= G, ++tcur;
+            int tload = -1;               // tile position whose width idesc holds
+            uint32_t idesc = idesc_f16(TN);  // the MMA's N: the tile's rows rounded up to 16 (grouped)
             for (int k = warp - 1; k < total; k += 2) {
                 const int x = k % XS, ab = k % AS, db = k % NACC;
+                if constexpr (GRP) {
+                    if (tcur != tload) {
+                        tload = tcur;
+                        idesc = idesc_f16((tile_at<GRP>(a, (int)blockIdx.x + tcur * (int)gridDim.x, TB).rows + 15) & ~15);
+                    }
+                    gk += 2;
+                    while (gk >= G) gk -= G, ++tcur;
+                }
                 if (!mbar_wait(bar(B_XFULL + x), (k / XS) & 1, lim) || !mbar_wait(bar(B_AFULL + ab), (k / AS) & 1, lim) ||
                     !mbar_wait(bar(B_DEMPTY + db), ((k / NACC) & 1) ^ 1, lim)) {
                     dead = true;
@@ -290,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
                 const uint64_t xo = (uint64_t)((x * X_BYTES) >> 4);
 #pragma unroll
                 for (int j = 0; j < GK / 16; ++j)
-                    mma_f16_ts(d, at + 8 * j, xd0 + xo + (uint64_t)((j / 4) * (XATOM >> 4) + (j % 4) * 2),
+                    mma_f16_ts(d, at + 8 * j, xd0 + xo + (uint64_t)((j / 4) * (XATOM >> 4) + (j % 4) * 2), idesc,
                                j ? 1u : 0u);
                 // One commit per step: its accumulator is ready for the epilogue, and its
                 // A tile and activation slot may be refilled.  A waiter for step j checks
@@ -392,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
             const uint32_t dt = tmem + tl + db * TN + cg * EPC;
 #pragma unroll
             for (int h = 0; h < EPC / CW; ++h) {
+                if (GRP && h * CW >= rows) break;  // columns past the tile's rows were not computed (warp-uniform)
                 uint32_t v[CW];
                 QL_TMEM_LD16(dt + h * CW, v);
                 QL_TMEM_WAIT16(v);
@@ -473,7 +503,8 @@ cudaError_t launch_prefill_a16(int fmt, const __half* xs, const float* xf, const
     if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
     A16Args a{};
     if ((e = make_tmap_2d(codes, N, K, K, GK, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d(xs, M, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) != cudaSuccess)
+    if ((e = make_tmap_2d(xs, M, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) != cudaSuccess ||
+        (e = make_tmap_2d(xs, M, 2LL * K, 2LL * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmXb)) != cudaSuccess)
         return e;
     a.sw = static_cast<const uint16_t*>(scales);
     a.xf = xf;
@@ -501,7 +532,9 @@ cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* x
     if ((e = make_tmap_2d(codes, (long long)E * N, K, K, GK, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) != cudaSuccess)
         return e;
     if ((e = make_tmap_2d(xs, rows_total, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) !=
-        cudaSuccess)
+            cudaSuccess ||
+        (e = make_tmap_2d(xs, rows_total, 2LL * K, 2LL * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmXb)) !=
+            cudaSuccess)
         return e;
     a.sw = static_cast<const uint16_t*>(scales);
     a.xf = xf;
