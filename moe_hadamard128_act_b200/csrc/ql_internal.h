@@ -148,8 +148,10 @@ struct MoeChunk {
     int expert, start, count;  // rows perm[start .. start+count) of the permuted order
 };
 size_t moe_max_chunks(int T, int topk, int E);
-// One tile of the grouped expert GEMM: `rows` permuted rows from `row0` (all
-// of one expert) against weight rows wb * 128 .. + 127 of that expert.
+// One tile of a grouped expert GEMM: `rows` permuted rows from `row0` (all
+// of one expert) against weight block wb of that expert (blocks of the GEMM's
+// height: 128 rows for the A16 and down-projection kernels, 192 for the E4M3
+// one).
 struct MoeTile {
     int expert, row0, rows, wb;
 };
