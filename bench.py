@@ -306,7 +306,10 @@ def run_extras(torch, Q, synth, dev, stream, hbm, sections=None):
                     c, s, zz = Q.qlinear_pack(fmt, N_FULL, K_FULL, W=Wd)
                 cp = [(c, s, zz)] + [(c.clone(), s.clone(), None if zz is None else zz.clone()) for _ in range(3)]
                 res = {}
-                for m in (1, 5, 16) if fmt == Q.I4_G64_BF16 else (1, 4, 16):
+                # above 16 rows int4 (and int5 up to 64) has no tensor-core prefill path: the decode
+                # kernel runs once per 16 rows, streaming the weight again each time
+                ms = {Q.I4_G64_BF16: (1, 5, 16, 64, 256), Q.I5Z_G128_F16: (1, 4, 16, 64)}.get(fmt, (1, 4, 16))
+                for m in ms:
                     x = bf(synth.activations(0, f"x_M{m}", m, K_FULL))
                     y = torch.empty((m, N_FULL), dtype=torch.float32, device=dev)
                     ws = torch.empty(Q.qlinear_workspace_size(fmt, 0, m, N_FULL, K_FULL), dtype=torch.uint8, device=dev)
@@ -320,6 +323,8 @@ def run_extras(torch, Q, synth, dev, stream, hbm, sections=None):
                     byts = cb + sb + zb + m * K_FULL * 2 + m * N_FULL * 4
                     res[str(m)] = {"us": us, "GB/s": byts / (us * 1e-6) / 1e9, "frac": byts / (us * 1e-6) / 1e9 / hbm,
                                    "us_gemm": 1e3 * t, "launches_per_call": per}
+                    if m > 16:
+                        res[str(m)]["TFLOPS"] = 2.0 * m * N_FULL * K_FULL / (us * 1e-6) / 1e12
                 out[name] = res
                 del cp, c, s, zz
             del Wd
