@@ -132,11 +132,9 @@ __device__ __forceinline__ void fold_chains(T (&acc)[CH][NT][4]) {
 // The per-group MMAs of one unit for the weight-only formats.
 // getx(nt, piece) returns the lane's 16-byte activation piece for n-tile nt.
 // yacc[nt][i] accumulates scale * partial; i = 0,1 row g, i = 2,3 row g + 8.
-// CH independent accumulation chains per group (see fold_chains): two by default
-// with a single n-tile; the MoE kernel asks for two at NT = 2 as well, since its
-// chunks mostly hold fewer than 9 rows and leave the second n-tile idle.
-template <int FMT, int NT, int CH = (NT == 1 ? 2 : 1), typename GetX>
+template <int FMT, int NT, typename GetX>
 __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1_live, float (&yacc)[NT][4]) {
+    constexpr int CH = NT == 1 ? 2 : 1;  // independent accumulation chains per group (see fold_chains)
     if constexpr (FMT == QL_I4_G64_BF16) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -332,10 +330,10 @@ __device__ __forceinline__ void unit_w8a8(const Regs<QL_I8A8_G128_BF16>& r, GetX
         for (int i = 0; i < 4; ++i) out[nt][i] = acc[0][nt][i];
 }
 
-// Format 7: fp32 sums of one group's E4M3 products, the same walk as unit_w8a8
-// (CH chains as for unit_a16).
-template <int NT, int CH = (NT == 1 ? 2 : 1), typename GetX>
+// Format 7: fp32 sums of one group's E4M3 products, the same walk as unit_w8a8.
+template <int NT, typename GetX>
 __device__ __forceinline__ void unit_e4m3(const Regs<QL_FP8A8_B128_BF16>& r, GetX getx, float (&out)[NT][4]) {
+    constexpr int CH = NT == 1 ? 2 : 1;
     float acc[CH][NT][4];
 #pragma unroll
     for (int ch = 0; ch < CH; ++ch)
@@ -379,13 +377,9 @@ __device__ __forceinline__ void mma_bf16(float d[4], uint32_t a0, uint32_t a1, u
 // operands as they are; the activation is three bf16 planes whose sum is the
 // fp32 value, so the three products summed in fp32 carry its full precision.
 // getx(nt, piece, plane) returns the lane's 16-byte piece (chunk c, or 4 + c)
-// of a plane.  No scale: the sums go into yacc, the odd k-steps through a
-// second chain (acc2) so that the twelve MMAs are not one dependent chain.
+// of a plane.  No scale: the sums go straight into yacc.
 template <int NT, typename GetX>
 __device__ __forceinline__ void unit_down(const Regs<kFmtDown>& r, GetX getx, bool nt1_live, float (&yacc)[NT][4]) {
-    float acc2[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc2[nt][0] = acc2[nt][1] = acc2[nt][2] = acc2[nt][3] = 0.0f;
 #pragma unroll
     for (int piece = 0; piece < 2; ++piece) {
 #pragma unroll
@@ -402,16 +396,11 @@ __device__ __forceinline__ void unit_down(const Regs<kFmtDown>& r, GetX getx, bo
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (nt == 1 && !nt1_live) continue;
-                    mma_bf16(s2 == 0 ? yacc[nt] : acc2[nt], a0, a1, a2, a3, s2 == 0 ? xv[nt].x : xv[nt].z,
-                             s2 == 0 ? xv[nt].y : xv[nt].w);
+                    mma_bf16(yacc[nt], a0, a1, a2, a3, s2 == 0 ? xv[nt].x : xv[nt].z, s2 == 0 ? xv[nt].y : xv[nt].w);
                 }
             }
         }
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) yacc[nt][i] += acc2[nt][i];
 }
 
 // ---------------------------------------------------------------------------
@@ -1108,7 +1097,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 // fp32 sums of the group's E4M3 products, then both scales: the block's weight
                 // scale and the scale of the column's token for this group.
                 float acc[NT][4];
-                unit_e4m3<NT, 2>(r, getx, acc);
+                unit_e4m3<NT>(r, getx, acc);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -1118,7 +1107,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                         yacc[nt][2 + i] = fmaf(r.s[1] * sx, acc[nt][2 + i], yacc[nt][2 + i]);
                     }
             } else {
-                unit_a16<FMT, NT, 2>(r, getx, chc.count > 8, yacc);
+                unit_a16<FMT, NT>(r, getx, chc.count > 8, yacc);
             }
             __syncwarp();
             if (issued < u1) issue(st);  // refill this slot with the unit kMoeStages ahead
