@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--extras", default=None,
                    help="comma-separated extras sections to run (decode, moe_decode, moe_prefill, moe_fp8a8_down, "
                         "prefill); default all")
+    p.add_argument("--extras-only", action="store_true",
+                   help="run only the extras and print them as one JSON line (the main run starts this as a "
+                        "child process, so a fault in a secondary workload cannot take the headline line with it)")
     p.add_argument("--ncu-case", choices=["skinny_w8a8", "prefill_w8a8", "prefill_fp8", "prefill_fp8a8", "prefill_w5a8",
                                           "moe_decode", "moe_decode_t1", "moe_prefill", "act_quant", "decode_w4a16",
                                           "decode_w5a16", "decode_w8a16", "decode_fp8", "moe_down"],
@@ -701,6 +704,50 @@ def ncu_case(name):
 # --------------------------------------------------------------------------
 # GPU arm
 # --------------------------------------------------------------------------
+def run_extras_child(args):
+    """Runs `bench.py --extras-only` as a child process and returns its extras dict, or
+    {"error": ...} when the child fails (its stderr, with the section markers, passes through)."""
+    import subprocess
+    cmd = [sys.executable, str(Path(__file__).resolve()), "--extras-only"]
+    if args.extras is not None:
+        cmd += ["--extras", args.extras]
+    try:
+        r = subprocess.run(cmd, stdout=subprocess.PIPE, stderr=None, text=True, timeout=1800)
+    except subprocess.TimeoutExpired:
+        return {"error": "extras child process timed out"}
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    if r.returncode != 0 or not lines:
+        print(f"[bench] extras failed: child exit code {r.returncode}", file=sys.stderr, flush=True)
+        return {"error": f"extras child process exited with code {r.returncode}"}
+    return json.loads(lines[-1])
+
+
+def extras_only(args):
+    """The secondary workloads alone (one GPU), printed as one JSON line."""
+    import torch
+
+    from moe_hadamard128_act_b200 import build as qbuild
+    from moe_hadamard128_act_b200 import qlinear as Q
+    from moe_hadamard128_act_b200 import synth
+
+    torch.cuda.set_device(0)
+    qbuild.build()
+    Q.lib()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    hbm = peaks()[0]
+    sections = None if args.extras is None else set(args.extras.split(","))
+    try:
+        extras = run_extras(torch, Q, synth, dev, stream, hbm, sections)
+    except Exception as ex:  # report what failed; the parent keeps its headline line either way
+        extras = {"error": f"{type(ex).__name__}: {ex}"}
+        print(f"[bench] extras failed: {extras['error']}", file=sys.stderr, flush=True)
+    st, bits = Q.ql_get_device_error(stream)
+    if st != 0 or bits:
+        extras["device_error"] = {"status": st, "bits": bits}
+    print(json.dumps(extras), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", 0))
@@ -710,6 +757,8 @@ def main():
         return run_reference(args, rank, world)
     if args.ncu_case:
         return ncu_case(args.ncu_case)
+    if args.extras_only:
+        return extras_only(args)
 
     import torch
     import torch.distributed as dist
@@ -936,21 +985,19 @@ def main():
     e2e = {"value": replicas_value(e2e_ms, world, e2e_steps, step_bytes()), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
-    extras = None
-    if not args.no_extras:
-        del copies, codes0, scales0
-        torch.cuda.empty_cache()
-        try:
-            sections = None if args.extras is None else set(args.extras.split(","))
-            extras = run_extras(torch, Q, synth, dev, stream, hbm, sections)
-        except Exception as ex:  # report, keep the headline line
-            extras = {"error": f"{type(ex).__name__}: {ex}"}
-            print(f"[bench] extras failed: {extras['error']}", file=sys.stderr, flush=True)
-
     st, bits = Q.ql_get_device_error(stream)
     if st != 0:
         raise RuntimeError(f"ql_get_device_error: status {st} ({Q.STATUS.get(st, st)}), bits {bits}, "
                            f"last CUDA error: {Q.lib().ql_last_cuda_error().decode()}")
+
+    extras = None
+    if not args.no_extras and world == 1:
+        # The secondary workloads run in a child process with its own CUDA context, after this
+        # one has released its buffers: whatever happens there, the headline line below stands.
+        del copies, codes0, scales0
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        extras = run_extras_child(args)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -110,7 +110,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // normal range); below that the rounding error is under 2^-39 of the row's
 // max, far beneath the fp32 accumulation error of the GEMM.
 // With inv != null the row is written to rows inv[t * topk + j] (j < topk,
-// negative entries skipped) instead of row t: the permuted order of the
+// negative entries skipped, entries at or past xs_rows flagged as
+// QL_DEVERR_BOUNDS and skipped) instead of row t: the permuted order of the
 // grouped expert GEMM.
 // Slots SL .. 31 of one int5 lane run starting at element b: the f16 activation
 // of the slot's code (i5_slot_code), divided by 2^o (i5_slot_off), to its
@@ -128,7 +129,7 @@ __device__ __forceinline__ void i5_stage_run(const float* r, float f, __half* ou
 
 __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M, int K, int rotate, int order,
                                                   __half* xs, float* xf, float* yz, long long nz, const int32_t* inv,
-                                                  int topk, float* xsum) {
+                                                  int topk, float* xsum, int xs_rows, unsigned* err) {
     extern __shared__ float row[];  // [K] fp32, then (natural order) [K] f16
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // let the GEMM start its weight stream
     zero_fill(yz, nz);  // the GEMM that follows accumulates into y (CTAs past M only help with this)
@@ -185,7 +186,11 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
         for (int idx = threadIdx.x; idx < nrep * K8; idx += 256) {
             const int j = idx / K8, c = idx - j * K8;
             const long long orow = inv ? (long long)__ldg(inv + (long long)t * topk + j) : (long long)t;
-            if (orow >= 0) reinterpret_cast<uint4*>(xs + orow * K)[c] = hrow[c];
+            if (orow >= xs_rows) {  // a permuted row outside xs (the permutation is device data): flag, skip
+                if (c == 0) atomicOr(err, (unsigned)QL_DEVERR_BOUNDS);
+            } else if (orow >= 0) {
+                reinterpret_cast<uint4*>(xs + orow * K)[c] = hrow[c];
+            }
         }
         return;
     }
@@ -350,7 +355,7 @@ cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, 
     const long long zc = zb < 2LL * di.sm_count ? zb : 2LL * di.sm_count;
     const int grid = (int)(M > zc ? M : zc);
     k_prep_a16<<<grid, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), M, K, rotate, order, xs, xf, yz, nz,
-                                       nullptr, 1, xsum);
+                                       nullptr, 1, xsum, M, di.err_word);
     return cudaGetLastError();
 }
 
@@ -363,8 +368,10 @@ cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, con
         e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
+    DeviceInfo di;
+    if ((e = device_info(&di)) != cudaSuccess) return e;
     k_prep_a16<<<T, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), T, K, rotate, XORD_NATURAL, xs, xf, nullptr, 0,
-                                    inv, topk, nullptr);
+                                    inv, topk, nullptr, T * topk, di.err_word);
     return cudaGetLastError();
 }
 

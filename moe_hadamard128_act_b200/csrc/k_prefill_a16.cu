@@ -166,6 +166,7 @@ struct A16Args {
     const int* n_tiles;
     const int32_t* perm;   // grouped: permuted row -> pair index t * topk + j
     int topk;
+    int E, max_tiles;      // grouped: experts, the tile table's capacity (bounds of its entries)
 };
 
 // The tile a CTA works on: expert, first activation row, rows, weight block.
@@ -203,7 +204,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_a16(const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int WB = (a.N + TM - 1) / TM, TB = (a.M + TN - 1) / TN;
     // dense: weight-block-major, t -> (wb = t / TB, tb = t % TB); grouped: the permute's table
-    const int tiles = GRP ? *a.n_tiles : WB * TB;
+    int tiles = GRP ? *a.n_tiles : WB * TB;
+    if (GRP) {
+        // The tile table comes from the permute kernel on the device: a CTA runs only if the
+        // count and every one of its tiles lie inside the buffers (else it flags and skips).
+        bool bad = tiles < 0 || tiles > a.max_tiles;
+        for (int t = blockIdx.x; !bad && t < tiles; t += gridDim.x) {
+            const MoeTile ti = a.tiles[t];
+            bad = ti.expert < 0 || ti.expert >= a.E || ti.rows < 1 || ti.rows > TN || ti.row0 < 0 ||
+                  ti.row0 + ti.rows > a.M || ti.wb < 0 || ti.wb >= WB;
+        }
+        if (bad) {
+            if (threadIdx.x == 0) atomicOr(a.err, (unsigned)QL_DEVERR_BOUNDS);
+            tiles = 0;
+        }
+    }
     const int my_tiles = (int)blockIdx.x < tiles ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int G = a.G;
     const int total = my_tiles * G;
@@ -548,6 +563,8 @@ cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* x
     a.n_tiles = n_tiles;
     a.perm = perm;
     a.topk = topk;
+    a.E = E;
+    a.max_tiles = max_tiles;
     const int grid = max_tiles < di.sm_count ? max_tiles : di.sm_count;
     return launch_any<true>(fmt, a, grid, s);
 }

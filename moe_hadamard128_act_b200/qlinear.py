@@ -32,6 +32,7 @@ FORMATS = (I8_G128_BF16, I8_G128_F16, I8A8_G128_BF16, I4_G64_BF16, I5Z_G128_F16,
 DEVERR_EXPERT_ID = 1
 DEVERR_CODE_RANGE = 2
 DEVERR_TIMEOUT = 4
+DEVERR_BOUNDS = 8
 
 A16_MAX_K = 32768  # QL_A16_MAX_K: largest K for the formats whose activations stay 16-bit
 
