@@ -359,21 +359,6 @@ cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, const int32_t* inv, int topk, __half* xs,
-                                    float* xf, cudaStream_t s) {
-    const size_t smem = (size_t)K * (sizeof(float) + sizeof(__half));  // the fp32 row and its f16 copy
-    cudaError_t e = prefer_max_shared(k_prep_a16);
-    if (e != cudaSuccess) return e;
-    if (smem > 48 * 1024) {
-        e = cudaFuncSetAttribute(k_prep_a16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    DeviceInfo di;
-    if ((e = device_info(&di)) != cudaSuccess) return e;
-    k_prep_a16<<<T, 256, smem, s>>>(static_cast<const __nv_bfloat16*>(x), T, K, rotate, XORD_NATURAL, xs, xf, nullptr, 0,
-                                    inv, topk, nullptr, T * topk, di.err_word);
-    return cudaGetLastError();
-}
 
 }  // namespace ql
 

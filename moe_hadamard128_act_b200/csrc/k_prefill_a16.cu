@@ -48,6 +48,10 @@
 // wait on that one commit, on a ring of 6 mbarriers (a multiple of the
 // activation, A-tile and accumulator ring depths).
 //
+// The grouped mode (GRP: the MoE experts' tiles from the permute kernel) is
+// not launched: it is withdrawn until the cause of an intermittent device
+// fault seen with it, in repeated calls at 2048 tokens x top-8, is found.
+//
 // All waits are bounded (200 ms); on a timeout the CTA sets QL_DEVERR_TIMEOUT
 // and winds down without leaving tensor memory allocated, MMAs running or
 // copies in flight.
@@ -534,39 +538,5 @@ cudaError_t launch_prefill_a16(int fmt, const __half* xs, const float* xf, const
     return launch_any<false>(fmt, a, grid, s);
 }
 
-cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* xf, const uint8_t* codes,
-                                       const void* scales, int E, int N, int K, int rows_total, const MoeTile* tiles,
-                                       const int* n_tiles, int max_tiles, const int32_t* perm, int topk, float* y,
-                                       cudaStream_t s) {
-    if (!prefill_a16_supported(fmt)) return cudaErrorInvalidValue;
-    DeviceInfo di;
-    cudaError_t e = device_info(&di);
-    if (e != cudaSuccess) return e;
-    if ((size_t)SMEM_BYTES > di.smem_optin) return cudaErrorInvalidValue;
-    A16Args a{};
-    if ((e = make_tmap_2d(codes, (long long)E * N, K, K, GK, TM, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmW)) != cudaSuccess)
-        return e;
-    if ((e = make_tmap_2d(xs, rows_total, 2LL * K, 2LL * K, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmX)) !=
-            cudaSuccess ||
-        (e = make_tmap_2d(xs, rows_total, 2LL * K, 2LL * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, &a.tmXb)) !=
-            cudaSuccess)
-        return e;
-    a.sw = static_cast<const uint16_t*>(scales);
-    a.xf = xf;
-    a.y = y;
-    a.err = di.err_word;
-    a.M = rows_total;
-    a.N = N;
-    a.G = K / GK;
-    a.ldy = N;
-    a.tiles = tiles;
-    a.n_tiles = n_tiles;
-    a.perm = perm;
-    a.topk = topk;
-    a.E = E;
-    a.max_tiles = max_tiles;
-    const int grid = max_tiles < di.sm_count ? max_tiles : di.sm_count;
-    return launch_any<true>(fmt, a, grid, s);
-}
 
 }  // namespace ql

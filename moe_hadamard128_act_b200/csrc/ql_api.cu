@@ -158,8 +158,12 @@ int x_order(int fmt) {
 }
 
 // The grouped tensor-core GEMM takes over once experts average this many rows.
+// The grouped tensor-core path runs format-7 experts only.  The int8 / FP8 experts with 16-bit
+// activations had one too (the A16 prefill kernel in grouped mode); it is withdrawn until the cause
+// of an intermittent device fault seen with it is found, and those experts take the chunked
+// grouped decode kernel at every batch size.
 bool moe_grouped(const ql_experts* ex, int T, int topk) {
-    return (long long)T * topk >= (long long)kMoePrefillMinRowsPerExpert * ex->E;
+    return ex->fmt == QL_FP8A8_B128_BF16 && (long long)T * topk >= (long long)kMoePrefillMinRowsPerExpert * ex->E;
 }
 // Format 7 experts, grouped: the permuted rows' scales [K/128][Mp], with the 132 columns past the last
 // row that a tile's 16-byte aligned scale copy may read.
@@ -184,9 +188,7 @@ MoeWs moe_ws(const ql_experts* ex, int T, int topk) {
     w.counts = o; o += align_up((size_t)ex->E * 4, 256);
     w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
     w.perm = o; o += align_up((size_t)T * topk * 4, 256);
-    w.max_tiles = !grp ? 0
-                  : e4 ? moe_max_tiles(T, topk, ex->E, kPrefillTileM, (ex->N + kPrefillTileN - 1) / kPrefillTileN)
-                       : moe_max_tiles(T, topk, ex->E, kPrefillA16Tokens, (ex->N + 127) / 128);
+    w.max_tiles = grp ? moe_max_tiles(T, topk, ex->E, kPrefillTileM, (ex->N + kPrefillTileN - 1) / kPrefillTileN) : 0;
     w.sw = 0;
     if (grp) {
         w.inv = o; o += align_up((size_t)T * topk * 4, 256);
@@ -626,7 +628,7 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     const int K = experts->K, N = experts->N;
     const int rot = (experts->flags & QL_HADAMARD) ? 1 : 0;
     cudaError_t e;
-    if (moe_grouped(experts, T, topk) && experts->fmt == QL_FP8A8_B128_BF16) {
+    if (moe_grouped(experts, T, topk)) {  // format 7
         // permute; E4M3 codes and scales straight into permuted order; the experts' weight scales
         // as fp32; the grouped E4M3 tensor-core GEMM with the un-permute in its stores
         MoePermuteOut po;
@@ -656,30 +658,6 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
         e = launch_prefill_e4m3_grouped(reinterpret_cast<const uint8_t*>(xs), xf, Mp,
                                         static_cast<const uint8_t*>(experts->codes), swT, experts->E, N, K, T * topk,
                                         po.tiles, nch, (int)w.max_tiles, perm, y, s);
-        trace_end(t, s);
-        return from_cuda(e);
-    }
-    if (moe_grouped(experts, T, topk)) {  // permute, stage x in permuted order, grouped tensor-core GEMM
-        MoePermuteOut po;
-        po.inv = reinterpret_cast<int32_t*>(b + w.inv);
-        po.tiles = reinterpret_cast<MoeTile*>(b + w.tiles);
-        po.n_tiles = nch;
-        po.tile_rows = kPrefillA16Tokens;
-        po.wblocks = (N + 127) / 128;
-        po.yz = y;  // rows of pairs with a bad expert id are zeroed
-        po.N = N;
-        int t = trace_begin(QL_KIND_MOE_PERMUTE, s);
-        e = launch_moe_permute(topk_ids, T, topk, experts->E, counts, offsets, perm, po, di.err_word, s);
-        trace_end(t, s);
-        if (e != cudaSuccess) return from_cuda(e);
-        t = trace_begin(QL_KIND_PREP_A16, s);
-        e = launch_prep_a16_scatter(x, T, K, rot, po.inv, topk, xs, xf, s);
-        trace_end(t, s);
-        if (e != cudaSuccess) return from_cuda(e);
-        t = trace_begin(QL_KIND_MOE_GEMM, s);
-        e = launch_prefill_a16_grouped(experts->fmt, xs, xf, static_cast<const uint8_t*>(experts->codes),
-                                       experts->scales, experts->E, N, K, T * topk, po.tiles, nch, (int)w.max_tiles,
-                                       perm, topk, y, s);
         trace_end(t, s);
         return from_cuda(e);
     }

@@ -65,10 +65,6 @@ cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8
 // point) and puts 2^24 into xf (the int5 codes enter the MMAs as exact subnormals u * 2^-24).
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s, float* xsum = nullptr);
-// The same for the grouped expert GEMM: token t's f16 row goes to rows
-// inv[t * topk + j] of xs (j < topk, rows < 0 skipped); xf stays per token.
-cudaError_t launch_prep_a16_scatter(const void* x, int T, int K, int rotate, const int32_t* inv, int topk, __half* xs,
-                                    float* xf, cudaStream_t s);
 
 // ---- packing ---------------------------------------------------------------------
 cudaError_t launch_pack_rtn(const float* W, int fmt, int flags, int N, int K, void* codes, void* scales,
@@ -171,13 +167,6 @@ struct MoePermuteOut {
     int N = 0;
 };
 size_t moe_max_tiles(int T, int topk, int E, int tile_rows, int wblocks);
-// Grouped over experts: codes [E][N][K] and scales stacked per expert, xs the
-// permuted rows (launch_prep_a16_scatter), tiles / n_tiles from the permute;
-// row r of a tile lands in y[perm[r]][0 .. N) scaled by xf[perm[r] / topk].
-cudaError_t launch_prefill_a16_grouped(int fmt, const __half* xs, const float* xf, const uint8_t* codes,
-                                       const void* scales, int E, int N, int K, int rows_total, const MoeTile* tiles,
-                                       const int* n_tiles, int max_tiles, const int32_t* perm, int topk, float* y,
-                                       cudaStream_t s);
 // Format 7 experts on the E4M3 tensor-core GEMM, grouped: qx the E4M3 codes of the permuted rows
 // [rows_total][K] with their scales sxT [K/128][Mp] (Mp % 4 == 0, at least 132 columns past the last
 // row), swT the experts' weight scales from launch_prefill_prep_blk (E blocks), tiles of

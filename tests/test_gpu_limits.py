@@ -36,7 +36,7 @@ def test_forward_parity_at_max_k(Q, fmt, M):
     assert_close(y.cpu().numpy(), ref, f"fmt {fmt} M {M} K {K}")
 
 
-@pytest.mark.parametrize("T", [16, 1024])  # the grouped skinny GEMM and the grouped tensor-core GEMM
+@pytest.mark.parametrize("T", [16, 1024])  # in-kernel ranking, then the permute kernel's chunks
 def test_moe_gate_up_max_experts(Q, T):
     E, topk, N, K = 1024, 8, 64, 128
     codes, scales = moe_weights(E, N, K, Q.I8_G128_BF16)

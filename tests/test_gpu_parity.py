@@ -284,7 +284,8 @@ def moe_weights(E, N, K, fmt, seed=9):
                                           (20, 32, 8, 130, 256), (40, 8, 3, 48, 128)])
 def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
     # T * topk <= 128: the expert GEMM ranks the ids itself; (20, 32, 8): 160 pairs, the
-    # permute kernel's chunk table; (40, 8, 3): the grouped tensor-core GEMM.
+    # permute kernel's chunk table; (40, 8, 3): format 7 on the grouped tensor-core GEMM, the other
+    # formats on the chunk table.
     codes, scales = moe_weights(E, N, K, fmt)
     ids, w = synth.routing(6, T, E, topk)
     x = x_bits(T, K, seed=13)
@@ -298,8 +299,9 @@ def test_moe_gate_up_parity(fmt, T, E, topk, N, K):
 @pytest.mark.parametrize("T,E,topk,N,K", [(64, 8, 4, 130, 384), (300, 16, 8, 200, 256), (50, 64, 8, 128, 128),
                                           (600, 8, 2, 400, 256)])
 def test_moe_gate_up_grouped_parity(fmt, T, E, topk, N, K):
-    # T * topk >= 8 E: the grouped tensor-core GEMM. (300, 16, 8): ~150 rows per expert, some over one
-    # 192-row block; N = 200: a ragged second weight block. (50, 64, 8): some experts get no rows.
+    # T * topk >= 8 E: format 7 on the grouped tensor-core GEMM, the formats with 16-bit activations
+    # on the weight-streaming kernel over the permute kernel's 16-row chunks.  (300, 16, 8): ~150
+    # rows per expert; N = 200: a ragged second weight block. (50, 64, 8): some experts get no rows.
     # (600, 8, 2): ~150 rows per expert, several 128-row tiles each; N = 400: three weight tiles of the
     # E4M3 GEMM (192 rows each), the last one ragged.
     codes, scales = moe_weights(E, N, K, fmt)
