@@ -99,9 +99,9 @@ typedef enum {
  * calls accept the flag and ignore it. */
 enum { QL_HADAMARD = 1, QL_SCALE_SEARCH = 2 };
 
-/* Bits of the device error word.  QL_DEVERR_BOUNDS: a grouped kernel found a
- * routing table entry (a tile or a permuted row) outside its buffers and skipped
- * it; the results of that call are incomplete. */
+/* Bits of the device error word.  QL_DEVERR_BOUNDS: a kernel found an index it
+ * reads from device memory (a routing table entry or a permuted row) outside its
+ * buffers and skipped it; the results of that call are incomplete. */
 enum { QL_DEVERR_EXPERT_ID = 1, QL_DEVERR_CODE_RANGE = 2, QL_DEVERR_TIMEOUT = 4, QL_DEVERR_BOUNDS = 8 };
 
 /* Human-readable name of a status. Never NULL. */

@@ -892,6 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const bool fused = a.ids != nullptr;
+    constexpr int CR = 8 * NT;  // rows per chunk of the fused mode: one or two n-tiles
     // Routing state of the fused mode, after the rings and barriers.
     int* const s_ids = reinterpret_cast<int*>(smem_raw + (base - raw) + moe_ring_bytes<FMT>() + kWarps * kMoeStages * 8);
     int* const s_perm = s_ids + kMoeFusedMaxPairs;   // permuted position -> pair index t * topk + j
@@ -931,14 +932,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
         int nv = 0;  // valid pairs: positions 0 .. nv - 1
         for (int j = 0; j < P; ++j) nv += s_ids[j] >= 0 && s_ids[j] < a.E;
         for (int p = threadIdx.x; p < nv; p += kThreads) {
-            if (s_bef[p] % 16) continue;  // a chunk starts at every 16th row of an expert's segment
+            if (s_bef[p] % CR) continue;  // a chunk starts at every CR-th row of an expert's segment
             int idx = 0;
-            for (int q = 0; q < p; ++q) idx += s_bef[q] % 16 == 0;
-            s_ch[idx] = MoeChunk{s_exp[p], p, min(16, s_cnt[p] - s_bef[p])};
+            for (int q = 0; q < p; ++q) idx += s_bef[q] % CR == 0;
+            s_ch[idx] = MoeChunk{s_exp[p], p, min(CR, s_cnt[p] - s_bef[p])};
         }
         if (threadIdx.x == 0) {
             int n = 0;
-            for (int q = 0; q < nv; ++q) n += s_bef[q] % 16 == 0;
+            for (int q = 0; q < nv; ++q) n += s_bef[q] % CR == 0;
             *s_nch = n;
         }
         __syncthreads();
@@ -1289,9 +1290,9 @@ cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        if ((e = cudaFuncSetAttribute(k_moe_tma<kFmtDown, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess)
-            return e;
+        for (auto kern : {k_moe_tma<kFmtDown, 1>, k_moe_tma<kFmtDown, 2>})
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return e;
         if (dev < 64) attr_set[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
@@ -1304,7 +1305,8 @@ cudaError_t launch_moe_down(const MoeArgs& in, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = a.ids ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k_moe_tma<kFmtDown, 2>, a);
+    // the fused mode cuts its own chunks at 8 rows (one n-tile); the permute's chunks hold up to 16
+    e = a.ids ? cudaLaunchKernelEx(&cfg, k_moe_tma<kFmtDown, 1>, a) : cudaLaunchKernelEx(&cfg, k_moe_tma<kFmtDown, 2>, a);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1325,7 +1327,8 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
         for (auto kern : {k_moe_tma<QL_I8_G128_BF16, 2>, k_moe_tma<QL_I8_G128_F16, 2>, k_moe_tma<QL_FP8_B128_BF16, 2>,
-                          k_moe_tma<QL_FP8A8_B128_BF16, 2>}) {
+                          k_moe_tma<QL_FP8A8_B128_BF16, 2>, k_moe_tma<QL_I8_G128_BF16, 1>, k_moe_tma<QL_I8_G128_F16, 1>,
+                          k_moe_tma<QL_FP8_B128_BF16, 1>, k_moe_tma<QL_FP8A8_B128_BF16, 1>}) {
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
                 return e;
         }
@@ -1347,11 +1350,15 @@ cudaError_t launch_moe_skinny(const MoeArgs& in, cudaStream_t s) {
         cudaError_t r = cudaLaunchKernelEx(&cfg, kern, a);
         return r != cudaSuccess ? r : cudaGetLastError();
     };
+    // The fused mode cuts its own chunks at 8 rows: one n-tile per MMA (NT = 1); the permute
+    // kernel's chunks hold up to 16 rows (NT = 2).
+    const bool one = a.ids != nullptr;
     switch (a.fmt) {
-    case QL_I8_G128_BF16: return run(k_moe_tma<QL_I8_G128_BF16, 2>);
-    case QL_I8_G128_F16: return run(k_moe_tma<QL_I8_G128_F16, 2>);
-    case QL_FP8_B128_BF16: return run(k_moe_tma<QL_FP8_B128_BF16, 2>);
-    case QL_FP8A8_B128_BF16: return run(k_moe_tma<QL_FP8A8_B128_BF16, 2>);
+    case QL_I8_G128_BF16: return one ? run(k_moe_tma<QL_I8_G128_BF16, 1>) : run(k_moe_tma<QL_I8_G128_BF16, 2>);
+    case QL_I8_G128_F16: return one ? run(k_moe_tma<QL_I8_G128_F16, 1>) : run(k_moe_tma<QL_I8_G128_F16, 2>);
+    case QL_FP8_B128_BF16: return one ? run(k_moe_tma<QL_FP8_B128_BF16, 1>) : run(k_moe_tma<QL_FP8_B128_BF16, 2>);
+    case QL_FP8A8_B128_BF16:
+        return one ? run(k_moe_tma<QL_FP8A8_B128_BF16, 1>) : run(k_moe_tma<QL_FP8A8_B128_BF16, 2>);
     default: return cudaErrorInvalidValue;
     }
 }
