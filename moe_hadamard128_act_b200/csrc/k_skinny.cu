@@ -1009,13 +1009,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     // The weight stream is running; the activations and the zeroed y come from the prologue.
     if (fused) asm volatile("griddepcontrol.wait;\n" ::: "memory");
     MoeChunk chc = chunks[cp.ch];  // the chunk being computed
-    int tok[NT];                     // this lane's tokens in it (-1: none): the MMA's B columns it loads
+    // This lane's activation row per n-tile (the MMA's B column it loads), as a byte pointer.  A
+    // lane past the chunk's rows loads the chunk's first row instead: its MMA column is computed
+    // and never stored, so no test sits in the fragment loads.
+    const uint8_t* xrow[NT];
     int ctok[NT][2];                 // format 7: the tokens of this lane's accumulator columns
     auto load_tokens = [&]() {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int slot = 8 * nt + g;  // (the down projection's activations are per pair)
-            tok[nt] = slot < chc.count ? perm[chc.start + slot] / (DOWN ? 1 : a.topk) : -1;
+            const int tk = perm[chc.start + (slot < chc.count ? slot : 0)] / (DOWN ? 1 : a.topk);
+            // row bytes: E4M3 codes K, f16 K * 2, the down projection's three bf16 planes K * 6
+            xrow[nt] = static_cast<const uint8_t*>(a.xs) + (long long)tk * a.K * (DOWN ? 6 : act8<FMT>() ? 1 : 2);
             if constexpr (act8<FMT>()) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
@@ -1075,23 +1080,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
             // The fragments read_unit_smem hands out pair with these 16-byte x pieces of the group
             // (the same order as the dense kernel's staged activations).
             auto getx = [&](int nt, int p) -> uint4 {
-                if (tok[nt] < 0) return make_uint4(0, 0, 0, 0);
                 if constexpr (act8<FMT>()) {  // E4M3 codes: the dense kernel's piece order, 16 B each
                     const int j = 4 * p + c;
-                    return __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.xs) +
-                                                                (long long)tok[nt] * a.K + grp * 128 + 16 * j));
+                    return __ldg(reinterpret_cast<const uint4*>(xrow[nt] + grp * 128 + 16 * j));
                 } else {
                     const int j = (p >> 1) * 8 + 2 * c + (p & 1);
-                    return __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(a.xs) +
-                                                                (long long)tok[nt] * a.K + grp * 128 + 8 * j));
+                    return __ldg(reinterpret_cast<const uint4*>(xrow[nt] + grp * 256 + 16 * j));
                 }
             };
             if constexpr (DOWN) {
                 auto getx3 = [&](int nt, int piece, int pl) -> uint4 {
-                    if (tok[nt] < 0) return make_uint4(0, 0, 0, 0);
-                    const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(a.xs) +
-                                              ((long long)tok[nt] * 3 + pl) * a.K + grp * 64 + 8 * (piece ? 4 + c : c);
-                    return __ldg(reinterpret_cast<const uint4*>(xr));
+                    return __ldg(reinterpret_cast<const uint4*>(xrow[nt] + ((long long)pl * a.K + grp * 64) * 2 +
+                                                                16 * (piece ? 4 + c : c)));
                 };
                 unit_down<NT>(r, getx3, chc.count > 8, yacc);
             } else if constexpr (act8<FMT>()) {
