@@ -987,15 +987,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     __syncwarp();
+    // The issue side's (chunk, slab): its weight row in the stacked experts and this lane's two
+    // scale rows, recomputed only when the slab changes (every G units).
+    int i_ch = -1, i_slab = -1, i_wrow = 0;
+    const uint16_t* i_srow[2] = {nullptr, nullptr};
     auto issue = [&](int st) {
-        const MoeChunk ch = chunks[ip.ch];
+        if (ip.ch != i_ch || ip.slab != i_slab) {
+            i_ch = ip.ch;
+            i_slab = ip.slab;
+            const MoeChunk ch = chunks[ip.ch];
+            i_wrow = ch.expert * a.N + ip.slab * 16;
+            if constexpr (!DOWN) {
+                const uint16_t* const se = sc0 + (long long)ch.expert * expert_scales;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int n = ip.slab * 16 + g + 8 * h;
+                    i_srow[h] = n < a.N ? se + (long long)(block_scaled<FMT>() ? (n >> 7) : n) * G : nullptr;
+                }
+            }
+        }
         if (lane == 0) {
             mbar_expect_tx(bars + 8 * st, SB);
-            tma_load_2d(ring + st * SB, &a.tmap, ip.grp * 128, ch.expert * a.N + ip.slab * 16, bars + 8 * st);
+            tma_load_2d(ring + st * SB, &a.tmap, ip.grp * 128, i_wrow, bars + 8 * st);
         }
-        if constexpr (!DOWN)
-            load_side_w<FMT, NT>(sd[st], sc0 + (long long)ch.expert * expert_scales, nullptr, a.N, G, ip.grp, ip.slab,
-                                 g);
+        if constexpr (!DOWN) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) sd[st].sw[h][0] = i_srow[h] ? (uint32_t)__ldg(i_srow[h] + ip.grp) : 0u;
+        }
         ip.next(slabs, G);
         ++issued;
     };
