@@ -546,25 +546,6 @@ struct Side {
 };
 
 template <int FMT, int NT>
-__device__ __forceinline__ void load_side_w(Side<FMT, NT>& d, const void* scales, const uint8_t* zeros, int N,
-                                            int Gtot, int gabs, int slab, int g) {
-    const uint16_t* sc = static_cast<const uint16_t*>(scales);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int n = slab * 16 + g + 8 * h;
-        const bool ok = n < N && sc;
-        if constexpr (FMT == QL_I4_G64_BF16) {  // the unit's two bf16 scales, adjacent: one 32-bit load
-            d.sw[h][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(sc + (long long)n * (2 * Gtot) + 2 * gabs)) : 0u;
-        } else if constexpr (block_scaled<FMT>()) {
-            d.sw[h][0] = ok ? __ldg(sc + (long long)(n >> 7) * Gtot + gabs) : 0u;
-        } else {
-            d.sw[h][0] = ok ? __ldg(sc + (long long)n * Gtot + gabs) : 0u;
-        }
-        if constexpr (FMT == QL_I5Z_G128_F16) d.z[h] = ok ? __ldg(zeros + (long long)n * Gtot + gabs) : 0u;
-    }
-}
-
-template <int FMT, int NT>
 __device__ __forceinline__ void load_side_x(Side<FMT, NT>& d, const float* sx, int M, int Gtot, int gabs, int c) {
     if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16) {  // int5: the tokens' group sums
 #pragma unroll
@@ -653,6 +634,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     __syncwarp();
     QL_PROF(7)
     // Issues slot s's TMA boxes (UPS consecutive groups of one slab) and fetches their side data.
+    // This lane's two scale rows (and int5 zero rows) of the issue side's slab, recomputed only when
+    // the slab changes; a row past N reads as scale 0.
+    int i_slab = -1;
+    const uint16_t* i_srow[2] = {nullptr, nullptr};
+    const uint8_t* i_zrow[2] = {nullptr, nullptr};
     auto issue = [&](int s) {
         if (lane == 0) {
             mbar_expect_tx(bars + 8 * s, SB);
@@ -661,9 +647,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 tma_load_2d(ring + s * SB + i * SB1, &a.tmap, (UPS * ip.grp(GP) + i) * URB, ip.slab * 16,
                             bars + 8 * s);
         }
+        if (ip.slab != i_slab) {
+            i_slab = ip.slab;
+            const uint16_t* const sc = static_cast<const uint16_t*>(a.scales);
 #pragma unroll
-        for (int i = 0; i < UPS; ++i)
-            load_side_w<FMT, NT>(sd[s][i], a.scales, a.zeros, a.N, a.Gtot, a.g0 + UPS * ip.grp(GP) + i, ip.slab, g);
+            for (int h = 0; h < 2; ++h) {
+                const int n = ip.slab * 16 + g + 8 * h;
+                const bool ok = n < a.N && sc;
+                const long long row = block_scaled<FMT>() ? (long long)(n >> 7) * a.Gtot
+                                      : FMT == QL_I4_G64_BF16 ? (long long)n * (2 * a.Gtot)
+                                                               : (long long)n * a.Gtot;
+                i_srow[h] = ok ? sc + row : nullptr;
+                if constexpr (FMT == QL_I5Z_G128_F16) i_zrow[h] = ok ? a.zeros + (long long)n * a.Gtot : nullptr;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < UPS; ++i) {
+            const int gabs = a.g0 + UPS * ip.grp(GP) + i;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if constexpr (FMT == QL_I4_G64_BF16)  // the unit's two bf16 scales, adjacent: one 32-bit load
+                    sd[s][i].sw[h][0] = i_srow[h] ? __ldg(reinterpret_cast<const uint32_t*>(i_srow[h] + 2 * gabs)) : 0u;
+                else
+                    sd[s][i].sw[h][0] = i_srow[h] ? (uint32_t)__ldg(i_srow[h] + gabs) : 0u;
+                if constexpr (FMT == QL_I5Z_G128_F16) sd[s][i].z[h] = i_zrow[h] ? __ldg(i_zrow[h] + gabs) : 0u;
+            }
+        }
     };
     // Start the weight stream first: it never depends on the kernel before.
 #pragma unroll
