@@ -105,7 +105,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // offset o; the 16-byte pieces of each group are also swapped pairwise in
 // their upper half (the shared-memory layout the GEMM reads without bank
 // conflicts); xsum[t][g] = the group's sum of f16(x * f) (for the zero point),
-// and xf = 2^24 / f (the codes enter the MMAs as u * 2^-24).
+// and xf = 2^24 / f (the codes enter the MMAs as u * 2^-24).  The natural
+// order with xsum requested is the int8 decode's: the same group sums and
+// 2^24 / f (its codes enter the MMAs as the subnormals (q + 128) * 2^-24).
 // f16 holds every bf16 value of the scaled row exactly down to 2^-14 (its
 // normal range); below that the rounding error is under 2^-39 of the row's
 // max, far beneath the fp32 accumulation error of the GEMM.
@@ -163,10 +165,20 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
         if (m > 0.0f && m <= 3.4e38f) frexpf(m, &e);
         e = max(-100, min(128, e));
         red[0] = ldexpf(1.0f, 15 - e);
-        xf[t] = ldexpf(1.0f, e - 15 + (order == XORD_I5 ? 24 : 0));
+        xf[t] = ldexpf(1.0f, e - 15 + (xsum ? 24 : 0));
     }
     __syncthreads();
     const float f = red[0];
+    if (xsum) {  // the groups' sums of the f16 activations (for the codes' offset)
+        for (int g = warp; g < K / 128; g += 8) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sum += __half2float(__float2half_rn(__fmul_rn(row[g * 128 + 4 * lane + i], f)));
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
+            if (lane == 0) xsum[(long long)t * (K / 128) + g] = sum;
+        }
+    }
     if (order == XORD_NATURAL) {  // converted once into shared memory, then 16-byte copies per output row
         uint4* const hrow = reinterpret_cast<uint4*>(row + K);  // [K / 8] x 8 f16
         const int K8 = K / 8;
@@ -195,17 +207,6 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
         return;
     }
     __half* out = xs + (long long)t * K;
-    if (order == XORD_I5) {
-        const int lane5 = threadIdx.x & 31, warp5 = threadIdx.x >> 5;
-        for (int g = warp5; g < K / 128; g += 8) {  // the groups' sums of the f16 activations
-            float sum = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) sum += __half2float(__float2half_rn(__fmul_rn(row[g * 128 + 4 * lane5 + i], f)));
-#pragma unroll
-            for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
-            if (lane5 == 0) xsum[(long long)t * (K / 128) + g] = sum;
-        }
-    }
     if (order == XORD_I5) {
         for (int run = threadIdx.x; run < K / 32; run += 256)  // one lane's 32 codes of a group
             i5_stage_run<0>(row + run * 32, f, out, run * 32);

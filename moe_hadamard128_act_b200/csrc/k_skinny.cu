@@ -74,6 +74,11 @@ struct Regs<kFmtDown> : Regs<QL_I8_G128_BF16> {};
 // per 128 (int8 for W8A8, E4M3 for format 7), multiplied on the byte MMAs.
 template <int FMT>
 __host__ __device__ constexpr bool act8() { return FMT == QL_I8A8_G128_BF16 || FMT == QL_FP8A8_B128_BF16; }
+// int8 codes with 16-bit activations: the codes enter the MMAs as subnormals (q + 128) * 2^-24,
+// and the offset comes off with the token's group sum (as the int5 zero point does).
+template <int FMT>
+__host__ __device__ constexpr bool i8sub() { return FMT == QL_I8_G128_BF16 || FMT == QL_I8_G128_F16; }
+constexpr float kI8Off = 7.62939453125e-06f;  // 128 * 2^-24
 // Weight scales per 128 x 128 block rather than per row.
 template <int FMT>
 __host__ __device__ constexpr bool block_scaled() { return FMT == QL_FP8_B128_BF16 || FMT == QL_FP8A8_B128_BF16; }
@@ -131,9 +136,11 @@ __device__ __forceinline__ void fold_chains(T (&acc)[CH][NT][4]) {
 
 // The per-group MMAs of one unit for the weight-only formats.
 // getx(nt, piece) returns the lane's 16-byte activation piece for n-tile nt.
+// X: the group sums of the lane's column tokens (int8 codes only: their subnormal offset).
 // yacc[nt][i] accumulates scale * partial; i = 0,1 row g, i = 2,3 row g + 8.
 template <int FMT, int NT, typename GetX>
-__device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1_live, float (&yacc)[NT][4]) {
+__device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1_live, const float (&X)[NT][2],
+                                         float (&yacc)[NT][4]) {
     constexpr int CH = NT == 1 ? 2 : 1;  // independent accumulation chains per group (see fold_chains)
     if constexpr (FMT == QL_I4_G64_BF16) {
 #pragma unroll
@@ -201,8 +208,8 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
                     a1 = e4m3x2_to_f16x2(w1);
                     a3 = e4m3x2_to_f16x2(w1 >> 16);
                 } else {
-                    i8x4_to_f16(word_of(r.w[0], s), a0, a2);
-                    i8x4_to_f16(word_of(r.w[1], s), a1, a3);
+                    i8x4_to_f16sub(word_of(r.w[0], s), a0, a2);
+                    i8x4_to_f16sub(word_of(r.w[1], s), a1, a3);
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -215,12 +222,12 @@ __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1
         }
         fold_chains<CH, NT>(acc);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            yacc[nt][0] = fmaf(r.s[0], acc[0][nt][0], yacc[nt][0]);
-            yacc[nt][1] = fmaf(r.s[0], acc[0][nt][1], yacc[nt][1]);
-            yacc[nt][2] = fmaf(r.s[1], acc[0][nt][2], yacc[nt][2]);
-            yacc[nt][3] = fmaf(r.s[1], acc[0][nt][3], yacc[nt][3]);
-        }
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = i8sub<FMT>() ? fmaf(-kI8Off, X[nt][i & 1], acc[0][nt][i]) : acc[0][nt][i];
+                yacc[nt][i] = fmaf(r.s[i >> 1], t, yacc[nt][i]);
+            }
     }
 }
 
@@ -547,7 +554,7 @@ struct Side {
 
 template <int FMT, int NT>
 __device__ __forceinline__ void load_side_x(Side<FMT, NT>& d, const float* sx, int M, int Gtot, int gabs, int c) {
-    if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16) {  // int5: the tokens' group sums
+    if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16 || i8sub<FMT>()) {  // int5, int8 A16: the group sums
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -727,8 +734,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     }
     // Per-token side data of the units already in flight: the activation scales (byte
     // activations) or the group sums (int5), written by the kernel before this one.
-    const float* const xside = FMT == QL_I5Z_G128_F16 ? a.xsum : a.xf;
-    if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16) {
+    const float* const xside = (FMT == QL_I5Z_G128_F16 || i8sub<FMT>()) ? a.xsum : a.xf;
+    if constexpr (act8<FMT>() || FMT == QL_I5Z_G128_F16 || i8sub<FMT>()) {
         UnitPos q = cp;
 #pragma unroll
         for (int s = 0; s < ST; ++s) {
@@ -832,7 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                 } else if constexpr (FMT == QL_I5Z_G128_F16) {
                     unit_i5<NT>(r, getx, nt1_live, sd[s][ui].sx, yacc);
                 } else {
-                    unit_a16<FMT, NT>(r, getx, nt1_live, yacc);
+                    unit_a16<FMT, NT>(r, getx, nt1_live, sd[s][ui].sx, yacc);
                 }
             }
             __syncwarp();
@@ -1040,6 +1047,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
     // lane past the chunk's rows loads the chunk's first row instead: its MMA column is computed
     // and never stored, so no test sits in the fragment loads.
     const uint8_t* xrow[NT];
+    const float* xsr[NT][2];  // int8 codes: the group-sum rows of this lane's accumulator columns (null: none)
     int ctok[NT][2];                 // format 7: the tokens of this lane's accumulator columns
     auto load_tokens = [&]() {
 #pragma unroll
@@ -1053,6 +1061,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                 for (int i = 0; i < 2; ++i) {
                     const int cs = 8 * nt + 2 * c + i;
                     ctok[nt][i] = cs < chc.count ? perm[chc.start + cs] / a.topk : -1;
+                }
+            }
+            if constexpr (i8sub<FMT>()) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int cs = 8 * nt + 2 * c + i;
+                    xsr[nt][i] = cs < chc.count ? a.xsum + (long long)(perm[chc.start + cs] / a.topk) * G : nullptr;
                 }
             }
         }
@@ -1135,7 +1150,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_moe_tma(const __grid_constant__
                         yacc[nt][2 + i] = fmaf(r.s[1] * sx, acc[nt][2 + i], yacc[nt][2 + i]);
                     }
             } else {
-                unit_a16<FMT, NT>(r, getx, chc.count > 8, yacc);
+                float X[NT][2];  // int8 codes: the column tokens' sums of this group's activations
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) X[nt][i] = i8sub<FMT>() && xsr[nt][i] ? __ldg(xsr[nt][i] + grp) : 0.0f;
+                unit_a16<FMT, NT>(r, getx, chc.count > 8, X, yacc);
             }
             __syncwarp();
             if (issued < u1) issue(st);  // refill this slot with the unit kMoeStages ahead

@@ -148,7 +148,8 @@ FwdWs forward_ws(int fmt, size_t M, size_t N, size_t K) {
     } else {
         w.x_bytes = align_up(M * K * 2, 256);
         w.f_bytes = align_up(M * 4, 256);
-        if (fmt == QL_I5Z_G128_F16) w.g_bytes = align_up(M * (K / 128) * 4, 256);  // the tokens' group sums
+        // the tokens' group sums: the int5 zero point, and the int8 codes' offset in the decode kernel
+        if (fmt == QL_I5Z_G128_F16 || fmt_i8_a16(fmt)) w.g_bytes = align_up(M * (K / 128) * 4, 256);
     }
     return w;
 }
@@ -169,7 +170,7 @@ bool moe_grouped(const ql_experts* ex, int T, int topk) {
 // row that a tile's 16-byte aligned scale copy may read.
 int moe_e4m3_mp(int T, int topk) { return (int)align_up((size_t)T * topk + 132, 4); }
 struct MoeWs {
-    size_t xs, xf, counts, offsets, perm, chunks, nch, inv, tiles, sw;
+    size_t xs, xf, xsum, counts, offsets, perm, chunks, nch, inv, tiles, sw;
     size_t max_tiles;
     size_t total;
 };
@@ -185,6 +186,9 @@ MoeWs moe_ws(const ql_experts* ex, int T, int topk) {
     const size_t G = (size_t)ex->K / 128;
     w.xs = o; o += align_up((size_t)(grp ? T * topk : T) * ex->K * (e4 ? 1 : 2), 256);
     w.xf = o; o += align_up(e4 ? (grp ? G * moe_e4m3_mp(T, topk) * 4 : (size_t)T * G * 4) : (size_t)T * 4, 256);
+    // int8 experts: each token's group sums of its f16 activations [T][K/128] (the codes' offset)
+    w.xsum = 0;
+    if (fmt_i8_a16(ex->fmt)) { w.xsum = o; o += align_up((size_t)T * G * 4, 256); }
     w.counts = o; o += align_up((size_t)ex->E * 4, 256);
     w.offsets = o; o += align_up(((size_t)ex->E + 1) * 4, 256);
     w.perm = o; o += align_up((size_t)T * topk * 4, 256);
@@ -426,7 +430,8 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         return from_cuda(e);
     }
     const long long ny = (long long)M * N;  // the prologue zeroes y for the accumulating GEMM
-    float* const xsum = fmt == QL_I5Z_G128_F16 ? reinterpret_cast<float*>(wsb + w.x_bytes + w.f_bytes) : nullptr;
+    float* const xsum = (fmt == QL_I5Z_G128_F16 || fmt_i8_a16(fmt)) ? reinterpret_cast<float*>(wsb + w.x_bytes + w.f_bytes)
+                                                                     : nullptr;
     if (fmt == QL_I8A8_G128_BF16) {
         const int t = trace_begin(QL_KIND_ACT_QUANT, s);
         e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, nullptr, 0, y, ny, s);
@@ -620,6 +625,7 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     uint8_t* b = static_cast<uint8_t*>(ws);
     __half* xs = reinterpret_cast<__half*>(b + w.xs);
     float* xf = reinterpret_cast<float*>(b + w.xf);
+    float* xsum = fmt_i8_a16(experts->fmt) ? reinterpret_cast<float*>(b + w.xsum) : nullptr;
     int32_t* counts = reinterpret_cast<int32_t*>(b + w.counts);
     int32_t* offsets = reinterpret_cast<int32_t*>(b + w.offsets);
     int32_t* perm = reinterpret_cast<int32_t*>(b + w.perm);
@@ -668,7 +674,7 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
                                   (long long)T * topk * N, s);
     } else {  // rotation, f16 staging, and the zeroing of y
         t = trace_begin(QL_KIND_PREP_A16, s);
-        e = launch_prep_a16(x, T, K, rot, XORD_NATURAL, xs, xf, y, (long long)T * topk * N, s);
+        e = launch_prep_a16(x, T, K, rot, XORD_NATURAL, xs, xf, y, (long long)T * topk * N, s, xsum);
     }
     trace_end(t, s);
     if (e != cudaSuccess) return from_cuda(e);
@@ -688,6 +694,7 @@ int moe_gate_up(const void* x, const int32_t* topk_ids, const float* topk_weight
     a.scales = experts->scales;
     a.xs = xs;
     a.xf = xf;
+    a.xsum = xsum;
     a.perm = perm;
     a.chunks = chunks;
     a.n_chunks = nch;

@@ -165,6 +165,16 @@ __device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& 
     hi = hadd2_u32(__byte_perm(u, 0x64646464u, 0x4342), 0xE480E480u);
 }
 
+// Four int8 codes (bytes 0..3 of w) -> f16x2 pairs lo = (c0, c1), hi = (c2, c3)
+// as subnormals: u = c + 128 placed in the low byte of a zero f16 is exactly
+// u * 2^-24.  A dot product over a group then carries 2^-24 * (sum c x + 128 sum x);
+// the caller takes the offset off with the activations' group sum.
+__device__ __forceinline__ void i8x4_to_f16sub(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    lo = __byte_perm(u, 0u, 0x4140);
+    hi = __byte_perm(u, 0u, 0x4342);
+}
+
 // Two e4m3 bytes (low, high) -> f16x2, exact (every e4m3 value is an f16).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
     __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xFFFFu), __NV_E4M3);

@@ -18,6 +18,8 @@ inline bool fmt_valid(int f) { return f >= QL_I8_G128_BF16 && f <= QL_FP8A8_B128
 // FP8 E4M3 weights with 128 x 128 block scales (formats 6 and 7 pack alike).
 inline bool fmt_fp8_weights(int f) { return f == QL_FP8_B128_BF16 || f == QL_FP8A8_B128_BF16; }
 inline bool fmt_scale_f16(int f) { return f == QL_I8_G128_F16 || f == QL_I5Z_G128_F16; }
+// int8 codes with 16-bit activations (formats 1 and 2).
+inline bool fmt_i8_a16(int f) { return f == QL_I8_G128_BF16 || f == QL_I8_G128_F16; }
 inline int fmt_group(int f) { return f == QL_I4_G64_BF16 ? 64 : 128; }
 // Bytes of one packed row of K codes.
 inline size_t fmt_row_bytes(int f, size_t K) {
@@ -81,7 +83,7 @@ struct SkinnyArgs {
     const uint8_t* zeros;  // int5: [N][Gtot]
     const void* xs;        // prepared activations, row stride ldx elements; offset to group g0
     const float* xf;       // A16: [M] inverse token factors; W8A8: sx [M][Gtot]
-    const float* xsum = nullptr;  // int5: each token's sums of its f16 activations per group [M][Gtot]
+    const float* xsum = nullptr;  // int5, int8 A16: each token's sums of its f16 activations per group [M][Gtot]
     float* y;              // [M][ldy]
     int32_t* acc;          // optional W8A8 group sums [M][N][Gtot]
     unsigned* err;         // device error word (filled by launch_skinny)
@@ -195,6 +197,7 @@ struct MoeArgs {
     const void* scales;    // [E][...] per the format
     const void* xs;        // prepared activations [T][K]: f16 in natural order, or E4M3 codes (format 7)
     const float* xf;       // [T] inverse token factors, or (format 7) activation scales [T][K/128]
+    const float* xsum = nullptr;  // int8 codes: each token's sums of its f16 activations per group [T][K/128]
     const int32_t* perm;   // [T*topk]
     const MoeChunk* chunks;
     const int* n_chunks;
