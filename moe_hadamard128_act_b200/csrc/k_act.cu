@@ -165,18 +165,19 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
         if (m > 0.0f && m <= 3.4e38f) frexpf(m, &e);
         e = max(-100, min(128, e));
         red[0] = ldexpf(1.0f, 15 - e);
-        xf[t] = ldexpf(1.0f, e - 15 + (xsum ? 24 : 0));
+        xf[t] = ldexpf(1.0f, e - 15 + (xsum && order != XORD_I4 ? 24 : 0));
     }
     __syncthreads();
     const float f = red[0];
-    if (xsum) {  // the groups' sums of the f16 activations (for the codes' offset)
+    if (xsum) {  // the groups' sums of the f16 activations (for the codes' offset); int4: per 64
+        const bool g64 = order == XORD_I4;
         for (int g = warp; g < K / 128; g += 8) {
             float sum = 0.0f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) sum += __half2float(__float2half_rn(__fmul_rn(row[g * 128 + 4 * lane + i], f)));
-#pragma unroll
-            for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
-            if (lane == 0) xsum[(long long)t * (K / 128) + g] = sum;
+            for (int m = g64 ? 8 : 16; m > 0; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
+            if (!g64 && lane == 0) xsum[(long long)t * (K / 128) + g] = sum;
+            if (g64 && (lane & 15) == 0) xsum[(long long)t * (K / 64) + 2 * g + (lane >> 4)] = sum;
         }
     }
     if (order == XORD_NATURAL) {  // converted once into shared memory, then 16-byte copies per output row
@@ -218,7 +219,10 @@ __global__ void __launch_bounds__(256) k_prep_a16(const __nv_bfloat16* x, int M,
             const int p = k & 7;
             src = (k & ~7) + ((p & 1) ? 4 + (p >> 1) : (p >> 1));
         }
-        out[k] = __float2half_rn(__fmul_rn(row[src], f));
+        __half h = __float2half_rn(__fmul_rn(row[src], f));
+        // int4: an odd k meets a high nibble, which enters the MMA as 16 u * 2^-24
+        if (order == XORD_I4 && (src & 1)) h = __float2half_rn(__fmul_rn(__half2float(h), 0.0625f));
+        out[k] = h;
     }
 }
 
@@ -341,7 +345,7 @@ cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8
 
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s, float* xsum) {
-    if (order == XORD_I5 && !xsum) return cudaErrorInvalidValue;
+    if ((order == XORD_I5 || order == XORD_I4) && !xsum) return cudaErrorInvalidValue;
     const size_t smem = (size_t)K * (sizeof(float) + sizeof(__half));  // the fp32 row and its f16 copy
     cudaError_t e = prefer_max_shared(k_prep_a16);
     if (e != cudaSuccess) return e;

@@ -134,7 +134,73 @@ __device__ __forceinline__ void fold_chains(T (&acc)[CH][NT][4]) {
             for (int i = 0; i < 4; ++i) acc[0][nt][i] += acc[ch][nt][i];
 }
 
-// The per-group MMAs of one unit for the weight-only formats.
+// One int4 unit (16 rows x 128 K: two 64-groups, each with its own scale).  The
+// activations of odd k, which meet the high nibbles, were staged divided by 16
+// (XORD_I4), so the operands need no shift to line the high nibble up:
+//  - one n-tile: the codes enter the MMAs as exact f16 subnormals with one mask
+//    each (low nibble u * 2^-24, high nibble in place 16 u * 2^-24), and the
+//    offset of q = u - 8 comes off with the token's sum over the 64-group, X
+//    (same units): y += s * (acc - 8 * 2^-24 * X), the scale carrying the 2^24
+//    back (side_to_regs).  X[2 i + h]: token 2 c + i, half h.
+//  - two n-tiles: the offset comes off in f16 instead (1024 + u - 1032 = q and
+//    1024 + 16 u - 1152 = 16 q, both exact); X is unused.
+constexpr float kI4Off = 4.76837158203125e-07f;  // 8 * 2^-24
+template <int NT, typename GetX>
+__device__ __forceinline__ void unit_i4(const Regs<QL_I4_G64_BF16>& r, GetX getx, bool nt1_live, const float (&X)[4],
+                                        float (&yacc)[NT][4]) {
+    constexpr int CH = NT == 1 ? 2 : 1;  // independent accumulation chains per group (see fold_chains)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float acc[CH][NT][4];
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0.0f;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            uint4 xv[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                if (nt == 0 || nt1_live) xv[nt] = getx(nt, 8 * h + p);
+            const uint32_t v0 = p == 0 ? r.w[0][h].x : r.w[0][h].y;  // row g: 8 codes of the lane's run
+            const uint32_t v1 = p == 0 ? r.w[1][h].x : r.w[1][h].y;  // row g + 8
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+                // bytes (sub, sub + 2): low nibbles -> k = 2 c, 2 c + 1; high nibbles -> 2 c + 8, 2 c + 9
+                const uint32_t w0 = sub == 0 ? v0 : v0 >> 8, w1 = sub == 0 ? v1 : v1 >> 8;
+                uint32_t a0, a1, a2, a3;
+                if constexpr (NT == 1) {
+                    a0 = w0 & 0x000F000Fu;
+                    a2 = w0 & 0x00F000F0u;
+                    a1 = w1 & 0x000F000Fu;
+                    a3 = w1 & 0x00F000F0u;
+                } else {
+                    a0 = hadd2_u32(and_or(w0, 0x000F000Fu, 0x64006400u), 0xE408E408u);
+                    a2 = hadd2_u32(and_or(w0, 0x00F000F0u, 0x64006400u), 0xE480E480u);
+                    a1 = hadd2_u32(and_or(w1, 0x000F000Fu, 0x64006400u), 0xE408E408u);
+                    a3 = hadd2_u32(and_or(w1, 0x00F000F0u, 0x64006400u), 0xE480E480u);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (nt == 1 && !nt1_live) continue;
+                    const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
+                    const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
+                    mma_f16(acc[sub % CH][nt], a0, a1, a2, a3, b0, b1);
+                }
+            }
+        }
+        fold_chains<CH, NT>(acc);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = NT == 1 ? fmaf(-kI4Off, X[2 * (i & 1) + h], acc[0][nt][i]) : acc[0][nt][i];
+                yacc[nt][i] = fmaf(r.s[i >> 1][h], t, yacc[nt][i]);
+            }
+    }
+}
+
+// The per-group MMAs of one unit for the byte weight-only formats (int8, E4M3).
 // getx(nt, piece) returns the lane's 16-byte activation piece for n-tile nt.
 // X: the group sums of the lane's column tokens (int8 codes only: their subnormal offset).
 // yacc[nt][i] accumulates scale * partial; i = 0,1 row g, i = 2,3 row g + 8.
@@ -142,50 +208,7 @@ template <int FMT, int NT, typename GetX>
 __device__ __forceinline__ void unit_a16(const Regs<FMT>& r, GetX getx, bool nt1_live, const float (&X)[NT][2],
                                          float (&yacc)[NT][4]) {
     constexpr int CH = NT == 1 ? 2 : 1;  // independent accumulation chains per group (see fold_chains)
-    if constexpr (FMT == QL_I4_G64_BF16) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float acc[CH][NT][4];
-#pragma unroll
-            for (int ch = 0; ch < CH; ++ch)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) acc[ch][nt][0] = acc[ch][nt][1] = acc[ch][nt][2] = acc[ch][nt][3] = 0.0f;
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                uint4 xv[NT];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    if (nt == 0 || nt1_live) xv[nt] = getx(nt, 8 * h + p);
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    // Nibble pairs at bits (8 sub, 8 sub + 16) and (8 sub + 4, 8 sub + 20): the low
-                    // nibble of each byte becomes 1024 + u and -1032 leaves q = u - 8; the high nibble,
-                    // masked in place, becomes 1024 + 16 u and one exact FMA (x / 16 - 72) leaves q.
-                    const uint32_t w0 = (p == 0 ? r.w[0][h].x : r.w[0][h].y) >> (8 * sub);
-                    const uint32_t w1 = (p == 0 ? r.w[1][h].x : r.w[1][h].y) >> (8 * sub);
-                    const uint32_t a0 = hadd2_u32(and_or(w0, 0x000F000Fu, 0x64006400u), 0xE408E408u);
-                    const uint32_t a2 = hfma2_u32(and_or(w0, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-                    const uint32_t a1 = hadd2_u32(and_or(w1, 0x000F000Fu, 0x64006400u), 0xE408E408u);
-                    const uint32_t a3 = hfma2_u32(and_or(w1, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        if (nt == 1 && !nt1_live) continue;
-                        const uint32_t b0 = sub == 0 ? xv[nt].x : xv[nt].z;
-                        const uint32_t b1 = sub == 0 ? xv[nt].y : xv[nt].w;
-                        mma_f16(acc[sub % CH][nt], a0, a1, a2, a3, b0, b1);
-                    }
-                }
-            }
-            fold_chains<CH, NT>(acc);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                yacc[nt][0] = fmaf(r.s[0][h], acc[0][nt][0], yacc[nt][0]);
-                yacc[nt][1] = fmaf(r.s[0][h], acc[0][nt][1], yacc[nt][1]);
-                yacc[nt][2] = fmaf(r.s[1][h], acc[0][nt][2], yacc[nt][2]);
-                yacc[nt][3] = fmaf(r.s[1][h], acc[0][nt][3], yacc[nt][3]);
-            }
-        }
-    } else {
+    {
         float acc[CH][NT][4];
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch)
@@ -470,11 +493,15 @@ __host__ __device__ constexpr size_t moe_ring_bytes() {
 }
 
 // Shared memory of the dense kernel staging `rows` token rows of XG groups.
+// srows: rows of the int4 one-n-tile kernel's staged group sums, [srows][XG][2] fp32.
 template <int FMT, int UPS>
-__host__ __device__ constexpr size_t tma_smem(int rows, int XG) {
+__host__ __device__ constexpr size_t tma_smem(int rows, int XG, int srows = 0) {
     return 1024 /* alignment slack */ + ring_bytes<FMT, UPS>() + (size_t)kWarps * stages_of<FMT, UPS>() * 8 + 16 +
-           (size_t)rows * ((size_t)XG * tx_group_bytes<FMT>() + tx_row_pad<FMT>());
+           (size_t)rows * ((size_t)XG * tx_group_bytes<FMT>() + tx_row_pad<FMT>()) + (size_t)srows * XG * 8;
 }
+// int4 with one n-tile offsets its subnormal codes with the tokens' 64-group sums (unit_i4).
+template <int FMT, int NT>
+__host__ __device__ constexpr bool i4_sums() { return FMT == QL_I4_G64_BF16 && NT == 1; }
 
 // Position in the unit stream: K part, row slab, group within the part.
 struct UnitPos {
@@ -576,8 +603,10 @@ __device__ __forceinline__ void side_to_regs(Regs<FMT>& r, const Side<FMT, NT>& 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         if constexpr (FMT == QL_I4_G64_BF16) {
-            r.s[h][0] = __uint_as_float(d.sw[h][0] << 16);
-            r.s[h][1] = __uint_as_float(d.sw[h][0] & 0xFFFF0000u);
+            // one n-tile: the unit's sums carry 2^-24 (the subnormal codes), the scale 2^24
+            constexpr float k = NT == 1 ? 16777216.0f : 1.0f;
+            r.s[h][0] = __uint_as_float(d.sw[h][0] << 16) * k;
+            r.s[h][1] = __uint_as_float(d.sw[h][0] & 0xFFFF0000u) * k;
         } else {
             r.s[h] = scale_value<FMT>(d.sw[h][0]);
         }
@@ -713,6 +742,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     uint32_t xrow_off[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) xrow_off[nt] = (uint32_t)((8 * nt + g < rows_x ? 8 * nt + g : rows_x) * R);
+    // int4, one n-tile: the group-sum rows of this lane's accumulator columns (tokens 2 c + i)
+    uint32_t srow_off[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) srow_off[i] = (uint32_t)(8 * (2 * c + i < rows_x ? 2 * c + i : 0) * a.XG);
     if (rows_x < NT * 8) {
         const int pieces = ngs * XGB / 16;
         for (int i = threadIdx.x; i < pieces; i += kThreads)
@@ -730,6 +763,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
             const long long ldx_b = a.ldx * (act8<FMT>() ? 1 : 2);
             for (int t = 0; t < rows_x; ++t)
                 bulk_load(xs_base + (uint32_t)(t * R), xsrc + t * ldx_b + (long long)gs0 * XGB, row_bytes, xbar);
+        }
+    }
+    // int4, one n-tile: the staged tokens' sums over each 64-group, [token][group][half], after
+    // the activation rows (a lane whose token is absent reads token 0's: its column is never stored).
+    const uint32_t xsum_s = xs_base + (uint32_t)((a.M < NT * 8 ? a.M + 1 : NT * 8) * R);
+    if constexpr (i4_sums<FMT, NT>()) {
+        const int per_row = 2 * ngs;
+        for (int i = threadIdx.x; i < rows_x * per_row; i += kThreads) {
+            const int t = i / per_row, j = i - t * per_row;
+            const float v = __ldg(a.xsum + (long long)t * 2 * a.Gtot + 2 * (a.g0 + gs0) + j);
+            asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(xsum_s + (uint32_t)(8 * (t * a.XG) + 4 * j)), "f"(v)
+                         : "memory");
         }
     }
     // Per-token side data of the units already in flight: the activation scales (byte
@@ -838,6 +883,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
                             yacc[nt][i] = fmaf(r.s[i >> 1] * sd[s][ui].sx[nt][i & 1], acc[nt][i], yacc[nt][i]);
                 } else if constexpr (FMT == QL_I5Z_G128_F16) {
                     unit_i5<NT>(r, getx, nt1_live, sd[s][ui].sx, yacc);
+                } else if constexpr (FMT == QL_I4_G64_BF16) {
+                    float X[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    if constexpr (i4_sums<FMT, NT>()) {
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+                            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];\n"
+                                         : "=f"(X[2 * i]), "=f"(X[2 * i + 1])
+                                         : "r"(xsum_s + srow_off[i] + (uint32_t)(8 * lg)));
+                    }
+                    unit_i4<NT>(r, getx, nt1_live, X, yacc);
                 } else {
                     unit_a16<FMT, NT>(r, getx, nt1_live, sd[s][ui].sx, yacc);
                 }
@@ -1185,11 +1240,12 @@ int swizzle_mode() {
                                  : (FMT == QL_I5Z_G128_F16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Groups of activations one CTA can stage for `rows` tokens next to its rings.
+// Groups of activations one CTA can stage for `rows` tokens (and `srows` rows of group sums)
+// next to its rings.
 template <int FMT, int UPS = 1>
-int max_staged_groups(int rows, size_t smem_optin) {
+int max_staged_groups(int rows, size_t smem_optin, int srows = 0) {
     for (int xg = 256; xg >= 1; --xg)
-        if (tma_smem<FMT, UPS>(rows, xg) <= smem_optin) return xg;
+        if (tma_smem<FMT, UPS>(rows, xg, srows) <= smem_optin) return xg;
     return 0;
 }
 
@@ -1217,7 +1273,8 @@ cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& d
     if (a.G % UPS) return cudaErrorInvalidValue;
     // token rows staged, plus one row of zeros for the lanes of absent tokens
     const int rows = a.M < NT * 8 ? a.M + 1 : NT * 8;
-    const int XG = max_staged_groups<FMT, UPS>(rows, di.smem_optin);
+    const int srows = i4_sums<FMT, NT>() ? std::min(a.M, NT * 8) : 0;
+    const int XG = max_staged_groups<FMT, UPS>(rows, di.smem_optin, srows);
     if (XG < UPS) return cudaErrorInvalidValue;
     a.XG = XG;
     // K parts in whole slots, so a slot never straddles two parts
@@ -1228,7 +1285,7 @@ cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& d
     cudaError_t e = make_tmap_2d(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw, unit_row_bytes<FMT>(), 16,
                                  swizzle_mode<FMT>(), &a.tmap);
     if (e != cudaSuccess) return e;
-    const size_t smem = tma_smem<FMT, UPS>(rows, XG);
+    const size_t smem = tma_smem<FMT, UPS>(rows, XG, srows);
     static bool attr_set[64] = {};  // per device ordinal
     int dev = 0;
     cudaGetDevice(&dev);

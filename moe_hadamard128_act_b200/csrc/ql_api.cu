@@ -148,8 +148,10 @@ FwdWs forward_ws(int fmt, size_t M, size_t N, size_t K) {
     } else {
         w.x_bytes = align_up(M * K * 2, 256);
         w.f_bytes = align_up(M * 4, 256);
-        // the tokens' group sums: the int5 zero point, and the int8 codes' offset in the decode kernel
+        // the tokens' group sums: the int5 zero point, and the int8 / int4 codes' offset in the decode
+        // kernel (int4: per 64-group)
         if (fmt == QL_I5Z_G128_F16 || fmt_i8_a16(fmt)) w.g_bytes = align_up(M * (K / 128) * 4, 256);
+        if (fmt == QL_I4_G64_BF16) w.g_bytes = align_up(M * (K / 64) * 4, 256);
     }
     return w;
 }
@@ -430,8 +432,9 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
         return from_cuda(e);
     }
     const long long ny = (long long)M * N;  // the prologue zeroes y for the accumulating GEMM
-    float* const xsum = (fmt == QL_I5Z_G128_F16 || fmt_i8_a16(fmt)) ? reinterpret_cast<float*>(wsb + w.x_bytes + w.f_bytes)
-                                                                     : nullptr;
+    float* const xsum = (fmt == QL_I5Z_G128_F16 || fmt == QL_I4_G64_BF16 || fmt_i8_a16(fmt))
+                            ? reinterpret_cast<float*>(wsb + w.x_bytes + w.f_bytes)
+                            : nullptr;
     if (fmt == QL_I8A8_G128_BF16) {
         const int t = trace_begin(QL_KIND_ACT_QUANT, s);
         e = launch_act_quant(x, M, K, rot, static_cast<int8_t*>(xs), xf, nullptr, 0, y, ny, s);
@@ -458,7 +461,7 @@ int qlinear_forward(const void* x, const void* W_packed, const void* scales, con
             a.zeros = zeros;
             a.xs = static_cast<const uint8_t*>(xs) + ((size_t)m0 * K + k0) * xelem;
             a.xf = act8 ? xf + (size_t)m0 * G : xf + m0;
-            a.xsum = xsum ? xsum + (size_t)m0 * G : nullptr;
+            a.xsum = xsum ? xsum + (size_t)m0 * G * (fmt == QL_I4_G64_BF16 ? 2 : 1) : nullptr;
             a.y = y + (size_t)m0 * N;
             a.acc = nullptr;
             a.M = M - m0 < 16 ? M - m0 : 16;

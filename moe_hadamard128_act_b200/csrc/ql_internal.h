@@ -64,7 +64,10 @@ cudaError_t launch_act_quant_e4m3(const void* x, int M, int K, int rotate, uint8
                                   float* yz, long long nz, cudaStream_t s, const int32_t* inv = nullptr,
                                   int topk = 0);
 // XORD_I5 also writes xsum [M][K/128] (each group's sum of the f16 activations, for the zero
-// point) and puts 2^24 into xf (the int5 codes enter the MMAs as exact subnormals u * 2^-24).
+// point) and puts 2^24 into xf (the int5 codes enter the MMAs as exact subnormals u * 2^-24);
+// so does any other order given an xsum, but XORD_I4: it stages the activations of odd k (the
+// high nibbles) divided by 16, writes the sums per 64-group, [M][K/64], and no 2^24 (the int4
+// kernel that uses the sums puts that factor into its scales).
 cudaError_t launch_prep_a16(const void* x, int M, int K, int rotate, int order, __half* xs, float* xf, float* yz,
                             long long nz, cudaStream_t s, float* xsum = nullptr);
 
@@ -83,7 +86,8 @@ struct SkinnyArgs {
     const uint8_t* zeros;  // int5: [N][Gtot]
     const void* xs;        // prepared activations, row stride ldx elements; offset to group g0
     const float* xf;       // A16: [M] inverse token factors; W8A8: sx [M][Gtot]
-    const float* xsum = nullptr;  // int5, int8 A16: each token's sums of its f16 activations per group [M][Gtot]
+    const float* xsum = nullptr;  // int5, int8 A16: each token's sums of its f16 activations per group [M][Gtot];
+                                  // int4: per 64-group [M][2 Gtot]
     float* y;              // [M][ldy]
     int32_t* acc;          // optional W8A8 group sums [M][N][Gtot]
     unsigned* err;         // device error word (filled by launch_skinny)
