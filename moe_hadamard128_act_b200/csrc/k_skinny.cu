@@ -527,6 +527,28 @@ struct UnitPos {
     __device__ __forceinline__ int grp(int GP) const { return part * GP + gi; }
 };
 
+// int4 with two units per ring slot loads the slot as one box of 16 rows x 128 bytes (both
+// groups of each row contiguous, 128-byte swizzle) instead of two 64-byte-wide boxes: one copy
+// per slot, and whole 128-byte row segments from DRAM.
+template <int FMT, int UPS>
+__host__ __device__ constexpr bool wide_i4() { return FMT == QL_I4_G64_BF16 && UPS == 2; }
+
+// The lane's int4 fragments of unit ui (0, 1) of a wide slot: its bytes 64 ui .. 64 ui + 63 of
+// each 128-byte row, 16-byte chunk j at j ^ (row & 7).  Each quarter-warp's eight 8-byte reads
+// hit eight distinct chunks of one 128-byte swizzle row: conflict-free.
+__device__ __forceinline__ void read_unit_i4_wide(Regs<QL_I4_G64_BF16>& r, uint32_t slot, int ui, int g, int c) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = g + 8 * h;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int j = 4 * ui + 2 * half + (c >> 1);
+            const uint32_t a = slot + row * 128 + ((j ^ (row & 7)) << 4) + 8 * (c & 1);
+            asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];\n" : "=r"(r.w[h][half].x), "=r"(r.w[h][half].y) : "r"(a));
+        }
+    }
+}
+
 // The lane's weight fragments of one unit, out of its ring slot.
 template <int FMT>
 __device__ __forceinline__ void read_unit_smem(Regs<FMT>& r, uint32_t st, int g, int c) {
@@ -678,10 +700,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
     auto issue = [&](int s) {
         if (lane == 0) {
             mbar_expect_tx(bars + 8 * s, SB);
+            if constexpr (wide_i4<FMT, UPS>()) {
+                tma_load_2d(ring + s * SB, &a.tmap, UPS * ip.grp(GP) * URB, ip.slab * 16, bars + 8 * s);
+            } else {
 #pragma unroll
-            for (int i = 0; i < UPS; ++i)
-                tma_load_2d(ring + s * SB + i * SB1, &a.tmap, (UPS * ip.grp(GP) + i) * URB, ip.slab * 16,
-                            bars + 8 * s);
+                for (int i = 0; i < UPS; ++i)
+                    tma_load_2d(ring + s * SB + i * SB1, &a.tmap, (UPS * ip.grp(GP) + i) * URB, ip.slab * 16,
+                                bars + 8 * s);
+            }
         }
         if (ip.slab != i_slab) {
             i_slab = ip.slab;
@@ -839,7 +865,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_skinny_tma(const __grid_constan
             for (int ui = 0; ui < UPS; ++ui) {
                 Regs<FMT> r;
                 side_to_regs<FMT, NT>(r, sd[s][ui]);
-                read_unit_smem<FMT>(r, ring + s * SB + ui * SB1, g, c);
+                if constexpr (wide_i4<FMT, UPS>())
+                    read_unit_i4_wide(r, ring + s * SB, ui, g, c);
+                else
+                    read_unit_smem<FMT>(r, ring + s * SB + ui * SB1, g, c);
                 const int grp = UPS * cp.grp(GP) + ui;
                 const int lg = grp - gs0;  // group index in the staged activations
                 auto getx = [&](int nt, int p) -> uint4 {
@@ -1282,8 +1311,10 @@ cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& d
     if (a.GP < 1) return cudaErrorInvalidValue;
     if ((long long)((a.N + 15) / 16) * a.G * (di.sm_count + 1) >= (1LL << 31)) return cudaErrorInvalidValue;
     a.err = di.err_word;
-    cudaError_t e = make_tmap_2d(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw, unit_row_bytes<FMT>(), 16,
-                                 swizzle_mode<FMT>(), &a.tmap);
+    constexpr bool wide = wide_i4<FMT, UPS>();
+    cudaError_t e = make_tmap_2d(a.W, a.N, (long long)a.G * unit_row_bytes<FMT>(), a.ldw,
+                                 wide ? 2 * unit_row_bytes<FMT>() : unit_row_bytes<FMT>(), 16,
+                                 wide ? (int)CU_TENSOR_MAP_SWIZZLE_128B : swizzle_mode<FMT>(), &a.tmap);
     if (e != cudaSuccess) return e;
     const size_t smem = tma_smem<FMT, UPS>(rows, XG, srows);
     static bool attr_set[64] = {};  // per device ordinal
