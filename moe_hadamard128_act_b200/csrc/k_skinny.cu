@@ -472,21 +472,24 @@ __host__ __device__ constexpr int tx_row_pad() {
 }
 
 // The nibble formats put UPS = 2 consecutive units of a row slab in one ring
-// slot (two TMA boxes, one barrier): the per-slot waits, refills and
-// bookkeeping then cover 2 KB (int4) or 2.5 KB (int5) of weights instead of
-// half that.  The 2.5 KB int5 slots take three ring stages instead of four.
+// slot (one barrier): the per-slot waits, refills and bookkeeping then cover
+// 2 KB (int4) or 2.5 KB (int5) of weights instead of half that.
+// Ring depth, measured per format at 1 to 16 tokens: the int4 and int5 two-unit slots run
+// best three deep, format 7 (byte activations, four k32 MMAs per unit) two deep, the rest four
+// deep.  Deeper rings were slower for every format: more copies in flight per SM do not raise
+// the DRAM rate here, they only leave less shared memory to the staged activations.
 template <int FMT, int UPS = 1>
 __host__ __device__ constexpr int stages_of() {
-    return (FMT == QL_I5Z_G128_F16 && UPS == 2) ? 3 : kStages;
+    return UPS == 2 ? 3 : (FMT == QL_FP8A8_B128_BF16 ? 2 : kStages);
 }
 template <int FMT, int UPS = 1>
 __host__ __device__ constexpr size_t ring_bytes() {
     return (size_t)kWarps * stages_of<FMT, UPS>() * UPS * stage_bytes<FMT>();
 }
 // The grouped (MoE) kernel's ring depth.  It reads its activations through L1 (a
-// chunk's tokens are scattered rows of the prepared x); six slots, which leave
-// less of the SM to L1, were measured slower at every decode batch size.
-constexpr int kMoeStages = 4;
+// chunk's tokens are scattered rows of the prepared x).  Measured per whole call at
+// 1, 8 and 16 tokens, two slots beat three, four and six at every batch size.
+constexpr int kMoeStages = 2;
 template <int FMT>
 __host__ __device__ constexpr size_t moe_ring_bytes() {
     return (size_t)kWarps * kMoeStages * stage_bytes<FMT>();
