@@ -475,12 +475,14 @@ __host__ __device__ constexpr int tx_row_pad() {
 // slot (one barrier): the per-slot waits, refills and bookkeeping then cover
 // 2 KB (int4) or 2.5 KB (int5) of weights instead of half that.
 // Ring depth, measured per format at 1 to 16 tokens: the int4 and int5 two-unit slots run
-// best three deep, format 7 (byte activations, four k32 MMAs per unit) two deep, the rest four
-// deep.  Deeper rings were slower for every format: more copies in flight per SM do not raise
-// the DRAM rate here, they only leave less shared memory to the staged activations.
+// best three deep, the byte formats' two-unit slots (4 KB) two deep, single-unit slots four
+// deep but format 7's two.  Deeper rings were slower for every format: more copies in flight
+// per SM do not raise the DRAM rate here, they only leave less shared memory to the staged
+// activations.
 template <int FMT, int UPS = 1>
 __host__ __device__ constexpr int stages_of() {
-    return UPS == 2 ? 3 : (FMT == QL_FP8A8_B128_BF16 ? 2 : kStages);
+    return UPS == 2 ? ((FMT == QL_I4_G64_BF16 || FMT == QL_I5Z_G128_F16) ? 3 : 2)
+                    : (FMT == QL_FP8A8_B128_BF16 ? 2 : kStages);
 }
 template <int FMT, int UPS = 1>
 __host__ __device__ constexpr size_t ring_bytes() {
@@ -1351,12 +1353,12 @@ cudaError_t run_skinny(const SkinnyArgs& in, cudaStream_t s, const DeviceInfo& d
 
 template <int FMT>
 cudaError_t run_skinny_fmt(const SkinnyArgs& a, cudaStream_t s, const DeviceInfo& di) {
-    if constexpr (FMT == QL_I4_G64_BF16 || FMT == QL_I5Z_G128_F16) {
-        // Two units per ring slot up to 8 tokens.  With 16 the doubled ring leaves room for
-        // fewer staged activation groups, K splits into more parts, and that costs more than
-        // the slots save.
-        if (a.G % 2 == 0 && a.M <= 8) return run_skinny<FMT, 1, false, 2>(a, s, di);
-    }
+    // Two units per ring slot up to 8 tokens, for every format (int8 and fp8: 4 KB slots two
+    // deep, the same 128 KB ring per SM as one-unit slots four deep, with half the waits,
+    // refills and bookkeeping).  With 16 tokens the nibble formats' doubled ring leaves room
+    // for fewer staged activation groups, K splits into more parts, and that costs more than
+    // the slots save.
+    if (a.G % 2 == 0 && a.M <= 8) return run_skinny<FMT, 1, false, 2>(a, s, di);
     if (a.M > 8) return run_skinny<FMT, 2, false>(a, s, di);
     return run_skinny<FMT, 1, false>(a, s, di);
 }
