@@ -1359,6 +1359,10 @@ cudaError_t run_skinny_fmt(const SkinnyArgs& a, cudaStream_t s, const DeviceInfo
     // for fewer staged activation groups, K splits into more parts, and that costs more than
     // the slots save.
     if (a.G % 2 == 0 && a.M <= 8) return run_skinny<FMT, 1, false, 2>(a, s, di);
+    // Two n-tiles: two-unit slots measured faster for the fp8 codes only (FP8 3%, format 7 7% at
+    // 16 tokens); the int8 formats ran slower with them (W8A8 spills at that register count).
+    if constexpr (FMT == QL_FP8_B128_BF16 || FMT == QL_FP8A8_B128_BF16)
+        if (a.G % 2 == 0 && a.M > 8) return run_skinny<FMT, 2, false, 2>(a, s, di);
     if (a.M > 8) return run_skinny<FMT, 2, false>(a, s, di);
     return run_skinny<FMT, 1, false>(a, s, di);
 }
