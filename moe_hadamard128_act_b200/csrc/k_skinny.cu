@@ -436,14 +436,14 @@ __device__ __forceinline__ void unit_down(const Regs<kFmtDown>& r, GetX getx, bo
 // ---------------------------------------------------------------------------
 // Dense skinny GEMM, TMA-fed.
 //
-// Every warp owns a ring of kStages shared-memory slots, one unit (16 rows of
-// the packed weight x one 128-K group) per slot.  Lane 0 keeps kStages units
-// in flight with cp.async.bulk.tensor (2-D tile [16 rows][unit bytes],
-// zero-filled past row N) completing on a per-slot mbarrier; the whole warp
-// waits on the slot, pulls its fragments out of shared memory, refills the
-// slot with the unit kStages ahead and computes.  With 16 warps x 4 slots x
-// 2 KB the SM keeps up to 128 KB of weight in flight without holding it in
-// registers.  Waits are bounded: a slot that never fills sets
+// Every warp owns a ring of shared-memory slots (stages_of below), each one or
+// two units (16 rows of the packed weight x one 128-K group).  Lane 0 keeps the
+// ring's slots in flight with cp.async.bulk.tensor (2-D tile [16 rows][unit
+// bytes], zero-filled past row N) completing on a per-slot mbarrier; the whole
+// warp waits on the slot, pulls its fragments out of shared memory, computes,
+// and refills the slot with the units a ring ahead.  At int8, 16 warps x 2
+// slots x 4 KB (or 4 x 2 KB) keep 128 KB of weight in flight per SM without
+// holding it in registers.  Waits are bounded: a slot that never fills sets
 // QL_DEVERR_TIMEOUT in the device error word and the CTA drains and returns.
 //
 // Units are numbered (K part, row slab, group within the part): a CTA's
@@ -595,7 +595,7 @@ __device__ unsigned long long g_skinny_prof[148 * 16];
 #define QL_PROF(slot)
 #endif
 
-// Per-unit side data, fetched kStages units ahead of use together with the
+// Per-unit side data, fetched a ring ahead of use together with the
 // weight tile: raw scale bits (converted only when the unit is computed, so
 // the loads never stall the issuing loop), int5 zero points, and for W8A8 the
 // activation scales of the lane's output tokens (W8A8 and format 7).
@@ -603,7 +603,7 @@ template <int FMT, int NT>
 struct Side {
     uint32_t sw[2][1];  // weight scale bits [row g / g+8] (int4: both 64-groups' bf16 scales in one word)
     uint32_t z[2];      // int5 zero points
-    float sx[NT][2];    // byte activations: scales of tokens 8nt + 2c + {0, 1}; int5: their group sums
+    float sx[NT][2];    // byte activations: scales of tokens 8nt + 2c + {0, 1}; int5, int8 A16: their group sums
 };
 
 template <int FMT, int NT>
