@@ -70,6 +70,10 @@ def test_packed_sizes_and_workspace_reject_bad_args(L):
     assert Q.qlinear_workspace_size(3, 2 | 1, 16, 21504, 5376) == Q.qlinear_workspace_size(3, 1, 16, 21504, 5376)
     assert Q.qlinear_workspace_size(1, 0, 16, 21504, 5376) >= 16 * 5376 * 2
     assert Q.qlinear_workspace_size(3, 1, 16, 21504, 5376) >= 16 * 5376 + 16 * 42 * 4
+    # the 16-bit activations, their token factors and the tokens' group sums (the decode kernels take
+    # the codes' offset off with them): per 128 for int8 and int5, per 64 for int4
+    for fmt, per in ((1, 128), (2, 128), (5, 128), (4, 64)):
+        assert Q.qlinear_workspace_size(fmt, 0, 16, 21504, 5376) >= 16 * 5376 * 2 + 16 * 4 + 16 * (5376 // per) * 4
     # format 7: E4M3 codes and their scales for the decode kernel (M <= 16); from 17 rows the tensor-core
     # GEMM also takes transposed scales and its weight-scale scratch
     assert 5376 + 42 * 4 <= Q.qlinear_workspace_size(7, 1, 1, 21504, 5376) < 42 * 21504 * 4
