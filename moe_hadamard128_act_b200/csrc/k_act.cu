@@ -108,6 +108,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_act_quant(const __nv_bf
 // and xf = 2^24 / f (the codes enter the MMAs as u * 2^-24).  The natural
 // order with xsum requested is the int8 decode's: the same group sums and
 // 2^24 / f (its codes enter the MMAs as the subnormals (q + 128) * 2^-24).
+// For int4 the activations of odd k (those that meet a byte's high nibble,
+// which the decode GEMM uses in place as 16 u * 2^-24) are stored divided by
+// 16, xsum holds the sums per 64-group, [M][K/64], and xf stays 1 / f (the
+// int4 GEMM puts the 2^24 into its scales where it needs it).
 // f16 holds every bf16 value of the scaled row exactly down to 2^-14 (its
 // normal range); below that the rounding error is under 2^-39 of the row's
 // max, far beneath the fp32 accumulation error of the GEMM.
